@@ -1,0 +1,367 @@
+"""Pins of the CPU oracle to facts that do not come from the oracle itself: hand-worked cases,
+closed forms, invariants, brute force on tiny inputs and library routines (torch dtype casts,
+numpy float64 matmul). Each test names the oracle function it pins."""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+
+
+def _bf16_bits(t):
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+# --------------------------------------------------------------------------------------------
+# number formats
+# --------------------------------------------------------------------------------------------
+
+def test_bf16_value_all_patterns_match_torch():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ref = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).double().numpy()
+    got = oracle.bf16_value(bits)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+
+
+def test_bf16_round_matches_torch_on_f32_values_and_ties():
+    rng = np.random.default_rng(1)
+    u = rng.integers(0, 2 ** 32, 200000, dtype=np.uint64).astype(np.uint32)
+    u = u[((u >> 23) & 0xFF) != 0xFF]                       # finite only
+    ties = (u & 0xFFFF0000) | 0x8000                        # exact halfway cases
+    f = np.concatenate([u, ties]).view(np.float32)
+    ref = _bf16_bits(torch.from_numpy(f).to(torch.bfloat16))
+    got = oracle.bf16_round(f.astype(np.float64))
+    assert np.array_equal(got, ref)
+
+
+def test_bf16_round_is_a_single_rounding_of_the_double():
+    # 1 + 2^-8 + 2^-40 lies just above the halfway point between 1 and 1 + 2^-7: the nearest bf16
+    # is 1 + 2^-7. Rounding to f32 first would land exactly on the tie and go to even (1.0).
+    v = np.array([1 + 2.0 ** -8 + 2.0 ** -40, -(1 + 2.0 ** -8 + 2.0 ** -40), 1 + 2.0 ** -8], np.float64)
+    got = oracle.bf16_value(oracle.bf16_round(v))
+    assert list(got) == [1 + 2.0 ** -7, -(1 + 2.0 ** -7), 1.0]
+
+
+def test_e4m3_value_all_codes_match_torch():
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).double().numpy()
+    got = oracle.e4m3_value(codes)
+    nan = np.isnan(ref)
+    assert nan.sum() == 2 and np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+    assert got[0x7E] == 448.0 and got[0x01] == 2.0 ** -9 and got[0x08] == 2.0 ** -6
+
+
+def test_e4m3_encode_matches_torch_in_range_and_saturates():
+    rng = np.random.default_rng(2)
+    vals = np.concatenate([
+        rng.uniform(-448, 448, 100000), rng.normal(0, 1, 100000), rng.normal(0, 0.01, 50000),
+    ]).astype(np.float32)
+    grid = oracle.e4m3_value(np.arange(0, 0x7F, dtype=np.uint8))   # all finite non-negative values
+    mids = ((grid[1:] + grid[:-1]) / 2).astype(np.float32)           # exact ties (representable in f32)
+    vals = np.concatenate([vals, mids, -mids, grid.astype(np.float32)])
+    ref = torch.from_numpy(vals).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = oracle.e4m3_encode(vals)
+    assert np.array_equal(got, ref)
+    sat = oracle.e4m3_encode(np.array([448.0, 460.0, 470.0, 1e6, -500.0], np.float32))
+    assert list(sat) == [0x7E, 0x7E, 0x7E, 0x7E, 0xFE]
+
+
+# --------------------------------------------------------------------------------------------
+# routing
+# --------------------------------------------------------------------------------------------
+
+def test_route_closed_forms():
+    ids, w = oracle.route_topk(np.array([[0.0, math.log(3.0)]], np.float32), 2)
+    assert ids.tolist() == [[1, 0]]
+    assert abs(w[0, 0] - 0.75) < 2e-7 and abs(w[0, 1] - 0.25) < 2e-7
+    # all logits equal, k = E: ties go to the lower index, weights exactly 1/E
+    ids, w = oracle.route_topk(np.zeros((3, 8), np.float32), 8)
+    assert ids.tolist() == [list(range(8))] * 3
+    assert np.all(w == np.float32(0.125))
+    # k = 1: weight exactly 1
+    ids, w = oracle.route_topk(np.array([[0.3, -2.0, 5.0, 5.0]], np.float32), 1)
+    assert ids.tolist() == [[2]] and w[0, 0] == 1.0
+
+
+def test_route_brute_force_against_numpy():
+    rng = np.random.default_rng(3)
+    for trial in range(200):
+        T, E = int(rng.integers(1, 9)), int(rng.integers(1, 40))
+        k = int(rng.integers(1, E + 1))
+        lg = rng.normal(size=(T, E)).astype(np.float32)
+        if trial % 3 == 0:                                 # force ties
+            lg = np.round(lg * 2) / 2
+        ids, w = oracle.route_topk(lg, k)
+        for t in range(T):
+            order = sorted(range(E), key=lambda e: (-float(lg[t, e]), e))[:k]
+            assert ids[t].tolist() == order
+            ex = np.exp(lg[t, order].astype(np.float64) - lg[t, order[0]])
+            ref = (ex / ex.sum()).astype(np.float32)
+            assert np.array_equal(w[t], ref)
+            assert abs(float(w[t].astype(np.float64).sum()) - 1.0) <= 1e-6
+
+
+# --------------------------------------------------------------------------------------------
+# alignment
+# --------------------------------------------------------------------------------------------
+
+def test_align_hand_worked(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "align_hand.json")))
+    s, e, n = oracle.align(np.array(g["topk_ids"], np.int32), g["E"], g["block_m"])
+    assert s.tolist() == g["sorted_ids"]
+    assert e.tolist() == g["expert_ids"]
+    assert n == g["num_tokens_padded"]
+
+
+def _align_numpy(ids, E, B):
+    flat = ids.reshape(-1)
+    n = flat.size
+    cap = n + E * (B - 1)
+    sorted_ids = np.full(cap, n, np.int32)
+    expert_ids = np.full(-(-cap // B), -1, np.int32)
+    order = np.argsort(flat, kind="stable")            # by expert, ties by slot
+    counts = np.bincount(flat, minlength=E)
+    pos, src = 0, 0
+    for e in range(E):
+        c = int(counts[e])
+        sorted_ids[pos:pos + c] = order[src:src + c]
+        p = -(-c // B) * B
+        expert_ids[pos // B:(pos + p) // B] = e
+        pos += p
+        src += c
+    return sorted_ids, expert_ids, pos
+
+
+def test_align_brute_force_and_invariants():
+    rng = np.random.default_rng(4)
+    for _ in range(300):
+        T, E = int(rng.integers(0, 9)), int(rng.integers(1, 7))
+        k = int(rng.integers(1, min(3, E) + 1))
+        B = int(rng.choice([1, 2, 3, 4, 8, 16]))
+        ids = np.array([rng.permutation(E)[:k] for _ in range(T)], np.int32).reshape(T, k)
+        s, e, n = oracle.align(ids, E, B)
+        rs, re_, rn = _align_numpy(ids, E, B)
+        assert np.array_equal(s, rs) and np.array_equal(e, re_) and n == rn
+        flat = ids.reshape(-1)
+        real = s[:n][s[:n] < T * k]
+        assert sorted(real.tolist()) == list(range(T * k))      # every slot exactly once
+        for b in range(n // B):                                  # one expert per block
+            blk = s[b * B:(b + 1) * B]
+            assert all(flat[f] == e[b] for f in blk if f < T * k)
+        assert n == sum(-(-int(c) // B) * B for c in np.bincount(flat, minlength=E))
+
+
+# --------------------------------------------------------------------------------------------
+# W4A16 layer
+# --------------------------------------------------------------------------------------------
+
+def _hand_case(g, case):
+    H, I, E, T = g["H"], g["I"], g["E"], g["T"]
+    x = np.zeros((T, H), np.float32)
+    for t, c, v in g["x_nonzero"]:
+        x[t, c] = v
+    dw = np.uint32(int(g["default_word"], 16)).view(np.int32)
+    w13q = np.full((E, 2 * I, H // 8), dw, np.int32)
+    w2q = np.full((E, H, I // 8), dw, np.int32)
+    w13s = np.full((E, 2 * I, H // 32), g["default_scale_w13"], np.float32)
+    w2s = np.full((E, H, I // 32), g["default_scale_w2"], np.float32)
+    for e, r, wi, word in g["w13_words"]:
+        w13q[e, r, wi] = np.uint32(int(word, 16)).view(np.int32)
+    for e, r, wi, word in g["w2_words"]:
+        w2q[e, r, wi] = np.uint32(int(word, 16)).view(np.int32)
+    for e, r, gi, s in g["w13_scales"]:
+        w13s[e, r, gi] = s
+    for e, r, gi, s in g["w2_scales"]:
+        w2s[e, r, gi] = s
+    xb = _bf16_bits(torch.from_numpy(x).to(torch.bfloat16))
+    w13sb = _bf16_bits(torch.from_numpy(w13s).to(torch.bfloat16))
+    w2sb = _bf16_bits(torch.from_numpy(w2s).to(torch.bfloat16))
+    logits = np.array(case["logits"], np.float32)
+    return xb, logits, w13q, w13sb, w2q, w2sb
+
+
+def test_w4a16_hand_worked(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "w4a16_hand.json")))
+    for case in g["cases"]:
+        xb, logits, w13q, w13s, w2q, w2s = _hand_case(g, case)
+        out = oracle.moe_w4a16(xb, logits, case["k"], w13q, w13s, w2q, w2s)
+        ref = np.zeros_like(out)
+        for t, m, v in case["out_nonzero"]:
+            ref[t, m] = v
+        tol = case["rel_tol"] * np.abs(ref) + 1e-300
+        assert np.all(np.abs(out - ref) <= tol), (out[np.nonzero(ref)], ref[np.nonzero(ref)])
+
+
+def _np_unpack_w4(q, s):
+    """Independent numpy restatement of the INT4 group-32 format (for library-matmul pins)."""
+    q = q.view(np.uint32)
+    N, K8 = q.shape
+    codes = np.stack([(q >> (4 * j)) & 15 for j in range(8)], axis=-1).reshape(N, K8 * 8)
+    scale = torch.from_numpy(s.view(np.int16)).view(torch.bfloat16).double().numpy()
+    return (codes.astype(np.float64) - 8.0) * np.repeat(scale, 32, axis=1)
+
+
+def _np_bf16(v):
+    """bf16 rounding via torch (library); exact on these inputs (values come from f32 math below)."""
+    return torch.from_numpy(np.ascontiguousarray(v)).to(torch.bfloat16).double().numpy()
+
+
+def _np_ffn_w4(xd, w13, w2, I):
+    g = xd @ w13[:I].T
+    u = xd @ w13[I:].T
+    a = g / (1.0 + np.exp(-g)) * u
+    return a, w2
+
+
+def test_w4a16_dense_equivalence_with_uniform_routing():
+    """k = E and equal logits: every expert is selected with weight exactly 1/E, so the layer is
+    (1/E) * sum_e FFN_e(x); FFN_e evaluated with numpy float64 matmul on the unpacked weights."""
+    wl = W.WORKLOADS["tiny_w4a16"]
+    d = W.make_moe(wl, T=4, E=8, k=8, H=128, I=64)
+    x = W.np_bits(d["x"])
+    logits = np.zeros((4, 8), np.float32)
+    w13q, w13s, w2q, w2s = (W.np_bits(d[n]) for n in ("w13q", "w13s", "w2q", "w2s"))
+    out, h = oracle.moe_w4a16(x, logits, 8, w13q, w13s, w2q, w2s, want_h=True)
+    xd = oracle.bf16_value(x)  # exact
+    ref = np.zeros_like(out)
+    for e in range(8):
+        w13 = _np_unpack_w4(w13q[e], w13s[e])
+        w2 = _np_unpack_w4(w2q[e], w2s[e])
+        a, _ = _np_ffn_w4(xd, w13, w2, 64)
+        # h must be bf16(a): compare the oracle's intermediate to the rounding of numpy's a
+        hv = oracle.bf16_value(h[:, e, :])
+        assert np.all(np.abs(hv - a) <= np.abs(a) * 2.0 ** -8 + 1e-30)
+        ref += (1.0 / 8.0) * (hv @ w2.T)
+    assert np.allclose(out, ref, rtol=1e-12, atol=1e-15)
+
+
+def test_w4a16_single_expert_is_dense_gemm():
+    """k = 1 and one dominant logit: every token goes to expert 5 with weight 1."""
+    wl = W.WORKLOADS["tiny_w4a16"]
+    d = W.make_moe(wl, T=6, E=8, k=1, H=256, I=128)
+    x = W.np_bits(d["x"])
+    logits = np.zeros((6, 8), np.float32)
+    logits[:, 5] = 10.0
+    w13q, w13s, w2q, w2s = (W.np_bits(d[n]) for n in ("w13q", "w13s", "w2q", "w2s"))
+    out = oracle.moe_w4a16(x, logits, 1, w13q, w13s, w2q, w2s)
+    xd = oracle.bf16_value(x)
+    w13 = _np_unpack_w4(w13q[5], w13s[5])
+    w2 = _np_unpack_w4(w2q[5], w2s[5])
+    a, _ = _np_ffn_w4(xd, w13, w2, 128)
+    ref = _np_bf16(a) @ w2.T
+    # a from numpy and from the oracle may differ in the last double bit, which can flip a bf16
+    # rounding of h; bound that by one bf16 ulp of h per term
+    bound = (np.abs(a) * 2.0 ** -8) @ np.abs(w2.T) + 1e-12
+    assert np.all(np.abs(out - ref) <= bound)
+    assert np.allclose(out, ref, rtol=1e-6, atol=1e-9)
+
+
+def test_w4a16_dequant_matches_numpy_unpack():
+    d = W.make_moe(W.WORKLOADS["tiny_w4a16"], T=1, E=1, k=1, H=128, I=64)
+    q, s = W.np_bits(d["w13q"])[0], W.np_bits(d["w13s"])[0]
+    assert np.array_equal(oracle.w4a16_dequant(q, s), _np_unpack_w4(q, s))
+
+
+def test_w4a16_combine_weights_sum_to_one_on_workload_logits():
+    for name in ("tiny_w4a16", "decode_w4a16", "prefill_w4a16", "moe_fp8"):
+        wl = W.WORKLOADS[name]
+        lg = W.router_logits(wl, min(wl.T, 512), wl.E).numpy()
+        ids, w = oracle.route_topk(lg, wl.k)
+        assert np.all(np.abs(w.astype(np.float64).sum(1) - 1.0) <= 1e-6)
+        assert all(len(set(r)) == wl.k for r in ids.tolist())
+
+
+# --------------------------------------------------------------------------------------------
+# FP8
+# --------------------------------------------------------------------------------------------
+
+def test_fp8_act_quant_matches_torch_quantizer():
+    rng = np.random.default_rng(5)
+    x = torch.from_numpy(rng.normal(size=(37, 512)).astype(np.float32)).to(torch.bfloat16)
+    x[3, :128] = 0.0                                  # all-zero group: scale 1e-10/448
+    x[4, 128:256] = 1000.0
+    q, s = oracle.fp8_act_quant(_bf16_bits(x))
+    rq, rs = W.quantize_fp8_rows(x.float())
+    assert np.array_equal(q, rq.numpy()) and np.array_equal(s, rs.numpy())
+
+
+def test_fp8_closed_form_ones():
+    K, N = 7168, 256
+    a = np.full((2, K), 1.0, np.float32)
+    q, s = oracle.fp8_act_quant(_bf16_bits(torch.from_numpy(a).to(torch.bfloat16)))
+    assert np.all(q == 0x7E) and np.all(s == np.float32(1.0) / np.float32(448.0))
+    B = np.full((N, K), 0x7E, np.uint8)
+    Bs = np.full((N // 128, K // 128), np.float32(0.5) / np.float32(448.0), np.float32)
+    C = oracle.fp8_block_matmul(q, s, B, Bs)
+    assert np.all(np.abs(C - 0.5 * K) <= 1e-6 * 0.5 * K)
+
+
+def test_fp8_block_scale_indexing():
+    """One nonzero element per K block with power-of-two scales: C[m, n] = sum_kb
+    As[m, kb] * Bs[n // 128, kb] exactly, which fails for any transposed or shifted scale index."""
+    M, N, K = 3, 384, 512
+    one = 0x38                                                   # E4M3 code of 1.0
+    A = np.zeros((M, K), np.uint8)
+    B = np.zeros((N, K), np.uint8)
+    A[:, ::128] = one
+    B[:, 5::128] = 0
+    B[:, ::128] = one
+    As = np.array([[2.0 ** (kb + 4 * m) for kb in range(K // 128)] for m in range(M)], np.float32)
+    Bs = np.array([[2.0 ** (-2 * kb - 8 * nb) for kb in range(K // 128)] for nb in range(N // 128)], np.float32)
+    C = oracle.fp8_block_matmul(A, As, B, Bs)
+    for m in range(M):
+        for n in (0, 127, 128, 300, 383):
+            assert C[m, n] == sum(2.0 ** (kb + 4 * m) * 2.0 ** (-2 * kb - 8 * (n // 128)) for kb in range(K // 128))
+
+
+def test_fp8_dense_matches_numpy_matmul():
+    d = W.make_dense_fp8(W.WORKLOADS["dense_fp8"], 16, N=256, K=1024)
+    A, As, B, Bs = (d[n].numpy() for n in ("A", "As", "B", "Bs"))
+    C = oracle.fp8_block_matmul(A, As, B, Bs)
+    Ad = torch.from_numpy(A).view(torch.float8_e4m3fn).double().numpy() * np.repeat(As, 128, 1)
+    Bd = torch.from_numpy(B).view(torch.float8_e4m3fn).double().numpy() * np.repeat(np.repeat(Bs, 128, 0), 128, 1)
+    ref = Ad @ Bd.T
+    assert np.allclose(C, ref, rtol=1e-12, atol=1e-12)
+
+
+def _torch_fp8_rows(v32):
+    q, s = W.quantize_fp8_rows(torch.from_numpy(np.ascontiguousarray(v32)))
+    return q.numpy(), s.numpy()
+
+
+def test_fp8_moe_dense_equivalence_with_uniform_routing():
+    """k = E, equal logits: out = (1/E) sum_e FFN_e(x) with FFN_e from numpy float64 matmul on
+    decoded E4M3 weights and a torch-quantized intermediate."""
+    T, E, H, I = 3, 4, 256, 256
+    d = W.make_moe(W.WORKLOADS["moe_fp8"], T=T, E=E, k=E, H=H, I=I)
+    x = W.np_bits(d["x"])
+    w13, w13s, w2, w2s = (W.np_bits(d[n]) for n in ("w13", "w13s", "w2", "w2s"))
+    logits = np.zeros((T, E), np.float32)
+    out, hq, hs = oracle.moe_fp8(x, logits, E, w13, w13s, w2, w2s, want_h=True)
+    xq, xs = _torch_fp8_rows(d["x"].float().numpy())
+
+    def deq(q, s, bn=128):
+        v = torch.from_numpy(q).view(torch.float8_e4m3fn).double().numpy()
+        return v * np.repeat(np.repeat(s, bn, 0), 128, 1)
+
+    xd = torch.from_numpy(xq).view(torch.float8_e4m3fn).double().numpy() * np.repeat(xs, 128, 1)
+    ref = np.zeros_like(out)
+    for e in range(E):
+        g = xd @ deq(w13[e, :I], w13s[e, :I // 128]).T
+        u = xd @ deq(w13[e, I:], w13s[e, I // 128:]).T
+        a = (g / (1 + np.exp(-g)) * u).astype(np.float32)
+        q2, s2 = _torch_fp8_rows(a)
+        # the oracle's intermediate codes may differ from numpy's at exact rounding boundaries
+        # (a differs in the last f32 bit); they agree on almost every element
+        assert np.mean(hq[:, e, :] == q2) > 0.99
+        hd = torch.from_numpy(hq[:, e, :].copy()).view(torch.float8_e4m3fn).double().numpy() * np.repeat(hs[:, e, :], 128, 1)
+        ref += 0.25 * (hd @ deq(w2[e], w2s[e]).T)
+    assert np.allclose(out, ref, rtol=1e-10, atol=1e-12)

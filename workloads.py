@@ -1,0 +1,201 @@
+"""Seeded synthetic inputs for the quantized routed-MoE layer, shared by the CUDA path's tests and
+benchmark and by the CPU oracle. This module holds none of the layer's arithmetic: it draws
+random numbers and encodes synthetic checkpoints with torch's own dtype casts.
+
+Workloads (all seed 0, one independent random stream per (workload, tensor, expert)):
+
+  tiny_w4a16     T=16, H=512, I=256, E=8, top-2; router logits N(0,1)
+  decode_w4a16   T=32, H=7168, I=2048 (gate+up N=4096), E=384, top-8; router logits U[0,1)
+  prefill_w4a16  the decode shapes with T=8192; logits N(0,1) plus a per-expert Zipf bias
+  dense_fp8      A [M, 7168] (M = 1, 2, 4, ..., 4096), B [24576, 7168], E4M3 block-FP8
+  moe_fp8        T=4096, H=7168, I=2048, E=256, top-8, E4M3 block-FP8, Zipf-biased logits
+
+Recipes:
+  * x: bf16 of N(0,1) f32 draws.
+  * W4A16 weights: f32 N(0, 0.02) draws quantized per 32 consecutive inputs to unsigned INT4 with
+    scale = bf16(max|w| / 7) and code = clamp(round_half_even(w / scale) + 8, 0, 15) (code 8 for
+    an all-zero group), packed 8 codes per int32, code j of a word in bits [4j, 4j+4).
+  * FP8 weights: f32 N(0, 0.02) draws, one f32 scale max(amax, 1e-10)/448 per [128, 128] block,
+    codes = E4M3(w / scale) (torch's float8_e4m3fn cast).
+  * dense_fp8 activations: bf16 N(0,1) draws quantized per row and 128-column group the same way.
+  * Zipf bias: bias_e = -1.1 * ln(rank_e) with rank a seeded permutation of 1..E, added (f32) to
+    N(0,1) logits, so routed rows per expert are skewed: many experts get no rows, a few get
+    more than a thousand.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import numpy as np
+import torch
+
+SEED = 0
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    kind: str              # "w4a16", "fp8" (MoE layers) or "dense_fp8"
+    wid: int               # stream id of the workload
+    T: int = 0
+    H: int = 0
+    I: int = 0
+    E: int = 0
+    k: int = 0
+    logits: str = "normal"  # "normal", "uniform" or "zipf"
+    M_list: tuple = field(default_factory=tuple)
+    N: int = 0
+    K: int = 0
+
+
+WORKLOADS = {
+    "tiny_w4a16": Workload("tiny_w4a16", "w4a16", 0, T=16, H=512, I=256, E=8, k=2, logits="normal"),
+    "decode_w4a16": Workload("decode_w4a16", "w4a16", 1, T=32, H=7168, I=2048, E=384, k=8, logits="uniform"),
+    "prefill_w4a16": Workload("prefill_w4a16", "w4a16", 2, T=8192, H=7168, I=2048, E=384, k=8, logits="zipf"),
+    "dense_fp8": Workload("dense_fp8", "dense_fp8", 3, M_list=tuple(2 ** i for i in range(13)), N=24576, K=7168),
+    "moe_fp8": Workload("moe_fp8", "fp8", 4, T=4096, H=7168, I=2048, E=256, k=8, logits="zipf"),
+}
+
+# tensor stream ids
+_X, _LOGITS, _RANKS, _W13, _W2, _A, _B = range(7)
+
+
+def generator(wid: int, tensor: int, expert: int = 0, device="cpu", seed: int = SEED) -> torch.Generator:
+    state = np.random.SeedSequence([seed, wid, tensor, expert]).generate_state(2, dtype=np.uint32)
+    g = torch.Generator(device=device)
+    g.manual_seed(int(state[0]) << 32 | int(state[1]))
+    return g
+
+
+def bf16_normal(shape, g, device) -> torch.Tensor:
+    return torch.randn(shape, generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+
+
+def router_logits(wl: Workload, T: int, E: int, device="cpu", wid=None) -> torch.Tensor:
+    wid = wl.wid if wid is None else wid
+    g = generator(wid, _LOGITS, device=device)
+    if wl.logits == "uniform":
+        return torch.rand((T, E), generator=g, device=device, dtype=torch.float32)
+    z = torch.randn((T, E), generator=g, device=device, dtype=torch.float32)
+    if wl.logits == "zipf":
+        gr = generator(wid, _RANKS, device="cpu")
+        rank = torch.randperm(E, generator=gr).to(torch.float64) + 1.0
+        bias = (-1.1 * torch.log(rank)).to(torch.float32).to(device)
+        z = z + bias[None, :]
+    return z
+
+
+def quantize_w4_group32(w: torch.Tensor):
+    """f32 [N, K] -> (codes packed int32 [N, K/8], bf16 scales [N, K/32])."""
+    N, K = w.shape
+    wg = w.view(N, K // 32, 32)
+    scale = (wg.abs().amax(-1) / 7.0).to(torch.bfloat16)
+    sf = scale.float()[..., None]
+    safe = torch.where(sf > 0, sf, torch.ones_like(sf))
+    q = torch.where(sf > 0, torch.round(wg / safe) + 8.0, torch.full_like(wg, 8.0)).clamp(0, 15)
+    q = q.to(torch.int64).view(N, K // 8, 8)
+    shifts = torch.arange(0, 32, 4, device=w.device, dtype=torch.int64)
+    packed = (q << shifts).sum(-1)
+    packed = packed - ((packed >> 31) & 1) * (1 << 32)       # uint32 bit pattern as int32
+    return packed.to(torch.int32).contiguous(), scale.contiguous()
+
+
+def quantize_fp8_blocks(w: torch.Tensor, bn: int = 128, bk: int = 128):
+    """f32 [N, K] -> (E4M3 codes uint8 [N, K], f32 scales [N/bn, K/bk])."""
+    N, K = w.shape
+    wb = w.view(N // bn, bn, K // bk, bk)
+    amax = wb.abs().amax(dim=(1, 3))
+    scale = torch.clamp(amax, min=1e-10) / 448.0
+    q = (wb / scale[:, None, :, None]).to(torch.float8_e4m3fn)
+    return q.view(N, K).view(torch.uint8).contiguous(), scale.contiguous()
+
+
+def quantize_fp8_rows(a: torch.Tensor, group: int = 128):
+    """f32 [M, K] -> (E4M3 codes uint8 [M, K], f32 scales [M, K/group])."""
+    M, K = a.shape
+    ag = a.view(M, K // group, group)
+    scale = torch.clamp(ag.abs().amax(-1), min=1e-10) / 448.0
+    q = (ag / scale[..., None]).to(torch.float8_e4m3fn)
+    return q.view(M, K).view(torch.uint8).contiguous(), scale.contiguous()
+
+
+def make_moe(wl: Workload, device="cpu", T=None, E=None, k=None, H=None, I=None):
+    """Inputs of a routed MoE workload. Overrides let tests reuse a recipe at other sizes."""
+    T = wl.T if T is None else T
+    E = wl.E if E is None else E
+    k = wl.k if k is None else k
+    H = wl.H if H is None else H
+    I = wl.I if I is None else I
+    x = bf16_normal((T, H), generator(wl.wid, _X, device=device), device)
+    logits = router_logits(wl, T, E, device)
+    d = dict(x=x, logits=logits, T=T, H=H, I=I, E=E, k=k, kind=wl.kind)
+    if wl.kind == "w4a16":
+        w13q = torch.empty((E, 2 * I, H // 8), dtype=torch.int32, device=device)
+        w13s = torch.empty((E, 2 * I, H // 32), dtype=torch.bfloat16, device=device)
+        w2q = torch.empty((E, H, I // 8), dtype=torch.int32, device=device)
+        w2s = torch.empty((E, H, I // 32), dtype=torch.bfloat16, device=device)
+        for e in range(E):
+            g = generator(wl.wid, _W13, e, device=device)
+            w13q[e], w13s[e] = quantize_w4_group32(torch.randn((2 * I, H), generator=g, device=device) * 0.02)
+            g = generator(wl.wid, _W2, e, device=device)
+            w2q[e], w2s[e] = quantize_w4_group32(torch.randn((H, I), generator=g, device=device) * 0.02)
+        d.update(w13q=w13q, w13s=w13s, w2q=w2q, w2s=w2s)
+    elif wl.kind == "fp8":
+        w13 = torch.empty((E, 2 * I, H), dtype=torch.uint8, device=device)
+        w13s = torch.empty((E, 2 * I // 128, H // 128), dtype=torch.float32, device=device)
+        w2 = torch.empty((E, H, I), dtype=torch.uint8, device=device)
+        w2s = torch.empty((E, H // 128, I // 128), dtype=torch.float32, device=device)
+        for e in range(E):
+            g = generator(wl.wid, _W13, e, device=device)
+            w13[e], w13s[e] = quantize_fp8_blocks(torch.randn((2 * I, H), generator=g, device=device) * 0.02)
+            g = generator(wl.wid, _W2, e, device=device)
+            w2[e], w2s[e] = quantize_fp8_blocks(torch.randn((H, I), generator=g, device=device) * 0.02)
+        d.update(w13=w13, w13s=w13s, w2=w2, w2s=w2s)
+    else:
+        raise ValueError(wl.kind)
+    return d
+
+
+def make_dense_fp8(wl: Workload, M: int, device="cpu", N=None, K=None):
+    """A (quantized per row and 128-group) [M, K] and B (block-quantized) [N, K]. Rows of A do not
+    depend on M: A for M rows is the first M rows of the largest draw."""
+    N = wl.N if N is None else N
+    K = wl.K if K is None else K
+    Mmax = max(M, max(wl.M_list) if wl.M_list else M)
+    a = bf16_normal((Mmax, K), generator(wl.wid, _A, device=device), device)[:M].float()
+    Aq, As = quantize_fp8_rows(a)
+    gb = generator(wl.wid, _B, device=device)
+    Bq, Bs = quantize_fp8_blocks(torch.randn((N, K), generator=gb, device=device) * 0.02)
+    return dict(A=Aq, As=As, B=Bq, Bs=Bs, M=M, N=N, K=K)
+
+
+def np_bits(t: torch.Tensor) -> np.ndarray:
+    """Host numpy view of a tensor's raw storage: bf16 -> uint16, everything else as is."""
+    t = t.detach().contiguous().cpu()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).numpy().view(np.uint16)
+    return t.numpy()
+
+
+def moe_flops(T: int, k: int, H: int, I: int) -> float:
+    """Algorithmic FLOPs of the layer: 2 per multiply-add of gate/up (N=2I, K=H) and of down
+    (N=H, K=I), over the T*k routed rows (padding excluded)."""
+    return 2.0 * T * k * (2 * I * H + H * I)
+
+
+def w4a16_expert_bytes(H: int, I: int) -> int:
+    """Packed codes + bf16 scales of one expert's gate/up and down matrices."""
+    return (2 * I * H) // 2 + (2 * I * H // 32) * 2 + (H * I) // 2 + (H * I // 32) * 2
+
+
+def fp8_expert_bytes(H: int, I: int) -> int:
+    return 2 * I * H + (2 * I // 128) * (H // 128) * 4 + H * I + (H // 128) * (I // 128) * 4
+
+
+def cdiv(a: int, b: int) -> int:
+    return -(-a // b)
+
+
+__all__ = ["WORKLOADS", "Workload", "make_moe", "make_dense_fp8", "np_bits", "moe_flops",
+           "w4a16_expert_bytes", "fp8_expert_bytes", "router_logits", "cdiv", "math"]
