@@ -1,0 +1,447 @@
+"""Benchmark of the routed, weight-quantized MoE expert layer on B200.
+
+Headline (one JSON line on rank 0): the decode W4A16 layer (T=32 tokens, H=7168, I=2048,
+E=384 experts, top-8, INT4 group-32 weights with bf16 scales), one step = one full layer forward
+(route, align, gate/up + SiLU*up, down + routing weight, combine) through the C ABI.
+  value  = weight bytes of the experts the step touches / device time per step (GB/s)
+  e2e    = the same with the step's input copied from pinned host memory and its output read back
+           inside the timed region
+  roofline = the dominant kernel (gate/up) against the measured HBM copy bandwidth
+The same line carries the prefill W4A16 layer (T=8192, Zipf-skewed routing), the block-FP8 MoE
+layer (T=4096, E=256) and the dense block-FP8 matmul sweep as secondary measurements.
+
+--impl reference times the CPU oracle (oracle/, the one other consumer allowed here) on a bounded
+sample of the same workload, on the host cores. Multi-GPU (--gpus N under torchrun): independent
+replicas, one per rank, no collective on the data path ("replicas only"); value is the sum over
+ranks of bytes / the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "MoE layer TFLOP/s + weight GB/s vs roofline (decode T=32, prefill T=8192)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------------------------
+# distributed plumbing (replicas only)
+# ---------------------------------------------------------------------------------------------
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", str(self.dev)], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        loaded = [v for v in sm if mx is None or v >= 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------------------------
+# timing helpers
+# ---------------------------------------------------------------------------------------------
+
+def timed_steps(fn, steps, warmup, flush=None, world=1):
+    """Device time per step (ms): CUDA events around each step on the current stream, L2 flushed
+    between steps outside the events; barrier + synchronize on both sides."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in evs:
+        if flush is not None:
+            flush()
+        a.record()
+        fn()
+        b.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def src_sha(*names):
+    h = hashlib.sha256()
+    for n in names:
+        h.update(open(os.path.join(ROOT, "quantized_mixture_experts_align_b200", "csrc", n), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(key, sha):
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(key)
+    if not d or d.get("src_sha") != sha:
+        return None
+    return d.get("bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------------------------
+# workloads
+# ---------------------------------------------------------------------------------------------
+
+def touched_experts(moeq, d):
+    ids, _ = moeq.moe_route_topk(d["logits"], d["k"])
+    return int(torch.unique(ids).numel())
+
+
+def run_w4a16(moeq, d, steps, warmup, flush, world, trace=False):
+    out = torch.empty((d["T"], d["H"]), dtype=torch.bfloat16, device="cuda")
+    ws = moeq.workspace(moeq.moe_w4a16_workspace_size(d["T"], d["H"], d["I"], d["E"], d["k"]), "cuda")
+
+    def step():
+        moeq.moe_w4a16_forward(d["x"], d["logits"], d["k"], d["w13q"], d["w13s"], d["w2q"], d["w2s"], out=out, ws=ws)
+
+    if trace:
+        for _ in range(warmup):
+            step()
+        torch.cuda.synchronize()
+        moeq.moe_trace_read(reset=True)
+        moeq.moe_trace_enable(True)
+    ms = timed_steps(step, steps, 0 if trace else warmup, flush, world)
+    stages = None
+    if trace:
+        moeq.moe_trace_enable(False)
+        stages = moeq.moe_trace_read(reset=True)
+    return ms, stages, out
+
+
+def run_fp8(moeq, d, steps, warmup, flush, world):
+    out = torch.empty((d["T"], d["H"]), dtype=torch.bfloat16, device="cuda")
+    ws = moeq.workspace(moeq.moe_w8a8_block_fp8_workspace_size(d["T"], d["H"], d["I"], d["E"], d["k"]), "cuda")
+
+    def step():
+        moeq.moe_w8a8_block_fp8_forward(d["x"], d["logits"], d["k"], d["w13"], d["w13s"], d["w2"], d["w2s"], out=out,
+                                        ws=ws)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    moeq.moe_trace_read(reset=True)
+    moeq.moe_trace_enable(True)
+    ms = timed_steps(step, steps, 0, flush, world)
+    moeq.moe_trace_enable(False)
+    return ms, moeq.moe_trace_read(reset=True)
+
+
+def e2e_w4a16(moeq, d, steps, warmup, world):
+    """Same layer through the C ABI with the step's inputs in pinned host memory: H2D of x and
+    the router logits, the forward, D2H of the output, all inside the timed region."""
+    hx = d["x"].cpu().pin_memory()
+    hl = d["logits"].cpu().pin_memory()
+    hout = torch.empty((d["T"], d["H"]), dtype=torch.bfloat16).pin_memory()
+    dx = torch.empty_like(d["x"])
+    dl = torch.empty_like(d["logits"])
+    out = torch.empty((d["T"], d["H"]), dtype=torch.bfloat16, device="cuda")
+    ws = moeq.workspace(moeq.moe_w4a16_workspace_size(d["T"], d["H"], d["I"], d["E"], d["k"]), "cuda")
+
+    def step():
+        dx.copy_(hx, non_blocking=True)
+        dl.copy_(hl, non_blocking=True)
+        moeq.moe_w4a16_forward(dx, dl, d["k"], d["w13q"], d["w13s"], d["w2q"], d["w2s"], out=out, ws=ws)
+        hout.copy_(out, non_blocking=True)
+
+    ms = timed_steps(step, steps, warmup, None, world)
+    h2d = hx.numel() * hx.element_size() + hl.numel() * hl.element_size()
+    d2h = hout.numel() * hout.element_size()
+    return ms, h2d, d2h
+
+
+def oracle_sample_time(d, ntok):
+    """Seconds the CPU oracle takes for `ntok` tokens of the workload (host copies excluded)."""
+    import oracle
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from tests._util import host_moe_weights
+    x = W.np_bits(d["x"])
+    logits = W.np_bits(d["logits"])
+    toks = np.arange(ntok, dtype=np.int32)
+    ids, _ = oracle.route_topk(logits[:ntok], d["k"])
+    hw = host_moe_weights(d, ids.ravel())
+    t0 = time.perf_counter()
+    if d["kind"] == "w4a16":
+        oracle.moe_w4a16(x, logits, d["k"], hw["w13q"], hw["w13s"], hw["w2q"], hw["w2s"], tokens=toks)
+    else:
+        oracle.moe_fp8(x, logits, d["k"], hw["w13"], hw["w13s"], hw["w2"], hw["w2s"], tokens=toks)
+    return time.perf_counter() - t0
+
+
+def cpu_info():
+    model = ""
+    try:
+        for ln in open("/proc/cpuinfo"):
+            if ln.startswith("model name"):
+                model = ln.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    return model
+
+
+# ---------------------------------------------------------------------------------------------
+# arms
+# ---------------------------------------------------------------------------------------------
+
+def reference_arm(args, rank, world):
+    """The CPU oracle, as it stands, on a bounded sample of the decode workload per step."""
+    if rank != 0:
+        return
+    import oracle
+    wl = W.WORKLOADS["decode_w4a16"]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    d = W.make_moe(wl, device=dev)
+    T = d["T"]
+    n_active = int(np.unique(oracle.route_topk(W.np_bits(d["logits"]), d["k"])[0]).size)
+    gbytes = n_active * W.w4a16_expert_bytes(d["H"], d["I"]) / 1e9
+    ntok = 1
+    for _ in range(args.warmup):
+        oracle_sample_time(d, ntok)
+    times = [oracle_sample_time(d, ntok) for _ in range(args.steps)]
+    step_s = statistics.mean(times) * T / ntok          # extrapolated full step
+    value = gbytes / step_s
+    cores = oracle.threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "decode_w4a16 T=32 H=7168 I=2048 E=384 k=8 (INT4 group-32, bf16 scales)"},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{ntok} of {T} tokens per step, time x{T // ntok}; host CPU: {cpu_info()}"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="moeq", choices=["moeq", "reference"])
+    ap.add_argument("--headline-only", action="store_true", help="skip the secondary workloads")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    rank, world, local = dist_setup(args.gpus)
+    if args.impl == "reference":
+        reference_arm(args, rank, world)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+
+    import quantized_mixture_experts_align_b200 as moeq
+    moeq.lib()
+    peaks, peak_src = load_peaks()
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+
+    def flush():
+        flush_buf.fill_(1)
+
+    # ---- headline: decode W4A16 -----------------------------------------------------------
+    d = W.make_moe(W.WORKLOADS["decode_w4a16"], device="cuda")
+    n_active = touched_experts(moeq, d)
+    w13_bytes = W.w4a16_expert_bytes(d["H"], d["I"]) * 2 // 3
+    step_bytes = n_active * W.w4a16_expert_bytes(d["H"], d["I"])
+    flops = W.moe_flops(d["T"], d["k"], d["H"], d["I"])
+    dev_index = torch.cuda.current_device()
+    with ClockSampler(dev_index) as clk:
+        ms, stages, _ = run_w4a16(moeq, d, args.steps, args.warmup, flush, world, trace=True)
+    ms_step = max_over_ranks(statistics.mean(ms), world)
+    value = world * step_bytes / (ms_step * 1e-3) / 1e9
+    gu_ms, gu_calls = stages["gate_up"]
+    gu_avg = gu_ms / max(gu_calls, 1)
+    gu_bytes = n_active * (d["H"] * 2 * d["I"] // 2 + d["H"] // 32 * 2 * d["I"] * 2)
+    achieved = gu_bytes / (gu_avg * 1e-3) / 1e9
+    sha = src_sha("w4a16_mma.cu", "common.cuh")
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": traffic_for("w4a16_gate_up_decode", sha),
+                "kernel": "w4a16_grouped_mma_kernel<8,4,GATEUP> (gate/up + SiLU*up)",
+                "algorithmic_bytes_per_launch": gu_bytes, "launch_ms": gu_avg,
+                "peak_source": f"{peak_src} hbm_gbs (copy)"}
+    del w13_bytes
+
+    e2e_ms, h2d, d2h = e2e_w4a16(moeq, d, args.steps, args.warmup, world)
+    e2e_step = max_over_ranks(statistics.mean(e2e_ms), world)
+    e2e = {"value": world * step_bytes / (e2e_step * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "ms_per_step": e2e_step}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "decode_w4a16 T=32 H=7168 I=2048 E=384 k=8 (INT4 group-32, bf16 scales)",
+                   "touched_experts": n_active, "weight_bytes_per_step": step_bytes,
+                   "l2": f"flushed between steps ({L2_FLUSH_BYTES >> 20} MB write), outside the timed events",
+                   "parallelism": f"replicas x{world}"},
+        "tflops": world * flops / (ms_step * 1e-3) / 1e12,
+        "roofline": roofline,
+        "stages_ms": {k: v[0] / max(v[1], 1) for k, v in stages.items() if v[1]},
+        "e2e": e2e,
+        "gpu_launches": 5 * args.steps,
+    }
+
+    # ---- secondary workloads -----------------------------------------------------------------
+    if not args.headline_only:
+        also = {}
+        dp = W.make_moe(W.WORKLOADS["prefill_w4a16"], device="cuda")
+        pms, pst, _ = run_w4a16(moeq, dp, max(3, args.steps // 4), 3, None, world, trace=True)
+        pflops = W.moe_flops(dp["T"], dp["k"], dp["H"], dp["I"])
+        pstep = max_over_ranks(statistics.mean(pms), world)
+        also["prefill_w4a16"] = {
+            "workload": "T=8192 H=7168 I=2048 E=384 k=8, Zipf-biased routing", "ms_per_step": pstep,
+            "tflops": pflops / (pstep * 1e-3) / 1e12,
+            "frac_of_bf16_peak": pflops / (pstep * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"],
+            "peak_tflops": peaks["bf16_tflops_sustained"], "peak_source": f"{peak_src} bf16 sustained",
+            "stages_ms": {k: v[0] / max(v[1], 1) for k, v in pst.items() if v[1]}}
+        del dp
+        torch.cuda.empty_cache()
+        df = W.make_moe(W.WORKLOADS["moe_fp8"], device="cuda")
+        fms, fst = run_fp8(moeq, df, max(3, args.steps // 4), 3, None, world)
+        fflops = W.moe_flops(df["T"], df["k"], df["H"], df["I"])
+        fstep = max_over_ranks(statistics.mean(fms), world)
+        fp8_peak = 2.0 * peaks["bf16_tflops_sustained"]
+        also["moe_fp8"] = {
+            "workload": "T=4096 H=7168 I=2048 E=256 k=8, block-FP8 [128,128], Zipf-biased routing",
+            "ms_per_step": fstep, "tflops": fflops / (fstep * 1e-3) / 1e12,
+            "frac_of_fp8_peak": fflops / (fstep * 1e-3) / 1e12 / fp8_peak,
+            "peak_tflops": fp8_peak, "peak_source": f"2 x {peak_src} bf16 sustained (nominal fp8/bf16 ratio)",
+            "stages_ms": {k: v[0] / max(v[1], 1) for k, v in fst.items() if v[1]}}
+        del df
+        torch.cuda.empty_cache()
+        sweep = {}
+        wl = W.WORKLOADS["dense_fp8"]
+        for M in wl.M_list:
+            dd = W.make_dense_fp8(wl, M, device="cuda")
+            C = torch.empty((M, wl.N), dtype=torch.bfloat16, device="cuda")
+            fn = lambda: moeq.w8a8_block_fp8_matmul(dd["A"], dd["As"], dd["B"], dd["Bs"], out=C)
+            dms = statistics.mean(timed_steps(fn, max(3, args.steps // 4), 3, flush, world))
+            byts = wl.N * wl.K + dd["Bs"].numel() * 4 + M * wl.K + M * (wl.K // 128) * 4 + 2 * M * wl.N
+            fl = 2.0 * M * wl.N * wl.K
+            sweep[M] = {"ms": dms, "tflops": fl / (dms * 1e-3) / 1e12, "gbs": byts / (dms * 1e-3) / 1e9,
+                        "hbm_frac": byts / (dms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                        "fp8_frac": fl / (dms * 1e-3) / 1e12 / (2.0 * peaks["bf16_tflops"])}
+            del dd, C
+        also["dense_fp8_sweep"] = {"workload": "A [M,7168] x B [24576,7168] block-FP8, C bf16", "by_M": sweep}
+        line["also"] = also
+
+    line["clocks"] = clk.summary()
+
+    # ---- CPU baseline: the oracle as it stands, bounded sample, rank 0 only --------------------
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        ntok = 1
+        t_s = oracle_sample_time(d, ntok)
+        full_s = t_s * d["T"] / ntok
+        line["cpu_baseline"] = {"value": step_bytes / full_s / 1e9, "unit": "GB/s", "cores": oracle.threads(),
+                                "kind": "oracle",
+                                "sample": f"{ntok} of {d['T']} decode tokens timed ({t_s:.1f} s), scaled x{d['T']}; "
+                                          f"host CPU: {cpu_info()}"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

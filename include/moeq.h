@@ -1,0 +1,168 @@
+/*
+ * moeq — routed Mixture-of-Experts expert layer with quantized weights, for NVIDIA B200 (sm_100a).
+ *
+ * C ABI of libmoeq.so. Plain pointers and sizes only.
+ *
+ * Conventions for every entry point below:
+ *  - Pointers to tensors are caller-owned DEVICE memory (cudaMalloc, a torch CUDA tensor, ...).
+ *    The library never allocates, frees or keeps a pointer past the call. Scratch memory comes
+ *    from the caller through `ws` / `ws_bytes`, sized by the matching *_workspace_size().
+ *  - All tensors are dense, row-major, contiguous. bf16 values are passed as uint16_t bit
+ *    patterns, E4M3 ("fn" variant: max 448, no infinities) values as uint8_t bit patterns.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream). Every call only
+ *    enqueues work on that stream and returns; no call synchronizes with the host or reads
+ *    device data back, so a sequence of calls can be captured in a CUDA graph.
+ *  - Status: 0 on success, else one of the MOEQ_ERR_* codes; the calling thread's last error
+ *    message is available from moe_last_error(). Arguments are validated on the host before
+ *    anything is enqueued; a rejected call enqueues nothing. No C++ exception crosses the ABI.
+ *  - Device data must satisfy the documented value ranges (e.g. expert ids in [0, E)); kernels
+ *    skip out-of-range ids instead of writing out of bounds.
+ *
+ * Sources, cited by page title and section:
+ *  [CHORD] "vLLM x Novita AI: Chord W4A16 INT4 MoE Kernel for Kimi K2.x" (Novita blog).
+ *  [SGL]   "SGLang W8A8 Block FP8 quantized kernel config files: analysis and tuning guide"
+ *          (xdnf.cn article on SGLang's fp8_kernel.py).
+ */
+#ifndef MOEQ_H
+#define MOEQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOEQ_API __attribute__((visibility("default")))
+#else
+#define MOEQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOEQ_OK 0
+#define MOEQ_ERR_INVALID_ARG 1    /* null pointer, negative or inconsistent size */
+#define MOEQ_ERR_UNSUPPORTED 2    /* shape, alignment or quantization scheme this library does not run */
+#define MOEQ_ERR_WORKSPACE 3      /* ws_bytes smaller than the matching *_workspace_size() */
+#define MOEQ_ERR_CUDA 4           /* a CUDA launch or API call failed (message has the CUDA error) */
+#define MOEQ_ERR_DEVICE_TIMEOUT 5 /* a kernel gave up a bounded wait (reported by moe_device_status) */
+
+/* Message of the calling thread's last failed call ("" if none). Valid until the next call. */
+MOEQ_API const char *moe_last_error(void);
+
+/* Library version string. */
+MOEQ_API const char *moe_version(void);
+
+/*
+ * Top-k softmax routing, renormalised over the selected experts ([CHORD], "vLLM integration":
+ * the layer consumes routing produced upstream; the definition taken is softmax over the E
+ * logits, keep the k largest, divide by their sum).
+ *   logits   f32 [T, E], finite values
+ *   topk_ids i32 [T, k] out: expert of slot (t, j), in (logit descending, index ascending) order
+ *   topk_w   f32 [T, k] out: exp(l - l_max) / sum over the k selected, computed in double
+ * Limits: 1 <= k <= 32, k <= E <= 1024, T >= 0.
+ */
+MOEQ_API int moe_route_topk(const float *logits, int T, int E, int k, int32_t *topk_ids, float *topk_w,
+                   void *stream);
+
+/*
+ * Token-to-expert alignment ([CHORD], "Two kernel families": the indexed kernels consume
+ * sorted_ids / expert_ids / num_tokens_padded; figure 3: padding guards live in the indices,
+ * activations are not padded; "vLLM integration": buffers are over-allocated so that no host
+ * read of the routed count is needed).
+ *   topk_ids  i32 [T, k], values in [0, E)
+ *   sorted_ids i32 [T*k + E*(block_m-1)] out: for experts in ascending order, the flat slots
+ *              f = t*k + j routed to it in ascending f, padded with the value T*k to a multiple
+ *              of block_m; entries past num_tokens_padded also hold T*k
+ *   expert_ids i32 [ceil((T*k + E*(block_m-1)) / block_m)] out: expert of each block of
+ *              block_m entries, -1 past num_tokens_padded
+ *   num_tokens_padded i32 [1] out: sum over experts of ceil(count / block_m) * block_m
+ * Bit-exact (integer). Limits: 1 <= block_m <= 256, E <= 1024, T*k <= 2^24.
+ */
+MOEQ_API int moe_align(const int32_t *topk_ids, int T, int k, int E, int block_m, int32_t *sorted_ids,
+              int32_t *expert_ids, int32_t *num_tokens_padded, void *stream);
+
+/*
+ * Per-token, per-128-column-group FP8 quantization of activations ([SGL], "Background": As is
+ * the per token-group quantization scale matrix of the activations):
+ *   s = max(max|x_group|, 1e-10) / 448 (IEEE f32 division), q = E4M3(x / s) rounded to nearest
+ *   even with saturation to +-448.
+ *   x bf16 [rows, cols]; q e4m3 [rows, cols] out; s f32 [rows, cols/128] out. cols % 128 == 0.
+ */
+MOEQ_API int moe_fp8_act_quant(const uint16_t *x, int rows, int cols, uint8_t *q, float *s, void *stream);
+
+/*
+ * W4A16 routed expert layer ([CHORD], "vLLM integration": uint4 codes, group 32, BF16 scales,
+ * the pack-quantized INT4 group-32 checkpoint shape; "SM90 grouped kernels": codes [G, N, K],
+ * scales [G, N, K/32]):
+ *   out[t] = sum_j topk_w[t, j] * W2[e_j] . bf16( silu(W13_gate[e_j] . x[t]) * (W13_up[e_j] . x[t]) )
+ *   x      bf16 [T, H]
+ *   logits f32 [T, E] (routing is computed inside, as moe_route_topk)
+ *   w13_q  i32 [E, 2I, H/8]  codes of the fused gate (rows [0, I)) and up (rows [I, 2I))
+ *          projections; nibble j of word w holds input column 8w + j in bits [4j, 4j+4); the
+ *          value of code q is (q - 8) * scale
+ *   w13_s  bf16 [E, 2I, H/32] one scale per 32 consecutive input columns
+ *   w2_q   i32 [E, H, I/8], w2_s bf16 [E, H, I/32]  down projection, same format
+ *   out    bf16 [T, H] out
+ *   topk_ids_out i32 [T, k], topk_w_out f32 [T, k]: optional (may be NULL) copies of the routing
+ *   ws     scratch of at least moe_w4a16_workspace_size(T, H, I, E, k) bytes, 256-byte aligned
+ * Limits: H % 128 == 0, I % 128 == 0, 1 <= k <= 32, k <= E <= 1024, T >= 0.
+ */
+MOEQ_API size_t moe_w4a16_workspace_size(int T, int H, int I, int E, int k);
+MOEQ_API int moe_w4a16_forward(const uint16_t *x, const float *logits, int T, int H, int I, int E, int k,
+                      const int32_t *w13_q, const uint16_t *w13_s, const int32_t *w2_q,
+                      const uint16_t *w2_s, uint16_t *out, int32_t *topk_ids_out,
+                      float *topk_w_out, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * W8A8 block-FP8 routed expert layer ([SGL], "Background": E4M3 weights with one f32 scale per
+ * [128, 128] block, activations E4M3 with one f32 scale per token and 128-column group):
+ *   the input is quantized as moe_fp8_act_quant; g, u = block-scaled products with W13[e];
+ *   a = silu(g) * u is quantized the same way per slot and 128-column group; y = block-scaled
+ *   product with W2[e]; out[t] = sum_j topk_w[t, j] * y_j.
+ *   w13 e4m3 [E, 2I, H], w13_s f32 [E, 2I/128, H/128]; w2 e4m3 [E, H, I], w2_s f32 [E, H/128, I/128]
+ *   other arguments as moe_w4a16_forward.
+ * Limits: H % 128 == 0, I % 128 == 0, 1 <= k <= 32, k <= E <= 1024.
+ */
+MOEQ_API size_t moe_w8a8_block_fp8_workspace_size(int T, int H, int I, int E, int k);
+MOEQ_API int moe_w8a8_block_fp8_forward(const uint16_t *x, const float *logits, int T, int H, int I, int E,
+                               int k, const uint8_t *w13, const float *w13_s, const uint8_t *w2,
+                               const float *w2_s, uint16_t *out, int32_t *topk_ids_out,
+                               float *topk_w_out, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Dense block-FP8 matmul ([SGL], "Background": w8a8_block_fp8_matmul(A, B, As, Bs, block_size,
+ * output_dtype)):  C[m, n] = sum_kb As[m, kb] * Bs[n/128, kb] * sum_{k in block kb} A[m,k] B[n,k]
+ *   A e4m3 [M, K], As f32 [M, K/128], B e4m3 [N, K], Bs f32 [ceil(N/128), ceil(K/128)],
+ *   C bf16 [M, N] out. block_n and block_k must both be 128 ([SGL], "Config directory & naming":
+ *   almost every entry uses block_shape [128, 128]); K % 128 == 0, N % 128 == 0
+ *   (the page's shape check: ceil(N/block_n) == rows of Bs, ceil(K/block_k) == columns of Bs).
+ */
+MOEQ_API int w8a8_block_fp8_matmul(const uint8_t *A, const float *As, const uint8_t *B, const float *Bs,
+                          int M, int N, int K, int block_n, int block_k, uint16_t *C, void *stream);
+
+/*
+ * Stage tracing, a diagnostic that is off by default. While enabled, every forward / matmul call
+ * brackets each of its kernel stages with a pair of CUDA events recorded on the call's stream
+ * (the library creates the events on first use, on the current device; do not enable tracing
+ * during stream capture). moe_trace_read() waits for the recorded events, adds their durations
+ * to per-stage totals and writes the first min(n_stages, 7) totals (milliseconds) and call
+ * counts (either pointer may be NULL); it returns 7, the number of stages, or MOEQ_ERR_CUDA.
+ * `reset` != 0 clears the totals after reading. Stage indices: 0 route_topk, 1 align,
+ * 2 fp8_act_quant, 3 gate_up (with SiLU*up), 4 down (with the routing weight), 5 combine,
+ * 6 dense block-FP8 matmul.
+ */
+MOEQ_API int moe_trace_enable(int enable);
+MOEQ_API int moe_trace_read(double *stage_ms, long long *stage_calls, int n_stages, int reset);
+
+/*
+ * Sticky device status of the library's kernels on the current device: 0 if no kernel has
+ * reported a problem, else MOEQ_ERR_DEVICE_TIMEOUT. This call synchronizes with the device (it
+ * is a diagnostic, not part of the forward path); `clear` != 0 resets the status.
+ */
+MOEQ_API int moe_device_status(int clear);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOEQ_H */

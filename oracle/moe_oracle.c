@@ -304,6 +304,18 @@ int orc_moe_w4a16(const uint16_t *x, const float *logits, int T, int H, int I, i
 /* The W8A8 block-FP8 expert layer, for a chosen list of tokens                                */
 /* ------------------------------------------------------------------------------------------ */
 
+/* Decoded E4M3 values, filled from e4m3_value() before any parallel region (a cache of the
+ * decoder above, so the inner loops do not call ldexp). */
+static double e4m3_table[256];
+static int e4m3_table_ready = 0;
+
+static void e4m3_table_init(void)
+{
+    if (e4m3_table_ready) return;
+    for (int c = 0; c < 256; ++c) e4m3_table[c] = e4m3_value((uint8_t)c);
+    e4m3_table_ready = 1;
+}
+
 /* Block-scaled dot product of one activation row and one weight row over K ([SGL],
  * "Background": each [BLOCK_N, BLOCK_K] = [128, 128] weight block has its own scale, the
  * activations one scale per token and 128-column group):
@@ -313,7 +325,7 @@ static double fp8_row_dot(const uint8_t *a, const float *as, const uint8_t *b, c
     double acc = 0.0;
     for (int kb = 0; kb < K / 128; ++kb) {
         double part = 0.0;
-        for (int c = kb * 128; c < kb * 128 + 128; ++c) part += e4m3_value(a[c]) * e4m3_value(b[c]);
+        for (int c = kb * 128; c < kb * 128 + 128; ++c) part += e4m3_table[a[c]] * e4m3_table[b[c]];
         acc += (double)as[kb] * (double)bs[kb] * part;
     }
     return acc;
@@ -332,6 +344,7 @@ int orc_moe_fp8(const uint16_t *x, const float *logits, int T, int H, int I, int
     if (H % 128 || I % 128 || H < 128 || I < 128 || k < 1 || k > E) return 1;
     for (int i = 0; i < ntok; ++i)
         if (tokens[i] < 0 || tokens[i] >= T) return 1;
+    e4m3_table_init();
     int32_t *ids = (int32_t *)malloc(sizeof(int32_t) * (size_t)k);
     float *w = (float *)malloc(sizeof(float) * (size_t)k);
     uint8_t *xq = (uint8_t *)malloc((size_t)H);
@@ -385,6 +398,7 @@ int orc_fp8_block_matmul(const uint8_t *A, const float *As, const uint8_t *B, co
     for (int i = 0; i < nrows; ++i)
         if (rows[i] < 0 || rows[i] >= M) return 1;
     int KB = K / 128;
+    e4m3_table_init();
 #pragma omp parallel for collapse(2) schedule(static)
     for (int i = 0; i < nrows; ++i)
         for (int n = 0; n < N; ++n) {

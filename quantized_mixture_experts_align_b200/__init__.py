@@ -1,0 +1,202 @@
+"""Python binding of libmoeq.so, the sm_100a library for the routed, weight-quantized
+Mixture-of-Experts expert layer. Every function has the name of the C entry point it calls
+(declared in include/moeq.h) and only marshals arguments: torch CUDA tensors in, their device
+pointers and sizes to the C ABI, the status checked. All computation runs in the library's CUDA
+kernels; there is no CPU or PyTorch fallback - a missing library or a non-CUDA tensor raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmoeq.so")
+
+MOEQ_OK, MOEQ_ERR_INVALID_ARG, MOEQ_ERR_UNSUPPORTED, MOEQ_ERR_WORKSPACE, MOEQ_ERR_CUDA, MOEQ_ERR_DEVICE_TIMEOUT = range(6)
+
+
+class MoeqError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"moeq error {code}: {msg}")
+        self.code = code
+
+
+_lib = None
+
+_V, _I, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+_SIGNATURES = {
+    "moe_last_error": ([], ctypes.c_char_p),
+    "moe_version": ([], ctypes.c_char_p),
+    "moe_route_topk": ([_V, _I, _I, _I, _V, _V, _V], _I),
+    "moe_align": ([_V, _I, _I, _I, _I, _V, _V, _V, _V], _I),
+    "moe_fp8_act_quant": ([_V, _I, _I, _V, _V, _V], _I),
+    "moe_w4a16_workspace_size": ([_I, _I, _I, _I, _I], _Z),
+    "moe_w4a16_forward": ([_V, _V, _I, _I, _I, _I, _I, _V, _V, _V, _V, _V, _V, _V, _V, _Z, _V], _I),
+    "moe_w8a8_block_fp8_workspace_size": ([_I, _I, _I, _I, _I], _Z),
+    "moe_w8a8_block_fp8_forward": ([_V, _V, _I, _I, _I, _I, _I, _V, _V, _V, _V, _V, _V, _V, _V, _Z, _V], _I),
+    "w8a8_block_fp8_matmul": ([_V, _V, _V, _V, _I, _I, _I, _I, _I, _V, _V], _I),
+    "moe_trace_enable": ([_I], _I),
+    "moe_trace_read": ([_V, _V, _I, _I], _I),
+    "moe_device_status": ([_I], _I),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmoeq.so (built in-tree by build.py). Raises if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is not built; run quantized_mixture_experts_align_b200/build.py")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = L
+    return _lib
+
+
+def exported_symbols() -> list[str]:
+    return list(_SIGNATURES)
+
+
+def _check(rc: int):
+    if rc != MOEQ_OK:
+        raise MoeqError(rc, lib().moe_last_error().decode())
+
+
+def _dev(t: torch.Tensor | None, name: str, dtype=None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise ValueError(f"{name} must have dtype {dtype}, got {t.dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+_BF16 = (torch.bfloat16, torch.int16, torch.uint16)
+_U8 = (torch.uint8, torch.float8_e4m3fn)
+
+
+def version() -> str:
+    return lib().moe_version().decode()
+
+
+def moe_route_topk(logits: torch.Tensor, k: int, topk_ids=None, topk_w=None, stream=None):
+    T, E = logits.shape
+    topk_ids = torch.empty((T, k), dtype=torch.int32, device=logits.device) if topk_ids is None else topk_ids
+    topk_w = torch.empty((T, k), dtype=torch.float32, device=logits.device) if topk_w is None else topk_w
+    _check(lib().moe_route_topk(_dev(logits, "logits", torch.float32), T, E, k, _dev(topk_ids, "topk_ids", torch.int32),
+                                _dev(topk_w, "topk_w", torch.float32), _stream(stream)))
+    return topk_ids, topk_w
+
+
+def moe_align(topk_ids: torch.Tensor, E: int, block_m: int, stream=None):
+    T, k = topk_ids.shape
+    cap = T * k + E * (block_m - 1)
+    dev = topk_ids.device
+    sorted_ids = torch.empty(cap, dtype=torch.int32, device=dev)
+    expert_ids = torch.empty(-(-cap // block_m), dtype=torch.int32, device=dev)
+    ntp = torch.empty(1, dtype=torch.int32, device=dev)
+    _check(lib().moe_align(_dev(topk_ids, "topk_ids", torch.int32), T, k, E, block_m, _dev(sorted_ids, "sorted_ids"),
+                           _dev(expert_ids, "expert_ids"), _dev(ntp, "ntp"), _stream(stream)))
+    return sorted_ids, expert_ids, ntp
+
+
+def moe_fp8_act_quant(x: torch.Tensor, stream=None):
+    rows, cols = x.shape
+    q = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+    s = torch.empty((rows, cols // 128), dtype=torch.float32, device=x.device)
+    _check(lib().moe_fp8_act_quant(_dev(x, "x", _BF16), rows, cols, _dev(q, "q"), _dev(s, "s"), _stream(stream)))
+    return q, s
+
+
+def moe_w4a16_workspace_size(T: int, H: int, I: int, E: int, k: int) -> int:
+    return int(lib().moe_w4a16_workspace_size(T, H, I, E, k))
+
+
+def moe_w8a8_block_fp8_workspace_size(T: int, H: int, I: int, E: int, k: int) -> int:
+    return int(lib().moe_w8a8_block_fp8_workspace_size(T, H, I, E, k))
+
+
+def workspace(nbytes: int, device) -> torch.Tensor:
+    """A device scratch buffer for the *_forward calls (torch allocations are 256-byte aligned)."""
+    return torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device)
+
+
+def moe_w4a16_forward(x, logits, k, w13_q, w13_s, w2_q, w2_s, out=None, ws=None, topk_ids_out=None,
+                      topk_w_out=None, stream=None):
+    T, H = x.shape
+    E = logits.shape[1]
+    I = w2_q.shape[2] * 8
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device) if out is None else out
+    need = moe_w4a16_workspace_size(T, H, I, E, k)
+    ws = workspace(need, x.device) if ws is None else ws
+    _check(lib().moe_w4a16_forward(
+        _dev(x, "x", _BF16), _dev(logits, "logits", torch.float32), T, H, I, E, k,
+        _dev(w13_q, "w13_q", torch.int32), _dev(w13_s, "w13_s", _BF16), _dev(w2_q, "w2_q", torch.int32),
+        _dev(w2_s, "w2_s", _BF16), _dev(out, "out", _BF16), _dev(topk_ids_out, "topk_ids_out", torch.int32),
+        _dev(topk_w_out, "topk_w_out", torch.float32), _dev(ws, "ws"), ws.numel() * ws.element_size(),
+        _stream(stream)))
+    return out
+
+
+def moe_w8a8_block_fp8_forward(x, logits, k, w13, w13_s, w2, w2_s, out=None, ws=None, topk_ids_out=None,
+                               topk_w_out=None, stream=None):
+    T, H = x.shape
+    E = logits.shape[1]
+    I = w2.shape[2]
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device) if out is None else out
+    need = moe_w8a8_block_fp8_workspace_size(T, H, I, E, k)
+    ws = workspace(need, x.device) if ws is None else ws
+    _check(lib().moe_w8a8_block_fp8_forward(
+        _dev(x, "x", _BF16), _dev(logits, "logits", torch.float32), T, H, I, E, k,
+        _dev(w13, "w13", _U8), _dev(w13_s, "w13_s", torch.float32), _dev(w2, "w2", _U8),
+        _dev(w2_s, "w2_s", torch.float32), _dev(out, "out", _BF16), _dev(topk_ids_out, "topk_ids_out", torch.int32),
+        _dev(topk_w_out, "topk_w_out", torch.float32), _dev(ws, "ws"), ws.numel() * ws.element_size(),
+        _stream(stream)))
+    return out
+
+
+def w8a8_block_fp8_matmul(A, As, B, Bs, block_size=(128, 128), out=None, stream=None):
+    M, K = A.shape
+    N = B.shape[0]
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=A.device) if out is None else out
+    _check(lib().w8a8_block_fp8_matmul(
+        _dev(A, "A", _U8), _dev(As, "As", torch.float32), _dev(B, "B", _U8), _dev(Bs, "Bs", torch.float32),
+        M, N, K, int(block_size[0]), int(block_size[1]), _dev(out, "out", _BF16), _stream(stream)))
+    return out
+
+
+TRACE_STAGES = ("route_topk", "align", "fp8_act_quant", "gate_up", "down", "combine", "dense_fp8")
+
+
+def moe_trace_enable(enable: bool = True):
+    _check(lib().moe_trace_enable(1 if enable else 0))
+
+
+def moe_trace_read(reset: bool = False) -> dict:
+    """{stage name: (total ms, calls)} of the kernel stages recorded since the last reset."""
+    n = len(TRACE_STAGES)
+    ms = (ctypes.c_double * n)()
+    calls = (ctypes.c_longlong * n)()
+    rc = lib().moe_trace_read(ctypes.cast(ms, ctypes.c_void_p), ctypes.cast(calls, ctypes.c_void_p), n,
+                              1 if reset else 0)
+    if rc != n:
+        _check(rc)
+    return {name: (ms[i], calls[i]) for i, name in enumerate(TRACE_STAGES)}
+
+
+def moe_device_status(clear: bool = False) -> int:
+    return int(lib().moe_device_status(1 if clear else 0))

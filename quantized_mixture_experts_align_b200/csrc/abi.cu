@@ -1,0 +1,533 @@
+// C ABI of libmoeq.so: argument validation, workspace layout, schedule choice and the launch
+// sequence of each entry point. Declarations and contracts are in include/moeq.h.
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+#define MOEQ_VERSION "moeq 0.1 (sm_100a)"
+
+namespace moeq {
+
+static thread_local char g_err[512] = "";
+
+int set_error(int code, const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+int check_launch(const char *what)
+{
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return set_error(MOEQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+    return MOEQ_OK;
+}
+
+__device__ int g_device_status = 0;
+
+// SM count of the current device, looked up once per device.
+static int num_sms()
+{
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cache[dev] == 0) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        cache[dev] = n > 0 ? n : 148;
+    }
+    return cache[dev];
+}
+
+// ---- stage tracing (diagnostic, off by default) ---------------------------------------------
+// When enabled, each kernel stage of a call is bracketed by a CUDA event pair recorded on the
+// call's stream; moe_trace_read() waits for the recorded pairs and accumulates their durations.
+namespace trace {
+enum { ROUTE = 0, ALIGN, ACT_QUANT, GATE_UP, DOWN, COMBINE, DENSE, NSTAGE };
+struct Rec {
+    cudaEvent_t a, b;
+    int stage;
+};
+static std::mutex mu;
+static bool enabled = false;
+static std::vector<Rec> pending;
+static std::vector<cudaEvent_t> spare;
+static double sum_ms[NSTAGE];
+static long long calls[NSTAGE];
+constexpr size_t kMaxPending = 1 << 16;
+
+static cudaEvent_t take_event()
+{
+    if (!spare.empty()) {
+        cudaEvent_t e = spare.back();
+        spare.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+}
+
+struct Scope {
+    Rec r{nullptr, nullptr, 0};
+    cudaStream_t s;
+    bool on = false;
+    Scope(int stage, cudaStream_t st) : s(st)
+    {
+        std::lock_guard<std::mutex> g(mu);
+        if (!enabled || pending.size() >= kMaxPending) return;
+        r.a = take_event();
+        r.b = take_event();
+        r.stage = stage;
+        on = r.a && r.b && cudaEventRecord(r.a, s) == cudaSuccess;
+    }
+    ~Scope()
+    {
+        if (!on) return;
+        std::lock_guard<std::mutex> g(mu);
+        if (cudaEventRecord(r.b, s) == cudaSuccess) pending.push_back(r);
+    }
+};
+}  // namespace trace
+
+// ---- schedule --------------------------------------------------------------------------------
+// The routed rows per expert (tok_e = T*k/E), not the token count, decides the tile ("vLLM x
+// Novita AI: Chord W4A16 INT4 MoE Kernel for Kimi K2.x", sections "Summary" and "H200 prefill
+// and TP8": block-M chosen from tokens per expert). Without a host read of the routing, the
+// mean tok_e picks block_m: decode shapes get block-M 8 (the page's decode profile).
+static int pick_block_m(long T, int k, int E)
+{
+    const double tok_e = (double)T * k / (double)E;
+    if (tok_e <= 2.0) return 8;
+    if (tok_e <= 8.0) return 16;
+    if (tok_e <= 24.0) return 32;
+    return 64;
+}
+
+static int pick_block_m_dense(int M)
+{
+    if (M <= 8) return 8;
+    if (M <= 16) return 16;
+    if (M <= 32) return 32;
+    return 64;
+}
+
+// ---- workspace ---------------------------------------------------------------------------------
+struct Carve {
+    char *base;
+    size_t used = 0;
+    explicit Carve(void *p) : base(static_cast<char *>(p)) {}
+    template <class Tp>
+    Tp *take(size_t count)
+    {
+        Tp *p = base ? reinterpret_cast<Tp *>(base + used) : nullptr;
+        used += align256(count * sizeof(Tp));
+        return p;
+    }
+};
+
+struct RouteBufs {
+    int32_t *ids;
+    float *w;
+    int32_t *sorted;
+    int32_t *eids;
+    int32_t *ntp;
+    int block_m;
+    int max_blocks;
+};
+
+static RouteBufs carve_route(Carve &c, long T, int k, int E, int block_m)
+{
+    RouteBufs r;
+    const size_t n = (size_t)T * k;
+    const size_t cap = n + (size_t)E * (block_m - 1);
+    r.block_m = block_m;
+    r.max_blocks = (int)cdivz(cap, block_m);
+    r.ids = c.take<int32_t>(n);
+    r.w = c.take<float>(n);
+    r.sorted = c.take<int32_t>(cap);
+    r.eids = c.take<int32_t>((size_t)r.max_blocks);
+    r.ntp = c.take<int32_t>(1);
+    return r;
+}
+
+static size_t w4a16_layout(Carve &c, long T, int H, int I, int E, int k, RouteBufs *rb, uint16_t **h, float **ys)
+{
+    RouteBufs r = carve_route(c, T, k, E, pick_block_m(T, k, E));
+    uint16_t *hp = c.take<uint16_t>((size_t)T * k * I);
+    float *yp = c.take<float>((size_t)T * k * H);
+    if (rb) *rb = r;
+    if (h) *h = hp;
+    if (ys) *ys = yp;
+    return c.used;
+}
+
+static size_t fp8_layout(Carve &c, long T, int H, int I, int E, int k, RouteBufs *rb, uint8_t **xq, float **xs,
+                         uint8_t **hq, float **hs, float **ys)
+{
+    RouteBufs r = carve_route(c, T, k, E, pick_block_m(T, k, E));
+    uint8_t *xqp = c.take<uint8_t>((size_t)T * H);
+    float *xsp = c.take<float>((size_t)T * (H / 128));
+    uint8_t *hqp = c.take<uint8_t>((size_t)T * k * I);
+    float *hsp = c.take<float>((size_t)T * k * (I / 128));
+    float *yp = c.take<float>((size_t)T * k * H);
+    if (rb) *rb = r;
+    if (xq) *xq = xqp;
+    if (xs) *xs = xsp;
+    if (hq) *hq = hqp;
+    if (hs) *hs = hsp;
+    if (ys) *ys = yp;
+    return c.used;
+}
+
+// ---- validation ----------------------------------------------------------------------------------
+static int check_routing_shape(long T, int E, int k)
+{
+    if (T < 0) return set_error(MOEQ_ERR_INVALID_ARG, "T must be >= 0 (got %ld)", T);
+    if (E < 1 || E > kMaxExperts)
+        return set_error(MOEQ_ERR_UNSUPPORTED, "E must be in [1, %d] (got %d)", kMaxExperts, E);
+    if (k < 1 || k > kMaxTopK || k > E)
+        return set_error(MOEQ_ERR_UNSUPPORTED, "k must be in [1, min(%d, E)] (got k=%d, E=%d)", kMaxTopK, k, E);
+    if (T * (long)k > (1L << 24)) return set_error(MOEQ_ERR_UNSUPPORTED, "T*k must be <= 2^24 (got %ld)", T * k);
+    return MOEQ_OK;
+}
+
+static int check_layer_shape(long T, int H, int I, int E, int k)
+{
+    int rc = check_routing_shape(T, E, k);
+    if (rc) return rc;
+    if (H < 128 || H % 128) return set_error(MOEQ_ERR_UNSUPPORTED, "H must be a positive multiple of 128 (got %d)", H);
+    if (I < 128 || I % 128) return set_error(MOEQ_ERR_UNSUPPORTED, "I must be a positive multiple of 128 (got %d)", I);
+    return MOEQ_OK;
+}
+
+#define MOEQ_REQUIRE(ptr)                                                                       \
+    do {                                                                                        \
+        if ((ptr) == nullptr) return set_error(MOEQ_ERR_INVALID_ARG, "%s must not be NULL", #ptr); \
+    } while (0)
+
+}  // namespace moeq
+
+using namespace moeq;
+
+extern "C" {
+
+const char *moe_last_error(void) { return g_err; }
+
+const char *moe_version(void) { return MOEQ_VERSION; }
+
+int moe_route_topk(const float *logits, int T, int E, int k, int32_t *topk_ids, float *topk_w, void *stream)
+{
+    g_err[0] = 0;
+    int rc = check_routing_shape(T, E, k);
+    if (rc) return rc;
+    if (T == 0) return MOEQ_OK;
+    MOEQ_REQUIRE(logits);
+    MOEQ_REQUIRE(topk_ids);
+    MOEQ_REQUIRE(topk_w);
+    launch_route_topk(logits, T, E, k, topk_ids, topk_w, (cudaStream_t)stream);
+    return check_launch("moe_route_topk");
+}
+
+int moe_align(const int32_t *topk_ids, int T, int k, int E, int block_m, int32_t *sorted_ids, int32_t *expert_ids,
+              int32_t *num_tokens_padded, void *stream)
+{
+    g_err[0] = 0;
+    if (T < 0 || k < 1) return set_error(MOEQ_ERR_INVALID_ARG, "need T >= 0 and k >= 1 (got T=%d, k=%d)", T, k);
+    if (E < 1 || E > kMaxExperts) return set_error(MOEQ_ERR_UNSUPPORTED, "E must be in [1, %d] (got %d)", kMaxExperts, E);
+    if (block_m < 1 || block_m > 256) return set_error(MOEQ_ERR_UNSUPPORTED, "block_m must be in [1, 256] (got %d)", block_m);
+    if ((long)T * k > (1L << 24)) return set_error(MOEQ_ERR_UNSUPPORTED, "T*k must be <= 2^24");
+    MOEQ_REQUIRE(sorted_ids);
+    MOEQ_REQUIRE(expert_ids);
+    MOEQ_REQUIRE(num_tokens_padded);
+    if (T > 0) MOEQ_REQUIRE(topk_ids);
+    launch_align(topk_ids, T * k, E, block_m, sorted_ids, expert_ids, num_tokens_padded, (cudaStream_t)stream);
+    return check_launch("moe_align");
+}
+
+int moe_fp8_act_quant(const uint16_t *x, int rows, int cols, uint8_t *q, float *s, void *stream)
+{
+    g_err[0] = 0;
+    if (rows < 0) return set_error(MOEQ_ERR_INVALID_ARG, "rows must be >= 0 (got %d)", rows);
+    if (cols < 128 || cols % 128) return set_error(MOEQ_ERR_UNSUPPORTED, "cols must be a positive multiple of 128 (got %d)", cols);
+    if (rows == 0) return MOEQ_OK;
+    MOEQ_REQUIRE(x);
+    MOEQ_REQUIRE(q);
+    MOEQ_REQUIRE(s);
+    launch_fp8_act_quant(x, rows, cols, q, s, (cudaStream_t)stream);
+    return check_launch("moe_fp8_act_quant");
+}
+
+size_t moe_w4a16_workspace_size(int T, int H, int I, int E, int k)
+{
+    if (check_layer_shape(T, H, I, E, k)) return 0;
+    Carve c(nullptr);
+    return w4a16_layout(c, T, H, I, E, k, nullptr, nullptr, nullptr);
+}
+
+int moe_w4a16_forward(const uint16_t *x, const float *logits, int T, int H, int I, int E, int k,
+                      const int32_t *w13_q, const uint16_t *w13_s, const int32_t *w2_q, const uint16_t *w2_s,
+                      uint16_t *out, int32_t *topk_ids_out, float *topk_w_out, void *ws, size_t ws_bytes,
+                      void *stream)
+{
+    g_err[0] = 0;
+    int rc = check_layer_shape(T, H, I, E, k);
+    if (rc) return rc;
+    if (T == 0) return MOEQ_OK;
+    MOEQ_REQUIRE(x);
+    MOEQ_REQUIRE(logits);
+    MOEQ_REQUIRE(w13_q);
+    MOEQ_REQUIRE(w13_s);
+    MOEQ_REQUIRE(w2_q);
+    MOEQ_REQUIRE(w2_s);
+    MOEQ_REQUIRE(out);
+    MOEQ_REQUIRE(ws);
+    if (reinterpret_cast<uintptr_t>(ws) & 255) return set_error(MOEQ_ERR_INVALID_ARG, "ws must be 256-byte aligned");
+    const size_t need = moe_w4a16_workspace_size(T, H, I, E, k);
+    if (ws_bytes < need) return set_error(MOEQ_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, need);
+
+    cudaStream_t s = (cudaStream_t)stream;
+    Carve c(ws);
+    RouteBufs r;
+    uint16_t *h;
+    float *ys;
+    w4a16_layout(c, T, H, I, E, k, &r, &h, &ys);
+    int32_t *ids = topk_ids_out ? topk_ids_out : r.ids;
+    float *tw = topk_w_out ? topk_w_out : r.w;
+    const int n = T * k;
+
+    {
+        trace::Scope ts(trace::ROUTE, s);
+        launch_route_topk(logits, T, E, k, ids, tw, s);
+    }
+    {
+        trace::Scope ts(trace::ALIGN, s);
+        launch_align(ids, n, E, r.block_m, r.sorted, r.eids, r.ntp, s);
+    }
+
+    W4GroupedArgs a{};
+    a.E = E;
+    a.sorted_ids = r.sorted;
+    a.expert_ids = r.eids;
+    a.num_tokens_padded = r.ntp;
+    a.n_slots = n;
+    a.topk_w = tw;
+    // gate/up + SiLU*up
+    a.act = x;
+    a.act_row_div = k;
+    a.wq = w13_q;
+    a.ws = w13_s;
+    a.K = H;
+    a.n_out = I;
+    a.n_rows = 2 * I;
+    a.h_out = h;
+    {
+        trace::Scope ts(trace::GATE_UP, s);
+        launch_w4a16_grouped_mma(a, MODE_GATEUP, r.block_m, r.max_blocks, s);
+    }
+    // down, routing weight applied per slot
+    a.act = h;
+    a.act_row_div = 1;
+    a.wq = w2_q;
+    a.ws = w2_s;
+    a.K = I;
+    a.n_out = H;
+    a.n_rows = H;
+    a.y_out = ys;
+    {
+        trace::Scope ts(trace::DOWN, s);
+        launch_w4a16_grouped_mma(a, MODE_DOWN, r.block_m, r.max_blocks, s);
+    }
+    {
+        trace::Scope ts(trace::COMBINE, s);
+        launch_combine(ys, T, k, H, out, num_sms(), s);
+    }
+    return check_launch("moe_w4a16_forward");
+}
+
+size_t moe_w8a8_block_fp8_workspace_size(int T, int H, int I, int E, int k)
+{
+    if (check_layer_shape(T, H, I, E, k)) return 0;
+    Carve c(nullptr);
+    return fp8_layout(c, T, H, I, E, k, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr);
+}
+
+int moe_w8a8_block_fp8_forward(const uint16_t *x, const float *logits, int T, int H, int I, int E, int k,
+                               const uint8_t *w13, const float *w13_s, const uint8_t *w2, const float *w2_s,
+                               uint16_t *out, int32_t *topk_ids_out, float *topk_w_out, void *ws, size_t ws_bytes,
+                               void *stream)
+{
+    g_err[0] = 0;
+    int rc = check_layer_shape(T, H, I, E, k);
+    if (rc) return rc;
+    if (T == 0) return MOEQ_OK;
+    MOEQ_REQUIRE(x);
+    MOEQ_REQUIRE(logits);
+    MOEQ_REQUIRE(w13);
+    MOEQ_REQUIRE(w13_s);
+    MOEQ_REQUIRE(w2);
+    MOEQ_REQUIRE(w2_s);
+    MOEQ_REQUIRE(out);
+    MOEQ_REQUIRE(ws);
+    if (reinterpret_cast<uintptr_t>(ws) & 255) return set_error(MOEQ_ERR_INVALID_ARG, "ws must be 256-byte aligned");
+    const size_t need = moe_w8a8_block_fp8_workspace_size(T, H, I, E, k);
+    if (ws_bytes < need) return set_error(MOEQ_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, need);
+
+    cudaStream_t s = (cudaStream_t)stream;
+    Carve c(ws);
+    RouteBufs r;
+    uint8_t *xq, *hq;
+    float *xs, *hs, *ys;
+    fp8_layout(c, T, H, I, E, k, &r, &xq, &xs, &hq, &hs, &ys);
+    int32_t *ids = topk_ids_out ? topk_ids_out : r.ids;
+    float *tw = topk_w_out ? topk_w_out : r.w;
+    const int n = T * k;
+
+    {
+        trace::Scope ts(trace::ROUTE, s);
+        launch_route_topk(logits, T, E, k, ids, tw, s);
+    }
+    {
+        trace::Scope ts(trace::ALIGN, s);
+        launch_align(ids, n, E, r.block_m, r.sorted, r.eids, r.ntp, s);
+    }
+    {
+        trace::Scope ts(trace::ACT_QUANT, s);
+        launch_fp8_act_quant(x, T, H, xq, xs, s);
+    }
+
+    F8GroupedArgs a{};
+    a.E = E;
+    a.sorted_ids = r.sorted;
+    a.expert_ids = r.eids;
+    a.num_tokens_padded = r.ntp;
+    a.n_slots = n;
+    a.topk_w = tw;
+    a.act = xq;
+    a.act_s = xs;
+    a.act_row_div = k;
+    a.w = w13;
+    a.w_s = w13_s;
+    a.K = H;
+    a.n_out = I;
+    a.n_rows = 2 * I;
+    a.hq_out = hq;
+    a.hs_out = hs;
+    {
+        trace::Scope ts(trace::GATE_UP, s);
+        launch_fp8_grouped_mma(a, MODE_GATEUP, r.block_m, r.max_blocks, s);
+    }
+    a.act = hq;
+    a.act_s = hs;
+    a.act_row_div = 1;
+    a.w = w2;
+    a.w_s = w2_s;
+    a.K = I;
+    a.n_out = H;
+    a.n_rows = H;
+    a.y_out = ys;
+    {
+        trace::Scope ts(trace::DOWN, s);
+        launch_fp8_grouped_mma(a, MODE_DOWN, r.block_m, r.max_blocks, s);
+    }
+    {
+        trace::Scope ts(trace::COMBINE, s);
+        launch_combine(ys, T, k, H, out, num_sms(), s);
+    }
+    return check_launch("moe_w8a8_block_fp8_forward");
+}
+
+int w8a8_block_fp8_matmul(const uint8_t *A, const float *As, const uint8_t *B, const float *Bs, int M, int N, int K,
+                          int block_n, int block_k, uint16_t *C, void *stream)
+{
+    g_err[0] = 0;
+    if (block_n != 128 || block_k != 128)
+        return set_error(MOEQ_ERR_UNSUPPORTED, "block_size must be [128, 128] (got [%d, %d])", block_n, block_k);
+    if (M < 0 || N < 1 || K < 1) return set_error(MOEQ_ERR_INVALID_ARG, "bad sizes M=%d N=%d K=%d", M, N, K);
+    if (K % 128) return set_error(MOEQ_ERR_UNSUPPORTED, "K must be a multiple of 128 (got %d)", K);
+    if (N % 128) return set_error(MOEQ_ERR_UNSUPPORTED, "N must be a multiple of 128 (got %d)", N);
+    if (M == 0) return MOEQ_OK;
+    MOEQ_REQUIRE(A);
+    MOEQ_REQUIRE(As);
+    MOEQ_REQUIRE(B);
+    MOEQ_REQUIRE(Bs);
+    MOEQ_REQUIRE(C);
+    F8GroupedArgs a{};
+    a.act = A;
+    a.act_s = As;
+    a.act_row_div = 1;
+    a.w = B;
+    a.w_s = Bs;
+    a.K = K;
+    a.n_out = N;
+    a.n_rows = N;
+    a.E = 1;
+    a.n_slots = M;
+    a.c_out = C;
+    const int bm = pick_block_m_dense(M);
+    {
+        trace::Scope ts(trace::DENSE, (cudaStream_t)stream);
+        launch_fp8_grouped_mma(a, MODE_DENSE, bm, cdiv(M, bm), (cudaStream_t)stream);
+    }
+    return check_launch("w8a8_block_fp8_matmul");
+}
+
+int moe_trace_enable(int enable)
+{
+    g_err[0] = 0;
+    std::lock_guard<std::mutex> g(trace::mu);
+    trace::enabled = enable != 0;
+    return MOEQ_OK;
+}
+
+int moe_trace_read(double *stage_ms, long long *stage_calls, int n_stages, int reset)
+{
+    g_err[0] = 0;
+    std::lock_guard<std::mutex> g(trace::mu);
+    for (const trace::Rec &r : trace::pending) {
+        float ms = 0.f;
+        cudaError_t e = cudaEventSynchronize(r.b);
+        if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, r.a, r.b);
+        if (e != cudaSuccess) {
+            trace::pending.clear();
+            return set_error(MOEQ_ERR_CUDA, "moe_trace_read: %s", cudaGetErrorString(e));
+        }
+        trace::sum_ms[r.stage] += ms;
+        trace::calls[r.stage] += 1;
+        trace::spare.push_back(r.a);
+        trace::spare.push_back(r.b);
+    }
+    trace::pending.clear();
+    for (int i = 0; i < n_stages && i < trace::NSTAGE; ++i) {
+        if (stage_ms) stage_ms[i] = trace::sum_ms[i];
+        if (stage_calls) stage_calls[i] = trace::calls[i];
+    }
+    if (reset)
+        for (int i = 0; i < trace::NSTAGE; ++i) { trace::sum_ms[i] = 0.0; trace::calls[i] = 0; }
+    return trace::NSTAGE;
+}
+
+int moe_device_status(int clear)
+{
+    g_err[0] = 0;
+    int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_device_status, sizeof v);
+    if (e != cudaSuccess) return set_error(MOEQ_ERR_CUDA, "moe_device_status: %s", cudaGetErrorString(e));
+    if (clear) {
+        const int z = 0;
+        e = cudaMemcpyToSymbol(g_device_status, &z, sizeof z);
+        if (e != cudaSuccess) return set_error(MOEQ_ERR_CUDA, "moe_device_status: %s", cudaGetErrorString(e));
+    }
+    return v ? MOEQ_ERR_DEVICE_TIMEOUT : MOEQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,58 @@
+// Kernel launchers of the moeq library (internal; the public surface is include/moeq.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moeq {
+
+enum { MODE_GATEUP = 0, MODE_DOWN = 1, MODE_DENSE = 2 };
+
+struct W4GroupedArgs {
+    const uint16_t *act;     // gate/up: x [T, K]; down: h [T*k, K]  (bf16)
+    int act_row_div;         // activation row of a slot = slot / act_row_div (k for x, 1 for h)
+    const int32_t *wq;       // [E, n_rows, K/8]
+    const uint16_t *ws;      // [E, n_rows, K/32] bf16
+    int K;
+    int n_out;               // gate/up: I (weights hold 2I rows); down: H
+    int n_rows;              // weight rows per expert
+    int E;
+    const int32_t *sorted_ids;
+    const int32_t *expert_ids;
+    const int32_t *num_tokens_padded;
+    int n_slots;             // T*k; sorted_ids entries >= n_slots are padding
+    const float *topk_w;     // [T*k] (down)
+    uint16_t *h_out;         // [T*k, I] bf16 (gate/up)
+    float *y_out;            // [T*k, H] f32, routing weight applied (down)
+};
+
+struct F8GroupedArgs {
+    const uint8_t *act;      // gate/up: xq [T, K]; down: hq [T*k, K]; dense: A [M, K]
+    const float *act_s;      // [rows, K/128]
+    int act_row_div;
+    const uint8_t *w;        // [E, n_rows, K]
+    const float *w_s;        // [E, n_rows/128, K/128]
+    int K;
+    int n_out;
+    int n_rows;
+    int E;
+    const int32_t *sorted_ids;
+    const int32_t *expert_ids;
+    const int32_t *num_tokens_padded;
+    int n_slots;             // T*k (grouped) or M (dense)
+    const float *topk_w;
+    uint8_t *hq_out;         // [T*k, I]
+    float *hs_out;           // [T*k, I/128]
+    float *y_out;            // [T*k, H]
+    uint16_t *c_out;         // dense: [M, N] bf16
+};
+
+void launch_route_topk(const float *logits, int T, int E, int k, int32_t *ids, float *w, cudaStream_t s);
+void launch_align(const int32_t *topk_ids, int n, int E, int B, int32_t *sorted_ids, int32_t *expert_ids,
+                  int32_t *ntp, cudaStream_t s);
+void launch_combine(const float *ys, int T, int k, int H, uint16_t *out, int num_sms, cudaStream_t s);
+void launch_fp8_act_quant(const uint16_t *x, int rows, int cols, uint8_t *q, float *s, cudaStream_t st);
+void launch_w4a16_grouped_mma(const W4GroupedArgs &a, int mode, int block_m, int max_blocks, cudaStream_t s);
+void launch_fp8_grouped_mma(const F8GroupedArgs &a, int mode, int block_m, int max_blocks, cudaStream_t s);
+
+}  // namespace moeq

@@ -1,0 +1,206 @@
+// Routing (top-k softmax, renormalised) and token-to-expert alignment kernels.
+//
+// Alignment follows "vLLM x Novita AI: Chord W4A16 INT4 MoE Kernel for Kimi K2.x", sections
+// "Two kernel families" (sorted_ids / expert_ids / num_tokens_padded) and figure 3 (padding
+// guards live in the indices, activations are not padded). The stable within-expert order and
+// the pad value T*k are this library's reading; they make the outputs bit-reproducible.
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace moeq {
+
+// ------------------------------------------------------------------------------------------
+// Routing: one warp per token. Lane l holds logits l, l+32, ... in registers; k rounds of a
+// warp arg-max (value descending, index ascending) pick the experts, then lane j < k turns its
+// pick into exp(l_j - l_max) in double and every lane sums them in slot order.
+// ------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict__ logits, int T, int E,
+                                                         int k, int32_t *__restrict__ ids,
+                                                         float *__restrict__ w)
+{
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (t >= T) return;
+    const float *row = logits + (size_t)t * E;
+    float v[kMaxExperts / 32];
+#pragma unroll
+    for (int i = 0; i < kMaxExperts / 32; ++i) {
+        const int e = lane + 32 * i;
+        v[i] = (e < E) ? __ldg(row + e) : 0.0f;
+    }
+    uint32_t taken = 0;
+    float my_v = 0.0f;
+    int my_e = 0;
+    for (int j = 0; j < k; ++j) {
+        float bv = 0.0f;
+        int be = 0x7FFFFFFF;
+#pragma unroll
+        for (int i = 0; i < kMaxExperts / 32; ++i) {
+            const int e = lane + 32 * i;
+            if (e < E && !((taken >> i) & 1u)) {
+                if (be == 0x7FFFFFFF || v[i] > bv) { bv = v[i]; be = e; }
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, off);
+            const int oe = __shfl_xor_sync(0xFFFFFFFFu, be, off);
+            const bool better = (oe != 0x7FFFFFFF) &&
+                                (be == 0x7FFFFFFF || ov > bv || (ov == bv && oe < be));
+            if (better) { bv = ov; be = oe; }
+        }
+        if ((be & 31) == lane) taken |= 1u << (be >> 5);
+        if (lane == j) { my_v = bv; my_e = be; }
+    }
+    const float vmax = __shfl_sync(0xFFFFFFFFu, my_v, 0);
+    const double d = (lane < k) ? exp((double)my_v - (double)vmax) : 0.0;
+    double den = 0.0;
+    for (int j = 0; j < k; ++j) den += __shfl_sync(0xFFFFFFFFu, d, j);
+    if (lane < k) {
+        ids[(size_t)t * k + lane] = my_e;
+        w[(size_t)t * k + lane] = (float)(d / den);
+    }
+}
+
+void launch_route_topk(const float *logits, int T, int E, int k, int32_t *ids, float *w, cudaStream_t s)
+{
+    if (T <= 0) return;
+    const int warps = 8;
+    route_topk_kernel<<<cdiv(T, warps), warps * 32, 0, s>>>(logits, T, E, k, ids, w);
+}
+
+// ------------------------------------------------------------------------------------------
+// Alignment: one CTA of 1024 threads.
+//  1. per-expert counts (shared-memory atomics; order-free);
+//  2. exclusive scan of the padded counts -> each expert's offset; expert_ids and pads written;
+//  3. stable scatter in tiles of 1024 slots: a slot's position is its expert's offset + slots of
+//     that expert in earlier tiles + those in earlier warps of this tile + its rank in its warp
+//     (__match_any_sync peers below its lane).
+// ------------------------------------------------------------------------------------------
+constexpr int kAlignThreads = 1024;
+constexpr int kAlignWarps = kAlignThreads / 32;
+
+__global__ void __launch_bounds__(kAlignThreads) align_kernel(const int32_t *__restrict__ topk_ids, int n,
+                                                              int E, int B, int32_t *__restrict__ sorted_ids,
+                                                              int32_t *__restrict__ expert_ids,
+                                                              int32_t *__restrict__ num_tokens_padded)
+{
+    __shared__ int cnt[kMaxExperts];
+    __shared__ int off[kMaxExperts + 1];
+    __shared__ int cursor[kMaxExperts];
+    __shared__ uint8_t hist[kMaxExperts][kAlignWarps];  // per tile: count of expert e in warp w
+    __shared__ int warp_sums[kAlignWarps];
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int e = tid; e < E; e += kAlignThreads) { cnt[e] = 0; cursor[e] = 0; }
+    for (int i = tid; i < kMaxExperts * kAlignWarps / 4; i += kAlignThreads)
+        reinterpret_cast<uint32_t *>(&hist[0][0])[i] = 0u;
+    __syncthreads();
+
+    for (int f = tid; f < n; f += kAlignThreads) {
+        const int e = topk_ids[f];
+        if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
+    }
+    __syncthreads();
+
+    // exclusive scan of padded counts, one expert per thread (E <= 1024)
+    const int padded = (tid < E) ? (cnt[tid] + B - 1) / B * B : 0;
+    int incl = padded;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int ws = warp_sums[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xFFFFFFFFu, ws, o);
+            if (lane >= o) ws += y;
+        }
+        warp_sums[lane] = ws;  // inclusive over warps
+    }
+    __syncthreads();
+    const int excl = incl - padded + (warp > 0 ? warp_sums[warp - 1] : 0);
+    if (tid < E) off[tid] = excl;
+    const int total = warp_sums[kAlignWarps - 1];
+    if (tid == 0) { off[E] = total; *num_tokens_padded = total; }
+    __syncthreads();
+
+    // block ids and pad entries of each expert's range, then the tail past the total
+    const long cap = (long)n + (long)E * (B - 1);
+    const long nblk = (cap + B - 1) / B;
+    if (tid < E) {
+        const int c = cnt[tid];
+        for (int i = excl + c; i < excl + padded; ++i) sorted_ids[i] = n;
+        for (int b = excl / B; b < (excl + padded) / B; ++b) expert_ids[b] = tid;
+    }
+    for (long i = total + tid; i < cap; i += kAlignThreads) sorted_ids[i] = n;
+    for (long b = total / B + tid; b < nblk; b += kAlignThreads) expert_ids[b] = -1;
+
+    // stable scatter
+    const unsigned lt_mask = (1u << lane) - 1u;
+    for (int base = 0; base < n; base += kAlignThreads) {
+        const int f = base + tid;
+        int e = (f < n) ? topk_ids[f] : -1;
+        if (e < 0 || e >= E) e = -1;
+        const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
+        const int rank = __popc(peers & lt_mask);
+        const bool leader = (peers & lt_mask) == 0u;
+        if (e >= 0 && leader) hist[e][warp] = (uint8_t)__popc(peers);
+        __syncthreads();
+        if (e >= 0) {
+            int before = 0;
+            for (int w = 0; w < warp; ++w) before += hist[e][w];
+            sorted_ids[off[e] + cursor[e] + before + rank] = f;
+        }
+        __syncthreads();
+        if (e >= 0 && leader) {
+            atomicAdd(&cursor[e], __popc(peers));
+            hist[e][warp] = 0;
+        }
+        __syncthreads();
+    }
+}
+
+void launch_align(const int32_t *topk_ids, int n, int E, int B, int32_t *sorted_ids, int32_t *expert_ids,
+                  int32_t *ntp, cudaStream_t s)
+{
+    align_kernel<<<1, kAlignThreads, 0, s>>>(topk_ids, n, E, B, sorted_ids, expert_ids, ntp);
+}
+
+// ------------------------------------------------------------------------------------------
+// Top-k weighted combine: out[t, :] = bf16( sum_j ys[t*k + j, :] ), the slot rows already
+// carrying their routing weight. f32 sums in slot order.
+// ------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ ys, int T, int k, int H,
+                                                      uint16_t *__restrict__ out)
+{
+    const int H4 = H / 4;
+    const long total = (long)T * H4;
+    for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < total; i += (long)gridDim.x * blockDim.x) {
+        const long t = i / H4;
+        const int c = (int)(i - t * H4);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < k; ++j) {
+            const float4 v = __ldg(reinterpret_cast<const float4 *>(ys + ((size_t)t * k + j) * H) + c);
+            acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+        }
+        uint2 o;
+        o.x = pack_bf16x2(acc.x, acc.y);
+        o.y = pack_bf16x2(acc.z, acc.w);
+        reinterpret_cast<uint2 *>(out + (size_t)t * H)[c] = o;
+    }
+}
+
+void launch_combine(const float *ys, int T, int k, int H, uint16_t *out, int num_sms, cudaStream_t s)
+{
+    if (T <= 0) return;
+    const long total = (long)T * (H / 4);
+    const int blocks = (int)((total + 255) / 256 < (long)num_sms * 8 ? (total + 255) / 256 : (long)num_sms * 8);
+    combine_kernel<<<blocks, 256, 0, s>>>(ys, T, k, H, out);
+}
+
+}  // namespace moeq

@@ -1,0 +1,82 @@
+"""Helpers shared by the GPU parity tests: input synthesis on the device, host copies for the
+oracle, and the layer tolerance check."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import workloads as W
+
+# Layer-output tolerances: |gpu - ref| <= tol * (|ref| + rms(ref)), element-wise.
+TOL_W4A16 = 2e-2
+TOL_FP8 = 3e-2
+
+
+def assert_layer_close(gpu: np.ndarray, ref: np.ndarray, tol: float, what: str = ""):
+    gpu = np.asarray(gpu, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert gpu.shape == ref.shape, (gpu.shape, ref.shape)
+    assert np.all(np.isfinite(gpu)), f"{what}: non-finite GPU output"
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    err = np.abs(gpu - ref)
+    bound = tol * (np.abs(ref) + rms)
+    bad = err > bound
+    if bad.any():
+        i = np.unravel_index(np.argmax(err / bound), err.shape)
+        raise AssertionError(f"{what}: {bad.sum()} of {bad.size} elements out of tolerance; worst at {i}: "
+                             f"gpu={gpu[i]!r} ref={ref[i]!r} bound={bound[i]!r} (rms {rms:.3g})")
+
+
+def bf16_to_f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def host_moe_weights(d: dict, experts) -> dict:
+    """Host numpy copies of the weights of the given experts, laid out full-size (untouched
+    experts stay zero pages) so the oracle can index them by expert id."""
+    out = {}
+    names = ("w13q", "w13s", "w2q", "w2s") if d["kind"] == "w4a16" else ("w13", "w13s", "w2", "w2s")
+    for n in names:
+        t = d[n]
+        np_dtype = {torch.int32: np.int32, torch.bfloat16: np.uint16, torch.uint8: np.uint8,
+                    torch.float32: np.float32}[t.dtype]
+        arr = np.zeros(tuple(t.shape), np_dtype)
+        for e in sorted(set(int(v) for v in experts)):
+            arr[e] = W.np_bits(t[e])
+        out[n] = arr
+    return out
+
+
+def oracle_layer(d: dict, tokens, want_h=False):
+    """Oracle output rows for `tokens` of a generated MoE workload (float64 [len(tokens), H])."""
+    import oracle
+    x = W.np_bits(d["x"])
+    logits = W.np_bits(d["logits"])
+    ids, _ = oracle.route_topk(logits[np.asarray(tokens)], d["k"])
+    hw = host_moe_weights(d, ids.ravel())
+    if d["kind"] == "w4a16":
+        return oracle.moe_w4a16(x, logits, d["k"], hw["w13q"], hw["w13s"], hw["w2q"], hw["w2s"], tokens=tokens,
+                                want_h=want_h)
+    return oracle.moe_fp8(x, logits, d["k"], hw["w13"], hw["w13s"], hw["w2"], hw["w2s"], tokens=tokens,
+                          want_h=want_h)
+
+
+def sample_tokens(d: dict, n: int, seed: int = 0) -> np.ndarray:
+    """Seeded token sample that includes the first and last token and tokens routed to the most
+    and least loaded experts."""
+    import oracle
+    T = d["T"]
+    if T <= n:
+        return np.arange(T, dtype=np.int32)
+    logits = W.np_bits(d["logits"])
+    ids, _ = oracle.route_topk(logits, d["k"])
+    counts = np.bincount(ids.ravel(), minlength=d["E"])
+    heavy = int(np.argmax(counts))
+    light = int(np.argmin(np.where(counts > 0, counts, 1 << 30)))
+    pick = {0, T - 1}
+    pick.add(int(np.nonzero((ids == heavy).any(1))[0][0]))
+    pick.add(int(np.nonzero((ids == light).any(1))[0][0]))
+    rng = np.random.default_rng(seed)
+    while len(pick) < n:
+        pick.add(int(rng.integers(0, T)))
+    return np.array(sorted(pick), dtype=np.int32)

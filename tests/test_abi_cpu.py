@@ -1,0 +1,97 @@
+"""CPU-side checks of the C ABI: the library builds, loads and exports every entry point that
+include/moeq.h declares, and host-side validation rejects bad arguments before any device work
+(no GPU is touched: every call here fails validation before the first CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import quantized_mixture_experts_align_b200 as moeq
+from quantized_mixture_experts_align_b200 import build as moeq_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    moeq_build.build()
+    return moeq.lib()
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "moeq.h")).read()
+    return re.findall(r"^MOEQ_API\s+[\w\s\*]*?\b(\w+)\s*\(", text, flags=re.M)
+
+
+def test_header_declares_the_boundary():
+    names = set(_declared())
+    for need in ("moe_route_topk", "moe_align", "moe_w4a16_forward", "moe_w8a8_block_fp8_forward",
+                 "w8a8_block_fp8_matmul", "moe_fp8_act_quant", "moe_last_error"):
+        assert need in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in _declared():
+        assert hasattr(L, name), name
+    assert set(_declared()) <= set(moeq.exported_symbols())
+
+
+def test_version(L):
+    assert "sm_100a" in moeq.version()
+
+
+def test_workspace_sizes(L):
+    a = moeq.moe_w4a16_workspace_size(32, 7168, 2048, 384, 8)
+    n = 32 * 8
+    assert a >= n * 2048 * 2 + n * 7168 * 4                   # h + weighted slot outputs
+    assert moeq.moe_w4a16_workspace_size(8192, 7168, 2048, 384, 8) > a
+    assert moeq.moe_w8a8_block_fp8_workspace_size(4096, 7168, 2048, 256, 8) > 0
+    assert moeq.moe_w4a16_workspace_size(32, 100, 2048, 384, 8) == 0      # unsupported H
+    assert moeq.moe_w4a16_workspace_size(32, 7168, 2048, 4, 8) == 0       # k > E
+
+
+def _rc(L, name, *args):
+    fn = getattr(L, name)
+    return fn(*args)
+
+
+def test_validation_rejects_before_device_work(L):
+    N = None
+    # route: k > E, E too large, k > 32
+    assert _rc(L, "moe_route_topk", N, 4, 8, 9, N, N, N) == moeq.MOEQ_ERR_UNSUPPORTED
+    assert _rc(L, "moe_route_topk", N, 4, 2000, 8, N, N, N) == moeq.MOEQ_ERR_UNSUPPORTED
+    assert _rc(L, "moe_route_topk", N, 4, 64, 33, N, N, N) == moeq.MOEQ_ERR_UNSUPPORTED
+    assert _rc(L, "moe_route_topk", N, 4, 64, 8, N, N, N) == moeq.MOEQ_ERR_INVALID_ARG   # NULL logits
+    assert b"logits" in L.moe_last_error()
+    # align: bad block size, negative T, NULL outputs
+    assert _rc(L, "moe_align", N, 3, 2, 3, 0, N, N, N, N) == moeq.MOEQ_ERR_UNSUPPORTED
+    assert _rc(L, "moe_align", N, -1, 2, 3, 4, N, N, N, N) == moeq.MOEQ_ERR_INVALID_ARG
+    assert _rc(L, "moe_align", N, 3, 2, 3, 4, N, N, N, N) == moeq.MOEQ_ERR_INVALID_ARG
+    # act quant: ragged columns
+    assert _rc(L, "moe_fp8_act_quant", N, 4, 100, N, N, N) == moeq.MOEQ_ERR_UNSUPPORTED
+    # forward: unsupported H / I, workspace too small, misaligned workspace
+    fwd = (N, N, 32, 7000, 2048, 384, 8, N, N, N, N, N, N, N, N, 0, N)
+    assert _rc(L, "moe_w4a16_forward", *fwd) == moeq.MOEQ_ERR_UNSUPPORTED
+    fwd = (N, N, 32, 7168, 2000, 384, 8, N, N, N, N, N, N, N, N, 0, N)
+    assert _rc(L, "moe_w8a8_block_fp8_forward", *fwd) == moeq.MOEQ_ERR_UNSUPPORTED
+    p = ctypes.c_void_p(256)
+    fwd = (p, p, 32, 7168, 2048, 384, 8, p, p, p, p, p, N, N, p, 10, N)
+    assert _rc(L, "moe_w4a16_forward", *fwd) == moeq.MOEQ_ERR_WORKSPACE
+    assert b"workspace" in L.moe_last_error()
+    q = ctypes.c_void_p(257)
+    fwd = (p, p, 32, 7168, 2048, 384, 8, p, p, p, p, p, N, N, q, 1 << 40, N)
+    assert _rc(L, "moe_w4a16_forward", *fwd) == moeq.MOEQ_ERR_INVALID_ARG
+    # dense matmul: block size must be [128, 128]; K, N multiples of 128
+    assert _rc(L, "w8a8_block_fp8_matmul", N, N, N, N, 4, 256, 256, 64, 128, N, N) == moeq.MOEQ_ERR_UNSUPPORTED
+    assert _rc(L, "w8a8_block_fp8_matmul", N, N, N, N, 4, 256, 200, 128, 128, N, N) == moeq.MOEQ_ERR_UNSUPPORTED
+    assert _rc(L, "w8a8_block_fp8_matmul", N, N, N, N, 4, 200, 256, 128, 128, N, N) == moeq.MOEQ_ERR_UNSUPPORTED
+    # T == 0 / M == 0 are valid no-ops
+    assert _rc(L, "moe_route_topk", N, 0, 8, 2, N, N, N) == 0
+    assert _rc(L, "w8a8_block_fp8_matmul", N, N, N, N, 0, 256, 256, 128, 128, N, N) == 0
+
+
+def test_binding_refuses_cpu_tensors(L):
+    import torch
+    with pytest.raises(ValueError):
+        moeq.moe_route_topk(torch.zeros(4, 8), 2)
