@@ -114,6 +114,32 @@ MOEQ_API int moe_w4a16_forward(const uint16_t *x, const float *logits, int T, in
                       float *topk_w_out, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * Scratch-free W4A16 layer forward. The pages have no counterpart of this entry point: it exists
+ * for callers that cannot allocate device memory where they run the layer, such as a plugin or
+ * custom-op host that only hands over its input and output buffers, or a serving runtime that
+ * plans all device memory at start-up and forbids allocation afterwards. It computes what
+ * moe_w4a16_forward computes, with the same arguments minus ws / ws_bytes; the caller still
+ * passes (and owns) the inputs and outputs.
+ *  - Its scratch is one static device array of MOEQ_NOALLOC_SCRATCH_BYTES (16 MiB) inside this
+ *    library; every GPU that loads the library holds it until the process exits.
+ *  - Shapes whose moe_w4a16_workspace_size() exceeds that size are rejected with
+ *    MOEQ_ERR_WORKSPACE before anything is enqueued (at H=7168, I=2048, E=384, k=8 the limit is
+ *    T <= 63 tokens).
+ *  - The call allocates nothing: no cudaMalloc, cudaFree or other allocating routine.
+ *  - The first call on each device does a one-time set-up, the lookup of the array's device
+ *    address (cudaGetSymbolAddress, with that device current); make that first call before any
+ *    stream capture.
+ *  - Every call shares the one array, which keeps the last call's contents; nothing in it needs to
+ *    start at zero. Calls that can overlap on the GPU (other streams, other host threads) race on
+ *    the array: serialize them.
+ */
+#define MOEQ_NOALLOC_SCRATCH_BYTES (16u << 20)
+MOEQ_API int moe_w4a16_forward_noalloc(const uint16_t *x, const float *logits, int T, int H, int I, int E,
+                                       int k, const int32_t *w13_q, const uint16_t *w13_s,
+                                       const int32_t *w2_q, const uint16_t *w2_s, uint16_t *out,
+                                       int32_t *topk_ids_out, float *topk_w_out, void *stream);
+
+/*
  * W8A8 block-FP8 routed expert layer ([SGL], "Background": E4M3 weights with one f32 scale per
  * [128, 128] block, activations E4M3 with one f32 scale per token and 128-column group):
  *   the input is quantized as moe_fp8_act_quant; g, u = block-scaled products with W13[e];

@@ -34,6 +34,7 @@ _SIGNATURES = {
     "moe_fp8_act_quant": ([_V, _I, _I, _V, _V, _V], _I),
     "moe_w4a16_workspace_size": ([_I, _I, _I, _I, _I], _Z),
     "moe_w4a16_forward": ([_V, _V, _I, _I, _I, _I, _I, _V, _V, _V, _V, _V, _V, _V, _V, _Z, _V], _I),
+    "moe_w4a16_forward_noalloc": ([_V, _V, _I, _I, _I, _I, _I, _V, _V, _V, _V, _V, _V, _V, _V], _I),
     "moe_w8a8_block_fp8_workspace_size": ([_I, _I, _I, _I, _I], _Z),
     "moe_w8a8_block_fp8_forward": ([_V, _V, _I, _I, _I, _I, _I, _V, _V, _V, _V, _V, _V, _V, _V, _Z, _V], _I),
     "w8a8_block_fp8_matmul": ([_V, _V, _V, _V, _I, _I, _I, _I, _I, _V, _V], _I),
@@ -149,6 +150,22 @@ def moe_w4a16_forward(x, logits, k, w13_q, w13_s, w2_q, w2_s, out=None, ws=None,
         _dev(w2_s, "w2_s", _BF16), _dev(out, "out", _BF16), _dev(topk_ids_out, "topk_ids_out", torch.int32),
         _dev(topk_w_out, "topk_w_out", torch.float32), _dev(ws, "ws"), ws.numel() * ws.element_size(),
         _stream(stream)))
+    return out
+
+
+def moe_w4a16_forward_noalloc(x, logits, k, w13_q, w13_s, w2_q, w2_s, out=None, topk_ids_out=None,
+                              topk_w_out=None, stream=None):
+    """moe_w4a16_forward without a caller workspace: the library's built-in static device scratch
+    is used (for callers that cannot allocate device memory; shapes up to a fixed size)."""
+    T, H = x.shape
+    E = logits.shape[1]
+    I = w2_q.shape[2] * 8
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device) if out is None else out
+    _check(lib().moe_w4a16_forward_noalloc(
+        _dev(x, "x", _BF16), _dev(logits, "logits", torch.float32), T, H, I, E, k,
+        _dev(w13_q, "w13_q", torch.int32), _dev(w13_s, "w13_s", _BF16), _dev(w2_q, "w2_q", torch.int32),
+        _dev(w2_s, "w2_s", _BF16), _dev(out, "out", _BF16), _dev(topk_ids_out, "topk_ids_out", torch.int32),
+        _dev(topk_w_out, "topk_w_out", torch.float32), _stream(stream)))
     return out
 
 
