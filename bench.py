@@ -319,6 +319,8 @@ def main():
     ap.add_argument("--impl", default="moeq", choices=["moeq", "reference"])
     ap.add_argument("--headline-only", action="store_true", help="skip the secondary workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="override E of the headline workload (small cases for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -339,7 +341,7 @@ def main():
         flush_buf.fill_(1)
 
     # ---- headline: decode W4A16 -----------------------------------------------------------
-    d = W.make_moe(W.WORKLOADS["decode_w4a16"], device="cuda")
+    d = W.make_moe(W.WORKLOADS["decode_w4a16"], device="cuda", E=args.experts)
     n_active = touched_experts(moeq, d)
     w13_bytes = W.w4a16_expert_bytes(d["H"], d["I"]) * 2 // 3
     step_bytes = n_active * W.w4a16_expert_bytes(d["H"], d["I"])
@@ -370,7 +372,7 @@ def main():
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": "decode_w4a16 T=32 H=7168 I=2048 E=384 k=8 (INT4 group-32, bf16 scales)",
+        "config": {"workload": f"decode_w4a16 T=32 H=7168 I=2048 E={d['E']} k=8 (INT4 group-32, bf16 scales)",
                    "touched_experts": n_active, "weight_bytes_per_step": step_bytes,
                    "l2": f"flushed between steps ({L2_FLUSH_BYTES >> 20} MB write), outside the timed events",
                    "parallelism": f"replicas x{world}"},

@@ -8,9 +8,11 @@
 // Work split: one CTA per (align block of BM slots = grid x, tile of output features = grid y);
 // consecutive CTAs take consecutive blocks, so the blocks of one expert share its weights in L2.
 // Each warp owns 16 (gate/up) or 32 (down) output rows for the whole K range and streams its
-// packed weights straight from HBM into registers (16 B per lane per 128 inputs, no shared-memory round trip:
-// the decode shapes are HBM-bound and every weight byte is used by exactly one warp). A
-// dequantized 32-bit word feeds two m16n8k16 k-steps directly as A fragments.
+// packed weights from HBM through its own multi-stage cp.async ring in shared memory (16 B per
+// lane per 128 inputs per row set; five stages in flight hide the HBM latency without holding
+// registers). Every weight byte is used by exactly one warp, so the dequantized weights never go
+// back to shared memory: a dequantized 32-bit word feeds two m16n8k16 k-steps directly as A
+// fragments.
 //
 // Input permutation. The sum over K does not care about order, so inside a 128-input
 // "quad-group" lane t (of a 4-lane quad) takes the 32 inputs of group t = 16 contiguous bytes of
@@ -53,6 +55,12 @@ __device__ __forceinline__ void act_pairs(const uint4 &v, uint32_t (&b)[4])
 
 }  // namespace
 
+// Per-warp weight ring: each stage holds one 128-input quad-group of the warp's 4 row sets
+// (16 B per lane per row set, lane-private slots) and their 4 bf16 scales per row (8 B per row,
+// copied by lane (g, t) for row set t, row g and shared across the warp).
+constexpr int kW4Stages = 6;
+constexpr int kW4StageBytes = 4 * 32 * 16 + 4 * 8 * 8;  // 2048 B codes + 256 B scales
+
 // MODE_GATEUP: rows [f0, f0+16) (gate) and [I + f0, I + f0 + 16) (up) of W13; epilogue writes
 //              h[slot, f] = bf16(silu(gate) * up).
 // MODE_DOWN:   rows [r0, r0+32) of W2; epilogue writes ys[slot, r] = topk_w[slot] * y (f32).
@@ -60,6 +68,9 @@ template <int BM, int WARPS, int MODE>
 __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4GroupedArgs a)
 {
     constexpr int MS = BM / 8;  // token sub-tiles of 8 columns
+    constexpr int S = kW4Stages;
+    constexpr bool kActPrefetch = MS <= 2;
+    extern __shared__ __align__(16) unsigned char smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
     const int blk = blockIdx.x;
@@ -92,10 +103,26 @@ __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4Grouped
 
     const int32_t *wq = a.wq + (size_t)e * a.n_rows * KW;
     const uint16_t *wsc = a.ws + (size_t)e * a.n_rows * KG;
-    const int32_t *wr[4] = {wq + (size_t)(rowA + g) * KW, wq + (size_t)(rowA + g + 8) * KW,
-                            wq + (size_t)(rowB + g) * KW, wq + (size_t)(rowB + g + 8) * KW};
-    const uint16_t *sr[4] = {wsc + (size_t)(rowA + g) * KG, wsc + (size_t)(rowA + g + 8) * KG,
-                             wsc + (size_t)(rowB + g) * KG, wsc + (size_t)(rowB + g + 8) * KG};
+    const int row_of_set[4] = {rowA + g, rowA + g + 8, rowB + g, rowB + g + 8};
+    const int32_t *wr[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) wr[r] = wq + (size_t)row_of_set[r] * KW + 4 * t;
+    const uint16_t *my_scale_row = wsc + (size_t)row_of_set[t] * KG;  // copied by this lane
+
+    unsigned char *ring = smem + (size_t)warp * S * kW4StageBytes;
+    auto code_slot = [&](int st, int r) { return ring + st * kW4StageBytes + r * 512 + lane * 16; };
+    auto scale_slot = [&](int st, int r, int gg) { return ring + st * kW4StageBytes + 2048 + (r * 8 + gg) * 8; };
+
+    const int NQ = K / 128;
+    auto issue = [&](int q) {
+        if (q < NQ) {
+            const int st = q % S;
+#pragma unroll
+            for (int r = 0; r < 4; ++r) cp_async16_stream(code_slot(st, r), wr[r] + 16 * q);
+            cp_async8(scale_slot(st, t, g), my_scale_row + 4 * q);
+        }
+        cp_async_commit();  // possibly empty: keeps the group count uniform
+    };
 
     float accA[MS][4], accB[MS][4];
 #pragma unroll
@@ -103,24 +130,43 @@ __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4Grouped
 #pragma unroll
         for (int i = 0; i < 4; ++i) { accA[s][i] = 0.f; accB[s][i] = 0.f; }
 
-    const int NQ = K / 128;
-    uint4 wcur[4];
 #pragma unroll
-    for (int r = 0; r < 4; ++r) wcur[r] = ld_stream_v4(wr[r] + 4 * t);
+    for (int q = 0; q < S - 1; ++q) issue(q);
+
+    uint4 xcur[kActPrefetch ? MS : 1][4];
+    if (kActPrefetch) {
+#pragma unroll
+        for (int s = 0; s < MS; ++s)
+#pragma unroll
+            for (int m = 0; m < 4; ++m)
+                xcur[s][m] = act_row[s] ? ld_v4(act_row[s] + 32 * t + 8 * m) : make_uint4(0u, 0u, 0u, 0u);
+    }
 
     for (int q = 0; q < NQ; ++q) {
-        // prefetch the next quad-group's words while this one is consumed
-        uint4 wnext[4];
-        const int qn = (q + 1 < NQ) ? q + 1 : q;
+        cp_async_wait<S - 2>();
+        __syncwarp();
+        const int st = q % S;
+        uint4 wcur[4];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) wnext[r] = ld_stream_v4(wr[r] + 16 * qn + 4 * t);
+        for (int r = 0; r < 4; ++r) wcur[r] = *reinterpret_cast<const uint4 *>(code_slot(st, r));
         uint32_t sc[4];
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
-            const uint32_t s16 = __ldg(sr[r] + 4 * q + t);
+            const uint32_t s16 = reinterpret_cast<const uint16_t *>(scale_slot(st, r, g))[t];
             sc[r] = s16 | (s16 << 16);
         }
+        issue(q + S - 1);  // refills the slot every lane finished reading in iteration q - 1
+
+        uint4 xnext[kActPrefetch ? MS : 1][4];
         const int kofs = 128 * q + 32 * t;
+        if (kActPrefetch) {
+            const int kn = (q + 1 < NQ) ? kofs + 128 : kofs;
+#pragma unroll
+            for (int s = 0; s < MS; ++s)
+#pragma unroll
+                for (int m = 0; m < 4; ++m)
+                    xnext[s][m] = act_row[s] ? ld_v4(act_row[s] + kn + 8 * m) : make_uint4(0u, 0u, 0u, 0u);
+        }
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
             const uint32_t words[4] = {(&wcur[0].x)[m], (&wcur[1].x)[m], (&wcur[2].x)[m], (&wcur[3].x)[m]};
@@ -129,8 +175,9 @@ __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4Grouped
             for (int r = 0; r < 4; ++r) d[r] = dequant_word(words[r], sc[r]);
 #pragma unroll
             for (int s = 0; s < MS; ++s) {
-                uint4 xv = make_uint4(0u, 0u, 0u, 0u);
-                if (act_row[s]) xv = ld_v4(act_row[s] + kofs + 8 * m);
+                uint4 xv;
+                if (kActPrefetch) xv = xcur[s][m];
+                else xv = act_row[s] ? ld_v4(act_row[s] + kofs + 8 * m) : make_uint4(0u, 0u, 0u, 0u);
                 uint32_t b[4];
                 act_pairs(xv, b);
                 // k-step 2m: pairs 0/1; k-step 2m+1: pairs 2/3
@@ -140,9 +187,14 @@ __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4Grouped
                 mma_bf16_16816(accB[s], d[2].p[2], d[3].p[2], d[2].p[3], d[3].p[3], b[2], b[3]);
             }
         }
+        if (kActPrefetch) {
 #pragma unroll
-        for (int r = 0; r < 4; ++r) wcur[r] = wnext[r];
+            for (int s = 0; s < MS; ++s)
+#pragma unroll
+                for (int m = 0; m < 4; ++m) xcur[s][m] = xnext[s][m];
+        }
     }
+    cp_async_wait<0>();
 
     // epilogue: lane holds rows (g, g+8) x columns (2t, 2t+1) of each sub-tile
 #pragma unroll
@@ -171,8 +223,15 @@ template <int BM, int WARPS, int MODE>
 static void launch_bm(const W4GroupedArgs &a, int max_blocks, cudaStream_t s)
 {
     const int rows_per_cta = (MODE == MODE_GATEUP ? 16 : 32) * WARPS;
+    const size_t smem = (size_t)WARPS * kW4Stages * kW4StageBytes;
+    static bool attr_set = false;  // per template instance; the attribute is per function
+    if (!attr_set) {
+        cudaFuncSetAttribute(w4a16_grouped_mma_kernel<BM, WARPS, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+        attr_set = true;
+    }
     dim3 grid(max_blocks, cdiv(a.n_out, rows_per_cta));
-    w4a16_grouped_mma_kernel<BM, WARPS, MODE><<<grid, WARPS * 32, 0, s>>>(a);
+    w4a16_grouped_mma_kernel<BM, WARPS, MODE><<<grid, WARPS * 32, smem, s>>>(a);
 }
 
 void launch_w4a16_grouped_mma(const W4GroupedArgs &a, int mode, int block_m, int max_blocks, cudaStream_t s)
