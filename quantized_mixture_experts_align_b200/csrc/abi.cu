@@ -9,6 +9,7 @@
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "tc_common.cuh"
 
 #define MOEQ_VERSION "moeq 0.1 (sm_100a)"
 
@@ -31,8 +32,6 @@ int check_launch(const char *what)
     if (e != cudaSuccess) return set_error(MOEQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
     return MOEQ_OK;
 }
-
-__device__ int g_device_status = 0;
 
 // SM count of the current device, looked up once per device.
 static int num_sms()
@@ -112,6 +111,10 @@ static int pick_block_m(long T, int k, int E)
     if (tok_e <= 24.0) return 32;
     return 64;
 }
+
+// Dense block-FP8: from this many rows on, the tcgen05 kernel (128-row tiles, tensor-core bound)
+// replaces the register-fed swap-AB kernel (weight-streaming, HBM bound).
+static int kDenseTcMinM = 128;
 
 static int pick_block_m_dense(int M)
 {
@@ -473,6 +476,14 @@ int w8a8_block_fp8_matmul(const uint8_t *A, const float *As, const uint8_t *B, c
     a.E = 1;
     a.n_slots = M;
     a.c_out = C;
+    if (M >= kDenseTcMinM) {
+        Fp8TcArgs t{As, Bs, C, M, N, K, device_status_ptr()};
+        if (!t.status) return set_error(MOEQ_ERR_CUDA, "w8a8_block_fp8_matmul: no device status word");
+        trace::Scope ts(trace::DENSE, (cudaStream_t)stream);
+        const int rc = launch_fp8_tc_gemm(t, A, B, (cudaStream_t)stream);
+        if (rc) return rc;
+        return check_launch("w8a8_block_fp8_matmul");
+    }
     const int bm = pick_block_m_dense(M);
     {
         trace::Scope ts(trace::DENSE, (cudaStream_t)stream);
@@ -519,12 +530,14 @@ int moe_trace_read(double *stage_ms, long long *stage_calls, int n_stages, int r
 int moe_device_status(int clear)
 {
     g_err[0] = 0;
+    int *p = device_status_ptr();
+    if (!p) return set_error(MOEQ_ERR_CUDA, "moe_device_status: no device status word");
     int v = 0;
-    cudaError_t e = cudaMemcpyFromSymbol(&v, g_device_status, sizeof v);
+    cudaError_t e = cudaMemcpy(&v, p, sizeof v, cudaMemcpyDeviceToHost);
     if (e != cudaSuccess) return set_error(MOEQ_ERR_CUDA, "moe_device_status: %s", cudaGetErrorString(e));
     if (clear) {
         const int z = 0;
-        e = cudaMemcpyToSymbol(g_device_status, &z, sizeof z);
+        e = cudaMemcpy(p, &z, sizeof z, cudaMemcpyHostToDevice);
         if (e != cudaSuccess) return set_error(MOEQ_ERR_CUDA, "moe_device_status: %s", cudaGetErrorString(e));
     }
     return v ? MOEQ_ERR_DEVICE_TIMEOUT : MOEQ_OK;

@@ -47,6 +47,14 @@ struct F8GroupedArgs {
     uint16_t *c_out;         // dense: [M, N] bf16
 };
 
+struct Fp8TcArgs {
+    const float *As;   // [M, K/128]
+    const float *Bs;   // [N/128, K/128]
+    uint16_t *C;       // [M, N] bf16
+    int M, N, K;
+    int *status;       // kernel status word (bounded waits that gave up)
+};
+
 void launch_route_topk(const float *logits, int T, int E, int k, int32_t *ids, float *w, cudaStream_t s);
 void launch_align(const int32_t *topk_ids, int n, int E, int B, int32_t *sorted_ids, int32_t *expert_ids,
                   int32_t *ntp, cudaStream_t s);
@@ -54,5 +62,7 @@ void launch_combine(const float *ys, int T, int k, int H, uint16_t *out, int num
 void launch_fp8_act_quant(const uint16_t *x, int rows, int cols, uint8_t *q, float *s, cudaStream_t st);
 void launch_w4a16_grouped_mma(const W4GroupedArgs &a, int mode, int block_m, int max_blocks, cudaStream_t s);
 void launch_fp8_grouped_mma(const F8GroupedArgs &a, int mode, int block_m, int max_blocks, cudaStream_t s);
+// tcgen05 block-FP8 GEMM: A [M, K] and B [N, K] E4M3, K % 128 == 0, N % 128 == 0. Returns a status.
+int launch_fp8_tc_gemm(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B, cudaStream_t s);
 
 }  // namespace moeq

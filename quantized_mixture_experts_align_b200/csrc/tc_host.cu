@@ -1,0 +1,61 @@
+// Host utilities of the tensor-core kernels: TMA tensor maps (encoded through the driver entry
+// point, so the library needs no link-time dependency on libcuda) and the device status word that
+// kernels with bounded waits write when a wait gives up.
+#include <mutex>
+
+#include "tc_common.cuh"
+
+namespace moeq {
+
+__device__ int g_device_status = 0;
+
+namespace {
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+std::mutex g_mu;
+EncodeTiledFn g_encode = nullptr;
+int *g_status_addr[64] = {};
+}  // namespace
+
+int make_tmap_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype, int elem_bytes, uint64_t rows,
+                 uint64_t cols, uint32_t box_rows, uint32_t box_cols)
+{
+    {
+        std::lock_guard<std::mutex> g(g_mu);
+        if (!g_encode) {
+            void *fn = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            const cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+            if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
+                return set_error(MOEQ_ERR_CUDA, "cuTensorMapEncodeTiled unavailable: %s", cudaGetErrorString(e));
+            g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+        }
+    }
+    if (reinterpret_cast<uintptr_t>(base) % 16 || (cols * elem_bytes) % 16)
+        return set_error(MOEQ_ERR_UNSUPPORTED, "tensor map: base and row pitch must be 16-byte aligned");
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * (uint64_t)elem_bytes};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint32_t estride[2] = {1, 1};
+    const CUresult r = g_encode(map, dtype, 2, const_cast<void *>(base), dims, strides, box, estride,
+                                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return set_error(MOEQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+    return MOEQ_OK;
+}
+
+int *device_status_ptr()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> g(g_mu);
+    if (!g_status_addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+        g_status_addr[dev] = static_cast<int *>(p);
+    }
+    return g_status_addr[dev];
+}
+
+}  // namespace moeq

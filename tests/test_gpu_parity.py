@@ -249,7 +249,13 @@ def test_dense_fp8_small_shapes_all_rows(M):
     _dense_parity(M, 512, 1024, np.arange(M, dtype=np.int32))
 
 
-@pytest.mark.parametrize("M", [1, 16, 128, 4096])
+@pytest.mark.parametrize("M,N,K", [(128, 256, 1024), (200, 512, 512), (300, 384, 896), (1000, 256, 7168)])
+def test_dense_fp8_tensor_core_shapes_all_rows(M, N, K):
+    """Row counts at and past the tcgen05 threshold, ragged M tails, N not a multiple of 256."""
+    _dense_parity(M, N, K, np.arange(M, dtype=np.int32))
+
+
+@pytest.mark.parametrize("M", [1, 16, 128, 1000, 4096])
 def test_dense_fp8_full_shape_sampled(M):
     rows = np.unique(np.array([0, M - 1, M // 2, M // 3], np.int32))
     _dense_parity(M, 24576, 7168, rows)
