@@ -174,21 +174,33 @@ static size_t w4a16_layout(Carve &c, long T, int H, int I, int E, int k, RouteBu
     return c.used;
 }
 
+// Block-FP8 layer schedule: from this many routed rows per expert on (mean T*k/E), the grouped
+// GEMMs run on the tensor-core kernel over 128-row expert blocks; below, the register-fed swap-AB
+// kernel streams the weights for the few rows each expert has.
+static bool fp8_use_tc(long T, int k, int E) { return (double)T * k / (double)E >= 16.0; }
+
 static size_t fp8_layout(Carve &c, long T, int H, int I, int E, int k, RouteBufs *rb, uint8_t **xq, float **xs,
-                         uint8_t **hq, float **hs, float **ys)
+                         uint8_t **hq, float **hs, float **ys, uint8_t **xg = nullptr, float **xsg = nullptr)
 {
-    RouteBufs r = carve_route(c, T, k, E, pick_block_m(T, k, E));
+    const bool tcp = fp8_use_tc(T, k, E);
+    RouteBufs r = carve_route(c, T, k, E, tcp ? 128 : pick_block_m(T, k, E));
+    const size_t cap = (size_t)T * k + (size_t)E * (r.block_m - 1);   // aligned rows
+    const size_t hrows = tcp ? cap : (size_t)T * k;                     // h rows: aligned or by slot
     uint8_t *xqp = c.take<uint8_t>((size_t)T * H);
     float *xsp = c.take<float>((size_t)T * (H / 128));
-    uint8_t *hqp = c.take<uint8_t>((size_t)T * k * I);
-    float *hsp = c.take<float>((size_t)T * k * (I / 128));
+    uint8_t *hqp = c.take<uint8_t>(hrows * I);
+    float *hsp = c.take<float>(hrows * (I / 128));
     float *yp = c.take<float>((size_t)T * k * H);
+    uint8_t *xgp = tcp ? c.take<uint8_t>(cap * H) : nullptr;
+    float *xsgp = tcp ? c.take<float>(cap * (H / 128)) : nullptr;
     if (rb) *rb = r;
     if (xq) *xq = xqp;
     if (xs) *xs = xsp;
     if (hq) *hq = hqp;
     if (hs) *hs = hsp;
     if (ys) *ys = yp;
+    if (xg) *xg = xgp;
+    if (xsg) *xsg = xsgp;
     return c.used;
 }
 
@@ -388,12 +400,13 @@ int moe_w8a8_block_fp8_forward(const uint16_t *x, const float *logits, int T, in
     cudaStream_t s = (cudaStream_t)stream;
     Carve c(ws);
     RouteBufs r;
-    uint8_t *xq, *hq;
-    float *xs, *hs, *ys;
-    fp8_layout(c, T, H, I, E, k, &r, &xq, &xs, &hq, &hs, &ys);
+    uint8_t *xq, *hq, *xg;
+    float *xs, *hs, *ys, *xsg;
+    fp8_layout(c, T, H, I, E, k, &r, &xq, &xs, &hq, &hs, &ys, &xg, &xsg);
     int32_t *ids = topk_ids_out ? topk_ids_out : r.ids;
     float *tw = topk_w_out ? topk_w_out : r.w;
     const int n = T * k;
+    const bool tcp = fp8_use_tc(T, k, E);
 
     {
         trace::Scope ts(trace::ROUTE, s);
@@ -406,41 +419,83 @@ int moe_w8a8_block_fp8_forward(const uint16_t *x, const float *logits, int T, in
     {
         trace::Scope ts(trace::ACT_QUANT, s);
         launch_fp8_act_quant(x, T, H, xq, xs, s);
+        if (tcp) launch_gather_fp8_rows(xq, xs, H, k, r.sorted, r.ntp, n, r.max_blocks * 128, xg, xsg, num_sms(), s);
     }
 
-    F8GroupedArgs a{};
-    a.E = E;
-    a.sorted_ids = r.sorted;
-    a.expert_ids = r.eids;
-    a.num_tokens_padded = r.ntp;
-    a.n_slots = n;
-    a.topk_w = tw;
-    a.act = xq;
-    a.act_s = xs;
-    a.act_row_div = k;
-    a.w = w13;
-    a.w_s = w13_s;
-    a.K = H;
-    a.n_out = I;
-    a.n_rows = 2 * I;
-    a.hq_out = hq;
-    a.hs_out = hs;
-    {
-        trace::Scope ts(trace::GATE_UP, s);
-        launch_fp8_grouped_mma(a, MODE_GATEUP, r.block_m, r.max_blocks, s);
-    }
-    a.act = hq;
-    a.act_s = hs;
-    a.act_row_div = 1;
-    a.w = w2;
-    a.w_s = w2_s;
-    a.K = I;
-    a.n_out = H;
-    a.n_rows = H;
-    a.y_out = ys;
-    {
-        trace::Scope ts(trace::DOWN, s);
-        launch_fp8_grouped_mma(a, MODE_DOWN, r.block_m, r.max_blocks, s);
+    if (tcp) {
+        int *status = device_status_ptr();
+        if (!status) return set_error(MOEQ_ERR_CUDA, "moe_w8a8_block_fp8_forward: no device status word");
+        const int cap = r.max_blocks * 128;
+        Fp8TcArgs t{};
+        t.status = status;
+        t.E = E;
+        t.sorted_ids = r.sorted;
+        t.expert_ids = r.eids;
+        t.ntp = r.ntp;
+        t.n_slots = n;
+        t.topk_w = tw;
+        // gate/up + SiLU*up + E4M3 quantization of the intermediate (rows in aligned order)
+        t.a_scale = xsg;
+        t.b_scale = w13_s;
+        t.M = cap;
+        t.N = I;
+        t.K = H;
+        t.rows_per_expert = 2 * I;
+        t.hq = hq;
+        t.hs = hs;
+        int rc;
+        {
+            trace::Scope ts(trace::GATE_UP, s);
+            rc = launch_fp8_tc_grouped(t, TC_GATEUP, xg, w13, E, r.max_blocks, s);
+        }
+        if (rc) return rc;
+        // down, routing weight applied, rows scattered back to their slots
+        t.a_scale = hs;
+        t.b_scale = w2_s;
+        t.N = H;
+        t.K = I;
+        t.rows_per_expert = H;
+        t.ys = ys;
+        {
+            trace::Scope ts(trace::DOWN, s);
+            rc = launch_fp8_tc_grouped(t, TC_DOWN, hq, w2, E, r.max_blocks, s);
+        }
+        if (rc) return rc;
+    } else {
+        F8GroupedArgs a{};
+        a.E = E;
+        a.sorted_ids = r.sorted;
+        a.expert_ids = r.eids;
+        a.num_tokens_padded = r.ntp;
+        a.n_slots = n;
+        a.topk_w = tw;
+        a.act = xq;
+        a.act_s = xs;
+        a.act_row_div = k;
+        a.w = w13;
+        a.w_s = w13_s;
+        a.K = H;
+        a.n_out = I;
+        a.n_rows = 2 * I;
+        a.hq_out = hq;
+        a.hs_out = hs;
+        {
+            trace::Scope ts(trace::GATE_UP, s);
+            launch_fp8_grouped_mma(a, MODE_GATEUP, r.block_m, r.max_blocks, s);
+        }
+        a.act = hq;
+        a.act_s = hs;
+        a.act_row_div = 1;
+        a.w = w2;
+        a.w_s = w2_s;
+        a.K = I;
+        a.n_out = H;
+        a.n_rows = H;
+        a.y_out = ys;
+        {
+            trace::Scope ts(trace::DOWN, s);
+            launch_fp8_grouped_mma(a, MODE_DOWN, r.block_m, r.max_blocks, s);
+        }
     }
     {
         trace::Scope ts(trace::COMBINE, s);
@@ -477,7 +532,14 @@ int w8a8_block_fp8_matmul(const uint8_t *A, const float *As, const uint8_t *B, c
     a.n_slots = M;
     a.c_out = C;
     if (M >= kDenseTcMinM) {
-        Fp8TcArgs t{As, Bs, C, M, N, K, device_status_ptr()};
+        Fp8TcArgs t{};
+        t.a_scale = As;
+        t.b_scale = Bs;
+        t.C = C;
+        t.M = M;
+        t.N = N;
+        t.K = K;
+        t.status = device_status_ptr();
         if (!t.status) return set_error(MOEQ_ERR_CUDA, "w8a8_block_fp8_matmul: no device status word");
         trace::Scope ts(trace::DENSE, (cudaStream_t)stream);
         const int rc = launch_fp8_tc_gemm(t, A, B, (cudaStream_t)stream);

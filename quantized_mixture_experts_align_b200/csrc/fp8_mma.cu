@@ -45,6 +45,39 @@ void launch_fp8_act_quant(const uint16_t *x, int rows, int cols, uint8_t *q, flo
 }
 
 // ------------------------------------------------------------------------------------------
+// Gather of quantized rows into aligned (expert-contiguous) order: one warp per row, 16-byte
+// copies; padding rows (pad slot, or past the padded count) are written as zeros.
+// ------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) gather_fp8_rows_kernel(const uint8_t *__restrict__ xq,
+                                                              const float *__restrict__ xs, int H, int k,
+                                                              const int32_t *__restrict__ sorted_ids,
+                                                              const int32_t *__restrict__ ntp, int n_slots,
+                                                              int cap_rows, uint8_t *__restrict__ xg,
+                                                              float *__restrict__ xsg)
+{
+    const int lane = threadIdx.x & 31;
+    const int rows = min(__ldg(ntp), cap_rows);
+    const int G = H / 128;
+    for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += gridDim.x * (blockDim.x >> 5)) {
+        const int slot = __ldg(sorted_ids + r);
+        const bool real = slot < n_slots;
+        const uint4 *src = reinterpret_cast<const uint4 *>(xq + (size_t)(real ? slot / k : 0) * H);
+        uint4 *dst = reinterpret_cast<uint4 *>(xg + (size_t)r * H);
+        for (int i = lane; i < H / 16; i += 32) dst[i] = real ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
+        for (int i = lane; i < G; i += 32) xsg[(size_t)r * G + i] = real ? __ldg(xs + (size_t)(slot / k) * G + i) : 0.f;
+    }
+}
+
+void launch_gather_fp8_rows(const uint8_t *xq, const float *xs, int H, int k, const int32_t *sorted_ids,
+                            const int32_t *ntp, int n_slots, int cap_rows, uint8_t *xg, float *xsg, int num_sms,
+                            cudaStream_t s)
+{
+    if (cap_rows <= 0) return;
+    const int blocks = min(cdiv(cap_rows, 8), num_sms * 8);
+    gather_fp8_rows_kernel<<<blocks, 256, 0, s>>>(xq, xs, H, k, sorted_ids, ntp, n_slots, cap_rows, xg, xsg);
+}
+
+// ------------------------------------------------------------------------------------------
 // Block-scaled FP8 GEMM, weights as MMA A (16 rows per tile), tokens as MMA B (8 per sub-tile).
 // Lane t of a quad reads 16 contiguous bytes per 64 inputs; its 4 words feed two k-steps as the
 // A (and, for the token column, B) fragments directly - both operands use the same permutation

@@ -47,12 +47,25 @@ struct F8GroupedArgs {
     uint16_t *c_out;         // dense: [M, N] bf16
 };
 
+enum { TC_DENSE = 0, TC_GATEUP = 1, TC_DOWN = 2 };
+
 struct Fp8TcArgs {
-    const float *As;   // [M, K/128]
-    const float *Bs;   // [N/128, K/128]
-    uint16_t *C;       // [M, N] bf16
-    int M, N, K;
-    int *status;       // kernel status word (bounded waits that gave up)
+    const float *a_scale;   // [M, K/128]: As (dense) or the gathered / intermediate row scales
+    const float *b_scale;   // dense: Bs [N/128, K/128]; grouped: weight scales [E, rows/128, K/128]
+    int M, N, K;            // A rows; output columns (dense N, gate/up I, down H); inputs
+    int *status;            // kernel status word (bounded waits that gave up)
+    uint16_t *C;            // dense: [M, N] bf16
+    // grouped
+    int E;
+    int rows_per_expert;    // weight rows per expert (2I or H)
+    const int32_t *sorted_ids;
+    const int32_t *expert_ids;
+    const int32_t *ntp;
+    int n_slots;
+    const float *topk_w;
+    uint8_t *hq;            // gate/up out: [M, N] E4M3
+    float *hs;              // gate/up out: [M, N/128]
+    float *ys;              // down out: [n_slots, N] f32, routing weight applied
 };
 
 void launch_route_topk(const float *logits, int T, int E, int k, int32_t *ids, float *w, cudaStream_t s);
@@ -64,5 +77,14 @@ void launch_w4a16_grouped_mma(const W4GroupedArgs &a, int mode, int block_m, int
 void launch_fp8_grouped_mma(const F8GroupedArgs &a, int mode, int block_m, int max_blocks, cudaStream_t s);
 // tcgen05 block-FP8 GEMM: A [M, K] and B [N, K] E4M3, K % 128 == 0, N % 128 == 0. Returns a status.
 int launch_fp8_tc_gemm(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B, cudaStream_t s);
+// tcgen05 grouped block-FP8 GEMM over expert-contiguous rows A [M, K] (128-row blocks, one expert
+// each, per expert_ids / ntp) and weights W [E * rows_per_expert, K]; mode TC_GATEUP or TC_DOWN.
+int launch_fp8_tc_grouped(const Fp8TcArgs &a, int mode, const uint8_t *A, const uint8_t *W, int E, int max_blocks,
+                          cudaStream_t s);
+// Copies E4M3 rows (and their scales) of the routed slots into aligned order: row r takes token
+// sorted_ids[r] / k; padding rows become zero.
+void launch_gather_fp8_rows(const uint8_t *xq, const float *xs, int H, int k, const int32_t *sorted_ids,
+                            const int32_t *ntp, int n_slots, int cap_rows, uint8_t *xg, float *xsg, int num_sms,
+                            cudaStream_t s);
 
 }  // namespace moeq

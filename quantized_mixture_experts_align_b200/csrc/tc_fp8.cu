@@ -18,6 +18,14 @@
 //               (= tile rows) and one half of the columns, keeps the running f32 sums in
 //               registers, and finally writes bf16 C.
 // Every wait is bounded; a wait that gives up flags the kernel status word and the CTA drains.
+//
+// The same kernel runs the grouped expert GEMMs of the block-FP8 MoE layer over expert-contiguous
+// rows (the routed slots gathered in aligned order, every 128-row block owned by one expert):
+//   TC_GATEUP  B stage = 128 gate rows + 128 up rows of the block's expert; the epilogue forms
+//              a = silu(g) * u and quantizes it per row and 128-feature group to E4M3 + f32 scale
+//              (the two column halves of a row meet through shared memory for the group max);
+//   TC_DOWN    B = 256 rows of W2[e]; the epilogue multiplies by the slot's routing weight and
+//              writes the f32 slot row for the combine.
 #include "kernels.cuh"
 #include "tc_common.cuh"
 
@@ -38,15 +46,16 @@ struct Fp8TcShape {
     static constexpr int kStageBytes = kABytes + kBBytes;
     static constexpr int kTmemCols = 2 * BN;  // two partial buffers (256 or 512 columns)
     static constexpr int kColsPerWarp = BN / 2;
-    static constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + 1024 + 256;
+    static constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + 1024 + 256 + 2 * 128 * 4;
 };
 
-template <int BN>
+template <int BN, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     fp8_tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                        Fp8TcArgs a)
 {
     using Sh = Fp8TcShape<BN>;
+    static_assert(MODE != TC_GATEUP || BN == 256, "gate/up tiles hold 128 gate + 128 up columns");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + kStages * Sh::kStageBytes);
@@ -59,8 +68,32 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int m0 = blockIdx.x * kBM;  // consecutive CTAs share a B (weight) tile in L2
-    const int n0 = blockIdx.y * BN;
     const int KB = a.K / kBK;
+    // output columns of this tile and the weight rows (in the [E * rows, K] weight matrix) loaded
+    // into the B stage: dense and down take BN consecutive rows; gate/up takes 128 gate + 128 up
+    int n0, brow0, brow1 = 0;
+    const float *bscale0, *bscale1 = nullptr;
+    if (MODE == TC_DENSE) {
+        n0 = blockIdx.y * BN;
+        brow0 = n0;
+        bscale0 = a.b_scale + (size_t)(n0 / 128) * KB;
+    } else {
+        if (m0 >= __ldg(a.ntp)) return;  // uniform over the CTA, before any barrier or allocation
+        const int e = __ldg(a.expert_ids + blockIdx.x);
+        if (e < 0 || e >= a.E) return;
+        const float *ws = a.b_scale + (size_t)e * (a.rows_per_expert / 128) * KB;
+        if (MODE == TC_GATEUP) {
+            n0 = blockIdx.y * 128;                      // feature tile
+            brow0 = e * a.rows_per_expert + n0;         // gate rows
+            brow1 = e * a.rows_per_expert + a.N + n0;   // up rows
+            bscale0 = ws + (size_t)(n0 / 128) * KB;
+            bscale1 = ws + (size_t)((a.N + n0) / 128) * KB;
+        } else {
+            n0 = blockIdx.y * BN;
+            brow0 = e * a.rows_per_expert + n0;
+            bscale0 = ws + (size_t)(n0 / 128) * KB;
+        }
+    }
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -92,7 +125,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint8_t *sa = smem + s * Sh::kStageBytes;
                 tc::mbar_arrive_expect_tx(&full[s], Sh::kStageBytes);
                 tc::tma_load_2d(sa, &tmA, &full[s], kb * kBK, m0);
-                tc::tma_load_2d(sa + Sh::kABytes, &tmB, &full[s], kb * kBK, n0);
+                if (MODE == TC_GATEUP) {
+                    tc::tma_load_2d(sa + Sh::kABytes, &tmB, &full[s], kb * kBK, brow0);
+                    tc::tma_load_2d(sa + Sh::kABytes + 128 * kBK, &tmB, &full[s], kb * kBK, brow1);
+                } else {
+                    tc::tma_load_2d(sa + Sh::kABytes, &tmB, &full[s], kb * kBK, brow0);
+                }
                 issued = kb + 1;
             }
             // no copy may still be landing in shared memory when the CTA exits
@@ -125,25 +163,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int ew = warp - 2, quarter = warp & 3, half = ew >> 2;
         const int row = quarter * 32 + lane;
         const int m = m0 + row;
-        const int col0 = half * COLS;
-        const float *as_row = a.As + (size_t)(m < a.M ? m : a.M - 1) * KB;
-        const float *bs_row = a.Bs + (size_t)((n0 + col0) / 128) * KB;
+        // TMEM columns of this warp: one contiguous half of the tile, or (gate/up) 64 gate columns
+        // and the 64 matching up columns
+        const int c_first = (MODE == TC_GATEUP) ? 64 * half : half * COLS;
+        const int c_second = (MODE == TC_GATEUP) ? 128 + 64 * half : half * COLS + COLS / 2;
+        const float *as_row = a.a_scale + (size_t)(m < a.M ? m : a.M - 1) * KB;
+        const float *bs_first = (MODE == TC_GATEUP) ? bscale0 : bscale0 + (size_t)((half * COLS) / 128) * KB;
+        const float *bs_second = (MODE == TC_GATEUP) ? bscale1 : bs_first;
         float acc[COLS];
 #pragma unroll
         for (int j = 0; j < COLS; ++j) acc[j] = 0.f;
         bool ok = true;
         for (int kb = 0; kb < KB && ok; ++kb) {
             const int buf = kb & 1;
-            const float sc = __ldg(as_row + kb) * __ldg(bs_row + kb);
+            const float sa = __ldg(as_row + kb);
+            const float sc0 = sa * __ldg(bs_first + kb), sc1 = sa * __ldg(bs_second + kb);
             // every lane waits, then the warp agrees: the tensor-memory loads below are warp-wide
             ok = __all_sync(0xFFFFFFFFu, tc::mbar_wait(&tfull[buf], (kb >> 1) & 1, abort_flag, a.status));
             if (!ok) break;
             tc::fence_after_sync();
-            const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + buf * BN + col0;
+            const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + buf * BN;
 #pragma unroll
             for (int c = 0; c < COLS / 32; ++c) {
+                const bool second = c >= COLS / 64;
+                const int col = (second ? c_second : c_first) + (c % (COLS / 64)) * 32;
+                const float sc = second ? sc1 : sc0;
                 uint32_t r[32];
-                tc::tmem_ld32(taddr + c * 32, r);
+                tc::tmem_ld32(taddr + col, r);
                 tc::tmem_wait_ld();
 #pragma unroll
                 for (int j = 0; j < 32; ++j) acc[c * 32 + j] = fmaf(__uint_as_float(r[j]), sc, acc[c * 32 + j]);
@@ -152,16 +198,57 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&tempty[buf]);
         }
-        if (ok && m < a.M) {
-            uint16_t *crow = a.C + (size_t)m * a.N + n0 + col0;
+        if (MODE == TC_DENSE) {
+            if (ok && m < a.M) {
+                uint16_t *crow = a.C + (size_t)m * a.N + n0 + half * COLS;
 #pragma unroll
-            for (int j = 0; j < COLS; j += 8) {
-                uint4 v;
-                v.x = pack_bf16x2(acc[j], acc[j + 1]);
-                v.y = pack_bf16x2(acc[j + 2], acc[j + 3]);
-                v.z = pack_bf16x2(acc[j + 4], acc[j + 5]);
-                v.w = pack_bf16x2(acc[j + 6], acc[j + 7]);
-                *reinterpret_cast<uint4 *>(crow + j) = v;
+                for (int j = 0; j < COLS; j += 8) {
+                    uint4 v;
+                    v.x = pack_bf16x2(acc[j], acc[j + 1]);
+                    v.y = pack_bf16x2(acc[j + 2], acc[j + 3]);
+                    v.z = pack_bf16x2(acc[j + 4], acc[j + 5]);
+                    v.w = pack_bf16x2(acc[j + 6], acc[j + 7]);
+                    *reinterpret_cast<uint4 *>(crow + j) = v;
+                }
+            }
+        } else if (MODE == TC_GATEUP) {
+            // a = silu(g) * u for features n0 + 64 half + j; E4M3 per row and 128-feature group
+            float amax = 0.f;
+#pragma unroll
+            for (int j = 0; j < 64; ++j) {
+                acc[j] = silu_f32(acc[j]) * acc[64 + j];
+                amax = fmaxf(amax, fabsf(acc[j]));
+            }
+            float *red = reinterpret_cast<float *>(tmem_slot + 4);  // [2][128] group maxima
+            red[half * 128 + row] = amax;
+            asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory");
+            amax = fmaxf(red[row], red[128 + row]);
+            const float sc = __fdiv_rn(fmaxf(amax, 1e-10f), 448.0f);
+            if (ok) {
+                uint8_t *hrow = a.hq + (size_t)m * a.N + n0 + 64 * half;
+#pragma unroll
+                for (int j = 0; j < 64; j += 16) {
+                    uint4 v;
+                    uint32_t *w = &v.x;
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) {
+                        const uint32_t lo = pack_e4m3x2(__fdiv_rn(acc[j + 4 * p], sc), __fdiv_rn(acc[j + 4 * p + 1], sc));
+                        const uint32_t hi = pack_e4m3x2(__fdiv_rn(acc[j + 4 * p + 2], sc), __fdiv_rn(acc[j + 4 * p + 3], sc));
+                        w[p] = lo | (hi << 16);
+                    }
+                    *reinterpret_cast<uint4 *>(hrow + j) = v;
+                }
+                if (half == 0) a.hs[(size_t)m * (a.N / 128) + n0 / 128] = sc;
+            }
+        } else {
+            const int slot = __ldg(a.sorted_ids + m);
+            if (ok && slot < a.n_slots) {
+                const float wt = __ldg(a.topk_w + slot);
+                float *yrow = a.ys + (size_t)slot * a.N + n0 + half * COLS;
+#pragma unroll
+                for (int j = 0; j < COLS; j += 4)
+                    *reinterpret_cast<float4 *>(yrow + j) =
+                        make_float4(wt * acc[j], wt * acc[j + 1], wt * acc[j + 2], wt * acc[j + 3]);
             }
         }
     }
@@ -171,22 +258,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 1) tc::tmem_dealloc(tmem, Sh::kTmemCols);
 }
 
-template <int BN>
-int launch_bn(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B, cudaStream_t s)
+template <int BN, int MODE>
+int launch_tc(const Fp8TcArgs &a, const CUtensorMap &tmA, const CUtensorMap &tmB, int grid_x, int grid_y,
+              cudaStream_t s)
 {
     using Sh = Fp8TcShape<BN>;
-    CUtensorMap tmA, tmB;
-    int rc = make_tmap_2d(&tmA, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.M, (uint64_t)a.K, kBM, kBK);
-    if (rc) return rc;
-    rc = make_tmap_2d(&tmB, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.N, (uint64_t)a.K, BN, kBK);
-    if (rc) return rc;
     static bool attr = false;
     if (!attr) {
-        cudaFuncSetAttribute(fp8_tc_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Sh::kSmemBytes);
+        const cudaError_t e = cudaFuncSetAttribute(fp8_tc_gemm_kernel<BN, MODE>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Sh::kSmemBytes);
+        if (e != cudaSuccess)
+            return set_error(MOEQ_ERR_CUDA, "tcgen05 FP8 GEMM: shared-memory attribute: %s", cudaGetErrorString(e));
         attr = true;
     }
-    dim3 grid(cdiv(a.M, kBM), a.N / BN);
-    fp8_tc_gemm_kernel<BN><<<grid, kThreads, Sh::kSmemBytes, s>>>(tmA, tmB, a);
+    if (grid_x <= 0 || grid_y <= 0) return MOEQ_OK;
+    fp8_tc_gemm_kernel<BN, MODE><<<dim3(grid_x, grid_y), kThreads, Sh::kSmemBytes, s>>>(tmA, tmB, a);
     return MOEQ_OK;
 }
 
@@ -194,8 +280,29 @@ int launch_bn(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B, cudaStream
 
 int launch_fp8_tc_gemm(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B, cudaStream_t s)
 {
-    if (a.N % 256 == 0) return launch_bn<256>(a, A, B, s);
-    return launch_bn<128>(a, A, B, s);
+    const int bn = (a.N % 256 == 0) ? 256 : 128;
+    CUtensorMap tmA, tmB;
+    int rc = make_tmap_2d(&tmA, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.M, (uint64_t)a.K, kBM, kBK);
+    if (rc) return rc;
+    rc = make_tmap_2d(&tmB, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.N, (uint64_t)a.K, bn, kBK);
+    if (rc) return rc;
+    if (bn == 256) return launch_tc<256, TC_DENSE>(a, tmA, tmB, cdiv(a.M, kBM), a.N / 256, s);
+    return launch_tc<128, TC_DENSE>(a, tmA, tmB, cdiv(a.M, kBM), a.N / 128, s);
+}
+
+int launch_fp8_tc_grouped(const Fp8TcArgs &a, int mode, const uint8_t *A, const uint8_t *W, int E, int max_blocks,
+                          cudaStream_t s)
+{
+    CUtensorMap tmA, tmB;
+    int rc = make_tmap_2d(&tmA, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.M, (uint64_t)a.K, kBM, kBK);
+    if (rc) return rc;
+    const uint32_t box = (mode == TC_GATEUP || a.N % 256 != 0) ? 128 : 256;
+    rc = make_tmap_2d(&tmB, W, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)E * a.rows_per_expert, (uint64_t)a.K, box,
+                      kBK);
+    if (rc) return rc;
+    if (mode == TC_GATEUP) return launch_tc<256, TC_GATEUP>(a, tmA, tmB, max_blocks, a.N / 128, s);
+    if (a.N % 256 == 0) return launch_tc<256, TC_DOWN>(a, tmA, tmB, max_blocks, a.N / 256, s);
+    return launch_tc<128, TC_DOWN>(a, tmA, tmB, max_blocks, a.N / 128, s);
 }
 
 }  // namespace moeq

@@ -224,14 +224,22 @@ def test_fp8_moe_full_sampled():
     _layer_parity(d, sample_tokens(d, 8), TOL_FP8, "moe_fp8")
 
 
-@pytest.mark.parametrize("T,E,k,logit_mode", [(1, 8, 2, "normal"), (150, 4, 1, "one"), (33, 8, 8, "equal")])
-def test_fp8_moe_edge_cases(T, E, k, logit_mode):
-    d = W.make_moe(W.WORKLOADS["moe_fp8"], device=DEV, T=T, E=E, k=k, H=256, I=256)
+@pytest.mark.parametrize("T,E,k,H,logit_mode", [
+    (1, 8, 2, 256, "normal"),      # register-fed path (few rows per expert)
+    (150, 4, 1, 256, "one"),       # tensor-core path, one expert takes every token
+    (33, 8, 8, 256, "equal"),      # k = E
+    (100, 4, 2, 384, "zipf"),      # H not a multiple of 256: 128-column down tiles; empty experts
+    (517, 24, 6, 512, "zipf"),     # many expert blocks, ragged tails
+])
+def test_fp8_moe_edge_cases(T, E, k, H, logit_mode):
+    d = W.make_moe(W.WORKLOADS["moe_fp8"], device=DEV, T=T, E=E, k=k, H=H, I=256)
     if logit_mode == "one":
         d["logits"] = torch.zeros((T, E), device=DEV)
         d["logits"][:, 2] = 5.0
     elif logit_mode == "equal":
         d["logits"] = torch.zeros((T, E), device=DEV)
+    elif logit_mode == "zipf":
+        d["logits"] = W.router_logits(W.WORKLOADS["moe_fp8"], T, E, device=DEV)
     _layer_parity(d, np.arange(T, dtype=np.int32), TOL_FP8, f"fp8 T={T} E={E} k={k}")
 
 
