@@ -163,14 +163,25 @@ static RouteBufs carve_route(Carve &c, long T, int k, int E, int block_m)
     return r;
 }
 
-static size_t w4a16_layout(Carve &c, long T, int H, int I, int E, int k, RouteBufs *rb, uint16_t **h, float **ys)
+// W4A16 layer schedule: from this many routed rows per expert on (mean T*k/E), the grouped GEMMs
+// run on the tensor-core kernels over 128-row expert blocks (weights dequantized into tensor
+// memory); below, the register-fed swap-AB kernels stream the weights for the few rows each
+// expert has (HBM bound).
+static bool w4_use_tc(long T, int k, int E) { return (double)T * k / (double)E >= 16.0; }
+
+static size_t w4a16_layout(Carve &c, long T, int H, int I, int E, int k, RouteBufs *rb, uint16_t **h, float **ys,
+                           uint16_t **xg = nullptr)
 {
-    RouteBufs r = carve_route(c, T, k, E, pick_block_m(T, k, E));
-    uint16_t *hp = c.take<uint16_t>((size_t)T * k * I);
+    const bool tcp = w4_use_tc(T, k, E);
+    RouteBufs r = carve_route(c, T, k, E, tcp ? 128 : pick_block_m(T, k, E));
+    const size_t cap = (size_t)r.max_blocks * r.block_m;
+    uint16_t *hp = c.take<uint16_t>((tcp ? cap : (size_t)T * k) * I);
     float *yp = c.take<float>((size_t)T * k * H);
+    uint16_t *xgp = tcp ? c.take<uint16_t>(cap * H) : nullptr;
     if (rb) *rb = r;
     if (h) *h = hp;
     if (ys) *ys = yp;
+    if (xg) *xg = xgp;
     return c.used;
 }
 
@@ -313,12 +324,13 @@ int moe_w4a16_forward(const uint16_t *x, const float *logits, int T, int H, int 
     cudaStream_t s = (cudaStream_t)stream;
     Carve c(ws);
     RouteBufs r;
-    uint16_t *h;
+    uint16_t *h, *xg;
     float *ys;
-    w4a16_layout(c, T, H, I, E, k, &r, &h, &ys);
+    w4a16_layout(c, T, H, I, E, k, &r, &h, &ys, &xg);
     int32_t *ids = topk_ids_out ? topk_ids_out : r.ids;
     float *tw = topk_w_out ? topk_w_out : r.w;
     const int n = T * k;
+    const bool tcp = w4_use_tc(T, k, E);
 
     {
         trace::Scope ts(trace::ROUTE, s);
@@ -329,38 +341,80 @@ int moe_w4a16_forward(const uint16_t *x, const float *logits, int T, int H, int 
         launch_align(ids, n, E, r.block_m, r.sorted, r.eids, r.ntp, s);
     }
 
-    W4GroupedArgs a{};
-    a.E = E;
-    a.sorted_ids = r.sorted;
-    a.expert_ids = r.eids;
-    a.num_tokens_padded = r.ntp;
-    a.n_slots = n;
-    a.topk_w = tw;
-    // gate/up + SiLU*up
-    a.act = x;
-    a.act_row_div = k;
-    a.wq = w13_q;
-    a.ws = w13_s;
-    a.K = H;
-    a.n_out = I;
-    a.n_rows = 2 * I;
-    a.h_out = h;
-    {
-        trace::Scope ts(trace::GATE_UP, s);
-        launch_w4a16_grouped_mma(a, MODE_GATEUP, r.block_m, r.max_blocks, s);
-    }
-    // down, routing weight applied per slot
-    a.act = h;
-    a.act_row_div = 1;
-    a.wq = w2_q;
-    a.ws = w2_s;
-    a.K = I;
-    a.n_out = H;
-    a.n_rows = H;
-    a.y_out = ys;
-    {
-        trace::Scope ts(trace::DOWN, s);
-        launch_w4a16_grouped_mma(a, MODE_DOWN, r.block_m, r.max_blocks, s);
+    if (tcp) {
+        int *status = device_status_ptr();
+        if (!status) return set_error(MOEQ_ERR_CUDA, "moe_w4a16_forward: no device status word");
+        const int cap = r.max_blocks * 128;
+        {
+            trace::Scope ts(trace::ACT_QUANT, s);  // the activation gather takes the act-prep slot
+            launch_gather_bf16_perm(x, H, k, r.sorted, r.ntp, n, cap, xg, num_sms(), s);
+        }
+        W4TcArgs t{};
+        t.status = status;
+        t.E = E;
+        t.sorted_ids = r.sorted;
+        t.expert_ids = r.eids;
+        t.ntp = r.ntp;
+        t.n_slots = n;
+        t.topk_w = tw;
+        t.M = cap;
+        t.N = I;
+        t.K = H;
+        t.rows_per_expert = 2 * I;
+        t.wq = w13_q;
+        t.ws = w13_s;
+        t.h_out = h;
+        int rc;
+        {
+            trace::Scope ts(trace::GATE_UP, s);
+            rc = launch_w4a16_tc(t, TC_GATEUP, xg, r.max_blocks, s);
+        }
+        if (rc) return rc;
+        t.N = H;
+        t.K = I;
+        t.rows_per_expert = H;
+        t.wq = w2_q;
+        t.ws = w2_s;
+        t.ys = ys;
+        {
+            trace::Scope ts(trace::DOWN, s);
+            rc = launch_w4a16_tc(t, TC_DOWN, h, r.max_blocks, s);
+        }
+        if (rc) return rc;
+    } else {
+        W4GroupedArgs a{};
+        a.E = E;
+        a.sorted_ids = r.sorted;
+        a.expert_ids = r.eids;
+        a.num_tokens_padded = r.ntp;
+        a.n_slots = n;
+        a.topk_w = tw;
+        // gate/up + SiLU*up
+        a.act = x;
+        a.act_row_div = k;
+        a.wq = w13_q;
+        a.ws = w13_s;
+        a.K = H;
+        a.n_out = I;
+        a.n_rows = 2 * I;
+        a.h_out = h;
+        {
+            trace::Scope ts(trace::GATE_UP, s);
+            launch_w4a16_grouped_mma(a, MODE_GATEUP, r.block_m, r.max_blocks, s);
+        }
+        // down, routing weight applied per slot
+        a.act = h;
+        a.act_row_div = 1;
+        a.wq = w2_q;
+        a.ws = w2_s;
+        a.K = I;
+        a.n_out = H;
+        a.n_rows = H;
+        a.y_out = ys;
+        {
+            trace::Scope ts(trace::DOWN, s);
+            launch_w4a16_grouped_mma(a, MODE_DOWN, r.block_m, r.max_blocks, s);
+        }
     }
     {
         trace::Scope ts(trace::COMBINE, s);

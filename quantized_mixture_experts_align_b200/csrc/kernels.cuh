@@ -68,6 +68,22 @@ struct Fp8TcArgs {
     float *ys;              // down out: [n_slots, N] f32, routing weight applied
 };
 
+struct W4TcArgs {
+    int M, N, K;            // activation rows (aligned capacity); output features / rows; inputs
+    int *status;
+    int E;
+    int rows_per_expert;    // 2I (gate/up) or H (down)
+    const int32_t *wq;      // [E * rows_per_expert, K/8]
+    const uint16_t *ws;     // [E * rows_per_expert, K/32] bf16
+    const int32_t *sorted_ids;
+    const int32_t *expert_ids;
+    const int32_t *ntp;
+    int n_slots;
+    const float *topk_w;
+    uint16_t *h_out;        // gate/up: [M, N] bf16, pair-permuted inside 8-element chunks
+    float *ys;              // down: [n_slots, N] f32, routing weight applied
+};
+
 void launch_route_topk(const float *logits, int T, int E, int k, int32_t *ids, float *w, cudaStream_t s);
 void launch_align(const int32_t *topk_ids, int n, int E, int B, int32_t *sorted_ids, int32_t *expert_ids,
                   int32_t *ntp, cudaStream_t s);
@@ -81,6 +97,11 @@ int launch_fp8_tc_gemm(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B, c
 // each, per expert_ids / ntp) and weights W [E * rows_per_expert, K]; mode TC_GATEUP or TC_DOWN.
 int launch_fp8_tc_grouped(const Fp8TcArgs &a, int mode, const uint8_t *A, const uint8_t *W, int E, int max_blocks,
                           cudaStream_t s);
+// tcgen05 W4A16 grouped GEMM over aligned activation rows (bf16 [M, K], pair-permuted); mode
+// TC_GATEUP (h = silu(gate) * up, written pair-permuted) or TC_DOWN (weighted slot rows).
+int launch_w4a16_tc(const W4TcArgs &a, int mode, const uint16_t *act, int max_blocks, cudaStream_t s);
+void launch_gather_bf16_perm(const uint16_t *x, int H, int k, const int32_t *sorted_ids, const int32_t *ntp,
+                             int n_slots, int cap_rows, uint16_t *xg, int num_sms, cudaStream_t s);
 // Copies E4M3 rows (and their scales) of the routed slots into aligned order: row r takes token
 // sorted_ids[r] / k; padding rows become zero.
 void launch_gather_fp8_rows(const uint8_t *xq, const float *xs, int H, int k, const int32_t *sorted_ids,

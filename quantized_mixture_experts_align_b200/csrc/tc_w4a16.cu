@@ -1,0 +1,339 @@
+// W4A16 grouped expert GEMMs on the 5th-generation tensor cores (tcgen05, sm_100a), for expert
+// blocks with many routed rows (prefill).
+//
+// "vLLM x Novita AI: Chord W4A16 INT4 MoE Kernel for Kimi K2.x": INT4 group-32 codes with bf16
+// scales ("vLLM integration"), dequantized by subtracting the zero point and then scaling in
+// bf16 ("H200 and Blackwell indexed decode"), the dequantization of the next stage overlapped
+// with the pending MMAs ("H200 prefill and TP8"), a TMA producer feeding MMA consumers ("SM90
+// grouped kernels"). Re-derived for tcgen05:
+//
+// Weights take the MMA's A side and live in TENSOR memory: dequantization warps turn the packed
+// codes into bf16 in registers and store them with tcgen05.st, so dequantized weights never pass
+// through shared memory (a bf16 B-side tile would cost its shared-memory bandwidth twice, on
+// write and on every MMA read). The activations (routed rows gathered in aligned order, one
+// expert per 128-row block) are the B side, loaded by TMA with the 128-byte swizzle.
+//   D[weight rows, tokens] += A_tmem[weight rows, K] * B_smem[tokens, K]^T   (M = N = 128, K = 16)
+// The nibble pairs that one shift + LOP3 extracts, (q0,q4) (q1,q5) (q2,q6) (q3,q7) of each
+// 32-bit word, become consecutive K in tensor memory, so the activations are stored with the
+// same order inside every 8-element chunk (done by the gather and by the gate/up epilogue).
+//
+// CTA = one 128-row activation block of one expert x 128 output features, 10 warps:
+//   warp 0      TMA producer of the activation tiles [128 tokens x 64 inputs] (4 stages);
+//   warp 1      tensor-memory allocation; lane 0 issues the MMAs (gate/up: one MMA into each of
+//               the two accumulators per 16 inputs) and commits;
+//   warps 2-9   dequantization: each thread owns one weight row (gate/up: warps of the first
+//               set the gate rows, of the second set the up rows; down: the two sets split each
+//               64-input step), prefetches its packed codes and scales through a private
+//               8-deep cp.async ring, and writes the dequantized step to a tensor-memory stage;
+//               then the epilogue: gate/up writes h = bf16(silu(g) * u) in the permuted order,
+//               down writes the routing-weighted f32 slot rows.
+#include "kernels.cuh"
+#include "tc_common.cuh"
+
+namespace moeq {
+
+namespace {
+
+constexpr int kTok = 128;     // tokens per tile = aligned block size
+constexpr int kKs = 64;       // inputs per pipeline step
+constexpr int kStages = 4;    // activation tiles (shared memory) and weight stages (tensor memory)
+constexpr int kRing = 8;      // per-thread packed-code prefetch depth, in steps
+constexpr int kDeqWarps = 8;
+constexpr int kDeqThreads = kDeqWarps * 32;
+constexpr int kThreads = (2 + kDeqWarps) * 32;
+
+template <int MODE>
+struct W4TcShape {
+    static constexpr bool kGU = MODE == TC_GATEUP;
+    static constexpr int kAccCols = kGU ? 2 * kTok : kTok;          // D_gate | D_up, or D
+    static constexpr int kAStageCols = kGU ? kKs : kKs / 2;          // bf16 pairs per stage
+    static constexpr int kTmemCols = kGU ? 512 : 256;
+    static_assert(kAccCols + kStages * kAStageCols <= kTmemCols, "tensor memory budget");
+    static constexpr int kBTile = kTok * kKs * 2;                    // 16 KB
+    static constexpr int kCodeParts = kGU ? 2 : 1;                   // 16-byte parts per thread per step
+    static constexpr size_t kCodeRing = (size_t)kRing * kCodeParts * kDeqThreads * 16;
+    static constexpr size_t kScaleRing = (size_t)kRing * kDeqThreads * 4;
+    static constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kBTile + kCodeRing + kScaleRing + 256;
+};
+
+__device__ __forceinline__ void cp_async4(void *dst, const void *src)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
+}
+
+// (q - 8) * scale in bf16 for the pairs (q0,q4) (q1,q5) (q2,q6) (q3,q7) of one code word
+__device__ __forceinline__ void dequant4(uint32_t w, uint32_t scale2, uint32_t *out)
+{
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t v = lop3_and_or(w >> (4 * i), 0x000F000Fu, 0x43004300u);  // 128 + q, exact
+        out[i] = bf16x2_mul(bf16x2_sub(v, 0x43084308u), scale2);                  // (q - 8), then * s
+    }
+}
+
+// position of feature f inside its 8-element chunk after the pair permutation
+__device__ __forceinline__ int perm_pos(int f)
+{
+    const int i = f & 7;
+    return (f & ~7) + (i < 4 ? 2 * i : 2 * (i - 4) + 1);
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+    w4a16_tc_kernel(const __grid_constant__ CUtensorMap tmX, W4TcArgs a)
+{
+    using Sh = W4TcShape<MODE>;
+    constexpr bool GU = Sh::kGU;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *btiles = smem;
+    uint8_t *code_ring = btiles + kStages * Sh::kBTile;
+    uint8_t *scale_ring = code_ring + Sh::kCodeRing;
+    uint64_t *b_full = reinterpret_cast<uint64_t *>(scale_ring + Sh::kScaleRing);
+    uint64_t *a_full = b_full + kStages;
+    uint64_t *empty = a_full + kStages;
+    uint64_t *acc_full = empty + kStages;
+    uint64_t *mma_done = acc_full + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int r0 = blockIdx.x * kTok;
+    if (r0 >= __ldg(a.ntp)) return;  // uniform over the CTA, before any barrier or allocation
+    const int e = __ldg(a.expert_ids + blockIdx.x);
+    if (e < 0 || e >= a.E) return;
+    const int n0 = blockIdx.y * 128;  // output features (gate/up) or output rows (down)
+    const int K = a.K, NS = K / kKs;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            tc::mbar_init(&b_full[s], 1);
+            tc::mbar_init(&a_full[s], kDeqWarps);
+            tc::mbar_init(&empty[s], 1);
+        }
+        tc::mbar_init(acc_full, 1);
+        tc::mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        tc::fence_barrier_init();
+    }
+    if (warp == 1) tc::tmem_alloc(tmem_slot, Sh::kTmemCols);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            tc::prefetch_tmap(&tmX);
+            int issued = 0;
+            for (int ks = 0; ks < NS; ++ks) {
+                const int s = ks % kStages;
+                if (ks >= kStages && !tc::mbar_wait(&empty[s], ((ks / kStages) & 1) ^ 1, abort_flag, a.status)) break;
+                tc::mbar_arrive_expect_tx(&b_full[s], Sh::kBTile);
+                tc::tma_load_2d(btiles + s * Sh::kBTile, &tmX, &b_full[s], ks * kKs, r0);
+                issued = ks + 1;
+            }
+            for (int ks = issued - kStages > 0 ? issued - kStages : 0; ks < issued; ++ks)
+                tc::mbar_drain(&b_full[ks % kStages], (ks / kStages) & 1, a.status);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = tc::idesc_f32(tc::kFmtBF16, tc::kFmtBF16, 128, kTok);
+            for (int ks = 0; ks < NS; ++ks) {
+                const int s = ks % kStages;
+                const uint32_t par = (ks / kStages) & 1;
+                if (!tc::mbar_wait(&b_full[s], par, abort_flag, a.status)) break;
+                if (!tc::mbar_wait(&a_full[s], par, abort_flag, a.status)) break;
+                tc::fence_after_sync();
+                const uint64_t bdesc = tc::smem_desc_sw128(btiles + s * Sh::kBTile);
+                const uint32_t astage = tmem + Sh::kAccCols + s * Sh::kAStageCols;
+#pragma unroll
+                for (int kk = 0; kk < kKs / 16; ++kk) {
+                    const uint32_t acc = (ks > 0 || kk > 0) ? 1u : 0u;
+                    if (GU) {
+                        tc::mma_f16_ts(tmem, astage + kk * 8, bdesc + 2 * kk, idesc, acc);
+                        tc::mma_f16_ts(tmem + kTok, astage + kKs / 2 + kk * 8, bdesc + 2 * kk, idesc, acc);
+                    } else {
+                        tc::mma_f16_ts(tmem, astage + kk * 8, bdesc + 2 * kk, idesc, acc);
+                    }
+                }
+                tc::mma_commit(&empty[s]);
+            }
+            tc::mma_commit(acc_full);
+            tc::mma_commit(mma_done);
+            tc::mbar_drain(mma_done, 0, a.status);
+        }
+    } else {
+        // ---- dequantization ----
+        const int dw = warp - 2, quarter = warp & 3, set = dw >> 2;
+        const int t = dw * 32 + lane;               // ring slot owner
+        const int row = quarter * 32 + lane;        // tensor-memory lane = weight row in the tile
+        const int grow = e * a.rows_per_expert + (GU ? (set ? a.N : 0) + n0 + row : n0 + row);
+        const int32_t *wrow = a.wq + (size_t)grow * (K / 8);
+        const uint16_t *srow = a.ws + (size_t)grow * (K / 32);
+        auto code_slot = [&](int slot, int part) {
+            return code_ring + ((size_t)(slot * Sh::kCodeParts + part) * kDeqThreads + t) * 16;
+        };
+        auto issue = [&](int ks) {
+            if (ks < NS) {
+                const int slot = ks % kRing;
+                if (GU) {
+                    cp_async16_stream(code_slot(slot, 0), wrow + ks * 8);
+                    cp_async16_stream(code_slot(slot, 1), wrow + ks * 8 + 4);
+                } else {
+                    cp_async16_stream(code_slot(slot, 0), wrow + ks * 8 + 4 * set);
+                }
+                cp_async4(scale_ring + ((size_t)slot * kDeqThreads + t) * 4, srow + ks * 2);
+            }
+            cp_async_commit();
+        };
+#pragma unroll
+        for (int ks = 0; ks < kRing - 1; ++ks) issue(ks);
+        bool ok = true;
+        for (int ks = 0; ks < NS && ok; ++ks) {
+            cp_async_wait<kRing - 2>();
+            const int slot = ks % kRing;
+            const uint4 c0 = *reinterpret_cast<const uint4 *>(code_slot(slot, 0));
+            uint4 c1 = make_uint4(0u, 0u, 0u, 0u);
+            if (GU) c1 = *reinterpret_cast<const uint4 *>(code_slot(slot, 1));
+            const uint32_t sc = *reinterpret_cast<const uint32_t *>(scale_ring + ((size_t)slot * kDeqThreads + t) * 4);
+            issue(ks + kRing - 1);  // refills the slot read in step ks - 1
+            uint32_t pairs[GU ? 32 : 16];
+            const uint32_t s_lo = (sc & 0xFFFFu) * 0x10001u, s_hi = (sc >> 16) * 0x10001u;
+            if (GU) {
+                dequant4(c0.x, s_lo, pairs + 0);
+                dequant4(c0.y, s_lo, pairs + 4);
+                dequant4(c0.z, s_lo, pairs + 8);
+                dequant4(c0.w, s_lo, pairs + 12);
+                dequant4(c1.x, s_hi, pairs + 16);
+                dequant4(c1.y, s_hi, pairs + 20);
+                dequant4(c1.z, s_hi, pairs + 24);
+                dequant4(c1.w, s_hi, pairs + 28);
+            } else {
+                const uint32_t s2 = set ? s_hi : s_lo;
+                dequant4(c0.x, s2, pairs + 0);
+                dequant4(c0.y, s2, pairs + 4);
+                dequant4(c0.z, s2, pairs + 8);
+                dequant4(c0.w, s2, pairs + 12);
+            }
+            const int s = ks % kStages;
+            if (ks >= kStages)
+                ok = __all_sync(0xFFFFFFFFu, tc::mbar_wait(&empty[s], ((ks / kStages) & 1) ^ 1, abort_flag, a.status));
+            if (!ok) break;
+            tc::fence_after_sync();
+            const uint32_t col = Sh::kAccCols + s * Sh::kAStageCols + (GU ? set * (kKs / 2) : set * (kKs / 4));
+            const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + col;
+            if (GU) tc::tmem_st32(taddr, pairs);
+            else tc::tmem_st16(taddr, pairs);
+            tc::tmem_wait_st();
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&a_full[s]);
+        }
+        cp_async_wait<0>();
+
+        // ---- epilogue: tokens [64 set, 64 set + 64) of the tile ----
+        ok = ok && __all_sync(0xFFFFFFFFu, tc::mbar_wait(acc_full, 0, abort_flag, a.status));
+        if (ok) {
+            tc::fence_after_sync();
+            const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+            for (int c = 0; c < 2; ++c) {
+                const int tok0 = set * 64 + c * 32;
+                uint32_t g[32];
+                tc::tmem_ld32(lane_base + tok0, g);
+                if (GU) {
+                    uint32_t u[32];
+                    tc::tmem_ld32(lane_base + kTok + tok0, u);
+                    tc::tmem_wait_ld();
+                    const int f = n0 + row;
+                    uint16_t *hcol = a.h_out + perm_pos(f);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const float hv = silu_f32(__uint_as_float(g[j])) * __uint_as_float(u[j]);
+                        hcol[(size_t)(r0 + tok0 + j) * a.N] = f32_to_bf16(hv);
+                    }
+                } else {
+                    tc::tmem_wait_ld();
+                    const int my_slot = __ldg(a.sorted_ids + r0 + tok0 + lane);
+                    const float my_w = (my_slot < a.n_slots) ? __ldg(a.topk_w + my_slot) : 0.f;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int slot = __shfl_sync(0xFFFFFFFFu, my_slot, j);
+                        const float wt = __shfl_sync(0xFFFFFFFFu, my_w, j);
+                        if (slot < a.n_slots) a.ys[(size_t)slot * a.N + n0 + row] = wt * __uint_as_float(g[j]);
+                    }
+                }
+            }
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp == 1) tc::tmem_dealloc(tmem, Sh::kTmemCols);
+}
+
+// Gather of bf16 activation rows into aligned order with the pair permutation inside every
+// 8-element chunk; one warp per row, padding rows zero.
+__global__ void __launch_bounds__(256) gather_bf16_perm_kernel(const uint16_t *__restrict__ x, int H, int k,
+                                                               const int32_t *__restrict__ sorted_ids,
+                                                               const int32_t *__restrict__ ntp, int n_slots,
+                                                               int cap_rows, uint16_t *__restrict__ xg)
+{
+    const int lane = threadIdx.x & 31;
+    const int rows = min(__ldg(ntp), cap_rows);
+    for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += gridDim.x * (blockDim.x >> 5)) {
+        const int slot = __ldg(sorted_ids + r);
+        const bool real = slot < n_slots;
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)(real ? slot / k : 0) * H);
+        uint4 *dst = reinterpret_cast<uint4 *>(xg + (size_t)r * H);
+        for (int i = lane; i < H / 8; i += 32) {
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (real) {
+                const uint4 u = __ldg(src + i);
+                v.x = prmt(u.x, u.z, 0x5410u);  // (x0, x4)
+                v.y = prmt(u.x, u.z, 0x7632u);  // (x1, x5)
+                v.z = prmt(u.y, u.w, 0x5410u);  // (x2, x6)
+                v.w = prmt(u.y, u.w, 0x7632u);  // (x3, x7)
+            }
+            dst[i] = v;
+        }
+    }
+}
+
+template <int MODE>
+int launch_mode(const W4TcArgs &a, const CUtensorMap &tm, int grid_x, int grid_y, cudaStream_t s)
+{
+    using Sh = W4TcShape<MODE>;
+    static bool attr = false;
+    if (!attr) {
+        const cudaError_t e =
+            cudaFuncSetAttribute(w4a16_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Sh::kSmemBytes);
+        if (e != cudaSuccess)
+            return set_error(MOEQ_ERR_CUDA, "tcgen05 W4A16 GEMM: shared-memory attribute: %s", cudaGetErrorString(e));
+        attr = true;
+    }
+    if (grid_x <= 0 || grid_y <= 0) return MOEQ_OK;
+    w4a16_tc_kernel<MODE><<<dim3(grid_x, grid_y), kThreads, Sh::kSmemBytes, s>>>(tm, a);
+    return MOEQ_OK;
+}
+
+}  // namespace
+
+int launch_w4a16_tc(const W4TcArgs &a, int mode, const uint16_t *act, int max_blocks, cudaStream_t s)
+{
+    CUtensorMap tm;
+    const int rc = make_tmap_2d(&tm, act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.M, (uint64_t)a.K, kTok, kKs);
+    if (rc) return rc;
+    if (mode == TC_GATEUP) return launch_mode<TC_GATEUP>(a, tm, max_blocks, a.N / 128, s);
+    return launch_mode<TC_DOWN>(a, tm, max_blocks, a.N / 128, s);
+}
+
+void launch_gather_bf16_perm(const uint16_t *x, int H, int k, const int32_t *sorted_ids, const int32_t *ntp,
+                             int n_slots, int cap_rows, uint16_t *xg, int num_sms, cudaStream_t s)
+{
+    if (cap_rows <= 0) return;
+    const int blocks = min(cdiv(cap_rows, 8), num_sms * 8);
+    gather_bf16_perm_kernel<<<blocks, 256, 0, s>>>(x, H, k, sorted_ids, ntp, n_slots, cap_rows, xg);
+}
+
+}  // namespace moeq
