@@ -311,6 +311,33 @@ def reference_arm(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def only_arm(args, moeq, rank, world):
+    """One workload alone, for profiler captures of a small case; prints a JSON line of timings."""
+    name = args.only
+    if name == "dense_fp8":
+        wl = W.WORKLOADS[name]
+        M = args.tokens or 4096
+        dd = W.make_dense_fp8(wl, M, device="cuda")
+        C = torch.empty((M, wl.N), dtype=torch.bfloat16, device="cuda")
+        ms = timed_steps(lambda: moeq.w8a8_block_fp8_matmul(dd["A"], dd["As"], dd["B"], dd["Bs"], out=C),
+                         args.steps, args.warmup, None, world)
+        line = {"only": name, "M": M, "ms": statistics.mean(ms), "tflops": 2.0 * M * wl.N * wl.K / statistics.mean(ms) / 1e9}
+    else:
+        d = W.make_moe(W.WORKLOADS[name], device="cuda", T=args.tokens, E=args.experts)
+        if d["kind"] == "w4a16":
+            ms, st, _ = run_w4a16(moeq, d, args.steps, args.warmup, None, world, trace=True)
+        else:
+            ms, st = run_fp8(moeq, d, args.steps, args.warmup, None, world)
+        fl = W.moe_flops(d["T"], d["k"], d["H"], d["I"])
+        line = {"only": name, "T": d["T"], "E": d["E"], "ms": statistics.mean(ms),
+                "tflops": fl / statistics.mean(ms) / 1e9,
+                "stages_ms": {k: v[0] / max(v[1], 1) for k, v in st.items() if v[1]}}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -320,7 +347,10 @@ def main():
     ap.add_argument("--headline-only", action="store_true", help="skip the secondary workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--experts", type=int, default=None,
-                    help="override E of the headline workload (small cases for profiler captures)")
+                    help="override E of the workload (small cases for profiler captures)")
+    ap.add_argument("--tokens", type=int, default=None, help="override T of the workload (with --only)")
+    ap.add_argument("--only", choices=["prefill_w4a16", "moe_fp8", "dense_fp8"], default=None,
+                    help="time one secondary workload alone (small cases for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -335,6 +365,9 @@ def main():
     import quantized_mixture_experts_align_b200 as moeq
     moeq.lib()
     peaks, peak_src = load_peaks()
+    if args.only:
+        only_arm(args, moeq, rank, world)
+        return
     flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
 
     def flush():

@@ -67,7 +67,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m0 = blockIdx.x * kBM;  // consecutive CTAs share a B (weight) tile in L2
+    // dense: grid x = row tiles, so consecutive CTAs share a B (weight) tile in L2; grouped: grid
+    // x = output tiles, so the tiles of one expert block run back to back and its activation rows
+    // come from DRAM once
+    const int m0 = (MODE == TC_DENSE ? blockIdx.x : blockIdx.y) * kBM;
     const int KB = a.K / kBK;
     // output columns of this tile and the weight rows (in the [E * rows, K] weight matrix) loaded
     // into the B stage: dense and down take BN consecutive rows; gate/up takes 128 gate + 128 up
@@ -79,17 +82,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         bscale0 = a.b_scale + (size_t)(n0 / 128) * KB;
     } else {
         if (m0 >= __ldg(a.ntp)) return;  // uniform over the CTA, before any barrier or allocation
-        const int e = __ldg(a.expert_ids + blockIdx.x);
+        const int e = __ldg(a.expert_ids + blockIdx.y);
         if (e < 0 || e >= a.E) return;
         const float *ws = a.b_scale + (size_t)e * (a.rows_per_expert / 128) * KB;
         if (MODE == TC_GATEUP) {
-            n0 = blockIdx.y * 128;                      // feature tile
+            n0 = blockIdx.x * 128;                      // feature tile
             brow0 = e * a.rows_per_expert + n0;         // gate rows
             brow1 = e * a.rows_per_expert + a.N + n0;   // up rows
             bscale0 = ws + (size_t)(n0 / 128) * KB;
             bscale1 = ws + (size_t)((a.N + n0) / 128) * KB;
         } else {
-            n0 = blockIdx.y * BN;
+            n0 = blockIdx.x * BN;
             brow0 = e * a.rows_per_expert + n0;
             bscale0 = ws + (size_t)(n0 / 128) * KB;
         }
@@ -300,9 +303,9 @@ int launch_fp8_tc_grouped(const Fp8TcArgs &a, int mode, const uint8_t *A, const 
     rc = make_tmap_2d(&tmB, W, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)E * a.rows_per_expert, (uint64_t)a.K, box,
                       kBK);
     if (rc) return rc;
-    if (mode == TC_GATEUP) return launch_tc<256, TC_GATEUP>(a, tmA, tmB, max_blocks, a.N / 128, s);
-    if (a.N % 256 == 0) return launch_tc<256, TC_DOWN>(a, tmA, tmB, max_blocks, a.N / 256, s);
-    return launch_tc<128, TC_DOWN>(a, tmA, tmB, max_blocks, a.N / 128, s);
+    if (mode == TC_GATEUP) return launch_tc<256, TC_GATEUP>(a, tmA, tmB, a.N / 128, max_blocks, s);
+    if (a.N % 256 == 0) return launch_tc<256, TC_DOWN>(a, tmA, tmB, a.N / 256, max_blocks, s);
+    return launch_tc<128, TC_DOWN>(a, tmA, tmB, a.N / 128, max_blocks, s);
 }
 
 }  // namespace moeq

@@ -17,16 +17,15 @@
 // 32-bit word, become consecutive K in tensor memory, so the activations are stored with the
 // same order inside every 8-element chunk (done by the gather and by the gate/up epilogue).
 //
-// CTA = one 128-row activation block of one expert x 128 output features, 10 warps:
+// CTA = one 128-row activation block of one expert x 128 output features:
 //   warp 0      TMA producer of the activation tiles [128 tokens x 64 inputs] (4 stages);
 //   warp 1      tensor-memory allocation; lane 0 issues the MMAs (gate/up: one MMA into each of
 //               the two accumulators per 16 inputs) and commits;
-//   warps 2-9   dequantization: each thread owns one weight row (gate/up: warps of the first
-//               set the gate rows, of the second set the up rows; down: the two sets split each
-//               64-input step), prefetches its packed codes and scales through a private
-//               8-deep cp.async ring, and writes the dequantized step to a tensor-memory stage;
-//               then the epilogue: gate/up writes h = bf16(silu(g) * u) in the permuted order,
-//               down writes the routing-weighted f32 slot rows.
+//   warps 2..  dequantization (gate/up 16 warps, down 8): a thread owns one weight row and a
+//               part of each 64-input step (gate/up: one matrix, half the step; down: half), prefetches its packed codes and scales through a private 8-deep cp.async
+//               ring, and writes the dequantized part to a tensor-memory stage; then the
+//               epilogue: gate/up writes h = bf16(silu(g) * u) in the permuted order, down
+//               writes the routing-weighted f32 slot rows.
 #include "kernels.cuh"
 #include "tc_common.cuh"
 
@@ -37,21 +36,28 @@ namespace {
 constexpr int kTok = 128;     // tokens per tile = aligned block size
 constexpr int kKs = 64;       // inputs per pipeline step
 constexpr int kStages = 4;    // activation tiles (shared memory) and weight stages (tensor memory)
-constexpr int kRing = 8;      // per-thread packed-code prefetch depth, in steps
-constexpr int kDeqWarps = 8;
-constexpr int kDeqThreads = kDeqWarps * 32;
-constexpr int kThreads = (2 + kDeqWarps) * 32;
 
-template <int MODE>
+// DW dequantization warps: 4 tensor-memory lane quarters x (DW / 4) "sets". A set is, for
+// gate/up, a (matrix, K part) pair (matrix = set % 2), for down a K part; each thread converts
+// kWords code words of one weight row per 64-input step.
+template <int MODE, int DW>
 struct W4TcShape {
     static constexpr bool kGU = MODE == TC_GATEUP;
+    // per-thread packed-code prefetch depth, in steps (down: shallower, so two CTAs fit an SM)
+    static constexpr int kRing = kGU ? 8 : 6;
+    static constexpr int kSets = DW / 4;
+    static constexpr int kKParts = kGU ? kSets / 2 : kSets;
+    static constexpr int kWords = 8 / kKParts;                       // code words per thread per step
+    static constexpr int kCodeBytes = kWords * 4;                    // 32, 16 or 8
+    static constexpr int kDeqThreads = DW * 32;
+    static constexpr int kThreads = (2 + DW) * 32;
     static constexpr int kAccCols = kGU ? 2 * kTok : kTok;          // D_gate | D_up, or D
     static constexpr int kAStageCols = kGU ? kKs : kKs / 2;          // bf16 pairs per stage
     static constexpr int kTmemCols = kGU ? 512 : 256;
     static_assert(kAccCols + kStages * kAStageCols <= kTmemCols, "tensor memory budget");
+    static_assert(kKParts >= 1 && kWords >= 2, "dequantization split");
     static constexpr int kBTile = kTok * kKs * 2;                    // 16 KB
-    static constexpr int kCodeParts = kGU ? 2 : 1;                   // 16-byte parts per thread per step
-    static constexpr size_t kCodeRing = (size_t)kRing * kCodeParts * kDeqThreads * 16;
+    static constexpr size_t kCodeRing = (size_t)kRing * kDeqThreads * kCodeBytes;
     static constexpr size_t kScaleRing = (size_t)kRing * kDeqThreads * 4;
     static constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kBTile + kCodeRing + kScaleRing + 256;
 };
@@ -59,6 +65,26 @@ struct W4TcShape {
 __device__ __forceinline__ void cp_async4(void *dst, const void *src)
 {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
+}
+
+template <int BYTES>
+__device__ __forceinline__ void cp_async_codes(void *dst, const void *src)
+{
+    if (BYTES == 8) {
+        cp_async8(dst, src);
+    } else {
+#pragma unroll
+        for (int p = 0; p < BYTES / 16; ++p)
+            cp_async16_stream(static_cast<uint8_t *>(dst) + 16 * p, static_cast<const uint8_t *>(src) + 16 * p);
+    }
+}
+
+template <int N>
+__device__ __forceinline__ void tmem_st_n(uint32_t taddr, const uint32_t *r)
+{
+    if (N == 8) tc::tmem_st8(taddr, *reinterpret_cast<const uint32_t(*)[8]>(r));
+    else if (N == 16) tc::tmem_st16(taddr, r);
+    else tc::tmem_st32(taddr, r);
 }
 
 // (q - 8) * scale in bf16 for the pairs (q0,q4) (q1,q5) (q2,q6) (q3,q7) of one code word
@@ -78,11 +104,13 @@ __device__ __forceinline__ int perm_pos(int f)
     return (f & ~7) + (i < 4 ? 2 * i : 2 * (i - 4) + 1);
 }
 
-template <int MODE>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int MODE, int DW>
+__global__ void __launch_bounds__((2 + DW) * 32, 1)
     w4a16_tc_kernel(const __grid_constant__ CUtensorMap tmX, W4TcArgs a)
 {
-    using Sh = W4TcShape<MODE>;
+    using Sh = W4TcShape<MODE, DW>;
+    constexpr int kDeqThreads = Sh::kDeqThreads;
+    constexpr int kRing = Sh::kRing;
     constexpr bool GU = Sh::kGU;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -98,17 +126,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int r0 = blockIdx.x * kTok;
+    // grid x = output tiles, grid y = token blocks: the tiles of one block run back to back, so
+    // the block's activation rows come from DRAM once and from L2 for the other tiles, and
+    // consecutive blocks of one expert find its weights in L2
+    const int r0 = blockIdx.y * kTok;
     if (r0 >= __ldg(a.ntp)) return;  // uniform over the CTA, before any barrier or allocation
-    const int e = __ldg(a.expert_ids + blockIdx.x);
+    const int e = __ldg(a.expert_ids + blockIdx.y);
     if (e < 0 || e >= a.E) return;
-    const int n0 = blockIdx.y * 128;  // output features (gate/up) or output rows (down)
+    const int n0 = blockIdx.x * 128;  // output features (gate/up) or output rows (down)
     const int K = a.K, NS = K / kKs;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             tc::mbar_init(&b_full[s], 1);
-            tc::mbar_init(&a_full[s], kDeqWarps);
+            tc::mbar_init(&a_full[s], DW);
             tc::mbar_init(&empty[s], 1);
         }
         tc::mbar_init(acc_full, 1);
@@ -166,23 +197,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ---- dequantization ----
         const int dw = warp - 2, quarter = warp & 3, set = dw >> 2;
-        const int t = dw * 32 + lane;               // ring slot owner
-        const int row = quarter * 32 + lane;        // tensor-memory lane = weight row in the tile
-        const int grow = e * a.rows_per_expert + (GU ? (set ? a.N : 0) + n0 + row : n0 + row);
-        const int32_t *wrow = a.wq + (size_t)grow * (K / 8);
+        const int matrix = GU ? (set & 1) : 0;                   // gate/up: 0 gate, 1 up
+        const int kpart = GU ? (set >> 1) : set;                 // which words of each step
+        const int t = dw * 32 + lane;                            // ring slot owner
+        const int row = quarter * 32 + lane;                     // tensor-memory lane = weight row
+        const int grow = e * a.rows_per_expert + (GU ? (matrix ? a.N : 0) + n0 + row : n0 + row);
+        const int32_t *wrow = a.wq + (size_t)grow * (K / 8) + kpart * Sh::kWords;
         const uint16_t *srow = a.ws + (size_t)grow * (K / 32);
-        auto code_slot = [&](int slot, int part) {
-            return code_ring + ((size_t)(slot * Sh::kCodeParts + part) * kDeqThreads + t) * 16;
-        };
+        auto code_slot = [&](int slot) { return code_ring + ((size_t)slot * kDeqThreads + t) * Sh::kCodeBytes; };
         auto issue = [&](int ks) {
             if (ks < NS) {
                 const int slot = ks % kRing;
-                if (GU) {
-                    cp_async16_stream(code_slot(slot, 0), wrow + ks * 8);
-                    cp_async16_stream(code_slot(slot, 1), wrow + ks * 8 + 4);
-                } else {
-                    cp_async16_stream(code_slot(slot, 0), wrow + ks * 8 + 4 * set);
-                }
+                cp_async_codes<Sh::kCodeBytes>(code_slot(slot), wrow + ks * 8);
                 cp_async4(scale_ring + ((size_t)slot * kDeqThreads + t) * 4, srow + ks * 2);
             }
             cp_async_commit();
@@ -193,38 +219,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int ks = 0; ks < NS && ok; ++ks) {
             cp_async_wait<kRing - 2>();
             const int slot = ks % kRing;
-            const uint4 c0 = *reinterpret_cast<const uint4 *>(code_slot(slot, 0));
-            uint4 c1 = make_uint4(0u, 0u, 0u, 0u);
-            if (GU) c1 = *reinterpret_cast<const uint4 *>(code_slot(slot, 1));
+            uint32_t words[Sh::kWords];  // vector reads: a warp reads one contiguous span, no bank conflicts
+            if (Sh::kWords == 2) {
+                const uint2 v = *reinterpret_cast<const uint2 *>(code_slot(slot));
+                words[0] = v.x;
+                words[1 % Sh::kWords] = v.y;
+            } else {
+#pragma unroll
+                for (int j = 0; j < Sh::kWords; j += 4) {
+                    const uint4 v = reinterpret_cast<const uint4 *>(code_slot(slot))[j / 4];
+                    words[j] = v.x;
+                    words[(j + 1) % Sh::kWords] = v.y;
+                    words[(j + 2) % Sh::kWords] = v.z;
+                    words[(j + 3) % Sh::kWords] = v.w;
+                }
+            }
             const uint32_t sc = *reinterpret_cast<const uint32_t *>(scale_ring + ((size_t)slot * kDeqThreads + t) * 4);
             issue(ks + kRing - 1);  // refills the slot read in step ks - 1
-            uint32_t pairs[GU ? 32 : 16];
-            const uint32_t s_lo = (sc & 0xFFFFu) * 0x10001u, s_hi = (sc >> 16) * 0x10001u;
-            if (GU) {
-                dequant4(c0.x, s_lo, pairs + 0);
-                dequant4(c0.y, s_lo, pairs + 4);
-                dequant4(c0.z, s_lo, pairs + 8);
-                dequant4(c0.w, s_lo, pairs + 12);
-                dequant4(c1.x, s_hi, pairs + 16);
-                dequant4(c1.y, s_hi, pairs + 20);
-                dequant4(c1.z, s_hi, pairs + 24);
-                dequant4(c1.w, s_hi, pairs + 28);
-            } else {
-                const uint32_t s2 = set ? s_hi : s_lo;
-                dequant4(c0.x, s2, pairs + 0);
-                dequant4(c0.y, s2, pairs + 4);
-                dequant4(c0.z, s2, pairs + 8);
-                dequant4(c0.w, s2, pairs + 12);
+            uint32_t pairs[4 * Sh::kWords];
+#pragma unroll
+            for (int j = 0; j < Sh::kWords; ++j) {
+                const int group = (kpart * Sh::kWords + j) / 4;  // 0 or 1 inside the 64-input step
+                const uint32_t s16 = group ? (sc >> 16) : (sc & 0xFFFFu);
+                dequant4(words[j], s16 * 0x10001u, pairs + 4 * j);
             }
             const int s = ks % kStages;
             if (ks >= kStages)
                 ok = __all_sync(0xFFFFFFFFu, tc::mbar_wait(&empty[s], ((ks / kStages) & 1) ^ 1, abort_flag, a.status));
             if (!ok) break;
             tc::fence_after_sync();
-            const uint32_t col = Sh::kAccCols + s * Sh::kAStageCols + (GU ? set * (kKs / 2) : set * (kKs / 4));
-            const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + col;
-            if (GU) tc::tmem_st32(taddr, pairs);
-            else tc::tmem_st16(taddr, pairs);
+            const uint32_t col = Sh::kAccCols + s * Sh::kAStageCols + matrix * (kKs / 2) + kpart * 4 * Sh::kWords;
+            tmem_st_n<4 * Sh::kWords>(tmem + ((uint32_t)(quarter * 32) << 16) + col, pairs);
             tc::tmem_wait_st();
             tc::fence_before_sync();
             __syncwarp();
@@ -232,13 +257,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         cp_async_wait<0>();
 
-        // ---- epilogue: tokens [64 set, 64 set + 64) of the tile ----
+        // ---- epilogue: tokens [set * 128 / kSets, +128 / kSets) of the tile ----
         ok = ok && __all_sync(0xFFFFFFFFu, tc::mbar_wait(acc_full, 0, abort_flag, a.status));
         if (ok) {
             tc::fence_after_sync();
             const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-            for (int c = 0; c < 2; ++c) {
-                const int tok0 = set * 64 + c * 32;
+            constexpr int kTokPerSet = kTok / Sh::kSets;
+            for (int c = 0; c < kTokPerSet / 32; ++c) {
+                const int tok0 = set * kTokPerSet + c * 32;
                 uint32_t g[32];
                 tc::tmem_ld32(lane_base + tok0, g);
                 if (GU) {
@@ -300,20 +326,20 @@ __global__ void __launch_bounds__(256) gather_bf16_perm_kernel(const uint16_t *_
     }
 }
 
-template <int MODE>
+template <int MODE, int DW>
 int launch_mode(const W4TcArgs &a, const CUtensorMap &tm, int grid_x, int grid_y, cudaStream_t s)
 {
-    using Sh = W4TcShape<MODE>;
+    using Sh = W4TcShape<MODE, DW>;
     static bool attr = false;
     if (!attr) {
-        const cudaError_t e =
-            cudaFuncSetAttribute(w4a16_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Sh::kSmemBytes);
+        const cudaError_t e = cudaFuncSetAttribute(w4a16_tc_kernel<MODE, DW>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Sh::kSmemBytes);
         if (e != cudaSuccess)
             return set_error(MOEQ_ERR_CUDA, "tcgen05 W4A16 GEMM: shared-memory attribute: %s", cudaGetErrorString(e));
         attr = true;
     }
     if (grid_x <= 0 || grid_y <= 0) return MOEQ_OK;
-    w4a16_tc_kernel<MODE><<<dim3(grid_x, grid_y), kThreads, Sh::kSmemBytes, s>>>(tm, a);
+    w4a16_tc_kernel<MODE, DW><<<dim3(grid_x, grid_y), Sh::kThreads, Sh::kSmemBytes, s>>>(tm, a);
     return MOEQ_OK;
 }
 
@@ -324,8 +350,9 @@ int launch_w4a16_tc(const W4TcArgs &a, int mode, const uint16_t *act, int max_bl
     CUtensorMap tm;
     const int rc = make_tmap_2d(&tm, act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.M, (uint64_t)a.K, kTok, kKs);
     if (rc) return rc;
-    if (mode == TC_GATEUP) return launch_mode<TC_GATEUP>(a, tm, max_blocks, a.N / 128, s);
-    return launch_mode<TC_DOWN>(a, tm, max_blocks, a.N / 128, s);
+    // gate/up: 16 dequantization warps; down (shorter K, two CTAs per SM): 8
+    if (mode == TC_GATEUP) return launch_mode<TC_GATEUP, 16>(a, tm, a.N / 128, max_blocks, s);
+    return launch_mode<TC_DOWN, 8>(a, tm, a.N / 128, max_blocks, s);
 }
 
 void launch_gather_bf16_perm(const uint16_t *x, int H, int k, const int32_t *sorted_ids, const int32_t *ntp,
