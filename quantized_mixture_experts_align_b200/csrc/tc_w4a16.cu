@@ -18,14 +18,17 @@
 // same order inside every 8-element chunk (done by the gather and by the gate/up epilogue).
 //
 // CTA = one 128-row activation block of one expert x 128 output features:
-//   warp 0      TMA producer of the activation tiles [128 tokens x 64 inputs] (4 stages);
+//   warp 0      TMA producer of the activation tiles [128 tokens x 64 inputs] (gate/up 8
+//               stages, down 4), released by their own barriers so the producer runs ahead of
+//               the 4 tensor-memory weight stages;
 //   warp 1      tensor-memory allocation; lane 0 issues the MMAs (gate/up: one MMA into each of
 //               the two accumulators per 16 inputs) and commits;
 //   warps 2..  dequantization (gate/up 16 warps, down 8): a thread owns one weight row and a
-//               part of each 64-input step (gate/up: one matrix, half the step; down: half), prefetches its packed codes and scales through a private 8-deep cp.async
-//               ring, and writes the dequantized part to a tensor-memory stage; then the
-//               epilogue: gate/up writes h = bf16(silu(g) * u) in the permuted order, down
-//               writes the routing-weighted f32 slot rows.
+//               part of each 64-input step (gate/up: one matrix, half the step; down: half),
+//               prefetches its packed codes and scales through a private 6-deep cp.async ring,
+//               and writes the dequantized part to a tensor-memory stage; then the epilogue:
+//               gate/up writes h = bf16(silu(g) * u) in the permuted order, down writes the
+//               routing-weighted f32 slot rows.
 #include "kernels.cuh"
 #include "tc_common.cuh"
 
@@ -35,7 +38,7 @@ namespace {
 
 constexpr int kTok = 128;     // tokens per tile = aligned block size
 constexpr int kKs = 64;       // inputs per pipeline step
-constexpr int kStages = 4;    // activation tiles (shared memory) and weight stages (tensor memory)
+constexpr int kStages = 4;    // dequantized weight stages (tensor memory)
 
 // DW dequantization warps: 4 tensor-memory lane quarters x (DW / 4) "sets". A set is, for
 // gate/up, a (matrix, K part) pair (matrix = set % 2), for down a K part; each thread converts
@@ -43,8 +46,10 @@ constexpr int kStages = 4;    // activation tiles (shared memory) and weight sta
 template <int MODE, int DW>
 struct W4TcShape {
     static constexpr bool kGU = MODE == TC_GATEUP;
-    // per-thread packed-code prefetch depth, in steps (down: shallower, so two CTAs fit an SM)
-    static constexpr int kRing = kGU ? 8 : 6;
+    // per-thread packed-code prefetch depth, in steps, and activation-tile stages (shared
+    // memory); down keeps both shallower so two CTAs fit an SM
+    static constexpr int kRing = 6;
+    static constexpr int kBStages = kGU ? 8 : 4;
     static constexpr int kSets = DW / 4;
     static constexpr int kKParts = kGU ? kSets / 2 : kSets;
     static constexpr int kWords = 8 / kKParts;                       // code words per thread per step
@@ -59,7 +64,7 @@ struct W4TcShape {
     static constexpr int kBTile = kTok * kKs * 2;                    // 16 KB
     static constexpr size_t kCodeRing = (size_t)kRing * kDeqThreads * kCodeBytes;
     static constexpr size_t kScaleRing = (size_t)kRing * kDeqThreads * 4;
-    static constexpr size_t kSmemBytes = 1024 + (size_t)kStages * kBTile + kCodeRing + kScaleRing + 256;
+    static constexpr size_t kSmemBytes = 1024 + (size_t)kBStages * kBTile + kCodeRing + kScaleRing + 256;
 };
 
 __device__ __forceinline__ void cp_async4(void *dst, const void *src)
@@ -111,14 +116,16 @@ __global__ void __launch_bounds__((2 + DW) * 32, 1)
     using Sh = W4TcShape<MODE, DW>;
     constexpr int kDeqThreads = Sh::kDeqThreads;
     constexpr int kRing = Sh::kRing;
+    constexpr int kBStages = Sh::kBStages;
     constexpr bool GU = Sh::kGU;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *btiles = smem;
-    uint8_t *code_ring = btiles + kStages * Sh::kBTile;
+    uint8_t *code_ring = btiles + kBStages * Sh::kBTile;
     uint8_t *scale_ring = code_ring + Sh::kCodeRing;
     uint64_t *b_full = reinterpret_cast<uint64_t *>(scale_ring + Sh::kScaleRing);
-    uint64_t *a_full = b_full + kStages;
+    uint64_t *b_empty = b_full + kBStages;
+    uint64_t *a_full = b_empty + kBStages;
     uint64_t *empty = a_full + kStages;
     uint64_t *acc_full = empty + kStages;
     uint64_t *mma_done = acc_full + 1;
@@ -137,8 +144,11 @@ __global__ void __launch_bounds__((2 + DW) * 32, 1)
     const int K = a.K, NS = K / kKs;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kBStages; ++s) {
             tc::mbar_init(&b_full[s], 1);
+            tc::mbar_init(&b_empty[s], 1);
+        }
+        for (int s = 0; s < kStages; ++s) {
             tc::mbar_init(&a_full[s], DW);
             tc::mbar_init(&empty[s], 1);
         }
@@ -158,25 +168,25 @@ __global__ void __launch_bounds__((2 + DW) * 32, 1)
             tc::prefetch_tmap(&tmX);
             int issued = 0;
             for (int ks = 0; ks < NS; ++ks) {
-                const int s = ks % kStages;
-                if (ks >= kStages && !tc::mbar_wait(&empty[s], ((ks / kStages) & 1) ^ 1, abort_flag, a.status)) break;
+                const int s = ks % kBStages;
+                if (ks >= kBStages && !tc::mbar_wait(&b_empty[s], ((ks / kBStages) & 1) ^ 1, abort_flag, a.status))
+                    break;
                 tc::mbar_arrive_expect_tx(&b_full[s], Sh::kBTile);
                 tc::tma_load_2d(btiles + s * Sh::kBTile, &tmX, &b_full[s], ks * kKs, r0);
                 issued = ks + 1;
             }
-            for (int ks = issued - kStages > 0 ? issued - kStages : 0; ks < issued; ++ks)
-                tc::mbar_drain(&b_full[ks % kStages], (ks / kStages) & 1, a.status);
+            for (int ks = issued - kBStages > 0 ? issued - kBStages : 0; ks < issued; ++ks)
+                tc::mbar_drain(&b_full[ks % kBStages], (ks / kBStages) & 1, a.status);
         }
     } else if (warp == 1) {
         if (lane == 0) {
             constexpr uint32_t idesc = tc::idesc_f32(tc::kFmtBF16, tc::kFmtBF16, 128, kTok);
             for (int ks = 0; ks < NS; ++ks) {
-                const int s = ks % kStages;
-                const uint32_t par = (ks / kStages) & 1;
-                if (!tc::mbar_wait(&b_full[s], par, abort_flag, a.status)) break;
-                if (!tc::mbar_wait(&a_full[s], par, abort_flag, a.status)) break;
+                const int s = ks % kStages, sb = ks % kBStages;
+                if (!tc::mbar_wait(&b_full[sb], (ks / kBStages) & 1, abort_flag, a.status)) break;
+                if (!tc::mbar_wait(&a_full[s], (ks / kStages) & 1, abort_flag, a.status)) break;
                 tc::fence_after_sync();
-                const uint64_t bdesc = tc::smem_desc_sw128(btiles + s * Sh::kBTile);
+                const uint64_t bdesc = tc::smem_desc_sw128(btiles + sb * Sh::kBTile);
                 const uint32_t astage = tmem + Sh::kAccCols + s * Sh::kAStageCols;
 #pragma unroll
                 for (int kk = 0; kk < kKs / 16; ++kk) {
@@ -189,6 +199,7 @@ __global__ void __launch_bounds__((2 + DW) * 32, 1)
                     }
                 }
                 tc::mma_commit(&empty[s]);
+                tc::mma_commit(&b_empty[sb]);
             }
             tc::mma_commit(acc_full);
             tc::mma_commit(mma_done);
