@@ -9,7 +9,7 @@
 // consecutive CTAs take consecutive blocks, so the blocks of one expert share its weights in L2.
 // Each warp owns 16 (gate/up) or 32 (down) output rows for the whole K range and streams its
 // packed weights from HBM through its own multi-stage cp.async ring in shared memory (16 B per
-// lane per 128 inputs per row set; five stages in flight hide the HBM latency without holding
+// lane per 128 inputs per row set; three stages in flight hide the HBM latency without holding
 // registers). Every weight byte is used by exactly one warp, so the dequantized weights never go
 // back to shared memory: a dequantized 32-bit word feeds two m16n8k16 k-steps directly as A
 // fragments.
@@ -57,8 +57,10 @@ __device__ __forceinline__ void act_pairs(const uint4 &v, uint32_t (&b)[4])
 
 // Per-warp weight ring: each stage holds one 128-input quad-group of the warp's 4 row sets
 // (16 B per lane per row set, lane-private slots) and their 4 bf16 scales per row (8 B per row,
-// copied by lane (g, t) for row set t, row g and shared across the warp).
-constexpr int kW4Stages = 6;
+// copied by lane (g, t) for row set t, row g and shared across the warp). Four stages measured
+// best: a deeper ring takes shared memory from the L1 share of the unified L1/shared storage,
+// which the activation and scale loads use.
+constexpr int kW4Stages = 4;
 constexpr int kW4StageBytes = 4 * 32 * 16 + 4 * 8 * 8;  // 2048 B codes + 256 B scales
 
 // MODE_GATEUP: rows [f0, f0+16) (gate) and [I + f0, I + f0 + 16) (up) of W13; epilogue writes
