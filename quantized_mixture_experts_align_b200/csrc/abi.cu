@@ -112,9 +112,9 @@ static int pick_block_m(long T, int k, int E)
     return 64;
 }
 
-// Dense block-FP8: from this many rows on, the tcgen05 kernel (128-row tiles, tensor-core bound)
-// replaces the register-fed swap-AB kernel (weight-streaming, HBM bound).
-static int kDenseTcMinM = 128;
+// Dense block-FP8: up to 16 rows the register-fed kernel (K split over warps) streams the
+// weights; from 17 rows on, the tcgen05 kernel (128-row tiles). Chosen from measured M sweeps.
+static int kDenseTcMinM = 17;
 
 static int pick_block_m_dense(int M)
 {
@@ -603,7 +603,7 @@ int w8a8_block_fp8_matmul(const uint8_t *A, const float *As, const uint8_t *B, c
     const int bm = pick_block_m_dense(M);
     {
         trace::Scope ts(trace::DENSE, (cudaStream_t)stream);
-        launch_fp8_grouped_mma(a, MODE_DENSE, bm, cdiv(M, bm), (cudaStream_t)stream);
+        launch_fp8_dense_splitk(a, bm, (cudaStream_t)stream);
     }
     return check_launch("w8a8_block_fp8_matmul");
 }

@@ -91,6 +91,8 @@ void launch_combine(const float *ys, int T, int k, int H, uint16_t *out, int num
 void launch_fp8_act_quant(const uint16_t *x, int rows, int cols, uint8_t *q, float *s, cudaStream_t st);
 void launch_w4a16_grouped_mma(const W4GroupedArgs &a, int mode, int block_m, int max_blocks, cudaStream_t s);
 void launch_fp8_grouped_mma(const F8GroupedArgs &a, int mode, int block_m, int max_blocks, cudaStream_t s);
+// Dense block-FP8 for few rows: K split over the 4 warps of a CTA, 32 weight rows per CTA.
+void launch_fp8_dense_splitk(const F8GroupedArgs &a, int block_m, cudaStream_t s);
 // tcgen05 block-FP8 GEMM: A [M, K] and B [N, K] E4M3, K % 128 == 0, N % 128 == 0. Returns a status.
 int launch_fp8_tc_gemm(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B, cudaStream_t s);
 // tcgen05 grouped block-FP8 GEMM over expert-contiguous rows A [M, K] (128-row blocks, one expert

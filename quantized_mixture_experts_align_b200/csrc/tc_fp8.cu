@@ -44,7 +44,7 @@ struct Fp8TcShape {
     static constexpr int kABytes = kBM * kBK;
     static constexpr int kBBytes = BN * kBK;
     static constexpr int kStageBytes = kABytes + kBBytes;
-    static constexpr int kTmemCols = 2 * BN;  // two partial buffers (256 or 512 columns)
+    static constexpr int kTmemCols = 2 * BN;  // two partial buffers (128, 256 or 512 columns)
     static constexpr int kColsPerWarp = BN / 2;
     static constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + 1024 + 256 + 2 * 128 * 4;
 };
@@ -188,8 +188,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + buf * BN;
 #pragma unroll
             for (int c = 0; c < COLS / 32; ++c) {
-                const bool second = c >= COLS / 64;
-                const int col = (second ? c_second : c_first) + (c % (COLS / 64)) * 32;
+                // gate/up: chunks 0-1 gate, 2-3 up; otherwise one contiguous run of columns
+                const bool second = (MODE == TC_GATEUP) && c >= 2;
+                const int col = (MODE == TC_GATEUP) ? (second ? c_second : c_first) + (c & 1) * 32 : c_first + c * 32;
                 const float sc = second ? sc1 : sc0;
                 uint32_t r[32];
                 tc::tmem_ld32(taddr + col, r);
@@ -283,14 +284,18 @@ int launch_tc(const Fp8TcArgs &a, const CUtensorMap &tmA, const CUtensorMap &tmB
 
 int launch_fp8_tc_gemm(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B, cudaStream_t s)
 {
-    const int bn = (a.N % 256 == 0) ? 256 : 128;
+    // Up to 64 rows the weights stream once (HBM bound) and narrow 64-column tiles give every SM
+    // several CTAs; from 65 rows, 256-column tiles (more weight bytes in flight per SM, fewer
+    // activation re-reads; tensor bound for many rows). Chosen from measured M sweeps.
+    const int bn = (a.M <= 64) ? 64 : (a.N % 256 == 0) ? 256 : 128;
     CUtensorMap tmA, tmB;
     int rc = make_tmap_2d(&tmA, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.M, (uint64_t)a.K, kBM, kBK);
     if (rc) return rc;
     rc = make_tmap_2d(&tmB, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.N, (uint64_t)a.K, bn, kBK);
     if (rc) return rc;
     if (bn == 256) return launch_tc<256, TC_DENSE>(a, tmA, tmB, cdiv(a.M, kBM), a.N / 256, s);
-    return launch_tc<128, TC_DENSE>(a, tmA, tmB, cdiv(a.M, kBM), a.N / 128, s);
+    if (bn == 128) return launch_tc<128, TC_DENSE>(a, tmA, tmB, cdiv(a.M, kBM), a.N / 128, s);
+    return launch_tc<64, TC_DENSE>(a, tmA, tmB, cdiv(a.M, kBM), a.N / 64, s);
 }
 
 int launch_fp8_tc_grouped(const Fp8TcArgs &a, int mode, const uint8_t *A, const uint8_t *W, int E, int max_blocks,
