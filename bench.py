@@ -71,11 +71,20 @@ def barrier(world):
 
 
 def max_over_ranks(v: float, world: int) -> float:
+    """Max of a per-rank value over all ranks (timings: the slowest rank sets the job's time)."""
     if world == 1:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_value(units_per_rank: float, ms_per_rank: float, world: int) -> tuple[float, float]:
+    """Whole-job throughput of `world` independent replicas: all ranks' units over the slowest
+    rank's time. Returns (units per second, slowest ms)."""
+    ms = max_over_ranks(ms_per_rank, world)
+    return world * units_per_rank / (ms * 1e-3), ms
 
 
 # ---------------------------------------------------------------------------------------------
@@ -292,7 +301,9 @@ def reference_arm(args, rank, world):
     T = d["T"]
     n_active = int(np.unique(oracle.route_topk(W.np_bits(d["logits"]), d["k"])[0]).size)
     gbytes = n_active * W.w4a16_expert_bytes(d["H"], d["I"]) / 1e9
-    ntok = 1
+    # each step: the oracle over a bounded sample of the decode batch (4 of its 32 tokens, ~0.2 s
+    # on 16 cores), scaled to the full step, so --steps K --warmup W ends within minutes
+    ntok = 4
     for _ in range(args.warmup):
         oracle_sample_time(d, ntok)
     times = [oracle_sample_time(d, ntok) for _ in range(args.steps)]
@@ -382,8 +393,7 @@ def main():
     dev_index = torch.cuda.current_device()
     with ClockSampler(dev_index) as clk:
         ms, stages, _ = run_w4a16(moeq, d, args.steps, args.warmup, flush, world, trace=True)
-    ms_step = max_over_ranks(statistics.mean(ms), world)
-    value = world * step_bytes / (ms_step * 1e-3) / 1e9
+    value, ms_step = job_value(step_bytes / 1e9, statistics.mean(ms), world)
     gu_ms, gu_calls = stages["gate_up"]
     gu_avg = gu_ms / max(gu_calls, 1)
     gu_bytes = n_active * (d["H"] * 2 * d["I"] // 2 + d["H"] // 32 * 2 * d["I"] * 2)
@@ -397,8 +407,8 @@ def main():
     del w13_bytes
 
     e2e_ms, h2d, d2h = e2e_w4a16(moeq, d, args.steps, args.warmup, world)
-    e2e_step = max_over_ranks(statistics.mean(e2e_ms), world)
-    e2e = {"value": world * step_bytes / (e2e_step * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+    e2e_value, e2e_step = job_value(step_bytes / 1e9, statistics.mean(e2e_ms), world)
+    e2e = {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h, "ms_per_step": e2e_step}
 
     line = {
@@ -465,13 +475,15 @@ def main():
     # ---- CPU baseline: the oracle as it stands, bounded sample, rank 0 only --------------------
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
-        ntok = 1
-        t_s = oracle_sample_time(d, ntok)
-        full_s = t_s * d["T"] / ntok
+        # whole decode steps (all T tokens), repeated until about 10 s of CPU work
+        times = []
+        while sum(times) < 10.0 and len(times) < 20:
+            times.append(oracle_sample_time(d, d["T"]))
+        full_s = statistics.mean(times)
         line["cpu_baseline"] = {"value": step_bytes / full_s / 1e9, "unit": "GB/s", "cores": oracle.threads(),
                                 "kind": "oracle",
-                                "sample": f"{ntok} of {d['T']} decode tokens timed ({t_s:.1f} s), scaled x{d['T']}; "
-                                          f"host CPU: {cpu_info()}"}
+                                "sample": f"{len(times)} full decode steps ({d['T']} tokens each, {sum(times):.1f} s "
+                                          f"total); host CPU: {cpu_info()}"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

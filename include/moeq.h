@@ -187,6 +187,17 @@ MOEQ_API int moe_trace_read(double *stage_ms, long long *stage_calls, int n_stag
  */
 MOEQ_API int moe_device_status(int clear);
 
+/*
+ * Failure-detection self-test (diagnostic; the pages have no counterpart). Every wait inside the
+ * tensor-core kernels is bounded: a wait that gives up sets the device status word and its CTA
+ * drains and exits, so a stuck pipeline surfaces as MOEQ_ERR_DEVICE_TIMEOUT from
+ * moe_device_status() instead of a hung GPU. This call enqueues a one-CTA kernel that runs the
+ * same bounded wait on a barrier nothing ever arrives at, with a short poll limit; afterwards
+ * moe_device_status() reports MOEQ_ERR_DEVICE_TIMEOUT (clear it with moe_device_status(1)).
+ * No fault, trap or hang is involved; the context stays usable.
+ */
+MOEQ_API int moe_selftest_bounded_wait(void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -41,6 +41,7 @@ _SIGNATURES = {
     "moe_trace_enable": ([_I], _I),
     "moe_trace_read": ([_V, _V, _I, _I], _I),
     "moe_device_status": ([_I], _I),
+    "moe_selftest_bounded_wait": ([_V], _I),
 }
 
 
@@ -213,6 +214,10 @@ def moe_trace_read(reset: bool = False) -> dict:
     if rc != n:
         _check(rc)
     return {name: (ms[i], calls[i]) for i, name in enumerate(TRACE_STAGES)}
+
+
+def moe_selftest_bounded_wait(stream=None):
+    _check(lib().moe_selftest_bounded_wait(_stream(stream)))
 
 
 def moe_device_status(clear: bool = False) -> int:

@@ -643,6 +643,14 @@ int moe_trace_read(double *stage_ms, long long *stage_calls, int n_stages, int r
     return trace::NSTAGE;
 }
 
+int moe_selftest_bounded_wait(void *stream)
+{
+    g_err[0] = 0;
+    const int rc = launch_selftest_bounded_wait((cudaStream_t)stream);
+    if (rc) return rc;
+    return check_launch("moe_selftest_bounded_wait");
+}
+
 int moe_device_status(int clear)
 {
     g_err[0] = 0;

@@ -53,9 +53,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
 
 // Wait for the phase with the given parity to complete; false (and `*abort` set, status word
 // written) if it does not within kMaxPolls polls or if another thread already gave up.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort, int *status)
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort, int *status,
+                                          uint32_t max_polls = kMaxPolls)
 {
-    for (uint32_t i = 0; i < kMaxPolls; ++i) {
+    for (uint32_t i = 0; i < max_polls; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 255u) == 255u && *abort) return false;
     }
@@ -207,5 +208,7 @@ int make_tmap_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype, 
 
 // Host: device address of the library's kernel status word on the current device.
 int *device_status_ptr();
+// Host: launches the bounded-wait self-test kernel (see moe_selftest_bounded_wait).
+int launch_selftest_bounded_wait(cudaStream_t s);
 
 }  // namespace moeq

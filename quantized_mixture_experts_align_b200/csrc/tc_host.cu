@@ -45,6 +45,29 @@ int make_tmap_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype, 
     return MOEQ_OK;
 }
 
+// A wait that can never complete (nothing arrives on the barrier), given a short poll limit: the
+// bounded-wait helper every tensor-core kernel uses must give up and flag the status word.
+__global__ void selftest_bounded_wait_kernel(uint32_t polls, int *status)
+{
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        tc::mbar_init(&bar, 1);
+        abort_flag = 0;
+        tc::fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) tc::mbar_wait(&bar, 0, &abort_flag, status, polls);
+}
+
+int launch_selftest_bounded_wait(cudaStream_t s)
+{
+    int *status = device_status_ptr();
+    if (!status) return set_error(MOEQ_ERR_CUDA, "moe_selftest_bounded_wait: no device status word");
+    selftest_bounded_wait_kernel<<<1, 32, 0, s>>>(4096u, status);
+    return MOEQ_OK;
+}
+
 int *device_status_ptr()
 {
     int dev = 0;
