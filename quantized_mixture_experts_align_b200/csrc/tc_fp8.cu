@@ -143,17 +143,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         if (lane == 0) {
             constexpr uint32_t idesc = tc::idesc_f32(tc::kFmtE4M3, tc::kFmtE4M3, kBM, BN);
+            const uint64_t a_base = tc::smem_desc_sw128(smem);
             for (int kb = 0; kb < KB; ++kb) {
                 const int s = kb % kStages, buf = kb & 1;
                 if (!tc::mbar_wait(&full[s], (kb / kStages) & 1, abort_flag, a.status)) break;
                 if (kb >= 2 && !tc::mbar_wait(&tempty[buf], ((kb >> 1) & 1) ^ 1, abort_flag, a.status)) break;
                 tc::fence_after_sync();
-                const uint8_t *sa = smem + s * Sh::kStageBytes;
-                const uint64_t adesc = tc::smem_desc_sw128(sa);
-                const uint64_t bdesc = tc::smem_desc_sw128(sa + Sh::kABytes);
+                // lean issue path: descriptors from a precomputed base; the first MMA of each K block
+                // starts the partial, the other three always accumulate
+                const uint64_t adesc = a_base + (uint64_t)((s * Sh::kStageBytes) >> 4);
+                const uint64_t bdesc = adesc + (uint64_t)(Sh::kABytes >> 4);
+                const uint32_t d = tmem + buf * BN;
+                tc::mma_f8f6f4_ss(d, adesc, bdesc, idesc, 0u);
 #pragma unroll
-                for (int kk = 0; kk < kBK / 32; ++kk)
-                    tc::mma_f8f6f4_ss(tmem + buf * BN, adesc + 2 * kk, bdesc + 2 * kk, idesc, kk > 0 ? 1u : 0u);
+                for (int kk = 1; kk < kBK / 32; ++kk) tc::mma_f8f6f4_ss_acc(d, adesc + 2 * kk, bdesc + 2 * kk, idesc);
                 tc::mma_commit(&empty[s]);
                 tc::mma_commit(&tfull[buf]);
             }

@@ -181,21 +181,29 @@ __global__ void __launch_bounds__((2 + DW) * 32, 1)
     } else if (warp == 1) {
         if (lane == 0) {
             constexpr uint32_t idesc = tc::idesc_f32(tc::kFmtBF16, tc::kFmtBF16, 128, kTok);
+            // lean issue path: stage bases precomputed, the first step peeled, then MMAs that always
+            // accumulate (the dequantization warps keep this SM's issue slots busy)
+            const uint32_t a_base = tmem + Sh::kAccCols;
+            const uint64_t b_base = tc::smem_desc_sw128(btiles);
             for (int ks = 0; ks < NS; ++ks) {
                 const int s = ks % kStages, sb = ks % kBStages;
                 if (!tc::mbar_wait(&b_full[sb], (ks / kBStages) & 1, abort_flag, a.status)) break;
                 if (!tc::mbar_wait(&a_full[s], (ks / kStages) & 1, abort_flag, a.status)) break;
                 tc::fence_after_sync();
-                const uint64_t bdesc = tc::smem_desc_sw128(btiles + sb * Sh::kBTile);
-                const uint32_t astage = tmem + Sh::kAccCols + s * Sh::kAStageCols;
+                const uint64_t bdesc = b_base + (uint64_t)((sb * Sh::kBTile) >> 4);
+                const uint32_t astage = a_base + s * Sh::kAStageCols;
+                if (ks == 0) {
 #pragma unroll
-                for (int kk = 0; kk < kKs / 16; ++kk) {
-                    const uint32_t acc = (ks > 0 || kk > 0) ? 1u : 0u;
-                    if (GU) {
+                    for (int kk = 0; kk < kKs / 16; ++kk) {
+                        const uint32_t acc = kk > 0 ? 1u : 0u;
                         tc::mma_f16_ts(tmem, astage + kk * 8, bdesc + 2 * kk, idesc, acc);
-                        tc::mma_f16_ts(tmem + kTok, astage + kKs / 2 + kk * 8, bdesc + 2 * kk, idesc, acc);
-                    } else {
-                        tc::mma_f16_ts(tmem, astage + kk * 8, bdesc + 2 * kk, idesc, acc);
+                        if (GU) tc::mma_f16_ts(tmem + kTok, astage + kKs / 2 + kk * 8, bdesc + 2 * kk, idesc, acc);
+                    }
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < kKs / 16; ++kk) {
+                        tc::mma_f16_ts_acc(tmem, astage + kk * 8, bdesc + 2 * kk, idesc);
+                        if (GU) tc::mma_f16_ts_acc(tmem + kTok, astage + kKs / 2 + kk * 8, bdesc + 2 * kk, idesc);
                     }
                 }
                 tc::mma_commit(&empty[s]);
