@@ -164,7 +164,7 @@ static RouteBufs carve_route(Carve &c, long T, int k, int E, int block_m)
 }
 
 // W4A16 layer schedule: from this many routed rows per expert on (mean T*k/E), the grouped GEMMs
-// run on the tensor-core kernels over 128-row expert blocks (weights dequantized into tensor
+// run on the tensor-core kernels over 256-row expert blocks (weights dequantized into tensor
 // memory); below, the register-fed swap-AB kernels stream the weights for the few rows each
 // expert has (HBM bound).
 static bool w4_use_tc(long T, int k, int E) { return (double)T * k / (double)E >= 16.0; }
@@ -173,7 +173,7 @@ static size_t w4a16_layout(Carve &c, long T, int H, int I, int E, int k, RouteBu
                            uint16_t **xg = nullptr)
 {
     const bool tcp = w4_use_tc(T, k, E);
-    RouteBufs r = carve_route(c, T, k, E, tcp ? 128 : pick_block_m(T, k, E));
+    RouteBufs r = carve_route(c, T, k, E, tcp ? 256 : pick_block_m(T, k, E));  // tensor-core tiles: 256 rows
     const size_t cap = (size_t)r.max_blocks * r.block_m;
     uint16_t *hp = c.take<uint16_t>((tcp ? cap : (size_t)T * k) * I);
     float *yp = c.take<float>((size_t)T * k * H);
@@ -344,7 +344,7 @@ int moe_w4a16_forward(const uint16_t *x, const float *logits, int T, int H, int 
     if (tcp) {
         int *status = device_status_ptr();
         if (!status) return set_error(MOEQ_ERR_CUDA, "moe_w4a16_forward: no device status word");
-        const int cap = r.max_blocks * 128;
+        const int cap = r.max_blocks * r.block_m;
         {
             trace::Scope ts(trace::ACT_QUANT, s);  // the activation gather takes the act-prep slot
             launch_gather_bf16_perm(x, H, k, r.sorted, r.ntp, n, cap, xg, num_sms(), s);

@@ -136,6 +136,12 @@ __device__ __forceinline__ void cp_async8(void *dst, const void *src)
     asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
 }
 
+// 4 bytes (4-byte aligned source and destination)
+__device__ __forceinline__ void cp_async4_ca(void *dst, const void *src)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
+}
+
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 
 template <int N>

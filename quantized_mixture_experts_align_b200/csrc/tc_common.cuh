@@ -65,6 +65,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     return false;
 }
 
+// Warp-wide wait: lane 0 polls, the warp agrees on the result (tensor-memory operations that
+// follow are warp-collective and ordered after the wait by the warp synchronization).
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort, int *status)
+{
+    bool ok = true;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, status);
+    return __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+}
+
 // Bounded wait that ignores the abort flag: used to drain copies / MMAs still in flight before a
 // CTA releases its shared or tensor memory.
 __device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity, int *status)

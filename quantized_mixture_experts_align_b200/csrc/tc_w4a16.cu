@@ -11,24 +11,27 @@
 // codes into bf16 in registers and store them with tcgen05.st, so dequantized weights never pass
 // through shared memory (a bf16 B-side tile would cost its shared-memory bandwidth twice, on
 // write and on every MMA read). The activations (routed rows gathered in aligned order, one
-// expert per 128-row block) are the B side, loaded by TMA with the 128-byte swizzle.
-//   D[weight rows, tokens] += A_tmem[weight rows, K] * B_smem[tokens, K]^T   (M = N = 128, K = 16)
+// expert per 256-row block) are the B side, loaded by TMA with the 128-byte swizzle.
+//   D[weight rows, tokens] += A_tmem[128 weight rows, K] * B_smem[tokens, K]^T   (M = 128, K = 16)
+// A tile serves up to 256 tokens, so each dequantized weight feeds 256 rows of MMA work: the
+// dequantization, not the MMA, bounds this kernel, and the wide tile halves it per FLOP. The
+// MMA's N is the block's real row count rounded up to 16, so padding rows cost no MMA work.
 // The nibble pairs that one shift + LOP3 extracts, (q0,q4) (q1,q5) (q2,q6) (q3,q7) of each
 // 32-bit word, become consecutive K in tensor memory, so the activations are stored with the
 // same order inside every 8-element chunk (done by the gather and by the gate/up epilogue).
 //
-// CTA = one 128-row activation block of one expert x 128 output features:
-//   warp 0      TMA producer of the activation tiles [128 tokens x 64 inputs] (gate/up 8
-//               stages, down 4), released by their own barriers so the producer runs ahead of
-//               the 4 tensor-memory weight stages;
-//   warp 1      tensor-memory allocation; lane 0 issues the MMAs (gate/up: one MMA into each of
-//               the two accumulators per 16 inputs) and commits;
-//   warps 2..  dequantization (gate/up 16 warps, down 8): a thread owns one weight row and a
-//               part of each 64-input step (gate/up: one matrix, half the step; down: half),
-//               prefetches its packed codes and scales through a private 6-deep cp.async ring,
-//               and writes the dequantized part to a tensor-memory stage; then the epilogue:
-//               gate/up writes h = bf16(silu(g) * u) in the permuted order, down writes the
-//               routing-weighted f32 slot rows.
+// CTA = one 256-row activation block of one expert x (gate/up: 64 features, gate rows in tensor
+// lanes 0-63 and the matching up rows in lanes 64-127; down: 128 output rows):
+//   warp 0      TMA producer of the activation tiles [256 tokens x 64 inputs] (4 stages, own
+//               barriers);
+//   warp 1      tensor-memory allocation; lane 0 issues 4 MMAs (K = 16) per 64-input step into
+//               the one accumulator and commits;
+//   warps 2-9   dequantization: a thread owns one weight row (tensor lane) and half of each
+//               64-input step, prefetches its packed codes and scale through a private 6-deep
+//               cp.async ring, and writes the dequantized half-step to one of 4 tensor-memory
+//               stages; then the epilogue: gate/up passes the up values through shared memory
+//               to the warps holding the gate values, which write h = bf16(silu(g) * u) in the
+//               permuted order; down writes the routing-weighted f32 slot rows.
 #include "kernels.cuh"
 #include "tc_common.cuh"
 
@@ -36,61 +39,23 @@ namespace moeq {
 
 namespace {
 
-constexpr int kTok = 128;     // tokens per tile = aligned block size
+constexpr int kTok = 256;     // tokens per tile = aligned block size
 constexpr int kKs = 64;       // inputs per pipeline step
 constexpr int kStages = 4;    // dequantized weight stages (tensor memory)
-
-// DW dequantization warps: 4 tensor-memory lane quarters x (DW / 4) "sets". A set is, for
-// gate/up, a (matrix, K part) pair (matrix = set % 2), for down a K part; each thread converts
-// kWords code words of one weight row per 64-input step.
-template <int MODE, int DW>
-struct W4TcShape {
-    static constexpr bool kGU = MODE == TC_GATEUP;
-    // per-thread packed-code prefetch depth, in steps, and activation-tile stages (shared
-    // memory); down keeps both shallower so two CTAs fit an SM
-    static constexpr int kRing = 6;
-    static constexpr int kBStages = kGU ? 8 : 4;
-    static constexpr int kSets = DW / 4;
-    static constexpr int kKParts = kGU ? kSets / 2 : kSets;
-    static constexpr int kWords = 8 / kKParts;                       // code words per thread per step
-    static constexpr int kCodeBytes = kWords * 4;                    // 32, 16 or 8
-    static constexpr int kDeqThreads = DW * 32;
-    static constexpr int kThreads = (2 + DW) * 32;
-    static constexpr int kAccCols = kGU ? 2 * kTok : kTok;          // D_gate | D_up, or D
-    static constexpr int kAStageCols = kGU ? kKs : kKs / 2;          // bf16 pairs per stage
-    static constexpr int kTmemCols = kGU ? 512 : 256;
-    static_assert(kAccCols + kStages * kAStageCols <= kTmemCols, "tensor memory budget");
-    static_assert(kKParts >= 1 && kWords >= 2, "dequantization split");
-    static constexpr int kBTile = kTok * kKs * 2;                    // 16 KB
-    static constexpr size_t kCodeRing = (size_t)kRing * kDeqThreads * kCodeBytes;
-    static constexpr size_t kScaleRing = (size_t)kRing * kDeqThreads * 4;
-    static constexpr size_t kSmemBytes = 1024 + (size_t)kBStages * kBTile + kCodeRing + kScaleRing + 256;
-};
-
-__device__ __forceinline__ void cp_async4(void *dst, const void *src)
-{
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
-}
-
-template <int BYTES>
-__device__ __forceinline__ void cp_async_codes(void *dst, const void *src)
-{
-    if (BYTES == 8) {
-        cp_async8(dst, src);
-    } else {
-#pragma unroll
-        for (int p = 0; p < BYTES / 16; ++p)
-            cp_async16_stream(static_cast<uint8_t *>(dst) + 16 * p, static_cast<const uint8_t *>(src) + 16 * p);
-    }
-}
-
-template <int N>
-__device__ __forceinline__ void tmem_st_n(uint32_t taddr, const uint32_t *r)
-{
-    if (N == 8) tc::tmem_st8(taddr, *reinterpret_cast<const uint32_t(*)[8]>(r));
-    else if (N == 16) tc::tmem_st16(taddr, r);
-    else tc::tmem_st32(taddr, r);
-}
+constexpr int kBStages = 4;   // activation tiles (shared memory)
+constexpr int kRing = 6;      // per-thread packed-code prefetch depth, in steps
+constexpr int kDeqWarps = 8;  // 2 per tensor-memory lane quarter, each half of every step
+constexpr int kDeqThreads = kDeqWarps * 32;
+constexpr int kThreads = (2 + kDeqWarps) * 32;
+constexpr int kAccCols = kTok;                  // one accumulator [128 lanes x 256 tokens]
+constexpr int kAStageCols = kKs / 2;            // 64 bf16 inputs = 32 columns
+constexpr int kTmemCols = 512;                  // 256 + 4 x 32 used, power of two allocated
+constexpr int kBTile = kTok * kKs * 2;          // 32 KB
+constexpr size_t kCodeRing = (size_t)kRing * kDeqThreads * 16;
+constexpr size_t kScaleRing = (size_t)kRing * kDeqThreads * 4;
+constexpr size_t kSmemBytes = 1024 + (size_t)kBStages * kBTile + kCodeRing + kScaleRing + 256;
+static_assert(kAccCols + kStages * kAStageCols <= kTmemCols, "tensor memory budget");
+static_assert(64 * kTok * 4 <= kBStages * kBTile, "gate/up exchange fits in the activation ring");
 
 // (q - 8) * scale in bf16 for the pairs (q0,q4) (q1,q5) (q2,q6) (q3,q7) of one code word
 __device__ __forceinline__ void dequant4(uint32_t w, uint32_t scale2, uint32_t *out)
@@ -109,21 +74,16 @@ __device__ __forceinline__ int perm_pos(int f)
     return (f & ~7) + (i < 4 ? 2 * i : 2 * (i - 4) + 1);
 }
 
-template <int MODE, int DW>
-__global__ void __launch_bounds__((2 + DW) * 32, 1)
-    w4a16_tc_kernel(const __grid_constant__ CUtensorMap tmX, W4TcArgs a)
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_constant__ CUtensorMap tmX, W4TcArgs a)
 {
-    using Sh = W4TcShape<MODE, DW>;
-    constexpr int kDeqThreads = Sh::kDeqThreads;
-    constexpr int kRing = Sh::kRing;
-    constexpr int kBStages = Sh::kBStages;
-    constexpr bool GU = Sh::kGU;
+    constexpr bool GU = MODE == TC_GATEUP;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *btiles = smem;
-    uint8_t *code_ring = btiles + kBStages * Sh::kBTile;
-    uint8_t *scale_ring = code_ring + Sh::kCodeRing;
-    uint64_t *b_full = reinterpret_cast<uint64_t *>(scale_ring + Sh::kScaleRing);
+    uint8_t *code_ring = btiles + kBStages * kBTile;
+    uint8_t *scale_ring = code_ring + kCodeRing;
+    uint64_t *b_full = reinterpret_cast<uint64_t *>(scale_ring + kScaleRing);
     uint64_t *b_empty = b_full + kBStages;
     uint64_t *a_full = b_empty + kBStages;
     uint64_t *empty = a_full + kStages;
@@ -140,8 +100,11 @@ __global__ void __launch_bounds__((2 + DW) * 32, 1)
     if (r0 >= __ldg(a.ntp)) return;  // uniform over the CTA, before any barrier or allocation
     const int e = __ldg(a.expert_ids + blockIdx.y);
     if (e < 0 || e >= a.E) return;
-    const int n0 = blockIdx.x * 128;  // output features (gate/up) or output rows (down)
+    const int n0 = blockIdx.x * (GU ? 64 : 128);  // first output feature (gate/up) or row (down)
     const int K = a.K, NS = K / kKs;
+    // real rows of this block: the expert's slots come first, padding after
+    const int valid = __syncthreads_count(threadIdx.x < kTok && __ldg(a.sorted_ids + r0 + threadIdx.x) < a.n_slots);
+    const int n_mma = (valid + 15) & ~15;  // MMA N: multiple of 16 in [16, 256]
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kBStages; ++s) {
@@ -149,7 +112,7 @@ __global__ void __launch_bounds__((2 + DW) * 32, 1)
             tc::mbar_init(&b_empty[s], 1);
         }
         for (int s = 0; s < kStages; ++s) {
-            tc::mbar_init(&a_full[s], DW);
+            tc::mbar_init(&a_full[s], kDeqWarps);
             tc::mbar_init(&empty[s], 1);
         }
         tc::mbar_init(acc_full, 1);
@@ -157,7 +120,7 @@ __global__ void __launch_bounds__((2 + DW) * 32, 1)
         *abort_flag = 0;
         tc::fence_barrier_init();
     }
-    if (warp == 1) tc::tmem_alloc(tmem_slot, Sh::kTmemCols);
+    if (warp == 1) tc::tmem_alloc(tmem_slot, kTmemCols);
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
@@ -171,8 +134,8 @@ __global__ void __launch_bounds__((2 + DW) * 32, 1)
                 const int s = ks % kBStages;
                 if (ks >= kBStages && !tc::mbar_wait(&b_empty[s], ((ks / kBStages) & 1) ^ 1, abort_flag, a.status))
                     break;
-                tc::mbar_arrive_expect_tx(&b_full[s], Sh::kBTile);
-                tc::tma_load_2d(btiles + s * Sh::kBTile, &tmX, &b_full[s], ks * kKs, r0);
+                tc::mbar_arrive_expect_tx(&b_full[s], kBTile);
+                tc::tma_load_2d(btiles + s * kBTile, &tmX, &b_full[s], ks * kKs, r0);
                 issued = ks + 1;
             }
             for (int ks = issued - kBStages > 0 ? issued - kBStages : 0; ks < issued; ++ks)
@@ -180,31 +143,25 @@ __global__ void __launch_bounds__((2 + DW) * 32, 1)
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            constexpr uint32_t idesc = tc::idesc_f32(tc::kFmtBF16, tc::kFmtBF16, 128, kTok);
+            const uint32_t idesc = tc::idesc_f32(tc::kFmtBF16, tc::kFmtBF16, 128, n_mma);
             // lean issue path: stage bases precomputed, the first step peeled, then MMAs that always
             // accumulate (the dequantization warps keep this SM's issue slots busy)
-            const uint32_t a_base = tmem + Sh::kAccCols;
+            const uint32_t a_base = tmem + kAccCols;
             const uint64_t b_base = tc::smem_desc_sw128(btiles);
             for (int ks = 0; ks < NS; ++ks) {
                 const int s = ks % kStages, sb = ks % kBStages;
                 if (!tc::mbar_wait(&b_full[sb], (ks / kBStages) & 1, abort_flag, a.status)) break;
                 if (!tc::mbar_wait(&a_full[s], (ks / kStages) & 1, abort_flag, a.status)) break;
                 tc::fence_after_sync();
-                const uint64_t bdesc = b_base + (uint64_t)((sb * Sh::kBTile) >> 4);
-                const uint32_t astage = a_base + s * Sh::kAStageCols;
+                const uint64_t bdesc = b_base + (uint64_t)((sb * kBTile) >> 4);
+                const uint32_t astage = a_base + s * kAStageCols;
                 if (ks == 0) {
 #pragma unroll
-                    for (int kk = 0; kk < kKs / 16; ++kk) {
-                        const uint32_t acc = kk > 0 ? 1u : 0u;
-                        tc::mma_f16_ts(tmem, astage + kk * 8, bdesc + 2 * kk, idesc, acc);
-                        if (GU) tc::mma_f16_ts(tmem + kTok, astage + kKs / 2 + kk * 8, bdesc + 2 * kk, idesc, acc);
-                    }
+                    for (int kk = 0; kk < kKs / 16; ++kk)
+                        tc::mma_f16_ts(tmem, astage + kk * 8, bdesc + 2 * kk, idesc, kk > 0 ? 1u : 0u);
                 } else {
 #pragma unroll
-                    for (int kk = 0; kk < kKs / 16; ++kk) {
-                        tc::mma_f16_ts_acc(tmem, astage + kk * 8, bdesc + 2 * kk, idesc);
-                        if (GU) tc::mma_f16_ts_acc(tmem + kTok, astage + kKs / 2 + kk * 8, bdesc + 2 * kk, idesc);
-                    }
+                    for (int kk = 0; kk < kKs / 16; ++kk) tc::mma_f16_ts_acc(tmem, astage + kk * 8, bdesc + 2 * kk, idesc);
                 }
                 tc::mma_commit(&empty[s]);
                 tc::mma_commit(&b_empty[sb]);
@@ -215,98 +172,115 @@ __global__ void __launch_bounds__((2 + DW) * 32, 1)
         }
     } else {
         // ---- dequantization ----
-        const int dw = warp - 2, quarter = warp & 3, set = dw >> 2;
-        const int matrix = GU ? (set & 1) : 0;                   // gate/up: 0 gate, 1 up
-        const int kpart = GU ? (set >> 1) : set;                 // which words of each step
+        const int dw = warp - 2, quarter = warp & 3, half = dw >> 2;
         const int t = dw * 32 + lane;                            // ring slot owner
         const int row = quarter * 32 + lane;                     // tensor-memory lane = weight row
-        const int grow = e * a.rows_per_expert + (GU ? (matrix ? a.N : 0) + n0 + row : n0 + row);
-        const int32_t *wrow = a.wq + (size_t)grow * (K / 8) + kpart * Sh::kWords;
-        const uint16_t *srow = a.ws + (size_t)grow * (K / 32);
-        auto code_slot = [&](int slot) { return code_ring + ((size_t)slot * kDeqThreads + t) * Sh::kCodeBytes; };
+        const int grow = GU ? e * a.rows_per_expert + (row < 64 ? 0 : a.N) + n0 + (row & 63)
+                            : e * a.rows_per_expert + n0 + row;
+        const int32_t *wrow = a.wq + (size_t)grow * (K / 8) + half * 4;  // 4 words = 32 inputs
+        const uint16_t *srow = a.ws + (size_t)grow * (K / 32);  // 4-byte aligned: K / 32 is even
+        auto code_slot = [&](int slot) { return code_ring + ((size_t)slot * kDeqThreads + t) * 16; };
+        auto scale_slot = [&](int slot) { return scale_ring + ((size_t)slot * kDeqThreads + t) * 4; };
         auto issue = [&](int ks) {
             if (ks < NS) {
                 const int slot = ks % kRing;
-                cp_async_codes<Sh::kCodeBytes>(code_slot(slot), wrow + ks * 8);
-                cp_async4(scale_ring + ((size_t)slot * kDeqThreads + t) * 4, srow + ks * 2);
+                cp_async16_stream(code_slot(slot), wrow + ks * 8);
+                cp_async4_ca(scale_slot(slot), srow + ks * 2);  // both group scales of the step
             }
             cp_async_commit();
         };
 #pragma unroll
         for (int ks = 0; ks < kRing - 1; ++ks) issue(ks);
+        // The stores of step ks are waited for (tcgen05.wait::st) only after the dequantization of
+        // step ks + 1, so the tensor-memory write latency hides behind that work.
         bool ok = true;
+        int pending = -1;
         for (int ks = 0; ks < NS && ok; ++ks) {
             cp_async_wait<kRing - 2>();
             const int slot = ks % kRing;
-            uint32_t words[Sh::kWords];  // vector reads: a warp reads one contiguous span, no bank conflicts
-            if (Sh::kWords == 2) {
-                const uint2 v = *reinterpret_cast<const uint2 *>(code_slot(slot));
-                words[0] = v.x;
-                words[1 % Sh::kWords] = v.y;
-            } else {
-#pragma unroll
-                for (int j = 0; j < Sh::kWords; j += 4) {
-                    const uint4 v = reinterpret_cast<const uint4 *>(code_slot(slot))[j / 4];
-                    words[j] = v.x;
-                    words[(j + 1) % Sh::kWords] = v.y;
-                    words[(j + 2) % Sh::kWords] = v.z;
-                    words[(j + 3) % Sh::kWords] = v.w;
-                }
-            }
-            const uint32_t sc = *reinterpret_cast<const uint32_t *>(scale_ring + ((size_t)slot * kDeqThreads + t) * 4);
+            const uint4 c = *reinterpret_cast<const uint4 *>(code_slot(slot));  // a warp reads 512 contiguous bytes
+            const uint32_t sc = *reinterpret_cast<const uint32_t *>(scale_slot(slot));
+            const uint32_t s16 = half ? (sc >> 16) : (sc & 0xFFFFu);  // the group of this half-step
             issue(ks + kRing - 1);  // refills the slot read in step ks - 1
-            uint32_t pairs[4 * Sh::kWords];
-#pragma unroll
-            for (int j = 0; j < Sh::kWords; ++j) {
-                const int group = (kpart * Sh::kWords + j) / 4;  // 0 or 1 inside the 64-input step
-                const uint32_t s16 = group ? (sc >> 16) : (sc & 0xFFFFu);
-                dequant4(words[j], s16 * 0x10001u, pairs + 4 * j);
+            const uint32_t s2 = prmt(s16, s16, 0x1010u);
+            uint32_t pairs[16];
+            dequant4(c.x, s2, pairs + 0);
+            dequant4(c.y, s2, pairs + 4);
+            dequant4(c.z, s2, pairs + 8);
+            dequant4(c.w, s2, pairs + 12);
+            if (pending >= 0) {
+                tc::tmem_wait_st();
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&a_full[pending % kStages]);
+                pending = -1;
             }
             const int s = ks % kStages;
-            if (ks >= kStages)
-                ok = __all_sync(0xFFFFFFFFu, tc::mbar_wait(&empty[s], ((ks / kStages) & 1) ^ 1, abort_flag, a.status));
+            if (ks >= kStages) ok = tc::mbar_wait_warp(&empty[s], ((ks / kStages) & 1) ^ 1, abort_flag, a.status);
             if (!ok) break;
             tc::fence_after_sync();
-            const uint32_t col = Sh::kAccCols + s * Sh::kAStageCols + matrix * (kKs / 2) + kpart * 4 * Sh::kWords;
-            tmem_st_n<4 * Sh::kWords>(tmem + ((uint32_t)(quarter * 32) << 16) + col, pairs);
+            tc::tmem_st16(tmem + ((uint32_t)(quarter * 32) << 16) + kAccCols + s * kAStageCols + half * 16, pairs);
+            pending = ks;
+        }
+        if (pending >= 0) {
             tc::tmem_wait_st();
             tc::fence_before_sync();
             __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&a_full[s]);
+            if (lane == 0) tc::mbar_arrive(&a_full[pending % kStages]);
         }
         cp_async_wait<0>();
 
-        // ---- epilogue: tokens [set * 128 / kSets, +128 / kSets) of the tile ----
-        ok = ok && __all_sync(0xFFFFFFFFu, tc::mbar_wait(acc_full, 0, abort_flag, a.status));
-        if (ok) {
-            tc::fence_after_sync();
-            const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-            constexpr int kTokPerSet = kTok / Sh::kSets;
-            for (int c = 0; c < kTokPerSet / 32; ++c) {
-                const int tok0 = set * kTokPerSet + c * 32;
-                uint32_t g[32];
-                tc::tmem_ld32(lane_base + tok0, g);
-                if (GU) {
+        // ---- epilogue: tokens [128 half, 128 half + 128) of the tile, chunks of 32 ----
+        ok = ok && tc::mbar_wait_warp(acc_full, 0, abort_flag, a.status);
+        const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+        if (GU) {
+            // up values (lanes 64-127) go through shared memory (the activation ring is free once
+            // every MMA has completed) to the warps holding the matching gate values (lanes 0-63)
+            float *up_s = reinterpret_cast<float *>(btiles);  // [token][feature 0..63]
+            if (ok) tc::fence_after_sync();
+            if (ok && quarter >= 2) {
+                for (int c = 0; c < 4; ++c) {
+                    const int tok0 = half * 128 + c * 32;
+                    if (tok0 >= n_mma) break;
                     uint32_t u[32];
-                    tc::tmem_ld32(lane_base + kTok + tok0, u);
+                    tc::tmem_ld32(lane_base + tok0, u);
                     tc::tmem_wait_ld();
-                    const int f = n0 + row;
-                    uint16_t *hcol = a.h_out + perm_pos(f);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) up_s[(tok0 + j) * 64 + (row - 64)] = __uint_as_float(u[j]);
+                }
+            }
+            asm volatile("bar.sync 1, %0;" ::"n"(kDeqThreads) : "memory");
+            if (ok && quarter < 2) {
+                const int f = n0 + row;
+                uint16_t *hcol = a.h_out + perm_pos(f);
+                for (int c = 0; c < 4; ++c) {
+                    const int tok0 = half * 128 + c * 32;
+                    if (tok0 >= n_mma) break;
+                    uint32_t g[32];
+                    tc::tmem_ld32(lane_base + tok0, g);
+                    tc::tmem_wait_ld();
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
-                        const float hv = silu_f32(__uint_as_float(g[j])) * __uint_as_float(u[j]);
+                        const float hv = silu_f32(__uint_as_float(g[j])) * up_s[(tok0 + j) * 64 + row];
                         hcol[(size_t)(r0 + tok0 + j) * a.N] = f32_to_bf16(hv);
                     }
-                } else {
-                    tc::tmem_wait_ld();
-                    const int my_slot = __ldg(a.sorted_ids + r0 + tok0 + lane);
-                    const float my_w = (my_slot < a.n_slots) ? __ldg(a.topk_w + my_slot) : 0.f;
+                }
+            }
+        } else if (ok) {
+            tc::fence_after_sync();
+            for (int c = 0; c < 4; ++c) {
+                const int tok0 = half * 128 + c * 32;
+                if (tok0 >= n_mma) break;
+                uint32_t y[32];
+                tc::tmem_ld32(lane_base + tok0, y);
+                tc::tmem_wait_ld();
+                const int my_slot = __ldg(a.sorted_ids + r0 + tok0 + lane);
+                const float my_w = (my_slot < a.n_slots) ? __ldg(a.topk_w + my_slot) : 0.f;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int slot = __shfl_sync(0xFFFFFFFFu, my_slot, j);
-                        const float wt = __shfl_sync(0xFFFFFFFFu, my_w, j);
-                        if (slot < a.n_slots) a.ys[(size_t)slot * a.N + n0 + row] = wt * __uint_as_float(g[j]);
-                    }
+                for (int j = 0; j < 32; ++j) {
+                    const int slot = __shfl_sync(0xFFFFFFFFu, my_slot, j);
+                    const float wt = __shfl_sync(0xFFFFFFFFu, my_w, j);
+                    if (slot < a.n_slots) a.ys[(size_t)slot * a.N + n0 + row] = wt * __uint_as_float(y[j]);
                 }
             }
         }
@@ -314,7 +288,7 @@ __global__ void __launch_bounds__((2 + DW) * 32, 1)
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
-    if (warp == 1) tc::tmem_dealloc(tmem, Sh::kTmemCols);
+    if (warp == 1) tc::tmem_dealloc(tmem, kTmemCols);
 }
 
 // Gather of bf16 activation rows into aligned order with the pair permutation inside every
@@ -345,20 +319,19 @@ __global__ void __launch_bounds__(256) gather_bf16_perm_kernel(const uint16_t *_
     }
 }
 
-template <int MODE, int DW>
+template <int MODE>
 int launch_mode(const W4TcArgs &a, const CUtensorMap &tm, int grid_x, int grid_y, cudaStream_t s)
 {
-    using Sh = W4TcShape<MODE, DW>;
     static bool attr = false;
     if (!attr) {
-        const cudaError_t e = cudaFuncSetAttribute(w4a16_tc_kernel<MODE, DW>,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Sh::kSmemBytes);
+        const cudaError_t e =
+            cudaFuncSetAttribute(w4a16_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
         if (e != cudaSuccess)
             return set_error(MOEQ_ERR_CUDA, "tcgen05 W4A16 GEMM: shared-memory attribute: %s", cudaGetErrorString(e));
         attr = true;
     }
     if (grid_x <= 0 || grid_y <= 0) return MOEQ_OK;
-    w4a16_tc_kernel<MODE, DW><<<dim3(grid_x, grid_y), Sh::kThreads, Sh::kSmemBytes, s>>>(tm, a);
+    w4a16_tc_kernel<MODE><<<dim3(grid_x, grid_y), kThreads, kSmemBytes, s>>>(tm, a);
     return MOEQ_OK;
 }
 
@@ -369,9 +342,8 @@ int launch_w4a16_tc(const W4TcArgs &a, int mode, const uint16_t *act, int max_bl
     CUtensorMap tm;
     const int rc = make_tmap_2d(&tm, act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.M, (uint64_t)a.K, kTok, kKs);
     if (rc) return rc;
-    // gate/up: 16 dequantization warps; down (shorter K, two CTAs per SM): 8
-    if (mode == TC_GATEUP) return launch_mode<TC_GATEUP, 16>(a, tm, a.N / 128, max_blocks, s);
-    return launch_mode<TC_DOWN, 8>(a, tm, a.N / 128, max_blocks, s);
+    if (mode == TC_GATEUP) return launch_mode<TC_GATEUP>(a, tm, a.N / 64, max_blocks, s);
+    return launch_mode<TC_DOWN>(a, tm, a.N / 128, max_blocks, s);
 }
 
 void launch_gather_bf16_perm(const uint16_t *x, int H, int k, const int32_t *sorted_ids, const int32_t *ntp,
