@@ -231,11 +231,13 @@ constexpr uint32_t kFmtBF16 = 1;  // kind::f16
 
 }  // namespace tc
 
-// Host: a 2-D tensor map over a row-major [rows, cols] matrix of 1- or 2-byte elements, tile box
-// [box_rows, box_cols] with the 128-byte swizzle (box_cols * element size must be 128). Rows past
-// the end read as zero.
+// Host: a 2-D tensor map over a row-major [rows, cols] matrix, tile box [box_rows, box_cols]. With
+// swizzle128 the box lands in shared memory in the 128-byte swizzled K-major layout the MMA
+// descriptors expect (box_cols * element size must then be 128); without it the box is stored
+// row-major and densely packed (box_cols * element size a multiple of 16). Rows past the end read
+// as zero.
 int make_tmap_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype, int elem_bytes, uint64_t rows,
-                 uint64_t cols, uint32_t box_rows, uint32_t box_cols);
+                 uint64_t cols, uint32_t box_rows, uint32_t box_cols, bool swizzle128 = true);
 
 // Host: device address of the library's kernel status word on the current device.
 int *device_status_ptr();

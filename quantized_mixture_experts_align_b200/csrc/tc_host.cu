@@ -19,7 +19,7 @@ int *g_status_addr[64] = {};
 }  // namespace
 
 int make_tmap_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype, int elem_bytes, uint64_t rows,
-                 uint64_t cols, uint32_t box_rows, uint32_t box_cols)
+                 uint64_t cols, uint32_t box_rows, uint32_t box_cols, bool swizzle128)
 {
     {
         std::lock_guard<std::mutex> g(g_mu);
@@ -34,12 +34,16 @@ int make_tmap_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype, 
     }
     if (reinterpret_cast<uintptr_t>(base) % 16 || (cols * elem_bytes) % 16)
         return set_error(MOEQ_ERR_UNSUPPORTED, "tensor map: base and row pitch must be 16-byte aligned");
+    if ((box_cols * (uint64_t)elem_bytes) % 16 || (swizzle128 && box_cols * (uint64_t)elem_bytes != 128))
+        return set_error(MOEQ_ERR_UNSUPPORTED, "tensor map: box inner extent %u x %d bytes not supported", box_cols,
+                         elem_bytes);
     const cuuint64_t dims[2] = {cols, rows};
     const cuuint64_t strides[1] = {cols * (uint64_t)elem_bytes};
     const cuuint32_t box[2] = {box_cols, box_rows};
     const cuuint32_t estride[2] = {1, 1};
     const CUresult r = g_encode(map, dtype, 2, const_cast<void *>(base), dims, strides, box, estride,
-                                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return set_error(MOEQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
     return MOEQ_OK;

@@ -22,10 +22,13 @@
 //
 // CTA = one 256-row activation block of one expert x (gate/up: 64 features, gate rows in tensor
 // lanes 0-63 and the matching up rows in lanes 64-127; down: 128 output rows):
-//   warp 0      TMA producer of the activation tiles [256 tokens x 64 inputs] (4 stages, own
-//               barriers);
+//   warp 0      TMA producer of the activation tiles [256 tokens x 64 inputs] (4 stages); a
+//               tile's bytes complete on the same "stage ready" barrier the dequantization warps
+//               arrive on, and one commit per step frees both the weight stage and the tile;
 //   warp 1      tensor-memory allocation; lane 0 issues 4 MMAs (K = 16) per 64-input step into
-//               the one accumulator and commits;
+//               the one accumulator and commits. This single thread is the pipeline's critical
+//               path on sm_100a (an MMA issue costs ~50-65 cycles, a barrier wait ~47 even when
+//               the phase is complete), so it waits on one barrier and commits once per step;
 //   warps 2-9   dequantization: a thread owns one weight row (tensor lane) and half of each
 //               64-input step, prefetches its packed codes and scale through a private 6-deep
 //               cp.async ring, and writes the dequantized half-step to one of 4 tensor-memory
@@ -55,6 +58,7 @@ constexpr size_t kCodeRing = (size_t)kRing * kDeqThreads * 16;
 constexpr size_t kScaleRing = (size_t)kRing * kDeqThreads * 4;
 constexpr size_t kSmemBytes = 1024 + (size_t)kBStages * kBTile + kCodeRing + kScaleRing + 256;
 static_assert(kAccCols + kStages * kAStageCols <= kTmemCols, "tensor memory budget");
+static_assert(kBStages == kStages, "one stage-free barrier serves the activation and weight stages");
 static_assert(64 * kTok * 4 <= kBStages * kBTile, "gate/up exchange fits in the activation ring");
 
 // (q - 8) * scale in bf16 for the pairs (q0,q4) (q1,q5) (q2,q6) (q3,q7) of one code word
@@ -83,9 +87,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
     uint8_t *btiles = smem;
     uint8_t *code_ring = btiles + kBStages * kBTile;
     uint8_t *scale_ring = code_ring + kCodeRing;
-    uint64_t *b_full = reinterpret_cast<uint64_t *>(scale_ring + kScaleRing);
-    uint64_t *b_empty = b_full + kBStages;
-    uint64_t *a_full = b_empty + kBStages;
+    uint64_t *a_full = reinterpret_cast<uint64_t *>(scale_ring + kScaleRing);
     uint64_t *empty = a_full + kStages;
     uint64_t *acc_full = empty + kStages;
     uint64_t *mma_done = acc_full + 1;
@@ -107,12 +109,8 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
     const int n_mma = (valid + 15) & ~15;  // MMA N: multiple of 16 in [16, 256]
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kBStages; ++s) {
-            tc::mbar_init(&b_full[s], 1);
-            tc::mbar_init(&b_empty[s], 1);
-        }
         for (int s = 0; s < kStages; ++s) {
-            tc::mbar_init(&a_full[s], kDeqWarps);
+            tc::mbar_init(&a_full[s], kDeqWarps + 1);
             tc::mbar_init(&empty[s], 1);
         }
         tc::mbar_init(acc_full, 1);
@@ -132,14 +130,16 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
             int issued = 0;
             for (int ks = 0; ks < NS; ++ks) {
                 const int s = ks % kBStages;
-                if (ks >= kBStages && !tc::mbar_wait(&b_empty[s], ((ks / kBStages) & 1) ^ 1, abort_flag, a.status))
+                if (ks >= kBStages && !tc::mbar_wait(&empty[s], ((ks / kBStages) & 1) ^ 1, abort_flag, a.status))
                     break;
-                tc::mbar_arrive_expect_tx(&b_full[s], kBTile);
-                tc::tma_load_2d(btiles + s * kBTile, &tmX, &b_full[s], ks * kKs, r0);
+                // the tile's bytes complete on the stage's a_full barrier (dequantization warps + this
+                // arrival): the MMA thread waits on one barrier per step
+                tc::mbar_arrive_expect_tx(&a_full[s], kBTile);
+                tc::tma_load_2d(btiles + s * kBTile, &tmX, &a_full[s], ks * kKs, r0);
                 issued = ks + 1;
             }
             for (int ks = issued - kBStages > 0 ? issued - kBStages : 0; ks < issued; ++ks)
-                tc::mbar_drain(&b_full[ks % kBStages], (ks / kBStages) & 1, a.status);
+                tc::mbar_drain(&a_full[ks % kBStages], (ks / kBStages) & 1, a.status);
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -149,8 +149,9 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
             const uint32_t a_base = tmem + kAccCols;
             const uint64_t b_base = tc::smem_desc_sw128(btiles);
             for (int ks = 0; ks < NS; ++ks) {
-                const int s = ks % kStages, sb = ks % kBStages;
-                if (!tc::mbar_wait(&b_full[sb], (ks / kBStages) & 1, abort_flag, a.status)) break;
+                const int s = ks % kStages, sb = ks % kBStages;  // equal: one stage index
+                // one wait per step: a_full completes when the weight stage and the activation tile
+                // are both in place
                 if (!tc::mbar_wait(&a_full[s], (ks / kStages) & 1, abort_flag, a.status)) break;
                 tc::fence_after_sync();
                 const uint64_t bdesc = b_base + (uint64_t)((sb * kBTile) >> 4);
@@ -163,8 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
 #pragma unroll
                     for (int kk = 0; kk < kKs / 16; ++kk) tc::mma_f16_ts_acc(tmem, astage + kk * 8, bdesc + 2 * kk, idesc);
                 }
-                tc::mma_commit(&empty[s]);
-                tc::mma_commit(&b_empty[sb]);
+                tc::mma_commit(&empty[s]);  // frees the weight stage and the activation tile
             }
             tc::mma_commit(acc_full);
             tc::mma_commit(mma_done);
@@ -193,6 +193,13 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
         for (int ks = 0; ks < kRing - 1; ++ks) issue(ks);
         // The stores of step ks are waited for (tcgen05.wait::st) only after the dequantization of
         // step ks + 1, so the tensor-memory write latency hides behind that work.
+        auto stage_ready = [&](int j) -> bool {
+            tc::tmem_wait_st();
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&a_full[j % kStages]);
+            return true;
+        };
         bool ok = true;
         int pending = -1;
         for (int ks = 0; ks < NS && ok; ++ks) {
@@ -209,11 +216,9 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
             dequant4(c.z, s2, pairs + 8);
             dequant4(c.w, s2, pairs + 12);
             if (pending >= 0) {
-                tc::tmem_wait_st();
-                tc::fence_before_sync();
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&a_full[pending % kStages]);
+                ok = stage_ready(pending);
                 pending = -1;
+                if (!ok) break;
             }
             const int s = ks % kStages;
             if (ks >= kStages) ok = tc::mbar_wait_warp(&empty[s], ((ks / kStages) & 1) ^ 1, abort_flag, a.status);
@@ -222,12 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
             tc::tmem_st16(tmem + ((uint32_t)(quarter * 32) << 16) + kAccCols + s * kAStageCols + half * 16, pairs);
             pending = ks;
         }
-        if (pending >= 0) {
-            tc::tmem_wait_st();
-            tc::fence_before_sync();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&a_full[pending % kStages]);
-        }
+        if (pending >= 0) ok = stage_ready(pending);
         cp_async_wait<0>();
 
         // ---- epilogue: tokens [128 half, 128 half + 128) of the tile, chunks of 32 ----
