@@ -22,16 +22,19 @@
 //
 // CTA = one 256-row activation block of one expert x (gate/up: 64 features, gate rows in tensor
 // lanes 0-63 and the matching up rows in lanes 64-127; down: 128 output rows):
-//   warp 0      TMA producer of the activation tiles [256 tokens x 64 inputs] (4 stages); a
+//   warp 0      TMA producer of the activation tiles [256 tokens x 128 inputs] (3 stages, two
+//               128-byte-swizzled halves of 64 inputs each); a
 //               tile's bytes complete on the same "stage ready" barrier the dequantization warps
 //               arrive on, and one commit per step frees both the weight stage and the tile;
-//   warp 1      tensor-memory allocation; lane 0 issues 4 MMAs (K = 16) per 64-input step into
-//               the one accumulator and commits. This single thread is the pipeline's critical
-//               path on sm_100a (an MMA issue costs ~50-65 cycles, a barrier wait ~47 even when
-//               the phase is complete), so it waits on one barrier and commits once per step;
+//   warp 1      tensor-memory allocation; lane 0 issues 8 MMAs (K = 16) per 128-input step into
+//               the one accumulator and commits. On sm_100a a pipeline step costs several hundred
+//               cycles of synchronization whatever work it carries (an MMA issue ~50-65 cycles, a
+//               barrier wait ~47 even when the phase is complete, more under load), so the steps
+//               are long and the MMA thread waits on one barrier and commits once per step;
 //   warps 2-9   dequantization: a thread owns one weight row (tensor lane) and half of each
-//               64-input step, prefetches its packed codes and scale through a private 6-deep
-//               cp.async ring, and writes the dequantized half-step to one of 4 tensor-memory
+//               128-input step (32 bytes of codes, 2 group scales), prefetches them through a
+//               private 3-deep cp.async ring, and writes the dequantized half-step to one of 3
+//               tensor-memory
 //               stages; then the epilogue: gate/up passes the up values through shared memory
 //               to the warps holding the gate values, which write h = bf16(silu(g) * u) in the
 //               permuted order; down writes the routing-weighted f32 slot rows.
@@ -43,18 +46,19 @@ namespace moeq {
 namespace {
 
 constexpr int kTok = 256;     // tokens per tile = aligned block size
-constexpr int kKs = 64;       // inputs per pipeline step
-constexpr int kStages = 4;    // dequantized weight stages (tensor memory)
-constexpr int kBStages = 4;   // activation tiles (shared memory)
-constexpr int kRing = 6;      // per-thread packed-code prefetch depth, in steps
+constexpr int kKs = 128;      // inputs per pipeline step (8 MMAs per barrier round trip)
+constexpr int kStages = 3;    // dequantized weight stages (tensor memory)
+constexpr int kBStages = 3;   // activation tiles (shared memory)
+constexpr int kRing = 3;      // per-thread packed-code prefetch depth, in steps
 constexpr int kDeqWarps = 8;  // 2 per tensor-memory lane quarter, each half of every step
 constexpr int kDeqThreads = kDeqWarps * 32;
 constexpr int kThreads = (2 + kDeqWarps) * 32;
 constexpr int kAccCols = kTok;                  // one accumulator [128 lanes x 256 tokens]
-constexpr int kAStageCols = kKs / 2;            // 64 bf16 inputs = 32 columns
-constexpr int kTmemCols = 512;                  // 256 + 4 x 32 used, power of two allocated
-constexpr int kBTile = kTok * kKs * 2;          // 32 KB
-constexpr size_t kCodeRing = (size_t)kRing * kDeqThreads * 16;
+constexpr int kAStageCols = kKs / 2;            // 128 bf16 inputs = 64 columns
+constexpr int kTmemCols = 512;                  // 256 + 3 x 64 used, power of two allocated
+constexpr int kBTile = kTok * kKs * 2;          // 64 KB: two 128-byte-swizzled halves of 64 inputs
+constexpr int kBHalf = kBTile / 2;
+constexpr size_t kCodeRing = (size_t)kRing * kDeqThreads * 32;
 constexpr size_t kScaleRing = (size_t)kRing * kDeqThreads * 4;
 constexpr size_t kSmemBytes = 1024 + (size_t)kBStages * kBTile + kCodeRing + kScaleRing + 256;
 static_assert(kAccCols + kStages * kAStageCols <= kTmemCols, "tensor memory budget");
@@ -136,6 +140,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
                 // arrival): the MMA thread waits on one barrier per step
                 tc::mbar_arrive_expect_tx(&a_full[s], kBTile);
                 tc::tma_load_2d(btiles + s * kBTile, &tmX, &a_full[s], ks * kKs, r0);
+                tc::tma_load_2d(btiles + s * kBTile + kBHalf, &tmX, &a_full[s], ks * kKs + kKs / 2, r0);
                 issued = ks + 1;
             }
             for (int ks = issued - kBStages > 0 ? issued - kBStages : 0; ks < issued; ++ks)
@@ -159,10 +164,12 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
                 if (ks == 0) {
 #pragma unroll
                     for (int kk = 0; kk < kKs / 16; ++kk)
-                        tc::mma_f16_ts(tmem, astage + kk * 8, bdesc + 2 * kk, idesc, kk > 0 ? 1u : 0u);
+                        tc::mma_f16_ts(tmem, astage + kk * 8, bdesc + (kk >> 2) * (kBHalf >> 4) + 2 * (kk & 3), idesc,
+                                       kk > 0 ? 1u : 0u);
                 } else {
 #pragma unroll
-                    for (int kk = 0; kk < kKs / 16; ++kk) tc::mma_f16_ts_acc(tmem, astage + kk * 8, bdesc + 2 * kk, idesc);
+                    for (int kk = 0; kk < kKs / 16; ++kk)
+                        tc::mma_f16_ts_acc(tmem, astage + kk * 8, bdesc + (kk >> 2) * (kBHalf >> 4) + 2 * (kk & 3), idesc);
                 }
                 tc::mma_commit(&empty[s]);  // frees the weight stage and the activation tile
             }
@@ -177,15 +184,17 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
         const int row = quarter * 32 + lane;                     // tensor-memory lane = weight row
         const int grow = GU ? e * a.rows_per_expert + (row < 64 ? 0 : a.N) + n0 + (row & 63)
                             : e * a.rows_per_expert + n0 + row;
-        const int32_t *wrow = a.wq + (size_t)grow * (K / 8) + half * 4;  // 4 words = 32 inputs
-        const uint16_t *srow = a.ws + (size_t)grow * (K / 32);  // 4-byte aligned: K / 32 is even
-        auto code_slot = [&](int slot) { return code_ring + ((size_t)slot * kDeqThreads + t) * 16; };
+        const int32_t *wrow = a.wq + (size_t)grow * (K / 8) + half * 8;  // 8 words = 64 inputs
+        // the two group scales of this thread's 64 inputs: 4-byte aligned (rows are K/16 bytes apart)
+        const uint16_t *srow = a.ws + (size_t)grow * (K / 32) + half * 2;
+        auto code_slot = [&](int slot) { return code_ring + ((size_t)slot * kDeqThreads + t) * 32; };
         auto scale_slot = [&](int slot) { return scale_ring + ((size_t)slot * kDeqThreads + t) * 4; };
         auto issue = [&](int ks) {
             if (ks < NS) {
                 const int slot = ks % kRing;
-                cp_async16_stream(code_slot(slot), wrow + ks * 8);
-                cp_async4_ca(scale_slot(slot), srow + ks * 2);  // both group scales of the step
+                cp_async16_stream(code_slot(slot), wrow + ks * 16);
+                cp_async16_stream(code_slot(slot) + 16, wrow + ks * 16 + 4);
+                cp_async4_ca(scale_slot(slot), srow + ks * 4);
             }
             cp_async_commit();
         };
@@ -205,16 +214,20 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
         for (int ks = 0; ks < NS && ok; ++ks) {
             cp_async_wait<kRing - 2>();
             const int slot = ks % kRing;
-            const uint4 c = *reinterpret_cast<const uint4 *>(code_slot(slot));  // a warp reads 512 contiguous bytes
+            const uint4 c0 = *reinterpret_cast<const uint4 *>(code_slot(slot));
+            const uint4 c1 = *reinterpret_cast<const uint4 *>(code_slot(slot) + 16);
             const uint32_t sc = *reinterpret_cast<const uint32_t *>(scale_slot(slot));
-            const uint32_t s16 = half ? (sc >> 16) : (sc & 0xFFFFu);  // the group of this half-step
             issue(ks + kRing - 1);  // refills the slot read in step ks - 1
-            const uint32_t s2 = prmt(s16, s16, 0x1010u);
-            uint32_t pairs[16];
-            dequant4(c.x, s2, pairs + 0);
-            dequant4(c.y, s2, pairs + 4);
-            dequant4(c.z, s2, pairs + 8);
-            dequant4(c.w, s2, pairs + 12);
+            const uint32_t sa = prmt(sc, sc, 0x1010u), sb = prmt(sc, sc, 0x3232u);  // groups 0 and 1
+            uint32_t pairs[32];
+            dequant4(c0.x, sa, pairs + 0);
+            dequant4(c0.y, sa, pairs + 4);
+            dequant4(c0.z, sa, pairs + 8);
+            dequant4(c0.w, sa, pairs + 12);
+            dequant4(c1.x, sb, pairs + 16);
+            dequant4(c1.y, sb, pairs + 20);
+            dequant4(c1.z, sb, pairs + 24);
+            dequant4(c1.w, sb, pairs + 28);
             if (pending >= 0) {
                 ok = stage_ready(pending);
                 pending = -1;
@@ -224,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
             if (ks >= kStages) ok = tc::mbar_wait_warp(&empty[s], ((ks / kStages) & 1) ^ 1, abort_flag, a.status);
             if (!ok) break;
             tc::fence_after_sync();
-            tc::tmem_st16(tmem + ((uint32_t)(quarter * 32) << 16) + kAccCols + s * kAStageCols + half * 16, pairs);
+            tc::tmem_st32(tmem + ((uint32_t)(quarter * 32) << 16) + kAccCols + s * kAStageCols + half * 32, pairs);
             pending = ks;
         }
         if (pending >= 0) ok = stage_ready(pending);
@@ -340,7 +353,7 @@ int launch_mode(const W4TcArgs &a, const CUtensorMap &tm, int grid_x, int grid_y
 int launch_w4a16_tc(const W4TcArgs &a, int mode, const uint16_t *act, int max_blocks, cudaStream_t s)
 {
     CUtensorMap tm;
-    const int rc = make_tmap_2d(&tm, act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.M, (uint64_t)a.K, kTok, kKs);
+    const int rc = make_tmap_2d(&tm, act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.M, (uint64_t)a.K, kTok, kKs / 2);
     if (rc) return rc;
     if (mode == TC_GATEUP) return launch_mode<TC_GATEUP>(a, tm, a.N / 64, max_blocks, s);
     return launch_mode<TC_DOWN>(a, tm, a.N / 128, max_blocks, s);
