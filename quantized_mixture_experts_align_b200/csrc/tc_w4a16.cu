@@ -31,9 +31,9 @@
 //               cycles of synchronization whatever work it carries (an MMA issue ~50-65 cycles, a
 //               barrier wait ~47 even when the phase is complete, more under load), so the steps
 //               are long and the MMA thread waits on one barrier and commits once per step;
-//   warps 2-9   dequantization: a thread owns one weight row (tensor lane) and half of each
-//               128-input step (32 bytes of codes, 2 group scales), prefetches them through a
-//               private 3-deep cp.async ring, and writes the dequantized half-step to one of 3
+//   warps 2-17  dequantization: a thread owns one weight row (tensor lane) and a 32-input slice
+//               of each 128-input step (16 bytes of codes, 1 group scale), prefetches them through
+//               a private 3-deep cp.async ring, and writes the dequantized slice to one of 3
 //               tensor-memory
 //               stages; then the epilogue: gate/up passes the up values through shared memory
 //               to the warps holding the gate values, which write h = bf16(silu(g) * u) in the
@@ -50,15 +50,18 @@ constexpr int kKs = 128;      // inputs per pipeline step (8 MMAs per barrier ro
 constexpr int kStages = 3;    // dequantized weight stages (tensor memory)
 constexpr int kBStages = 3;   // activation tiles (shared memory)
 constexpr int kRing = 3;      // per-thread packed-code prefetch depth, in steps
-constexpr int kDeqWarps = 8;  // 2 per tensor-memory lane quarter, each half of every step
+constexpr int kDeqWarps = 16;  // 4 per tensor-memory lane quarter, each a quarter of every step
 constexpr int kDeqThreads = kDeqWarps * 32;
+constexpr int kSplit = kDeqWarps / 4;           // K slices of a step (one per warp of a lane quarter)
+constexpr int kThrK = kKs / kSplit;             // 32 inputs per thread per step: 4 code words, 1 group
+static_assert(kThrK == 32, "one scale group per thread and step");
 constexpr int kThreads = (2 + kDeqWarps) * 32;
 constexpr int kAccCols = kTok;                  // one accumulator [128 lanes x 256 tokens]
 constexpr int kAStageCols = kKs / 2;            // 128 bf16 inputs = 64 columns
 constexpr int kTmemCols = 512;                  // 256 + 3 x 64 used, power of two allocated
 constexpr int kBTile = kTok * kKs * 2;          // 64 KB: two 128-byte-swizzled halves of 64 inputs
 constexpr int kBHalf = kBTile / 2;
-constexpr size_t kCodeRing = (size_t)kRing * kDeqThreads * 32;
+constexpr size_t kCodeRing = (size_t)kRing * kDeqThreads * 16;
 constexpr size_t kScaleRing = (size_t)kRing * kDeqThreads * 4;
 constexpr size_t kSmemBytes = 1024 + (size_t)kBStages * kBTile + kCodeRing + kScaleRing + 256;
 static_assert(kAccCols + kStages * kAStageCols <= kTmemCols, "tensor memory budget");
@@ -179,22 +182,22 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
         }
     } else {
         // ---- dequantization ----
-        const int dw = warp - 2, quarter = warp & 3, half = dw >> 2;
+        const int dw = warp - 2, quarter = warp & 3, kq = dw >> 2;  // lane quarter, K slice
         const int t = dw * 32 + lane;                            // ring slot owner
         const int row = quarter * 32 + lane;                     // tensor-memory lane = weight row
         const int grow = GU ? e * a.rows_per_expert + (row < 64 ? 0 : a.N) + n0 + (row & 63)
                             : e * a.rows_per_expert + n0 + row;
-        const int32_t *wrow = a.wq + (size_t)grow * (K / 8) + half * 8;  // 8 words = 64 inputs
-        // the two group scales of this thread's 64 inputs: 4-byte aligned (rows are K/16 bytes apart)
-        const uint16_t *srow = a.ws + (size_t)grow * (K / 32) + half * 2;
-        auto code_slot = [&](int slot) { return code_ring + ((size_t)slot * kDeqThreads + t) * 32; };
+        const int32_t *wrow = a.wq + (size_t)grow * (K / 8) + kq * 4;  // 4 words = 32 inputs
+        // the group scale of this thread's 32 inputs comes with its neighbour's in one aligned
+        // 4-byte copy (rows are K/16 bytes apart, K a multiple of 128)
+        const uint16_t *srow = a.ws + (size_t)grow * (K / 32) + (kq & ~1);
+        auto code_slot = [&](int slot) { return code_ring + ((size_t)slot * kDeqThreads + t) * 16; };
         auto scale_slot = [&](int slot) { return scale_ring + ((size_t)slot * kDeqThreads + t) * 4; };
         auto issue = [&](int ks) {
             if (ks < NS) {
                 const int slot = ks % kRing;
-                cp_async16_stream(code_slot(slot), wrow + ks * 16);
-                cp_async16_stream(code_slot(slot) + 16, wrow + ks * 16 + 4);
-                cp_async4_ca(scale_slot(slot), srow + ks * 4);
+                cp_async16_stream(code_slot(slot), wrow + ks * (kKs / 8));
+                cp_async4_ca(scale_slot(slot), srow + ks * (kKs / 32));
             }
             cp_async_commit();
         };
@@ -214,20 +217,15 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
         for (int ks = 0; ks < NS && ok; ++ks) {
             cp_async_wait<kRing - 2>();
             const int slot = ks % kRing;
-            const uint4 c0 = *reinterpret_cast<const uint4 *>(code_slot(slot));
-            const uint4 c1 = *reinterpret_cast<const uint4 *>(code_slot(slot) + 16);
+            const uint4 c = *reinterpret_cast<const uint4 *>(code_slot(slot));  // a warp reads 512 contiguous bytes
             const uint32_t sc = *reinterpret_cast<const uint32_t *>(scale_slot(slot));
             issue(ks + kRing - 1);  // refills the slot read in step ks - 1
-            const uint32_t sa = prmt(sc, sc, 0x1010u), sb = prmt(sc, sc, 0x3232u);  // groups 0 and 1
-            uint32_t pairs[32];
-            dequant4(c0.x, sa, pairs + 0);
-            dequant4(c0.y, sa, pairs + 4);
-            dequant4(c0.z, sa, pairs + 8);
-            dequant4(c0.w, sa, pairs + 12);
-            dequant4(c1.x, sb, pairs + 16);
-            dequant4(c1.y, sb, pairs + 20);
-            dequant4(c1.z, sb, pairs + 24);
-            dequant4(c1.w, sb, pairs + 28);
+            const uint32_t s2 = prmt(sc, sc, (kq & 1) ? 0x3232u : 0x1010u);  // this slice's group, twice
+            uint32_t pairs[16];
+            dequant4(c.x, s2, pairs + 0);
+            dequant4(c.y, s2, pairs + 4);
+            dequant4(c.z, s2, pairs + 8);
+            dequant4(c.w, s2, pairs + 12);
             if (pending >= 0) {
                 ok = stage_ready(pending);
                 pending = -1;
@@ -237,13 +235,13 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
             if (ks >= kStages) ok = tc::mbar_wait_warp(&empty[s], ((ks / kStages) & 1) ^ 1, abort_flag, a.status);
             if (!ok) break;
             tc::fence_after_sync();
-            tc::tmem_st32(tmem + ((uint32_t)(quarter * 32) << 16) + kAccCols + s * kAStageCols + half * 32, pairs);
+            tc::tmem_st16(tmem + ((uint32_t)(quarter * 32) << 16) + kAccCols + s * kAStageCols + kq * (kThrK / 2), pairs);
             pending = ks;
         }
         if (pending >= 0) ok = stage_ready(pending);
         cp_async_wait<0>();
 
-        // ---- epilogue: tokens [128 half, 128 half + 128) of the tile, chunks of 32 ----
+        // ---- epilogue: tokens [64 kq, 64 kq + 64) of the tile, chunks of 32 ----
         ok = ok && tc::mbar_wait_warp(acc_full, 0, abort_flag, a.status);
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
         if (GU) {
@@ -252,8 +250,8 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
             float *up_s = reinterpret_cast<float *>(btiles);  // [token][feature 0..63]
             if (ok) tc::fence_after_sync();
             if (ok && quarter >= 2) {
-                for (int c = 0; c < 4; ++c) {
-                    const int tok0 = half * 128 + c * 32;
+                for (int c = 0; c < kTok / kSplit / 32; ++c) {
+                    const int tok0 = kq * (kTok / kSplit) + c * 32;
                     if (tok0 >= n_mma) break;
                     uint32_t u[32];
                     tc::tmem_ld32(lane_base + tok0, u);
@@ -266,8 +264,8 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
             if (ok && quarter < 2) {
                 const int f = n0 + row;
                 uint16_t *hcol = a.h_out + perm_pos(f);
-                for (int c = 0; c < 4; ++c) {
-                    const int tok0 = half * 128 + c * 32;
+                for (int c = 0; c < kTok / kSplit / 32; ++c) {
+                    const int tok0 = kq * (kTok / kSplit) + c * 32;
                     if (tok0 >= n_mma) break;
                     uint32_t g[32];
                     tc::tmem_ld32(lane_base + tok0, g);
@@ -281,8 +279,8 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
             }
         } else if (ok) {
             tc::fence_after_sync();
-            for (int c = 0; c < 4; ++c) {
-                const int tok0 = half * 128 + c * 32;
+            for (int c = 0; c < kTok / kSplit / 32; ++c) {
+                const int tok0 = kq * (kTok / kSplit) + c * 32;
                 if (tok0 >= n_mma) break;
                 uint32_t y[32];
                 tc::tmem_ld32(lane_base + tok0, y);
