@@ -8,15 +8,16 @@
 // acc += As * Bs * partial, with two partial buffers so the MMAs of block kb+1 run while block kb
 // is promoted.
 //
-// CTA = one 128 x BN output tile, 10 warps:
+// CTA = one 128 x BN output tile, 18 warps:
 //   warp 0      TMA producer: A [128 x 128 B] and B [BN x 128 B] tiles per K block, 128-byte
 //               swizzle, into a 4-stage shared-memory ring (mbarrier transaction counts);
 //   warp 1      allocates tensor memory; lane 0 issues 4 tcgen05.mma (K = 32 each) per K block
 //               into partial buffer kb % 2 and commits to the stage's "empty" and the buffer's
 //               "full" barriers;
-//   warps 2-9   promotion and epilogue: warp w reads tensor-memory lanes 32 (w % 4) .. +31
-//               (= tile rows) and one half of the columns, keeps the running f32 sums in
-//               registers, and finally writes bf16 C.
+//   warps 2-17  promotion and epilogue: warp w reads tensor-memory lanes 32 (w % 4) .. +31
+//               (= tile rows) and one quarter of the columns, keeps the running f32 sums in
+//               registers (the next block's scales are loaded while the partial is awaited),
+//               and finally writes bf16 C.
 // Every wait is bounded; a wait that gives up flags the kernel status word and the CTA drains.
 //
 // The same kernel runs the grouped expert GEMMs of the block-FP8 MoE layer over expert-contiguous
@@ -35,26 +36,36 @@ namespace {
 
 constexpr int kBM = 128;
 constexpr int kBK = 128;  // one scale block; bytes = elements for E4M3
-constexpr int kStages = 4;
-constexpr int kEpiWarps = 8;
-constexpr int kThreads = (2 + kEpiWarps) * 32;
+// promotion warps: 4 per tensor-memory lane quarter (each a quarter of the columns) for gate/up,
+// whose epilogue is the heaviest; 2 per quarter (each half of the columns) otherwise, which
+// leaves the MMA thread's SM sub-partition less crowded (both chosen from measured A/B runs)
+__host__ __device__ constexpr int epi_warps(int mode) { return mode == TC_GATEUP ? 16 : 8; }
+__host__ __device__ constexpr int fp8_threads(int mode) { return (2 + epi_warps(mode)) * 32; }
 
-template <int BN>
+// PAIR: a cluster of 2 CTAs runs one 256 x BN tile with cta_group::2 MMAs; each CTA loads its 128
+// rows of A and half of the BN weight rows, so a CTA moves 32 KB instead of 48 KB from L2 per K
+// block for the same MMA work, and the smaller stages make a 6-deep ring.
+template <int BN, bool PAIR, int MODE>
 struct Fp8TcShape {
+    static constexpr int kStages = PAIR ? 6 : 4;
     static constexpr int kABytes = kBM * kBK;
-    static constexpr int kBBytes = BN * kBK;
+    static constexpr int kBBytes = (PAIR ? BN / 2 : BN) * kBK;
     static constexpr int kStageBytes = kABytes + kBBytes;
     static constexpr int kTmemCols = 2 * BN;  // two partial buffers (128, 256 or 512 columns)
-    static constexpr int kColsPerWarp = BN / 2;
-    static constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + 1024 + 256 + 2 * 128 * 4;
+    static constexpr int kSlices = epi_warps(MODE) / 4;  // column slices per lane quarter
+    static constexpr int kColsPerWarp = BN / kSlices;
+    static constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + 1024 + 256 + kSlices * 128 * 4;
 };
 
-template <int BN, int MODE>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int BN, int MODE, bool PAIR>
+__global__ void __launch_bounds__(fp8_threads(MODE), 1)
     fp8_tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                        Fp8TcArgs a)
 {
-    using Sh = Fp8TcShape<BN>;
+    using Sh = Fp8TcShape<BN, PAIR, MODE>;
+    constexpr int kStages = Sh::kStages;
+    constexpr int kEpiWarps = epi_warps(MODE);
+    static_assert(!PAIR || BN == 256, "pair tiles are 256 x 256");
     static_assert(MODE != TC_GATEUP || BN == 256, "gate/up tiles hold 128 gate + 128 up columns");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -70,7 +81,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // dense: grid x = row tiles, so consecutive CTAs share a B (weight) tile in L2; grouped: grid
     // x = output tiles, so the tiles of one expert block run back to back and its activation rows
     // come from DRAM once
-    const int m0 = (MODE == TC_DENSE ? blockIdx.x : blockIdx.y) * kBM;
+    // pair: rank 0 holds rows [0, 128) of the 256-row tile, rank 1 rows [128, 256); x counts CTAs
+    const uint32_t rank = PAIR ? tc::cluster_rank() : 0u;
+    const int tile_x = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+    const int m0 = PAIR ? (MODE == TC_DENSE ? tile_x : (int)blockIdx.y) * 2 * kBM + (int)rank * kBM
+                        : (MODE == TC_DENSE ? tile_x : (int)blockIdx.y) * kBM;
     const int KB = a.K / kBK;
     // output columns of this tile and the weight rows (in the [E * rows, K] weight matrix) loaded
     // into the B stage: dense and down take BN consecutive rows; gate/up takes 128 gate + 128 up
@@ -81,22 +96,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         brow0 = n0;
         bscale0 = a.b_scale + (size_t)(n0 / 128) * KB;
     } else {
-        if (m0 >= __ldg(a.ntp)) return;  // uniform over the CTA, before any barrier or allocation
+        // uniform over the CTA (and the pair: both test the pair's first row), before any barrier
+        if ((PAIR ? (int)blockIdx.y * 2 * kBM : m0) >= __ldg(a.ntp)) return;
         const int e = __ldg(a.expert_ids + blockIdx.y);
         if (e < 0 || e >= a.E) return;
         const float *ws = a.b_scale + (size_t)e * (a.rows_per_expert / 128) * KB;
         if (MODE == TC_GATEUP) {
-            n0 = blockIdx.x * 128;                      // feature tile
+            n0 = tile_x * 128;                          // feature tile
             brow0 = e * a.rows_per_expert + n0;         // gate rows
             brow1 = e * a.rows_per_expert + a.N + n0;   // up rows
             bscale0 = ws + (size_t)(n0 / 128) * KB;
             bscale1 = ws + (size_t)((a.N + n0) / 128) * KB;
         } else {
-            n0 = blockIdx.x * BN;
+            n0 = tile_x * BN;
             brow0 = e * a.rows_per_expert + n0;
             bscale0 = ws + (size_t)(n0 / 128) * KB;
         }
     }
+    // weight rows this CTA loads: all BN, or (pair) its half: gate/up rank 0 the gate rows, rank 1
+    // the up rows; dense / down rank r the rows [128 r, 128 r + 128) of the tile
+    const int brow_own = !PAIR ? brow0 : (MODE == TC_GATEUP ? (rank ? brow1 : brow0) : brow0 + (int)rank * 128);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -105,15 +124,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             tc::mbar_init(&tfull[b], 1);
-            tc::mbar_init(&tempty[b], kEpiWarps);
+            tc::mbar_init(&tempty[b], kEpiWarps * (PAIR ? 2 : 1));  // pair: both CTAs' promotion warps
         }
         tc::mbar_init(mma_done, 1);
         *abort_flag = 0;
         tc::fence_barrier_init();
     }
-    if (warp == 1) tc::tmem_alloc(tmem_slot, Sh::kTmemCols);
+    if (warp == 1) {
+        if (PAIR) tc::tmem_alloc_pair(tmem_slot, Sh::kTmemCols);
+        else tc::tmem_alloc(tmem_slot, Sh::kTmemCols);
+    }
     tc::fence_before_sync();
-    __syncthreads();
+    if (PAIR) tc::cluster_sync();  // both CTAs' barriers exist before any copy or arrival crosses over
+    else __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
 
@@ -126,6 +149,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int s = kb % kStages;
                 if (kb >= kStages && !tc::mbar_wait(&empty[s], ((kb / kStages) & 1) ^ 1, abort_flag, a.status)) break;
                 uint8_t *sa = smem + s * Sh::kStageBytes;
+                if (PAIR) {
+                    // both CTAs' bytes complete on rank 0's barrier, which alone expects them
+                    const uint32_t fb = tc::cluster_addr(&full[s], 0);
+                    if (rank == 0) tc::mbar_arrive_expect_tx(&full[s], 2 * Sh::kStageBytes);
+                    tc::tma_load_2d_pair(sa, &tmA, fb, kb * kBK, m0);
+                    tc::tma_load_2d_pair(sa + Sh::kABytes, &tmB, fb, kb * kBK, brow_own);
+                    issued = kb + 1;
+                    continue;
+                }
                 tc::mbar_arrive_expect_tx(&full[s], Sh::kStageBytes);
                 tc::tma_load_2d(sa, &tmA, &full[s], kb * kBK, m0);
                 if (MODE == TC_GATEUP) {
@@ -136,13 +168,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 issued = kb + 1;
             }
-            // no copy may still be landing in shared memory when the CTA exits
-            for (int kb = issued - kStages > 0 ? issued - kStages : 0; kb < issued; ++kb)
-                tc::mbar_drain(&full[kb % kStages], (kb / kStages) & 1, a.status);
+            // no copy may still be landing in shared memory when the CTA exits (pair: rank 0's
+            // barrier counts both CTAs' bytes; rank 1 is held by the final cluster barrier)
+            if (!PAIR || rank == 0)
+                for (int kb = issued - kStages > 0 ? issued - kStages : 0; kb < issued; ++kb)
+                    tc::mbar_drain(&full[kb % kStages], (kb / kStages) & 1, a.status);
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            constexpr uint32_t idesc = tc::idesc_f32(tc::kFmtE4M3, tc::kFmtE4M3, kBM, BN);
+        if (PAIR && rank != 0) {
+            // the peer issues nothing; it waits (bounded) until the pair's MMAs, which write its
+            // tensor memory and read its shared memory, are done
+            if (lane == 0) tc::mbar_drain(mma_done, 0, a.status);
+        } else if (lane == 0) {
+            constexpr uint32_t idesc = tc::idesc_f32(tc::kFmtE4M3, tc::kFmtE4M3, PAIR ? 2 * kBM : kBM, BN);
             const uint64_t a_base = tc::smem_desc_sw128(smem);
             for (int kb = 0; kb < KB; ++kb) {
                 const int s = kb % kStages, buf = kb & 1;
@@ -154,60 +192,84 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint64_t adesc = a_base + (uint64_t)((s * Sh::kStageBytes) >> 4);
                 const uint64_t bdesc = adesc + (uint64_t)(Sh::kABytes >> 4);
                 const uint32_t d = tmem + buf * BN;
-                tc::mma_f8f6f4_ss(d, adesc, bdesc, idesc, 0u);
+                if (PAIR) {
+                    tc::mma_f8f6f4_ss_pair(d, adesc, bdesc, idesc, 0u);
 #pragma unroll
-                for (int kk = 1; kk < kBK / 32; ++kk) tc::mma_f8f6f4_ss_acc(d, adesc + 2 * kk, bdesc + 2 * kk, idesc);
-                tc::mma_commit(&empty[s]);
-                tc::mma_commit(&tfull[buf]);
+                    for (int kk = 1; kk < kBK / 32; ++kk)
+                        tc::mma_f8f6f4_ss_pair_acc(d, adesc + 2 * kk, bdesc + 2 * kk, idesc);
+                    tc::mma_commit_pair(&empty[s], 0x3);
+                    tc::mma_commit_pair(&tfull[buf], 0x3);
+                } else {
+                    tc::mma_f8f6f4_ss(d, adesc, bdesc, idesc, 0u);
+#pragma unroll
+                    for (int kk = 1; kk < kBK / 32; ++kk)
+                        tc::mma_f8f6f4_ss_acc(d, adesc + 2 * kk, bdesc + 2 * kk, idesc);
+                    tc::mma_commit(&empty[s]);
+                    tc::mma_commit(&tfull[buf]);
+                }
             }
             // every MMA issued must finish before tensor memory is released
-            tc::mma_commit(mma_done);
+            if (PAIR) tc::mma_commit_pair(mma_done, 0x3);
+            else tc::mma_commit(mma_done);
             tc::mbar_drain(mma_done, 0, a.status);
         }
     } else {
+        // warp w: tensor-memory lanes 32 (w % 4) .. +31 (= tile rows) and column slice cq
         constexpr int COLS = Sh::kColsPerWarp;
-        const int ew = warp - 2, quarter = warp & 3, half = ew >> 2;
+        constexpr int GF = 128 / Sh::kSlices;  // gate/up: gate features per warp
+        const int ew = warp - 2, quarter = warp & 3, cq = ew >> 2;
         const int row = quarter * 32 + lane;
         const int m = m0 + row;
-        // TMEM columns of this warp: one contiguous half of the tile, or (gate/up) 64 gate columns
-        // and the 64 matching up columns
-        const int c_first = (MODE == TC_GATEUP) ? 64 * half : half * COLS;
-        const int c_second = (MODE == TC_GATEUP) ? 128 + 64 * half : half * COLS + COLS / 2;
+        // TMEM columns of this warp: one contiguous slice of the tile, or (gate/up) GF gate
+        // columns and the GF matching up columns
+        const int c_first = (MODE == TC_GATEUP) ? GF * cq : cq * COLS;
+        const int c_second = (MODE == TC_GATEUP) ? 128 + GF * cq : 0;
         const float *as_row = a.a_scale + (size_t)(m < a.M ? m : a.M - 1) * KB;
-        const float *bs_first = (MODE == TC_GATEUP) ? bscale0 : bscale0 + (size_t)((half * COLS) / 128) * KB;
+        const float *bs_first = (MODE == TC_GATEUP) ? bscale0 : bscale0 + (size_t)((cq * COLS) / 128) * KB;
         const float *bs_second = (MODE == TC_GATEUP) ? bscale1 : bs_first;
         float acc[COLS];
 #pragma unroll
         for (int j = 0; j < COLS; ++j) acc[j] = 0.f;
         bool ok = true;
+        // the scales of block kb + 1 are loaded while block kb's partial is awaited
+        float n_sa = __ldg(as_row), n_b0 = __ldg(bs_first), n_b1 = __ldg(bs_second);
         for (int kb = 0; kb < KB && ok; ++kb) {
             const int buf = kb & 1;
-            const float sa = __ldg(as_row + kb);
-            const float sc0 = sa * __ldg(bs_first + kb), sc1 = sa * __ldg(bs_second + kb);
-            // every lane waits, then the warp agrees: the tensor-memory loads below are warp-wide
-            ok = __all_sync(0xFFFFFFFFu, tc::mbar_wait(&tfull[buf], (kb >> 1) & 1, abort_flag, a.status));
+            const float sc0 = n_sa * n_b0, sc1 = n_sa * n_b1;
+            if (kb + 1 < KB) {
+                n_sa = __ldg(as_row + kb + 1);
+                n_b0 = __ldg(bs_first + kb + 1);
+                n_b1 = __ldg(bs_second + kb + 1);
+            }
+            // lane 0 waits, the warp agrees: the tensor-memory loads below are warp-wide
+            ok = tc::mbar_wait_warp(&tfull[buf], (kb >> 1) & 1, abort_flag, a.status);
             if (!ok) break;
             tc::fence_after_sync();
             const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + buf * BN;
+            // 16-column loads keep the registers to acc[] + 16
 #pragma unroll
-            for (int c = 0; c < COLS / 32; ++c) {
-                // gate/up: chunks 0-1 gate, 2-3 up; otherwise one contiguous run of columns
-                const bool second = (MODE == TC_GATEUP) && c >= 2;
-                const int col = (MODE == TC_GATEUP) ? (second ? c_second : c_first) + (c & 1) * 32 : c_first + c * 32;
+            for (int c = 0; c < COLS / 16; ++c) {
+                // gate/up: the first GF / 16 chunks gate, the rest up; otherwise one contiguous run
+                const bool second = (MODE == TC_GATEUP) && c >= GF / 16;
+                const int col = (MODE == TC_GATEUP) ? (second ? c_second + (c - GF / 16) * 16 : c_first + c * 16)
+                                                    : c_first + c * 16;
                 const float sc = second ? sc1 : sc0;
-                uint32_t r[32];
-                tc::tmem_ld32(taddr + col, r);
+                uint32_t r[16];
+                tc::tmem_ld16(taddr + col, r);
                 tc::tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) acc[c * 32 + j] = fmaf(__uint_as_float(r[j]), sc, acc[c * 32 + j]);
+                for (int j = 0; j < 16; ++j) acc[c * 16 + j] = fmaf(__uint_as_float(r[j]), sc, acc[c * 16 + j]);
             }
             tc::fence_before_sync();
             __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&tempty[buf]);
+            if (lane == 0) {
+                if (PAIR && rank != 0) tc::mbar_arrive_cluster(tc::cluster_addr(&tempty[buf], 0));  // the issuer's
+                else tc::mbar_arrive(&tempty[buf]);
+            }
         }
         if (MODE == TC_DENSE) {
             if (ok && m < a.M) {
-                uint16_t *crow = a.C + (size_t)m * a.N + n0 + half * COLS;
+                uint16_t *crow = a.C + (size_t)m * a.N + n0 + cq * COLS;
 #pragma unroll
                 for (int j = 0; j < COLS; j += 8) {
                     uint4 v;
@@ -219,22 +281,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         } else if (MODE == TC_GATEUP) {
-            // a = silu(g) * u for features n0 + 64 half + j; E4M3 per row and 128-feature group
+            // a = silu(g) * u for features n0 + GF cq + j; E4M3 per row and 128-feature group
             float amax = 0.f;
 #pragma unroll
-            for (int j = 0; j < 64; ++j) {
-                acc[j] = silu_f32(acc[j]) * acc[64 + j];
+            for (int j = 0; j < GF; ++j) {
+                acc[j] = silu_f32(acc[j]) * acc[GF + j];
                 amax = fmaxf(amax, fabsf(acc[j]));
             }
-            float *red = reinterpret_cast<float *>(tmem_slot + 4);  // [2][128] group maxima
-            red[half * 128 + row] = amax;
+            float *red = reinterpret_cast<float *>(tmem_slot + 4);  // [slices][128] slice maxima
+            red[cq * 128 + row] = amax;
             asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory");
-            amax = fmaxf(red[row], red[128 + row]);
+            amax = red[row];
+#pragma unroll
+            for (int q = 1; q < Sh::kSlices; ++q) amax = fmaxf(amax, red[q * 128 + row]);
             const float sc = __fdiv_rn(fmaxf(amax, 1e-10f), 448.0f);
             if (ok) {
-                uint8_t *hrow = a.hq + (size_t)m * a.N + n0 + 64 * half;
+                uint8_t *hrow = a.hq + (size_t)m * a.N + n0 + GF * cq;
 #pragma unroll
-                for (int j = 0; j < 64; j += 16) {
+                for (int j = 0; j < GF; j += 16) {
                     uint4 v;
                     uint32_t *w = &v.x;
 #pragma unroll
@@ -245,13 +309,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     *reinterpret_cast<uint4 *>(hrow + j) = v;
                 }
-                if (half == 0) a.hs[(size_t)m * (a.N / 128) + n0 / 128] = sc;
+                if (cq == 0) a.hs[(size_t)m * (a.N / 128) + n0 / 128] = sc;
             }
         } else {
             const int slot = __ldg(a.sorted_ids + m);
             if (ok && slot < a.n_slots) {
                 const float wt = __ldg(a.topk_w + slot);
-                float *yrow = a.ys + (size_t)slot * a.N + n0 + half * COLS;
+                float *yrow = a.ys + (size_t)slot * a.N + n0 + cq * COLS;
 #pragma unroll
                 for (int j = 0; j < COLS; j += 4)
                     *reinterpret_cast<float4 *>(yrow + j) =
@@ -260,26 +324,49 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
     tc::fence_before_sync();
-    __syncthreads();
+    if (PAIR) tc::cluster_sync();  // neither CTA leaves while the pair's copies or MMAs use it
+    else __syncthreads();
     tc::fence_after_sync();
-    if (warp == 1) tc::tmem_dealloc(tmem, Sh::kTmemCols);
+    if (warp == 1) {
+        if (PAIR) tc::tmem_dealloc_pair(tmem, Sh::kTmemCols);
+        else tc::tmem_dealloc(tmem, Sh::kTmemCols);
+    }
 }
 
-template <int BN, int MODE>
+template <int BN, int MODE, bool PAIR = false>
 int launch_tc(const Fp8TcArgs &a, const CUtensorMap &tmA, const CUtensorMap &tmB, int grid_x, int grid_y,
               cudaStream_t s)
 {
-    using Sh = Fp8TcShape<BN>;
+    using Sh = Fp8TcShape<BN, PAIR, MODE>;
+    constexpr int kThreads = fp8_threads(MODE);
     static bool attr = false;
     if (!attr) {
-        const cudaError_t e = cudaFuncSetAttribute(fp8_tc_gemm_kernel<BN, MODE>,
+        const cudaError_t e = cudaFuncSetAttribute(fp8_tc_gemm_kernel<BN, MODE, PAIR>,
                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Sh::kSmemBytes);
         if (e != cudaSuccess)
             return set_error(MOEQ_ERR_CUDA, "tcgen05 FP8 GEMM: shared-memory attribute: %s", cudaGetErrorString(e));
         attr = true;
     }
     if (grid_x <= 0 || grid_y <= 0) return MOEQ_OK;
-    fp8_tc_gemm_kernel<BN, MODE><<<dim3(grid_x, grid_y), kThreads, Sh::kSmemBytes, s>>>(tmA, tmB, a);
+    if (!PAIR) {
+        fp8_tc_gemm_kernel<BN, MODE, PAIR><<<dim3(grid_x, grid_y), kThreads, Sh::kSmemBytes, s>>>(tmA, tmB, a);
+        return MOEQ_OK;
+    }
+    // clusters of 2 CTAs along x (grid_x even): the pair of one 256-row tile
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid_x, grid_y);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = Sh::kSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr_c[1];
+    attr_c[0].id = cudaLaunchAttributeClusterDimension;
+    attr_c[0].val.clusterDim.x = 2;
+    attr_c[0].val.clusterDim.y = 1;
+    attr_c[0].val.clusterDim.z = 1;
+    cfg.attrs = attr_c;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, fp8_tc_gemm_kernel<BN, MODE, PAIR>, tmA, tmB, a);
+    if (e != cudaSuccess) return set_error(MOEQ_ERR_CUDA, "tcgen05 FP8 pair GEMM launch: %s", cudaGetErrorString(e));
     return MOEQ_OK;
 }
 
@@ -290,12 +377,15 @@ int launch_fp8_tc_gemm(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B, c
     // Up to 64 rows the weights stream once (HBM bound) and narrow 64-column tiles give every SM
     // several CTAs; from 65 rows, 256-column tiles (more weight bytes in flight per SM, fewer
     // activation re-reads; tensor bound for many rows). Chosen from measured M sweeps.
+    // From 256 rows, CTA pairs (256 x 256 tiles, half the weight rows per CTA).
     const int bn = (a.M <= 64) ? 64 : (a.N % 256 == 0) ? 256 : 128;
+    const bool pair = bn == 256 && a.M >= 256;
     CUtensorMap tmA, tmB;
     int rc = make_tmap_2d(&tmA, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.M, (uint64_t)a.K, kBM, kBK);
     if (rc) return rc;
-    rc = make_tmap_2d(&tmB, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.N, (uint64_t)a.K, bn, kBK);
+    rc = make_tmap_2d(&tmB, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.N, (uint64_t)a.K, pair ? 128 : bn, kBK);
     if (rc) return rc;
+    if (pair) return launch_tc<256, TC_DENSE, true>(a, tmA, tmB, 2 * cdiv(a.M, 2 * kBM), a.N / 256, s);
     if (bn == 256) return launch_tc<256, TC_DENSE>(a, tmA, tmB, cdiv(a.M, kBM), a.N / 256, s);
     if (bn == 128) return launch_tc<128, TC_DENSE>(a, tmA, tmB, cdiv(a.M, kBM), a.N / 128, s);
     return launch_tc<64, TC_DENSE>(a, tmA, tmB, cdiv(a.M, kBM), a.N / 64, s);

@@ -257,9 +257,11 @@ def test_dense_fp8_small_shapes_all_rows(M):
     _dense_parity(M, 512, 1024, np.arange(M, dtype=np.int32))
 
 
-@pytest.mark.parametrize("M,N,K", [(128, 256, 1024), (200, 512, 512), (300, 384, 896), (1000, 256, 7168)])
+@pytest.mark.parametrize("M,N,K", [(128, 256, 1024), (200, 512, 512), (300, 384, 896), (1000, 256, 7168),
+                                   (256, 512, 384), (257, 768, 640), (640, 256, 1152)])
 def test_dense_fp8_tensor_core_shapes_all_rows(M, N, K):
-    """Row counts at and past the tcgen05 threshold, ragged M tails, N not a multiple of 256."""
+    """Row counts at and past the tcgen05 threshold and the CTA-pair threshold (256 rows), ragged M
+    tails, N not a multiple of 256."""
     _dense_parity(M, N, K, np.arange(M, dtype=np.int32))
 
 
