@@ -169,8 +169,15 @@ static RouteBufs carve_route(Carve &c, long T, int k, int E, int block_m)
 // expert has (HBM bound).
 static bool w4_use_tc(long T, int k, int E) { return (double)T * k / (double)E >= 16.0; }
 
+// Within the tensor-core schedule, expert blocks with at most this many real rows (the tail of a
+// skewed routing) run on the register-fed kernel: a tcgen05 block dequantizes its whole weight
+// tile whatever its row count, while the register-fed kernel streams the weights once at HBM rate.
+// Measured on the Zipf prefill (T=8192, E=384): 8 rows beat 16, 32 and 64 (at 64 rows per block
+// the legacy mma.sync rate, not the weight stream, bounds the register-fed kernel).
+constexpr int kW4SmallRows = 8;
+
 static size_t w4a16_layout(Carve &c, long T, int H, int I, int E, int k, RouteBufs *rb, uint16_t **h, float **ys,
-                           uint16_t **xg = nullptr)
+                           uint16_t **xg = nullptr, uint16_t **h_small = nullptr)
 {
     const bool tcp = w4_use_tc(T, k, E);
     RouteBufs r = carve_route(c, T, k, E, tcp ? 256 : pick_block_m(T, k, E));  // tensor-core tiles: 256 rows
@@ -178,10 +185,13 @@ static size_t w4a16_layout(Carve &c, long T, int H, int I, int E, int k, RouteBu
     uint16_t *hp = c.take<uint16_t>((tcp ? cap : (size_t)T * k) * I);
     float *yp = c.take<float>((size_t)T * k * H);
     uint16_t *xgp = tcp ? c.take<uint16_t>(cap * H) : nullptr;
+    // small blocks of the tensor-core schedule: h in slot order, natural feature order
+    uint16_t *hsp = tcp ? c.take<uint16_t>((size_t)T * k * I) : nullptr;
     if (rb) *rb = r;
     if (h) *h = hp;
     if (ys) *ys = yp;
     if (xg) *xg = xgp;
+    if (h_small) *h_small = hsp;
     return c.used;
 }
 
@@ -324,9 +334,9 @@ int moe_w4a16_forward(const uint16_t *x, const float *logits, int T, int H, int 
     cudaStream_t s = (cudaStream_t)stream;
     Carve c(ws);
     RouteBufs r;
-    uint16_t *h, *xg;
+    uint16_t *h, *xg, *h_small;
     float *ys;
-    w4a16_layout(c, T, H, I, E, k, &r, &h, &ys, &xg);
+    w4a16_layout(c, T, H, I, E, k, &r, &h, &ys, &xg, &h_small);
     int32_t *ids = topk_ids_out ? topk_ids_out : r.ids;
     float *tw = topk_w_out ? topk_w_out : r.w;
     const int n = T * k;
@@ -364,10 +374,29 @@ int moe_w4a16_forward(const uint16_t *x, const float *logits, int T, int H, int 
         t.wq = w13_q;
         t.ws = w13_s;
         t.h_out = h;
+        t.small_rows = kW4SmallRows;
+        // the small blocks: register-fed kernel over the same 256-row alignment, h in slot order
+        W4GroupedArgs g{};
+        g.E = E;
+        g.sorted_ids = r.sorted;
+        g.expert_ids = r.eids;
+        g.num_tokens_padded = r.ntp;
+        g.n_slots = n;
+        g.topk_w = tw;
+        g.blk_stride = r.block_m;
+        g.act = x;
+        g.act_row_div = k;
+        g.wq = w13_q;
+        g.ws = w13_s;
+        g.K = H;
+        g.n_out = I;
+        g.n_rows = 2 * I;
+        g.h_out = h_small;
         int rc;
         {
             trace::Scope ts(trace::GATE_UP, s);
             rc = launch_w4a16_tc(t, TC_GATEUP, xg, r.max_blocks, s);
+            launch_w4a16_grouped_mma(g, MODE_GATEUP, kW4SmallRows, r.max_blocks, s);
         }
         if (rc) return rc;
         t.N = H;
@@ -376,9 +405,18 @@ int moe_w4a16_forward(const uint16_t *x, const float *logits, int T, int H, int 
         t.wq = w2_q;
         t.ws = w2_s;
         t.ys = ys;
+        g.act = h_small;
+        g.act_row_div = 1;
+        g.wq = w2_q;
+        g.ws = w2_s;
+        g.K = I;
+        g.n_out = H;
+        g.n_rows = H;
+        g.y_out = ys;
         {
             trace::Scope ts(trace::DOWN, s);
             rc = launch_w4a16_tc(t, TC_DOWN, h, r.max_blocks, s);
+            launch_w4a16_grouped_mma(g, MODE_DOWN, kW4SmallRows, r.max_blocks, s);
         }
         if (rc) return rc;
     } else {

@@ -24,6 +24,9 @@ struct W4GroupedArgs {
     const float *topk_w;     // [T*k] (down)
     uint16_t *h_out;         // [T*k, I] bf16 (gate/up)
     float *y_out;            // [T*k, H] f32, routing weight applied (down)
+    // 0: align blocks of BM rows. Otherwise the alignment has blocks of blk_stride rows and the
+    // kernel takes only those with at most BM real rows (the rest belong to the tensor-core path)
+    int blk_stride;
 };
 
 struct F8GroupedArgs {
@@ -82,6 +85,7 @@ struct W4TcArgs {
     const float *topk_w;
     uint16_t *h_out;        // gate/up: [M, N] bf16, pair-permuted inside 8-element chunks
     float *ys;              // down: [n_slots, N] f32, routing weight applied
+    int small_rows;         // blocks with at most this many real rows are left to the register-fed path
 };
 
 void launch_route_topk(const float *logits, int T, int E, int k, int32_t *ids, float *w, cudaStream_t s);

@@ -114,6 +114,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
     // real rows of this block: the expert's slots come first, padding after
     const int valid = __syncthreads_count(threadIdx.x < kTok && __ldg(a.sorted_ids + r0 + threadIdx.x) < a.n_slots);
     const int n_mma = (valid + 15) & ~15;  // MMA N: multiple of 16 in [16, 256]
+    if (valid <= a.small_rows) return;      // left to the register-fed kernel (uniform, before any barrier)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {

@@ -76,7 +76,10 @@ __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4Grouped
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
     const int blk = blockIdx.x;
-    if (blk * BM >= __ldg(a.num_tokens_padded)) return;
+    const int base = blk * (a.blk_stride ? a.blk_stride : BM);  // first aligned row of the block
+    if (base >= __ldg(a.num_tokens_padded)) return;
+    // strided: blocks with more than BM real rows are the tensor-core path's (real rows come first)
+    if (a.blk_stride && __ldg(a.sorted_ids + base + BM) < a.n_slots) return;
     const int e = __ldg(a.expert_ids + blk);
     if (e < 0 || e >= a.E) return;
 
@@ -99,7 +102,7 @@ __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4Grouped
     const uint16_t *act_row[MS];
 #pragma unroll
     for (int s = 0; s < MS; ++s) {
-        const int slot = __ldg(a.sorted_ids + blk * BM + 8 * s + g);
+        const int slot = __ldg(a.sorted_ids + base + 8 * s + g);
         act_row[s] = (slot < a.n_slots) ? a.act + (size_t)(slot / a.act_row_div) * K : nullptr;
     }
 
@@ -203,7 +206,7 @@ __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4Grouped
     for (int s = 0; s < MS; ++s) {
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
-            const int slot = __ldg(a.sorted_ids + blk * BM + 8 * s + 2 * t + c);
+            const int slot = __ldg(a.sorted_ids + base + 8 * s + 2 * t + c);
             if (slot >= a.n_slots) continue;
             if (MODE == MODE_GATEUP) {
                 uint16_t *h = a.h_out + (size_t)slot * a.n_out;

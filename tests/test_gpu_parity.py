@@ -196,6 +196,7 @@ def test_w4a16_prefill_sampled():
     (37, 16, 16, 256, 128, "equal"),      # k = E, uniform weights 1/E
     (5, 1024, 32, 256, 128, "normal"),    # largest E and k
     (300, 64, 6, 384, 256, "zipf"),       # skewed, empty experts, ragged blocks
+    (400, 32, 2, 256, 128, "split"),      # tensor-core schedule with blocks of exactly 8 and 9 rows
 ])
 def test_w4a16_edge_cases(T, E, k, H, I, logit_mode):
     wl = W.WORKLOADS["tiny_w4a16"]
@@ -207,6 +208,19 @@ def test_w4a16_edge_cases(T, E, k, H, I, logit_mode):
         d["logits"] = torch.zeros((T, E), device=DEV)
     elif logit_mode == "zipf":
         d["logits"] = W.router_logits(W.WORKLOADS["prefill_w4a16"], T, E, device=DEV)
+    elif logit_mode == "split":
+        # experts 0/1 take 300 tokens (full 256-row blocks + a tail), 2/3 exactly 8 (the register-fed
+        # side of the small-block threshold), 4/5 exactly 9 (the tensor-core side), the rest 1-5
+        first = np.zeros(T, np.int64)
+        first[:300] = 0
+        first[300:308] = 2
+        first[308:317] = 4
+        first[317:] = 6 + (np.arange(T - 317) % 20)
+        lg = torch.zeros((T, E), device=DEV)
+        idx = torch.as_tensor(first, device=DEV)
+        lg[torch.arange(T, device=DEV), idx] = 5.0
+        lg[torch.arange(T, device=DEV), idx + 1] = 4.0
+        d["logits"] = lg
     _layer_parity(d, np.arange(T, dtype=np.int32), TOL_W4A16, f"w4a16 T={T} E={E} k={k}")
 
 
