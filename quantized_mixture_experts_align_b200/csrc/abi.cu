@@ -175,6 +175,7 @@ static bool w4_use_tc(long T, int k, int E) { return (double)T * k / (double)E >
 // Measured on the Zipf prefill (T=8192, E=384): 8 rows beat 16, 32 and 64 (at 64 rows per block
 // the legacy mma.sync rate, not the weight stream, bounds the register-fed kernel).
 constexpr int kW4SmallRows = 8;
+static_assert(kW4SmallRows == 8, "the strided register-fed instantiation is built for 8-row tiles");
 
 static size_t w4a16_layout(Carve &c, long T, int H, int I, int E, int k, RouteBufs *rb, uint16_t **h, float **ys,
                            uint16_t **xg = nullptr, uint16_t **h_small = nullptr)

@@ -66,7 +66,7 @@ constexpr int kW4StageBytes = 4 * 32 * 16 + 4 * 8 * 8;  // 2048 B codes + 256 B 
 // MODE_GATEUP: rows [f0, f0+16) (gate) and [I + f0, I + f0 + 16) (up) of W13; epilogue writes
 //              h[slot, f] = bf16(silu(gate) * up).
 // MODE_DOWN:   rows [r0, r0+32) of W2; epilogue writes ys[slot, r] = topk_w[slot] * y (f32).
-template <int BM, int WARPS, int MODE>
+template <int BM, int WARPS, int MODE, bool STRIDED>
 __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4GroupedArgs a)
 {
     constexpr int MS = BM / 8;  // token sub-tiles of 8 columns
@@ -76,10 +76,10 @@ __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4Grouped
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
     const int blk = blockIdx.x;
-    const int base = blk * (a.blk_stride ? a.blk_stride : BM);  // first aligned row of the block
+    const int base = blk * (STRIDED ? a.blk_stride : BM);  // first aligned row of the block
     if (base >= __ldg(a.num_tokens_padded)) return;
     // strided: blocks with more than BM real rows are the tensor-core path's (real rows come first)
-    if (a.blk_stride && __ldg(a.sorted_ids + base + BM) < a.n_slots) return;
+    if (STRIDED && __ldg(a.sorted_ids + base + BM) < a.n_slots) return;
     const int e = __ldg(a.expert_ids + blk);
     if (e < 0 || e >= a.E) return;
 
@@ -224,28 +224,34 @@ __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4Grouped
     }
 }
 
-template <int BM, int WARPS, int MODE>
+template <int BM, int WARPS, int MODE, bool STRIDED>
 static void launch_bm(const W4GroupedArgs &a, int max_blocks, cudaStream_t s)
 {
     const int rows_per_cta = (MODE == MODE_GATEUP ? 16 : 32) * WARPS;
     const size_t smem = (size_t)WARPS * kW4Stages * kW4StageBytes;
     static bool attr_set = false;  // per template instance; the attribute is per function
     if (!attr_set) {
-        cudaFuncSetAttribute(w4a16_grouped_mma_kernel<BM, WARPS, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(w4a16_grouped_mma_kernel<BM, WARPS, MODE, STRIDED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
         attr_set = true;
     }
     dim3 grid(max_blocks, cdiv(a.n_out, rows_per_cta));
-    w4a16_grouped_mma_kernel<BM, WARPS, MODE><<<grid, WARPS * 32, smem, s>>>(a);
+    w4a16_grouped_mma_kernel<BM, WARPS, MODE, STRIDED><<<grid, WARPS * 32, smem, s>>>(a);
 }
 
 void launch_w4a16_grouped_mma(const W4GroupedArgs &a, int mode, int block_m, int max_blocks, cudaStream_t s)
 {
     if (max_blocks <= 0) return;
-#define MOEQ_W4_CASE(BMV)                                                   \
-    case BMV:                                                               \
-        if (mode == MODE_GATEUP) launch_bm<BMV, 4, MODE_GATEUP>(a, max_blocks, s); \
-        else launch_bm<BMV, 4, MODE_DOWN>(a, max_blocks, s);                \
+    if (a.blk_stride) {  // small blocks of the tensor-core schedule
+        if (block_m != 8) return;
+        if (mode == MODE_GATEUP) launch_bm<8, 4, MODE_GATEUP, true>(a, max_blocks, s);
+        else launch_bm<8, 4, MODE_DOWN, true>(a, max_blocks, s);
+        return;
+    }
+#define MOEQ_W4_CASE(BMV)                                                          \
+    case BMV:                                                                      \
+        if (mode == MODE_GATEUP) launch_bm<BMV, 4, MODE_GATEUP, false>(a, max_blocks, s); \
+        else launch_bm<BMV, 4, MODE_DOWN, false>(a, max_blocks, s);                \
         break;
     switch (block_m) {
         MOEQ_W4_CASE(8)
