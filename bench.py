@@ -244,6 +244,49 @@ def measure_fp8_peak():
         return {"error": f"{type(exc).__name__}: {exc}"[:200]}
 
 
+def launch_overhead_w4a16(moeq, d, steps, warmup):
+    """Launch overhead of the decode layer: host time to enqueue one eager forward (the C ABI
+    call with its five launches) and one CUDA-graph replay of the same forward, and the device
+    time per step of back-to-back eager calls and graph replays (no L2 flush: launch gaps show)."""
+    out = torch.empty((d["T"], d["H"]), dtype=torch.bfloat16, device="cuda")
+    ws = moeq.workspace(moeq.moe_w4a16_workspace_size(d["T"], d["H"], d["I"], d["E"], d["k"]), "cuda")
+
+    def step():
+        moeq.moe_w4a16_forward(d["x"], d["logits"], d["k"], d["w13q"], d["w13s"], d["w2q"], d["w2s"], out=out, ws=ws)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for _ in range(warmup):
+            step()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    torch.cuda.synchronize()
+
+    def back_to_back(fn):
+        fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0 = time.perf_counter()
+        e0.record()
+        for _ in range(steps):
+            fn()
+        e1.record()
+        host_us = (time.perf_counter() - t0) / steps * 1e6
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps, host_us
+
+    eager_ms, eager_host = back_to_back(step)
+    graph_ms, graph_host = back_to_back(g.replay)
+    del g
+    return {"eager_ms_per_step": eager_ms, "graph_ms_per_step": graph_ms, "eager_host_submit_us": eager_host,
+            "graph_host_submit_us": graph_host, "steps": steps,
+            "how": "back-to-back steps on one stream, no L2 flush; host time = enqueue time per step"}
+
+
 def run_w4a16(moeq, d, steps, warmup, flush, world, trace=False):
     out = torch.empty((d["T"], d["H"]), dtype=torch.bfloat16, device="cuda")
     ws = moeq.workspace(moeq.moe_w4a16_workspace_size(d["T"], d["H"], d["I"], d["E"], d["k"]), "cuda")
@@ -460,6 +503,7 @@ def main():
     e2e_value, e2e_step = job_value(step_bytes / 1e9, statistics.mean(e2e_ms), world)
     e2e = {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h, "ms_per_step": e2e_step}
+    launch = launch_overhead_w4a16(moeq, d, args.steps, args.warmup)
 
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -473,6 +517,7 @@ def main():
         "roofline": roofline,
         "stages_ms": {k: v[0] / max(v[1], 1) for k, v in stages.items() if v[1]},
         "e2e": e2e,
+        "launch_overhead": launch,
         "gpu_launches": 5 * args.steps,
     }
 
