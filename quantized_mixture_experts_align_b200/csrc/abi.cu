@@ -177,14 +177,14 @@ static bool w4_use_tc(long T, int k, int E) { return (double)T * k / (double)E >
 constexpr int kW4SmallRows = 8;
 static_assert(kW4SmallRows == 8, "the strided register-fed instantiation is built for 8-row tiles");
 
-static size_t w4a16_layout(Carve &c, long T, int H, int I, int E, int k, RouteBufs *rb, uint16_t **h, float **ys,
+static size_t w4a16_layout(Carve &c, long T, int H, int I, int E, int k, RouteBufs *rb, uint16_t **h, uint16_t **ys,
                            uint16_t **xg = nullptr, uint16_t **h_small = nullptr)
 {
     const bool tcp = w4_use_tc(T, k, E);
     RouteBufs r = carve_route(c, T, k, E, tcp ? 256 : pick_block_m(T, k, E));  // tensor-core tiles: 256 rows
     const size_t cap = (size_t)r.max_blocks * r.block_m;
     uint16_t *hp = c.take<uint16_t>((tcp ? cap : (size_t)T * k) * I);
-    float *yp = c.take<float>((size_t)T * k * H);
+    uint16_t *yp = c.take<uint16_t>((size_t)T * k * H);  // weighted slot rows (bf16) for the combine
     uint16_t *xgp = tcp ? c.take<uint16_t>(cap * H) : nullptr;
     // small blocks of the tensor-core schedule: h in slot order, natural feature order
     uint16_t *hsp = tcp ? c.take<uint16_t>((size_t)T * k * I) : nullptr;
@@ -202,7 +202,7 @@ static size_t w4a16_layout(Carve &c, long T, int H, int I, int E, int k, RouteBu
 static bool fp8_use_tc(long T, int k, int E) { return (double)T * k / (double)E >= 16.0; }
 
 static size_t fp8_layout(Carve &c, long T, int H, int I, int E, int k, RouteBufs *rb, uint8_t **xq, float **xs,
-                         uint8_t **hq, float **hs, float **ys, uint8_t **xg = nullptr, float **xsg = nullptr)
+                         uint8_t **hq, float **hs, uint16_t **ys, uint8_t **xg = nullptr, float **xsg = nullptr)
 {
     const bool tcp = fp8_use_tc(T, k, E);
     RouteBufs r = carve_route(c, T, k, E, tcp ? 128 : pick_block_m(T, k, E));
@@ -212,7 +212,7 @@ static size_t fp8_layout(Carve &c, long T, int H, int I, int E, int k, RouteBufs
     float *xsp = c.take<float>((size_t)T * (H / 128));
     uint8_t *hqp = c.take<uint8_t>(hrows * I);
     float *hsp = c.take<float>(hrows * (I / 128));
-    float *yp = c.take<float>((size_t)T * k * H);
+    uint16_t *yp = c.take<uint16_t>((size_t)T * k * H);  // weighted slot rows (bf16) for the combine
     uint8_t *xgp = tcp ? c.take<uint8_t>(cap * H) : nullptr;
     float *xsgp = tcp ? c.take<float>(cap * (H / 128)) : nullptr;
     if (rb) *rb = r;
@@ -336,7 +336,7 @@ int moe_w4a16_forward(const uint16_t *x, const float *logits, int T, int H, int 
     Carve c(ws);
     RouteBufs r;
     uint16_t *h, *xg, *h_small;
-    float *ys;
+    uint16_t *ys;
     w4a16_layout(c, T, H, I, E, k, &r, &h, &ys, &xg, &h_small);
     int32_t *ids = topk_ids_out ? topk_ids_out : r.ids;
     float *tw = topk_w_out ? topk_w_out : r.w;
@@ -494,7 +494,8 @@ int moe_w8a8_block_fp8_forward(const uint16_t *x, const float *logits, int T, in
     Carve c(ws);
     RouteBufs r;
     uint8_t *xq, *hq, *xg;
-    float *xs, *hs, *ys, *xsg;
+    float *xs, *hs, *xsg;
+    uint16_t *ys;
     fp8_layout(c, T, H, I, E, k, &r, &xq, &xs, &hq, &hs, &ys, &xg, &xsg);
     int32_t *ids = topk_ids_out ? topk_ids_out : r.ids;
     float *tw = topk_w_out ? topk_w_out : r.w;

@@ -245,11 +245,11 @@ __global__ void __launch_bounds__(WARPS * 32) fp8_grouped_mma_kernel(F8GroupedAr
                     const int slot = __ldg(a.sorted_ids + j);
                     if (slot >= a.n_slots) continue;
                     const float wt = __ldg(a.topk_w + slot);
-                    float *y = a.y_out + (size_t)slot * a.n_out;
-                    y[rowA + g] = wt * accA[s][c];
-                    y[rowA + g + 8] = wt * accA[s][2 + c];
-                    y[rowB + g] = wt * accB[s][c];
-                    y[rowB + g + 8] = wt * accB[s][2 + c];
+                    uint16_t *y = a.y_out + (size_t)slot * a.n_out;
+                    y[rowA + g] = f32_to_bf16(wt * accA[s][c]);
+                    y[rowA + g + 8] = f32_to_bf16(wt * accA[s][2 + c]);
+                    y[rowB + g] = f32_to_bf16(wt * accB[s][c]);
+                    y[rowB + g + 8] = f32_to_bf16(wt * accB[s][2 + c]);
                 }
             }
         }

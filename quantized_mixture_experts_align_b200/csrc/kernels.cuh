@@ -23,7 +23,7 @@ struct W4GroupedArgs {
     int n_slots;             // T*k; sorted_ids entries >= n_slots are padding
     const float *topk_w;     // [T*k] (down)
     uint16_t *h_out;         // [T*k, I] bf16 (gate/up)
-    float *y_out;            // [T*k, H] f32, routing weight applied (down)
+    uint16_t *y_out;         // [T*k, H] bf16, routing weight applied (down)
     // 0: align blocks of BM rows. Otherwise the alignment has blocks of blk_stride rows and the
     // kernel takes only those with at most BM real rows (the rest belong to the tensor-core path)
     int blk_stride;
@@ -46,7 +46,7 @@ struct F8GroupedArgs {
     const float *topk_w;
     uint8_t *hq_out;         // [T*k, I]
     float *hs_out;           // [T*k, I/128]
-    float *y_out;            // [T*k, H]
+    uint16_t *y_out;         // [T*k, H] bf16, routing weight applied (down)
     uint16_t *c_out;         // dense: [M, N] bf16
 };
 
@@ -68,7 +68,7 @@ struct Fp8TcArgs {
     const float *topk_w;
     uint8_t *hq;            // gate/up out: [M, N] E4M3
     float *hs;              // gate/up out: [M, N/128]
-    float *ys;              // down out: [n_slots, N] f32, routing weight applied
+    uint16_t *ys;           // down out: [n_slots, N] bf16, routing weight applied
 };
 
 struct W4TcArgs {
@@ -84,14 +84,14 @@ struct W4TcArgs {
     int n_slots;
     const float *topk_w;
     uint16_t *h_out;        // gate/up: [M, N] bf16, pair-permuted inside 8-element chunks
-    float *ys;              // down: [n_slots, N] f32, routing weight applied
+    uint16_t *ys;           // down: [n_slots, N] bf16, routing weight applied
     int small_rows;         // blocks with at most this many real rows are left to the register-fed path
 };
 
 void launch_route_topk(const float *logits, int T, int E, int k, int32_t *ids, float *w, cudaStream_t s);
 void launch_align(const int32_t *topk_ids, int n, int E, int B, int32_t *sorted_ids, int32_t *expert_ids,
                   int32_t *ntp, cudaStream_t s);
-void launch_combine(const float *ys, int T, int k, int H, uint16_t *out, int num_sms, cudaStream_t s);
+void launch_combine(const uint16_t *ys, int T, int k, int H, uint16_t *out, int num_sms, cudaStream_t s);
 void launch_fp8_act_quant(const uint16_t *x, int rows, int cols, uint8_t *q, float *s, cudaStream_t st);
 void launch_w4a16_grouped_mma(const W4GroupedArgs &a, int mode, int block_m, int max_blocks, cudaStream_t s);
 void launch_fp8_grouped_mma(const F8GroupedArgs &a, int mode, int block_m, int max_blocks, cudaStream_t s);

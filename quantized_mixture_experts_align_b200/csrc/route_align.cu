@@ -172,33 +172,40 @@ void launch_align(const int32_t *topk_ids, int n, int E, int B, int32_t *sorted_
 }
 
 // ------------------------------------------------------------------------------------------
-// Top-k weighted combine: out[t, :] = bf16( sum_j ys[t*k + j, :] ), the slot rows already
+// Top-k weighted combine: out[t, :] = bf16( sum_j ys[t*k + j, :] ), the slot rows (bf16) already
 // carrying their routing weight. f32 sums in slot order.
 // ------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ ys, int T, int k, int H,
+__global__ void __launch_bounds__(256) combine_kernel(const uint16_t *__restrict__ ys, int T, int k, int H,
                                                       uint16_t *__restrict__ out)
 {
-    const int H4 = H / 4;
-    const long total = (long)T * H4;
+    const int H8 = H / 8;
+    const long total = (long)T * H8;
     for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < total; i += (long)gridDim.x * blockDim.x) {
-        const long t = i / H4;
-        const int c = (int)(i - t * H4);
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        const long t = i / H8;
+        const int c = (int)(i - t * H8);
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         for (int j = 0; j < k; ++j) {
-            const float4 v = __ldg(reinterpret_cast<const float4 *>(ys + ((size_t)t * k + j) * H) + c);
-            acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(ys + ((size_t)t * k + j) * H) + c);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                acc[2 * q] += __uint_as_float(w[q] << 16);
+                acc[2 * q + 1] += __uint_as_float(w[q] & 0xFFFF0000u);
+            }
         }
-        uint2 o;
-        o.x = pack_bf16x2(acc.x, acc.y);
-        o.y = pack_bf16x2(acc.z, acc.w);
-        reinterpret_cast<uint2 *>(out + (size_t)t * H)[c] = o;
+        uint4 o;
+        o.x = pack_bf16x2(acc[0], acc[1]);
+        o.y = pack_bf16x2(acc[2], acc[3]);
+        o.z = pack_bf16x2(acc[4], acc[5]);
+        o.w = pack_bf16x2(acc[6], acc[7]);
+        reinterpret_cast<uint4 *>(out + (size_t)t * H)[c] = o;
     }
 }
 
-void launch_combine(const float *ys, int T, int k, int H, uint16_t *out, int num_sms, cudaStream_t s)
+void launch_combine(const uint16_t *ys, int T, int k, int H, uint16_t *out, int num_sms, cudaStream_t s)
 {
     if (T <= 0) return;
-    const long total = (long)T * (H / 4);
+    const long total = (long)T * (H / 8);
     const int blocks = (int)((total + 255) / 256 < (long)num_sms * 8 ? (total + 255) / 256 : (long)num_sms * 8);
     combine_kernel<<<blocks, 256, 0, s>>>(ys, T, k, H, out);
 }

@@ -26,7 +26,7 @@
 //              a = silu(g) * u and quantizes it per row and 128-feature group to E4M3 + f32 scale
 //              (the two column halves of a row meet through shared memory for the group max);
 //   TC_DOWN    B = 256 rows of W2[e]; the epilogue multiplies by the slot's routing weight and
-//              writes the f32 slot row for the combine.
+//              writes the bf16 slot row for the combine.
 #include "kernels.cuh"
 #include "tc_common.cuh"
 
@@ -315,11 +315,16 @@ __global__ void __launch_bounds__(fp8_threads(MODE), 1)
             const int slot = __ldg(a.sorted_ids + m);
             if (ok && slot < a.n_slots) {
                 const float wt = __ldg(a.topk_w + slot);
-                float *yrow = a.ys + (size_t)slot * a.N + n0 + cq * COLS;
+                uint16_t *yrow = a.ys + (size_t)slot * a.N + n0 + cq * COLS;
 #pragma unroll
-                for (int j = 0; j < COLS; j += 4)
-                    *reinterpret_cast<float4 *>(yrow + j) =
-                        make_float4(wt * acc[j], wt * acc[j + 1], wt * acc[j + 2], wt * acc[j + 3]);
+                for (int j = 0; j < COLS; j += 8) {
+                    uint4 v;
+                    v.x = pack_bf16x2(wt * acc[j], wt * acc[j + 1]);
+                    v.y = pack_bf16x2(wt * acc[j + 2], wt * acc[j + 3]);
+                    v.z = pack_bf16x2(wt * acc[j + 4], wt * acc[j + 5]);
+                    v.w = pack_bf16x2(wt * acc[j + 6], wt * acc[j + 7]);
+                    *reinterpret_cast<uint4 *>(yrow + j) = v;
+                }
             }
         }
     }

@@ -37,7 +37,7 @@
 //               tensor-memory
 //               stages; then the epilogue: gate/up passes the up values through shared memory
 //               to the warps holding the gate values, which write h = bf16(silu(g) * u) in the
-//               permuted order; down writes the routing-weighted f32 slot rows.
+//               permuted order; down writes the routing-weighted bf16 slot rows.
 #include "kernels.cuh"
 #include "tc_common.cuh"
 
@@ -292,7 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
                 for (int j = 0; j < 32; ++j) {
                     const int slot = __shfl_sync(0xFFFFFFFFu, my_slot, j);
                     const float wt = __shfl_sync(0xFFFFFFFFu, my_w, j);
-                    if (slot < a.n_slots) a.ys[(size_t)slot * a.N + n0 + row] = wt * __uint_as_float(y[j]);
+                    if (slot < a.n_slots) a.ys[(size_t)slot * a.N + n0 + row] = f32_to_bf16(wt * __uint_as_float(y[j]));
                 }
             }
         }

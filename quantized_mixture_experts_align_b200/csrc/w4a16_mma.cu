@@ -214,11 +214,11 @@ __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4Grouped
                 h[rowA + g + 8] = f32_to_bf16(silu_f32(accA[s][2 + c]) * accB[s][2 + c]);
             } else {
                 const float wt = __ldg(a.topk_w + slot);
-                float *y = a.y_out + (size_t)slot * a.n_out;
-                y[rowA + g] = wt * accA[s][c];
-                y[rowA + g + 8] = wt * accA[s][2 + c];
-                y[rowB + g] = wt * accB[s][c];
-                y[rowB + g + 8] = wt * accB[s][2 + c];
+                uint16_t *y = a.y_out + (size_t)slot * a.n_out;
+                y[rowA + g] = f32_to_bf16(wt * accA[s][c]);
+                y[rowA + g + 8] = f32_to_bf16(wt * accA[s][2 + c]);
+                y[rowB + g] = f32_to_bf16(wt * accB[s][c]);
+                y[rowB + g + 8] = f32_to_bf16(wt * accB[s][2 + c]);
             }
         }
     }

@@ -44,7 +44,7 @@ def test_version(L):
 def test_workspace_sizes(L):
     a = moeq.moe_w4a16_workspace_size(32, 7168, 2048, 384, 8)
     n = 32 * 8
-    assert a >= n * 2048 * 2 + n * 7168 * 4                   # h + weighted slot outputs
+    assert a >= n * 2048 * 2 + n * 7168 * 2                   # h + weighted slot outputs (both bf16)
     assert moeq.moe_w4a16_workspace_size(8192, 7168, 2048, 384, 8) > a
     assert moeq.moe_w8a8_block_fp8_workspace_size(4096, 7168, 2048, 256, 8) > 0
     assert moeq.moe_w4a16_workspace_size(32, 100, 2048, 384, 8) == 0      # unsupported H

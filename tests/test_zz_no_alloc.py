@@ -40,9 +40,9 @@ def test_noalloc_forward_matches_workspace_forward_on_two_calls():
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
     H, I, E, k = 7168, 2048, 384, 8
-    assert moeq.moe_w4a16_workspace_size(63, H, I, E, k) <= 16 << 20 < moeq.moe_w4a16_workspace_size(64, H, I, E, k)
-    x = torch.zeros((64, H), dtype=torch.bfloat16, device=DEV)
-    logits = torch.zeros((64, E), device=DEV)
+    assert moeq.moe_w4a16_workspace_size(113, H, I, E, k) <= 16 << 20 < moeq.moe_w4a16_workspace_size(114, H, I, E, k)
+    x = torch.zeros((114, H), dtype=torch.bfloat16, device=DEV)
+    logits = torch.zeros((114, E), device=DEV)
     # rejected before any device work, so the weight contents do not matter
     w13q = torch.empty((E, 2 * I, H // 8), dtype=torch.int32, device=DEV)
     w13s = torch.empty((E, 2 * I, H // 32), dtype=torch.bfloat16, device=DEV)
