@@ -76,10 +76,18 @@ MOEQ_API int moe_route_topk(const float *logits, int T, int E, int k, int32_t *t
  *   expert_ids i32 [ceil((T*k + E*(block_m-1)) / block_m)] out: expert of each block of
  *              block_m entries, -1 past num_tokens_padded
  *   num_tokens_padded i32 [1] out: sum over experts of ceil(count / block_m) * block_m
+ *   ws, ws_bytes: caller-owned device scratch (256-byte aligned) of moe_align_workspace_size()
+ *              bytes; with it, more than 8192 slots are aligned by many CTAs (per-chunk counts,
+ *              one scan, per-chunk stable scatter), without it (NULL / too small) by one CTA.
+ *              Same result either way.
  * Bit-exact (integer). Limits: 1 <= block_m <= 256, E <= 1024, T*k <= 2^24.
  */
 MOEQ_API int moe_align(const int32_t *topk_ids, int T, int k, int E, int block_m, int32_t *sorted_ids,
-              int32_t *expert_ids, int32_t *num_tokens_padded, void *stream);
+              int32_t *expert_ids, int32_t *num_tokens_padded, void *ws, size_t ws_bytes, void *stream);
+
+/* Scratch bytes moe_align uses for T*k slots over E experts (0: none needed; 0 also for invalid
+ * arguments, which moe_align itself rejects). */
+MOEQ_API size_t moe_align_workspace_size(int T, int k, int E);
 
 /*
  * Per-token, per-128-column-group FP8 quantization of activations ([SGL], "Background": As is

@@ -30,7 +30,8 @@ _SIGNATURES = {
     "moe_last_error": ([], ctypes.c_char_p),
     "moe_version": ([], ctypes.c_char_p),
     "moe_route_topk": ([_V, _I, _I, _I, _V, _V, _V], _I),
-    "moe_align": ([_V, _I, _I, _I, _I, _V, _V, _V, _V], _I),
+    "moe_align": ([_V, _I, _I, _I, _I, _V, _V, _V, _V, _Z, _V], _I),
+    "moe_align_workspace_size": ([_I, _I, _I], _Z),
     "moe_fp8_act_quant": ([_V, _I, _I, _V, _V, _V], _I),
     "moe_w4a16_workspace_size": ([_I, _I, _I, _I, _I], _Z),
     "moe_w4a16_forward": ([_V, _V, _I, _I, _I, _I, _I, _V, _V, _V, _V, _V, _V, _V, _V, _Z, _V], _I),
@@ -104,15 +105,25 @@ def moe_route_topk(logits: torch.Tensor, k: int, topk_ids=None, topk_w=None, str
     return topk_ids, topk_w
 
 
-def moe_align(topk_ids: torch.Tensor, E: int, block_m: int, stream=None):
+def moe_align_workspace_size(T: int, k: int, E: int) -> int:
+    return int(lib().moe_align_workspace_size(T, k, E))
+
+
+def moe_align(topk_ids: torch.Tensor, E: int, block_m: int, ws=None, stream=None):
+    """ws: None allocates the scratch moe_align_workspace_size asks for; pass an empty tensor to
+    run without scratch (the one-CTA kernel)."""
     T, k = topk_ids.shape
     cap = T * k + E * (block_m - 1)
     dev = topk_ids.device
     sorted_ids = torch.empty(cap, dtype=torch.int32, device=dev)
     expert_ids = torch.empty(-(-cap // block_m), dtype=torch.int32, device=dev)
     ntp = torch.empty(1, dtype=torch.int32, device=dev)
+    if ws is None:
+        ws = workspace(moe_align_workspace_size(T, k, E), dev)
+    nbytes = ws.numel() * ws.element_size()
     _check(lib().moe_align(_dev(topk_ids, "topk_ids", torch.int32), T, k, E, block_m, _dev(sorted_ids, "sorted_ids"),
-                           _dev(expert_ids, "expert_ids"), _dev(ntp, "ntp"), _stream(stream)))
+                           _dev(expert_ids, "expert_ids"), _dev(ntp, "ntp"), _dev(ws, "ws") if nbytes else None,
+                           nbytes, _stream(stream)))
     return sorted_ids, expert_ids, ntp
 
 

@@ -144,6 +144,7 @@ struct RouteBufs {
     int32_t *sorted;
     int32_t *eids;
     int32_t *ntp;
+    int32_t *scratch;  // per-chunk expert counts of the many-CTA alignment (null: one-CTA kernel)
     int block_m;
     int max_blocks;
 };
@@ -160,6 +161,8 @@ static RouteBufs carve_route(Carve &c, long T, int k, int E, int block_m)
     r.sorted = c.take<int32_t>(cap);
     r.eids = c.take<int32_t>((size_t)r.max_blocks);
     r.ntp = c.take<int32_t>(1);
+    const size_t sb = align_scratch_bytes((int)n, E);
+    r.scratch = sb ? c.take<int32_t>(sb / sizeof(int32_t)) : nullptr;
     return r;
 }
 
@@ -275,8 +278,14 @@ int moe_route_topk(const float *logits, int T, int E, int k, int32_t *topk_ids, 
     return check_launch("moe_route_topk");
 }
 
+size_t moe_align_workspace_size(int T, int k, int E)
+{
+    if (T < 0 || k < 1 || E < 1 || E > kMaxExperts || (long)T * k > (1L << 24)) return 0;
+    return align_scratch_bytes(T * k, E);
+}
+
 int moe_align(const int32_t *topk_ids, int T, int k, int E, int block_m, int32_t *sorted_ids, int32_t *expert_ids,
-              int32_t *num_tokens_padded, void *stream)
+              int32_t *num_tokens_padded, void *ws, size_t ws_bytes, void *stream)
 {
     g_err[0] = 0;
     if (T < 0 || k < 1) return set_error(MOEQ_ERR_INVALID_ARG, "need T >= 0 and k >= 1 (got T=%d, k=%d)", T, k);
@@ -287,7 +296,12 @@ int moe_align(const int32_t *topk_ids, int T, int k, int E, int block_m, int32_t
     MOEQ_REQUIRE(expert_ids);
     MOEQ_REQUIRE(num_tokens_padded);
     if (T > 0) MOEQ_REQUIRE(topk_ids);
-    launch_align(topk_ids, T * k, E, block_m, sorted_ids, expert_ids, num_tokens_padded, (cudaStream_t)stream);
+    const size_t need = align_scratch_bytes(T * k, E);
+    if (need && ws && (reinterpret_cast<uintptr_t>(ws) & 255))
+        return set_error(MOEQ_ERR_INVALID_ARG, "ws must be 256-byte aligned");
+    int32_t *scratch = (need && ws && ws_bytes >= need) ? static_cast<int32_t *>(ws) : nullptr;
+    launch_align(topk_ids, T * k, E, block_m, sorted_ids, expert_ids, num_tokens_padded, scratch,
+                 (cudaStream_t)stream);
     return check_launch("moe_align");
 }
 
@@ -349,7 +363,7 @@ int moe_w4a16_forward(const uint16_t *x, const float *logits, int T, int H, int 
     }
     {
         trace::Scope ts(trace::ALIGN, s);
-        launch_align(ids, n, E, r.block_m, r.sorted, r.eids, r.ntp, s);
+        launch_align(ids, n, E, r.block_m, r.sorted, r.eids, r.ntp, r.scratch, s);
     }
 
     if (tcp) {
@@ -358,7 +372,7 @@ int moe_w4a16_forward(const uint16_t *x, const float *logits, int T, int H, int 
         const int cap = r.max_blocks * r.block_m;
         {
             trace::Scope ts(trace::ACT_QUANT, s);  // the activation gather takes the act-prep slot
-            launch_gather_bf16_perm(x, H, k, r.sorted, r.ntp, n, cap, xg, num_sms(), s);
+            launch_gather_bf16_perm(x, H, k, r.sorted, r.ntp, n, cap, kW4SmallRows, xg, num_sms(), s);
         }
         W4TcArgs t{};
         t.status = status;
@@ -508,7 +522,7 @@ int moe_w8a8_block_fp8_forward(const uint16_t *x, const float *logits, int T, in
     }
     {
         trace::Scope ts(trace::ALIGN, s);
-        launch_align(ids, n, E, r.block_m, r.sorted, r.eids, r.ntp, s);
+        launch_align(ids, n, E, r.block_m, r.sorted, r.eids, r.ntp, r.scratch, s);
     }
     {
         trace::Scope ts(trace::ACT_QUANT, s);

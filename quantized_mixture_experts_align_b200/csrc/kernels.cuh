@@ -89,8 +89,11 @@ struct W4TcArgs {
 };
 
 void launch_route_topk(const float *logits, int T, int E, int k, int32_t *ids, float *w, cudaStream_t s);
+// Scratch (bytes) the alignment of n slots over E experts uses; 0 = the one-CTA kernel, which
+// also runs when launch_align gets no scratch.
+size_t align_scratch_bytes(int n, int E);
 void launch_align(const int32_t *topk_ids, int n, int E, int B, int32_t *sorted_ids, int32_t *expert_ids,
-                  int32_t *ntp, cudaStream_t s);
+                  int32_t *ntp, int32_t *scratch, cudaStream_t s);
 void launch_combine(const uint16_t *ys, int T, int k, int H, uint16_t *out, int num_sms, cudaStream_t s);
 void launch_fp8_act_quant(const uint16_t *x, int rows, int cols, uint8_t *q, float *s, cudaStream_t st);
 void launch_w4a16_grouped_mma(const W4GroupedArgs &a, int mode, int block_m, int max_blocks, cudaStream_t s);
@@ -107,7 +110,7 @@ int launch_fp8_tc_grouped(const Fp8TcArgs &a, int mode, const uint8_t *A, const 
 // TC_GATEUP (h = silu(gate) * up, written pair-permuted) or TC_DOWN (weighted slot rows).
 int launch_w4a16_tc(const W4TcArgs &a, int mode, const uint16_t *act, int max_blocks, cudaStream_t s);
 void launch_gather_bf16_perm(const uint16_t *x, int H, int k, const int32_t *sorted_ids, const int32_t *ntp,
-                             int n_slots, int cap_rows, uint16_t *xg, int num_sms, cudaStream_t s);
+                             int n_slots, int cap_rows, int small_rows, uint16_t *xg, int num_sms, cudaStream_t s);
 // Copies E4M3 rows (and their scales) of the routed slots into aligned order: row r takes token
 // sorted_ids[r] / k; padding rows become zero.
 void launch_gather_fp8_rows(const uint8_t *xq, const float *xs, int H, int k, const int32_t *sorted_ids,

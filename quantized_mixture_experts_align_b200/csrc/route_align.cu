@@ -165,9 +165,144 @@ __global__ void __launch_bounds__(kAlignThreads) align_kernel(const int32_t *__r
     }
 }
 
-void launch_align(const int32_t *topk_ids, int n, int E, int B, int32_t *sorted_ids, int32_t *expert_ids,
-                  int32_t *ntp, cudaStream_t s)
+// ------------------------------------------------------------------------------------------
+// Alignment over many CTAs (large T*k), same result as align_kernel:
+//  1. align_count_kernel: chunk c of kChunk slots -> its per-expert counts hist[c][e]
+//     (warp-aggregated shared-memory atomics: one atomic per expert and warp);
+//  2. align_scan_kernel (one CTA): per expert, the totals and the exclusive prefix over chunks;
+//     the padded scan gives each expert's offset; hist[c][e] becomes the position of chunk c's
+//     first slot of expert e; expert_ids, pads, tail and num_tokens_padded are written;
+//  3. align_scatter_kernel: chunk c places its slots at hist[c][e] + their stable rank within
+//     the chunk (tiles of 256 slots as in align_kernel).
+// ------------------------------------------------------------------------------------------
+constexpr int kChunkThreads = 256;
+constexpr int kChunkWarps = kChunkThreads / 32;
+constexpr int kChunk = 2048;  // slots per chunk (8 tiles of 256)
+constexpr int kAlignOneCtaMax = 8192;  // up to this many slots the one-CTA kernel is faster
+
+__global__ void __launch_bounds__(kChunkThreads) align_count_kernel(const int32_t *__restrict__ topk_ids, int n,
+                                                                   int E, int32_t *__restrict__ hist)
 {
+    __shared__ int cnt[kMaxExperts];
+    const int tid = threadIdx.x, lane = tid & 31;
+    for (int e = tid; e < E; e += kChunkThreads) cnt[e] = 0;
+    __syncthreads();
+    const int f0 = blockIdx.x * kChunk;
+    for (int i = tid; i < kChunk; i += kChunkThreads) {
+        const int f = f0 + i;
+        int e = (f < n) ? __ldg(topk_ids + f) : -1;
+        if (e < 0 || e >= E) e = -1;
+        const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
+        if (e >= 0 && (peers & ((1u << lane) - 1u)) == 0u) atomicAdd(&cnt[e], __popc(peers));
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += kChunkThreads) hist[(size_t)blockIdx.x * E + e] = cnt[e];
+}
+
+__global__ void __launch_bounds__(kAlignThreads) align_scan_kernel(int n, int E, int B, int n_chunks,
+                                                                  int32_t *__restrict__ hist,
+                                                                  int32_t *__restrict__ sorted_ids,
+                                                                  int32_t *__restrict__ expert_ids,
+                                                                  int32_t *__restrict__ num_tokens_padded)
+{
+    __shared__ int warp_sums[kAlignWarps];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    int cnt = 0;
+    if (tid < E)
+        for (int c = 0; c < n_chunks; ++c) cnt += hist[(size_t)c * E + tid];
+    const int padded = (tid < E) ? (cnt + B - 1) / B * B : 0;
+    int incl = padded;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int ws = warp_sums[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xFFFFFFFFu, ws, o);
+            if (lane >= o) ws += y;
+        }
+        warp_sums[lane] = ws;
+    }
+    __syncthreads();
+    const int excl = incl - padded + (warp > 0 ? warp_sums[warp - 1] : 0);
+    const int total = warp_sums[kAlignWarps - 1];
+    if (tid == 0) *num_tokens_padded = total;
+    const long cap = (long)n + (long)E * (B - 1);
+    const long nblk = (cap + B - 1) / B;
+    if (tid < E) {
+        int pos = excl;  // chunk c's first slot of this expert
+        for (int c = 0; c < n_chunks; ++c) {
+            const int h = hist[(size_t)c * E + tid];
+            hist[(size_t)c * E + tid] = pos;
+            pos += h;
+        }
+        for (int i = excl + cnt; i < excl + padded; ++i) sorted_ids[i] = n;
+        for (int b = excl / B; b < (excl + padded) / B; ++b) expert_ids[b] = tid;
+    }
+    for (long i = total + tid; i < cap; i += kAlignThreads) sorted_ids[i] = n;
+    for (long b = total / B + tid; b < nblk; b += kAlignThreads) expert_ids[b] = -1;
+}
+
+__global__ void __launch_bounds__(kChunkThreads) align_scatter_kernel(const int32_t *__restrict__ topk_ids, int n,
+                                                                     int E, const int32_t *__restrict__ base,
+                                                                     int32_t *__restrict__ sorted_ids)
+{
+    __shared__ int cursor[kMaxExperts];
+    __shared__ uint8_t hist[kMaxExperts][kChunkWarps];  // per tile: count of expert e in warp w
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int32_t *my_base = base + (size_t)blockIdx.x * E;
+    for (int e = tid; e < E; e += kChunkThreads) {
+        cursor[e] = __ldg(my_base + e);
+#pragma unroll
+        for (int w = 0; w < kChunkWarps; ++w) hist[e][w] = 0;
+    }
+    __syncthreads();
+    const unsigned lt_mask = (1u << lane) - 1u;
+    const int f0 = blockIdx.x * kChunk;
+    for (int t0 = 0; t0 < kChunk; t0 += kChunkThreads) {
+        const int f = f0 + t0 + tid;
+        int e = (f < n) ? __ldg(topk_ids + f) : -1;
+        if (e < 0 || e >= E) e = -1;
+        const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
+        const int rank = __popc(peers & lt_mask);
+        const bool leader = (peers & lt_mask) == 0u;
+        if (e >= 0 && leader) hist[e][warp] = (uint8_t)__popc(peers);
+        __syncthreads();
+        if (e >= 0) {
+            int before = 0;
+#pragma unroll
+            for (int w = 0; w < kChunkWarps; ++w) before += (w < warp) ? hist[e][w] : 0;
+            sorted_ids[cursor[e] + before + rank] = f;
+        }
+        __syncthreads();
+        if (e >= 0 && leader) {
+            atomicAdd(&cursor[e], __popc(peers));
+            hist[e][warp] = 0;
+        }
+        __syncthreads();
+    }
+}
+
+size_t align_scratch_bytes(int n, int E)
+{
+    return n > kAlignOneCtaMax ? (size_t)cdiv(n, kChunk) * E * sizeof(int32_t) : 0;
+}
+
+void launch_align(const int32_t *topk_ids, int n, int E, int B, int32_t *sorted_ids, int32_t *expert_ids,
+                  int32_t *ntp, int32_t *scratch, cudaStream_t s)
+{
+    if (n > kAlignOneCtaMax && scratch) {
+        const int chunks = cdiv(n, kChunk);
+        align_count_kernel<<<chunks, kChunkThreads, 0, s>>>(topk_ids, n, E, scratch);
+        align_scan_kernel<<<1, kAlignThreads, 0, s>>>(n, E, B, chunks, scratch, sorted_ids, expert_ids, ntp);
+        align_scatter_kernel<<<chunks, kChunkThreads, 0, s>>>(topk_ids, n, E, scratch, sorted_ids);
+        return;
+    }
     align_kernel<<<1, kAlignThreads, 0, s>>>(topk_ids, n, E, B, sorted_ids, expert_ids, ntp);
 }
 

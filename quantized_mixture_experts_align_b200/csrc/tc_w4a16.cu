@@ -304,17 +304,25 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
 }
 
 // Gather of bf16 activation rows into aligned order with the pair permutation inside every
-// 8-element chunk; one warp per row, padding rows zero.
+// 8-element chunk; one warp per row. Only the rows the MMAs read are written: the real rows and
+// the zero padding up to the block's real count rounded up to 16 (the MMA's N); blocks with at
+// most small_rows real rows belong to the register-fed kernel, which reads x itself.
 __global__ void __launch_bounds__(256) gather_bf16_perm_kernel(const uint16_t *__restrict__ x, int H, int k,
                                                                const int32_t *__restrict__ sorted_ids,
                                                                const int32_t *__restrict__ ntp, int n_slots,
-                                                               int cap_rows, uint16_t *__restrict__ xg)
+                                                               int cap_rows, int small_rows,
+                                                               uint16_t *__restrict__ xg)
 {
     const int lane = threadIdx.x & 31;
     const int rows = min(__ldg(ntp), cap_rows);
     for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += gridDim.x * (blockDim.x >> 5)) {
         const int slot = __ldg(sorted_ids + r);
         const bool real = slot < n_slots;
+        // real rows come first in a block: a 16-row group is read iff its first row is real, and
+        // the block is the register-fed kernel's iff its row small_rows is padding
+        const int blk0 = r & ~(kTok - 1);
+        if (!real && __ldg(sorted_ids + (r & ~15)) >= n_slots) continue;
+        if (small_rows > 0 && __ldg(sorted_ids + blk0 + small_rows) >= n_slots) continue;
         const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)(real ? slot / k : 0) * H);
         uint4 *dst = reinterpret_cast<uint4 *>(xg + (size_t)r * H);
         for (int i = lane; i < H / 8; i += 32) {
@@ -359,11 +367,11 @@ int launch_w4a16_tc(const W4TcArgs &a, int mode, const uint16_t *act, int max_bl
 }
 
 void launch_gather_bf16_perm(const uint16_t *x, int H, int k, const int32_t *sorted_ids, const int32_t *ntp,
-                             int n_slots, int cap_rows, uint16_t *xg, int num_sms, cudaStream_t s)
+                             int n_slots, int cap_rows, int small_rows, uint16_t *xg, int num_sms, cudaStream_t s)
 {
     if (cap_rows <= 0) return;
     const int blocks = min(cdiv(cap_rows, 8), num_sms * 8);
-    gather_bf16_perm_kernel<<<blocks, 256, 0, s>>>(x, H, k, sorted_ids, ntp, n_slots, cap_rows, xg);
+    gather_bf16_perm_kernel<<<blocks, 256, 0, s>>>(x, H, k, sorted_ids, ntp, n_slots, cap_rows, small_rows, xg);
 }
 
 }  // namespace moeq

@@ -65,9 +65,9 @@ def test_validation_rejects_before_device_work(L):
     assert _rc(L, "moe_route_topk", N, 4, 64, 8, N, N, N) == moeq.MOEQ_ERR_INVALID_ARG   # NULL logits
     assert b"logits" in L.moe_last_error()
     # align: bad block size, negative T, NULL outputs
-    assert _rc(L, "moe_align", N, 3, 2, 3, 0, N, N, N, N) == moeq.MOEQ_ERR_UNSUPPORTED
-    assert _rc(L, "moe_align", N, -1, 2, 3, 4, N, N, N, N) == moeq.MOEQ_ERR_INVALID_ARG
-    assert _rc(L, "moe_align", N, 3, 2, 3, 4, N, N, N, N) == moeq.MOEQ_ERR_INVALID_ARG
+    assert _rc(L, "moe_align", N, 3, 2, 3, 0, N, N, N, N, 0, N) == moeq.MOEQ_ERR_UNSUPPORTED
+    assert _rc(L, "moe_align", N, -1, 2, 3, 4, N, N, N, N, 0, N) == moeq.MOEQ_ERR_INVALID_ARG
+    assert _rc(L, "moe_align", N, 3, 2, 3, 4, N, N, N, N, 0, N) == moeq.MOEQ_ERR_INVALID_ARG
     # act quant: ragged columns
     assert _rc(L, "moe_fp8_act_quant", N, 4, 100, N, N, N) == moeq.MOEQ_ERR_UNSUPPORTED
     # forward: unsupported H / I, workspace too small, misaligned workspace

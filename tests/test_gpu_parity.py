@@ -106,6 +106,29 @@ def test_align_edges():
     _check_align(torch.zeros((0, 2), dtype=torch.int32, device=DEV), 4, 8)
 
 
+@pytest.mark.parametrize("B", [1, 8, 64, 128, 256])
+def test_align_many_cta_matches_one_cta_and_oracle(B):
+    """Past 8192 slots the alignment runs over many CTAs (per-chunk counts, scan, per-chunk stable
+    scatter); it must equal the oracle and the one-CTA kernel (run without scratch) exactly:
+    ragged chunk tails, one expert taking most slots (Zipf), E = 1024."""
+    g = torch.Generator(device="cpu").manual_seed(31)
+    cases = [
+        (W.router_logits(W.WORKLOADS["prefill_w4a16"], 3001, 384, device=DEV), 384, 8),   # 24008 slots
+        (torch.randn((2500, 1024), generator=g).to(DEV), 1024, 4),                        # 10000 slots
+    ]
+    for logits, E, k in cases:
+        ids, _ = moeq.moe_route_topk(logits, k)
+        assert moeq.moe_align_workspace_size(ids.shape[0], k, E) > 0
+        _check_align(ids, E, B)
+        s0, e0, n0 = moeq.moe_align(ids, E, B, ws=torch.empty(0, dtype=torch.uint8, device=DEV))
+        s1, e1, n1 = moeq.moe_align(ids, E, B)
+        torch.cuda.synchronize()
+        assert torch.equal(s0, s1) and torch.equal(e0, e1) and torch.equal(n0, n1)
+    skew = torch.zeros((9000, 1), dtype=torch.int32)
+    skew[::7] = 5
+    _check_align(skew.to(DEV), 8, B)
+
+
 # --------------------------------------------------------------------------------------------
 # FP8 activation quantizer (bit-exact: same IEEE division and RNE rounding)
 # --------------------------------------------------------------------------------------------
