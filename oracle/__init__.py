@@ -135,6 +135,23 @@ def fp8_block_matmul(A, As, B, Bs, rows=None):
     return C
 
 
+def grouped_w4a16(A, wq, ws, expert_of_row, rows=None):
+    """C rows (float64 [len(rows), N]) of the grouped W4A16 GEMM: row m times the dequantized
+    weights of expert expert_of_row[m] (zeros where it is -1). A bf16 bits [M, K]; wq int32
+    [G, N, K/8]; ws bf16 bits [G, N, K/32]."""
+    A = np.ascontiguousarray(A, dtype=np.uint16)
+    wq = np.ascontiguousarray(wq, dtype=np.int32)
+    ws = np.ascontiguousarray(ws, dtype=np.uint16)
+    eor = np.ascontiguousarray(expert_of_row, dtype=np.int32)
+    M, K = A.shape
+    G, N = wq.shape[0], wq.shape[1]
+    r = _tokens(rows, M)
+    C = np.zeros((len(r), N), np.float64)
+    _check(lib().orc_grouped_w4a16(_p(A), M, K, _p(wq), _p(ws), G, N, _p(eor), _p(r), len(r), _p(C)),
+           "grouped_w4a16")
+    return C
+
+
 # ---- format primitives (for the pins) ------------------------------------------------------
 
 def bf16_round(v: np.ndarray) -> np.ndarray:

@@ -410,6 +410,39 @@ int orc_fp8_block_matmul(const uint8_t *A, const float *As, const uint8_t *B, co
 }
 
 /* ------------------------------------------------------------------------------------------ */
+/* Grouped W4A16 GEMM ([CHORD], "SM90 grouped kernels": the contiguous layout concatenates the
+ * rows of each expert, padded to 128-row boundaries, with m_indices holding each row's expert
+ * and -1 on padding; the masked layout gives every expert a fixed budget of max_m rows of which
+ * masked_m are real, and consumers ignore the rest). Both are, per real row m with expert e:
+ *   C[m, n] = sum_c A[m, c] * ((q[e, n, c] - 8) * s[e, n, c / 32])
+ * READING: the pages print no formula; this is the plain product of the activation row with the
+ * dequantized weights of its expert, A taken as exact bf16 values, in double. The expert of a
+ * row is given per row (expert_of_row, -1 = not computed), which covers both layouts.         */
+/* ------------------------------------------------------------------------------------------ */
+
+int orc_grouped_w4a16(const uint16_t *A, int M, int K, const int32_t *wq, const uint16_t *ws, int G, int N,
+                      const int32_t *expert_of_row, const int32_t *rows, int nrows, double *C)
+{
+    if (K % 32 || K < 32 || N < 1 || G < 1) return 1;
+    for (int i = 0; i < nrows; ++i)
+        if (rows[i] < 0 || rows[i] >= M) return 1;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int i = 0; i < nrows; ++i)
+        for (int n = 0; n < N; ++n) {
+            int m = rows[i];
+            int e = expert_of_row[m];
+            double acc = 0.0;
+            if (e >= 0 && e < G) {
+                const int32_t *q = wq + (size_t)e * N * (K / 8);
+                const uint16_t *sc = ws + (size_t)e * N * (K / 32);
+                for (int c = 0; c < K; ++c) acc += bf16_value(A[(size_t)m * K + c]) * w4_value(q, sc, K, n, c);
+            }
+            C[(size_t)i * N + n] = acc;
+        }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------------------------ */
 /* Format primitives exported for the pins                                                     */
 /* ------------------------------------------------------------------------------------------ */
 

@@ -270,6 +270,42 @@ def test_w4a16_dequant_matches_numpy_unpack():
     assert np.array_equal(oracle.w4a16_dequant(q, s), _np_unpack_w4(q, s))
 
 
+def test_grouped_w4a16_matches_numpy_on_numpy_unpacked_weights():
+    """Library special case: each row times its expert's weights, unpacked by numpy (not by the
+    oracle) and multiplied with float64 matmul; -1 rows are not computed (zeros)."""
+    d = W.make_moe(W.WORKLOADS["tiny_w4a16"], T=1, E=3, k=1, H=128, I=64)
+    wq, ws = W.np_bits(d["w13q"]), W.np_bits(d["w13s"])          # [3, 128, 16], [3, 128, 4]
+    g = np.random.default_rng(3)
+    A = _bf16_bits(torch.from_numpy(g.standard_normal((9, 128)).astype(np.float32)).to(torch.bfloat16))
+    eor = np.array([0, 0, 2, -1, 1, 2, -1, 0, 1], np.int32)
+    got = oracle.grouped_w4a16(A, wq, ws, eor)
+    Ad = torch.from_numpy(A.view(np.int16)).view(torch.bfloat16).double().numpy()   # bits -> values (torch)
+    for m in range(9):
+        if eor[m] < 0:
+            assert np.all(got[m] == 0.0)
+            continue
+        ref = _np_unpack_w4(wq[eor[m]], ws[eor[m]]) @ Ad[m]
+        assert np.allclose(got[m], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_grouped_w4a16_closed_form_and_nibble_order():
+    """Codes all 9 with scale 0.5 and A of ones give K * 0.5; one code 10 at input column 37 (word
+    4, nibble 5) of row 3 of expert 1 adds exactly A[m, 37] * 0.5 there."""
+    G, N, K = 2, 4, 64
+    wq = np.full((G, N, K // 8), np.int32(np.uint32(0x99999999).view(np.int32)), np.int32)
+    ws = np.full((G, N, K // 32), 0x3F00, np.uint16)                        # bf16 0.5
+    A = np.full((3, K), 0x3F80, np.uint16)                                  # bf16 1.0
+    C = oracle.grouped_w4a16(A, wq, ws, np.array([0, 1, -1], np.int32))
+    assert np.all(C[0] == K * 0.5) and np.all(C[1] == K * 0.5) and np.all(C[2] == 0.0)
+    word = np.uint32(0x99999999) & ~np.uint32(0xF << 20) | np.uint32(0xA << 20)
+    wq[1, 3, 4] = np.int32(word.view(np.int32))
+    A[1, 37] = 0x4040                                                       # bf16 3.0
+    C = oracle.grouped_w4a16(A, wq, ws, np.array([0, 1, -1], np.int32))
+    # row 3: 63 columns of 1.0 * 0.5, column 37 of 3.0 * (10 - 8) * 0.5; row 2: column 37 at 0.5
+    assert C[1, 3] == (K - 1) * 0.5 + 3.0 * 1.0 and C[1, 2] == (K - 1) * 0.5 + 3.0 * 0.5
+    assert np.all(C[0] == K * 0.5)
+
+
 def test_w4a16_combine_weights_sum_to_one_on_workload_logits():
     for name in ("tiny_w4a16", "decode_w4a16", "prefill_w4a16", "moe_fp8"):
         wl = W.WORKLOADS[name]
