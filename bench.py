@@ -542,7 +542,44 @@ def main():
             "weight_gbs": pbytes / (pstep * 1e-3) / 1e9, "active_experts": int((prows > 0).sum()),
             "skew_aware_roof_ms": proof, "frac_of_skew_aware_roof": proof / pstep,
             "stages_ms": {k: v[0] / max(v[1], 1) for k, v in pst.items() if v[1]}}
-        del dp
+        # grouped W4A16 GEMM, contiguous layout: the prefill routing's rows per expert, each
+        # expert padded to 128 rows (m_indices -1), its W13 (N = 2I = 4096, K = H = 7168)
+        pad = [int(c) + (-int(c)) % 128 for c in prows]
+        m_idx = torch.cat([torch.cat([torch.full((int(c),), e, dtype=torch.int32),
+                                      torch.full((p - int(c),), -1, dtype=torch.int32)])
+                           for e, (c, p) in enumerate(zip(prows, pad)) if p]).cuda()
+        gA = W.bf16_normal((m_idx.numel(), dp["H"]), W.generator(90, 0, device="cuda"), "cuda")
+        gC = torch.empty((m_idx.numel(), 2 * dp["I"]), dtype=torch.bfloat16, device="cuda")
+        gws = moeq.workspace(moeq.lib().moe_w4a16_grouped_contiguous_workspace_size(
+            m_idx.numel(), dp["H"], 2 * dp["I"], dp["E"]), "cuda")
+        gms = timed_steps(lambda: moeq.moe_w4a16_grouped_contiguous(gA, dp["w13q"], dp["w13s"], m_idx, out=gC, ws=gws),
+                          max(3, args.steps // 4), 3, None, world)
+        gstep = max_over_ranks(statistics.mean(gms), world)
+        gfl = 2.0 * int(prows.sum()) * 2 * dp["I"] * dp["H"]
+        also["grouped_w4a16_contiguous"] = {
+            "workload": f"prefill routing rows per expert padded to 128 ({m_idx.numel()} rows), N=4096 K=7168, E=384",
+            "ms_per_step": gstep, "tflops": gfl / (gstep * 1e-3) / 1e12,
+            "frac_of_bf16_peak": gfl / (gstep * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"]}
+        del gA, gC, gws, m_idx, dp
+        torch.cuda.empty_cache()
+        # masked layout: the decode routing's rows per expert in budgets of 16 rows, expected_m 1
+        dd8 = W.make_moe(W.WORKLOADS["decode_w4a16"], device="cuda")
+        drows = expert_rows(moeq, dd8)
+        max_m = 16
+        masked = torch.as_tensor(np.minimum(drows, max_m).astype(np.int32)).cuda()
+        mA = W.bf16_normal((dd8["E"] * max_m, dd8["H"]), W.generator(91, 0, device="cuda"), "cuda")
+        mC = torch.empty((dd8["E"] * max_m, 2 * dd8["I"]), dtype=torch.bfloat16, device="cuda")
+        mws = moeq.workspace(moeq.lib().moe_w4a16_grouped_masked_workspace_size(
+            dd8["E"], max_m, dd8["H"], 2 * dd8["I"], 1), "cuda")
+        mms = timed_steps(lambda: moeq.moe_w4a16_grouped_masked(mA, dd8["w13q"], dd8["w13s"], masked, 1, out=mC, ws=mws),
+                          args.steps, 3, flush, world)
+        mstep = max_over_ranks(statistics.mean(mms), world)
+        mbytes = int((drows > 0).sum()) * (W.w4a16_expert_bytes(dd8["H"], dd8["I"]) * 2 // 3)
+        also["grouped_w4a16_masked"] = {
+            "workload": f"decode routing rows per expert in budgets of {max_m} rows, N=4096 K=7168, E=384, expected_m 1",
+            "ms_per_step": mstep, "weight_gbs": mbytes / (mstep * 1e-3) / 1e9,
+            "hbm_frac": mbytes / (mstep * 1e-3) / 1e9 / peaks["hbm_gbs"], "active_experts": int((drows > 0).sum())}
+        del mA, mC, mws, dd8
         torch.cuda.empty_cache()
         df = W.make_moe(W.WORKLOADS["moe_fp8"], device="cuda")
         fms, fst = run_fp8(moeq, df, max(3, args.steps // 4), 3, None, world)

@@ -164,6 +164,34 @@ MOEQ_API int moe_w8a8_block_fp8_forward(const uint16_t *x, const float *logits, 
                                float *topk_w_out, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * Grouped W4A16 GEMM on the layer's kernels, for callers that route themselves ([CHORD], "SM90
+ * grouped kernels": the contiguous prefill layout concatenates each expert's rows, padded to
+ * 128-row boundaries, with m_indices holding each row's expert and -1 on padding; the masked
+ * decode layout gives every expert a fixed budget of max_m rows, masked_m of them real, and
+ * consumers ignore the rest; expected_m is the host-side rows-per-expert hint that picks the
+ * launch). For every real row m with expert e:
+ *   C[m, n] = bf16( sum_c A[m, c] * (q[e, n, c] - 8) * s[e, n, c / 32] )   (f32 accumulation)
+ *   A    bf16 [M, K] (contiguous) or [G * max_m, K] (masked, expert e's rows at e * max_m)
+ *   w_q  i32 [G, N, K/8], w_s bf16 [G, N, K/32]: the layer's INT4 group-32 format
+ *   m_indices i32 [M] (contiguous): expert of each row in [0, G), -1 = padding (any order works;
+ *        the 128-row padding of the pages' layout is not required)
+ *   masked_m i32 [G] (masked, device): real rows per expert (values above max_m count as max_m)
+ *   C    bf16 [M, N] / [G * max_m, N] out; padding / masked-out rows are not written
+ *   ws, ws_bytes: device scratch (256-byte aligned) of the matching *_workspace_size() bytes
+ * Limits: K % 128 == 0, N % 128 == 0 (both >= 128), 1 <= G <= 1024, rows <= 2^24. Schedule as the
+ * layer's down GEMM: at >= 16 rows per expert (M / G, or expected_m) tcgen05 over 256-row blocks
+ * with blocks of <= 8 rows on the register-fed kernel, below that the register-fed kernel.
+ */
+MOEQ_API size_t moe_w4a16_grouped_contiguous_workspace_size(int M, int K, int N, int G);
+MOEQ_API int moe_w4a16_grouped_contiguous(const uint16_t *A, int M, int K, const int32_t *w_q, const uint16_t *w_s,
+                                          int G, int N, const int32_t *m_indices, uint16_t *C, void *ws,
+                                          size_t ws_bytes, void *stream);
+MOEQ_API size_t moe_w4a16_grouped_masked_workspace_size(int G, int max_m, int K, int N, int expected_m);
+MOEQ_API int moe_w4a16_grouped_masked(const uint16_t *A, int G, int max_m, int K, const int32_t *w_q,
+                                      const uint16_t *w_s, int N, const int32_t *masked_m, int expected_m, uint16_t *C,
+                                      void *ws, size_t ws_bytes, void *stream);
+
+/*
  * Dense block-FP8 matmul ([SGL], "Background": w8a8_block_fp8_matmul(A, B, As, Bs, block_size,
  * output_dtype)):  C[m, n] = sum_kb As[m, kb] * Bs[n/128, kb] * sum_{k in block kb} A[m,k] B[n,k]
  *   A e4m3 [M, K], As f32 [M, K/128], B e4m3 [N, K], Bs f32 [ceil(N/128), ceil(K/128)],

@@ -39,6 +39,10 @@ _SIGNATURES = {
     "moe_w8a8_block_fp8_workspace_size": ([_I, _I, _I, _I, _I], _Z),
     "moe_w8a8_block_fp8_forward": ([_V, _V, _I, _I, _I, _I, _I, _V, _V, _V, _V, _V, _V, _V, _V, _Z, _V], _I),
     "w8a8_block_fp8_matmul": ([_V, _V, _V, _V, _I, _I, _I, _I, _I, _V, _V], _I),
+    "moe_w4a16_grouped_contiguous_workspace_size": ([_I, _I, _I, _I], _Z),
+    "moe_w4a16_grouped_contiguous": ([_V, _I, _I, _V, _V, _I, _I, _V, _V, _V, _Z, _V], _I),
+    "moe_w4a16_grouped_masked_workspace_size": ([_I, _I, _I, _I, _I], _Z),
+    "moe_w4a16_grouped_masked": ([_V, _I, _I, _I, _V, _V, _I, _V, _I, _V, _V, _Z, _V], _I),
     "moe_trace_enable": ([_I], _I),
     "moe_trace_read": ([_V, _V, _I, _I], _I),
     "moe_device_status": ([_I], _I),
@@ -205,6 +209,38 @@ def w8a8_block_fp8_matmul(A, As, B, Bs, block_size=(128, 128), out=None, stream=
     _check(lib().w8a8_block_fp8_matmul(
         _dev(A, "A", _U8), _dev(As, "As", torch.float32), _dev(B, "B", _U8), _dev(Bs, "Bs", torch.float32),
         M, N, K, int(block_size[0]), int(block_size[1]), _dev(out, "out", _BF16), _stream(stream)))
+    return out
+
+
+def moe_w4a16_grouped_contiguous(A, w_q, w_s, m_indices, out=None, ws=None, stream=None):
+    """Grouped W4A16 GEMM, contiguous layout: C[m] = A[m] . dequant(W[m_indices[m]]) for rows with
+    m_indices >= 0 (other rows of out are left as they are). A bf16 [M, K]; w_q int32 [G, N, K/8];
+    w_s bf16 [G, N, K/32]; m_indices int32 [M]."""
+    M, K = A.shape
+    G, N = w_q.shape[0], w_q.shape[1]
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=A.device) if out is None else out
+    ws = workspace(lib().moe_w4a16_grouped_contiguous_workspace_size(M, K, N, G), A.device) if ws is None else ws
+    _check(lib().moe_w4a16_grouped_contiguous(
+        _dev(A, "A", _BF16), M, K, _dev(w_q, "w_q", torch.int32), _dev(w_s, "w_s", _BF16), G, N,
+        _dev(m_indices, "m_indices", torch.int32), _dev(out, "out", _BF16), _dev(ws, "ws"),
+        ws.numel() * ws.element_size(), _stream(stream)))
+    return out
+
+
+def moe_w4a16_grouped_masked(A, w_q, w_s, masked_m, expected_m, out=None, ws=None, stream=None):
+    """Grouped W4A16 GEMM, masked layout: A bf16 [G, max_m, K] (or [G * max_m, K]); the first
+    masked_m[e] rows of expert e's budget are computed, the rest of out is left as it is.
+    expected_m: host-side rows-per-expert hint for the launch. Returns out [G * max_m, N]."""
+    G, N = w_q.shape[0], w_q.shape[1]
+    K = A.shape[-1]
+    max_m = A.numel() // (G * K)
+    out = torch.empty((G * max_m, N), dtype=torch.bfloat16, device=A.device) if out is None else out
+    ws = workspace(lib().moe_w4a16_grouped_masked_workspace_size(G, max_m, K, N, expected_m), A.device) \
+        if ws is None else ws
+    _check(lib().moe_w4a16_grouped_masked(
+        _dev(A, "A", _BF16), G, max_m, K, _dev(w_q, "w_q", torch.int32), _dev(w_s, "w_s", _BF16), N,
+        _dev(masked_m, "masked_m", torch.int32), int(expected_m), _dev(out, "out", _BF16), _dev(ws, "ws"),
+        ws.numel() * ws.element_size(), _stream(stream)))
     return out
 
 

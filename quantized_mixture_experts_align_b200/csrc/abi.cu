@@ -476,6 +476,152 @@ int moe_w4a16_forward(const uint16_t *x, const float *logits, int T, int H, int 
     return check_launch("moe_w4a16_forward");
 }
 
+// ------------------------------------------------------------------------------------------
+// Grouped W4A16 GEMM, contiguous and masked layouts (per-row expert map -> alignment with k = 1,
+// then the down-mode kernels with unit weights write each real row of C).
+// ------------------------------------------------------------------------------------------
+
+static size_t grouped_layout(Carve &c, long M, int K, int G, int rows_hint, RouteBufs *rb, int32_t **ids,
+                             uint16_t **xg)
+{
+    const bool tcp = rows_hint >= 16;  // same rule as the layer: rows per expert
+    int32_t *idp = c.take<int32_t>((size_t)M);
+    RouteBufs r = carve_route(c, M, 1, G, tcp ? 256 : pick_block_m((long)rows_hint * G, 1, G));
+    uint16_t *xgp = tcp ? c.take<uint16_t>((size_t)r.max_blocks * r.block_m * K) : nullptr;
+    if (rb) *rb = r;
+    if (ids) *ids = idp;
+    if (xg) *xg = xgp;
+    return c.used;
+}
+
+static int check_grouped_shape(long M, int K, int N, int G)
+{
+    if (M < 0) return set_error(MOEQ_ERR_INVALID_ARG, "row count must be >= 0 (got %ld)", M);
+    if (M > (1L << 24)) return set_error(MOEQ_ERR_UNSUPPORTED, "row count must be <= 2^24 (got %ld)", M);
+    if (K < 128 || K % 128) return set_error(MOEQ_ERR_UNSUPPORTED, "K must be a positive multiple of 128 (got %d)", K);
+    if (N < 128 || N % 128) return set_error(MOEQ_ERR_UNSUPPORTED, "N must be a positive multiple of 128 (got %d)", N);
+    if (G < 1 || G > kMaxExperts) return set_error(MOEQ_ERR_UNSUPPORTED, "G must be in [1, %d] (got %d)", kMaxExperts, G);
+    return MOEQ_OK;
+}
+
+size_t moe_w4a16_grouped_contiguous_workspace_size(int M, int K, int N, int G)
+{
+    if (check_grouped_shape(M, K, N, G)) return 0;
+    Carve c(nullptr);
+    return grouped_layout(c, M, K, G, M / G, nullptr, nullptr, nullptr);
+}
+
+size_t moe_w4a16_grouped_masked_workspace_size(int G, int max_m, int K, int N, int expected_m)
+{
+    if (max_m < 0 || check_grouped_shape((long)G * max_m, K, N, G)) return 0;
+    Carve c(nullptr);
+    return grouped_layout(c, (long)G * max_m, K, G, expected_m, nullptr, nullptr, nullptr);
+}
+
+static int grouped_forward(const char *name, const uint16_t *A, long M, int K, const int32_t *wq, const uint16_t *wsc,
+                           int G, int N, const int32_t *m_indices, const int32_t *masked_m, int max_m, int rows_hint,
+                           uint16_t *C, void *ws, size_t ws_bytes, void *stream)
+{
+    MOEQ_REQUIRE(A);
+    MOEQ_REQUIRE(wq);
+    MOEQ_REQUIRE(wsc);
+    MOEQ_REQUIRE(C);
+    MOEQ_REQUIRE(ws);
+    if (!m_indices && !masked_m) return set_error(MOEQ_ERR_INVALID_ARG, "%s: no row-to-expert map", name);
+    if (reinterpret_cast<uintptr_t>(ws) & 255) return set_error(MOEQ_ERR_INVALID_ARG, "ws must be 256-byte aligned");
+    Carve need_c(nullptr);
+    const size_t need = grouped_layout(need_c, M, K, G, rows_hint, nullptr, nullptr, nullptr);
+    if (ws_bytes < need) return set_error(MOEQ_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, need);
+    cudaStream_t s = (cudaStream_t)stream;
+    Carve c(ws);
+    RouteBufs r;
+    int32_t *idp;
+    uint16_t *xg;
+    grouped_layout(c, M, K, G, rows_hint, &r, &idp, &xg);
+    const int n = (int)M;
+    const int32_t *ids = m_indices;
+    {
+        trace::Scope ts(trace::ALIGN, s);
+        if (masked_m) {
+            launch_masked_rows(masked_m, G, max_m, idp, num_sms(), s);
+            ids = idp;
+        }
+        launch_align(ids, n, G, r.block_m, r.sorted, r.eids, r.ntp, r.scratch, s);
+    }
+    W4GroupedArgs g{};
+    g.E = G;
+    g.sorted_ids = r.sorted;
+    g.expert_ids = r.eids;
+    g.num_tokens_padded = r.ntp;
+    g.n_slots = n;
+    g.topk_w = nullptr;  // weight 1: plain grouped GEMM
+    g.act = A;
+    g.act_row_div = 1;   // k = 1: the slot is the row
+    g.wq = wq;
+    g.ws = wsc;
+    g.K = K;
+    g.n_out = N;
+    g.n_rows = N;
+    g.y_out = C;
+    trace::Scope ts(trace::DOWN, s);
+    if (xg) {
+        int *status = device_status_ptr();
+        if (!status) return set_error(MOEQ_ERR_CUDA, "%s: no device status word", name);
+        const int cap = r.max_blocks * r.block_m;
+        launch_gather_bf16_perm(A, K, 1, r.sorted, r.ntp, n, cap, kW4SmallRows, xg, num_sms(), s);
+        W4TcArgs t{};
+        t.status = status;
+        t.E = G;
+        t.sorted_ids = r.sorted;
+        t.expert_ids = r.eids;
+        t.ntp = r.ntp;
+        t.n_slots = n;
+        t.topk_w = nullptr;
+        t.M = cap;
+        t.N = N;
+        t.K = K;
+        t.rows_per_expert = N;
+        t.wq = wq;
+        t.ws = wsc;
+        t.ys = C;
+        t.small_rows = kW4SmallRows;
+        const int rc = launch_w4a16_tc(t, TC_DOWN, xg, r.max_blocks, s);
+        if (rc) return rc;
+        g.blk_stride = r.block_m;
+        launch_w4a16_grouped_mma(g, MODE_DOWN, kW4SmallRows, r.max_blocks, s);
+    } else {
+        launch_w4a16_grouped_mma(g, MODE_DOWN, r.block_m, r.max_blocks, s);
+    }
+    return check_launch(name);
+}
+
+int moe_w4a16_grouped_contiguous(const uint16_t *A, int M, int K, const int32_t *w_q, const uint16_t *w_s, int G, int N,
+                                 const int32_t *m_indices, uint16_t *C, void *ws, size_t ws_bytes, void *stream)
+{
+    g_err[0] = 0;
+    int rc = check_grouped_shape(M, K, N, G);
+    if (rc) return rc;
+    if (M == 0) return MOEQ_OK;
+    MOEQ_REQUIRE(m_indices);
+    return grouped_forward("moe_w4a16_grouped_contiguous", A, M, K, w_q, w_s, G, N, m_indices, nullptr, 0, M / G, C,
+                           ws, ws_bytes, stream);
+}
+
+int moe_w4a16_grouped_masked(const uint16_t *A, int G, int max_m, int K, const int32_t *w_q, const uint16_t *w_s, int N,
+                             const int32_t *masked_m, int expected_m, uint16_t *C, void *ws, size_t ws_bytes,
+                             void *stream)
+{
+    g_err[0] = 0;
+    if (max_m < 0) return set_error(MOEQ_ERR_INVALID_ARG, "max_m must be >= 0 (got %d)", max_m);
+    if (expected_m < 0) return set_error(MOEQ_ERR_INVALID_ARG, "expected_m must be >= 0 (got %d)", expected_m);
+    int rc = check_grouped_shape((long)G * max_m, K, N, G);
+    if (rc) return rc;
+    if (max_m == 0) return MOEQ_OK;
+    MOEQ_REQUIRE(masked_m);
+    return grouped_forward("moe_w4a16_grouped_masked", A, (long)G * max_m, K, w_q, w_s, G, N, nullptr, masked_m, max_m,
+                           expected_m, C, ws, ws_bytes, stream);
+}
+
 size_t moe_w8a8_block_fp8_workspace_size(int T, int H, int I, int E, int k)
 {
     if (check_layer_shape(T, H, I, E, k)) return 0;

@@ -21,7 +21,7 @@ struct W4GroupedArgs {
     const int32_t *expert_ids;
     const int32_t *num_tokens_padded;
     int n_slots;             // T*k; sorted_ids entries >= n_slots are padding
-    const float *topk_w;     // [T*k] (down)
+    const float *topk_w;     // [T*k] (down); null: weight 1 (plain grouped GEMM)
     uint16_t *h_out;         // [T*k, I] bf16 (gate/up)
     uint16_t *y_out;         // [T*k, H] bf16, routing weight applied (down)
     // 0: align blocks of BM rows. Otherwise the alignment has blocks of blk_stride rows and the
@@ -92,6 +92,7 @@ void launch_route_topk(const float *logits, int T, int E, int k, int32_t *ids, f
 // Scratch (bytes) the alignment of n slots over E experts uses; 0 = the one-CTA kernel, which
 // also runs when launch_align gets no scratch.
 size_t align_scratch_bytes(int n, int E);
+void launch_masked_rows(const int32_t *masked_m, int G, int max_m, int32_t *ids, int num_sms, cudaStream_t s);
 void launch_align(const int32_t *topk_ids, int n, int E, int B, int32_t *sorted_ids, int32_t *expert_ids,
                   int32_t *ntp, int32_t *scratch, cudaStream_t s);
 void launch_combine(const uint16_t *ys, int T, int k, int H, uint16_t *out, int num_sms, cudaStream_t s);

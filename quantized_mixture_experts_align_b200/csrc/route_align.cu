@@ -288,6 +288,27 @@ __global__ void __launch_bounds__(kChunkThreads) align_scatter_kernel(const int3
     }
 }
 
+// Masked grouped layout: row e * max_m + r belongs to expert e when r < masked_m[e], else to none
+// (-1), which the alignment skips.
+__global__ void __launch_bounds__(256) masked_rows_kernel(const int32_t *__restrict__ masked_m, int G, int max_m,
+                                                          int32_t *__restrict__ ids)
+{
+    const long total = (long)G * max_m;
+    for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < total; i += (long)gridDim.x * blockDim.x) {
+        const int e = (int)(i / max_m);
+        const int r = (int)(i - (long)e * max_m);
+        ids[i] = (r < __ldg(masked_m + e)) ? e : -1;
+    }
+}
+
+void launch_masked_rows(const int32_t *masked_m, int G, int max_m, int32_t *ids, int num_sms, cudaStream_t s)
+{
+    const long total = (long)G * max_m;
+    if (total <= 0) return;
+    const int blocks = (int)((total + 255) / 256 < (long)num_sms * 4 ? (total + 255) / 256 : (long)num_sms * 4);
+    masked_rows_kernel<<<blocks, 256, 0, s>>>(masked_m, G, max_m, ids);
+}
+
 size_t align_scratch_bytes(int n, int E)
 {
     return n > kAlignOneCtaMax ? (size_t)cdiv(n, kChunk) * E * sizeof(int32_t) : 0;

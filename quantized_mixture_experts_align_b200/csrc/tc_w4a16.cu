@@ -287,7 +287,8 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
                 tc::tmem_ld32(lane_base + tok0, y);
                 tc::tmem_wait_ld();
                 const int my_slot = __ldg(a.sorted_ids + r0 + tok0 + lane);
-                const float my_w = (my_slot < a.n_slots) ? __ldg(a.topk_w + my_slot) : 0.f;
+                // no routing weights (plain grouped GEMM): weight 1
+                const float my_w = (my_slot < a.n_slots) ? (a.topk_w ? __ldg(a.topk_w + my_slot) : 1.f) : 0.f;
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
                     const int slot = __shfl_sync(0xFFFFFFFFu, my_slot, j);

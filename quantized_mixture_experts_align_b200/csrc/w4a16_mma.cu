@@ -65,7 +65,8 @@ constexpr int kW4StageBytes = 4 * 32 * 16 + 4 * 8 * 8;  // 2048 B codes + 256 B 
 
 // MODE_GATEUP: rows [f0, f0+16) (gate) and [I + f0, I + f0 + 16) (up) of W13; epilogue writes
 //              h[slot, f] = bf16(silu(gate) * up).
-// MODE_DOWN:   rows [r0, r0+32) of W2; epilogue writes ys[slot, r] = topk_w[slot] * y (f32).
+// MODE_DOWN:   rows [r0, r0+32) of W2; epilogue writes ys[slot, r] = bf16(topk_w[slot] * y) (weight 1
+//              without routing weights: the plain grouped GEMM).
 template <int BM, int WARPS, int MODE, bool STRIDED>
 __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4GroupedArgs a)
 {
@@ -213,7 +214,7 @@ __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4Grouped
                 h[rowA + g] = f32_to_bf16(silu_f32(accA[s][c]) * accB[s][c]);
                 h[rowA + g + 8] = f32_to_bf16(silu_f32(accA[s][2 + c]) * accB[s][2 + c]);
             } else {
-                const float wt = __ldg(a.topk_w + slot);
+                const float wt = a.topk_w ? __ldg(a.topk_w + slot) : 1.f;
                 uint16_t *y = a.y_out + (size_t)slot * a.n_out;
                 y[rowA + g] = f32_to_bf16(wt * accA[s][c]);
                 y[rowA + g + 8] = f32_to_bf16(wt * accA[s][2 + c]);

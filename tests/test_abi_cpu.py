@@ -86,6 +86,23 @@ def test_validation_rejects_before_device_work(L):
     assert _rc(L, "w8a8_block_fp8_matmul", N, N, N, N, 4, 256, 256, 64, 128, N, N) == moeq.MOEQ_ERR_UNSUPPORTED
     assert _rc(L, "w8a8_block_fp8_matmul", N, N, N, N, 4, 256, 200, 128, 128, N, N) == moeq.MOEQ_ERR_UNSUPPORTED
     assert _rc(L, "w8a8_block_fp8_matmul", N, N, N, N, 4, 200, 256, 128, 128, N, N) == moeq.MOEQ_ERR_UNSUPPORTED
+    # grouped W4A16 GEMM: shapes, row map, workspace
+    gc = lambda M, K, Nn, G, idx, ws, wsb: _rc(L, "moe_w4a16_grouped_contiguous", p, M, K, p, p, G, Nn, idx, p, ws, wsb, N)
+    assert gc(64, 100, 256, 4, p, p, 1 << 40) == moeq.MOEQ_ERR_UNSUPPORTED       # K % 128
+    assert gc(64, 256, 200, 4, p, p, 1 << 40) == moeq.MOEQ_ERR_UNSUPPORTED       # N % 128
+    assert gc(64, 256, 256, 0, p, p, 1 << 40) == moeq.MOEQ_ERR_UNSUPPORTED       # G
+    assert gc(64, 256, 256, 4, N, p, 1 << 40) == moeq.MOEQ_ERR_INVALID_ARG       # NULL m_indices
+    assert gc(64, 256, 256, 4, p, p, 10) == moeq.MOEQ_ERR_WORKSPACE
+    assert gc(0, 256, 256, 4, N, N, 0) == moeq.MOEQ_OK                           # no rows: no-op
+    assert moeq.lib().moe_w4a16_grouped_contiguous_workspace_size(64, 100, 256, 4) == 0
+    gm = lambda G, mm, K, Nn, masked, em: _rc(L, "moe_w4a16_grouped_masked", p, G, mm, K, p, p, Nn, masked, em, p, p,
+                                              1 << 40, N)
+    assert gm(4, 16, 256, 256, N, 4) == moeq.MOEQ_ERR_INVALID_ARG                # NULL masked_m
+    assert gm(4, -1, 256, 256, p, 4) == moeq.MOEQ_ERR_INVALID_ARG                # max_m < 0
+    assert gm(4, 16, 256, 256, p, -2) == moeq.MOEQ_ERR_INVALID_ARG               # expected_m < 0
+    assert gm(2000, 16, 256, 256, p, 4) == moeq.MOEQ_ERR_UNSUPPORTED             # G > 1024
+    assert moeq.lib().moe_w4a16_grouped_masked_workspace_size(8, 64, 256, 384, 48) > \
+        moeq.lib().moe_w4a16_grouped_masked_workspace_size(8, 64, 256, 384, 4)   # tensor-core gather buffer
     # T == 0 / M == 0 are valid no-ops
     assert _rc(L, "moe_route_topk", N, 0, 8, 2, N, N, N) == 0
     assert _rc(L, "w8a8_block_fp8_matmul", N, N, N, N, 0, 256, 256, 128, 128, N, N) == 0
