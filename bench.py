@@ -474,8 +474,14 @@ def main():
         return
     flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
 
+    flush_words = flush_buf.view(torch.int32)
+
     def flush():
+        # write a buffer larger than L2, then read it back: the timed step starts with a cold L2
+        # holding only clean lines (a write alone leaves ~L2-size dirty lines whose write-back
+        # would land inside the next timed step: ~9 us on a 176 MB weight stream)
         flush_buf.fill_(1)
+        flush_words.max()
 
     # ---- headline: decode W4A16 -----------------------------------------------------------
     d = W.make_moe(W.WORKLOADS["decode_w4a16"], device="cuda", E=args.experts)
@@ -511,7 +517,8 @@ def main():
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": f"decode_w4a16 T=32 H=7168 I=2048 E={d['E']} k=8 (INT4 group-32, bf16 scales)",
                    "touched_experts": n_active, "weight_bytes_per_step": step_bytes,
-                   "l2": f"flushed between steps ({L2_FLUSH_BYTES >> 20} MB write), outside the timed events",
+                   "l2": f"flushed between steps ({L2_FLUSH_BYTES >> 20} MB written then read: cold, clean L2), "
+                         "outside the timed events",
                    "parallelism": f"replicas x{world}"},
         "tflops": world * flops / (ms_step * 1e-3) / 1e12,
         "roofline": roofline,

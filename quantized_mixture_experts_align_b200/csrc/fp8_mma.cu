@@ -86,9 +86,7 @@ void launch_gather_fp8_rows(const uint8_t *xq, const float *xs, int H, int k, co
 // MODE_GATEUP: rows [f0, f0+16) gate and [I+f0, ...) up; WARPS = 8 so a CTA covers the 128
 //              features of one intermediate quantization group; epilogue quantizes silu(g)*u
 //              per slot and 128-group to E4M3 + f32 scale.
-// MODE_DOWN:   rows [r0, r0+32); epilogue writes ys[slot, r] = topk_w[slot] * y (f32).
-// MODE_DENSE:  as DOWN for a plain [M, K] x [N, K] product, row m of A is token m; epilogue
-//              writes C[m, r] as bf16.
+// MODE_DOWN:   rows [r0, r0+32); epilogue writes ys[slot, r] = topk_w[slot] * y (bf16).
 // ------------------------------------------------------------------------------------------
 template <int BM, int WARPS, int MODE>
 __global__ void __launch_bounds__(WARPS * 32) fp8_grouped_mma_kernel(F8GroupedArgs a)
@@ -98,12 +96,9 @@ __global__ void __launch_bounds__(WARPS * 32) fp8_grouped_mma_kernel(F8GroupedAr
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
     const int blk = blockIdx.x;
-    int e = 0;
-    if (MODE != MODE_DENSE) {
-        if (blk * BM >= __ldg(a.num_tokens_padded)) return;
-        e = __ldg(a.expert_ids + blk);
-        if (e < 0 || e >= a.E) return;
-    }
+    if (blk * BM >= __ldg(a.num_tokens_padded)) return;
+    const int e = __ldg(a.expert_ids + blk);
+    if (e < 0 || e >= a.E) return;
     const int tile = blockIdx.y * WARPS + warp;
     int rowA, rowB;
     bool active;
@@ -129,7 +124,7 @@ __global__ void __launch_bounds__(WARPS * 32) fp8_grouped_mma_kernel(F8GroupedAr
 #pragma unroll
         for (int c = -1; c < 2; ++c) {
             const int j = blk * BM + 8 * s + (c < 0 ? g : 2 * t + c);
-            const int slot = (MODE == MODE_DENSE) ? ((j < a.n_slots) ? j : a.n_slots) : __ldg(a.sorted_ids + j);
+            const int slot = __ldg(a.sorted_ids + j);
             const bool ok = slot < a.n_slots;
             const size_t arow = ok ? (size_t)(slot / a.act_row_div) : 0;
             if (c < 0) act_row[s] = ok ? a.act + arow * K : nullptr;
@@ -234,150 +229,16 @@ __global__ void __launch_bounds__(WARPS * 32) fp8_grouped_mma_kernel(F8GroupedAr
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
                 const int j = blk * BM + 8 * s + 2 * t + c;
-                if (MODE == MODE_DENSE) {
-                    if (j >= a.n_slots) continue;
-                    uint16_t *crow = a.c_out + (size_t)j * a.n_out;
-                    crow[rowA + g] = f32_to_bf16(accA[s][c]);
-                    crow[rowA + g + 8] = f32_to_bf16(accA[s][2 + c]);
-                    crow[rowB + g] = f32_to_bf16(accB[s][c]);
-                    crow[rowB + g + 8] = f32_to_bf16(accB[s][2 + c]);
-                } else {
-                    const int slot = __ldg(a.sorted_ids + j);
-                    if (slot >= a.n_slots) continue;
-                    const float wt = __ldg(a.topk_w + slot);
-                    uint16_t *y = a.y_out + (size_t)slot * a.n_out;
-                    y[rowA + g] = f32_to_bf16(wt * accA[s][c]);
-                    y[rowA + g + 8] = f32_to_bf16(wt * accA[s][2 + c]);
-                    y[rowB + g] = f32_to_bf16(wt * accB[s][c]);
-                    y[rowB + g + 8] = f32_to_bf16(wt * accB[s][2 + c]);
-                }
+                const int slot = __ldg(a.sorted_ids + j);
+                if (slot >= a.n_slots) continue;
+                const float wt = __ldg(a.topk_w + slot);
+                uint16_t *y = a.y_out + (size_t)slot * a.n_out;
+                y[rowA + g] = f32_to_bf16(wt * accA[s][c]);
+                y[rowA + g + 8] = f32_to_bf16(wt * accA[s][2 + c]);
+                y[rowB + g] = f32_to_bf16(wt * accB[s][c]);
+                y[rowB + g + 8] = f32_to_bf16(wt * accB[s][2 + c]);
             }
         }
-    }
-}
-
-// ------------------------------------------------------------------------------------------
-// Dense block-FP8 for few rows (M <= 128): the weights are streamed once, so the kernel is HBM
-// bound and needs many bytes in flight. A CTA owns 32 weight rows (two 16-row MMA tiles) for
-// all M rows; its 4 warps split K into contiguous quarters (each warp reads sequential row
-// segments, one 128-wide K block ahead in registers) and add their partial sums through shared
-// memory. 24576 weight rows give 768 CTAs, five per SM.
-// ------------------------------------------------------------------------------------------
-template <int BM>
-__global__ void __launch_bounds__(128) fp8_dense_splitk_kernel(F8GroupedArgs a)
-{
-    constexpr int MS = BM / 8;
-    constexpr int KSPLIT = 4;
-    __shared__ float part[KSPLIT - 1][MS][8][32];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int g = lane >> 2, t = lane & 3;
-    const int m0 = blockIdx.x * BM;
-    const int rowA = blockIdx.y * 32, rowB = rowA + 16;
-    const int K = a.K, KB = K / 128;
-    const int kb0 = warp * KB / KSPLIT, kb1 = (warp + 1) * KB / KSPLIT;
-
-    const uint8_t *act_row[MS];
-    const float *col_scale[MS][2];
-#pragma unroll
-    for (int s = 0; s < MS; ++s) {
-        const int j = m0 + 8 * s + g;
-        act_row[s] = (j < a.n_slots) ? a.act + (size_t)j * K : nullptr;
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-            const int jc = m0 + 8 * s + 2 * t + c;
-            col_scale[s][c] = (jc < a.n_slots) ? a.act_s + (size_t)jc * KB : nullptr;
-        }
-    }
-    const uint8_t *wr[4] = {a.w + (size_t)(rowA + g) * K, a.w + (size_t)(rowA + g + 8) * K,
-                            a.w + (size_t)(rowB + g) * K, a.w + (size_t)(rowB + g + 8) * K};
-    const float *srA = a.w_s + (size_t)(rowA / 128) * KB;
-
-    float acc[MS][2][4];
-#pragma unroll
-    for (int s = 0; s < MS; ++s)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) { acc[s][0][i] = 0.f; acc[s][1][i] = 0.f; }
-
-    // one K block ahead in registers where the accumulators leave room (up to 16 rows)
-    constexpr bool kPrefetch = MS <= 2;
-    uint4 cur[2][4], nxt[kPrefetch ? 2 : 1][4];
-    auto load_kb = [&](int kb, uint4 (&v)[2][4]) {
-#pragma unroll
-        for (int c = 0; c < 2; ++c)
-#pragma unroll
-            for (int r = 0; r < 4; ++r) v[c][r] = ld_stream_v4(wr[r] + kb * 128 + c * 64 + 16 * t);
-    };
-    if (kPrefetch && kb0 < kb1) load_kb(kb0, cur);
-    for (int kb = kb0; kb < kb1; ++kb) {
-        if (kPrefetch) {
-            if (kb + 1 < kb1) load_kb(kb + 1, *reinterpret_cast<uint4(*)[2][4]>(&nxt));
-        } else {
-            load_kb(kb, cur);
-        }
-        const float sw = __ldg(srA + kb);  // rows rowA..rowA+31 share one 128-row scale block
-#pragma unroll
-        for (int s = 0; s < MS; ++s) {
-            float tA[4] = {0.f, 0.f, 0.f, 0.f}, tB[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                uint4 xv = make_uint4(0u, 0u, 0u, 0u);
-                if (act_row[s]) xv = ld_v4(act_row[s] + kb * 128 + c * 64 + 16 * t);
-                mma_e4m3_16832(tA, cur[c][0].x, cur[c][1].x, cur[c][0].y, cur[c][1].y, xv.x, xv.y);
-                mma_e4m3_16832(tB, cur[c][2].x, cur[c][3].x, cur[c][2].y, cur[c][3].y, xv.x, xv.y);
-                mma_e4m3_16832(tA, cur[c][0].z, cur[c][1].z, cur[c][0].w, cur[c][1].w, xv.z, xv.w);
-                mma_e4m3_16832(tB, cur[c][2].z, cur[c][3].z, cur[c][2].w, cur[c][3].w, xv.z, xv.w);
-            }
-            const float x0 = col_scale[s][0] ? __ldg(col_scale[s][0] + kb) * sw : 0.f;
-            const float x1 = col_scale[s][1] ? __ldg(col_scale[s][1] + kb) * sw : 0.f;
-            acc[s][0][0] += tA[0] * x0; acc[s][0][1] += tA[1] * x1;
-            acc[s][0][2] += tA[2] * x0; acc[s][0][3] += tA[3] * x1;
-            acc[s][1][0] += tB[0] * x0; acc[s][1][1] += tB[1] * x1;
-            acc[s][1][2] += tB[2] * x0; acc[s][1][3] += tB[3] * x1;
-        }
-        if (kPrefetch) {
-#pragma unroll
-            for (int c = 0; c < 2; ++c)
-#pragma unroll
-                for (int r = 0; r < 4; ++r) cur[c][r] = (&nxt[0][0])[c * 4 + r];
-        }
-    }
-    // reduce the K quarters
-    if (warp > 0) {
-#pragma unroll
-        for (int s = 0; s < MS; ++s)
-#pragma unroll
-            for (int i = 0; i < 8; ++i) part[warp - 1][s][i][lane] = acc[s][i >> 2][i & 3];
-    }
-    __syncthreads();
-    if (warp == 0) {
-#pragma unroll
-        for (int s = 0; s < MS; ++s) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-#pragma unroll
-                for (int w = 0; w < KSPLIT - 1; ++w) acc[s][i >> 2][i & 3] += part[w][s][i][lane];
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                const int j = m0 + 8 * s + 2 * t + c;
-                if (j >= a.n_slots) continue;
-                uint16_t *crow = a.c_out + (size_t)j * a.n_out;
-                crow[rowA + g] = f32_to_bf16(acc[s][0][c]);
-                crow[rowA + g + 8] = f32_to_bf16(acc[s][0][2 + c]);
-                crow[rowB + g] = f32_to_bf16(acc[s][1][c]);
-                crow[rowB + g + 8] = f32_to_bf16(acc[s][1][2 + c]);
-            }
-        }
-    }
-}
-
-void launch_fp8_dense_splitk(const F8GroupedArgs &a, int block_m, cudaStream_t s)
-{
-    const dim3 grid(cdiv(a.n_slots, block_m), a.n_out / 32);
-    switch (block_m) {
-        case 8: fp8_dense_splitk_kernel<8><<<grid, 128, 0, s>>>(a); break;
-        case 16: fp8_dense_splitk_kernel<16><<<grid, 128, 0, s>>>(a); break;
-        case 32: fp8_dense_splitk_kernel<32><<<grid, 128, 0, s>>>(a); break;
-        default: fp8_dense_splitk_kernel<64><<<grid, 128, 0, s>>>(a); break;
     }
 }
 
@@ -396,8 +257,7 @@ void launch_fp8_grouped_mma(const F8GroupedArgs &a, int mode, int block_m, int m
 #define MOEQ_F8_CASE(BMV)                                                          \
     case BMV:                                                                      \
         if (mode == MODE_GATEUP) launch_f8<BMV, MODE_GATEUP>(a, max_blocks, s);    \
-        else if (mode == MODE_DOWN) launch_f8<BMV, MODE_DOWN>(a, max_blocks, s);   \
-        else launch_f8<BMV, MODE_DENSE>(a, max_blocks, s);                         \
+        else launch_f8<BMV, MODE_DOWN>(a, max_blocks, s);                          \
         break;
     switch (block_m) {
         MOEQ_F8_CASE(8)

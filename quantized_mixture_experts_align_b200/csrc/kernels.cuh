@@ -6,7 +6,7 @@
 
 namespace moeq {
 
-enum { MODE_GATEUP = 0, MODE_DOWN = 1, MODE_DENSE = 2 };
+enum { MODE_GATEUP = 0, MODE_DOWN = 1 };
 
 struct W4GroupedArgs {
     const uint16_t *act;     // gate/up: x [T, K]; down: h [T*k, K]  (bf16)
@@ -42,12 +42,11 @@ struct F8GroupedArgs {
     const int32_t *sorted_ids;
     const int32_t *expert_ids;
     const int32_t *num_tokens_padded;
-    int n_slots;             // T*k (grouped) or M (dense)
+    int n_slots;             // T*k
     const float *topk_w;
     uint8_t *hq_out;         // [T*k, I]
     float *hs_out;           // [T*k, I/128]
     uint16_t *y_out;         // [T*k, H] bf16, routing weight applied (down)
-    uint16_t *c_out;         // dense: [M, N] bf16
 };
 
 enum { TC_DENSE = 0, TC_GATEUP = 1, TC_DOWN = 2 };
@@ -99,10 +98,12 @@ void launch_combine(const uint16_t *ys, int T, int k, int H, uint16_t *out, int 
 void launch_fp8_act_quant(const uint16_t *x, int rows, int cols, uint8_t *q, float *s, cudaStream_t st);
 void launch_w4a16_grouped_mma(const W4GroupedArgs &a, int mode, int block_m, int max_blocks, cudaStream_t s);
 void launch_fp8_grouped_mma(const F8GroupedArgs &a, int mode, int block_m, int max_blocks, cudaStream_t s);
-// Dense block-FP8 for few rows: K split over the 4 warps of a CTA, 32 weight rows per CTA.
-void launch_fp8_dense_splitk(const F8GroupedArgs &a, int block_m, cudaStream_t s);
 // tcgen05 block-FP8 GEMM: A [M, K] and B [N, K] E4M3, K % 128 == 0, N % 128 == 0. Returns a status.
 int launch_fp8_tc_gemm(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B, cudaStream_t s);
+// Dense block-FP8 GEMM for M <= fp8_skinny_max_rows() rows (swap-AB tcgen05 tiles of 128 weight
+// rows, K split over a cluster of `split` CTAs reduced through distributed shared memory).
+int fp8_skinny_max_rows();
+int launch_fp8_tc_skinny(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B, int split, cudaStream_t s);
 // tcgen05 grouped block-FP8 GEMM over expert-contiguous rows A [M, K] (128-row blocks, one expert
 // each, per expert_ids / ntp) and weights W [E * rows_per_expert, K]; mode TC_GATEUP or TC_DOWN.
 int launch_fp8_tc_grouped(const Fp8TcArgs &a, int mode, const uint8_t *A, const uint8_t *W, int E, int max_blocks,

@@ -379,11 +379,10 @@ int launch_tc(const Fp8TcArgs &a, const CUtensorMap &tmA, const CUtensorMap &tmB
 
 int launch_fp8_tc_gemm(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B, cudaStream_t s)
 {
-    // Up to 64 rows the weights stream once (HBM bound) and narrow 64-column tiles give every SM
-    // several CTAs; from 65 rows, 256-column tiles (more weight bytes in flight per SM, fewer
-    // activation re-reads; tensor bound for many rows). Chosen from measured M sweeps.
-    // From 256 rows, CTA pairs (256 x 256 tiles, half the weight rows per CTA).
-    const int bn = (a.M <= 64) ? 64 : (a.N % 256 == 0) ? 256 : 128;
+    // Rows past 64 (fewer go to the swap-AB kernel): 256-column tiles (more weight bytes in flight
+    // per SM, fewer activation re-reads; tensor bound for many rows), chosen from measured M
+    // sweeps; from 256 rows, CTA pairs (256 x 256 tiles, half the weight rows per CTA).
+    const int bn = (a.N % 256 == 0) ? 256 : 128;
     const bool pair = bn == 256 && a.M >= 256;
     CUtensorMap tmA, tmB;
     int rc = make_tmap_2d(&tmA, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.M, (uint64_t)a.K, kBM, kBK);
@@ -392,8 +391,7 @@ int launch_fp8_tc_gemm(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B, c
     if (rc) return rc;
     if (pair) return launch_tc<256, TC_DENSE, true>(a, tmA, tmB, 2 * cdiv(a.M, 2 * kBM), a.N / 256, s);
     if (bn == 256) return launch_tc<256, TC_DENSE>(a, tmA, tmB, cdiv(a.M, kBM), a.N / 256, s);
-    if (bn == 128) return launch_tc<128, TC_DENSE>(a, tmA, tmB, cdiv(a.M, kBM), a.N / 128, s);
-    return launch_tc<64, TC_DENSE>(a, tmA, tmB, cdiv(a.M, kBM), a.N / 64, s);
+    return launch_tc<128, TC_DENSE>(a, tmA, tmB, cdiv(a.M, kBM), a.N / 128, s);
 }
 
 int launch_fp8_tc_grouped(const Fp8TcArgs &a, int mode, const uint8_t *A, const uint8_t *W, int E, int max_blocks,

@@ -294,6 +294,14 @@ def test_dense_fp8_small_shapes_all_rows(M):
     _dense_parity(M, 512, 1024, np.arange(M, dtype=np.int32))
 
 
+@pytest.mark.parametrize("M,N,K", [(5, 256, 896), (70, 1280, 2944), (17, 384, 384), (128, 384, 1024),
+                                   (120, 128, 7168), (33, 24576 // 16, 7168)])
+def test_dense_fp8_skinny_split_shapes_all_rows(M, N, K):
+    """The few-row path splits K over a cluster of CTAs: cluster sizes that do not divide the K
+    blocks (7 CTAs over 7 blocks, 8 CTAs over 23), every padded row count (16 .. 128), one tile."""
+    _dense_parity(M, N, K, np.arange(M, dtype=np.int32))
+
+
 @pytest.mark.parametrize("M,N,K", [(128, 256, 1024), (200, 512, 512), (300, 384, 896), (1000, 256, 7168),
                                    (256, 512, 384), (257, 768, 640), (640, 256, 1152)])
 def test_dense_fp8_tensor_core_shapes_all_rows(M, N, K):
