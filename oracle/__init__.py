@@ -135,6 +135,24 @@ def fp8_block_matmul(A, As, B, Bs, rows=None):
     return C
 
 
+def fp8_channel_matmul(A, As, B, Bs, rows=None):
+    """C rows (float64 [len(rows), N]) of the channelwise FP8 product As[m] Bs[n] (A_q B_q^T)[m, n].
+    A uint8 E4M3 [M, K], As f32 [M], B uint8 E4M3 [N, K], Bs f32 [N]."""
+    A = np.ascontiguousarray(A, dtype=np.uint8)
+    B = np.ascontiguousarray(B, dtype=np.uint8)
+    As = np.ascontiguousarray(As, dtype=np.float32).reshape(-1)
+    Bs = np.ascontiguousarray(Bs, dtype=np.float32).reshape(-1)
+    M, K = A.shape
+    N = B.shape[0]
+    if As.size != M or Bs.size != N or B.shape[1] != K:
+        raise ValueError("fp8_channel_matmul: shapes")
+    r = _tokens(rows, M)
+    C = np.zeros((len(r), N), np.float64)
+    _check(lib().orc_fp8_channel_matmul(_p(A), _p(As), _p(B), _p(Bs), M, N, K, _p(r), len(r), _p(C)),
+           "fp8_channel_matmul")
+    return C
+
+
 def grouped_w4a16(A, wq, ws, expert_of_row, rows=None):
     """C rows (float64 [len(rows), N]) of the grouped W4A16 GEMM: row m times the dequantized
     weights of expert expert_of_row[m] (zeros where it is -1). A bf16 bits [M, K]; wq int32

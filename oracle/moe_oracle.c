@@ -410,6 +410,34 @@ int orc_fp8_block_matmul(const uint8_t *A, const float *As, const uint8_t *B, co
 }
 
 /* ------------------------------------------------------------------------------------------ */
+/* Dense channelwise FP8 matmul ([SGL], "JSON format": the channelwise variant is the W8A8 FP8
+ * GEMM with one scale per token of the activations and one per channel (output row) of the
+ * weights). READING: the pages name the scaling granularity and no formula; the plain reading is
+ *   C[m, n] = As[m] * Bs[n] * sum_c E4M3(A[m, c]) * E4M3(B[n, c])
+ * with A [M, K], As [M], B [N, K], Bs [N], in double.                                         */
+/* ------------------------------------------------------------------------------------------ */
+
+int orc_fp8_channel_matmul(const uint8_t *A, const float *As, const uint8_t *B, const float *Bs,
+                           int M, int N, int K, const int32_t *rows, int nrows, double *C)
+{
+    if (K < 1 || N < 1) return 1;
+    for (int i = 0; i < nrows; ++i)
+        if (rows[i] < 0 || rows[i] >= M) return 1;
+    e4m3_table_init();
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int i = 0; i < nrows; ++i)
+        for (int n = 0; n < N; ++n) {
+            int m = rows[i];
+            const uint8_t *a = A + (size_t)m * K;
+            const uint8_t *b = B + (size_t)n * K;
+            double dot = 0.0;
+            for (int c = 0; c < K; ++c) dot += e4m3_table[a[c]] * e4m3_table[b[c]];
+            C[(size_t)i * N + n] = (double)As[m] * (double)Bs[n] * dot;
+        }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------------------------ */
 /* Grouped W4A16 GEMM ([CHORD], "SM90 grouped kernels": the contiguous layout concatenates the
  * rows of each expert, padded to 128-row boundaries, with m_indices holding each row's expert
  * and -1 on padding; the masked layout gives every expert a fixed budget of max_m rows of which

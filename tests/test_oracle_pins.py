@@ -368,6 +368,54 @@ def test_fp8_dense_matches_numpy_matmul():
     assert np.allclose(C, ref, rtol=1e-12, atol=1e-12)
 
 
+def test_fp8_channel_matches_numpy_matmul():
+    """Channelwise product against numpy float64 matmul of the torch-decoded E4M3 operands, the
+    per-token scale on the rows and the per-channel scale on the columns."""
+    d = W.make_dense_fp8_channel(W.WORKLOADS["dense_fp8_channel"], 24, N=384, K=640)
+    A, As, B, Bs = (d[n].numpy() for n in ("A", "As", "B", "Bs"))
+    assert As.shape == (24,) and Bs.shape == (384,)
+    C = oracle.fp8_channel_matmul(A, As, B, Bs)
+    Ad = torch.from_numpy(A).view(torch.float8_e4m3fn).double().numpy()
+    Bd = torch.from_numpy(B).view(torch.float8_e4m3fn).double().numpy()
+    ref = (Ad @ Bd.T) * As.astype(np.float64)[:, None] * Bs.astype(np.float64)[None, :]
+    assert np.allclose(C, ref, rtol=1e-12, atol=1e-12)
+    rows = np.array([23, 0, 7], np.int32)
+    assert np.array_equal(oracle.fp8_channel_matmul(A, As, B, Bs, rows=rows), C[rows])
+
+
+def test_fp8_channel_closed_form_and_scale_indexing():
+    """All codes 448 (0x7E) with As[m] = 2^m / 448 and Bs[n] = 3^(n % 5) / 448: C[m, n] =
+    K * 2^m * 3^(n % 5) exactly (M != N, so a transposed scale index cannot pass)."""
+    M, N, K = 3, 10, 96
+    A = np.full((M, K), 0x7E, np.uint8)
+    B = np.full((N, K), 0x7E, np.uint8)
+    As = np.array([2.0 ** m / 448.0 for m in range(M)], np.float32)
+    Bs = np.array([3.0 ** (n % 5) / 448.0 for n in range(N)], np.float32)
+    C = oracle.fp8_channel_matmul(A, As, B, Bs)
+    for m in range(M):
+        for n in range(N):
+            assert C[m, n] == pytest.approx(K * 2.0 ** m * 3.0 ** (n % 5), rel=1e-6)
+    # one code of -1.5 (0xBC) in row 1 of A at column 5 against 2.0 (0x40) in channel 7
+    A2 = np.zeros((M, K), np.uint8)
+    B2 = np.zeros((N, K), np.uint8)
+    A2[1, 5], B2[7, 5] = 0xBC, 0x40
+    ones = np.ones(M, np.float32), np.ones(N, np.float32)
+    C2 = oracle.fp8_channel_matmul(A2, ones[0], B2, ones[1])
+    assert C2[1, 7] == -3.0 and np.count_nonzero(C2) == 1
+
+
+def test_fp8_channel_equals_block_when_scales_are_constant_per_block():
+    """With As constant along K and Bs constant over each 128-row block, the channelwise and the
+    block-scaled definitions describe the same product: the two oracle functions agree."""
+    d = W.make_dense_fp8_channel(W.WORKLOADS["dense_fp8_channel"], 5, N=256, K=384)
+    A, As, B = d["A"].numpy(), d["As"].numpy(), d["B"].numpy()
+    Bs_blk = np.array([0.25, 3.0], np.float32)
+    Bs = np.repeat(Bs_blk, 128)
+    C = oracle.fp8_channel_matmul(A, As, B, Bs)
+    Cb = oracle.fp8_block_matmul(A, np.repeat(As[:, None], 3, 1), B, np.repeat(Bs_blk[:, None], 3, 1))
+    assert np.allclose(C, Cb, rtol=1e-12, atol=1e-12)
+
+
 def _torch_fp8_rows(v32):
     q, s = W.quantize_fp8_rows(torch.from_numpy(np.ascontiguousarray(v32)))
     return q.numpy(), s.numpy()

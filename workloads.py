@@ -55,6 +55,9 @@ WORKLOADS = {
     "prefill_w4a16": Workload("prefill_w4a16", "w4a16", 2, T=8192, H=7168, I=2048, E=384, k=8, logits="zipf"),
     "dense_fp8": Workload("dense_fp8", "dense_fp8", 3, M_list=tuple(2 ** i for i in range(13)), N=24576, K=7168),
     "moe_fp8": Workload("moe_fp8", "fp8", 4, T=4096, H=7168, I=2048, E=256, k=8, logits="zipf"),
+    # channelwise W8A8 FP8 GEMM at the N = K = 4096 shape the SGLang config page gives as its example
+    "dense_fp8_channel": Workload("dense_fp8_channel", "dense_fp8_channel", 5,
+                                  M_list=(1, 16, 64, 128, 256, 1024, 4096), N=4096, K=4096),
 }
 
 # tensor stream ids
@@ -170,6 +173,18 @@ def make_dense_fp8(wl: Workload, M: int, device="cpu", N=None, K=None):
     return dict(A=Aq, As=As, B=Bq, Bs=Bs, M=M, N=N, K=K)
 
 
+def make_dense_fp8_channel(wl: Workload, M: int, device="cpu", N=None, K=None):
+    """A quantized per token (one scale per row, As [M]) and B per channel (Bs [N]), E4M3."""
+    N = wl.N if N is None else N
+    K = wl.K if K is None else K
+    Mmax = max(M, max(wl.M_list) if wl.M_list else M)
+    a = bf16_normal((Mmax, K), generator(wl.wid, _A, device=device), device)[:M].float()
+    Aq, As = quantize_fp8_rows(a, group=K)
+    gb = generator(wl.wid, _B, device=device)
+    Bq, Bs = quantize_fp8_rows(torch.randn((N, K), generator=gb, device=device) * 0.02, group=K)
+    return dict(A=Aq, As=As.reshape(M).contiguous(), B=Bq, Bs=Bs.reshape(N).contiguous(), M=M, N=N, K=K)
+
+
 def np_bits(t: torch.Tensor) -> np.ndarray:
     """Host numpy view of a tensor's raw storage: bf16 -> uint16, everything else as is."""
     t = t.detach().contiguous().cpu()
@@ -197,5 +212,5 @@ def cdiv(a: int, b: int) -> int:
     return -(-a // b)
 
 
-__all__ = ["WORKLOADS", "Workload", "make_moe", "make_dense_fp8", "np_bits", "moe_flops",
+__all__ = ["WORKLOADS", "Workload", "make_moe", "make_dense_fp8", "make_dense_fp8_channel", "np_bits", "moe_flops",
            "w4a16_expert_bytes", "fp8_expert_bytes", "router_logits", "cdiv", "math"]
