@@ -426,6 +426,14 @@ def only_arm(args, moeq, rank, world):
         ms = timed_steps(lambda: moeq.w8a8_block_fp8_matmul(dd["A"], dd["As"], dd["B"], dd["Bs"], out=C),
                          args.steps, args.warmup, None, world)
         line = {"only": name, "M": M, "ms": statistics.mean(ms), "tflops": 2.0 * M * wl.N * wl.K / statistics.mean(ms) / 1e9}
+    elif name == "dense_fp8_channel":
+        wl = W.WORKLOADS[name]
+        M = args.tokens or 4096
+        dd = W.make_dense_fp8_channel(wl, M, device="cuda")
+        C = torch.empty((M, wl.N), dtype=torch.bfloat16, device="cuda")
+        ms = timed_steps(lambda: moeq.w8a8_channel_fp8_matmul(dd["A"], dd["As"], dd["B"], dd["Bs"], out=C),
+                         args.steps, args.warmup, None, world)
+        line = {"only": name, "M": M, "ms": statistics.mean(ms), "tflops": 2.0 * M * wl.N * wl.K / statistics.mean(ms) / 1e9}
     else:
         d = W.make_moe(W.WORKLOADS[name], device="cuda", T=args.tokens, E=args.experts)
         if d["kind"] == "w4a16":
@@ -453,7 +461,7 @@ def main():
     ap.add_argument("--experts", type=int, default=None,
                     help="override E of the workload (small cases for profiler captures)")
     ap.add_argument("--tokens", type=int, default=None, help="override T of the workload (with --only)")
-    ap.add_argument("--only", choices=["prefill_w4a16", "moe_fp8", "dense_fp8"], default=None,
+    ap.add_argument("--only", choices=["prefill_w4a16", "moe_fp8", "dense_fp8", "dense_fp8_channel"], default=None,
                     help="time one secondary workload alone (small cases for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -629,6 +637,27 @@ def main():
                                    "fp8_peak_tflops": fp8_burst,
                                    "fp8_peak_source": ("measured in this run (burst): " + fp8m["how"]) if "burst" in fp8m
                                    else f"2 x {peak_src} bf16 burst (nominal ratio)"}
+        # channelwise FP8 (per-token x per-channel scales) at the page's N = K = 4096 example, plus
+        # the block sweep's 24576 x 7168 weights at 4096 rows for comparison
+        cwl = W.WORKLOADS["dense_fp8_channel"]
+        csweep = {}
+        for (M, Nc, Kc) in [(M, cwl.N, cwl.K) for M in cwl.M_list] + [(4096, 24576, 7168)]:
+            dd = W.make_dense_fp8_channel(cwl, M, device="cuda", N=Nc, K=Kc)
+            C = torch.empty((M, Nc), dtype=torch.bfloat16, device="cuda")
+            fn = lambda: moeq.w8a8_channel_fp8_matmul(dd["A"], dd["As"], dd["B"], dd["Bs"], out=C)
+            dms = statistics.mean(timed_steps(fn, max(3, args.steps // 4), 3, flush, world))
+            byts = Nc * Kc + Nc * 4 + M * Kc + M * 4 + 2 * M * Nc
+            fl = 2.0 * M * Nc * Kc
+            csweep[f"M={M} N={Nc} K={Kc}"] = {
+                "ms": dms, "tflops": fl / (dms * 1e-3) / 1e12, "gbs": byts / (dms * 1e-3) / 1e9,
+                "hbm_frac": byts / (dms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                "fp8_frac": fl / (dms * 1e-3) / 1e12 / fp8_burst,
+                "roof_frac": max(byts / (peaks["hbm_gbs"] * 1e9), fl / (fp8_burst * 1e12)) / (dms * 1e-3)}
+            del dd, C
+        also["dense_fp8_channel_sweep"] = {
+            "workload": "A [M,K] e4m3 x As [M] per token, B [N,K] e4m3 x Bs [N] per channel, C bf16",
+            "by_shape": csweep, "fp8_peak_tflops": fp8_burst,
+            "roof": "max(bytes / measured HBM, flops / FP8 burst peak) / time"}
         line["also"] = also
 
     line["clocks"] = clk.summary()

@@ -197,10 +197,24 @@ MOEQ_API int moe_w4a16_grouped_masked(const uint16_t *A, int G, int max_m, int K
  *   A e4m3 [M, K], As f32 [M, K/128], B e4m3 [N, K], Bs f32 [ceil(N/128), ceil(K/128)],
  *   C bf16 [M, N] out. block_n and block_k must both be 128 ([SGL], "Config directory & naming":
  *   almost every entry uses block_shape [128, 128]); K % 128 == 0, N % 128 == 0
- *   (the page's shape check: ceil(N/block_n) == rows of Bs, ceil(K/block_k) == columns of Bs).
+ *   (the page's shape check: ceil(N/block_n) == rows of Bs, ceil(K/block_k) == columns of Bs);
+ *   A, B and C 16-byte aligned (else UNSUPPORTED).
  */
 MOEQ_API int w8a8_block_fp8_matmul(const uint8_t *A, const float *As, const uint8_t *B, const float *Bs,
                           int M, int N, int K, int block_n, int block_k, uint16_t *C, void *stream);
+
+/*
+ * Dense channelwise FP8 matmul ([SGL], "JSON format": the channelwise variant is the W8A8 FP8 GEMM
+ * with per-token activation scales and per-channel weight scales):
+ *   C[m, n] = bf16( As[m] * Bs[n] * sum_k A[m, k] * B[n, k] )   (f32 accumulation over all of K)
+ *   A e4m3 [M, K], As f32 [M], B e4m3 [N, K], Bs f32 [N], C bf16 [M, N] out; all device memory,
+ *   row-major, caller-owned; nothing allocated.
+ * Limits: K % 128 == 0, N % 128 == 0 (both >= 128), M >= 0 (0 is a no-op). Errors: INVALID_ARG for
+ * null pointers or negative sizes, UNSUPPORTED for other shapes or when A, B or C is not 16-byte
+ * aligned, CUDA_LAUNCH for a failed launch.
+ */
+MOEQ_API int w8a8_channel_fp8_matmul(const uint8_t *A, const float *As, const uint8_t *B, const float *Bs, int M, int N,
+                                     int K, uint16_t *C, void *stream);
 
 /*
  * Stage tracing, a diagnostic that is off by default. While enabled, every forward / matmul call

@@ -39,6 +39,7 @@ _SIGNATURES = {
     "moe_w8a8_block_fp8_workspace_size": ([_I, _I, _I, _I, _I], _Z),
     "moe_w8a8_block_fp8_forward": ([_V, _V, _I, _I, _I, _I, _I, _V, _V, _V, _V, _V, _V, _V, _V, _Z, _V], _I),
     "w8a8_block_fp8_matmul": ([_V, _V, _V, _V, _I, _I, _I, _I, _I, _V, _V], _I),
+    "w8a8_channel_fp8_matmul": ([_V, _V, _V, _V, _I, _I, _I, _V, _V], _I),
     "moe_w4a16_grouped_contiguous_workspace_size": ([_I, _I, _I, _I], _Z),
     "moe_w4a16_grouped_contiguous": ([_V, _I, _I, _V, _V, _I, _I, _V, _V, _V, _Z, _V], _I),
     "moe_w4a16_grouped_masked_workspace_size": ([_I, _I, _I, _I, _I], _Z),
@@ -209,6 +210,20 @@ def w8a8_block_fp8_matmul(A, As, B, Bs, block_size=(128, 128), out=None, stream=
     _check(lib().w8a8_block_fp8_matmul(
         _dev(A, "A", _U8), _dev(As, "As", torch.float32), _dev(B, "B", _U8), _dev(Bs, "Bs", torch.float32),
         M, N, K, int(block_size[0]), int(block_size[1]), _dev(out, "out", _BF16), _stream(stream)))
+    return out
+
+
+def w8a8_channel_fp8_matmul(A, As, B, Bs, out=None, stream=None):
+    """Channelwise FP8 product C = As[m] Bs[n] (A B^T)[m, n] in bf16. A uint8 E4M3 [M, K], As f32
+    [M], B uint8 E4M3 [N, K], Bs f32 [N]."""
+    M, K = A.shape
+    N = B.shape[0]
+    if As.numel() != M or Bs.numel() != N:
+        raise ValueError("w8a8_channel_fp8_matmul: As must hold M and Bs N scales")
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=A.device) if out is None else out
+    _check(lib().w8a8_channel_fp8_matmul(
+        _dev(A, "A", _U8), _dev(As, "As", torch.float32), _dev(B, "B", _U8), _dev(Bs, "Bs", torch.float32),
+        M, N, K, _dev(out, "out", _BF16), _stream(stream)))
     return out
 
 

@@ -777,6 +777,8 @@ int w8a8_block_fp8_matmul(const uint8_t *A, const float *As, const uint8_t *B, c
     MOEQ_REQUIRE(B);
     MOEQ_REQUIRE(Bs);
     MOEQ_REQUIRE(C);
+    if (reinterpret_cast<uintptr_t>(A) % 16 || reinterpret_cast<uintptr_t>(B) % 16 || reinterpret_cast<uintptr_t>(C) % 16)
+        return set_error(MOEQ_ERR_UNSUPPORTED, "w8a8_block_fp8_matmul: A, B and C must be 16-byte aligned");
     // up to 64 rows: swap-AB tiles with K split over a cluster (HBM bound); more rows: 128-row
     // activation tiles (CTA pairs from 256 rows)
     Fp8TcArgs t{};
@@ -790,10 +792,44 @@ int w8a8_block_fp8_matmul(const uint8_t *A, const float *As, const uint8_t *B, c
     if (!t.status) return set_error(MOEQ_ERR_CUDA, "w8a8_block_fp8_matmul: no device status word");
     trace::Scope ts(trace::DENSE, (cudaStream_t)stream);
     const int rc = M <= fp8_skinny_max_rows()
-                       ? launch_fp8_tc_skinny(t, A, B, pick_skinny_split(M, N, K), (cudaStream_t)stream)
+                       ? launch_fp8_tc_skinny(t, A, B, pick_skinny_split(M, N, K), false, (cudaStream_t)stream)
                        : launch_fp8_tc_gemm(t, A, B, (cudaStream_t)stream);
     if (rc) return rc;
     return check_launch("w8a8_block_fp8_matmul");
+}
+
+int w8a8_channel_fp8_matmul(const uint8_t *A, const float *As, const uint8_t *B, const float *Bs, int M, int N, int K,
+                            uint16_t *C, void *stream)
+{
+    g_err[0] = 0;
+    if (M < 0 || N < 1 || K < 1) return set_error(MOEQ_ERR_INVALID_ARG, "bad sizes M=%d N=%d K=%d", M, N, K);
+    if (K % 128) return set_error(MOEQ_ERR_UNSUPPORTED, "K must be a multiple of 128 (got %d)", K);
+    if (N % 128) return set_error(MOEQ_ERR_UNSUPPORTED, "N must be a multiple of 128 (got %d)", N);
+    if (M == 0) return MOEQ_OK;
+    MOEQ_REQUIRE(A);
+    MOEQ_REQUIRE(As);
+    MOEQ_REQUIRE(B);
+    MOEQ_REQUIRE(Bs);
+    MOEQ_REQUIRE(C);
+    if (reinterpret_cast<uintptr_t>(A) % 16 || reinterpret_cast<uintptr_t>(B) % 16 || reinterpret_cast<uintptr_t>(C) % 16)
+        return set_error(MOEQ_ERR_UNSUPPORTED, "w8a8_channel_fp8_matmul: A, B and C must be 16-byte aligned");
+    // up to 64 rows: swap-AB tiles, K split over a cluster; more rows: 128-row activation tiles
+    // (CTA pairs from 256 rows); both accumulate all of K in tensor memory and scale once
+    Fp8TcArgs t{};
+    t.a_scale = As;
+    t.b_scale = Bs;
+    t.C = C;
+    t.M = M;
+    t.N = N;
+    t.K = K;
+    t.status = device_status_ptr();
+    if (!t.status) return set_error(MOEQ_ERR_CUDA, "w8a8_channel_fp8_matmul: no device status word");
+    trace::Scope ts(trace::DENSE, (cudaStream_t)stream);
+    const int rc = M <= fp8_skinny_max_rows()
+                       ? launch_fp8_tc_skinny(t, A, B, pick_skinny_split(M, N, K), true, (cudaStream_t)stream)
+                       : launch_fp8_tc_channel(t, A, B, (cudaStream_t)stream);
+    if (rc) return rc;
+    return check_launch("w8a8_channel_fp8_matmul");
 }
 
 int moe_trace_enable(int enable)

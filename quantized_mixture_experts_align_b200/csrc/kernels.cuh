@@ -49,7 +49,9 @@ struct F8GroupedArgs {
     uint16_t *y_out;         // [T*k, H] bf16, routing weight applied (down)
 };
 
-enum { TC_DENSE = 0, TC_GATEUP = 1, TC_DOWN = 2 };
+// TC_DENSE_CW: dense channelwise FP8 (a_scale [M] per token, b_scale [N] per channel): the whole
+// K accumulates in one tensor-memory buffer and the scales are applied once, in the epilogue.
+enum { TC_DENSE = 0, TC_GATEUP = 1, TC_DOWN = 2, TC_DENSE_CW = 3 };
 
 struct Fp8TcArgs {
     const float *a_scale;   // [M, K/128]: As (dense) or the gathered / intermediate row scales
@@ -100,10 +102,15 @@ void launch_w4a16_grouped_mma(const W4GroupedArgs &a, int mode, int block_m, int
 void launch_fp8_grouped_mma(const F8GroupedArgs &a, int mode, int block_m, int max_blocks, cudaStream_t s);
 // tcgen05 block-FP8 GEMM: A [M, K] and B [N, K] E4M3, K % 128 == 0, N % 128 == 0. Returns a status.
 int launch_fp8_tc_gemm(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B, cudaStream_t s);
+// Dense channelwise FP8 GEMM (a_scale [M], b_scale [N]) for M > fp8_skinny_max_rows().
+int launch_fp8_tc_channel(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B, cudaStream_t s);
 // Dense block-FP8 GEMM for M <= fp8_skinny_max_rows() rows (swap-AB tcgen05 tiles of 128 weight
 // rows, K split over a cluster of `split` CTAs reduced through distributed shared memory).
 int fp8_skinny_max_rows();
-int launch_fp8_tc_skinny(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B, int split, cudaStream_t s);
+// channelwise: a_scale [M] per token and b_scale [N] per channel, the whole K accumulated in one
+// tensor-memory buffer.
+int launch_fp8_tc_skinny(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B, int split, bool channelwise,
+                         cudaStream_t s);
 // tcgen05 grouped block-FP8 GEMM over expert-contiguous rows A [M, K] (128-row blocks, one expert
 // each, per expert_ids / ntp) and weights W [E * rows_per_expert, K]; mode TC_GATEUP or TC_DOWN.
 int launch_fp8_tc_grouped(const Fp8TcArgs &a, int mode, const uint8_t *A, const uint8_t *W, int E, int max_blocks,

@@ -51,7 +51,8 @@ struct Fp8TcShape {
     static constexpr int kABytes = kBM * kBK;
     static constexpr int kBBytes = (PAIR ? BN / 2 : BN) * kBK;
     static constexpr int kStageBytes = kABytes + kBBytes;
-    static constexpr int kTmemCols = 2 * BN;  // two partial buffers (128, 256 or 512 columns)
+    // two partial buffers (128, 256 or 512 columns); channelwise: one accumulator over all of K
+    static constexpr int kTmemCols = MODE == TC_DENSE_CW ? BN : 2 * BN;
     static constexpr int kSlices = epi_warps(MODE) / 4;  // column slices per lane quarter
     static constexpr int kColsPerWarp = BN / kSlices;
     static constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + 1024 + 256 + kSlices * 128 * 4;
@@ -65,6 +66,7 @@ __global__ void __launch_bounds__(fp8_threads(MODE), 1)
     using Sh = Fp8TcShape<BN, PAIR, MODE>;
     constexpr int kStages = Sh::kStages;
     constexpr int kEpiWarps = epi_warps(MODE);
+    constexpr bool kDense = MODE == TC_DENSE || MODE == TC_DENSE_CW;
     static_assert(!PAIR || BN == 256, "pair tiles are 256 x 256");
     static_assert(MODE != TC_GATEUP || BN == 256, "gate/up tiles hold 128 gate + 128 up columns");
     extern __shared__ uint8_t smem_raw[];
@@ -84,17 +86,17 @@ __global__ void __launch_bounds__(fp8_threads(MODE), 1)
     // pair: rank 0 holds rows [0, 128) of the 256-row tile, rank 1 rows [128, 256); x counts CTAs
     const uint32_t rank = PAIR ? tc::cluster_rank() : 0u;
     const int tile_x = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
-    const int m0 = PAIR ? (MODE == TC_DENSE ? tile_x : (int)blockIdx.y) * 2 * kBM + (int)rank * kBM
-                        : (MODE == TC_DENSE ? tile_x : (int)blockIdx.y) * kBM;
+    const int m0 = PAIR ? (kDense ? tile_x : (int)blockIdx.y) * 2 * kBM + (int)rank * kBM
+                        : (kDense ? tile_x : (int)blockIdx.y) * kBM;
     const int KB = a.K / kBK;
     // output columns of this tile and the weight rows (in the [E * rows, K] weight matrix) loaded
     // into the B stage: dense and down take BN consecutive rows; gate/up takes 128 gate + 128 up
     int n0, brow0, brow1 = 0;
     const float *bscale0, *bscale1 = nullptr;
-    if (MODE == TC_DENSE) {
+    if (kDense) {
         n0 = blockIdx.y * BN;
         brow0 = n0;
-        bscale0 = a.b_scale + (size_t)(n0 / 128) * KB;
+        bscale0 = MODE == TC_DENSE_CW ? a.b_scale + n0 : a.b_scale + (size_t)(n0 / 128) * KB;
     } else {
         // uniform over the CTA (and the pair: both test the pair's first row), before any barrier
         if ((PAIR ? (int)blockIdx.y * 2 * kBM : m0) >= __ldg(a.ntp)) return;
@@ -183,35 +185,72 @@ __global__ void __launch_bounds__(fp8_threads(MODE), 1)
             constexpr uint32_t idesc = tc::idesc_f32(tc::kFmtE4M3, tc::kFmtE4M3, PAIR ? 2 * kBM : kBM, BN);
             const uint64_t a_base = tc::smem_desc_sw128(smem);
             for (int kb = 0; kb < KB; ++kb) {
-                const int s = kb % kStages, buf = kb & 1;
+                const int s = kb % kStages, buf = MODE == TC_DENSE_CW ? 0 : kb & 1;
                 if (!tc::mbar_wait(&full[s], (kb / kStages) & 1, abort_flag, a.status)) break;
-                if (kb >= 2 && !tc::mbar_wait(&tempty[buf], ((kb >> 1) & 1) ^ 1, abort_flag, a.status)) break;
+                if (MODE != TC_DENSE_CW && kb >= 2 &&
+                    !tc::mbar_wait(&tempty[buf], ((kb >> 1) & 1) ^ 1, abort_flag, a.status))
+                    break;
                 tc::fence_after_sync();
                 // lean issue path: descriptors from a precomputed base; the first MMA of each K block
                 // starts the partial, the other three always accumulate
                 const uint64_t adesc = a_base + (uint64_t)((s * Sh::kStageBytes) >> 4);
                 const uint64_t bdesc = adesc + (uint64_t)(Sh::kABytes >> 4);
                 const uint32_t d = tmem + buf * BN;
+                // channelwise: only the very first MMA starts the accumulator
+                const uint32_t first_acc = (MODE == TC_DENSE_CW && kb > 0) ? 1u : 0u;
                 if (PAIR) {
-                    tc::mma_f8f6f4_ss_pair(d, adesc, bdesc, idesc, 0u);
+                    tc::mma_f8f6f4_ss_pair(d, adesc, bdesc, idesc, first_acc);
 #pragma unroll
                     for (int kk = 1; kk < kBK / 32; ++kk)
                         tc::mma_f8f6f4_ss_pair_acc(d, adesc + 2 * kk, bdesc + 2 * kk, idesc);
                     tc::mma_commit_pair(&empty[s], 0x3);
-                    tc::mma_commit_pair(&tfull[buf], 0x3);
+                    if (MODE != TC_DENSE_CW) tc::mma_commit_pair(&tfull[buf], 0x3);
                 } else {
-                    tc::mma_f8f6f4_ss(d, adesc, bdesc, idesc, 0u);
+                    tc::mma_f8f6f4_ss(d, adesc, bdesc, idesc, first_acc);
 #pragma unroll
                     for (int kk = 1; kk < kBK / 32; ++kk)
                         tc::mma_f8f6f4_ss_acc(d, adesc + 2 * kk, bdesc + 2 * kk, idesc);
                     tc::mma_commit(&empty[s]);
-                    tc::mma_commit(&tfull[buf]);
+                    if (MODE != TC_DENSE_CW) tc::mma_commit(&tfull[buf]);
                 }
+            }
+            // channelwise: the accumulator is complete once every MMA issued so far has finished
+            if (MODE == TC_DENSE_CW) {
+                if (PAIR) tc::mma_commit_pair(&tfull[0], 0x3);
+                else tc::mma_commit(&tfull[0]);
             }
             // every MMA issued must finish before tensor memory is released
             if (PAIR) tc::mma_commit_pair(mma_done, 0x3);
             else tc::mma_commit(mma_done);
             tc::mbar_drain(mma_done, 0, a.status);
+        }
+    } else if (MODE == TC_DENSE_CW) {
+        // warp w: tensor-memory lanes 32 (w % 4) .. +31 (= tile rows) and column slice cq; one
+        // wait for the finished accumulator, then C = acc * As[m] * Bs[n] in bf16
+        constexpr int COLS = Sh::kColsPerWarp;
+        const int quarter = warp & 3, cq = (warp - 2) >> 2;
+        const int m = m0 + quarter * 32 + lane;
+        if (tc::mbar_wait_warp(&tfull[0], 0, abort_flag, a.status)) {
+            tc::fence_after_sync();
+            const float sa = __ldg(a.a_scale + (m < a.M ? m : a.M - 1));
+            const float *bs = bscale0 + cq * COLS;
+            const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + cq * COLS;
+            uint16_t *crow = a.C + (size_t)m * a.N + n0 + cq * COLS;
+#pragma unroll 1
+            for (int c = 0; c < COLS / 16; ++c) {
+                uint32_t r[16];
+                tc::tmem_ld16(taddr + c * 16, r);
+                tc::tmem_wait_ld();
+                if (m < a.M) {
+                    uint32_t o[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        o[j] = pack_bf16x2(__uint_as_float(r[2 * j]) * sa * __ldg(bs + c * 16 + 2 * j),
+                                           __uint_as_float(r[2 * j + 1]) * sa * __ldg(bs + c * 16 + 2 * j + 1));
+                    *reinterpret_cast<uint4 *>(crow + c * 16) = make_uint4(o[0], o[1], o[2], o[3]);
+                    *reinterpret_cast<uint4 *>(crow + c * 16 + 8) = make_uint4(o[4], o[5], o[6], o[7]);
+                }
+            }
         }
     } else {
         // warp w: tensor-memory lanes 32 (w % 4) .. +31 (= tile rows) and column slice cq
@@ -392,6 +431,21 @@ int launch_fp8_tc_gemm(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B, c
     if (pair) return launch_tc<256, TC_DENSE, true>(a, tmA, tmB, 2 * cdiv(a.M, 2 * kBM), a.N / 256, s);
     if (bn == 256) return launch_tc<256, TC_DENSE>(a, tmA, tmB, cdiv(a.M, kBM), a.N / 256, s);
     return launch_tc<128, TC_DENSE>(a, tmA, tmB, cdiv(a.M, kBM), a.N / 128, s);
+}
+
+int launch_fp8_tc_channel(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B, cudaStream_t s)
+{
+    // the block-scaled GEMM's tiles: 256 columns where N allows, CTA pairs from 256 rows
+    const int bn = (a.N % 256 == 0) ? 256 : 128;
+    const bool pair = bn == 256 && a.M >= 256;
+    CUtensorMap tmA, tmB;
+    int rc = make_tmap_2d(&tmA, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.M, (uint64_t)a.K, kBM, kBK);
+    if (rc) return rc;
+    rc = make_tmap_2d(&tmB, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.N, (uint64_t)a.K, pair ? 128 : bn, kBK);
+    if (rc) return rc;
+    if (pair) return launch_tc<256, TC_DENSE_CW, true>(a, tmA, tmB, 2 * cdiv(a.M, 2 * kBM), a.N / 256, s);
+    if (bn == 256) return launch_tc<256, TC_DENSE_CW>(a, tmA, tmB, cdiv(a.M, kBM), a.N / 256, s);
+    return launch_tc<128, TC_DENSE_CW>(a, tmA, tmB, cdiv(a.M, kBM), a.N / 128, s);
 }
 
 int launch_fp8_tc_grouped(const Fp8TcArgs &a, int mode, const uint8_t *A, const uint8_t *W, int E, int max_blocks,

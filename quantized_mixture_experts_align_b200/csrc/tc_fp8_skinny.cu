@@ -36,8 +36,9 @@ constexpr int kWBytes = kRows * kBK;
 
 // MP padded rows; G K blocks per pipeline step (one wait, one MMA batch, one commit and one
 // promotion pass per step: the hand-offs between the roles, not the bytes, set the time of a
-// step); TWO: the shared memory of two CTAs fits on one SM.
-template <int MP, int G, bool TWO>
+// step); TWO: the shared memory of two CTAs fits on one SM; CW: channelwise scales (per token,
+// per channel), the CTA's whole K range accumulated in one buffer and scaled once.
+template <int MP, int G, bool TWO, bool CW>
 struct SkinnyShape {
     static constexpr int kEpiWarps = MP <= 64 ? 4 : 8;        // <= 64 accumulators per thread
     static constexpr int kThreads = (2 + kEpiWarps) * 32;
@@ -45,7 +46,7 @@ struct SkinnyShape {
     static constexpr int kKbBytes = kWBytes + MP * kBK;       // one K block: weights + activations
     static constexpr int kStageBytes = G * kKbBytes;          // multiple of 1024 (MP >= 16)
     static constexpr int kStages = (TWO ? 104 * 1024 : 200 * 1024) / kStageBytes;
-    static constexpr int kBufCols = G * MP;                   // one partial buffer: G blocks
+    static constexpr int kBufCols = CW ? MP : G * MP;         // one partial buffer: G blocks
     static constexpr int kTmemCols = 2 * kBufCols < 32 ? 32 : 2 * kBufCols;
     static_assert(kStages >= 2, "at least two pipeline stages");
     static_assert(kTmemCols <= (TWO ? 256 : 512), "tensor memory of the CTAs on one SM");
@@ -67,12 +68,12 @@ __device__ __forceinline__ float4 ld_cluster_f32x4(uint32_t addr)
     return v;
 }
 
-template <int MP, int G, bool TWO>
-__global__ void __launch_bounds__(SkinnyShape<MP, G, TWO>::kThreads, TWO ? 2 : 1)
+template <int MP, int G, bool TWO, bool CW>
+__global__ void __launch_bounds__(SkinnyShape<MP, G, TWO, CW>::kThreads, TWO ? 2 : 1)
     fp8_tc_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                          Fp8TcArgs a, int split)
 {
-    using Sh = SkinnyShape<MP, G, TWO>;
+    using Sh = SkinnyShape<MP, G, TWO, CW>;
     constexpr int kStages = Sh::kStages, kEpiWarps = Sh::kEpiWarps, COLS = Sh::kCols;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -146,23 +147,44 @@ __global__ void __launch_bounds__(SkinnyShape<MP, G, TWO>::kThreads, TWO ? 2 : 1
             for (int i = 0; i < nstep; ++i) {
                 const int s = i % kStages, buf = i & 1, ng = min(G, nkb - i * G);
                 if (!tc::mbar_wait(&full[s], (i / kStages) & 1, abort_flag, a.status)) break;
-                if (i >= 2 && !tc::mbar_wait(&tempty[buf], ((i >> 1) & 1) ^ 1, abort_flag, a.status)) break;
+                if (!CW && i >= 2 && !tc::mbar_wait(&tempty[buf], ((i >> 1) & 1) ^ 1, abort_flag, a.status)) break;
                 tc::fence_after_sync();
                 for (int g = 0; g < ng; ++g) {
-                    // block g of the step: its own MP columns of the partial buffer
+                    // block g of the step: its own MP columns of the partial buffer (channelwise:
+                    // all blocks into one accumulator, started by the very first MMA)
                     const uint64_t wdesc = base + (uint64_t)((s * Sh::kStageBytes + g * Sh::kKbBytes) >> 4);
                     const uint64_t xdesc = wdesc + (uint64_t)(kWBytes >> 4);
-                    const uint32_t d = tmem + buf * Sh::kBufCols + g * MP;
-                    tc::mma_f8f6f4_ss(d, wdesc, xdesc, idesc, 0u);
+                    const uint32_t d = CW ? tmem : tmem + buf * Sh::kBufCols + g * MP;
+                    tc::mma_f8f6f4_ss(d, wdesc, xdesc, idesc, (CW && (i > 0 || g > 0)) ? 1u : 0u);
 #pragma unroll
                     for (int kk = 1; kk < kBK / 32; ++kk)
                         tc::mma_f8f6f4_ss_acc(d, wdesc + 2 * kk, xdesc + 2 * kk, idesc);
                 }
                 tc::mma_commit(&empty[s]);
-                tc::mma_commit(&tfull[buf]);
+                if (!CW) tc::mma_commit(&tfull[buf]);
             }
+            if (CW) tc::mma_commit(&tfull[0]);
             tc::mma_commit(mma_done);
             tc::mbar_drain(mma_done, 0, a.status);
+        }
+    } else if (CW) {
+        // one wait for the accumulated K range; acc = partial * As[m] * Bs[n0 + row] (padding
+        // rows m >= M get 0)
+        if (tc::mbar_wait_warp(&tfull[0], 0, abort_flag, a.status)) {
+            tc::fence_after_sync();
+            const float sb = __ldg(a.b_scale + n0 + row);
+            const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + cq * COLS;
+#pragma unroll
+            for (int c = 0; c < COLS / 16; ++c) {
+                uint32_t r[16];
+                tc::tmem_ld16(taddr + c * 16, r);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const int m = cq * COLS + c * 16 + j;
+                    acc[c * 16 + j] = m < a.M ? __uint_as_float(r[j]) * __ldg(a.a_scale + m) * sb : 0.f;
+                }
+            }
         }
     } else {
         // scale products of this CTA's K blocks: sct[i][m] = As[m, kb0 + i] * Bs[n0 / 128, kb0 + i]
@@ -240,10 +262,10 @@ __global__ void __launch_bounds__(SkinnyShape<MP, G, TWO>::kThreads, TWO ? 2 : 1
     if (warp == 1) tc::tmem_dealloc(tmem, Sh::kTmemCols);
 }
 
-template <int MP, int G, bool TWO>
+template <int MP, int G, bool TWO, bool CW>
 int launch_skinny(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B, int split, cudaStream_t s)
 {
-    using Sh = SkinnyShape<MP, G, TWO>;
+    using Sh = SkinnyShape<MP, G, TWO, CW>;
     const int KB = a.K / kBK;
     // the per-block scale table grows with K / split: more CTAs per tile for very deep K
     while (Sh::smem_bytes((KB + split - 1) / split) > (TWO ? 113 : 227) * 1024 && split < 8 && split < KB) ++split;
@@ -253,7 +275,7 @@ int launch_skinny(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B, int sp
                          a.K, smem);
     static int attr_bytes = 0;
     if (attr_bytes < (int)smem) {
-        const cudaError_t e = cudaFuncSetAttribute(fp8_tc_skinny_kernel<MP, G, TWO>,
+        const cudaError_t e = cudaFuncSetAttribute(fp8_tc_skinny_kernel<MP, G, TWO, CW>,
                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess)
             return set_error(MOEQ_ERR_CUDA, "tcgen05 FP8 skinny GEMM: shared-memory attribute: %s",
@@ -277,7 +299,7 @@ int launch_skinny(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B, int sp
     at[0].val.clusterDim.z = 1;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, fp8_tc_skinny_kernel<MP, G, TWO>, tmW, tmX, a, split);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, fp8_tc_skinny_kernel<MP, G, TWO, CW>, tmW, tmX, a, split);
     if (e != cudaSuccess) return set_error(MOEQ_ERR_CUDA, "tcgen05 FP8 skinny GEMM launch: %s", cudaGetErrorString(e));
     return MOEQ_OK;
 }
@@ -286,7 +308,8 @@ int launch_skinny(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B, int sp
 
 int fp8_skinny_max_rows() { return 64; }
 
-int launch_fp8_tc_skinny(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B, int split, cudaStream_t s)
+int launch_fp8_tc_skinny(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B, int split, bool channelwise,
+                         cudaStream_t s)
 {
     const int KB = a.K / kBK;
     if (a.M < 1 || a.M > fp8_skinny_max_rows() || a.N % kRows || a.K % kBK)
@@ -295,9 +318,14 @@ int launch_fp8_tc_skinny(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B,
     if (split > 8) split = 8;  // portable cluster size
     if (split > KB) split = KB;
     // two K blocks per step, two CTAs per SM (measured best for every row count up to 64)
-    if (a.M <= 16) return launch_skinny<16, 2, true>(a, A, B, split, s);
-    if (a.M <= 32) return launch_skinny<32, 2, true>(a, A, B, split, s);
-    return launch_skinny<64, 2, true>(a, A, B, split, s);
+    if (channelwise) {
+        if (a.M <= 16) return launch_skinny<16, 2, true, true>(a, A, B, split, s);
+        if (a.M <= 32) return launch_skinny<32, 2, true, true>(a, A, B, split, s);
+        return launch_skinny<64, 2, true, true>(a, A, B, split, s);
+    }
+    if (a.M <= 16) return launch_skinny<16, 2, true, false>(a, A, B, split, s);
+    if (a.M <= 32) return launch_skinny<32, 2, true, false>(a, A, B, split, s);
+    return launch_skinny<64, 2, true, false>(a, A, B, split, s);
 }
 
 }  // namespace moeq

@@ -27,7 +27,7 @@ def _declared():
 def test_header_declares_the_boundary():
     names = set(_declared())
     for need in ("moe_route_topk", "moe_align", "moe_w4a16_forward", "moe_w8a8_block_fp8_forward",
-                 "w8a8_block_fp8_matmul", "moe_fp8_act_quant", "moe_last_error"):
+                 "w8a8_block_fp8_matmul", "w8a8_channel_fp8_matmul", "moe_fp8_act_quant", "moe_last_error"):
         assert need in names
 
 
@@ -86,6 +86,17 @@ def test_validation_rejects_before_device_work(L):
     assert _rc(L, "w8a8_block_fp8_matmul", N, N, N, N, 4, 256, 256, 64, 128, N, N) == moeq.MOEQ_ERR_UNSUPPORTED
     assert _rc(L, "w8a8_block_fp8_matmul", N, N, N, N, 4, 256, 200, 128, 128, N, N) == moeq.MOEQ_ERR_UNSUPPORTED
     assert _rc(L, "w8a8_block_fp8_matmul", N, N, N, N, 4, 200, 256, 128, 128, N, N) == moeq.MOEQ_ERR_UNSUPPORTED
+    # channelwise dense matmul: K, N multiples of 128; aligned A, B, C; NULL scales
+    cw = lambda A_, As_, C_, M, Nn, K: _rc(L, "w8a8_channel_fp8_matmul", A_, As_, p, p, M, Nn, K, C_, N)
+    assert cw(p, p, p, 4, 256, 200) == moeq.MOEQ_ERR_UNSUPPORTED
+    assert cw(p, p, p, 4, 200, 256) == moeq.MOEQ_ERR_UNSUPPORTED
+    assert cw(p, N, p, 4, 256, 256) == moeq.MOEQ_ERR_INVALID_ARG
+    assert cw(p, p, p, -1, 256, 256) == moeq.MOEQ_ERR_INVALID_ARG
+    assert cw(p, p, ctypes.c_void_p(p.value + 8), 4, 256, 256) == moeq.MOEQ_ERR_UNSUPPORTED
+    assert cw(ctypes.c_void_p(p.value + 4), p, p, 4, 256, 256) == moeq.MOEQ_ERR_UNSUPPORTED
+    assert cw(N, N, N, 0, 256, 256) == moeq.MOEQ_OK
+    assert _rc(L, "w8a8_block_fp8_matmul", p, p, p, p, 4, 256, 256, 128, 128, ctypes.c_void_p(p.value + 2), N) == \
+        moeq.MOEQ_ERR_UNSUPPORTED
     # grouped W4A16 GEMM: shapes, row map, workspace
     gc = lambda M, K, Nn, G, idx, ws, wsb: _rc(L, "moe_w4a16_grouped_contiguous", p, M, K, p, p, G, Nn, idx, p, ws, wsb, N)
     assert gc(64, 100, 256, 4, p, p, 1 << 40) == moeq.MOEQ_ERR_UNSUPPORTED       # K % 128

@@ -316,6 +316,47 @@ def test_dense_fp8_full_shape_sampled(M):
     _dense_parity(M, 24576, 7168, rows)
 
 
+def _channel_parity(M, N, K, rows, what=""):
+    d = W.make_dense_fp8_channel(W.WORKLOADS["dense_fp8_channel"], M, device=DEV, N=N, K=K)
+    C = moeq.w8a8_channel_fp8_matmul(d["A"], d["As"], d["B"], d["Bs"])
+    torch.cuda.synchronize()
+    ref = oracle.fp8_channel_matmul(W.np_bits(d["A"]), W.np_bits(d["As"]), W.np_bits(d["B"]), W.np_bits(d["Bs"]),
+                                    rows=rows)
+    assert_layer_close(bf16_to_f64(C[torch.as_tensor(rows, device=DEV).long()]), ref, TOL_FP8,
+                       f"channelwise M={M} N={N} K={K} {what}")
+    assert moeq.moe_device_status() == 0
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 256, 1024), (5, 256, 896), (16, 128, 384), (33, 1280, 2944),
+                                   (64, 384, 128), (65, 256, 1024), (128, 384, 640), (200, 512, 512),
+                                   (256, 512, 384), (257, 768, 640), (640, 256, 1152)])
+def test_dense_fp8_channel_shapes_all_rows(M, N, K):
+    """Every schedule of the channelwise GEMM: the few-row swap-AB kernel (cluster K split, 16 /
+    32 / 64 padded rows), 128- and 256-column tiles, CTA pairs from 256 rows, ragged row tails."""
+    _channel_parity(M, N, K, np.arange(M, dtype=np.int32))
+
+
+@pytest.mark.parametrize("M", [1, 64, 4096])
+def test_dense_fp8_channel_page_shape_sampled(M):
+    """The N = K = 4096 shape of the SGLang channelwise config example, rows sampled."""
+    rows = np.unique(np.array([0, M - 1, M // 2, M // 3], np.int32))
+    _channel_parity(M, 4096, 4096, rows)
+
+
+def test_dense_fp8_channel_closed_form():
+    """All codes 448 with As[m] = 2^(m % 4) / 448 and Bs[n] = (1 + n % 3) / 448: C[m, n] =
+    K 2^(m % 4) (1 + n % 3), exact in bf16 for K = 1024 (row and column scale indexing)."""
+    for M in (3, 300):
+        N, K = 384, 1024
+        A = torch.full((M, K), 0x7E, dtype=torch.uint8, device=DEV)
+        B = torch.full((N, K), 0x7E, dtype=torch.uint8, device=DEV)
+        As = torch.tensor([2.0 ** (m % 4) / 448.0 for m in range(M)], device=DEV)
+        Bs = torch.tensor([(1 + n % 3) / 448.0 for n in range(N)], device=DEV)
+        C = moeq.w8a8_channel_fp8_matmul(A, As, B, Bs).double().cpu().numpy()
+        want = K * np.array([2.0 ** (m % 4) for m in range(M)])[:, None] * np.array([1 + n % 3 for n in range(N)])[None, :]
+        assert np.allclose(C, want, rtol=2 ** -8), f"M={M}"
+
+
 def test_dense_fp8_closed_form_ones():
     M, N, K = 4, 256, 7168
     A = torch.full((M, K), 0x7E, dtype=torch.uint8, device=DEV)
