@@ -58,6 +58,21 @@ struct Fp8TcShape {
     static constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + 1024 + 256 + kSlices * 128 * 4;
 };
 
+// partial-tile row pitch in floats for the K-split sum: BN + 4 keeps the float4 stores of 8
+// consecutive rows (one quarter warp) on distinct banks
+template <int BN>
+__host__ __device__ constexpr int kRedStride() { return BN + 4; }
+
+__device__ __forceinline__ float4 ld_cluster_f32x4(uint32_t addr)
+{
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
+
 template <int BN, int MODE, bool PAIR>
 __global__ void __launch_bounds__(fp8_threads(MODE), 1)
     fp8_tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -68,6 +83,8 @@ __global__ void __launch_bounds__(fp8_threads(MODE), 1)
     constexpr int kEpiWarps = epi_warps(MODE);
     constexpr bool kDense = MODE == TC_DENSE || MODE == TC_DENSE_CW;
     static_assert(!PAIR || BN == 256, "pair tiles are 256 x 256");
+    static_assert(PAIR || (size_t)kBM * kRedStride<BN>() * 4 <= (size_t)kStages * Sh::kStageBytes,
+                  "the K-split partial tile must fit in the stage ring");
     static_assert(MODE != TC_GATEUP || BN == 256, "gate/up tiles hold 128 gate + 128 up columns");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -89,6 +106,11 @@ __global__ void __launch_bounds__(fp8_threads(MODE), 1)
     const int m0 = PAIR ? (kDense ? tile_x : (int)blockIdx.y) * 2 * kBM + (int)rank * kBM
                         : (kDense ? tile_x : (int)blockIdx.y) * kBM;
     const int KB = a.K / kBK;
+    // K split (dense, no pair): the gridDim.z CTAs of a cluster take contiguous K-block ranges of
+    // the same tile and sum their partial tiles through distributed shared memory at the end
+    const int nsplit = (kDense && !PAIR) ? (int)gridDim.z : 1;
+    const int kb0 = (kDense && !PAIR) ? (int)blockIdx.z * KB / nsplit : 0;
+    const int nkb = (kDense && !PAIR) ? ((int)blockIdx.z + 1) * KB / nsplit - kb0 : KB;
     // output columns of this tile and the weight rows (in the [E * rows, K] weight matrix) loaded
     // into the B stage: dense and down take BN consecutive rows; gate/up takes 128 gate + 128 up
     int n0, brow0, brow1 = 0;
@@ -147,7 +169,7 @@ __global__ void __launch_bounds__(fp8_threads(MODE), 1)
             tc::prefetch_tmap(&tmA);
             tc::prefetch_tmap(&tmB);
             int issued = 0;
-            for (int kb = 0; kb < KB; ++kb) {
+            for (int kb = 0; kb < nkb; ++kb) {  // local index; x = (kb0 + kb) * kBK
                 const int s = kb % kStages;
                 if (kb >= kStages && !tc::mbar_wait(&empty[s], ((kb / kStages) & 1) ^ 1, abort_flag, a.status)) break;
                 uint8_t *sa = smem + s * Sh::kStageBytes;
@@ -161,12 +183,13 @@ __global__ void __launch_bounds__(fp8_threads(MODE), 1)
                     continue;
                 }
                 tc::mbar_arrive_expect_tx(&full[s], Sh::kStageBytes);
-                tc::tma_load_2d(sa, &tmA, &full[s], kb * kBK, m0);
+                const int x = (kb0 + kb) * kBK;
+                tc::tma_load_2d(sa, &tmA, &full[s], x, m0);
                 if (MODE == TC_GATEUP) {
-                    tc::tma_load_2d(sa + Sh::kABytes, &tmB, &full[s], kb * kBK, brow0);
-                    tc::tma_load_2d(sa + Sh::kABytes + 128 * kBK, &tmB, &full[s], kb * kBK, brow1);
+                    tc::tma_load_2d(sa + Sh::kABytes, &tmB, &full[s], x, brow0);
+                    tc::tma_load_2d(sa + Sh::kABytes + 128 * kBK, &tmB, &full[s], x, brow1);
                 } else {
-                    tc::tma_load_2d(sa + Sh::kABytes, &tmB, &full[s], kb * kBK, brow0);
+                    tc::tma_load_2d(sa + Sh::kABytes, &tmB, &full[s], x, brow0);
                 }
                 issued = kb + 1;
             }
@@ -184,7 +207,7 @@ __global__ void __launch_bounds__(fp8_threads(MODE), 1)
         } else if (lane == 0) {
             constexpr uint32_t idesc = tc::idesc_f32(tc::kFmtE4M3, tc::kFmtE4M3, PAIR ? 2 * kBM : kBM, BN);
             const uint64_t a_base = tc::smem_desc_sw128(smem);
-            for (int kb = 0; kb < KB; ++kb) {
+            for (int kb = 0; kb < nkb; ++kb) {
                 const int s = kb % kStages, buf = MODE == TC_DENSE_CW ? 0 : kb & 1;
                 if (!tc::mbar_wait(&full[s], (kb / kStages) & 1, abort_flag, a.status)) break;
                 if (MODE != TC_DENSE_CW && kb >= 2 &&
@@ -236,12 +259,22 @@ __global__ void __launch_bounds__(fp8_threads(MODE), 1)
             const float *bs = bscale0 + cq * COLS;
             const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + cq * COLS;
             uint16_t *crow = a.C + (size_t)m * a.N + n0 + cq * COLS;
+            float *red = reinterpret_cast<float *>(smem) + (size_t)(quarter * 32 + lane) * kRedStride<BN>() + cq * COLS;
 #pragma unroll 1
             for (int c = 0; c < COLS / 16; ++c) {
                 uint32_t r[16];
                 tc::tmem_ld16(taddr + c * 16, r);
                 tc::tmem_wait_ld();
-                if (m < a.M) {
+                if (nsplit > 1) {
+                    // K split: the scaled partial tile goes to shared memory for the cluster sum
+#pragma unroll
+                    for (int j = 0; j < 16; j += 4)
+                        *reinterpret_cast<float4 *>(red + c * 16 + j) = make_float4(
+                            __uint_as_float(r[j]) * sa * __ldg(bs + c * 16 + j),
+                            __uint_as_float(r[j + 1]) * sa * __ldg(bs + c * 16 + j + 1),
+                            __uint_as_float(r[j + 2]) * sa * __ldg(bs + c * 16 + j + 2),
+                            __uint_as_float(r[j + 3]) * sa * __ldg(bs + c * 16 + j + 3));
+                } else if (m < a.M) {
                     uint32_t o[8];
 #pragma unroll
                     for (int j = 0; j < 8; ++j)
@@ -263,19 +296,19 @@ __global__ void __launch_bounds__(fp8_threads(MODE), 1)
         // columns and the GF matching up columns
         const int c_first = (MODE == TC_GATEUP) ? GF * cq : cq * COLS;
         const int c_second = (MODE == TC_GATEUP) ? 128 + GF * cq : 0;
-        const float *as_row = a.a_scale + (size_t)(m < a.M ? m : a.M - 1) * KB;
-        const float *bs_first = (MODE == TC_GATEUP) ? bscale0 : bscale0 + (size_t)((cq * COLS) / 128) * KB;
-        const float *bs_second = (MODE == TC_GATEUP) ? bscale1 : bs_first;
+        const float *as_row = a.a_scale + (size_t)(m < a.M ? m : a.M - 1) * KB + kb0;
+        const float *bs_first = ((MODE == TC_GATEUP) ? bscale0 : bscale0 + (size_t)((cq * COLS) / 128) * KB) + kb0;
+        const float *bs_second = (MODE == TC_GATEUP) ? bscale1 + kb0 : bs_first;
         float acc[COLS];
 #pragma unroll
         for (int j = 0; j < COLS; ++j) acc[j] = 0.f;
         bool ok = true;
         // the scales of block kb + 1 are loaded while block kb's partial is awaited
         float n_sa = __ldg(as_row), n_b0 = __ldg(bs_first), n_b1 = __ldg(bs_second);
-        for (int kb = 0; kb < KB && ok; ++kb) {
+        for (int kb = 0; kb < nkb && ok; ++kb) {
             const int buf = kb & 1;
             const float sc0 = n_sa * n_b0, sc1 = n_sa * n_b1;
-            if (kb + 1 < KB) {
+            if (kb + 1 < nkb) {
                 n_sa = __ldg(as_row + kb + 1);
                 n_b0 = __ldg(bs_first + kb + 1);
                 n_b1 = __ldg(bs_second + kb + 1);
@@ -306,7 +339,14 @@ __global__ void __launch_bounds__(fp8_threads(MODE), 1)
                 else tc::mbar_arrive(&tempty[buf]);
             }
         }
-        if (MODE == TC_DENSE) {
+        if (MODE == TC_DENSE && nsplit > 1) {
+            // every MMA has completed (the last partial was awaited) and every copy landed: the
+            // ring holds this CTA's partial tile, rows padded to kRedStride floats
+            float *red = reinterpret_cast<float *>(smem) + (size_t)row * kRedStride<BN>() + cq * COLS;
+#pragma unroll
+            for (int j = 0; j < COLS; j += 4)
+                *reinterpret_cast<float4 *>(red + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+        } else if (MODE == TC_DENSE) {
             if (ok && m < a.M) {
                 uint16_t *crow = a.C + (size_t)m * a.N + n0 + cq * COLS;
 #pragma unroll
@@ -368,8 +408,39 @@ __global__ void __launch_bounds__(fp8_threads(MODE), 1)
         }
     }
     tc::fence_before_sync();
-    if (PAIR) tc::cluster_sync();  // neither CTA leaves while the pair's copies or MMAs use it
-    else __syncthreads();
+    if (kDense && !PAIR && nsplit > 1) {
+        // K split: rank r sums rows [128 r / S, 128 (r + 1) / S) of the S partial tiles in rank
+        // order (deterministic) and writes bf16 C; a second barrier keeps every CTA's partial tile
+        // alive until all ranks have read it
+        tc::cluster_sync();
+        const int r = (int)blockIdx.z;
+        const int row_lo = r * kBM / nsplit, row_hi = (r + 1) * kBM / nsplit;
+        constexpr int kUnits = BN / 4;
+        const float *red = reinterpret_cast<const float *>(smem);
+        for (int u = threadIdx.x; u < (row_hi - row_lo) * kUnits; u += fp8_threads(MODE)) {
+            const int row = row_lo + u / kUnits, col = (u % kUnits) * 4;
+            const int m = m0 + row;
+            if (m >= a.M) continue;
+            const float *src = red + (size_t)row * kRedStride<BN>() + col;
+            float4 t = ld_cluster_f32x4(tc::cluster_addr(src, 0));
+            for (int q = 1; q < nsplit; ++q) {
+                const float4 v = ld_cluster_f32x4(tc::cluster_addr(src, (uint32_t)q));
+                t.x += v.x;
+                t.y += v.y;
+                t.z += v.z;
+                t.w += v.w;
+            }
+            uint2 o;
+            o.x = pack_bf16x2(t.x, t.y);
+            o.y = pack_bf16x2(t.z, t.w);
+            *reinterpret_cast<uint2 *>(a.C + (size_t)m * a.N + n0 + col) = o;
+        }
+        tc::cluster_sync();
+    } else if (PAIR) {
+        tc::cluster_sync();  // neither CTA leaves while the pair's copies or MMAs use it
+    } else {
+        __syncthreads();
+    }
     tc::fence_after_sync();
     if (warp == 1) {
         if (PAIR) tc::tmem_dealloc_pair(tmem, Sh::kTmemCols);
@@ -379,7 +450,7 @@ __global__ void __launch_bounds__(fp8_threads(MODE), 1)
 
 template <int BN, int MODE, bool PAIR = false>
 int launch_tc(const Fp8TcArgs &a, const CUtensorMap &tmA, const CUtensorMap &tmB, int grid_x, int grid_y,
-              cudaStream_t s)
+              cudaStream_t s, int split = 1)
 {
     using Sh = Fp8TcShape<BN, PAIR, MODE>;
     constexpr int kThreads = fp8_threads(MODE);
@@ -392,60 +463,84 @@ int launch_tc(const Fp8TcArgs &a, const CUtensorMap &tmA, const CUtensorMap &tmB
         attr = true;
     }
     if (grid_x <= 0 || grid_y <= 0) return MOEQ_OK;
-    if (!PAIR) {
+    if (!PAIR && split <= 1) {
         fp8_tc_gemm_kernel<BN, MODE, PAIR><<<dim3(grid_x, grid_y), kThreads, Sh::kSmemBytes, s>>>(tmA, tmB, a);
         return MOEQ_OK;
     }
-    // clusters of 2 CTAs along x (grid_x even): the pair of one 256-row tile
+    // clusters of 2 CTAs along x (grid_x even): the pair of one 256-row tile; or (K split)
+    // clusters of `split` CTAs along z: the K ranges of one tile
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid_x, grid_y);
+    cfg.gridDim = dim3(grid_x, grid_y, PAIR ? 1 : split);
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = Sh::kSmemBytes;
     cfg.stream = s;
     cudaLaunchAttribute attr_c[1];
     attr_c[0].id = cudaLaunchAttributeClusterDimension;
-    attr_c[0].val.clusterDim.x = 2;
+    attr_c[0].val.clusterDim.x = PAIR ? 2 : 1;
     attr_c[0].val.clusterDim.y = 1;
-    attr_c[0].val.clusterDim.z = 1;
+    attr_c[0].val.clusterDim.z = PAIR ? 1 : split;
     cfg.attrs = attr_c;
     cfg.numAttrs = 1;
     const cudaError_t e = cudaLaunchKernelEx(&cfg, fp8_tc_gemm_kernel<BN, MODE, PAIR>, tmA, tmB, a);
-    if (e != cudaSuccess) return set_error(MOEQ_ERR_CUDA, "tcgen05 FP8 pair GEMM launch: %s", cudaGetErrorString(e));
+    if (e != cudaSuccess) return set_error(MOEQ_ERR_CUDA, "tcgen05 FP8 clustered GEMM launch: %s", cudaGetErrorString(e));
     return MOEQ_OK;
 }
 
 }  // namespace
 
+// Dense schedule, from measured sweeps (clean L2): single CTAs (128 x BN tiles) beat CTA pairs by
+// 3-5 % on the block-scaled GEMM at 512-4096 rows of 24576 x 7168 (437 vs 451 us at 2048 rows,
+// 824 vs 863 at 4096); on the channelwise GEMM the two tie, and pairs (half the B bytes per CTA)
+// are kept there once the tiles fill two waves. The K range is split over a cluster only when the
+// tiles fill less than half of the SMs (4096 x 4096 channelwise, 128-256 rows: 24.6 -> 20.5 us
+// with a split of 4); with more tiles every split measured slower.
+struct DenseSchedule {
+    bool pair;
+    int split;
+};
+static DenseSchedule pick_dense_schedule(int M, int N, int K, int bn, bool channelwise)
+{
+    const int KB = K / kBK, sms = 148;
+    const long tiles = (long)cdiv(M, kBM) * (N / bn);
+    if (channelwise && bn == 256 && M >= 256 && tiles >= 2 * sms) return {true, 1};
+    if (2 * tiles < sms) {
+        long sp = sms / tiles;
+        if (sp > 4) sp = 4;
+        if (sp > KB / 2) sp = KB / 2;
+        return {false, sp < 1 ? 1 : (int)sp};
+    }
+    return {false, 1};
+}
+
 int launch_fp8_tc_gemm(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B, cudaStream_t s)
 {
     // Rows past 64 (fewer go to the swap-AB kernel): 256-column tiles (more weight bytes in flight
-    // per SM, fewer activation re-reads; tensor bound for many rows), chosen from measured M
-    // sweeps; from 256 rows, CTA pairs (256 x 256 tiles, half the weight rows per CTA).
+    // per SM, fewer activation re-reads; tensor bound for many rows), chosen from measured M sweeps.
     const int bn = (a.N % 256 == 0) ? 256 : 128;
-    const bool pair = bn == 256 && a.M >= 256;
+    const DenseSchedule sch = pick_dense_schedule(a.M, a.N, a.K, bn, false);
     CUtensorMap tmA, tmB;
     int rc = make_tmap_2d(&tmA, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.M, (uint64_t)a.K, kBM, kBK);
     if (rc) return rc;
-    rc = make_tmap_2d(&tmB, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.N, (uint64_t)a.K, pair ? 128 : bn, kBK);
+    rc = make_tmap_2d(&tmB, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.N, (uint64_t)a.K, bn, kBK);
     if (rc) return rc;
-    if (pair) return launch_tc<256, TC_DENSE, true>(a, tmA, tmB, 2 * cdiv(a.M, 2 * kBM), a.N / 256, s);
-    if (bn == 256) return launch_tc<256, TC_DENSE>(a, tmA, tmB, cdiv(a.M, kBM), a.N / 256, s);
-    return launch_tc<128, TC_DENSE>(a, tmA, tmB, cdiv(a.M, kBM), a.N / 128, s);
+    if (bn == 256) return launch_tc<256, TC_DENSE>(a, tmA, tmB, cdiv(a.M, kBM), a.N / 256, s, sch.split);
+    return launch_tc<128, TC_DENSE>(a, tmA, tmB, cdiv(a.M, kBM), a.N / 128, s, sch.split);
 }
 
 int launch_fp8_tc_channel(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B, cudaStream_t s)
 {
-    // the block-scaled GEMM's tiles: 256 columns where N allows, CTA pairs from 256 rows
+    // the block-scaled GEMM's tiles and schedule: 256 columns where N allows, CTA pairs or a K split
     const int bn = (a.N % 256 == 0) ? 256 : 128;
-    const bool pair = bn == 256 && a.M >= 256;
+    const DenseSchedule sch = pick_dense_schedule(a.M, a.N, a.K, bn, true);
     CUtensorMap tmA, tmB;
     int rc = make_tmap_2d(&tmA, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.M, (uint64_t)a.K, kBM, kBK);
     if (rc) return rc;
-    rc = make_tmap_2d(&tmB, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.N, (uint64_t)a.K, pair ? 128 : bn, kBK);
+    rc = make_tmap_2d(&tmB, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.N, (uint64_t)a.K, sch.pair ? 128 : bn,
+                      kBK);
     if (rc) return rc;
-    if (pair) return launch_tc<256, TC_DENSE_CW, true>(a, tmA, tmB, 2 * cdiv(a.M, 2 * kBM), a.N / 256, s);
-    if (bn == 256) return launch_tc<256, TC_DENSE_CW>(a, tmA, tmB, cdiv(a.M, kBM), a.N / 256, s);
-    return launch_tc<128, TC_DENSE_CW>(a, tmA, tmB, cdiv(a.M, kBM), a.N / 128, s);
+    if (sch.pair) return launch_tc<256, TC_DENSE_CW, true>(a, tmA, tmB, 2 * cdiv(a.M, 2 * kBM), a.N / 256, s);
+    if (bn == 256) return launch_tc<256, TC_DENSE_CW>(a, tmA, tmB, cdiv(a.M, kBM), a.N / 256, s, sch.split);
+    return launch_tc<128, TC_DENSE_CW>(a, tmA, tmB, cdiv(a.M, kBM), a.N / 128, s, sch.split);
 }
 
 int launch_fp8_tc_grouped(const Fp8TcArgs &a, int mode, const uint8_t *A, const uint8_t *W, int E, int max_blocks,

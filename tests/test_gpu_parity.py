@@ -303,10 +303,12 @@ def test_dense_fp8_skinny_split_shapes_all_rows(M, N, K):
 
 
 @pytest.mark.parametrize("M,N,K", [(128, 256, 1024), (200, 512, 512), (300, 384, 896), (1000, 256, 7168),
-                                   (256, 512, 384), (257, 768, 640), (640, 256, 1152)])
+                                   (256, 512, 384), (257, 768, 640), (640, 256, 1152), (2048, 2048, 1024),
+                                   (2200, 2048, 1024)])
 def test_dense_fp8_tensor_core_shapes_all_rows(M, N, K):
-    """Row counts at and past the tcgen05 threshold and the CTA-pair threshold (256 rows), ragged M
-    tails, N not a multiple of 256."""
+    """Row counts past the few-row kernel: 128- and 256-column tiles, the K range split over
+    clusters of 2 to 4 CTAs where the tiles are few (uneven K ranges), ragged M tails, N not a
+    multiple of 256."""
     _dense_parity(M, N, K, np.arange(M, dtype=np.int32))
 
 
@@ -329,10 +331,12 @@ def _channel_parity(M, N, K, rows, what=""):
 
 @pytest.mark.parametrize("M,N,K", [(1, 256, 1024), (5, 256, 896), (16, 128, 384), (33, 1280, 2944),
                                    (64, 384, 128), (65, 256, 1024), (128, 384, 640), (200, 512, 512),
-                                   (256, 512, 384), (257, 768, 640), (640, 256, 1152)])
+                                   (256, 512, 384), (257, 768, 640), (640, 256, 1152), (2200, 2048, 1024),
+                                   (2400, 4096, 256)])
 def test_dense_fp8_channel_shapes_all_rows(M, N, K):
     """Every schedule of the channelwise GEMM: the few-row swap-AB kernel (cluster K split, 16 /
-    32 / 64 padded rows), 128- and 256-column tiles, CTA pairs from 256 rows, ragged row tails."""
+    32 / 64 padded rows), 128- and 256-column tiles with and without a cluster K split, CTA pairs
+    (2400 rows: two waves of tiles, a ragged 256-row pair tile), ragged row tails."""
     _channel_parity(M, N, K, np.arange(M, dtype=np.int32))
 
 
