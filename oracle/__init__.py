@@ -101,6 +101,25 @@ def moe_w4a16(x, logits, k, w13q, w13s, w2q, w2s, tokens=None, want_h=False):
     return (out, h) if want_h else out
 
 
+def moe_mxfp4(x, logits, k, w13q, w13s, w2q, w2s, tokens=None, want_h=False):
+    """As moe_w4a16 with MXFP4 weights: E2M1 codes int32 [E, rows, K/8] (INT4 nibble order) and
+    UE8M0 group-32 scales uint8 [E, rows, K/32]."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    logits = np.ascontiguousarray(logits, dtype=np.float32)
+    T, H = x.shape
+    E = logits.shape[1]
+    I = w2q.shape[2] * 8
+    tok = _tokens(tokens, T)
+    out = np.zeros((len(tok), H), np.float64)
+    h = np.zeros((len(tok), k, I), np.uint16) if want_h else None
+    args = [np.ascontiguousarray(a) for a in (w13q, w13s, w2q, w2s)]
+    assert args[0].dtype == np.int32 and args[1].dtype == np.uint8 and args[3].dtype == np.uint8
+    rc = lib().orc_moe_mxfp4(_p(x), _p(logits), T, H, I, E, k, *[_p(a) for a in args], _p(tok), len(tok),
+                             _p(out), _p(h) if h is not None else None)
+    _check(rc, "moe_mxfp4")
+    return (out, h) if want_h else out
+
+
 def moe_fp8(x, logits, k, w13, w13s, w2, w2s, tokens=None, want_h=False):
     """W8A8 block-FP8 layer output (float64 [len(tokens), H]); optionally the quantized
     intermediate (uint8 [len(tokens), k, I], f32 [len(tokens), k, I/128])."""
@@ -206,6 +225,22 @@ def w4a16_dequant(q: np.ndarray, s: np.ndarray) -> np.ndarray:
     N, K8 = q.shape
     out = np.zeros((N, K8 * 8), np.float64)
     _check(lib().orc_w4a16_dequant(_p(q), _p(s), N, K8 * 8, _p(out)), "w4a16_dequant")
+    return out
+
+
+def mxfp4_dequant(q: np.ndarray, s: np.ndarray) -> np.ndarray:
+    q = np.ascontiguousarray(q, dtype=np.int32)
+    s = np.ascontiguousarray(s, dtype=np.uint8)
+    N, K8 = q.shape
+    out = np.zeros((N, K8 * 8), np.float64)
+    _check(lib().orc_mxfp4_dequant(_p(q), _p(s), N, K8 * 8, _p(out)), "mxfp4_dequant")
+    return out
+
+
+def e2m1_value(c: np.ndarray) -> np.ndarray:
+    c = np.ascontiguousarray(c, dtype=np.uint8)
+    out = np.zeros(c.shape, np.float64)
+    lib().orc_e2m1_value(_p(c), _p(out), ctypes.c_long(c.size))
     return out
 
 

@@ -201,6 +201,33 @@ static double w4_value(const int32_t *q, const uint16_t *s, int K, int r, int c)
     return (double)(code - 8) * bf16_value(s[(size_t)r * (K / 32) + c / 32]);
 }
 
+/* E2M1, the 4-bit float of the MXFP4 format (lk_moe page, "Supported models & quant formats"
+ * lists MXFP4): 1 sign bit, 2 exponent bits with bias 1, 1 mantissa bit; exponent 0 is the
+ * subnormal range (value = mantissa / 2), so the magnitudes are 0, 0.5, 1, 1.5, 2, 3, 4, 6. */
+static double e2m1_value(unsigned code)
+{
+    unsigned e = (code >> 1) & 3u, m = code & 1u;
+    double mag = e ? ldexp(1.0 + 0.5 * (double)m, (int)e - 1) : 0.5 * (double)m;
+    return (code & 8u) ? -mag : mag;
+}
+
+/* MXFP4 weight element: E2M1 code (same packing as the INT4 format: nibble j of int32 word w is
+ * input 8w + j) times the power-of-two scale of its 32-input group, a UE8M0 byte s meaning
+ * 2^(s - 127). READING: the pages name the format only; this is the OCP microscaling layout with
+ * the layer's INT4 nibble order and group-32 scale shape. */
+static double fp4_value(const int32_t *q, const uint8_t *s, int K, int r, int c)
+{
+    uint32_t word = (uint32_t)q[(size_t)r * (K / 8) + c / 8];
+    unsigned code = (word >> (4 * (c % 8))) & 15u;
+    return e2m1_value(code) * ldexp(1.0, (int)s[(size_t)r * (K / 32) + c / 32] - 127);
+}
+
+/* fmt 0: INT4 (bf16 scales), fmt 1: MXFP4 (UE8M0 scales) */
+static double q4_value(int fmt, const int32_t *q, const void *s, int K, int r, int c)
+{
+    return fmt ? fp4_value(q, (const uint8_t *)s, K, r, c) : w4_value(q, (const uint16_t *)s, K, r, c);
+}
+
 /* ------------------------------------------------------------------------------------------ */
 /* FP8 per-token group-128 activation quantization ([SGL], "Background": As is the per
  * token-group quantization scale matrix of the activations; block_size [128, 128]).           */
@@ -252,10 +279,11 @@ static double silu(double g) { return g / (1.0 + exp(-g)); }
  *     y_m = sum_n h_n * W2[e][m, n]
  *   out = sum over the k selected experts of w * y     (the top-k weighted combine).
  * h_out (nullable, bf16 bits [ntok, k, I]) returns the intermediate of each slot. */
-int orc_moe_w4a16(const uint16_t *x, const float *logits, int T, int H, int I, int E, int k,
-                  const int32_t *w13q, const uint16_t *w13s, const int32_t *w2q, const uint16_t *w2s,
-                  const int32_t *tokens, int ntok, double *out, uint16_t *h_out)
+static int moe_q4_layer(int fmt, const uint16_t *x, const float *logits, int T, int H, int I, int E, int k,
+                        const int32_t *w13q, const void *w13s, const int32_t *w2q, const void *w2s,
+                        const int32_t *tokens, int ntok, double *out, uint16_t *h_out)
 {
+    const size_t sb = fmt ? 1 : 2;  /* bytes per scale */
     if (H % 32 || I % 32 || H < 32 || I < 32 || k < 1 || k > E) return 1;
     for (int i = 0; i < ntok; ++i)
         if (tokens[i] < 0 || tokens[i] >= T) return 1;
@@ -273,15 +301,15 @@ int orc_moe_w4a16(const uint16_t *x, const float *logits, int T, int H, int I, i
         for (int j = 0; j < k; ++j) {
             int e = ids[j];
             const int32_t *q13 = w13q + (size_t)e * 2 * I * (H / 8);
-            const uint16_t *s13 = w13s + (size_t)e * 2 * I * (H / 32);
+            const void *s13 = (const char *)w13s + (size_t)e * 2 * I * (H / 32) * sb;
             const int32_t *q2 = w2q + (size_t)e * H * (I / 8);
-            const uint16_t *s2 = w2s + (size_t)e * H * (I / 32);
+            const void *s2 = (const char *)w2s + (size_t)e * H * (I / 32) * sb;
 #pragma omp parallel for schedule(static)
             for (int n = 0; n < I; ++n) {
                 double g = 0.0, u = 0.0;
                 for (int c = 0; c < H; ++c) {
-                    g += xd[c] * w4_value(q13, s13, H, n, c);
-                    u += xd[c] * w4_value(q13, s13, H, I + n, c);
+                    g += xd[c] * q4_value(fmt, q13, s13, H, n, c);
+                    u += xd[c] * q4_value(fmt, q13, s13, H, I + n, c);
                 }
                 uint16_t hb = bf16_round(silu(g) * u);
                 h[n] = bf16_value(hb);
@@ -291,13 +319,29 @@ int orc_moe_w4a16(const uint16_t *x, const float *logits, int T, int H, int I, i
 #pragma omp parallel for schedule(static)
             for (int m = 0; m < H; ++m) {
                 double y = 0.0;
-                for (int n = 0; n < I; ++n) y += h[n] * w4_value(q2, s2, I, m, n);
+                for (int n = 0; n < I; ++n) y += h[n] * q4_value(fmt, q2, s2, I, m, n);
                 o[m] += wj * y;
             }
         }
     }
     free(ids); free(w); free(xd); free(h);
     return 0;
+}
+
+int orc_moe_w4a16(const uint16_t *x, const float *logits, int T, int H, int I, int E, int k,
+                  const int32_t *w13q, const uint16_t *w13s, const int32_t *w2q, const uint16_t *w2s,
+                  const int32_t *tokens, int ntok, double *out, uint16_t *h_out)
+{
+    return moe_q4_layer(0, x, logits, T, H, I, E, k, w13q, w13s, w2q, w2s, tokens, ntok, out, h_out);
+}
+
+/* The same layer with MXFP4 weights (E2M1 codes, UE8M0 group-32 scales [rows, K/32] bytes); the
+ * activations stay bf16 and the intermediate is rounded to bf16 as in the W4A16 layer. */
+int orc_moe_mxfp4(const uint16_t *x, const float *logits, int T, int H, int I, int E, int k,
+                  const int32_t *w13q, const uint8_t *w13s, const int32_t *w2q, const uint8_t *w2s,
+                  const int32_t *tokens, int ntok, double *out, uint16_t *h_out)
+{
+    return moe_q4_layer(1, x, logits, T, H, I, E, k, w13q, w13s, w2q, w2s, tokens, ntok, out, h_out);
 }
 
 /* ------------------------------------------------------------------------------------------ */
@@ -501,4 +545,17 @@ int orc_w4a16_dequant(const int32_t *q, const uint16_t *s, int N, int K, double 
     for (int r = 0; r < N; ++r)
         for (int c = 0; c < K; ++c) out[(size_t)r * K + c] = w4_value(q, s, K, r, c);
     return 0;
+}
+
+int orc_mxfp4_dequant(const int32_t *q, const uint8_t *s, int N, int K, double *out)
+{
+    if (K % 32 || K < 32) return 1;
+    for (int r = 0; r < N; ++r)
+        for (int c = 0; c < K; ++c) out[(size_t)r * K + c] = fp4_value(q, s, K, r, c);
+    return 0;
+}
+
+void orc_e2m1_value(const uint8_t *in, double *out, long n)
+{
+    for (long i = 0; i < n; ++i) out[i] = e2m1_value(in[i] & 15u);
 }

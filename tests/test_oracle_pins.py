@@ -416,6 +416,96 @@ def test_fp8_channel_equals_block_when_scales_are_constant_per_block():
     assert np.allclose(C, Cb, rtol=1e-12, atol=1e-12)
 
 
+# ---- MXFP4 (E2M1 codes, UE8M0 group-32 scales) ------------------------------------------------
+
+def _e2m1_via_e4m3(codes):
+    """E2M1 code -> value through torch's E4M3 decoder: every E2M1 value is an E4M3 value with the
+    same sign, exponent + 6 (bias 1 -> 7) and the mantissa bit moved to the top of three; the
+    E2M1 subnormal 0.5 is the E4M3 normal 2^-1 (code 0x30) and 0 is 0."""
+    codes = np.asarray(codes, np.uint8) & 15
+    e, m, sg = (codes >> 1) & 3, codes & 1, codes >> 3
+    e4 = np.where(e > 0, (sg << 7) | ((e + 6) << 3) | (m << 2), np.where(m == 1, (sg << 7) | 0x30, sg << 7))
+    return torch.from_numpy(e4.astype(np.uint8)).view(torch.float8_e4m3fn).double().numpy()
+
+
+def _mxfp4_numpy_dequant(q, s):
+    """numpy unpack of int32 words (nibble j = input 8w + j) times 2^(s - 127) per 32 inputs."""
+    q = np.asarray(q).view(np.uint32)
+    N, K8 = q.shape
+    codes = ((q[:, :, None] >> (4 * np.arange(8, dtype=np.uint32))) & 15).reshape(N, K8 * 8)
+    return _e2m1_via_e4m3(codes) * np.ldexp(1.0, np.repeat(s.astype(np.int64), 32, 1) - 127)
+
+
+def test_e2m1_all_codes_match_e4m3_route():
+    c = np.arange(16, dtype=np.uint8)
+    assert np.array_equal(oracle.e2m1_value(c), _e2m1_via_e4m3(c))
+    assert list(oracle.e2m1_value(c[:8])) == [0, 0.5, 1, 1.5, 2, 3, 4, 6]
+
+
+def test_mxfp4_dequant_hand_worked_and_numpy():
+    """Row 0: input 0 code 0x1 (0.5), input 9 code 0xF (-6), input 33 code 0x3 (1.5) with group
+    scales 2^(125-127) and 2^(130-127): -> 0.125, -1.5, 12.0; everything else code 0 -> 0."""
+    q = np.zeros((2, 8), np.uint32)
+    q[0, 0] = 0x1                      # input 0, nibble 0
+    q[0, 1] = 0xF << 4                 # input 9 = word 1, nibble 1
+    q[0, 4] = 0x3 << 4                 # input 33 = word 4, nibble 1
+    s = np.array([[125, 130], [0, 254]], np.uint8)
+    deq = oracle.mxfp4_dequant(q.view(np.int32), s)
+    want = np.zeros((2, 64))
+    want[0, 0], want[0, 9], want[0, 33] = 0.125, -1.5, 12.0
+    assert np.array_equal(deq, want)
+    d = W.make_moe(W.WORKLOADS["decode_mxfp4"], T=2, E=2, k=1, H=256, I=128)
+    for e in range(2):
+        qq, ss = W.np_bits(d["w13q"][e]), W.np_bits(d["w13s"][e])
+        assert np.array_equal(oracle.mxfp4_dequant(qq, ss), _mxfp4_numpy_dequant(qq, ss))
+
+
+def test_mxfp4_layer_equals_int4_layer_on_integer_weights():
+    """Weights whose MXFP4 values are the integers -6..6 (scale 2^0) written also as INT4 codes
+    q = value + 8 with bf16 scale 1: the MXFP4 and the INT4 layer oracles agree exactly."""
+    T, E, k, H, I = 3, 3, 2, 64, 32
+    rng = np.random.default_rng(5)
+    vals = np.array([0, 1, 2, 3, 4, 6, -1, -2, -3, -4, -6])
+    code_of = {0: 0, 1: 2, 2: 4, 3: 5, 4: 6, 6: 7, -1: 10, -2: 12, -3: 13, -4: 14, -6: 15}
+
+    def pack(v, table):
+        c = np.vectorize(table.__getitem__)(v).astype(np.uint32)
+        N, K = c.shape
+        return (c.reshape(N, K // 8, 8) << (4 * np.arange(8, dtype=np.uint32))).sum(-1).astype(np.uint32).view(np.int32)
+
+    v13 = rng.choice(vals, size=(E, 2 * I, H))
+    v2 = rng.choice(vals, size=(E, H, I))
+    fp4 = lambda v: np.stack([pack(x, code_of) for x in v])
+    int4 = lambda v: np.stack([pack(x, {u: u + 8 for u in vals}) for x in v])
+    one = 0x3F80
+    x = torch.randn(T, H).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    a = oracle.moe_mxfp4(x, logits, k, fp4(v13), np.full((E, 2 * I, H // 32), 127, np.uint8), fp4(v2),
+                         np.full((E, H, I // 32), 127, np.uint8))
+    b = oracle.moe_w4a16(x, logits, k, int4(v13), np.full((E, 2 * I, H // 32), one, np.uint16), int4(v2),
+                         np.full((E, H, I // 32), one, np.uint16))
+    assert np.array_equal(a, b)
+
+
+def test_mxfp4_layer_dense_equivalence_with_uniform_routing():
+    """k = E, equal logits: out = (1/E) sum_e FFN_e(x), FFN_e from numpy float64 matmul on the
+    torch/numpy-decoded weights and a torch-rounded bf16 intermediate."""
+    T, E, H, I = 3, 4, 128, 64
+    d = W.make_moe(W.WORKLOADS["decode_mxfp4"], T=T, E=E, k=E, H=H, I=I)
+    x = W.np_bits(d["x"])
+    w13q, w13s, w2q, w2s = (W.np_bits(d[n]) for n in ("w13q", "w13s", "w2q", "w2s"))
+    logits = np.zeros((T, E), np.float32)
+    out = oracle.moe_mxfp4(x, logits, E, w13q, w13s, w2q, w2s)
+    xd = d["x"].double().numpy()
+    ref = np.zeros_like(out)
+    for e in range(E):
+        w13 = _mxfp4_numpy_dequant(w13q[e], w13s[e])
+        g, u = xd @ w13[:I].T, xd @ w13[I:].T
+        h = torch.from_numpy(g / (1 + np.exp(-g)) * u).to(torch.bfloat16).double().numpy()
+        ref += 0.25 * (h @ _mxfp4_numpy_dequant(w2q[e], w2s[e]).T)
+    assert np.allclose(out, ref, rtol=1e-9, atol=1e-12)
+
+
 def _torch_fp8_rows(v32):
     q, s = W.quantize_fp8_rows(torch.from_numpy(np.ascontiguousarray(v32)))
     return q.numpy(), s.numpy()

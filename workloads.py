@@ -36,7 +36,7 @@ SEED = 0
 @dataclass(frozen=True)
 class Workload:
     name: str
-    kind: str              # "w4a16", "fp8" (MoE layers) or "dense_fp8"
+    kind: str              # "w4a16", "mxfp4", "fp8" (MoE layers) or "dense_fp8"
     wid: int               # stream id of the workload
     T: int = 0
     H: int = 0
@@ -55,6 +55,9 @@ WORKLOADS = {
     "prefill_w4a16": Workload("prefill_w4a16", "w4a16", 2, T=8192, H=7168, I=2048, E=384, k=8, logits="zipf"),
     "dense_fp8": Workload("dense_fp8", "dense_fp8", 3, M_list=tuple(2 ** i for i in range(13)), N=24576, K=7168),
     "moe_fp8": Workload("moe_fp8", "fp8", 4, T=4096, H=7168, I=2048, E=256, k=8, logits="zipf"),
+    # the decode and prefill layers with MXFP4 weights (E2M1 codes, UE8M0 group-32 scales)
+    "decode_mxfp4": Workload("decode_mxfp4", "mxfp4", 6, T=32, H=7168, I=2048, E=384, k=8, logits="uniform"),
+    "prefill_mxfp4": Workload("prefill_mxfp4", "mxfp4", 7, T=8192, H=7168, I=2048, E=384, k=8, logits="zipf"),
     # channelwise W8A8 FP8 GEMM at the N = K = 4096 shape the SGLang config page gives as its example
     "dense_fp8_channel": Workload("dense_fp8_channel", "dense_fp8_channel", 5,
                                   M_list=(1, 16, 64, 128, 256, 1024, 4096), N=4096, K=4096),
@@ -104,6 +107,35 @@ def quantize_w4_group32(w: torch.Tensor):
     return packed.to(torch.int32).contiguous(), scale.contiguous()
 
 
+_E2M1_GRID = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)
+
+
+def quantize_mxfp4_group32(w: torch.Tensor):
+    """f32 [N, K] -> (E2M1 codes packed int32 [N, K/8] in the INT4 nibble order, UE8M0 scales
+    uint8 [N, K/32]). Per group: the smallest power of two 2^(s-127) with amax / 2^(s-127) <= 6,
+    codes rounded to nearest (ties to the even code), an all-zero group gets s = 0 and code 0."""
+    N, K = w.shape
+    wg = w.double().view(N, K // 32, 32)
+    amax = wg.abs().amax(-1)
+    e = torch.ceil(torch.log2(torch.where(amax > 0, amax, torch.ones_like(amax)) / 6.0))
+    s = torch.where(amax > 0, (e + 127).clamp(0, 254), torch.zeros_like(e))
+    a = (wg / torch.pow(2.0, s - 127)[..., None]).abs().clamp(max=6.0)
+    grid = torch.tensor(_E2M1_GRID, dtype=torch.float64, device=w.device)
+    dist = (a[..., None] - grid).abs()
+    best = dist.min(-1, keepdim=True).values
+    # among the nearest grid points (one, or two at a tie) take the even code
+    idx = torch.arange(8, device=w.device)
+    cand = (dist <= best) & True
+    code = torch.where(cand & (idx % 2 == 0), idx, torch.full_like(idx, 99)).min(-1).values
+    code = torch.where((cand & (idx % 2 == 0)).any(-1), code, cand.int().argmax(-1))
+    code = code + 8 * ((wg < 0) & (code > 0)).to(code.dtype)
+    q = code.to(torch.int64).view(N, K // 8, 8)
+    shifts = torch.arange(0, 32, 4, device=w.device, dtype=torch.int64)
+    packed = (q << shifts).sum(-1)
+    packed = packed - ((packed >> 31) & 1) * (1 << 32)
+    return packed.to(torch.int32).contiguous(), s.to(torch.uint8).contiguous()
+
+
 def quantize_fp8_blocks(w: torch.Tensor, bn: int = 128, bk: int = 128):
     """f32 [N, K] -> (E4M3 codes uint8 [N, K], f32 scales [N/bn, K/bk])."""
     N, K = w.shape
@@ -133,16 +165,18 @@ def make_moe(wl: Workload, device="cpu", T=None, E=None, k=None, H=None, I=None)
     x = bf16_normal((T, H), generator(wl.wid, _X, device=device), device)
     logits = router_logits(wl, T, E, device)
     d = dict(x=x, logits=logits, T=T, H=H, I=I, E=E, k=k, kind=wl.kind)
-    if wl.kind == "w4a16":
+    if wl.kind in ("w4a16", "mxfp4"):
+        quant = quantize_w4_group32 if wl.kind == "w4a16" else quantize_mxfp4_group32
+        sdt = torch.bfloat16 if wl.kind == "w4a16" else torch.uint8
         w13q = torch.empty((E, 2 * I, H // 8), dtype=torch.int32, device=device)
-        w13s = torch.empty((E, 2 * I, H // 32), dtype=torch.bfloat16, device=device)
+        w13s = torch.empty((E, 2 * I, H // 32), dtype=sdt, device=device)
         w2q = torch.empty((E, H, I // 8), dtype=torch.int32, device=device)
-        w2s = torch.empty((E, H, I // 32), dtype=torch.bfloat16, device=device)
+        w2s = torch.empty((E, H, I // 32), dtype=sdt, device=device)
         for e in range(E):
             g = generator(wl.wid, _W13, e, device=device)
-            w13q[e], w13s[e] = quantize_w4_group32(torch.randn((2 * I, H), generator=g, device=device) * 0.02)
+            w13q[e], w13s[e] = quant(torch.randn((2 * I, H), generator=g, device=device) * 0.02)
             g = generator(wl.wid, _W2, e, device=device)
-            w2q[e], w2s[e] = quantize_w4_group32(torch.randn((H, I), generator=g, device=device) * 0.02)
+            w2q[e], w2s[e] = quant(torch.randn((H, I), generator=g, device=device) * 0.02)
         d.update(w13q=w13q, w13s=w13s, w2q=w2q, w2s=w2s)
     elif wl.kind == "fp8":
         w13 = torch.empty((E, 2 * I, H), dtype=torch.uint8, device=device)
