@@ -308,6 +308,20 @@ def run_w4a16(moeq, d, steps, warmup, flush, world, trace=False):
     return ms, stages, out
 
 
+def run_mxfp4(moeq, d, steps, warmup, flush, world):
+    """The MXFP4 layer: scale factors prepacked once (outside the timed steps), then forwards."""
+    out = torch.empty((d["T"], d["H"]), dtype=torch.bfloat16, device="cuda")
+    ws = moeq.workspace(moeq.lib().moe_mxfp4_workspace_size(d["T"], d["H"], d["I"], d["E"], d["k"]), "cuda")
+    if "w13f" not in d:
+        d["w13f"] = moeq.moe_mxfp4_prepack_scales(d["w13s"])
+        d["w2f"] = moeq.moe_mxfp4_prepack_scales(d["w2s"])
+
+    def step():
+        moeq.moe_mxfp4_forward(d["x"], d["logits"], d["k"], d["w13q"], d["w13f"], d["w2q"], d["w2f"], out=out, ws=ws)
+
+    return timed_steps(step, steps, warmup, flush, world)
+
+
 def run_fp8(moeq, d, steps, warmup, flush, world):
     out = torch.empty((d["T"], d["H"]), dtype=torch.bfloat16, device="cuda")
     ws = moeq.workspace(moeq.moe_w8a8_block_fp8_workspace_size(d["T"], d["H"], d["I"], d["E"], d["k"]), "cuda")
@@ -557,6 +571,32 @@ def main():
             "weight_gbs": pbytes / (pstep * 1e-3) / 1e9, "active_experts": int((prows > 0).sum()),
             "skew_aware_roof_ms": proof, "frac_of_skew_aware_roof": proof / pstep,
             "stages_ms": {k: v[0] / max(v[1], 1) for k, v in pst.items() if v[1]}}
+        # MXFP4 weights (E2M1 codes, UE8M0 group-32 scales) on the same layer: decode (T = 32,
+        # uniform routing) and prefill (T = 8192, Zipf routing) over one set of 384 experts
+        dm = W.make_moe(W.WORKLOADS["decode_mxfp4"], device="cuda")
+        mms = run_mxfp4(moeq, dm, max(3, args.steps // 2), 3, flush, world)
+        mstep = max_over_ranks(statistics.mean(mms), world)
+        mact = touched_experts(moeq, dm)
+        # bytes the hot path reads: E2M1 codes + the prepacked bf16 group factors (as the INT4
+        # format; the stored UE8M0 scales are 1 byte per group, 17/18 of this)
+        mbytes = mact * W.w4a16_expert_bytes(dm["H"], dm["I"])
+        also["decode_mxfp4"] = {
+            "workload": "T=32 H=7168 I=2048 E=384 k=8, MXFP4 weights, bf16 activations", "ms_per_step": mstep,
+            "weight_gbs": mbytes / (mstep * 1e-3) / 1e9,
+            "hbm_frac": mbytes / (mstep * 1e-3) / 1e9 / peaks["hbm_gbs"], "touched_experts": mact,
+            "weight_bytes_per_step": mbytes}
+        wlp = W.WORKLOADS["prefill_mxfp4"]
+        dpm = dict(dm)
+        dpm.update(T=wlp.T, x=W.bf16_normal((wlp.T, dm["H"]), W.generator(wlp.wid, 0, device="cuda"), "cuda"),
+                   logits=W.router_logits(wlp, wlp.T, dm["E"], "cuda"))
+        qms = run_mxfp4(moeq, dpm, max(3, args.steps // 4), 3, None, world)
+        qstep = max_over_ranks(statistics.mean(qms), world)
+        also["prefill_mxfp4"] = {
+            "workload": "T=8192 H=7168 I=2048 E=384 k=8, Zipf-biased routing, MXFP4 weights", "ms_per_step": qstep,
+            "tflops": pflops / (qstep * 1e-3) / 1e12,
+            "frac_of_bf16_peak": pflops / (qstep * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"]}
+        del dm, dpm
+        torch.cuda.empty_cache()
         # grouped W4A16 GEMM, contiguous layout: the prefill routing's rows per expert, each
         # expert padded to 128 rows (m_indices -1), its W13 (N = 2I = 4096, K = H = 7168)
         pad = [int(c) + (-int(c)) % 128 for c in prows]

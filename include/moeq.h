@@ -122,6 +122,27 @@ MOEQ_API int moe_w4a16_forward(const uint16_t *x, const float *logits, int T, in
                       float *topk_w_out, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * The same routed layer with MXFP4 weights (lk_moe page, "Supported models & quant formats": MXFP4;
+ * its launch example runs a 4-bit-weight, bf16-activation checkpoint on the weight-only MoE
+ * runner). A weight is E2M1(q) * 2^(s - 127): q an E2M1 code (1 sign, 2 exponent bits with bias 1,
+ * 1 mantissa bit; magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6) packed 8 per int32 in the INT4 nibble
+ * order above, s the UE8M0 scale byte of its 32-input group. Activations and the intermediate
+ * stay bf16 as in moe_w4a16_forward.
+ *   moe_mxfp4_prepack_scales: the n UE8M0 bytes -> n bf16 group factors 2^(s - 1), the form the
+ *     kernels multiply by (run once per weight tensor; codes s <= 128, i.e. group scales up to 2,
+ *     are exact; larger codes give +inf factors). Device memory, asynchronous on the stream.
+ *   moe_mxfp4_forward: w13_q i32 [E, 2I, H/8], w13_f bf16 [E, 2I, H/32] (prepacked factors),
+ *     w2_q i32 [E, H, I/8], w2_f bf16 [E, H, I/32]; everything else, the workspace
+ *     (moe_mxfp4_workspace_size, equal to the W4A16 one), limits and errors as moe_w4a16_forward.
+ */
+MOEQ_API int moe_mxfp4_prepack_scales(const uint8_t *ue8m0, long long n, uint16_t *factors, void *stream);
+MOEQ_API size_t moe_mxfp4_workspace_size(int T, int H, int I, int E, int k);
+MOEQ_API int moe_mxfp4_forward(const uint16_t *x, const float *logits, int T, int H, int I, int E, int k,
+                               const int32_t *w13_q, const uint16_t *w13_f, const int32_t *w2_q, const uint16_t *w2_f,
+                               uint16_t *out, int32_t *topk_ids_out, float *topk_w_out, void *ws, size_t ws_bytes,
+                               void *stream);
+
+/*
  * Scratch-free W4A16 layer forward. The pages have no counterpart of this entry point: it exists
  * for callers that cannot allocate device memory where they run the layer, such as a plugin or
  * custom-op host that only hands over its input and output buffers, or a serving runtime that

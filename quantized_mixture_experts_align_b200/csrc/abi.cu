@@ -329,10 +329,16 @@ size_t moe_w4a16_workspace_size(int T, int H, int I, int E, int k)
     return w4a16_layout(c, T, H, I, E, k, nullptr, nullptr, nullptr);
 }
 
-int moe_w4a16_forward(const uint16_t *x, const float *logits, int T, int H, int I, int E, int k,
-                      const int32_t *w13_q, const uint16_t *w13_s, const int32_t *w2_q, const uint16_t *w2_s,
-                      uint16_t *out, int32_t *topk_ids_out, float *topk_w_out, void *ws, size_t ws_bytes,
-                      void *stream)
+}  // extern "C"
+
+namespace moeq {
+// The 4-bit weight layer (fmt W4_INT4: codes - 8 times bf16 group scales; W4_FP4: E2M1 codes
+// times the bf16 group factors 2^(s - 1) of moe_mxfp4_prepack_scales): one schedule, the format
+// only changes the kernels' dequantization.
+static int w4_layer_forward(int fmt, const char *name, const uint16_t *x, const float *logits, int T, int H, int I,
+                            int E, int k, const int32_t *w13_q, const uint16_t *w13_s, const int32_t *w2_q,
+                            const uint16_t *w2_s, uint16_t *out, int32_t *topk_ids_out, float *topk_w_out, void *ws,
+                            size_t ws_bytes, void *stream)
 {
     g_err[0] = 0;
     int rc = check_layer_shape(T, H, I, E, k);
@@ -372,13 +378,14 @@ int moe_w4a16_forward(const uint16_t *x, const float *logits, int T, int H, int 
 
     if (tcp) {
         int *status = device_status_ptr();
-        if (!status) return set_error(MOEQ_ERR_CUDA, "moe_w4a16_forward: no device status word");
+        if (!status) return set_error(MOEQ_ERR_CUDA, "%s: no device status word", name);
         const int cap = r.max_blocks * r.block_m;
         {
             trace::Scope ts(trace::ACT_QUANT, s);  // the activation gather takes the act-prep slot
             launch_gather_bf16_perm(x, H, k, r.sorted, r.ntp, n, cap, kW4SmallRows, xg, num_sms(), s);
         }
         W4TcArgs t{};
+        t.fmt = fmt;
         t.status = status;
         t.E = E;
         t.sorted_ids = r.sorted;
@@ -396,6 +403,7 @@ int moe_w4a16_forward(const uint16_t *x, const float *logits, int T, int H, int 
         t.small_rows = kW4SmallRows;
         // the small blocks: register-fed kernel over the same 256-row alignment, h in slot order
         W4GroupedArgs g{};
+        g.fmt = fmt;
         g.E = E;
         g.sorted_ids = r.sorted;
         g.expert_ids = r.eids;
@@ -440,6 +448,7 @@ int moe_w4a16_forward(const uint16_t *x, const float *logits, int T, int H, int 
         if (rc) return rc;
     } else {
         W4GroupedArgs a{};
+        a.fmt = fmt;
         a.E = E;
         a.sorted_ids = r.sorted;
         a.expert_ids = r.eids;
@@ -477,7 +486,41 @@ int moe_w4a16_forward(const uint16_t *x, const float *logits, int T, int H, int 
         trace::Scope ts(trace::COMBINE, s);
         launch_combine(ys, T, k, H, out, num_sms(), s);
     }
-    return check_launch("moe_w4a16_forward");
+    return check_launch(name);
+}
+}  // namespace moeq
+
+extern "C" {
+
+int moe_w4a16_forward(const uint16_t *x, const float *logits, int T, int H, int I, int E, int k,
+                      const int32_t *w13_q, const uint16_t *w13_s, const int32_t *w2_q, const uint16_t *w2_s,
+                      uint16_t *out, int32_t *topk_ids_out, float *topk_w_out, void *ws, size_t ws_bytes,
+                      void *stream)
+{
+    return w4_layer_forward(W4_INT4, "moe_w4a16_forward", x, logits, T, H, I, E, k, w13_q, w13_s, w2_q, w2_s, out,
+                            topk_ids_out, topk_w_out, ws, ws_bytes, stream);
+}
+
+size_t moe_mxfp4_workspace_size(int T, int H, int I, int E, int k) { return moe_w4a16_workspace_size(T, H, I, E, k); }
+
+int moe_mxfp4_forward(const uint16_t *x, const float *logits, int T, int H, int I, int E, int k,
+                      const int32_t *w13_q, const uint16_t *w13_f, const int32_t *w2_q, const uint16_t *w2_f,
+                      uint16_t *out, int32_t *topk_ids_out, float *topk_w_out, void *ws, size_t ws_bytes,
+                      void *stream)
+{
+    return w4_layer_forward(W4_FP4, "moe_mxfp4_forward", x, logits, T, H, I, E, k, w13_q, w13_f, w2_q, w2_f, out,
+                            topk_ids_out, topk_w_out, ws, ws_bytes, stream);
+}
+
+int moe_mxfp4_prepack_scales(const uint8_t *ue8m0, long long n, uint16_t *factors, void *stream)
+{
+    g_err[0] = 0;
+    if (n < 0) return set_error(MOEQ_ERR_INVALID_ARG, "n must be >= 0 (got %lld)", n);
+    if (n == 0) return MOEQ_OK;
+    MOEQ_REQUIRE(ue8m0);
+    MOEQ_REQUIRE(factors);
+    launch_mxfp4_scale_factors(ue8m0, n, factors, num_sms(), (cudaStream_t)stream);
+    return check_launch("moe_mxfp4_prepack_scales");
 }
 
 // ------------------------------------------------------------------------------------------

@@ -61,6 +61,18 @@ __device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint3
     return r;
 }
 
+// E2M1 codes of nibbles P and P + 4 of a code word as bf16x2 holding 2^-126 times their values:
+// the sign goes to bit 15 (31) and the 2 exponent + 1 mantissa bits to bits [8:6] ([24:22]), so the
+// E2M1 exponent lands in the low bits of the bf16 exponent field and its subnormal (exponent 0,
+// value 0.5) on the bf16 subnormal 2^-127. One bf16 multiply by a group factor 2^(s - 1) then
+// gives value * 2^(s - 127) exactly.
+template <int P>
+__device__ __forceinline__ uint32_t e2m1_pair_pre(uint32_t w)
+{
+    const uint32_t mag = (P < 2 ? (w << (6 - 4 * P)) : (w >> (4 * P - 6))) & 0x01C001C0u;
+    return lop3_and_or(w << (12 - 4 * P), 0x80008000u, mag);
+}
+
 __device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b)
 {
     uint32_t r;

@@ -68,9 +68,18 @@ static_assert(kAccCols + kStages * kAStageCols <= kTmemCols, "tensor memory budg
 static_assert(kBStages == kStages, "one stage-free barrier serves the activation and weight stages");
 static_assert(64 * kTok * 4 <= kBStages * kBTile, "gate/up exchange fits in the activation ring");
 
-// (q - 8) * scale in bf16 for the pairs (q0,q4) (q1,q5) (q2,q6) (q3,q7) of one code word
+// (q - 8) * scale (INT4) or E2M1(q) * 2^(s - 1) (FP4, see e2m1_pair_pre) in bf16 for the pairs
+// (q0,q4) (q1,q5) (q2,q6) (q3,q7) of one code word
+template <int FMT>
 __device__ __forceinline__ void dequant4(uint32_t w, uint32_t scale2, uint32_t *out)
 {
+    if (FMT == W4_FP4) {
+        out[0] = bf16x2_mul(e2m1_pair_pre<0>(w), scale2);
+        out[1] = bf16x2_mul(e2m1_pair_pre<1>(w), scale2);
+        out[2] = bf16x2_mul(e2m1_pair_pre<2>(w), scale2);
+        out[3] = bf16x2_mul(e2m1_pair_pre<3>(w), scale2);
+        return;
+    }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const uint32_t v = lop3_and_or(w >> (4 * i), 0x000F000Fu, 0x43004300u);  // 128 + q, exact
@@ -85,7 +94,7 @@ __device__ __forceinline__ int perm_pos(int f)
     return (f & ~7) + (i < 4 ? 2 * i : 2 * (i - 4) + 1);
 }
 
-template <int MODE>
+template <int MODE, int FMT>
 __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_constant__ CUtensorMap tmX, W4TcArgs a)
 {
     constexpr bool GU = MODE == TC_GATEUP;
@@ -223,10 +232,10 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
             issue(ks + kRing - 1);  // refills the slot read in step ks - 1
             const uint32_t s2 = prmt(sc, sc, (kq & 1) ? 0x3232u : 0x1010u);  // this slice's group, twice
             uint32_t pairs[16];
-            dequant4(c.x, s2, pairs + 0);
-            dequant4(c.y, s2, pairs + 4);
-            dequant4(c.z, s2, pairs + 8);
-            dequant4(c.w, s2, pairs + 12);
+            dequant4<FMT>(c.x, s2, pairs + 0);
+            dequant4<FMT>(c.y, s2, pairs + 4);
+            dequant4<FMT>(c.z, s2, pairs + 8);
+            dequant4<FMT>(c.w, s2, pairs + 12);
             if (pending >= 0) {
                 ok = stage_ready(pending);
                 pending = -1;
@@ -340,19 +349,19 @@ __global__ void __launch_bounds__(256) gather_bf16_perm_kernel(const uint16_t *_
     }
 }
 
-template <int MODE>
+template <int MODE, int FMT>
 int launch_mode(const W4TcArgs &a, const CUtensorMap &tm, int grid_x, int grid_y, cudaStream_t s)
 {
     static bool attr = false;
     if (!attr) {
         const cudaError_t e =
-            cudaFuncSetAttribute(w4a16_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+            cudaFuncSetAttribute(w4a16_tc_kernel<MODE, FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
         if (e != cudaSuccess)
             return set_error(MOEQ_ERR_CUDA, "tcgen05 W4A16 GEMM: shared-memory attribute: %s", cudaGetErrorString(e));
         attr = true;
     }
     if (grid_x <= 0 || grid_y <= 0) return MOEQ_OK;
-    w4a16_tc_kernel<MODE><<<dim3(grid_x, grid_y), kThreads, kSmemBytes, s>>>(tm, a);
+    w4a16_tc_kernel<MODE, FMT><<<dim3(grid_x, grid_y), kThreads, kSmemBytes, s>>>(tm, a);
     return MOEQ_OK;
 }
 
@@ -363,8 +372,12 @@ int launch_w4a16_tc(const W4TcArgs &a, int mode, const uint16_t *act, int max_bl
     CUtensorMap tm;
     const int rc = make_tmap_2d(&tm, act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.M, (uint64_t)a.K, kTok, kKs / 2);
     if (rc) return rc;
-    if (mode == TC_GATEUP) return launch_mode<TC_GATEUP>(a, tm, a.N / 64, max_blocks, s);
-    return launch_mode<TC_DOWN>(a, tm, a.N / 128, max_blocks, s);
+    if (a.fmt == W4_FP4) {
+        if (mode == TC_GATEUP) return launch_mode<TC_GATEUP, W4_FP4>(a, tm, a.N / 64, max_blocks, s);
+        return launch_mode<TC_DOWN, W4_FP4>(a, tm, a.N / 128, max_blocks, s);
+    }
+    if (mode == TC_GATEUP) return launch_mode<TC_GATEUP, W4_INT4>(a, tm, a.N / 64, max_blocks, s);
+    return launch_mode<TC_DOWN, W4_INT4>(a, tm, a.N / 128, max_blocks, s);
 }
 
 void launch_gather_bf16_perm(const uint16_t *x, int H, int k, const int32_t *sorted_ids, const int32_t *ntp,

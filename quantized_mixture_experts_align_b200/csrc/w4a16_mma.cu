@@ -31,11 +31,20 @@ struct DeqWord {
     uint32_t p[4];  // bf16x2 pairs: (n0,n4) (n1,n5) (n2,n6) (n3,n7), already (q-8)*scale
 };
 
+template <int FMT>
 __device__ __forceinline__ DeqWord dequant_word(uint32_t w, uint32_t scale2)
 {
+    DeqWord d;
+    if (FMT == W4_FP4) {
+        // E2M1 code times the group factor 2^(s - 1) (see e2m1_pair_pre)
+        d.p[0] = bf16x2_mul(e2m1_pair_pre<0>(w), scale2);
+        d.p[1] = bf16x2_mul(e2m1_pair_pre<1>(w), scale2);
+        d.p[2] = bf16x2_mul(e2m1_pair_pre<2>(w), scale2);
+        d.p[3] = bf16x2_mul(e2m1_pair_pre<3>(w), scale2);
+        return d;
+    }
     const uint32_t magic = 0x43004300u;  // bf16 128.0 in both halves
     const uint32_t bias = 0x43084308u;   // bf16 136.0 = 128 + 8 (zero point) in both halves
-    DeqWord d;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const uint32_t v = lop3_and_or(w >> (4 * i), 0x000F000Fu, magic);  // 128 + q, exact
@@ -67,7 +76,7 @@ constexpr int kW4StageBytes = 4 * 32 * 16 + 4 * 8 * 8;  // 2048 B codes + 256 B 
 //              h[slot, f] = bf16(silu(gate) * up).
 // MODE_DOWN:   rows [r0, r0+32) of W2; epilogue writes ys[slot, r] = bf16(topk_w[slot] * y) (weight 1
 //              without routing weights: the plain grouped GEMM).
-template <int BM, int WARPS, int MODE, bool STRIDED>
+template <int BM, int WARPS, int MODE, bool STRIDED, int FMT>
 __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4GroupedArgs a)
 {
     constexpr int MS = BM / 8;  // token sub-tiles of 8 columns
@@ -178,7 +187,7 @@ __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4Grouped
             const uint32_t words[4] = {(&wcur[0].x)[m], (&wcur[1].x)[m], (&wcur[2].x)[m], (&wcur[3].x)[m]};
             DeqWord d[4];
 #pragma unroll
-            for (int r = 0; r < 4; ++r) d[r] = dequant_word(words[r], sc[r]);
+            for (int r = 0; r < 4; ++r) d[r] = dequant_word<FMT>(words[r], sc[r]);
 #pragma unroll
             for (int s = 0; s < MS; ++s) {
                 uint4 xv;
@@ -225,19 +234,35 @@ __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4Grouped
     }
 }
 
-template <int BM, int WARPS, int MODE, bool STRIDED>
-static void launch_bm(const W4GroupedArgs &a, int max_blocks, cudaStream_t s)
+template <int BM, int WARPS, int MODE, bool STRIDED, int FMT>
+static void launch_bm_fmt(const W4GroupedArgs &a, int max_blocks, cudaStream_t s)
 {
     const int rows_per_cta = (MODE == MODE_GATEUP ? 16 : 32) * WARPS;
     const size_t smem = (size_t)WARPS * kW4Stages * kW4StageBytes;
     static bool attr_set = false;  // per template instance; the attribute is per function
     if (!attr_set) {
-        cudaFuncSetAttribute(w4a16_grouped_mma_kernel<BM, WARPS, MODE, STRIDED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
+        cudaFuncSetAttribute(w4a16_grouped_mma_kernel<BM, WARPS, MODE, STRIDED, FMT>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         attr_set = true;
     }
     dim3 grid(max_blocks, cdiv(a.n_out, rows_per_cta));
-    w4a16_grouped_mma_kernel<BM, WARPS, MODE, STRIDED><<<grid, WARPS * 32, smem, s>>>(a);
+    w4a16_grouped_mma_kernel<BM, WARPS, MODE, STRIDED, FMT><<<grid, WARPS * 32, smem, s>>>(a);
+}
+
+template <int BM, int WARPS, int MODE, bool STRIDED>
+static void launch_bm(const W4GroupedArgs &a, int max_blocks, cudaStream_t s)
+{
+    if (a.fmt == W4_FP4) launch_bm_fmt<BM, WARPS, MODE, STRIDED, W4_FP4>(a, max_blocks, s);
+    else launch_bm_fmt<BM, WARPS, MODE, STRIDED, W4_INT4>(a, max_blocks, s);
+}
+
+// UE8M0 -> bf16 2^(s - 1): exponent field s + 126 (s <= 128); larger codes give +inf
+__global__ void mxfp4_scale_factor_kernel(const uint8_t *__restrict__ sc, long long n, uint16_t *__restrict__ f)
+{
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+        const uint32_t e = sc[i];
+        f[i] = e <= 128u ? (uint16_t)((e + 126u) << 7) : (uint16_t)0x7F80u;
+    }
 }
 
 void launch_w4a16_grouped_mma(const W4GroupedArgs &a, int mode, int block_m, int max_blocks, cudaStream_t s)
@@ -262,6 +287,13 @@ void launch_w4a16_grouped_mma(const W4GroupedArgs &a, int mode, int block_m, int
         default: break;
     }
 #undef MOEQ_W4_CASE
+}
+
+void launch_mxfp4_scale_factors(const uint8_t *s, long long n, uint16_t *f, int num_sms, cudaStream_t st)
+{
+    const long long want = (n + 255) / 256;
+    const int blocks = (int)(want < 8LL * num_sms ? want : 8LL * num_sms);
+    mxfp4_scale_factor_kernel<<<blocks, 256, 0, st>>>(s, n, f);
 }
 
 }  // namespace moeq

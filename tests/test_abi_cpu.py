@@ -86,6 +86,16 @@ def test_validation_rejects_before_device_work(L):
     assert _rc(L, "w8a8_block_fp8_matmul", N, N, N, N, 4, 256, 256, 64, 128, N, N) == moeq.MOEQ_ERR_UNSUPPORTED
     assert _rc(L, "w8a8_block_fp8_matmul", N, N, N, N, 4, 256, 200, 128, 128, N, N) == moeq.MOEQ_ERR_UNSUPPORTED
     assert _rc(L, "w8a8_block_fp8_matmul", N, N, N, N, 4, 200, 256, 128, 128, N, N) == moeq.MOEQ_ERR_UNSUPPORTED
+    # MXFP4 layer: the W4A16 validation; prepack: NULL / negative n
+    mx = (p, p, 32, 7168, 2048, 384, 8, p, p, p, p, p, N, N, p, 10, N)
+    assert _rc(L, "moe_mxfp4_forward", *mx) == moeq.MOEQ_ERR_WORKSPACE
+    assert _rc(L, "moe_mxfp4_forward", p, p, 32, 100, 2048, 384, 8, p, p, p, p, p, N, N, p, 1 << 40, N) == \
+        moeq.MOEQ_ERR_UNSUPPORTED
+    assert moeq.lib().moe_mxfp4_workspace_size(32, 7168, 2048, 384, 8) == \
+        moeq.lib().moe_w4a16_workspace_size(32, 7168, 2048, 384, 8) > 0
+    assert _rc(L, "moe_mxfp4_prepack_scales", N, 16, p, N) == moeq.MOEQ_ERR_INVALID_ARG
+    assert _rc(L, "moe_mxfp4_prepack_scales", p, -1, p, N) == moeq.MOEQ_ERR_INVALID_ARG
+    assert _rc(L, "moe_mxfp4_prepack_scales", N, 0, N, N) == moeq.MOEQ_OK
     # channelwise dense matmul: K, N multiples of 128; aligned A, B, C; NULL scales
     cw = lambda A_, As_, C_, M, Nn, K: _rc(L, "w8a8_channel_fp8_matmul", A_, As_, p, p, M, Nn, K, C_, N)
     assert cw(p, p, p, 4, 256, 200) == moeq.MOEQ_ERR_UNSUPPORTED

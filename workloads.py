@@ -107,27 +107,31 @@ def quantize_w4_group32(w: torch.Tensor):
     return packed.to(torch.int32).contiguous(), scale.contiguous()
 
 
-_E2M1_GRID = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)
+# midpoints between consecutive E2M1 magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6; a value on a midpoint
+# goes to the even code (the lower one for midpoints 0, 2, 4, 6, the upper one for 1, 3, 5)
+_E2M1_MIDS = (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0)
 
 
 def quantize_mxfp4_group32(w: torch.Tensor):
     """f32 [N, K] -> (E2M1 codes packed int32 [N, K/8] in the INT4 nibble order, UE8M0 scales
     uint8 [N, K/32]). Per group: the smallest power of two 2^(s-127) with amax / 2^(s-127) <= 6,
-    codes rounded to nearest (ties to the even code), an all-zero group gets s = 0 and code 0."""
+    codes rounded to nearest (ties to the even code); an all-zero group gets s = 0 and code 0."""
     N, K = w.shape
-    wg = w.double().view(N, K // 32, 32)
+    wg = w.float().view(N, K // 32, 32)
     amax = wg.abs().amax(-1)
-    e = torch.ceil(torch.log2(torch.where(amax > 0, amax, torch.ones_like(amax)) / 6.0))
-    s = torch.where(amax > 0, (e + 127).clamp(0, 254), torch.zeros_like(e))
+    pos = amax > 0
+    e = torch.ceil(torch.log2(torch.where(pos, amax, torch.ones_like(amax)) / 6.0))
+    # exact power-of-two boundary: keep the smallest exponent whose scaled amax is <= 6
+    e = torch.where(amax / torch.pow(2.0, e) > 6.0, e + 1, e)
+    e = torch.where(amax / torch.pow(2.0, e - 1) <= 6.0, e - 1, e)
+    s = torch.where(pos, (e + 127).clamp(0, 254), torch.zeros_like(e))
     a = (wg / torch.pow(2.0, s - 127)[..., None]).abs().clamp(max=6.0)
-    grid = torch.tensor(_E2M1_GRID, dtype=torch.float64, device=w.device)
-    dist = (a[..., None] - grid).abs()
-    best = dist.min(-1, keepdim=True).values
-    # among the nearest grid points (one, or two at a tie) take the even code
-    idx = torch.arange(8, device=w.device)
-    cand = (dist <= best) & True
-    code = torch.where(cand & (idx % 2 == 0), idx, torch.full_like(idx, 99)).min(-1).values
-    code = torch.where((cand & (idx % 2 == 0)).any(-1), code, cand.int().argmax(-1))
+    mids = torch.tensor(_E2M1_MIDS, dtype=torch.float32, device=w.device)
+    code = torch.bucketize(a, mids)                     # a <= mid -> lower code
+    on_mid = torch.zeros_like(a, dtype=torch.bool)
+    lower = code.clamp(max=6)
+    on_mid = (a == mids[lower]) & (lower % 2 == 1)      # ties at odd midpoints go up
+    code = code + on_mid.to(code.dtype)
     code = code + 8 * ((wg < 0) & (code > 0)).to(code.dtype)
     q = code.to(torch.int64).view(N, K // 8, 8)
     shifts = torch.arange(0, 32, 4, device=w.device, dtype=torch.int64)
