@@ -120,6 +120,28 @@ def moe_mxfp4(x, logits, k, w13q, w13s, w2q, w2s, tokens=None, want_h=False):
     return (out, h) if want_h else out
 
 
+def moe_nvfp4(x, logits, k, w13q, w13s, g13, w2q, w2s, g2, tokens=None, want_h=False):
+    """As moe_w4a16 with NVFP4 weights: E2M1 codes int32 [E, rows, K/8], E4M3 group-16 scales
+    uint8 [E, rows, K/16] and f32 tensor scales g13 [E] (gate/up) and g2 [E] (down)."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    logits = np.ascontiguousarray(logits, dtype=np.float32)
+    T, H = x.shape
+    E = logits.shape[1]
+    I = w2q.shape[2] * 8
+    tok = _tokens(tokens, T)
+    out = np.zeros((len(tok), H), np.float64)
+    h = np.zeros((len(tok), k, I), np.uint16) if want_h else None
+    q13, s13, q2, s2 = (np.ascontiguousarray(a) for a in (w13q, w13s, w2q, w2s))
+    assert q13.dtype == np.int32 and s13.dtype == np.uint8 and s2.dtype == np.uint8
+    assert s13.shape[-1] * 16 == H and s2.shape[-1] * 16 == I
+    g13 = np.ascontiguousarray(g13, dtype=np.float32).reshape(E)
+    g2 = np.ascontiguousarray(g2, dtype=np.float32).reshape(E)
+    rc = lib().orc_moe_nvfp4(_p(x), _p(logits), T, H, I, E, k, _p(q13), _p(s13), _p(g13), _p(q2), _p(s2), _p(g2),
+                             _p(tok), len(tok), _p(out), _p(h) if h is not None else None)
+    _check(rc, "moe_nvfp4")
+    return (out, h) if want_h else out
+
+
 def moe_fp8(x, logits, k, w13, w13s, w2, w2s, tokens=None, want_h=False):
     """W8A8 block-FP8 layer output (float64 [len(tokens), H]); optionally the quantized
     intermediate (uint8 [len(tokens), k, I], f32 [len(tokens), k, I/128])."""
@@ -234,6 +256,15 @@ def mxfp4_dequant(q: np.ndarray, s: np.ndarray) -> np.ndarray:
     N, K8 = q.shape
     out = np.zeros((N, K8 * 8), np.float64)
     _check(lib().orc_mxfp4_dequant(_p(q), _p(s), N, K8 * 8, _p(out)), "mxfp4_dequant")
+    return out
+
+
+def nvfp4_dequant(q: np.ndarray, s: np.ndarray, g: float) -> np.ndarray:
+    q = np.ascontiguousarray(q, dtype=np.int32)
+    s = np.ascontiguousarray(s, dtype=np.uint8)
+    N, K8 = q.shape
+    out = np.zeros((N, K8 * 8), np.float64)
+    _check(lib().orc_nvfp4_dequant(_p(q), _p(s), ctypes.c_float(g), N, K8 * 8, _p(out)), "nvfp4_dequant")
     return out
 
 

@@ -222,9 +222,22 @@ static double fp4_value(const int32_t *q, const uint8_t *s, int K, int r, int c)
     return e2m1_value(code) * ldexp(1.0, (int)s[(size_t)r * (K / 32) + c / 32] - 127);
 }
 
-/* fmt 0: INT4 (bf16 scales), fmt 1: MXFP4 (UE8M0 scales) */
+/* NVFP4 weight element without its tensor scale (lk_moe page, "Supported models & quant
+ * formats": NVFP4, compressed-tensors / modelopt): E2M1 code (INT4 nibble order) times the E4M3
+ * scale of its 16-input group, scales [rows, K/16] bytes. The per-tensor f32 scale multiplies the
+ * whole product and is applied by the caller. READING: the pages name the format only; this is
+ * the two-level NVFP4 layout (16-element E4M3 blocks, one f32 scale per weight tensor). */
+static double nvfp4_value(const int32_t *q, const uint8_t *s, int K, int r, int c)
+{
+    uint32_t word = (uint32_t)q[(size_t)r * (K / 8) + c / 8];
+    unsigned code = (word >> (4 * (c % 8))) & 15u;
+    return e2m1_value(code) * e4m3_value(s[(size_t)r * (K / 16) + c / 16]);
+}
+
+/* fmt 0: INT4 (bf16 scales per 32), 1: MXFP4 (UE8M0 scales per 32), 2: NVFP4 (E4M3 per 16) */
 static double q4_value(int fmt, const int32_t *q, const void *s, int K, int r, int c)
 {
+    if (fmt == 2) return nvfp4_value(q, (const uint8_t *)s, K, r, c);
     return fmt ? fp4_value(q, (const uint8_t *)s, K, r, c) : w4_value(q, (const uint16_t *)s, K, r, c);
 }
 
@@ -281,9 +294,11 @@ static double silu(double g) { return g / (1.0 + exp(-g)); }
  * h_out (nullable, bf16 bits [ntok, k, I]) returns the intermediate of each slot. */
 static int moe_q4_layer(int fmt, const uint16_t *x, const float *logits, int T, int H, int I, int E, int k,
                         const int32_t *w13q, const void *w13s, const int32_t *w2q, const void *w2s,
-                        const int32_t *tokens, int ntok, double *out, uint16_t *h_out)
+                        const float *g13, const float *g2, const int32_t *tokens, int ntok, double *out,
+                        uint16_t *h_out)
 {
-    const size_t sb = fmt ? 1 : 2;  /* bytes per scale */
+    const size_t sb = fmt ? 1 : 2;        /* bytes per scale */
+    const int gsz = fmt == 2 ? 16 : 32;   /* inputs per scale */
     if (H % 32 || I % 32 || H < 32 || I < 32 || k < 1 || k > E) return 1;
     for (int i = 0; i < ntok; ++i)
         if (tokens[i] < 0 || tokens[i] >= T) return 1;
@@ -301,9 +316,10 @@ static int moe_q4_layer(int fmt, const uint16_t *x, const float *logits, int T, 
         for (int j = 0; j < k; ++j) {
             int e = ids[j];
             const int32_t *q13 = w13q + (size_t)e * 2 * I * (H / 8);
-            const void *s13 = (const char *)w13s + (size_t)e * 2 * I * (H / 32) * sb;
+            const void *s13 = (const char *)w13s + (size_t)e * 2 * I * (H / gsz) * sb;
             const int32_t *q2 = w2q + (size_t)e * H * (I / 8);
-            const void *s2 = (const char *)w2s + (size_t)e * H * (I / 32) * sb;
+            const void *s2 = (const char *)w2s + (size_t)e * H * (I / gsz) * sb;
+            const double ts13 = g13 ? (double)g13[e] : 1.0, ts2 = g2 ? (double)g2[e] : 1.0;
 #pragma omp parallel for schedule(static)
             for (int n = 0; n < I; ++n) {
                 double g = 0.0, u = 0.0;
@@ -311,6 +327,8 @@ static int moe_q4_layer(int fmt, const uint16_t *x, const float *logits, int T, 
                     g += xd[c] * q4_value(fmt, q13, s13, H, n, c);
                     u += xd[c] * q4_value(fmt, q13, s13, H, I + n, c);
                 }
+                g *= ts13;
+                u *= ts13;
                 uint16_t hb = bf16_round(silu(g) * u);
                 h[n] = bf16_value(hb);
                 if (h_out) h_out[((size_t)i * k + j) * I + n] = hb;
@@ -320,7 +338,7 @@ static int moe_q4_layer(int fmt, const uint16_t *x, const float *logits, int T, 
             for (int m = 0; m < H; ++m) {
                 double y = 0.0;
                 for (int n = 0; n < I; ++n) y += h[n] * q4_value(fmt, q2, s2, I, m, n);
-                o[m] += wj * y;
+                o[m] += wj * ts2 * y;
             }
         }
     }
@@ -332,7 +350,7 @@ int orc_moe_w4a16(const uint16_t *x, const float *logits, int T, int H, int I, i
                   const int32_t *w13q, const uint16_t *w13s, const int32_t *w2q, const uint16_t *w2s,
                   const int32_t *tokens, int ntok, double *out, uint16_t *h_out)
 {
-    return moe_q4_layer(0, x, logits, T, H, I, E, k, w13q, w13s, w2q, w2s, tokens, ntok, out, h_out);
+    return moe_q4_layer(0, x, logits, T, H, I, E, k, w13q, w13s, w2q, w2s, NULL, NULL, tokens, ntok, out, h_out);
 }
 
 /* The same layer with MXFP4 weights (E2M1 codes, UE8M0 group-32 scales [rows, K/32] bytes); the
@@ -341,7 +359,19 @@ int orc_moe_mxfp4(const uint16_t *x, const float *logits, int T, int H, int I, i
                   const int32_t *w13q, const uint8_t *w13s, const int32_t *w2q, const uint8_t *w2s,
                   const int32_t *tokens, int ntok, double *out, uint16_t *h_out)
 {
-    return moe_q4_layer(1, x, logits, T, H, I, E, k, w13q, w13s, w2q, w2s, tokens, ntok, out, h_out);
+    return moe_q4_layer(1, x, logits, T, H, I, E, k, w13q, w13s, w2q, w2s, NULL, NULL, tokens, ntok, out, h_out);
+}
+
+/* The same layer with NVFP4 weights: E2M1 codes, E4M3 group-16 scales [rows, K/16] bytes and one
+ * f32 tensor scale per expert and matrix (g13 [E] for the fused gate/up, g2 [E] for down):
+ * W = E2M1(q) * E4M3(s) * g. READING: one tensor scale for the fused gate/up matrix. */
+int orc_moe_nvfp4(const uint16_t *x, const float *logits, int T, int H, int I, int E, int k,
+                  const int32_t *w13q, const uint8_t *w13s, const float *g13, const int32_t *w2q,
+                  const uint8_t *w2s, const float *g2, const int32_t *tokens, int ntok, double *out,
+                  uint16_t *h_out)
+{
+    if (H % 32 || I % 32) return 1;
+    return moe_q4_layer(2, x, logits, T, H, I, E, k, w13q, w13s, w2q, w2s, g13, g2, tokens, ntok, out, h_out);
 }
 
 /* ------------------------------------------------------------------------------------------ */
@@ -544,6 +574,14 @@ int orc_w4a16_dequant(const int32_t *q, const uint16_t *s, int N, int K, double 
     if (K % 32 || K < 32) return 1;
     for (int r = 0; r < N; ++r)
         for (int c = 0; c < K; ++c) out[(size_t)r * K + c] = w4_value(q, s, K, r, c);
+    return 0;
+}
+
+int orc_nvfp4_dequant(const int32_t *q, const uint8_t *s, float g, int N, int K, double *out)
+{
+    if (K % 32 || K < 32) return 1;
+    for (int r = 0; r < N; ++r)
+        for (int c = 0; c < K; ++c) out[(size_t)r * K + c] = nvfp4_value(q, s, K, r, c) * (double)g;
     return 0;
 }
 

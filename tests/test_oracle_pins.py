@@ -506,6 +506,71 @@ def test_mxfp4_layer_dense_equivalence_with_uniform_routing():
     assert np.allclose(out, ref, rtol=1e-9, atol=1e-12)
 
 
+# ---- NVFP4 (E2M1 codes, E4M3 group-16 scales, f32 tensor scale) -------------------------------
+
+def _nvfp4_numpy_dequant(q, s, g):
+    q = np.asarray(q).view(np.uint32)
+    N, K8 = q.shape
+    codes = ((q[:, :, None] >> (4 * np.arange(8, dtype=np.uint32))) & 15).reshape(N, K8 * 8)
+    sv = torch.from_numpy(np.ascontiguousarray(s)).view(torch.float8_e4m3fn).double().numpy()
+    return _e2m1_via_e4m3(codes) * np.repeat(sv, 16, 1) * float(g)
+
+
+def test_nvfp4_dequant_hand_worked_and_numpy():
+    """Input 0 code 0x2 (1.0) with scale 0x40 (2.0), input 17 code 0xB (-1.5) with 0x30 (0.5), input
+    40 code 0x7 (6.0) with 0x2C (0.375), tensor scale 0.5: 1.0, -0.375, 1.125 (group = input / 16)."""
+    q = np.zeros((1, 8), np.uint32)
+    q[0, 0] = 0x2
+    q[0, 2] = 0xB << 4                 # input 17 = word 2, nibble 1
+    q[0, 5] = 0x7                      # input 40 = word 5, nibble 0
+    s = np.array([[0x40, 0x30, 0x2C, 0x38]], np.uint8)
+    deq = oracle.nvfp4_dequant(q.view(np.int32), s, 0.5)
+    want = np.zeros((1, 64))
+    want[0, 0], want[0, 17], want[0, 40] = 1.0, -0.375, 1.125
+    assert np.array_equal(deq, want)
+    d = W.make_moe(W.WORKLOADS["decode_nvfp4"], T=2, E=2, k=1, H=256, I=128)
+    for e in range(2):
+        qq, ss, gg = W.np_bits(d["w13q"][e]), W.np_bits(d["w13s"][e]), float(d["g13"][e])
+        assert np.array_equal(oracle.nvfp4_dequant(qq, ss, gg), _nvfp4_numpy_dequant(qq, ss, gg))
+
+
+def test_nvfp4_layer_equals_mxfp4_layer_on_power_of_two_scales():
+    """E4M3 scales that are powers of two, equal over each 32 inputs, and tensor scales of 1: the
+    NVFP4 layer is the MXFP4 layer with UE8M0 codes log2(scale) + 127."""
+    T, E, k, H, I = 3, 3, 2, 64, 32
+    rng = np.random.default_rng(9)
+    q13 = rng.integers(0, 2 ** 31, size=(E, 2 * I, H // 8), dtype=np.int64).astype(np.uint32).view(np.int32)
+    q2 = rng.integers(0, 2 ** 31, size=(E, H, I // 8), dtype=np.int64).astype(np.uint32).view(np.int32)
+    p13 = rng.integers(-4, 3, size=(E, 2 * I, H // 32))
+    p2 = rng.integers(-4, 3, size=(E, H, I // 32))
+    e4m3_of = lambda p: ((p + 7) << 3).astype(np.uint8)           # 2^p, p in [-6, 8]
+    n13, n2 = np.repeat(e4m3_of(p13), 2, -1), np.repeat(e4m3_of(p2), 2, -1)
+    m13, m2 = (p13 + 127).astype(np.uint8), (p2 + 127).astype(np.uint8)
+    x = torch.randn(T, H).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    ones = np.ones(E, np.float32)
+    a = oracle.moe_nvfp4(x, logits, k, q13, n13, ones, q2, n2, ones)
+    b = oracle.moe_mxfp4(x, logits, k, q13, m13, q2, m2)
+    assert np.array_equal(a, b)
+
+
+def test_nvfp4_layer_dense_equivalence_with_uniform_routing():
+    T, E, H, I = 3, 4, 128, 64
+    d = W.make_moe(W.WORKLOADS["decode_nvfp4"], T=T, E=E, k=E, H=H, I=I)
+    x = W.np_bits(d["x"])
+    q13, s13, q2, s2 = (W.np_bits(d[n]) for n in ("w13q", "w13s", "w2q", "w2s"))
+    g13, g2 = d["g13"].numpy(), d["g2"].numpy()
+    out = oracle.moe_nvfp4(x, np.zeros((T, E), np.float32), E, q13, s13, g13, q2, s2, g2)
+    xd = d["x"].double().numpy()
+    ref = np.zeros_like(out)
+    for e in range(E):
+        w13 = _nvfp4_numpy_dequant(q13[e], s13[e], g13[e])
+        g, u = xd @ w13[:I].T, xd @ w13[I:].T
+        h = torch.from_numpy(g / (1 + np.exp(-g)) * u).to(torch.bfloat16).double().numpy()
+        ref += 0.25 * (h @ _nvfp4_numpy_dequant(q2[e], s2[e], g2[e]).T)
+    assert np.allclose(out, ref, rtol=1e-9, atol=1e-12)
+
+
 def _torch_fp8_rows(v32):
     q, s = W.quantize_fp8_rows(torch.from_numpy(np.ascontiguousarray(v32)))
     return q.numpy(), s.numpy()

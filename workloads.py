@@ -36,7 +36,7 @@ SEED = 0
 @dataclass(frozen=True)
 class Workload:
     name: str
-    kind: str              # "w4a16", "mxfp4", "fp8" (MoE layers) or "dense_fp8"
+    kind: str              # "w4a16", "mxfp4", "nvfp4", "fp8" (MoE layers) or "dense_fp8"
     wid: int               # stream id of the workload
     T: int = 0
     H: int = 0
@@ -58,6 +58,8 @@ WORKLOADS = {
     # the decode and prefill layers with MXFP4 weights (E2M1 codes, UE8M0 group-32 scales)
     "decode_mxfp4": Workload("decode_mxfp4", "mxfp4", 6, T=32, H=7168, I=2048, E=384, k=8, logits="uniform"),
     "prefill_mxfp4": Workload("prefill_mxfp4", "mxfp4", 7, T=8192, H=7168, I=2048, E=384, k=8, logits="zipf"),
+    # ... and with NVFP4 weights (E2M1 codes, E4M3 group-16 scales, one f32 scale per expert matrix)
+    "decode_nvfp4": Workload("decode_nvfp4", "nvfp4", 8, T=32, H=7168, I=2048, E=384, k=8, logits="uniform"),
     # channelwise W8A8 FP8 GEMM at the N = K = 4096 shape the SGLang config page gives as its example
     "dense_fp8_channel": Workload("dense_fp8_channel", "dense_fp8_channel", 5,
                                   M_list=(1, 16, 64, 128, 256, 1024, 4096), N=4096, K=4096),
@@ -140,6 +142,41 @@ def quantize_mxfp4_group32(w: torch.Tensor):
     return packed.to(torch.int32).contiguous(), s.to(torch.uint8).contiguous()
 
 
+def _e2m1_codes(a: torch.Tensor, neg: torch.Tensor) -> torch.Tensor:
+    """|values| already scaled into [0, 6] -> E2M1 codes (nearest, ties to the even code)."""
+    mids = torch.tensor(_E2M1_MIDS, dtype=torch.float32, device=a.device)
+    code = torch.bucketize(a, mids)
+    lower = code.clamp(max=6)
+    code = code + ((a == mids[lower]) & (lower % 2 == 1)).to(code.dtype)
+    return code + 8 * (neg & (code > 0)).to(code.dtype)
+
+
+def _pack_nibbles(code: torch.Tensor, N: int, K: int) -> torch.Tensor:
+    q = code.to(torch.int64).reshape(N, K // 8, 8)
+    shifts = torch.arange(0, 32, 4, device=code.device, dtype=torch.int64)
+    packed = (q << shifts).sum(-1)
+    packed = packed - ((packed >> 31) & 1) * (1 << 32)
+    return packed.to(torch.int32).contiguous()
+
+
+def quantize_nvfp4_group16(w: torch.Tensor):
+    """f32 [N, K] -> (E2M1 codes packed int32 [N, K/8], E4M3 scales uint8 [N, K/16], f32 tensor
+    scale g). g = amax / (6 * 448); a 16-group's scale is E4M3(amax_group / (6 g)) (torch's
+    rounding); codes are the group's values over E4M3(scale) * g, nearest with ties to even."""
+    N, K = w.shape
+    wf = w.float()
+    amax = wf.abs().max()
+    g = (amax / (6.0 * 448.0)).clamp(min=1e-30)
+    wg = wf.view(N, K // 16, 16)
+    sg = (wg.abs().amax(-1) / (6.0 * g)).to(torch.float8_e4m3fn)
+    sv = sg.float()
+    denom = (sv * g)[..., None]
+    a = torch.where(denom > 0, wg.abs() / torch.where(denom > 0, denom, torch.ones_like(denom)),
+                    torch.zeros_like(wg)).clamp(max=6.0)
+    code = _e2m1_codes(a, wg < 0)
+    return _pack_nibbles(code, N, K), sg.view(torch.uint8).contiguous(), g.reshape(1)
+
+
 def quantize_fp8_blocks(w: torch.Tensor, bn: int = 128, bk: int = 128):
     """f32 [N, K] -> (E4M3 codes uint8 [N, K], f32 scales [N/bn, K/bk])."""
     N, K = w.shape
@@ -182,6 +219,19 @@ def make_moe(wl: Workload, device="cpu", T=None, E=None, k=None, H=None, I=None)
             g = generator(wl.wid, _W2, e, device=device)
             w2q[e], w2s[e] = quant(torch.randn((H, I), generator=g, device=device) * 0.02)
         d.update(w13q=w13q, w13s=w13s, w2q=w2q, w2s=w2s)
+    elif wl.kind == "nvfp4":
+        w13q = torch.empty((E, 2 * I, H // 8), dtype=torch.int32, device=device)
+        w13s = torch.empty((E, 2 * I, H // 16), dtype=torch.uint8, device=device)
+        w2q = torch.empty((E, H, I // 8), dtype=torch.int32, device=device)
+        w2s = torch.empty((E, H, I // 16), dtype=torch.uint8, device=device)
+        g13 = torch.empty((E,), dtype=torch.float32, device=device)
+        g2 = torch.empty((E,), dtype=torch.float32, device=device)
+        for e in range(E):
+            g = generator(wl.wid, _W13, e, device=device)
+            w13q[e], w13s[e], g13[e:e + 1] = quantize_nvfp4_group16(torch.randn((2 * I, H), generator=g, device=device) * 0.02)
+            g = generator(wl.wid, _W2, e, device=device)
+            w2q[e], w2s[e], g2[e:e + 1] = quantize_nvfp4_group16(torch.randn((H, I), generator=g, device=device) * 0.02)
+        d.update(w13q=w13q, w13s=w13s, w2q=w2q, w2s=w2s, g13=g13, g2=g2)
     elif wl.kind == "fp8":
         w13 = torch.empty((E, 2 * I, H), dtype=torch.uint8, device=device)
         w13s = torch.empty((E, 2 * I // 128, H // 128), dtype=torch.float32, device=device)
