@@ -143,6 +143,25 @@ MOEQ_API int moe_mxfp4_forward(const uint16_t *x, const float *logits, int T, in
                                void *stream);
 
 /*
+ * The same routed layer with NVFP4 weights (lk_moe page, "Supported models & quant formats": NVFP4,
+ * compressed-tensors / modelopt). A weight is E2M1(q) * E4M3(s) * g: q an E2M1 code (INT4 nibble
+ * order), s the E4M3 scale byte of its 16-input group, g one f32 tensor scale per expert and matrix.
+ *   moe_nvfp4_prepack_scales: the n E4M3 bytes -> n bf16 factors E4M3(s) * 2^118 (exact for every
+ *     E4M3 value; NaN stays NaN), run once per weight tensor.
+ *   moe_nvfp4_forward: w13_q i32 [E, 2I, H/8], w13_f bf16 [E, 2I, H/16] (prepacked factors),
+ *     w13_g f32 [E] (one tensor scale for the fused gate/up matrix), w2_q i32 [E, H, I/8],
+ *     w2_f bf16 [E, H, I/16], w2_g f32 [E]; workspace moe_nvfp4_workspace_size (equal to the W4A16
+ *     one); everything else, limits and errors as moe_w4a16_forward (NULL w13_g / w2_g:
+ *     INVALID_ARG).
+ */
+MOEQ_API int moe_nvfp4_prepack_scales(const uint8_t *e4m3, long long n, uint16_t *factors, void *stream);
+MOEQ_API size_t moe_nvfp4_workspace_size(int T, int H, int I, int E, int k);
+MOEQ_API int moe_nvfp4_forward(const uint16_t *x, const float *logits, int T, int H, int I, int E, int k,
+                               const int32_t *w13_q, const uint16_t *w13_f, const float *w13_g, const int32_t *w2_q,
+                               const uint16_t *w2_f, const float *w2_g, uint16_t *out, int32_t *topk_ids_out,
+                               float *topk_w_out, void *ws, size_t ws_bytes, void *stream);
+
+/*
  * Scratch-free W4A16 layer forward. The pages have no counterpart of this entry point: it exists
  * for callers that cannot allocate device memory where they run the layer, such as a plugin or
  * custom-op host that only hands over its input and output buffers, or a serving runtime that

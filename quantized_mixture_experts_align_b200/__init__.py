@@ -37,6 +37,9 @@ _SIGNATURES = {
     "moe_w4a16_forward": ([_V, _V, _I, _I, _I, _I, _I, _V, _V, _V, _V, _V, _V, _V, _V, _Z, _V], _I),
     "moe_w4a16_forward_noalloc": ([_V, _V, _I, _I, _I, _I, _I, _V, _V, _V, _V, _V, _V, _V, _V], _I),
     "moe_mxfp4_prepack_scales": ([_V, ctypes.c_longlong, _V, _V], _I),
+    "moe_nvfp4_prepack_scales": ([_V, ctypes.c_longlong, _V, _V], _I),
+    "moe_nvfp4_workspace_size": ([_I, _I, _I, _I, _I], _Z),
+    "moe_nvfp4_forward": ([_V, _V, _I, _I, _I, _I, _I, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _Z, _V], _I),
     "moe_mxfp4_workspace_size": ([_I, _I, _I, _I, _I], _Z),
     "moe_mxfp4_forward": ([_V, _V, _I, _I, _I, _I, _I, _V, _V, _V, _V, _V, _V, _V, _V, _Z, _V], _I),
     "moe_w8a8_block_fp8_workspace_size": ([_I, _I, _I, _I, _I], _Z),
@@ -196,6 +199,35 @@ def moe_mxfp4_forward(x, logits, k, w13_q, w13_f, w2_q, w2_f, out=None, ws=None,
         _dev(x, "x", _BF16), _dev(logits, "logits", torch.float32), T, H, I, E, k,
         _dev(w13_q, "w13_q", torch.int32), _dev(w13_f, "w13_f", _BF16), _dev(w2_q, "w2_q", torch.int32),
         _dev(w2_f, "w2_f", _BF16), _dev(out, "out", _BF16), _dev(topk_ids_out, "topk_ids_out", torch.int32),
+        _dev(topk_w_out, "topk_w_out", torch.float32), _dev(ws, "ws"), ws.numel() * ws.element_size(),
+        _stream(stream)))
+    return out
+
+
+def moe_nvfp4_prepack_scales(s_e4m3, out=None, stream=None):
+    """E4M3 group scales (uint8, any shape) -> the bf16 factors E4M3(s) * 2^118 moe_nvfp4_forward
+    takes (same shape)."""
+    out = torch.empty(s_e4m3.shape, dtype=torch.bfloat16, device=s_e4m3.device) if out is None else out
+    _check(lib().moe_nvfp4_prepack_scales(_dev(s_e4m3, "s_e4m3", _U8), s_e4m3.numel(), _dev(out, "out", _BF16),
+                                          _stream(stream)))
+    return out
+
+
+def moe_nvfp4_forward(x, logits, k, w13_q, w13_f, w13_g, w2_q, w2_f, w2_g, out=None, ws=None, topk_ids_out=None,
+                      topk_w_out=None, stream=None):
+    """The routed layer with NVFP4 weights: E2M1 codes (int32, the INT4 packing), the prepacked
+    bf16 group-16 factors of moe_nvfp4_prepack_scales and the f32 tensor scales [E] per matrix."""
+    T, H = x.shape
+    E = logits.shape[1]
+    I = w2_q.shape[2] * 8
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device) if out is None else out
+    need = lib().moe_nvfp4_workspace_size(T, H, I, E, k)
+    ws = workspace(need, x.device) if ws is None else ws
+    _check(lib().moe_nvfp4_forward(
+        _dev(x, "x", _BF16), _dev(logits, "logits", torch.float32), T, H, I, E, k,
+        _dev(w13_q, "w13_q", torch.int32), _dev(w13_f, "w13_f", _BF16), _dev(w13_g, "w13_g", torch.float32),
+        _dev(w2_q, "w2_q", torch.int32), _dev(w2_f, "w2_f", _BF16), _dev(w2_g, "w2_g", torch.float32),
+        _dev(out, "out", _BF16), _dev(topk_ids_out, "topk_ids_out", torch.int32),
         _dev(topk_w_out, "topk_w_out", torch.float32), _dev(ws, "ws"), ws.numel() * ws.element_size(),
         _stream(stream)))
     return out

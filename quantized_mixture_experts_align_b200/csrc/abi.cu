@@ -338,7 +338,7 @@ namespace moeq {
 static int w4_layer_forward(int fmt, const char *name, const uint16_t *x, const float *logits, int T, int H, int I,
                             int E, int k, const int32_t *w13_q, const uint16_t *w13_s, const int32_t *w2_q,
                             const uint16_t *w2_s, uint16_t *out, int32_t *topk_ids_out, float *topk_w_out, void *ws,
-                            size_t ws_bytes, void *stream)
+                            size_t ws_bytes, void *stream, const float *g13 = nullptr, const float *g2 = nullptr)
 {
     g_err[0] = 0;
     int rc = check_layer_shape(T, H, I, E, k);
@@ -399,6 +399,7 @@ static int w4_layer_forward(int fmt, const char *name, const uint16_t *x, const 
         t.rows_per_expert = 2 * I;
         t.wq = w13_q;
         t.ws = w13_s;
+        t.wglobal = g13;
         t.h_out = h;
         t.small_rows = kW4SmallRows;
         // the small blocks: register-fed kernel over the same 256-row alignment, h in slot order
@@ -415,6 +416,7 @@ static int w4_layer_forward(int fmt, const char *name, const uint16_t *x, const 
         g.act_row_div = k;
         g.wq = w13_q;
         g.ws = w13_s;
+        g.wglobal = g13;
         g.K = H;
         g.n_out = I;
         g.n_rows = 2 * I;
@@ -431,11 +433,13 @@ static int w4_layer_forward(int fmt, const char *name, const uint16_t *x, const 
         t.rows_per_expert = H;
         t.wq = w2_q;
         t.ws = w2_s;
+        t.wglobal = g2;
         t.ys = ys;
         g.act = h_small;
         g.act_row_div = 1;
         g.wq = w2_q;
         g.ws = w2_s;
+        g.wglobal = g2;
         g.K = I;
         g.n_out = H;
         g.n_rows = H;
@@ -460,6 +464,7 @@ static int w4_layer_forward(int fmt, const char *name, const uint16_t *x, const 
         a.act_row_div = k;
         a.wq = w13_q;
         a.ws = w13_s;
+        a.wglobal = g13;
         a.K = H;
         a.n_out = I;
         a.n_rows = 2 * I;
@@ -473,6 +478,7 @@ static int w4_layer_forward(int fmt, const char *name, const uint16_t *x, const 
         a.act_row_div = 1;
         a.wq = w2_q;
         a.ws = w2_s;
+        a.wglobal = g2;
         a.K = I;
         a.n_out = H;
         a.n_rows = H;
@@ -510,6 +516,33 @@ int moe_mxfp4_forward(const uint16_t *x, const float *logits, int T, int H, int 
 {
     return w4_layer_forward(W4_FP4, "moe_mxfp4_forward", x, logits, T, H, I, E, k, w13_q, w13_f, w2_q, w2_f, out,
                             topk_ids_out, topk_w_out, ws, ws_bytes, stream);
+}
+
+size_t moe_nvfp4_workspace_size(int T, int H, int I, int E, int k) { return moe_w4a16_workspace_size(T, H, I, E, k); }
+
+int moe_nvfp4_forward(const uint16_t *x, const float *logits, int T, int H, int I, int E, int k,
+                      const int32_t *w13_q, const uint16_t *w13_f, const float *w13_g, const int32_t *w2_q,
+                      const uint16_t *w2_f, const float *w2_g, uint16_t *out, int32_t *topk_ids_out, float *topk_w_out,
+                      void *ws, size_t ws_bytes, void *stream)
+{
+    g_err[0] = 0;
+    if (T > 0) {
+        MOEQ_REQUIRE(w13_g);
+        MOEQ_REQUIRE(w2_g);
+    }
+    return w4_layer_forward(W4_NV, "moe_nvfp4_forward", x, logits, T, H, I, E, k, w13_q, w13_f, w2_q, w2_f, out,
+                            topk_ids_out, topk_w_out, ws, ws_bytes, stream, w13_g, w2_g);
+}
+
+int moe_nvfp4_prepack_scales(const uint8_t *e4m3, long long n, uint16_t *factors, void *stream)
+{
+    g_err[0] = 0;
+    if (n < 0) return set_error(MOEQ_ERR_INVALID_ARG, "n must be >= 0 (got %lld)", n);
+    if (n == 0) return MOEQ_OK;
+    MOEQ_REQUIRE(e4m3);
+    MOEQ_REQUIRE(factors);
+    launch_nvfp4_scale_factors(e4m3, n, factors, num_sms(), (cudaStream_t)stream);
+    return check_launch("moe_nvfp4_prepack_scales");
 }
 
 int moe_mxfp4_prepack_scales(const uint8_t *ue8m0, long long n, uint16_t *factors, void *stream)

@@ -8,12 +8,15 @@ namespace moeq {
 
 enum { MODE_GATEUP = 0, MODE_DOWN = 1 };
 
-// 4-bit weight formats: INT4 codes with zero point 8 times bf16 group scales, or E2M1 codes times
-// bf16 group factors 2^(s - 1) (MXFP4 after moe_mxfp4_prepack_scales)
-enum { W4_INT4 = 0, W4_FP4 = 1 };
+// 4-bit weight formats: INT4 codes with zero point 8 times bf16 group-32 scales; E2M1 codes times
+// bf16 group-32 factors 2^(s - 1) (MXFP4 after moe_mxfp4_prepack_scales); E2M1 codes times bf16
+// group-16 factors E4M3(s) * 2^118 (NVFP4 after moe_nvfp4_prepack_scales), the accumulators then
+// scaled by the expert's f32 tensor scale * 2^8 (wglobal)
+enum { W4_INT4 = 0, W4_FP4 = 1, W4_NV = 2 };
 
 struct W4GroupedArgs {
-    int fmt;                 // W4_INT4 / W4_FP4
+    int fmt;                 // W4_INT4 / W4_FP4 / W4_NV
+    const float *wglobal;    // W4_NV: f32 tensor scale per expert [E]
     const uint16_t *act;     // gate/up: x [T, K]; down: h [T*k, K]  (bf16)
     int act_row_div;         // activation row of a slot = slot / act_row_div (k for x, 1 for h)
     const int32_t *wq;       // [E, n_rows, K/8]
@@ -78,7 +81,8 @@ struct Fp8TcArgs {
 };
 
 struct W4TcArgs {
-    int fmt;                // W4_INT4 / W4_FP4
+    int fmt;                // W4_INT4 / W4_FP4 / W4_NV
+    const float *wglobal;   // W4_NV: f32 tensor scale per expert [E]
     int M, N, K;            // activation rows (aligned capacity); output features / rows; inputs
     int *status;
     int E;
@@ -106,6 +110,9 @@ void launch_combine(const uint16_t *ys, int T, int k, int H, uint16_t *out, int 
 // UE8M0 group scales s -> the bf16 factors 2^(s - 1) the FP4 dequantization multiplies by (s > 128
 // overflows to +inf: group scales above 2 are outside the supported range)
 void launch_mxfp4_scale_factors(const uint8_t *s, long long n, uint16_t *f, int num_sms, cudaStream_t st);
+// E4M3 group scales -> the bf16 factors E4M3(s) * 2^118 (exact: 4 significant bits, range 2^109 ..
+// 1.75 * 2^126) the NVFP4 dequantization multiplies by; E4M3 NaN stays NaN
+void launch_nvfp4_scale_factors(const uint8_t *s, long long n, uint16_t *f, int num_sms, cudaStream_t st);
 void launch_fp8_act_quant(const uint16_t *x, int rows, int cols, uint8_t *q, float *s, cudaStream_t st);
 void launch_w4a16_grouped_mma(const W4GroupedArgs &a, int mode, int block_m, int max_blocks, cudaStream_t s);
 void launch_fp8_grouped_mma(const F8GroupedArgs &a, int mode, int block_m, int max_blocks, cudaStream_t s);

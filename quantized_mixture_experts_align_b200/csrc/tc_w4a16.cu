@@ -73,7 +73,7 @@ static_assert(64 * kTok * 4 <= kBStages * kBTile, "gate/up exchange fits in the 
 template <int FMT>
 __device__ __forceinline__ void dequant4(uint32_t w, uint32_t scale2, uint32_t *out)
 {
-    if (FMT == W4_FP4) {
+    if (FMT == W4_FP4 || FMT == W4_NV) {
         out[0] = bf16x2_mul(e2m1_pair_pre<0>(w), scale2);
         out[1] = bf16x2_mul(e2m1_pair_pre<1>(w), scale2);
         out[2] = bf16x2_mul(e2m1_pair_pre<2>(w), scale2);
@@ -198,16 +198,18 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
         const int grow = GU ? e * a.rows_per_expert + (row < 64 ? 0 : a.N) + n0 + (row & 63)
                             : e * a.rows_per_expert + n0 + row;
         const int32_t *wrow = a.wq + (size_t)grow * (K / 8) + kq * 4;  // 4 words = 32 inputs
-        // the group scale of this thread's 32 inputs comes with its neighbour's in one aligned
-        // 4-byte copy (rows are K/16 bytes apart, K a multiple of 128)
-        const uint16_t *srow = a.ws + (size_t)grow * (K / 32) + (kq & ~1);
+        // the group-32 scale of this thread's 32 inputs comes with its neighbour's in one aligned
+        // 4-byte copy (rows are K/16 bytes apart, K a multiple of 128); group 16: its own two
+        // scales, the same aligned 4 bytes
+        constexpr int GS = FMT == W4_NV ? 16 : 32;
+        const uint16_t *srow = a.ws + (size_t)grow * (K / GS) + (FMT == W4_NV ? 2 * kq : (kq & ~1));
         auto code_slot = [&](int slot) { return code_ring + ((size_t)slot * kDeqThreads + t) * 16; };
         auto scale_slot = [&](int slot) { return scale_ring + ((size_t)slot * kDeqThreads + t) * 4; };
         auto issue = [&](int ks) {
             if (ks < NS) {
                 const int slot = ks % kRing;
                 cp_async16_stream(code_slot(slot), wrow + ks * (kKs / 8));
-                cp_async4_ca(scale_slot(slot), srow + ks * (kKs / 32));
+                cp_async4_ca(scale_slot(slot), srow + ks * (kKs / GS));
             }
             cp_async_commit();
         };
@@ -230,12 +232,14 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
             const uint4 c = *reinterpret_cast<const uint4 *>(code_slot(slot));  // a warp reads 512 contiguous bytes
             const uint32_t sc = *reinterpret_cast<const uint32_t *>(scale_slot(slot));
             issue(ks + kRing - 1);  // refills the slot read in step ks - 1
-            const uint32_t s2 = prmt(sc, sc, (kq & 1) ? 0x3232u : 0x1010u);  // this slice's group, twice
+            // this slice's group scale, twice (group 16: words 0-1 the first, words 2-3 the second)
+            const uint32_t s2 = prmt(sc, sc, (FMT != W4_NV && (kq & 1)) ? 0x3232u : 0x1010u);
+            const uint32_t s2h = FMT == W4_NV ? prmt(sc, sc, 0x3232u) : s2;
             uint32_t pairs[16];
             dequant4<FMT>(c.x, s2, pairs + 0);
             dequant4<FMT>(c.y, s2, pairs + 4);
-            dequant4<FMT>(c.z, s2, pairs + 8);
-            dequant4<FMT>(c.w, s2, pairs + 12);
+            dequant4<FMT>(c.z, s2h, pairs + 8);
+            dequant4<FMT>(c.w, s2h, pairs + 12);
             if (pending >= 0) {
                 ok = stage_ready(pending);
                 pending = -1;
@@ -254,6 +258,8 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
         // ---- epilogue: tokens [64 kq, 64 kq + 64) of the tile, chunks of 32 ----
         ok = ok && tc::mbar_wait_warp(acc_full, 0, abort_flag, a.status);
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+        // NVFP4: the accumulator carries 2^-8 / (tensor scale) of the product
+        const float gsc = FMT == W4_NV ? __ldg(a.wglobal + e) * 256.f : 1.f;
         if (GU) {
             // up values (lanes 64-127) go through shared memory (the activation ring is free once
             // every MMA has completed) to the warps holding the matching gate values (lanes 0-63)
@@ -267,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
                     tc::tmem_ld32(lane_base + tok0, u);
                     tc::tmem_wait_ld();
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) up_s[(tok0 + j) * 64 + (row - 64)] = __uint_as_float(u[j]);
+                    for (int j = 0; j < 32; ++j) up_s[(tok0 + j) * 64 + (row - 64)] = gsc * __uint_as_float(u[j]);
                 }
             }
             asm volatile("bar.sync 1, %0;" ::"n"(kDeqThreads) : "memory");
@@ -282,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
                     tc::tmem_wait_ld();
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
-                        const float hv = silu_f32(__uint_as_float(g[j])) * up_s[(tok0 + j) * 64 + row];
+                        const float hv = silu_f32(gsc * __uint_as_float(g[j])) * up_s[(tok0 + j) * 64 + row];
                         hcol[(size_t)(r0 + tok0 + j) * a.N] = f32_to_bf16(hv);
                     }
                 }
@@ -297,7 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
                 tc::tmem_wait_ld();
                 const int my_slot = __ldg(a.sorted_ids + r0 + tok0 + lane);
                 // no routing weights (plain grouped GEMM): weight 1
-                const float my_w = (my_slot < a.n_slots) ? (a.topk_w ? __ldg(a.topk_w + my_slot) : 1.f) : 0.f;
+                const float my_w = (my_slot < a.n_slots) ? (a.topk_w ? __ldg(a.topk_w + my_slot) : 1.f) * gsc : 0.f;
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
                     const int slot = __shfl_sync(0xFFFFFFFFu, my_slot, j);
@@ -375,6 +381,10 @@ int launch_w4a16_tc(const W4TcArgs &a, int mode, const uint16_t *act, int max_bl
     if (a.fmt == W4_FP4) {
         if (mode == TC_GATEUP) return launch_mode<TC_GATEUP, W4_FP4>(a, tm, a.N / 64, max_blocks, s);
         return launch_mode<TC_DOWN, W4_FP4>(a, tm, a.N / 128, max_blocks, s);
+    }
+    if (a.fmt == W4_NV) {
+        if (mode == TC_GATEUP) return launch_mode<TC_GATEUP, W4_NV>(a, tm, a.N / 64, max_blocks, s);
+        return launch_mode<TC_DOWN, W4_NV>(a, tm, a.N / 128, max_blocks, s);
     }
     if (mode == TC_GATEUP) return launch_mode<TC_GATEUP, W4_INT4>(a, tm, a.N / 64, max_blocks, s);
     return launch_mode<TC_DOWN, W4_INT4>(a, tm, a.N / 128, max_blocks, s);

@@ -35,7 +35,7 @@ template <int FMT>
 __device__ __forceinline__ DeqWord dequant_word(uint32_t w, uint32_t scale2)
 {
     DeqWord d;
-    if (FMT == W4_FP4) {
+    if (FMT == W4_FP4 || FMT == W4_NV) {
         // E2M1 code times the group factor 2^(s - 1) (see e2m1_pair_pre)
         d.p[0] = bf16x2_mul(e2m1_pair_pre<0>(w), scale2);
         d.p[1] = bf16x2_mul(e2m1_pair_pre<1>(w), scale2);
@@ -70,7 +70,9 @@ __device__ __forceinline__ void act_pairs(const uint4 &v, uint32_t (&b)[4])
 // best: a deeper ring takes shared memory from the L1 share of the unified L1/shared storage,
 // which the activation and scale loads use.
 constexpr int kW4Stages = 4;
-constexpr int kW4StageBytes = 4 * 32 * 16 + 4 * 8 * 8;  // 2048 B codes + 256 B scales
+// 2048 B codes + the scales of 4 row sets x 8 rows: 4 group-32 or 8 group-16 bf16 scales each
+__host__ __device__ constexpr int w4_scale_slot_bytes(int fmt) { return fmt == W4_NV ? 16 : 8; }
+__host__ __device__ constexpr int w4_stage_bytes(int fmt) { return 4 * 32 * 16 + 4 * 8 * w4_scale_slot_bytes(fmt); }
 
 // MODE_GATEUP: rows [f0, f0+16) (gate) and [I + f0, I + f0 + 16) (up) of W13; epilogue writes
 //              h[slot, f] = bf16(silu(gate) * up).
@@ -108,7 +110,9 @@ __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4Grouped
     // token columns this lane feeds as MMA B (column g of each sub-tile)
     const int K = a.K;
     const int KW = K / 8;    // int32 words per weight row
-    const int KG = K / 32;   // scale groups per weight row
+    constexpr int GS = FMT == W4_NV ? 16 : 32;   // inputs per scale
+    constexpr int SB = w4_stage_bytes(FMT), SS = w4_scale_slot_bytes(FMT);
+    const int KG = K / GS;   // scale groups per weight row
     const uint16_t *act_row[MS];
 #pragma unroll
     for (int s = 0; s < MS; ++s) {
@@ -124,9 +128,9 @@ __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4Grouped
     for (int r = 0; r < 4; ++r) wr[r] = wq + (size_t)row_of_set[r] * KW + 4 * t;
     const uint16_t *my_scale_row = wsc + (size_t)row_of_set[t] * KG;  // copied by this lane
 
-    unsigned char *ring = smem + (size_t)warp * S * kW4StageBytes;
-    auto code_slot = [&](int st, int r) { return ring + st * kW4StageBytes + r * 512 + lane * 16; };
-    auto scale_slot = [&](int st, int r, int gg) { return ring + st * kW4StageBytes + 2048 + (r * 8 + gg) * 8; };
+    unsigned char *ring = smem + (size_t)warp * S * SB;
+    auto code_slot = [&](int st, int r) { return ring + st * SB + r * 512 + lane * 16; };
+    auto scale_slot = [&](int st, int r, int gg) { return ring + st * SB + 2048 + (r * 8 + gg) * SS; };
 
     const int NQ = K / 128;
     auto issue = [&](int q) {
@@ -134,7 +138,8 @@ __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4Grouped
             const int st = q % S;
 #pragma unroll
             for (int r = 0; r < 4; ++r) cp_async16_stream(code_slot(st, r), wr[r] + 16 * q);
-            cp_async8(scale_slot(st, t, g), my_scale_row + 4 * q);
+            if (FMT == W4_NV) cp_async16_stream(scale_slot(st, t, g), my_scale_row + 8 * q);
+            else cp_async8(scale_slot(st, t, g), my_scale_row + 4 * q);
         }
         cp_async_commit();  // possibly empty: keeps the group count uniform
     };
@@ -164,11 +169,15 @@ __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4Grouped
         uint4 wcur[4];
 #pragma unroll
         for (int r = 0; r < 4; ++r) wcur[r] = *reinterpret_cast<const uint4 *>(code_slot(st, r));
-        uint32_t sc[4];
+        // this lane's 32 inputs: one group-32 scale, or (group 16) one for words 0-1, one for 2-3
+        uint32_t sc[4], sc_hi[4];
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
-            const uint32_t s16 = reinterpret_cast<const uint16_t *>(scale_slot(st, r, g))[t];
+            const uint16_t *sr = reinterpret_cast<const uint16_t *>(scale_slot(st, r, g));
+            const uint32_t s16 = sr[FMT == W4_NV ? 2 * t : t];
             sc[r] = s16 | (s16 << 16);
+            const uint32_t s16h = FMT == W4_NV ? sr[2 * t + 1] : s16;
+            sc_hi[r] = s16h | (s16h << 16);
         }
         issue(q + S - 1);  // refills the slot every lane finished reading in iteration q - 1
 
@@ -187,7 +196,7 @@ __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4Grouped
             const uint32_t words[4] = {(&wcur[0].x)[m], (&wcur[1].x)[m], (&wcur[2].x)[m], (&wcur[3].x)[m]};
             DeqWord d[4];
 #pragma unroll
-            for (int r = 0; r < 4; ++r) d[r] = dequant_word<FMT>(words[r], sc[r]);
+            for (int r = 0; r < 4; ++r) d[r] = dequant_word<FMT>(words[r], m < 2 ? sc[r] : sc_hi[r]);
 #pragma unroll
             for (int s = 0; s < MS; ++s) {
                 uint4 xv;
@@ -211,7 +220,15 @@ __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4Grouped
     }
     cp_async_wait<0>();
 
-    // epilogue: lane holds rows (g, g+8) x columns (2t, 2t+1) of each sub-tile
+    // epilogue: lane holds rows (g, g+8) x columns (2t, 2t+1) of each sub-tile; NVFP4 accumulators
+    // carry 2^-8 / (tensor scale) of the true product
+    if (FMT == W4_NV) {
+        const float gsc = __ldg(a.wglobal + e) * 256.f;
+#pragma unroll
+        for (int s = 0; s < MS; ++s)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) { accA[s][i] *= gsc; accB[s][i] *= gsc; }
+    }
 #pragma unroll
     for (int s = 0; s < MS; ++s) {
 #pragma unroll
@@ -238,7 +255,7 @@ template <int BM, int WARPS, int MODE, bool STRIDED, int FMT>
 static void launch_bm_fmt(const W4GroupedArgs &a, int max_blocks, cudaStream_t s)
 {
     const int rows_per_cta = (MODE == MODE_GATEUP ? 16 : 32) * WARPS;
-    const size_t smem = (size_t)WARPS * kW4Stages * kW4StageBytes;
+    const size_t smem = (size_t)WARPS * kW4Stages * w4_stage_bytes(FMT);
     static bool attr_set = false;  // per template instance; the attribute is per function
     if (!attr_set) {
         cudaFuncSetAttribute(w4a16_grouped_mma_kernel<BM, WARPS, MODE, STRIDED, FMT>,
@@ -253,6 +270,7 @@ template <int BM, int WARPS, int MODE, bool STRIDED>
 static void launch_bm(const W4GroupedArgs &a, int max_blocks, cudaStream_t s)
 {
     if (a.fmt == W4_FP4) launch_bm_fmt<BM, WARPS, MODE, STRIDED, W4_FP4>(a, max_blocks, s);
+    else if (a.fmt == W4_NV) launch_bm_fmt<BM, WARPS, MODE, STRIDED, W4_NV>(a, max_blocks, s);
     else launch_bm_fmt<BM, WARPS, MODE, STRIDED, W4_INT4>(a, max_blocks, s);
 }
 
@@ -287,6 +305,31 @@ void launch_w4a16_grouped_mma(const W4GroupedArgs &a, int mode, int block_m, int
         default: break;
     }
 #undef MOEQ_W4_CASE
+}
+
+// E4M3 -> bf16 of E4M3 * 2^118: sign, exponent e (bias 7) and 3 mantissa bits m; e = 0 is the
+// subnormal range m * 2^-9. The f32 product is exact and its upper half is the bf16 value.
+__global__ void nvfp4_scale_factor_kernel(const uint8_t *__restrict__ sc, long long n, uint16_t *__restrict__ f)
+{
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+        const uint32_t b = sc[i], e = (b >> 3) & 15u, m = b & 7u;
+        uint32_t bits;
+        if (e == 15u && m == 7u) {
+            bits = 0x7FC0u;                                          // NaN
+        } else {
+            const float v = e ? __uint_as_float(((e + 120u) << 23) | (m << 20))  // 2^(e-7) (1+m/8)
+                              : (float)m * 0x1p-9f;
+            bits = __float_as_uint(v * 0x1p118f) >> 16;
+        }
+        f[i] = (uint16_t)(bits | ((b & 0x80u) << 8));
+    }
+}
+
+void launch_nvfp4_scale_factors(const uint8_t *s, long long n, uint16_t *f, int num_sms, cudaStream_t st)
+{
+    const long long want = (n + 255) / 256;
+    const int blocks = (int)(want < 8LL * num_sms ? want : 8LL * num_sms);
+    nvfp4_scale_factor_kernel<<<blocks, 256, 0, st>>>(s, n, f);
 }
 
 void launch_mxfp4_scale_factors(const uint8_t *s, long long n, uint16_t *f, int num_sms, cudaStream_t st)

@@ -96,6 +96,13 @@ def test_validation_rejects_before_device_work(L):
     assert _rc(L, "moe_mxfp4_prepack_scales", N, 16, p, N) == moeq.MOEQ_ERR_INVALID_ARG
     assert _rc(L, "moe_mxfp4_prepack_scales", p, -1, p, N) == moeq.MOEQ_ERR_INVALID_ARG
     assert _rc(L, "moe_mxfp4_prepack_scales", N, 0, N, N) == moeq.MOEQ_OK
+    # NVFP4 layer: tensor scales required; prepack like MXFP4's
+    nv = lambda g13, g2: _rc(L, "moe_nvfp4_forward", p, p, 32, 7168, 2048, 384, 8, p, p, g13, p, p, g2, p, N, N, p,
+                             1 << 40, N)
+    assert nv(N, p) == moeq.MOEQ_ERR_INVALID_ARG and nv(p, N) == moeq.MOEQ_ERR_INVALID_ARG
+    assert _rc(L, "moe_nvfp4_prepack_scales", N, 16, p, N) == moeq.MOEQ_ERR_INVALID_ARG
+    assert moeq.lib().moe_nvfp4_workspace_size(32, 7168, 2048, 384, 8) == \
+        moeq.lib().moe_w4a16_workspace_size(32, 7168, 2048, 384, 8)
     # channelwise dense matmul: K, N multiples of 128; aligned A, B, C; NULL scales
     cw = lambda A_, As_, C_, M, Nn, K: _rc(L, "w8a8_channel_fp8_matmul", A_, As_, p, p, M, Nn, K, C_, N)
     assert cw(p, p, p, 4, 256, 200) == moeq.MOEQ_ERR_UNSUPPORTED
