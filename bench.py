@@ -597,6 +597,27 @@ def main():
             "frac_of_bf16_peak": pflops / (qstep * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"]}
         del dm, dpm
         torch.cuda.empty_cache()
+        # NVFP4 weights (E2M1 codes, E4M3 group-16 scales, f32 tensor scales) on the same layer
+        dn = W.make_moe(W.WORKLOADS["decode_nvfp4"], device="cuda")
+        dn["w13f"] = moeq.moe_nvfp4_prepack_scales(dn["w13s"])
+        dn["w2f"] = moeq.moe_nvfp4_prepack_scales(dn["w2s"])
+        nout = torch.empty((dn["T"], dn["H"]), dtype=torch.bfloat16, device="cuda")
+        nws = moeq.workspace(moeq.lib().moe_nvfp4_workspace_size(dn["T"], dn["H"], dn["I"], dn["E"], dn["k"]), "cuda")
+        nstep_fn = lambda: moeq.moe_nvfp4_forward(dn["x"], dn["logits"], dn["k"], dn["w13q"], dn["w13f"], dn["g13"],
+                                                  dn["w2q"], dn["w2f"], dn["g2"], out=nout, ws=nws)
+        nms = timed_steps(nstep_fn, max(3, args.steps // 2), 3, flush, world)
+        nstep = max_over_ranks(statistics.mean(nms), world)
+        nact = touched_experts(moeq, dn)
+        # bytes the hot path reads: codes + the prepacked bf16 group-16 factors
+        H_, I_ = dn["H"], dn["I"]
+        nexp = (2 * I_ * H_ + H_ * I_) // 2 + (2 * I_ * H_ + H_ * I_) // 16 * 2
+        also["decode_nvfp4"] = {
+            "workload": "T=32 H=7168 I=2048 E=384 k=8, NVFP4 weights, bf16 activations", "ms_per_step": nstep,
+            "weight_gbs": nact * nexp / (nstep * 1e-3) / 1e9,
+            "hbm_frac": nact * nexp / (nstep * 1e-3) / 1e9 / peaks["hbm_gbs"], "touched_experts": nact,
+            "weight_bytes_per_step": nact * nexp}
+        del dn, nout, nws
+        torch.cuda.empty_cache()
         # grouped W4A16 GEMM, contiguous layout: the prefill routing's rows per expert, each
         # expert padded to 128 rows (m_indices -1), its W13 (N = 2I = 4096, K = H = 7168)
         pad = [int(c) + (-int(c)) % 128 for c in prows]

@@ -169,15 +169,17 @@ __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4Grouped
         uint4 wcur[4];
 #pragma unroll
         for (int r = 0; r < 4; ++r) wcur[r] = *reinterpret_cast<const uint4 *>(code_slot(st, r));
-        // this lane's 32 inputs: one group-32 scale, or (group 16) one for words 0-1, one for 2-3
-        uint32_t sc[4], sc_hi[4];
+        // this lane's 32 inputs: one group-32 scale, or (group 16) one for words 0-1 and one for
+        // words 2-3 (sc holds both halves then)
+        uint32_t sc[4];
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
-            const uint16_t *sr = reinterpret_cast<const uint16_t *>(scale_slot(st, r, g));
-            const uint32_t s16 = sr[FMT == W4_NV ? 2 * t : t];
-            sc[r] = s16 | (s16 << 16);
-            const uint32_t s16h = FMT == W4_NV ? sr[2 * t + 1] : s16;
-            sc_hi[r] = s16h | (s16h << 16);
+            if (FMT == W4_NV) {
+                sc[r] = reinterpret_cast<const uint32_t *>(scale_slot(st, r, g))[t];  // (lo, hi)
+            } else {
+                const uint32_t s16 = reinterpret_cast<const uint16_t *>(scale_slot(st, r, g))[t];
+                sc[r] = s16 | (s16 << 16);
+            }
         }
         issue(q + S - 1);  // refills the slot every lane finished reading in iteration q - 1
 
@@ -196,7 +198,8 @@ __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4Grouped
             const uint32_t words[4] = {(&wcur[0].x)[m], (&wcur[1].x)[m], (&wcur[2].x)[m], (&wcur[3].x)[m]};
             DeqWord d[4];
 #pragma unroll
-            for (int r = 0; r < 4; ++r) d[r] = dequant_word<FMT>(words[r], m < 2 ? sc[r] : sc_hi[r]);
+            for (int r = 0; r < 4; ++r)
+                d[r] = dequant_word<FMT>(words[r], FMT != W4_NV ? sc[r] : prmt(sc[r], sc[r], m < 2 ? 0x1010u : 0x3232u));
 #pragma unroll
             for (int s = 0; s < MS; ++s) {
                 uint4 xv;
