@@ -74,15 +74,26 @@ def test_layer_graph_replay_matches_eager(case):
     assert moeq.moe_device_status() == 0
 
 
-@pytest.mark.parametrize("M", [8, 100, 512])  # split-K, single-CTA tcgen05, CTA-pair tcgen05
-def test_dense_fp8_graph_replay_matches_eager(M):
-    dd = W.make_dense_fp8(W.WORKLOADS["dense_fp8"], M, device=DEV, N=512, K=1024)
-    c_eager = torch.empty((M, 512), dtype=torch.bfloat16, device=DEV)
+@pytest.mark.parametrize("kind,M,N,K", [
+    ("block", 8, 512, 1024),       # swap-AB tiles, K split over a cluster of 8
+    ("block", 100, 512, 1024),     # 128-row tiles, K split over a cluster of 4
+    ("block", 512, 8192, 1024),    # 128-row tiles, no split
+    ("channel", 40, 512, 1024),    # channelwise swap-AB
+    ("channel", 2400, 4096, 256),  # channelwise CTA pairs
+])
+def test_dense_fp8_graph_replay_matches_eager(kind, M, N, K):
+    if kind == "block":
+        dd = W.make_dense_fp8(W.WORKLOADS["dense_fp8"], M, device=DEV, N=N, K=K)
+        mm = moeq.w8a8_block_fp8_matmul
+    else:
+        dd = W.make_dense_fp8_channel(W.WORKLOADS["dense_fp8_channel"], M, device=DEV, N=N, K=K)
+        mm = moeq.w8a8_channel_fp8_matmul
+    c_eager = torch.empty((M, N), dtype=torch.bfloat16, device=DEV)
     c_graph = torch.empty_like(c_eager)
-    g = _capture(lambda: moeq.w8a8_block_fp8_matmul(dd["A"], dd["As"], dd["B"], dd["Bs"], out=c_graph))
+    g = _capture(lambda: mm(dd["A"], dd["As"], dd["B"], dd["Bs"], out=c_graph))
     c_graph.zero_()
     g.replay()
-    moeq.w8a8_block_fp8_matmul(dd["A"], dd["As"], dd["B"], dd["Bs"], out=c_eager)
+    mm(dd["A"], dd["As"], dd["B"], dd["Bs"], out=c_eager)
     torch.cuda.synchronize()
     assert torch.equal(c_graph.view(torch.int16), c_eager.view(torch.int16))
     assert moeq.moe_device_status() == 0
