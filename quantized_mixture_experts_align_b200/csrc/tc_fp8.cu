@@ -51,8 +51,10 @@ struct Fp8TcShape {
     static constexpr int kABytes = kBM * kBK;
     static constexpr int kBBytes = (PAIR ? BN / 2 : BN) * kBK;
     static constexpr int kStageBytes = kABytes + kBBytes;
-    // two partial buffers (128, 256 or 512 columns); channelwise: one accumulator over all of K
-    static constexpr int kTmemCols = MODE == TC_DENSE_CW ? BN : 2 * BN;
+    // partial buffers: all 512 tensor-memory columns (4 of 128 or 2 of 256), so the MMAs run up to
+    // kNBuf - 1 K blocks ahead of the promotion; channelwise: one accumulator over all of K
+    static constexpr int kNBuf = MODE == TC_DENSE_CW ? 1 : (BN <= 128 ? 4 : 2);
+    static constexpr int kTmemCols = kNBuf * BN;
     static constexpr int kSlices = epi_warps(MODE) / 4;  // column slices per lane quarter
     static constexpr int kColsPerWarp = BN / kSlices;
     static constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + 1024 + 256 + kSlices * 128 * 4;
@@ -91,8 +93,10 @@ __global__ void __launch_bounds__(fp8_threads(MODE), 1)
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + kStages * Sh::kStageBytes);
     uint64_t *empty = full + kStages;
     uint64_t *tfull = empty + kStages;
-    uint64_t *tempty = tfull + 2;
-    uint64_t *mma_done = tempty + 2;
+    constexpr int NB = Sh::kNBuf;
+    static_assert((2 * kStages + 2 * NB + 1) * 8 + 16 <= 256, "barriers, tensor-memory slot and flag fit their region");
+    uint64_t *tempty = tfull + NB;
+    uint64_t *mma_done = tempty + NB;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -146,7 +150,7 @@ __global__ void __launch_bounds__(fp8_threads(MODE), 1)
             tc::mbar_init(&full[s], 1);
             tc::mbar_init(&empty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < NB; ++b) {
             tc::mbar_init(&tfull[b], 1);
             tc::mbar_init(&tempty[b], kEpiWarps * (PAIR ? 2 : 1));  // pair: both CTAs' promotion warps
         }
@@ -208,10 +212,10 @@ __global__ void __launch_bounds__(fp8_threads(MODE), 1)
             constexpr uint32_t idesc = tc::idesc_f32(tc::kFmtE4M3, tc::kFmtE4M3, PAIR ? 2 * kBM : kBM, BN);
             const uint64_t a_base = tc::smem_desc_sw128(smem);
             for (int kb = 0; kb < nkb; ++kb) {
-                const int s = kb % kStages, buf = MODE == TC_DENSE_CW ? 0 : kb & 1;
+                const int s = kb % kStages, buf = kb % NB;
                 if (!tc::mbar_wait(&full[s], (kb / kStages) & 1, abort_flag, a.status)) break;
-                if (MODE != TC_DENSE_CW && kb >= 2 &&
-                    !tc::mbar_wait(&tempty[buf], ((kb >> 1) & 1) ^ 1, abort_flag, a.status))
+                if (MODE != TC_DENSE_CW && kb >= NB &&
+                    !tc::mbar_wait(&tempty[buf], ((kb / NB) & 1) ^ 1, abort_flag, a.status))
                     break;
                 tc::fence_after_sync();
                 // lean issue path: descriptors from a precomputed base; the first MMA of each K block
@@ -306,7 +310,7 @@ __global__ void __launch_bounds__(fp8_threads(MODE), 1)
         // the scales of block kb + 1 are loaded while block kb's partial is awaited
         float n_sa = __ldg(as_row), n_b0 = __ldg(bs_first), n_b1 = __ldg(bs_second);
         for (int kb = 0; kb < nkb && ok; ++kb) {
-            const int buf = kb & 1;
+            const int buf = kb % NB;
             const float sc0 = n_sa * n_b0, sc1 = n_sa * n_b1;
             if (kb + 1 < nkb) {
                 n_sa = __ldg(as_row + kb + 1);
@@ -314,7 +318,7 @@ __global__ void __launch_bounds__(fp8_threads(MODE), 1)
                 n_b1 = __ldg(bs_second + kb + 1);
             }
             // lane 0 waits, the warp agrees: the tensor-memory loads below are warp-wide
-            ok = tc::mbar_wait_warp(&tfull[buf], (kb >> 1) & 1, abort_flag, a.status);
+            ok = tc::mbar_wait_warp(&tfull[buf], (kb / NB) & 1, abort_flag, a.status);
             if (!ok) break;
             tc::fence_after_sync();
             const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + buf * BN;

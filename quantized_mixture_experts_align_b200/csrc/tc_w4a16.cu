@@ -78,12 +78,12 @@ __device__ __forceinline__ void dequant4(uint32_t w, uint32_t scale2, uint32_t *
         out[1] = bf16x2_mul(e2m1_pair_pre<1>(w), scale2);
         out[2] = bf16x2_mul(e2m1_pair_pre<2>(w), scale2);
         out[3] = bf16x2_mul(e2m1_pair_pre<3>(w), scale2);
-        return;
-    }
+    } else {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint32_t v = lop3_and_or(w >> (4 * i), 0x000F000Fu, 0x43004300u);  // 128 + q, exact
-        out[i] = bf16x2_mul(bf16x2_sub(v, 0x43084308u), scale2);                  // (q - 8), then * s
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t v = lop3_and_or(w >> (4 * i), 0x000F000Fu, 0x43004300u);  // 128 + q, exact
+            out[i] = bf16x2_mul(bf16x2_sub(v, 0x43084308u), scale2);                  // (q - 8), then * s
+        }
     }
 }
 

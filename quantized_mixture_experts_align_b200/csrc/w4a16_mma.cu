@@ -41,14 +41,14 @@ __device__ __forceinline__ DeqWord dequant_word(uint32_t w, uint32_t scale2)
         d.p[1] = bf16x2_mul(e2m1_pair_pre<1>(w), scale2);
         d.p[2] = bf16x2_mul(e2m1_pair_pre<2>(w), scale2);
         d.p[3] = bf16x2_mul(e2m1_pair_pre<3>(w), scale2);
-        return d;
-    }
-    const uint32_t magic = 0x43004300u;  // bf16 128.0 in both halves
-    const uint32_t bias = 0x43084308u;   // bf16 136.0 = 128 + 8 (zero point) in both halves
+    } else {
+        const uint32_t magic = 0x43004300u;  // bf16 128.0 in both halves
+        const uint32_t bias = 0x43084308u;   // bf16 136.0 = 128 + 8 (zero point) in both halves
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint32_t v = lop3_and_or(w >> (4 * i), 0x000F000Fu, magic);  // 128 + q, exact
-        d.p[i] = bf16x2_mul(bf16x2_sub(v, bias), scale2);                 // (q - 8) exact, then * s
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t v = lop3_and_or(w >> (4 * i), 0x000F000Fu, magic);  // 128 + q, exact
+            d.p[i] = bf16x2_mul(bf16x2_sub(v, bias), scale2);                 // (q - 8) exact, then * s
+        }
     }
     return d;
 }
