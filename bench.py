@@ -616,7 +616,20 @@ def main():
             "weight_gbs": nact * nexp / (nstep * 1e-3) / 1e9,
             "hbm_frac": nact * nexp / (nstep * 1e-3) / 1e9 / peaks["hbm_gbs"], "touched_experts": nact,
             "weight_bytes_per_step": nact * nexp}
-        del dn, nout, nws
+        # NVFP4 prefill: the same experts, the prefill tokens and Zipf routing
+        pout = torch.empty((wlp.T, dn["H"]), dtype=torch.bfloat16, device="cuda")
+        pws = moeq.workspace(moeq.lib().moe_nvfp4_workspace_size(wlp.T, dn["H"], dn["I"], dn["E"], dn["k"]), "cuda")
+        px = W.bf16_normal((wlp.T, dn["H"]), W.generator(wlp.wid, 0, device="cuda"), "cuda")
+        plg = W.router_logits(wlp, wlp.T, dn["E"], "cuda")
+        pfn = lambda: moeq.moe_nvfp4_forward(px, plg, dn["k"], dn["w13q"], dn["w13f"], dn["g13"], dn["w2q"], dn["w2f"],
+                                             dn["g2"], out=pout, ws=pws)
+        pnms = timed_steps(pfn, max(3, args.steps // 4), 3, None, world)
+        pnstep = max_over_ranks(statistics.mean(pnms), world)
+        also["prefill_nvfp4"] = {
+            "workload": "T=8192 H=7168 I=2048 E=384 k=8, Zipf-biased routing, NVFP4 weights", "ms_per_step": pnstep,
+            "tflops": pflops / (pnstep * 1e-3) / 1e12,
+            "frac_of_bf16_peak": pflops / (pnstep * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"]}
+        del dn, nout, nws, pout, pws, px, plg
         torch.cuda.empty_cache()
         # grouped W4A16 GEMM, contiguous layout: the prefill routing's rows per expert, each
         # expert padded to 128 rows (m_indices -1), its W13 (N = 2I = 4096, K = H = 7168)
