@@ -97,6 +97,7 @@ struct W4TcArgs {
     uint16_t *h_out;        // gate/up: [M, N] bf16, pair-permuted inside 8-element chunks
     uint16_t *ys;           // down: [n_slots, N] bf16, routing weight applied
     int small_rows;         // blocks with at most this many real rows are left to the register-fed path
+    int tiles_per_cta;      // down: output tiles of 128 rows per CTA (set by the launcher)
 };
 
 void launch_route_topk(const float *logits, int T, int E, int k, int32_t *ids, float *w, cudaStream_t s);

@@ -48,6 +48,7 @@ namespace {
 constexpr int kTok = 256;     // tokens per tile = aligned block size
 constexpr int kKs = 128;      // inputs per pipeline step (8 MMAs per barrier round trip)
 constexpr int kStages = 3;    // dequantized weight stages (tensor memory)
+constexpr int kDownTilesPerCta = 4;  // down GEMM: 128-row output tiles run by one CTA
 constexpr int kBStages = 3;   // activation tiles (shared memory)
 constexpr int kRing = 3;      // per-thread packed-code prefetch depth, in steps
 constexpr int kDeqWarps = 16;  // 4 per tensor-memory lane quarter, each a quarter of every step
@@ -107,7 +108,8 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
     uint64_t *empty = a_full + kStages;
     uint64_t *acc_full = empty + kStages;
     uint64_t *mma_done = acc_full + 1;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
+    uint64_t *acc_empty = mma_done + 1;  // down, several output tiles: the accumulator has been read
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -118,8 +120,14 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
     if (r0 >= __ldg(a.ntp)) return;  // uniform over the CTA, before any barrier or allocation
     const int e = __ldg(a.expert_ids + blockIdx.y);
     if (e < 0 || e >= a.E) return;
-    const int n0 = blockIdx.x * (GU ? 64 : 128);  // first output feature (gate/up) or row (down)
-    const int K = a.K, NS = K / kKs;
+    // gate/up: one tile of 64 features; down: nt consecutive 128-row output tiles of the block, run
+    // back to back through one pipeline (the setup, the ring fill and the prefetch of the next
+    // tile's weights are shared; only the accumulator drains between tiles)
+    const int tpc = GU ? 1 : a.tiles_per_cta;
+    const int tile0 = blockIdx.x * tpc;
+    const int nt = GU ? 1 : min(tpc, a.N / 128 - tile0);
+    const int n0 = tile0 * (GU ? 64 : 128);  // first output feature (gate/up) or row (down)
+    const int K = a.K, NS = K / kKs, NT = nt * NS;  // K steps per tile, in all
     // real rows of this block: the expert's slots come first, padding after
     const int valid = __syncthreads_count(threadIdx.x < kTok && __ldg(a.sorted_ids + r0 + threadIdx.x) < a.n_slots);
     const int n_mma = (valid + 15) & ~15;  // MMA N: multiple of 16 in [16, 256]
@@ -132,6 +140,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
         }
         tc::mbar_init(acc_full, 1);
         tc::mbar_init(mma_done, 1);
+        tc::mbar_init(acc_empty, kDeqWarps);
         *abort_flag = 0;
         tc::fence_barrier_init();
     }
@@ -145,19 +154,19 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
         if (lane == 0) {
             tc::prefetch_tmap(&tmX);
             int issued = 0;
-            for (int ks = 0; ks < NS; ++ks) {
-                const int s = ks % kBStages;
-                if (ks >= kBStages && !tc::mbar_wait(&empty[s], ((ks / kBStages) & 1) ^ 1, abort_flag, a.status))
+            for (int gs = 0; gs < NT; ++gs) {  // global step: tile gs / NS, K step gs % NS
+                const int s = gs % kBStages, ks = gs % NS;
+                if (gs >= kBStages && !tc::mbar_wait(&empty[s], ((gs / kBStages) & 1) ^ 1, abort_flag, a.status))
                     break;
                 // the tile's bytes complete on the stage's a_full barrier (dequantization warps + this
                 // arrival): the MMA thread waits on one barrier per step
                 tc::mbar_arrive_expect_tx(&a_full[s], kBTile);
                 tc::tma_load_2d(btiles + s * kBTile, &tmX, &a_full[s], ks * kKs, r0);
                 tc::tma_load_2d(btiles + s * kBTile + kBHalf, &tmX, &a_full[s], ks * kKs + kKs / 2, r0);
-                issued = ks + 1;
+                issued = gs + 1;
             }
-            for (int ks = issued - kBStages > 0 ? issued - kBStages : 0; ks < issued; ++ks)
-                tc::mbar_drain(&a_full[ks % kBStages], (ks / kBStages) & 1, a.status);
+            for (int gs = issued - kBStages > 0 ? issued - kBStages : 0; gs < issued; ++gs)
+                tc::mbar_drain(&a_full[gs % kBStages], (gs / kBStages) & 1, a.status);
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -166,11 +175,15 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
             // accumulate (the dequantization warps keep this SM's issue slots busy)
             const uint32_t a_base = tmem + kAccCols;
             const uint64_t b_base = tc::smem_desc_sw128(btiles);
-            for (int ks = 0; ks < NS; ++ks) {
-                const int s = ks % kStages, sb = ks % kBStages;  // equal: one stage index
+            for (int gs = 0; gs < NT; ++gs) {
+                const int s = gs % kStages, sb = gs % kBStages, ks = gs % NS;  // equal: one stage index
+                // a new tile overwrites the accumulator: the previous tile's epilogue has read it
+                if (ks == 0 && gs > 0 &&
+                    !tc::mbar_wait(acc_empty, ((gs / NS - 1) & 1), abort_flag, a.status))
+                    break;
                 // one wait per step: a_full completes when the weight stage and the activation tile
                 // are both in place
-                if (!tc::mbar_wait(&a_full[s], (ks / kStages) & 1, abort_flag, a.status)) break;
+                if (!tc::mbar_wait(&a_full[s], (gs / kStages) & 1, abort_flag, a.status)) break;
                 tc::fence_after_sync();
                 const uint64_t bdesc = b_base + (uint64_t)((sb * kBTile) >> 4);
                 const uint32_t astage = a_base + s * kAStageCols;
@@ -185,8 +198,8 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
                         tc::mma_f16_ts_acc(tmem, astage + kk * 8, bdesc + (kk >> 2) * (kBHalf >> 4) + 2 * (kk & 3), idesc);
                 }
                 tc::mma_commit(&empty[s]);  // frees the weight stage and the activation tile
+                if (ks == NS - 1) tc::mma_commit(acc_full);  // this tile's accumulator is complete
             }
-            tc::mma_commit(acc_full);
             tc::mma_commit(mma_done);
             tc::mbar_drain(mma_done, 0, a.status);
         }
@@ -198,23 +211,25 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
         const int grow = GU ? e * a.rows_per_expert + (row < 64 ? 0 : a.N) + n0 + (row & 63)
                             : e * a.rows_per_expert + n0 + row;
         const int32_t *wrow = a.wq + (size_t)grow * (K / 8) + kq * 4;  // 4 words = 32 inputs
+        const size_t wtile = (size_t)128 * (K / 8);                     // next output tile (down)
         // the group-32 scale of this thread's 32 inputs comes with its neighbour's in one aligned
         // 4-byte copy (rows are K/16 bytes apart, K a multiple of 128); group 16: its own two
         // scales, the same aligned 4 bytes
         constexpr int GS = FMT == W4_NV ? 16 : 32;
         const uint16_t *srow = a.ws + (size_t)grow * (K / GS) + (FMT == W4_NV ? 2 * kq : (kq & ~1));
+        const size_t stile = (size_t)128 * (K / GS);
         auto code_slot = [&](int slot) { return code_ring + ((size_t)slot * kDeqThreads + t) * 16; };
         auto scale_slot = [&](int slot) { return scale_ring + ((size_t)slot * kDeqThreads + t) * 4; };
-        auto issue = [&](int ks) {
-            if (ks < NS) {
-                const int slot = ks % kRing;
-                cp_async16_stream(code_slot(slot), wrow + ks * (kKs / 8));
-                cp_async4_ca(scale_slot(slot), srow + ks * (kKs / GS));
+        auto issue = [&](int gs) {  // global step: the ring runs on into the next tile's weights
+            if (gs < NT) {
+                const int slot = gs % kRing, tt = gs / NS, ks = gs % NS;
+                cp_async16_stream(code_slot(slot), wrow + tt * wtile + ks * (kKs / 8));
+                cp_async4_ca(scale_slot(slot), srow + tt * stile + ks * (kKs / GS));
             }
             cp_async_commit();
         };
 #pragma unroll
-        for (int ks = 0; ks < kRing - 1; ++ks) issue(ks);
+        for (int gs = 0; gs < kRing - 1; ++gs) issue(gs);
         // The stores of step ks are waited for (tcgen05.wait::st) only after the dequantization of
         // step ks + 1, so the tensor-memory write latency hides behind that work.
         auto stage_ready = [&](int j) -> bool {
@@ -226,12 +241,14 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
         };
         bool ok = true;
         int pending = -1;
+        for (int tt = 0; tt < nt && ok; ++tt) {
         for (int ks = 0; ks < NS && ok; ++ks) {
+            const int gs = tt * NS + ks;
             cp_async_wait<kRing - 2>();
-            const int slot = ks % kRing;
+            const int slot = gs % kRing;
             const uint4 c = *reinterpret_cast<const uint4 *>(code_slot(slot));  // a warp reads 512 contiguous bytes
             const uint32_t sc = *reinterpret_cast<const uint32_t *>(scale_slot(slot));
-            issue(ks + kRing - 1);  // refills the slot read in step ks - 1
+            issue(gs + kRing - 1);  // refills the slot read in step gs - 1
             // this slice's group scale, twice (group 16: words 0-1 the first, words 2-3 the second)
             const uint32_t s2 = prmt(sc, sc, (FMT != W4_NV && (kq & 1)) ? 0x3232u : 0x1010u);
             const uint32_t s2h = FMT == W4_NV ? prmt(sc, sc, 0x3232u) : s2;
@@ -245,18 +262,19 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
                 pending = -1;
                 if (!ok) break;
             }
-            const int s = ks % kStages;
-            if (ks >= kStages) ok = tc::mbar_wait_warp(&empty[s], ((ks / kStages) & 1) ^ 1, abort_flag, a.status);
+            const int s = gs % kStages;
+            if (gs >= kStages) ok = tc::mbar_wait_warp(&empty[s], ((gs / kStages) & 1) ^ 1, abort_flag, a.status);
             if (!ok) break;
             tc::fence_after_sync();
             tc::tmem_st16(tmem + ((uint32_t)(quarter * 32) << 16) + kAccCols + s * kAStageCols + kq * (kThrK / 2), pairs);
-            pending = ks;
+            pending = gs;
         }
-        if (pending >= 0) ok = stage_ready(pending);
-        cp_async_wait<0>();
+        if (pending >= 0 && ok) ok = stage_ready(pending);
+        pending = -1;
 
-        // ---- epilogue: tokens [64 kq, 64 kq + 64) of the tile, chunks of 32 ----
-        ok = ok && tc::mbar_wait_warp(acc_full, 0, abort_flag, a.status);
+        // ---- epilogue of tile tt: tokens [64 kq, 64 kq + 64), chunks of 32 ----
+        ok = ok && tc::mbar_wait_warp(acc_full, tt & 1, abort_flag, a.status);
+        const int nrow0 = n0 + tt * 128;  // down: this tile's first output row
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
         // NVFP4: the accumulator carries 2^-8 / (tensor scale) of the product
         const float gsc = FMT == W4_NV ? __ldg(a.wglobal + e) * 256.f : 1.f;
@@ -293,25 +311,35 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
                     }
                 }
             }
-        } else if (ok) {
-            tc::fence_after_sync();
-            for (int c = 0; c < kTok / kSplit / 32; ++c) {
-                const int tok0 = kq * (kTok / kSplit) + c * 32;
-                if (tok0 >= n_mma) break;
-                uint32_t y[32];
-                tc::tmem_ld32(lane_base + tok0, y);
-                tc::tmem_wait_ld();
-                const int my_slot = __ldg(a.sorted_ids + r0 + tok0 + lane);
-                // no routing weights (plain grouped GEMM): weight 1
-                const float my_w = (my_slot < a.n_slots) ? (a.topk_w ? __ldg(a.topk_w + my_slot) : 1.f) * gsc : 0.f;
+        } else {
+            if (ok) {
+                tc::fence_after_sync();
+                for (int c = 0; c < kTok / kSplit / 32; ++c) {
+                    const int tok0 = kq * (kTok / kSplit) + c * 32;
+                    if (tok0 >= n_mma) break;
+                    uint32_t y[32];
+                    tc::tmem_ld32(lane_base + tok0, y);
+                    tc::tmem_wait_ld();
+                    const int my_slot = __ldg(a.sorted_ids + r0 + tok0 + lane);
+                    // no routing weights (plain grouped GEMM): weight 1
+                    const float my_w =
+                        (my_slot < a.n_slots) ? (a.topk_w ? __ldg(a.topk_w + my_slot) : 1.f) * gsc : 0.f;
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int slot = __shfl_sync(0xFFFFFFFFu, my_slot, j);
-                    const float wt = __shfl_sync(0xFFFFFFFFu, my_w, j);
-                    if (slot < a.n_slots) a.ys[(size_t)slot * a.N + n0 + row] = f32_to_bf16(wt * __uint_as_float(y[j]));
+                    for (int j = 0; j < 32; ++j) {
+                        const int slot = __shfl_sync(0xFFFFFFFFu, my_slot, j);
+                        const float wt = __shfl_sync(0xFFFFFFFFu, my_w, j);
+                        if (slot < a.n_slots)
+                            a.ys[(size_t)slot * a.N + nrow0 + row] = f32_to_bf16(wt * __uint_as_float(y[j]));
+                    }
                 }
             }
+            // this warp has read its accumulator lanes: the next tile's MMAs may overwrite them
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(acc_empty);
         }
+        }  // output tiles
+        cp_async_wait<0>();
     }
     tc::fence_before_sync();
     __syncthreads();
@@ -373,21 +401,27 @@ int launch_mode(const W4TcArgs &a, const CUtensorMap &tm, int grid_x, int grid_y
 
 }  // namespace
 
-int launch_w4a16_tc(const W4TcArgs &a, int mode, const uint16_t *act, int max_blocks, cudaStream_t s)
+int launch_w4a16_tc(const W4TcArgs &a_in, int mode, const uint16_t *act, int max_blocks, cudaStream_t s)
 {
     CUtensorMap tm;
-    const int rc = make_tmap_2d(&tm, act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a.M, (uint64_t)a.K, kTok, kKs / 2);
+    const int rc = make_tmap_2d(&tm, act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a_in.M, (uint64_t)a_in.K,
+                                kTok, kKs / 2);
     if (rc) return rc;
+    // down: several 128-row output tiles per CTA share one pipeline (set-up, ring fill, weight
+    // prefetch across the tile boundary)
+    W4TcArgs a = a_in;
+    a.tiles_per_cta = mode == TC_GATEUP ? 1 : kDownTilesPerCta;
+    const int gx = mode == TC_GATEUP ? a.N / 64 : cdiv(a.N / 128, a.tiles_per_cta);
     if (a.fmt == W4_FP4) {
-        if (mode == TC_GATEUP) return launch_mode<TC_GATEUP, W4_FP4>(a, tm, a.N / 64, max_blocks, s);
-        return launch_mode<TC_DOWN, W4_FP4>(a, tm, a.N / 128, max_blocks, s);
+        if (mode == TC_GATEUP) return launch_mode<TC_GATEUP, W4_FP4>(a, tm, gx, max_blocks, s);
+        return launch_mode<TC_DOWN, W4_FP4>(a, tm, gx, max_blocks, s);
     }
     if (a.fmt == W4_NV) {
-        if (mode == TC_GATEUP) return launch_mode<TC_GATEUP, W4_NV>(a, tm, a.N / 64, max_blocks, s);
-        return launch_mode<TC_DOWN, W4_NV>(a, tm, a.N / 128, max_blocks, s);
+        if (mode == TC_GATEUP) return launch_mode<TC_GATEUP, W4_NV>(a, tm, gx, max_blocks, s);
+        return launch_mode<TC_DOWN, W4_NV>(a, tm, gx, max_blocks, s);
     }
-    if (mode == TC_GATEUP) return launch_mode<TC_GATEUP, W4_INT4>(a, tm, a.N / 64, max_blocks, s);
-    return launch_mode<TC_DOWN, W4_INT4>(a, tm, a.N / 128, max_blocks, s);
+    if (mode == TC_GATEUP) return launch_mode<TC_GATEUP, W4_INT4>(a, tm, gx, max_blocks, s);
+    return launch_mode<TC_DOWN, W4_INT4>(a, tm, gx, max_blocks, s);
 }
 
 void launch_gather_bf16_perm(const uint16_t *x, int H, int k, const int32_t *sorted_ids, const int32_t *ntp,
