@@ -154,16 +154,22 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
         if (lane == 0) {
             tc::prefetch_tmap(&tmX);
             int issued = 0;
-            for (int gs = 0; gs < NT; ++gs) {  // global step: tile gs / NS, K step gs % NS
-                const int s = gs % kBStages, ks = gs % NS;
-                if (gs >= kBStages && !tc::mbar_wait(&empty[s], ((gs / kBStages) & 1) ^ 1, abort_flag, a.status))
-                    break;
-                // the tile's bytes complete on the stage's a_full barrier (dequantization warps + this
-                // arrival): the MMA thread waits on one barrier per step
-                tc::mbar_arrive_expect_tx(&a_full[s], kBTile);
-                tc::tma_load_2d(btiles + s * kBTile, &tmX, &a_full[s], ks * kKs, r0);
-                tc::tma_load_2d(btiles + s * kBTile + kBHalf, &tmX, &a_full[s], ks * kKs + kKs / 2, r0);
-                issued = gs + 1;
+            bool live = true;
+            for (int tt = 0, gs = 0; tt < nt && live; ++tt) {
+                for (int ks = 0; ks < NS; ++ks, ++gs) {  // gs: global step over the tiles
+                    const int s = gs % kBStages;
+                    if (gs >= kBStages &&
+                        !tc::mbar_wait(&empty[s], ((gs / kBStages) & 1) ^ 1, abort_flag, a.status)) {
+                        live = false;
+                        break;
+                    }
+                    // the tile's bytes complete on the stage's a_full barrier (dequantization warps +
+                    // this arrival): the MMA thread waits on one barrier per step
+                    tc::mbar_arrive_expect_tx(&a_full[s], kBTile);
+                    tc::tma_load_2d(btiles + s * kBTile, &tmX, &a_full[s], ks * kKs, r0);
+                    tc::tma_load_2d(btiles + s * kBTile + kBHalf, &tmX, &a_full[s], ks * kKs + kKs / 2, r0);
+                    issued = gs + 1;
+                }
             }
             for (int gs = issued - kBStages > 0 ? issued - kBStages : 0; gs < issued; ++gs)
                 tc::mbar_drain(&a_full[gs % kBStages], (gs / kBStages) & 1, a.status);
@@ -175,15 +181,18 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
             // accumulate (the dequantization warps keep this SM's issue slots busy)
             const uint32_t a_base = tmem + kAccCols;
             const uint64_t b_base = tc::smem_desc_sw128(btiles);
-            for (int gs = 0; gs < NT; ++gs) {
-                const int s = gs % kStages, sb = gs % kBStages, ks = gs % NS;  // equal: one stage index
-                // a new tile overwrites the accumulator: the previous tile's epilogue has read it
-                if (ks == 0 && gs > 0 &&
-                    !tc::mbar_wait(acc_empty, ((gs / NS - 1) & 1), abort_flag, a.status))
-                    break;
+            bool live = true;
+            for (int tt = 0, gs = 0; tt < nt && live; ++tt) {
+            // a new tile overwrites the accumulator: the previous tile's epilogue has read it
+            if (tt > 0 && !tc::mbar_wait(acc_empty, (tt - 1) & 1, abort_flag, a.status)) break;
+            for (int ks = 0; ks < NS; ++ks, ++gs) {
+                const int s = gs % kStages, sb = gs % kBStages;  // equal: one stage index
                 // one wait per step: a_full completes when the weight stage and the activation tile
                 // are both in place
-                if (!tc::mbar_wait(&a_full[s], (gs / kStages) & 1, abort_flag, a.status)) break;
+                if (!tc::mbar_wait(&a_full[s], (gs / kStages) & 1, abort_flag, a.status)) {
+                    live = false;
+                    break;
+                }
                 tc::fence_after_sync();
                 const uint64_t bdesc = b_base + (uint64_t)((sb * kBTile) >> 4);
                 const uint32_t astage = a_base + s * kAStageCols;
@@ -198,7 +207,8 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
                         tc::mma_f16_ts_acc(tmem, astage + kk * 8, bdesc + (kk >> 2) * (kBHalf >> 4) + 2 * (kk & 3), idesc);
                 }
                 tc::mma_commit(&empty[s]);  // frees the weight stage and the activation tile
-                if (ks == NS - 1) tc::mma_commit(acc_full);  // this tile's accumulator is complete
+            }
+            if (live) tc::mma_commit(acc_full);  // this tile's accumulator is complete
             }
             tc::mma_commit(mma_done);
             tc::mbar_drain(mma_done, 0, a.status);
@@ -220,16 +230,27 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
         const size_t stile = (size_t)128 * (K / GS);
         auto code_slot = [&](int slot) { return code_ring + ((size_t)slot * kDeqThreads + t) * 16; };
         auto scale_slot = [&](int slot) { return scale_ring + ((size_t)slot * kDeqThreads + t) * 4; };
-        auto issue = [&](int gs) {  // global step: the ring runs on into the next tile's weights
-            if (gs < NT) {
-                const int slot = gs % kRing, tt = gs / NS, ks = gs % NS;
-                cp_async16_stream(code_slot(slot), wrow + tt * wtile + ks * (kKs / 8));
-                cp_async4_ca(scale_slot(slot), srow + tt * stile + ks * (kKs / GS));
+        // prefetch position (global step pg = tile pt, K step pk): advanced by one per issue, so the
+        // ring runs on into the next tile's weights without a division
+        int pg = 0, pk = 0;
+        const int32_t *pw = wrow;
+        const uint16_t *ps = srow;
+        auto issue = [&]() {
+            if (pg < NT) {
+                const int slot = pg % kRing;
+                cp_async16_stream(code_slot(slot), pw + pk * (kKs / 8));
+                cp_async4_ca(scale_slot(slot), ps + pk * (kKs / GS));
+                ++pg;
+                if (++pk == NS) {
+                    pk = 0;
+                    pw += wtile;
+                    ps += stile;
+                }
             }
             cp_async_commit();
         };
 #pragma unroll
-        for (int gs = 0; gs < kRing - 1; ++gs) issue(gs);
+        for (int gs = 0; gs < kRing - 1; ++gs) issue();
         // The stores of step ks are waited for (tcgen05.wait::st) only after the dequantization of
         // step ks + 1, so the tensor-memory write latency hides behind that work.
         auto stage_ready = [&](int j) -> bool {
@@ -248,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
             const int slot = gs % kRing;
             const uint4 c = *reinterpret_cast<const uint4 *>(code_slot(slot));  // a warp reads 512 contiguous bytes
             const uint32_t sc = *reinterpret_cast<const uint32_t *>(scale_slot(slot));
-            issue(gs + kRing - 1);  // refills the slot read in step gs - 1
+            issue();  // step gs + kRing - 1: refills the slot read in step gs - 1
             // this slice's group scale, twice (group 16: words 0-1 the first, words 2-3 the second)
             const uint32_t s2 = prmt(sc, sc, (FMT != W4_NV && (kq & 1)) ? 0x3232u : 0x1010u);
             const uint32_t s2h = FMT == W4_NV ? prmt(sc, sc, 0x3232u) : s2;
