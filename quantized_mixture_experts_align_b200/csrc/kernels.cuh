@@ -78,6 +78,7 @@ struct Fp8TcArgs {
     uint8_t *hq;            // gate/up out: [M, N] E4M3
     float *hs;              // gate/up out: [M, N/128]
     uint16_t *ys;           // down out: [n_slots, N] bf16, routing weight applied
+    int tiles_per_cta;      // grouped down: output tiles per CTA (set by the launcher)
 };
 
 struct W4TcArgs {

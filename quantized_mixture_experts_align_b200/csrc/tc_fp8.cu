@@ -35,6 +35,7 @@ namespace moeq {
 namespace {
 
 constexpr int kBM = 128;
+constexpr int kFp8DownTilesPerCta = 4;  // grouped down GEMM: output tiles run by one CTA
 constexpr int kBK = 128;  // one scale block; bytes = elements for E4M3
 // promotion warps: 4 per tensor-memory lane quarter (each a quarter of the columns) for gate/up,
 // whose epilogue is the heaviest; 2 per quarter (each half of the columns) otherwise, which
@@ -136,7 +137,7 @@ __global__ void __launch_bounds__(fp8_threads(MODE), 1)
             bscale0 = ws + (size_t)(n0 / 128) * KB;
             bscale1 = ws + (size_t)((a.N + n0) / 128) * KB;
         } else {
-            n0 = tile_x * BN;
+            n0 = tile_x * a.tiles_per_cta * BN;  // the first of this CTA's output tiles
             brow0 = e * a.rows_per_expert + n0;
             bscale0 = ws + (size_t)(n0 / 128) * KB;
         }
@@ -144,6 +145,10 @@ __global__ void __launch_bounds__(fp8_threads(MODE), 1)
     // weight rows this CTA loads: all BN, or (pair) its half: gate/up rank 0 the gate rows, rank 1
     // the up rows; dense / down rank r the rows [128 r, 128 r + 128) of the tile
     const int brow_own = !PAIR ? brow0 : (MODE == TC_GATEUP ? (rank ? brow1 : brow0) : brow0 + (int)rank * 128);
+    // grouped down: ntl consecutive BN-column output tiles of the block run through one pipeline;
+    // the promotion warps hold the accumulator in registers, so the next tile's MMAs overlap this
+    // tile's epilogue
+    const int ntl = MODE == TC_DOWN ? min(a.tiles_per_cta, a.N / BN - tile_x * a.tiles_per_cta) : 1;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -173,9 +178,14 @@ __global__ void __launch_bounds__(fp8_threads(MODE), 1)
             tc::prefetch_tmap(&tmA);
             tc::prefetch_tmap(&tmB);
             int issued = 0;
-            for (int kb = 0; kb < nkb; ++kb) {  // local index; x = (kb0 + kb) * kBK
-                const int s = kb % kStages;
-                if (kb >= kStages && !tc::mbar_wait(&empty[s], ((kb / kStages) & 1) ^ 1, abort_flag, a.status)) break;
+            bool live = true;
+            for (int tt = 0, gs = 0; tt < ntl && live; ++tt)
+            for (int kb = 0; kb < nkb; ++kb, ++gs) {  // local K index, x = (kb0 + kb) * kBK; gs over tiles
+                const int s = gs % kStages;
+                if (gs >= kStages && !tc::mbar_wait(&empty[s], ((gs / kStages) & 1) ^ 1, abort_flag, a.status)) {
+                    live = false;
+                    break;
+                }
                 uint8_t *sa = smem + s * Sh::kStageBytes;
                 if (PAIR) {
                     // both CTAs' bytes complete on rank 0's barrier, which alone expects them
@@ -183,7 +193,7 @@ __global__ void __launch_bounds__(fp8_threads(MODE), 1)
                     if (rank == 0) tc::mbar_arrive_expect_tx(&full[s], 2 * Sh::kStageBytes);
                     tc::tma_load_2d_pair(sa, &tmA, fb, kb * kBK, m0);
                     tc::tma_load_2d_pair(sa + Sh::kABytes, &tmB, fb, kb * kBK, brow_own);
-                    issued = kb + 1;
+                    issued = gs + 1;
                     continue;
                 }
                 tc::mbar_arrive_expect_tx(&full[s], Sh::kStageBytes);
@@ -193,15 +203,15 @@ __global__ void __launch_bounds__(fp8_threads(MODE), 1)
                     tc::tma_load_2d(sa + Sh::kABytes, &tmB, &full[s], x, brow0);
                     tc::tma_load_2d(sa + Sh::kABytes + 128 * kBK, &tmB, &full[s], x, brow1);
                 } else {
-                    tc::tma_load_2d(sa + Sh::kABytes, &tmB, &full[s], x, brow0);
+                    tc::tma_load_2d(sa + Sh::kABytes, &tmB, &full[s], x, brow0 + tt * BN);
                 }
-                issued = kb + 1;
+                issued = gs + 1;
             }
             // no copy may still be landing in shared memory when the CTA exits (pair: rank 0's
             // barrier counts both CTAs' bytes; rank 1 is held by the final cluster barrier)
             if (!PAIR || rank == 0)
-                for (int kb = issued - kStages > 0 ? issued - kStages : 0; kb < issued; ++kb)
-                    tc::mbar_drain(&full[kb % kStages], (kb / kStages) & 1, a.status);
+                for (int gs = issued - kStages > 0 ? issued - kStages : 0; gs < issued; ++gs)
+                    tc::mbar_drain(&full[gs % kStages], (gs / kStages) & 1, a.status);
         }
     } else if (warp == 1) {
         if (PAIR && rank != 0) {
@@ -211,12 +221,16 @@ __global__ void __launch_bounds__(fp8_threads(MODE), 1)
         } else if (lane == 0) {
             constexpr uint32_t idesc = tc::idesc_f32(tc::kFmtE4M3, tc::kFmtE4M3, PAIR ? 2 * kBM : kBM, BN);
             const uint64_t a_base = tc::smem_desc_sw128(smem);
-            for (int kb = 0; kb < nkb; ++kb) {
-                const int s = kb % kStages, buf = kb % NB;
-                if (!tc::mbar_wait(&full[s], (kb / kStages) & 1, abort_flag, a.status)) break;
-                if (MODE != TC_DENSE_CW && kb >= NB &&
-                    !tc::mbar_wait(&tempty[buf], ((kb / NB) & 1) ^ 1, abort_flag, a.status))
+            bool live = true;
+            for (int tt = 0, gs = 0; tt < ntl && live; ++tt)
+            for (int kb = 0; kb < nkb; ++kb, ++gs) {
+                const int s = gs % kStages, buf = gs % NB;
+                if (!tc::mbar_wait(&full[s], (gs / kStages) & 1, abort_flag, a.status) ||
+                    (MODE != TC_DENSE_CW && gs >= NB &&
+                     !tc::mbar_wait(&tempty[buf], ((gs / NB) & 1) ^ 1, abort_flag, a.status))) {
+                    live = false;
                     break;
+                }
                 tc::fence_after_sync();
                 // lean issue path: descriptors from a precomputed base; the first MMA of each K block
                 // starts the partial, the other three always accumulate
@@ -301,16 +315,19 @@ __global__ void __launch_bounds__(fp8_threads(MODE), 1)
         const int c_first = (MODE == TC_GATEUP) ? GF * cq : cq * COLS;
         const int c_second = (MODE == TC_GATEUP) ? 128 + GF * cq : 0;
         const float *as_row = a.a_scale + (size_t)(m < a.M ? m : a.M - 1) * KB + kb0;
-        const float *bs_first = ((MODE == TC_GATEUP) ? bscale0 : bscale0 + (size_t)((cq * COLS) / 128) * KB) + kb0;
+        bool ok = true;
+        for (int tt = 0, gs = 0; tt < ntl && ok; ++tt) {
+        const int n0t = n0 + tt * BN;  // this tile's first output column
+        const float *bs_first =
+            ((MODE == TC_GATEUP) ? bscale0 : bscale0 + (size_t)((tt * BN + cq * COLS) / 128) * KB) + kb0;
         const float *bs_second = (MODE == TC_GATEUP) ? bscale1 + kb0 : bs_first;
         float acc[COLS];
 #pragma unroll
         for (int j = 0; j < COLS; ++j) acc[j] = 0.f;
-        bool ok = true;
         // the scales of block kb + 1 are loaded while block kb's partial is awaited
         float n_sa = __ldg(as_row), n_b0 = __ldg(bs_first), n_b1 = __ldg(bs_second);
-        for (int kb = 0; kb < nkb && ok; ++kb) {
-            const int buf = kb % NB;
+        for (int kb = 0; kb < nkb && ok; ++kb, ++gs) {
+            const int buf = gs % NB;
             const float sc0 = n_sa * n_b0, sc1 = n_sa * n_b1;
             if (kb + 1 < nkb) {
                 n_sa = __ldg(as_row + kb + 1);
@@ -318,7 +335,7 @@ __global__ void __launch_bounds__(fp8_threads(MODE), 1)
                 n_b1 = __ldg(bs_second + kb + 1);
             }
             // lane 0 waits, the warp agrees: the tensor-memory loads below are warp-wide
-            ok = tc::mbar_wait_warp(&tfull[buf], (kb / NB) & 1, abort_flag, a.status);
+            ok = tc::mbar_wait_warp(&tfull[buf], (gs / NB) & 1, abort_flag, a.status);
             if (!ok) break;
             tc::fence_after_sync();
             const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + buf * BN;
@@ -398,7 +415,7 @@ __global__ void __launch_bounds__(fp8_threads(MODE), 1)
             const int slot = __ldg(a.sorted_ids + m);
             if (ok && slot < a.n_slots) {
                 const float wt = __ldg(a.topk_w + slot);
-                uint16_t *yrow = a.ys + (size_t)slot * a.N + n0 + cq * COLS;
+                uint16_t *yrow = a.ys + (size_t)slot * a.N + n0t + cq * COLS;
 #pragma unroll
                 for (int j = 0; j < COLS; j += 8) {
                     uint4 v;
@@ -410,6 +427,7 @@ __global__ void __launch_bounds__(fp8_threads(MODE), 1)
                 }
             }
         }
+        }  // output tiles
     }
     tc::fence_before_sync();
     if (kDense && !PAIR && nsplit > 1) {
@@ -547,9 +565,13 @@ int launch_fp8_tc_channel(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B
     return launch_tc<128, TC_DENSE_CW>(a, tmA, tmB, cdiv(a.M, kBM), a.N / 128, s, sch.split);
 }
 
-int launch_fp8_tc_grouped(const Fp8TcArgs &a, int mode, const uint8_t *A, const uint8_t *W, int E, int max_blocks,
+int launch_fp8_tc_grouped(const Fp8TcArgs &a_in, int mode, const uint8_t *A, const uint8_t *W, int E, int max_blocks,
                           cudaStream_t s)
 {
+    // down: kFp8DownTilesPerCta output tiles per CTA (the K range is short, I = 2048: the fixed
+    // per-CTA cost is shared and the next tile's MMAs overlap the epilogue)
+    Fp8TcArgs a = a_in;
+    a.tiles_per_cta = mode == TC_DOWN ? kFp8DownTilesPerCta : 1;
     CUtensorMap tmA, tmB;
     int rc = make_tmap_2d(&tmA, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.M, (uint64_t)a.K, kBM, kBK);
     if (rc) return rc;
@@ -558,8 +580,9 @@ int launch_fp8_tc_grouped(const Fp8TcArgs &a, int mode, const uint8_t *A, const 
                       kBK);
     if (rc) return rc;
     if (mode == TC_GATEUP) return launch_tc<256, TC_GATEUP>(a, tmA, tmB, a.N / 128, max_blocks, s);
-    if (a.N % 256 == 0) return launch_tc<256, TC_DOWN>(a, tmA, tmB, a.N / 256, max_blocks, s);
-    return launch_tc<128, TC_DOWN>(a, tmA, tmB, a.N / 128, max_blocks, s);
+    if (a.N % 256 == 0)
+        return launch_tc<256, TC_DOWN>(a, tmA, tmB, cdiv(a.N / 256, a.tiles_per_cta), max_blocks, s);
+    return launch_tc<128, TC_DOWN>(a, tmA, tmB, cdiv(a.N / 128, a.tiles_per_cta), max_blocks, s);
 }
 
 }  // namespace moeq
