@@ -49,7 +49,6 @@ constexpr int kTok = 256;     // tokens per tile = aligned block size
 constexpr int kKs = 128;      // inputs per pipeline step (8 MMAs per barrier round trip)
 constexpr int kStages = 3;    // dequantized weight stages (tensor memory)
 constexpr int kDownTilesPerCta = 4;  // down GEMM: 128-row output tiles run by one CTA
-constexpr int kGateUpTilesPerCta = 2;  // gate/up GEMM: 64-feature tiles run by one CTA
 constexpr int kBStages = 3;   // activation tiles (shared memory)
 constexpr int kRing = 3;      // per-thread packed-code prefetch depth, in steps
 constexpr int kDeqWarps = 16;  // 4 per tensor-memory lane quarter, each a quarter of every step
@@ -121,14 +120,13 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
     if (r0 >= __ldg(a.ntp)) return;  // uniform over the CTA, before any barrier or allocation
     const int e = __ldg(a.expert_ids + blockIdx.y);
     if (e < 0 || e >= a.E) return;
-    // nt consecutive output tiles of the block (gate/up: 64 features, down: 128 rows) run back to
-    // back through one pipeline: the set-up, the ring fill and the prefetch of the next tile's
-    // weights are shared; only the accumulator drains between tiles
-    constexpr int kTileRows = GU ? 64 : 128;
-    const int tpc = a.tiles_per_cta;
+    // gate/up: one tile of 64 features; down: nt consecutive 128-row output tiles of the block, run
+    // back to back through one pipeline (the setup, the ring fill and the prefetch of the next
+    // tile's weights are shared; only the accumulator drains between tiles)
+    const int tpc = GU ? 1 : a.tiles_per_cta;
     const int tile0 = blockIdx.x * tpc;
-    const int nt = min(tpc, a.N / kTileRows - tile0);
-    const int n0 = tile0 * kTileRows;  // first output feature (gate/up) or row (down)
+    const int nt = GU ? 1 : min(tpc, a.N / 128 - tile0);
+    const int n0 = tile0 * (GU ? 64 : 128);  // first output feature (gate/up) or row (down)
     const int K = a.K, NS = K / kKs, NT = nt * NS;  // K steps per tile, in all
     // real rows of this block: the expert's slots come first, padding after
     const int valid = __syncthreads_count(threadIdx.x < kTok && __ldg(a.sorted_ids + r0 + threadIdx.x) < a.n_slots);
@@ -220,18 +218,16 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
         const int dw = warp - 2, quarter = warp & 3, kq = dw >> 2;  // lane quarter, K slice
         const int t = dw * 32 + lane;                            // ring slot owner
         const int row = quarter * 32 + lane;                     // tensor-memory lane = weight row
-        // gate/up: tensor lanes 2f and 2f + 1 hold the gate and the up row of feature n0 + f, so
-        // the epilogue pairs them with one lane shuffle
-        const int grow = GU ? e * a.rows_per_expert + ((row & 1) ? a.N : 0) + n0 + (row >> 1)
+        const int grow = GU ? e * a.rows_per_expert + (row < 64 ? 0 : a.N) + n0 + (row & 63)
                             : e * a.rows_per_expert + n0 + row;
         const int32_t *wrow = a.wq + (size_t)grow * (K / 8) + kq * 4;  // 4 words = 32 inputs
-        const size_t wtile = (size_t)kTileRows * (K / 8);               // next output tile
+        const size_t wtile = (size_t)128 * (K / 8);                     // next output tile (down)
         // the group-32 scale of this thread's 32 inputs comes with its neighbour's in one aligned
         // 4-byte copy (rows are K/16 bytes apart, K a multiple of 128); group 16: its own two
         // scales, the same aligned 4 bytes
         constexpr int GS = FMT == W4_NV ? 16 : 32;
         const uint16_t *srow = a.ws + (size_t)grow * (K / GS) + (FMT == W4_NV ? 2 * kq : (kq & ~1));
-        const size_t stile = (size_t)kTileRows * (K / GS);
+        const size_t stile = (size_t)128 * (K / GS);
         auto code_slot = [&](int slot) { return code_ring + ((size_t)slot * kDeqThreads + t) * 16; };
         auto scale_slot = [&](int slot) { return scale_ring + ((size_t)slot * kDeqThreads + t) * 4; };
         // prefetch position (global step pg = tile pt, K step pk): advanced by one per issue, so the
@@ -299,34 +295,43 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
 
         // ---- epilogue of tile tt: tokens [64 kq, 64 kq + 64), chunks of 32 ----
         ok = ok && tc::mbar_wait_warp(acc_full, tt & 1, abort_flag, a.status);
-        const int nrow0 = n0 + tt * kTileRows;  // this tile's first output row (down) / feature (gate/up)
+        const int nrow0 = n0 + tt * 128;  // down: this tile's first output row
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
         // NVFP4: the accumulator carries 2^-8 / (tensor scale) of the product
         const float gsc = FMT == W4_NV ? __ldg(a.wglobal + e) * 256.f : 1.f;
         if (GU) {
-            // even lane 2f: gate of feature n0 + 16 quarter + f, the odd lane next to it its up
-            if (ok) {
-                tc::fence_after_sync();
-                const int f = nrow0 + quarter * 16 + (lane >> 1);
+            // up values (lanes 64-127) go through shared memory (the activation ring is free once
+            // every MMA has completed) to the warps holding the matching gate values (lanes 0-63)
+            float *up_s = reinterpret_cast<float *>(btiles);  // [token][feature 0..63]
+            if (ok) tc::fence_after_sync();
+            if (ok && quarter >= 2) {
+                for (int c = 0; c < kTok / kSplit / 32; ++c) {
+                    const int tok0 = kq * (kTok / kSplit) + c * 32;
+                    if (tok0 >= n_mma) break;
+                    uint32_t u[32];
+                    tc::tmem_ld32(lane_base + tok0, u);
+                    tc::tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) up_s[(tok0 + j) * 64 + (row - 64)] = gsc * __uint_as_float(u[j]);
+                }
+            }
+            asm volatile("bar.sync 1, %0;" ::"n"(kDeqThreads) : "memory");
+            if (ok && quarter < 2) {
+                const int f = n0 + row;
                 uint16_t *hcol = a.h_out + perm_pos(f);
                 for (int c = 0; c < kTok / kSplit / 32; ++c) {
                     const int tok0 = kq * (kTok / kSplit) + c * 32;
                     if (tok0 >= n_mma) break;
-                    uint32_t v[32];
-                    tc::tmem_ld32(lane_base + tok0, v);
+                    uint32_t g[32];
+                    tc::tmem_ld32(lane_base + tok0, g);
                     tc::tmem_wait_ld();
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
-                        const float mine = gsc * __uint_as_float(v[j]);
-                        const float up = __shfl_xor_sync(0xFFFFFFFFu, mine, 1);
-                        if (!(lane & 1)) hcol[(size_t)(r0 + tok0 + j) * a.N] = f32_to_bf16(silu_f32(mine) * up);
+                        const float hv = silu_f32(gsc * __uint_as_float(g[j])) * up_s[(tok0 + j) * 64 + row];
+                        hcol[(size_t)(r0 + tok0 + j) * a.N] = f32_to_bf16(hv);
                     }
                 }
             }
-            // this warp has read its accumulator lanes: the next tile's MMAs may overwrite them
-            tc::fence_before_sync();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(acc_empty);
         } else {
             if (ok) {
                 tc::fence_after_sync();
@@ -426,8 +431,8 @@ int launch_w4a16_tc(const W4TcArgs &a_in, int mode, const uint16_t *act, int max
     // down: several 128-row output tiles per CTA share one pipeline (set-up, ring fill, weight
     // prefetch across the tile boundary)
     W4TcArgs a = a_in;
-    a.tiles_per_cta = mode == TC_GATEUP ? kGateUpTilesPerCta : kDownTilesPerCta;
-    const int gx = cdiv(a.N / (mode == TC_GATEUP ? 64 : 128), a.tiles_per_cta);
+    a.tiles_per_cta = mode == TC_GATEUP ? 1 : kDownTilesPerCta;
+    const int gx = mode == TC_GATEUP ? a.N / 64 : cdiv(a.N / 128, a.tiles_per_cta);
     if (a.fmt == W4_FP4) {
         if (mode == TC_GATEUP) return launch_mode<TC_GATEUP, W4_FP4>(a, tm, gx, max_blocks, s);
         return launch_mode<TC_DOWN, W4_FP4>(a, tm, gx, max_blocks, s);
