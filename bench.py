@@ -13,7 +13,9 @@ layer (T=4096, E=256) and the dense block-FP8 matmul sweep as secondary measurem
 --impl reference times the CPU oracle (oracle/, the one other consumer allowed here) on a bounded
 sample of the same workload, on the host cores. Multi-GPU (--gpus N under torchrun): independent
 replicas, one per rank, no collective on the data path ("replicas only"); value is the sum over
-ranks of bytes / the slowest rank's time.
+ranks of bytes / the slowest rank's time. --parallel ep|tp instead splits the one decode layer
+over the ranks (expert- or tensor-parallel shares, then an all-reduce of the output over NCCL);
+value is then the layer's weight bytes / the slowest rank's time (strong scaling).
 """
 from __future__ import annotations
 
@@ -429,6 +431,56 @@ def reference_arm(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def parallel_arm(args, moeq, rank, world, peaks, peak_src, flush):
+    """The decode W4A16 layer split over the ranks: expert-parallel (rank r holds experts
+    [r E/N, (r+1) E/N)) or tensor-parallel (rank r holds intermediate features [r I/N, (r+1) I/N) of
+    every expert). One step = this rank's share through the C ABI + the all-reduce (sum) of the
+    [T, H] bf16 output over the process group. The job's time is the slowest rank's."""
+    from quantized_mixture_experts_align_b200 import sharding as S
+    d = W.make_moe(W.WORKLOADS["decode_w4a16"], device="cuda", E=args.experts)
+    n_active = touched_experts(moeq, d)
+    step_bytes = n_active * W.w4a16_expert_bytes(d["H"], d["I"])  # every touched expert read once, job-wide
+    full = {n: d.pop(n) for n in ("w13q", "w13s", "w2q", "w2s")}
+    out = torch.empty((d["T"], d["H"]), dtype=torch.bfloat16, device="cuda")
+    if args.parallel == "ep":
+        w, base, local = S.shard_experts(full, "w4a16", rank, world)
+        ws = moeq.workspace(moeq.moe_w4a16_ep_workspace_size(d["T"], d["H"], d["I"], d["E"], d["k"], local), "cuda")
+        fn = lambda: S.forward_ep("w4a16", d["x"], d["logits"], d["k"], w, base, out=out, ws=ws)
+        shape = f"experts [{base}, {base + local}) of {d['E']} on rank {rank}"
+    else:
+        w = S.shard_intermediate(full, "w4a16", d["I"], rank, world)
+        ws = moeq.workspace(moeq.moe_w4a16_workspace_size(d["T"], d["H"], d["I"] // world, d["E"], d["k"]), "cuda")
+        fn = lambda: S.forward_tp("w4a16", d["x"], d["logits"], d["k"], w, out=out, ws=ws)
+        shape = f"features [{rank * d['I'] // world}, {(rank + 1) * d['I'] // world}) of {d['I']} on rank {rank}"
+    del full
+    torch.cuda.empty_cache()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        ms = timed_steps(fn, args.steps, args.warmup, flush, world)
+    ms_step = max_over_ranks(statistics.mean(ms), world)
+    value = step_bytes / (ms_step * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"decode_w4a16 T=32 H=7168 I=2048 E={d['E']} k=8 (INT4 group-32, bf16 scales)",
+                   "parallelism": f"{args.parallel}{world}", "rank0_share": shape,
+                   "touched_experts": n_active, "weight_bytes_per_step": step_bytes,
+                   "l2": f"flushed between steps ({L2_FLUSH_BYTES >> 20} MB written then read), outside the events",
+                   "collective": "all-reduce (sum) of the bf16 [T, H] output, NCCL" if world > 1 else "none (one rank)"},
+        "roofline": {"bound": "hbm", "achieved": value / world, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": value / world / peaks["hbm_gbs"], "traffic": None,
+                     "note": "whole step per GPU (share + all-reduce), not one kernel; the kernel roofline is on the "
+                             "default (replicas) line", "peak_source": f"{peak_src} hbm_gbs (copy)"},
+        "e2e": None,
+        "gpu_launches": 5 * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
 def only_arm(args, moeq, rank, world):
     """One workload alone, for profiler captures of a small case; prints a JSON line of timings."""
     name = args.only
@@ -475,6 +527,9 @@ def main():
     ap.add_argument("--experts", type=int, default=None,
                     help="override E of the workload (small cases for profiler captures)")
     ap.add_argument("--tokens", type=int, default=None, help="override T of the workload (with --only)")
+    ap.add_argument("--parallel", choices=["replicas", "ep", "tp"], default="replicas",
+                    help="replicas: one independent layer per rank (default); ep / tp: the decode layer split "
+                         "over the ranks (expert- / tensor-parallel shares + an all-reduce)")
     ap.add_argument("--only", choices=["prefill_w4a16", "moe_fp8", "dense_fp8", "dense_fp8_channel"], default=None,
                     help="time one secondary workload alone (small cases for profiler captures)")
     args = ap.parse_args()
@@ -504,6 +559,10 @@ def main():
         # would land inside the next timed step: ~9 us on a 176 MB weight stream)
         flush_buf.fill_(1)
         flush_words.max()
+
+    if args.parallel != "replicas":
+        parallel_arm(args, moeq, rank, world, peaks, peak_src, flush)
+        return
 
     # ---- headline: decode W4A16 -----------------------------------------------------------
     d = W.make_moe(W.WORKLOADS["decode_w4a16"], device="cuda", E=args.experts)

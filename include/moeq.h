@@ -162,6 +162,44 @@ MOEQ_API int moe_nvfp4_forward(const uint16_t *x, const float *logits, int T, in
                                float *topk_w_out, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * Expert-parallel forms of the layers ([CHORD], "Other deployment details" and the measured
+ * results: EP8, EP16 and EP32 deployments, where each GPU holds E / N of the experts). One call
+ * computes one rank's share of the layer:
+ *   out_r[t] = sum over the slots j of token t whose expert e_j lies in [ep_base, ep_base + ep_local)
+ *              of topk_w[t, j] * y_j           (y_j as in the single-GPU layer)
+ * so the layer's output is the sum of out_r over ranks whose ranges tile [0, E); the caller sums
+ * them (an all-reduce across GPUs). Routing still picks the top k of all E logits. Tokens with no
+ * slot on this rank get a zero row.
+ *   E          experts the routing picks from (logits are [T, E])
+ *   ep_base    first expert this call holds, ep_local how many (ep_local >= 1,
+ *              ep_base + ep_local <= E; else INVALID_ARG)
+ *   weights    only this rank's experts: w13 [ep_local, ...], w2 [ep_local, ...] (and w13_g / w2_g
+ *              [ep_local] for NVFP4), in the formats of the single-GPU entry points
+ *   topk_ids_out (nullable) receives the global expert ids
+ *   ws         moe_w4a16_ep_workspace_size (the three 4-bit formats) or
+ *              moe_w8a8_block_fp8_ep_workspace_size bytes
+ * The schedule follows the mean load of one expert, T * k / E, as on a single GPU.
+ * Tensor parallelism needs no entry point of its own: a rank that holds the intermediate features
+ * [r * I / N, (r + 1) * I / N) of every expert (those gate rows, those up rows, those down columns
+ * and their scales; I / N a multiple of 128) calls the single-GPU forward with I / N, and the
+ * ranks' outputs sum to the layer's.
+ */
+MOEQ_API size_t moe_w4a16_ep_workspace_size(int T, int H, int I, int E, int k, int ep_local);
+MOEQ_API int moe_w4a16_forward_ep(const uint16_t *x, const float *logits, int T, int H, int I, int E, int k,
+                                  int ep_base, int ep_local, const int32_t *w13_q, const uint16_t *w13_s,
+                                  const int32_t *w2_q, const uint16_t *w2_s, uint16_t *out, int32_t *topk_ids_out,
+                                  float *topk_w_out, void *ws, size_t ws_bytes, void *stream);
+MOEQ_API int moe_mxfp4_forward_ep(const uint16_t *x, const float *logits, int T, int H, int I, int E, int k,
+                                  int ep_base, int ep_local, const int32_t *w13_q, const uint16_t *w13_f,
+                                  const int32_t *w2_q, const uint16_t *w2_f, uint16_t *out, int32_t *topk_ids_out,
+                                  float *topk_w_out, void *ws, size_t ws_bytes, void *stream);
+MOEQ_API int moe_nvfp4_forward_ep(const uint16_t *x, const float *logits, int T, int H, int I, int E, int k,
+                                  int ep_base, int ep_local, const int32_t *w13_q, const uint16_t *w13_f,
+                                  const float *w13_g, const int32_t *w2_q, const uint16_t *w2_f, const float *w2_g,
+                                  uint16_t *out, int32_t *topk_ids_out, float *topk_w_out, void *ws,
+                                  size_t ws_bytes, void *stream);
+
+/*
  * Scratch-free W4A16 layer forward. The pages have no counterpart of this entry point: it exists
  * for callers that cannot allocate device memory where they run the layer, such as a plugin or
  * custom-op host that only hands over its input and output buffers, or a serving runtime that
@@ -202,6 +240,15 @@ MOEQ_API int moe_w8a8_block_fp8_forward(const uint16_t *x, const float *logits, 
                                int k, const uint8_t *w13, const float *w13_s, const uint8_t *w2,
                                const float *w2_s, uint16_t *out, int32_t *topk_ids_out,
                                float *topk_w_out, void *ws, size_t ws_bytes, void *stream);
+/* Expert-parallel form of the block-FP8 layer: as moe_w4a16_forward_ep above, with the weights
+ * w13 [ep_local, 2I, H], w13_s [ep_local, 2I/128, H/128], w2 [ep_local, H, I],
+ * w2_s [ep_local, H/128, I/128]. */
+MOEQ_API size_t moe_w8a8_block_fp8_ep_workspace_size(int T, int H, int I, int E, int k, int ep_local);
+MOEQ_API int moe_w8a8_block_fp8_forward_ep(const uint16_t *x, const float *logits, int T, int H, int I, int E,
+                                           int k, int ep_base, int ep_local, const uint8_t *w13,
+                                           const float *w13_s, const uint8_t *w2, const float *w2_s,
+                                           uint16_t *out, int32_t *topk_ids_out, float *topk_w_out, void *ws,
+                                           size_t ws_bytes, void *stream);
 
 /*
  * Grouped W4A16 GEMM on the layer's kernels, for callers that route themselves ([CHORD], "SM90

@@ -161,6 +161,54 @@ def moe_fp8(x, logits, k, w13, w13s, w2, w2s, tokens=None, want_h=False):
     return (out, hq, hs) if want_h else out
 
 
+_Q4_FORMATS = {"w4a16": (0, np.uint16), "mxfp4": (1, np.uint8), "nvfp4": (2, np.uint8)}
+
+
+def moe_q4_ep(fmt, x, logits, k, ep_base, w13q, w13s, w2q, w2s, g13=None, g2=None, tokens=None):
+    """One expert-parallel rank's share of the 4-bit layer (float64 [len(tokens), H]): the slots
+    whose expert lies in [ep_base, ep_base + ep_local), ep_local = len(w13q), the weights given
+    being those experts'. fmt "w4a16" (bf16 scale bits), "mxfp4" (UE8M0 bytes) or "nvfp4" (E4M3
+    bytes, with the tensor scales g13 / g2 [ep_local])."""
+    code, sdt = _Q4_FORMATS[fmt]
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    logits = np.ascontiguousarray(logits, dtype=np.float32)
+    T, H = x.shape
+    E = logits.shape[1]
+    I = w2q.shape[2] * 8
+    ep_local = w13q.shape[0]
+    tok = _tokens(tokens, T)
+    out = np.zeros((len(tok), H), np.float64)
+    q13, q2 = np.ascontiguousarray(w13q, dtype=np.int32), np.ascontiguousarray(w2q, dtype=np.int32)
+    s13, s2 = np.ascontiguousarray(w13s), np.ascontiguousarray(w2s)
+    assert s13.dtype == sdt and s2.dtype == sdt
+    gp = [None, None]
+    if code == 2:
+        g13 = np.ascontiguousarray(g13, dtype=np.float32).reshape(ep_local)
+        g2 = np.ascontiguousarray(g2, dtype=np.float32).reshape(ep_local)
+        gp = [_p(g13), _p(g2)]
+    rc = lib().orc_moe_q4_ep(code, _p(x), _p(logits), T, H, I, E, k, int(ep_base), ep_local, _p(q13), _p(s13), gp[0],
+                             _p(q2), _p(s2), gp[1], _p(tok), len(tok), _p(out))
+    _check(rc, "moe_q4_ep")
+    return out
+
+
+def moe_fp8_ep(x, logits, k, ep_base, w13, w13s, w2, w2s, tokens=None):
+    """One expert-parallel rank's share of the block-FP8 layer (float64 [len(tokens), H]), the
+    weights given being those of experts [ep_base, ep_base + len(w13))."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    logits = np.ascontiguousarray(logits, dtype=np.float32)
+    T, H = x.shape
+    E = logits.shape[1]
+    I = w2.shape[2]
+    tok = _tokens(tokens, T)
+    out = np.zeros((len(tok), H), np.float64)
+    args = [np.ascontiguousarray(a) for a in (w13, w13s, w2, w2s)]
+    rc = lib().orc_moe_fp8_ep(_p(x), _p(logits), T, H, I, E, k, int(ep_base), args[0].shape[0],
+                              *[_p(a) for a in args], _p(tok), len(tok), _p(out))
+    _check(rc, "moe_fp8_ep")
+    return out
+
+
 def fp8_block_matmul(A, As, B, Bs, rows=None):
     """C rows (float64 [len(rows), N]) of the dense block-FP8 product."""
     A = np.ascontiguousarray(A, dtype=np.uint8)

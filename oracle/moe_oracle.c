@@ -291,15 +291,20 @@ static double silu(double g) { return g / (1.0 + exp(-g)); }
  *     h_n = bf16( silu(g_n) * u_n )     (the A16 intermediate: activations are BF16)
  *     y_m = sum_n h_n * W2[e][m, n]
  *   out = sum over the k selected experts of w * y     (the top-k weighted combine).
- * h_out (nullable, bf16 bits [ntok, k, I]) returns the intermediate of each slot. */
+ * h_out (nullable, bf16 bits [ntok, k, I]) returns the intermediate of each slot.
+ * Expert parallelism ([CHORD] "Other deployment details": EP8 / EP16 / EP32, each GPU holding a
+ * share of the experts): with the weights of experts [ep_base, ep_base + ep_local) only, the sum
+ * above runs over the slots whose expert lies in that range (the routing still ranks all E);
+ * ep_base = 0, ep_local = E is the whole layer. Slots outside the range leave h_out untouched. */
 static int moe_q4_layer(int fmt, const uint16_t *x, const float *logits, int T, int H, int I, int E, int k,
                         const int32_t *w13q, const void *w13s, const int32_t *w2q, const void *w2s,
                         const float *g13, const float *g2, const int32_t *tokens, int ntok, double *out,
-                        uint16_t *h_out)
+                        uint16_t *h_out, int ep_base, int ep_local)
 {
     const size_t sb = fmt ? 1 : 2;        /* bytes per scale */
     const int gsz = fmt == 2 ? 16 : 32;   /* inputs per scale */
     if (H % 32 || I % 32 || H < 32 || I < 32 || k < 1 || k > E) return 1;
+    if (ep_base < 0 || ep_local < 1 || ep_base + ep_local > E) return 1;
     for (int i = 0; i < ntok; ++i)
         if (tokens[i] < 0 || tokens[i] >= T) return 1;
     int32_t *ids = (int32_t *)malloc(sizeof(int32_t) * (size_t)k);
@@ -314,7 +319,8 @@ static int moe_q4_layer(int fmt, const uint16_t *x, const float *logits, int T, 
         double *o = out + (size_t)i * H;
         for (int m = 0; m < H; ++m) o[m] = 0.0;
         for (int j = 0; j < k; ++j) {
-            int e = ids[j];
+            int e = ids[j] - ep_base;            /* index among the weights held */
+            if (e < 0 || e >= ep_local) continue;
             const int32_t *q13 = w13q + (size_t)e * 2 * I * (H / 8);
             const void *s13 = (const char *)w13s + (size_t)e * 2 * I * (H / gsz) * sb;
             const int32_t *q2 = w2q + (size_t)e * H * (I / 8);
@@ -350,7 +356,19 @@ int orc_moe_w4a16(const uint16_t *x, const float *logits, int T, int H, int I, i
                   const int32_t *w13q, const uint16_t *w13s, const int32_t *w2q, const uint16_t *w2s,
                   const int32_t *tokens, int ntok, double *out, uint16_t *h_out)
 {
-    return moe_q4_layer(0, x, logits, T, H, I, E, k, w13q, w13s, w2q, w2s, NULL, NULL, tokens, ntok, out, h_out);
+    return moe_q4_layer(0, x, logits, T, H, I, E, k, w13q, w13s, w2q, w2s, NULL, NULL, tokens, ntok, out, h_out, 0, E);
+}
+
+/* One expert-parallel rank's share of the 4-bit layer (fmt 0 INT4, 1 MXFP4, 2 NVFP4; scales as the
+ * single-format functions take them, g13 / g2 NULL except for NVFP4), weights of experts
+ * [ep_base, ep_base + ep_local) only. */
+int orc_moe_q4_ep(int fmt, const uint16_t *x, const float *logits, int T, int H, int I, int E, int k, int ep_base,
+                  int ep_local, const int32_t *w13q, const void *w13s, const float *g13, const int32_t *w2q,
+                  const void *w2s, const float *g2, const int32_t *tokens, int ntok, double *out)
+{
+    if (fmt < 0 || fmt > 2 || (fmt == 2 && (!g13 || !g2))) return 1;
+    return moe_q4_layer(fmt, x, logits, T, H, I, E, k, w13q, w13s, w2q, w2s, fmt == 2 ? g13 : NULL,
+                        fmt == 2 ? g2 : NULL, tokens, ntok, out, NULL, ep_base, ep_local);
 }
 
 /* The same layer with MXFP4 weights (E2M1 codes, UE8M0 group-32 scales [rows, K/32] bytes); the
@@ -359,7 +377,7 @@ int orc_moe_mxfp4(const uint16_t *x, const float *logits, int T, int H, int I, i
                   const int32_t *w13q, const uint8_t *w13s, const int32_t *w2q, const uint8_t *w2s,
                   const int32_t *tokens, int ntok, double *out, uint16_t *h_out)
 {
-    return moe_q4_layer(1, x, logits, T, H, I, E, k, w13q, w13s, w2q, w2s, NULL, NULL, tokens, ntok, out, h_out);
+    return moe_q4_layer(1, x, logits, T, H, I, E, k, w13q, w13s, w2q, w2s, NULL, NULL, tokens, ntok, out, h_out, 0, E);
 }
 
 /* The same layer with NVFP4 weights: E2M1 codes, E4M3 group-16 scales [rows, K/16] bytes and one
@@ -371,7 +389,7 @@ int orc_moe_nvfp4(const uint16_t *x, const float *logits, int T, int H, int I, i
                   uint16_t *h_out)
 {
     if (H % 32 || I % 32) return 1;
-    return moe_q4_layer(2, x, logits, T, H, I, E, k, w13q, w13s, w2q, w2s, g13, g2, tokens, ntok, out, h_out);
+    return moe_q4_layer(2, x, logits, T, H, I, E, k, w13q, w13s, w2q, w2s, g13, g2, tokens, ntok, out, h_out, 0, E);
 }
 
 /* ------------------------------------------------------------------------------------------ */
@@ -410,12 +428,15 @@ static double fp8_row_dot(const uint8_t *a, const float *as, const uint8_t *b, c
  * and the intermediate a = silu(g)*u is rounded to f32 and quantized the same way before the
  * down projection. READING: the intermediate quantizer sees the f32 value of a, as the input
  * quantizer sees the f32 value of the bf16 input.
- * hq_out/hs_out (nullable) return the quantized intermediate [ntok, k, I] / [ntok, k, I/128]. */
-int orc_moe_fp8(const uint16_t *x, const float *logits, int T, int H, int I, int E, int k,
-                const uint8_t *w13, const float *w13s, const uint8_t *w2, const float *w2s,
-                const int32_t *tokens, int ntok, double *out, uint8_t *hq_out, float *hs_out)
+ * hq_out/hs_out (nullable) return the quantized intermediate [ntok, k, I] / [ntok, k, I/128].
+ * ep_base / ep_local: the expert range whose weights are given, as in moe_q4_layer. */
+static int moe_fp8_layer(const uint16_t *x, const float *logits, int T, int H, int I, int E, int k,
+                         const uint8_t *w13, const float *w13s, const uint8_t *w2, const float *w2s,
+                         const int32_t *tokens, int ntok, double *out, uint8_t *hq_out, float *hs_out,
+                         int ep_base, int ep_local)
 {
     if (H % 128 || I % 128 || H < 128 || I < 128 || k < 1 || k > E) return 1;
+    if (ep_base < 0 || ep_local < 1 || ep_base + ep_local > E) return 1;
     for (int i = 0; i < ntok; ++i)
         if (tokens[i] < 0 || tokens[i] >= T) return 1;
     e4m3_table_init();
@@ -434,7 +455,8 @@ int orc_moe_fp8(const uint16_t *x, const float *logits, int T, int H, int I, int
         double *o = out + (size_t)i * H;
         for (int m = 0; m < H; ++m) o[m] = 0.0;
         for (int j = 0; j < k; ++j) {
-            int e = ids[j];
+            int e = ids[j] - ep_base;            /* index among the weights held */
+            if (e < 0 || e >= ep_local) continue;
             const uint8_t *W13 = w13 + (size_t)e * 2 * I * H;
             const float *S13 = w13s + (size_t)e * (2 * I / 128) * (H / 128);
             const uint8_t *W2 = w2 + (size_t)e * H * I;
@@ -457,6 +479,22 @@ int orc_moe_fp8(const uint16_t *x, const float *logits, int T, int H, int I, int
     }
     free(ids); free(w); free(xq); free(xs); free(a); free(hq); free(hs);
     return 0;
+}
+
+int orc_moe_fp8(const uint16_t *x, const float *logits, int T, int H, int I, int E, int k,
+                const uint8_t *w13, const float *w13s, const uint8_t *w2, const float *w2s,
+                const int32_t *tokens, int ntok, double *out, uint8_t *hq_out, float *hs_out)
+{
+    return moe_fp8_layer(x, logits, T, H, I, E, k, w13, w13s, w2, w2s, tokens, ntok, out, hq_out, hs_out, 0, E);
+}
+
+/* One expert-parallel rank's share of the block-FP8 layer (weights of [ep_base, ep_base + ep_local)). */
+int orc_moe_fp8_ep(const uint16_t *x, const float *logits, int T, int H, int I, int E, int k, int ep_base,
+                   int ep_local, const uint8_t *w13, const float *w13s, const uint8_t *w2, const float *w2s,
+                   const int32_t *tokens, int ntok, double *out)
+{
+    return moe_fp8_layer(x, logits, T, H, I, E, k, w13, w13s, w2, w2s, tokens, ntok, out, NULL, NULL, ep_base,
+                         ep_local);
 }
 
 /* ------------------------------------------------------------------------------------------ */

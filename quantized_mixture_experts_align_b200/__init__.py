@@ -44,6 +44,12 @@ _SIGNATURES = {
     "moe_mxfp4_forward": ([_V, _V, _I, _I, _I, _I, _I, _V, _V, _V, _V, _V, _V, _V, _V, _Z, _V], _I),
     "moe_w8a8_block_fp8_workspace_size": ([_I, _I, _I, _I, _I], _Z),
     "moe_w8a8_block_fp8_forward": ([_V, _V, _I, _I, _I, _I, _I, _V, _V, _V, _V, _V, _V, _V, _V, _Z, _V], _I),
+    "moe_w4a16_ep_workspace_size": ([_I, _I, _I, _I, _I, _I], _Z),
+    "moe_w4a16_forward_ep": ([_V, _V] + [_I] * 7 + [_V] * 8 + [_Z, _V], _I),
+    "moe_mxfp4_forward_ep": ([_V, _V] + [_I] * 7 + [_V] * 8 + [_Z, _V], _I),
+    "moe_nvfp4_forward_ep": ([_V, _V] + [_I] * 7 + [_V] * 10 + [_Z, _V], _I),
+    "moe_w8a8_block_fp8_ep_workspace_size": ([_I, _I, _I, _I, _I, _I], _Z),
+    "moe_w8a8_block_fp8_forward_ep": ([_V, _V] + [_I] * 7 + [_V] * 8 + [_Z, _V], _I),
     "w8a8_block_fp8_matmul": ([_V, _V, _V, _V, _I, _I, _I, _I, _I, _V, _V], _I),
     "w8a8_channel_fp8_matmul": ([_V, _V, _V, _V, _I, _I, _I, _V, _V], _I),
     "moe_w4a16_grouped_contiguous_workspace_size": ([_I, _I, _I, _I], _Z),
@@ -264,6 +270,68 @@ def moe_w8a8_block_fp8_forward(x, logits, k, w13, w13_s, w2, w2_s, out=None, ws=
         _dev(topk_w_out, "topk_w_out", torch.float32), _dev(ws, "ws"), ws.numel() * ws.element_size(),
         _stream(stream)))
     return out
+
+
+def moe_w4a16_ep_workspace_size(T: int, H: int, I: int, E: int, k: int, ep_local: int) -> int:
+    return int(lib().moe_w4a16_ep_workspace_size(T, H, I, E, k, ep_local))
+
+
+def moe_w8a8_block_fp8_ep_workspace_size(T: int, H: int, I: int, E: int, k: int, ep_local: int) -> int:
+    return int(lib().moe_w8a8_block_fp8_ep_workspace_size(T, H, I, E, k, ep_local))
+
+
+def _ep_call(name, x, logits, k, ep_base, weights, out, ws, topk_ids_out, topk_w_out, stream, I, ws_fn):
+    """Shared marshalling of the *_forward_ep entry points: weights = [(tensor, name, dtype), ...] of
+    ep_local experts, in the entry point's order."""
+    T, H = x.shape
+    E = logits.shape[1]
+    ep_local = weights[0][0].shape[0]
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device) if out is None else out
+    ws = workspace(ws_fn(T, H, I, E, k, ep_local), x.device) if ws is None else ws
+    _check(getattr(lib(), name)(
+        _dev(x, "x", _BF16), _dev(logits, "logits", torch.float32), T, H, I, E, k, int(ep_base), ep_local,
+        *[_dev(t, n, dt) for t, n, dt in weights], _dev(out, "out", _BF16),
+        _dev(topk_ids_out, "topk_ids_out", torch.int32), _dev(topk_w_out, "topk_w_out", torch.float32),
+        _dev(ws, "ws"), ws.numel() * ws.element_size(), _stream(stream)))
+    return out
+
+
+def moe_w4a16_forward_ep(x, logits, k, ep_base, w13_q, w13_s, w2_q, w2_s, out=None, ws=None, topk_ids_out=None,
+                         topk_w_out=None, stream=None):
+    """One expert-parallel rank's share of the W4A16 layer: the weights of experts
+    [ep_base, ep_base + len(w13_q)) only; the ranks' outputs sum to the layer's."""
+    return _ep_call("moe_w4a16_forward_ep", x, logits, k, ep_base,
+                    [(w13_q, "w13_q", torch.int32), (w13_s, "w13_s", _BF16), (w2_q, "w2_q", torch.int32),
+                     (w2_s, "w2_s", _BF16)], out, ws, topk_ids_out, topk_w_out, stream, w2_q.shape[2] * 8,
+                    moe_w4a16_ep_workspace_size)
+
+
+def moe_mxfp4_forward_ep(x, logits, k, ep_base, w13_q, w13_f, w2_q, w2_f, out=None, ws=None, topk_ids_out=None,
+                         topk_w_out=None, stream=None):
+    """One expert-parallel rank's share of the MXFP4 layer (prepacked factors)."""
+    return _ep_call("moe_mxfp4_forward_ep", x, logits, k, ep_base,
+                    [(w13_q, "w13_q", torch.int32), (w13_f, "w13_f", _BF16), (w2_q, "w2_q", torch.int32),
+                     (w2_f, "w2_f", _BF16)], out, ws, topk_ids_out, topk_w_out, stream, w2_q.shape[2] * 8,
+                    moe_w4a16_ep_workspace_size)
+
+
+def moe_nvfp4_forward_ep(x, logits, k, ep_base, w13_q, w13_f, w13_g, w2_q, w2_f, w2_g, out=None, ws=None,
+                         topk_ids_out=None, topk_w_out=None, stream=None):
+    """One expert-parallel rank's share of the NVFP4 layer (prepacked factors, tensor scales of the
+    rank's experts)."""
+    return _ep_call("moe_nvfp4_forward_ep", x, logits, k, ep_base,
+                    [(w13_q, "w13_q", torch.int32), (w13_f, "w13_f", _BF16), (w13_g, "w13_g", torch.float32),
+                     (w2_q, "w2_q", torch.int32), (w2_f, "w2_f", _BF16), (w2_g, "w2_g", torch.float32)],
+                    out, ws, topk_ids_out, topk_w_out, stream, w2_q.shape[2] * 8, moe_w4a16_ep_workspace_size)
+
+
+def moe_w8a8_block_fp8_forward_ep(x, logits, k, ep_base, w13, w13_s, w2, w2_s, out=None, ws=None, topk_ids_out=None,
+                                  topk_w_out=None, stream=None):
+    """One expert-parallel rank's share of the block-FP8 layer."""
+    return _ep_call("moe_w8a8_block_fp8_forward_ep", x, logits, k, ep_base,
+                    [(w13, "w13", _U8), (w13_s, "w13_s", torch.float32), (w2, "w2", _U8),
+                     (w2_s, "w2_s", torch.float32)], out, ws, topk_ids_out, topk_w_out, stream, w2.shape[2],
+                    moe_w8a8_block_fp8_ep_workspace_size)
 
 
 def w8a8_block_fp8_matmul(A, As, B, Bs, block_size=(128, 128), out=None, stream=None):

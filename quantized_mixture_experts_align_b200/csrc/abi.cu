@@ -184,11 +184,15 @@ static bool w4_use_tc(long T, int k, int E) { return (double)T * k / (double)E >
 constexpr int kW4SmallRows = 8;
 static_assert(kW4SmallRows == 8, "the strided register-fed instantiation is built for 8-row tiles");
 
+// E: experts whose weights the call holds (the alignment's capacity); E_sched (0: E): experts the
+// routing picks from, whose mean load T*k/E_sched picks the schedule (under expert parallelism a
+// rank holds E of the E_sched experts, and each of them still sees T*k/E_sched rows on average).
 static size_t w4a16_layout(Carve &c, long T, int H, int I, int E, int k, RouteBufs *rb, uint16_t **h, uint16_t **ys,
-                           uint16_t **xg = nullptr, uint16_t **h_small = nullptr)
+                           uint16_t **xg = nullptr, uint16_t **h_small = nullptr, int E_sched = 0)
 {
-    const bool tcp = w4_use_tc(T, k, E);
-    RouteBufs r = carve_route(c, T, k, E, tcp ? 256 : pick_block_m(T, k, E));  // tensor-core tiles: 256 rows
+    const int Es = E_sched > 0 ? E_sched : E;
+    const bool tcp = w4_use_tc(T, k, Es);
+    RouteBufs r = carve_route(c, T, k, E, tcp ? 256 : pick_block_m(T, k, Es));  // tensor-core tiles: 256 rows
     const size_t cap = (size_t)r.max_blocks * r.block_m;
     uint16_t *hp = c.take<uint16_t>((tcp ? cap : (size_t)T * k) * I);
     uint16_t *yp = c.take<uint16_t>((size_t)T * k * H);  // weighted slot rows (bf16) for the combine
@@ -208,11 +212,14 @@ static size_t w4a16_layout(Carve &c, long T, int H, int I, int E, int k, RouteBu
 // kernel streams the weights for the few rows each expert has.
 static bool fp8_use_tc(long T, int k, int E) { return (double)T * k / (double)E >= 16.0; }
 
+// E, E_sched: as w4a16_layout.
 static size_t fp8_layout(Carve &c, long T, int H, int I, int E, int k, RouteBufs *rb, uint8_t **xq, float **xs,
-                         uint8_t **hq, float **hs, uint16_t **ys, uint8_t **xg = nullptr, float **xsg = nullptr)
+                         uint8_t **hq, float **hs, uint16_t **ys, uint8_t **xg = nullptr, float **xsg = nullptr,
+                         int E_sched = 0)
 {
-    const bool tcp = fp8_use_tc(T, k, E);
-    RouteBufs r = carve_route(c, T, k, E, tcp ? 128 : pick_block_m(T, k, E));
+    const int Es = E_sched > 0 ? E_sched : E;
+    const bool tcp = fp8_use_tc(T, k, Es);
+    RouteBufs r = carve_route(c, T, k, E, tcp ? 128 : pick_block_m(T, k, Es));
     const size_t cap = (size_t)T * k + (size_t)E * (r.block_m - 1);   // aligned rows
     const size_t hrows = tcp ? cap : (size_t)T * k;                     // h rows: aligned or by slot
     uint8_t *xqp = c.take<uint8_t>((size_t)T * H);
@@ -251,6 +258,17 @@ static int check_layer_shape(long T, int H, int I, int E, int k)
     if (rc) return rc;
     if (H < 128 || H % 128) return set_error(MOEQ_ERR_UNSUPPORTED, "H must be a positive multiple of 128 (got %d)", H);
     if (I < 128 || I % 128) return set_error(MOEQ_ERR_UNSUPPORTED, "I must be a positive multiple of 128 (got %d)", I);
+    return MOEQ_OK;
+}
+
+// Expert parallelism: the call holds experts [ep_base, ep_base + ep_local) of the E the routing
+// picks from.
+static int check_expert_range(int E, int ep_base, int ep_local)
+{
+    if (ep_local < 1 || ep_base < 0 || ep_base > E - ep_local)
+        return set_error(MOEQ_ERR_INVALID_ARG,
+                         "expert range [ep_base, ep_base + ep_local) = [%d, %d) must be non-empty and lie in [0, E = %d)",
+                         ep_base, ep_base + ep_local, E);
     return MOEQ_OK;
 }
 
@@ -329,6 +347,13 @@ size_t moe_w4a16_workspace_size(int T, int H, int I, int E, int k)
     return w4a16_layout(c, T, H, I, E, k, nullptr, nullptr, nullptr);
 }
 
+size_t moe_w4a16_ep_workspace_size(int T, int H, int I, int E, int k, int ep_local)
+{
+    if (check_layer_shape(T, H, I, E, k) || check_expert_range(E, 0, ep_local)) return 0;
+    Carve c(nullptr);
+    return w4a16_layout(c, T, H, I, ep_local, k, nullptr, nullptr, nullptr, nullptr, nullptr, E);
+}
+
 }  // extern "C"
 
 namespace moeq {
@@ -338,11 +363,15 @@ namespace moeq {
 static int w4_layer_forward(int fmt, const char *name, const uint16_t *x, const float *logits, int T, int H, int I,
                             int E, int k, const int32_t *w13_q, const uint16_t *w13_s, const int32_t *w2_q,
                             const uint16_t *w2_s, uint16_t *out, int32_t *topk_ids_out, float *topk_w_out, void *ws,
-                            size_t ws_bytes, void *stream, const float *g13 = nullptr, const float *g2 = nullptr)
+                            size_t ws_bytes, void *stream, const float *g13 = nullptr, const float *g2 = nullptr,
+                            int ep_base = 0, int ep_local = 0)
 {
     g_err[0] = 0;
     int rc = check_layer_shape(T, H, I, E, k);
     if (rc) return rc;
+    const bool ep = ep_local > 0 || ep_base != 0;  // expert parallelism: weights of ep_local experts
+    if (ep && (rc = check_expert_range(E, ep_base, ep_local))) return rc;
+    const int Ew = ep ? ep_local : E;  // experts whose weights this call holds
     if (T == 0) return MOEQ_OK;
     MOEQ_REQUIRE(x);
     MOEQ_REQUIRE(logits);
@@ -353,7 +382,7 @@ static int w4_layer_forward(int fmt, const char *name, const uint16_t *x, const 
     MOEQ_REQUIRE(out);
     MOEQ_REQUIRE(ws);
     if (reinterpret_cast<uintptr_t>(ws) & 255) return set_error(MOEQ_ERR_INVALID_ARG, "ws must be 256-byte aligned");
-    const size_t need = moe_w4a16_workspace_size(T, H, I, E, k);
+    const size_t need = ep ? moe_w4a16_ep_workspace_size(T, H, I, E, k, ep_local) : moe_w4a16_workspace_size(T, H, I, E, k);
     if (ws_bytes < need) return set_error(MOEQ_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, need);
 
     cudaStream_t s = (cudaStream_t)stream;
@@ -361,19 +390,22 @@ static int w4_layer_forward(int fmt, const char *name, const uint16_t *x, const 
     RouteBufs r;
     uint16_t *h, *xg, *h_small;
     uint16_t *ys;
-    w4a16_layout(c, T, H, I, E, k, &r, &h, &ys, &xg, &h_small);
-    int32_t *ids = topk_ids_out ? topk_ids_out : r.ids;
+    w4a16_layout(c, T, H, I, Ew, k, &r, &h, &ys, &xg, &h_small, E);
+    // global picks to the caller's buffer (if any); under expert parallelism the alignment and the
+    // combine take the local ids (-1 for experts held elsewhere) in the route scratch
+    int32_t *ids = topk_ids_out ? topk_ids_out : (ep ? nullptr : r.ids);
+    int32_t *lids = ep ? r.ids : nullptr;
     float *tw = topk_w_out ? topk_w_out : r.w;
     const int n = T * k;
     const bool tcp = w4_use_tc(T, k, E);
 
     {
         trace::Scope ts(trace::ROUTE, s);
-        launch_route_topk(logits, T, E, k, ids, tw, s);
+        launch_route_topk(logits, T, E, k, ids, tw, s, lids, ep_base, ep_local);
     }
     {
         trace::Scope ts(trace::ALIGN, s);
-        launch_align(ids, n, E, r.block_m, r.sorted, r.eids, r.ntp, r.scratch, s);
+        launch_align(ep ? lids : ids, n, Ew, r.block_m, r.sorted, r.eids, r.ntp, r.scratch, s);
     }
 
     if (tcp) {
@@ -387,7 +419,7 @@ static int w4_layer_forward(int fmt, const char *name, const uint16_t *x, const 
         W4TcArgs t{};
         t.fmt = fmt;
         t.status = status;
-        t.E = E;
+        t.E = Ew;
         t.sorted_ids = r.sorted;
         t.expert_ids = r.eids;
         t.ntp = r.ntp;
@@ -405,7 +437,7 @@ static int w4_layer_forward(int fmt, const char *name, const uint16_t *x, const 
         // the small blocks: register-fed kernel over the same 256-row alignment, h in slot order
         W4GroupedArgs g{};
         g.fmt = fmt;
-        g.E = E;
+        g.E = Ew;
         g.sorted_ids = r.sorted;
         g.expert_ids = r.eids;
         g.num_tokens_padded = r.ntp;
@@ -453,7 +485,7 @@ static int w4_layer_forward(int fmt, const char *name, const uint16_t *x, const 
     } else {
         W4GroupedArgs a{};
         a.fmt = fmt;
-        a.E = E;
+        a.E = Ew;
         a.sorted_ids = r.sorted;
         a.expert_ids = r.eids;
         a.num_tokens_padded = r.ntp;
@@ -490,7 +522,7 @@ static int w4_layer_forward(int fmt, const char *name, const uint16_t *x, const 
     }
     {
         trace::Scope ts(trace::COMBINE, s);
-        launch_combine(ys, T, k, H, out, num_sms(), s);
+        launch_combine(ys, T, k, H, out, num_sms(), s, lids);
     }
     return check_launch(name);
 }
@@ -532,6 +564,43 @@ int moe_nvfp4_forward(const uint16_t *x, const float *logits, int T, int H, int 
     }
     return w4_layer_forward(W4_NV, "moe_nvfp4_forward", x, logits, T, H, I, E, k, w13_q, w13_f, w2_q, w2_f, out,
                             topk_ids_out, topk_w_out, ws, ws_bytes, stream, w13_g, w2_g);
+}
+
+int moe_w4a16_forward_ep(const uint16_t *x, const float *logits, int T, int H, int I, int E, int k, int ep_base,
+                         int ep_local, const int32_t *w13_q, const uint16_t *w13_s, const int32_t *w2_q,
+                         const uint16_t *w2_s, uint16_t *out, int32_t *topk_ids_out, float *topk_w_out, void *ws,
+                         size_t ws_bytes, void *stream)
+{
+    g_err[0] = 0;
+    if (int rc = check_expert_range(E, ep_base, ep_local)) return rc;
+    return w4_layer_forward(W4_INT4, "moe_w4a16_forward_ep", x, logits, T, H, I, E, k, w13_q, w13_s, w2_q, w2_s, out,
+                            topk_ids_out, topk_w_out, ws, ws_bytes, stream, nullptr, nullptr, ep_base, ep_local);
+}
+
+int moe_mxfp4_forward_ep(const uint16_t *x, const float *logits, int T, int H, int I, int E, int k, int ep_base,
+                         int ep_local, const int32_t *w13_q, const uint16_t *w13_f, const int32_t *w2_q,
+                         const uint16_t *w2_f, uint16_t *out, int32_t *topk_ids_out, float *topk_w_out, void *ws,
+                         size_t ws_bytes, void *stream)
+{
+    g_err[0] = 0;
+    if (int rc = check_expert_range(E, ep_base, ep_local)) return rc;
+    return w4_layer_forward(W4_FP4, "moe_mxfp4_forward_ep", x, logits, T, H, I, E, k, w13_q, w13_f, w2_q, w2_f, out,
+                            topk_ids_out, topk_w_out, ws, ws_bytes, stream, nullptr, nullptr, ep_base, ep_local);
+}
+
+int moe_nvfp4_forward_ep(const uint16_t *x, const float *logits, int T, int H, int I, int E, int k, int ep_base,
+                         int ep_local, const int32_t *w13_q, const uint16_t *w13_f, const float *w13_g,
+                         const int32_t *w2_q, const uint16_t *w2_f, const float *w2_g, uint16_t *out,
+                         int32_t *topk_ids_out, float *topk_w_out, void *ws, size_t ws_bytes, void *stream)
+{
+    g_err[0] = 0;
+    if (int rc = check_expert_range(E, ep_base, ep_local)) return rc;
+    if (T > 0) {
+        MOEQ_REQUIRE(w13_g);
+        MOEQ_REQUIRE(w2_g);
+    }
+    return w4_layer_forward(W4_NV, "moe_nvfp4_forward_ep", x, logits, T, H, I, E, k, w13_q, w13_f, w2_q, w2_f, out,
+                            topk_ids_out, topk_w_out, ws, ws_bytes, stream, w13_g, w2_g, ep_base, ep_local);
 }
 
 int moe_nvfp4_prepack_scales(const uint8_t *e4m3, long long n, uint16_t *factors, void *stream)
@@ -709,14 +778,25 @@ size_t moe_w8a8_block_fp8_workspace_size(int T, int H, int I, int E, int k)
     return fp8_layout(c, T, H, I, E, k, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr);
 }
 
-int moe_w8a8_block_fp8_forward(const uint16_t *x, const float *logits, int T, int H, int I, int E, int k,
-                               const uint8_t *w13, const float *w13_s, const uint8_t *w2, const float *w2_s,
-                               uint16_t *out, int32_t *topk_ids_out, float *topk_w_out, void *ws, size_t ws_bytes,
-                               void *stream)
+size_t moe_w8a8_block_fp8_ep_workspace_size(int T, int H, int I, int E, int k, int ep_local)
+{
+    if (check_layer_shape(T, H, I, E, k) || check_expert_range(E, 0, ep_local)) return 0;
+    Carve c(nullptr);
+    return fp8_layout(c, T, H, I, ep_local, k, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, E);
+}
+
+// The block-FP8 layer; ep_local > 0: expert parallelism over [ep_base, ep_base + ep_local).
+static int fp8_layer_forward(const char *name, const uint16_t *x, const float *logits, int T, int H, int I, int E,
+                             int k, const uint8_t *w13, const float *w13_s, const uint8_t *w2, const float *w2_s,
+                             uint16_t *out, int32_t *topk_ids_out, float *topk_w_out, void *ws, size_t ws_bytes,
+                             void *stream, int ep_base, int ep_local)
 {
     g_err[0] = 0;
     int rc = check_layer_shape(T, H, I, E, k);
     if (rc) return rc;
+    const bool ep = ep_local > 0 || ep_base != 0;
+    if (ep && (rc = check_expert_range(E, ep_base, ep_local))) return rc;
+    const int Ew = ep ? ep_local : E;  // experts whose weights this call holds
     if (T == 0) return MOEQ_OK;
     MOEQ_REQUIRE(x);
     MOEQ_REQUIRE(logits);
@@ -727,7 +807,8 @@ int moe_w8a8_block_fp8_forward(const uint16_t *x, const float *logits, int T, in
     MOEQ_REQUIRE(out);
     MOEQ_REQUIRE(ws);
     if (reinterpret_cast<uintptr_t>(ws) & 255) return set_error(MOEQ_ERR_INVALID_ARG, "ws must be 256-byte aligned");
-    const size_t need = moe_w8a8_block_fp8_workspace_size(T, H, I, E, k);
+    const size_t need = ep ? moe_w8a8_block_fp8_ep_workspace_size(T, H, I, E, k, ep_local)
+                           : moe_w8a8_block_fp8_workspace_size(T, H, I, E, k);
     if (ws_bytes < need) return set_error(MOEQ_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, need);
 
     cudaStream_t s = (cudaStream_t)stream;
@@ -736,19 +817,20 @@ int moe_w8a8_block_fp8_forward(const uint16_t *x, const float *logits, int T, in
     uint8_t *xq, *hq, *xg;
     float *xs, *hs, *xsg;
     uint16_t *ys;
-    fp8_layout(c, T, H, I, E, k, &r, &xq, &xs, &hq, &hs, &ys, &xg, &xsg);
-    int32_t *ids = topk_ids_out ? topk_ids_out : r.ids;
+    fp8_layout(c, T, H, I, Ew, k, &r, &xq, &xs, &hq, &hs, &ys, &xg, &xsg, E);
+    int32_t *ids = topk_ids_out ? topk_ids_out : (ep ? nullptr : r.ids);
+    int32_t *lids = ep ? r.ids : nullptr;
     float *tw = topk_w_out ? topk_w_out : r.w;
     const int n = T * k;
     const bool tcp = fp8_use_tc(T, k, E);
 
     {
         trace::Scope ts(trace::ROUTE, s);
-        launch_route_topk(logits, T, E, k, ids, tw, s);
+        launch_route_topk(logits, T, E, k, ids, tw, s, lids, ep_base, ep_local);
     }
     {
         trace::Scope ts(trace::ALIGN, s);
-        launch_align(ids, n, E, r.block_m, r.sorted, r.eids, r.ntp, r.scratch, s);
+        launch_align(ep ? lids : ids, n, Ew, r.block_m, r.sorted, r.eids, r.ntp, r.scratch, s);
     }
     {
         trace::Scope ts(trace::ACT_QUANT, s);
@@ -758,11 +840,11 @@ int moe_w8a8_block_fp8_forward(const uint16_t *x, const float *logits, int T, in
 
     if (tcp) {
         int *status = device_status_ptr();
-        if (!status) return set_error(MOEQ_ERR_CUDA, "moe_w8a8_block_fp8_forward: no device status word");
+        if (!status) return set_error(MOEQ_ERR_CUDA, "%s: no device status word", name);
         const int cap = r.max_blocks * 128;
         Fp8TcArgs t{};
         t.status = status;
-        t.E = E;
+        t.E = Ew;
         t.sorted_ids = r.sorted;
         t.expert_ids = r.eids;
         t.ntp = r.ntp;
@@ -780,7 +862,7 @@ int moe_w8a8_block_fp8_forward(const uint16_t *x, const float *logits, int T, in
         int rc;
         {
             trace::Scope ts(trace::GATE_UP, s);
-            rc = launch_fp8_tc_grouped(t, TC_GATEUP, xg, w13, E, r.max_blocks, s);
+            rc = launch_fp8_tc_grouped(t, TC_GATEUP, xg, w13, Ew, r.max_blocks, s);
         }
         if (rc) return rc;
         // down, routing weight applied, rows scattered back to their slots
@@ -792,12 +874,12 @@ int moe_w8a8_block_fp8_forward(const uint16_t *x, const float *logits, int T, in
         t.ys = ys;
         {
             trace::Scope ts(trace::DOWN, s);
-            rc = launch_fp8_tc_grouped(t, TC_DOWN, hq, w2, E, r.max_blocks, s);
+            rc = launch_fp8_tc_grouped(t, TC_DOWN, hq, w2, Ew, r.max_blocks, s);
         }
         if (rc) return rc;
     } else {
         F8GroupedArgs a{};
-        a.E = E;
+        a.E = Ew;
         a.sorted_ids = r.sorted;
         a.expert_ids = r.eids;
         a.num_tokens_padded = r.ntp;
@@ -833,9 +915,29 @@ int moe_w8a8_block_fp8_forward(const uint16_t *x, const float *logits, int T, in
     }
     {
         trace::Scope ts(trace::COMBINE, s);
-        launch_combine(ys, T, k, H, out, num_sms(), s);
+        launch_combine(ys, T, k, H, out, num_sms(), s, lids);
     }
-    return check_launch("moe_w8a8_block_fp8_forward");
+    return check_launch(name);
+}
+
+int moe_w8a8_block_fp8_forward(const uint16_t *x, const float *logits, int T, int H, int I, int E, int k,
+                               const uint8_t *w13, const float *w13_s, const uint8_t *w2, const float *w2_s,
+                               uint16_t *out, int32_t *topk_ids_out, float *topk_w_out, void *ws, size_t ws_bytes,
+                               void *stream)
+{
+    return fp8_layer_forward("moe_w8a8_block_fp8_forward", x, logits, T, H, I, E, k, w13, w13_s, w2, w2_s, out,
+                             topk_ids_out, topk_w_out, ws, ws_bytes, stream, 0, 0);
+}
+
+int moe_w8a8_block_fp8_forward_ep(const uint16_t *x, const float *logits, int T, int H, int I, int E, int k,
+                                  int ep_base, int ep_local, const uint8_t *w13, const float *w13_s, const uint8_t *w2,
+                                  const float *w2_s, uint16_t *out, int32_t *topk_ids_out, float *topk_w_out, void *ws,
+                                  size_t ws_bytes, void *stream)
+{
+    g_err[0] = 0;
+    if (int rc = check_expert_range(E, ep_base, ep_local)) return rc;
+    return fp8_layer_forward("moe_w8a8_block_fp8_forward_ep", x, logits, T, H, I, E, k, w13, w13_s, w2, w2_s, out,
+                             topk_ids_out, topk_w_out, ws, ws_bytes, stream, ep_base, ep_local);
 }
 
 int w8a8_block_fp8_matmul(const uint8_t *A, const float *As, const uint8_t *B, const float *Bs, int M, int N, int K,

@@ -101,14 +101,19 @@ struct W4TcArgs {
     int tiles_per_cta;      // down: output tiles of 128 rows per CTA (set by the launcher)
 };
 
-void launch_route_topk(const float *logits, int T, int E, int k, int32_t *ids, float *w, cudaStream_t s);
+// local_ids (nullable): the picks relative to the expert range [ep_base, ep_base + ep_local), -1
+// outside it; ids may be null when local_ids is given.
+void launch_route_topk(const float *logits, int T, int E, int k, int32_t *ids, float *w, cudaStream_t s,
+                       int32_t *local_ids = nullptr, int ep_base = 0, int ep_local = 0);
 // Scratch (bytes) the alignment of n slots over E experts uses; 0 = the one-CTA kernel, which
 // also runs when launch_align gets no scratch.
 size_t align_scratch_bytes(int n, int E);
 void launch_masked_rows(const int32_t *masked_m, int G, int max_m, int32_t *ids, int num_sms, cudaStream_t s);
 void launch_align(const int32_t *topk_ids, int n, int E, int B, int32_t *sorted_ids, int32_t *expert_ids,
                   int32_t *ntp, int32_t *scratch, cudaStream_t s);
-void launch_combine(const uint16_t *ys, int T, int k, int H, uint16_t *out, int num_sms, cudaStream_t s);
+// local_ids (nullable): slots with a negative id are left out of the sum.
+void launch_combine(const uint16_t *ys, int T, int k, int H, uint16_t *out, int num_sms, cudaStream_t s,
+                    const int32_t *local_ids = nullptr);
 // UE8M0 group scales s -> the bf16 factors 2^(s - 1) the FP4 dequantization multiplies by (s > 128
 // overflows to +inf: group scales above 2 are outside the supported range)
 void launch_mxfp4_scale_factors(const uint8_t *s, long long n, uint16_t *f, int num_sms, cudaStream_t st);

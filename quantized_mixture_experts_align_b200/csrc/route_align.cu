@@ -13,10 +13,14 @@ namespace moeq {
 // Routing: one warp per token. Lane l holds logits l, l+32, ... in registers; k rounds of a
 // warp arg-max (value descending, index ascending) pick the experts, then lane j < k turns its
 // pick into exp(l_j - l_max) in double and every lane sums them in slot order.
+// With local_ids (expert parallelism) the picks are also written relative to this rank's expert
+// range [ep_base, ep_base + ep_local), -1 for experts held elsewhere; ids may then be null.
 // ------------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict__ logits, int T, int E,
                                                          int k, int32_t *__restrict__ ids,
-                                                         float *__restrict__ w)
+                                                         float *__restrict__ w,
+                                                         int32_t *__restrict__ local_ids, int ep_base,
+                                                         int ep_local)
 {
     const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -57,16 +61,21 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict
     double den = 0.0;
     for (int j = 0; j < k; ++j) den += __shfl_sync(0xFFFFFFFFu, d, j);
     if (lane < k) {
-        ids[(size_t)t * k + lane] = my_e;
+        if (ids) ids[(size_t)t * k + lane] = my_e;
+        if (local_ids) {
+            const int le = my_e - ep_base;
+            local_ids[(size_t)t * k + lane] = (le >= 0 && le < ep_local) ? le : -1;
+        }
         w[(size_t)t * k + lane] = (float)(d / den);
     }
 }
 
-void launch_route_topk(const float *logits, int T, int E, int k, int32_t *ids, float *w, cudaStream_t s)
+void launch_route_topk(const float *logits, int T, int E, int k, int32_t *ids, float *w, cudaStream_t s,
+                       int32_t *local_ids, int ep_base, int ep_local)
 {
     if (T <= 0) return;
     const int warps = 8;
-    route_topk_kernel<<<cdiv(T, warps), warps * 32, 0, s>>>(logits, T, E, k, ids, w);
+    route_topk_kernel<<<cdiv(T, warps), warps * 32, 0, s>>>(logits, T, E, k, ids, w, local_ids, ep_base, ep_local);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -329,9 +338,11 @@ void launch_align(const int32_t *topk_ids, int n, int E, int B, int32_t *sorted_
 
 // ------------------------------------------------------------------------------------------
 // Top-k weighted combine: out[t, :] = bf16( sum_j ys[t*k + j, :] ), the slot rows (bf16) already
-// carrying their routing weight. f32 sums in slot order.
+// carrying their routing weight. f32 sums in slot order. With local_ids (expert parallelism) the
+// slots routed to experts of other ranks (-1) are left out: their rows of ys are never written.
 // ------------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) combine_kernel(const uint16_t *__restrict__ ys, int T, int k, int H,
+                                                      const int32_t *__restrict__ local_ids,
                                                       uint16_t *__restrict__ out)
 {
     const int H8 = H / 8;
@@ -341,6 +352,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t *__restrict
         const int c = (int)(i - t * H8);
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         for (int j = 0; j < k; ++j) {
+            if (local_ids && __ldg(local_ids + (size_t)t * k + j) < 0) continue;
             const uint4 v = __ldg(reinterpret_cast<const uint4 *>(ys + ((size_t)t * k + j) * H) + c);
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -358,12 +370,13 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t *__restrict
     }
 }
 
-void launch_combine(const uint16_t *ys, int T, int k, int H, uint16_t *out, int num_sms, cudaStream_t s)
+void launch_combine(const uint16_t *ys, int T, int k, int H, uint16_t *out, int num_sms, cudaStream_t s,
+                    const int32_t *local_ids)
 {
     if (T <= 0) return;
     const long total = (long)T * (H / 8);
     const int blocks = (int)((total + 255) / 256 < (long)num_sms * 8 ? (total + 255) / 256 : (long)num_sms * 8);
-    combine_kernel<<<blocks, 256, 0, s>>>(ys, T, k, H, out);
+    combine_kernel<<<blocks, 256, 0, s>>>(ys, T, k, H, local_ids, out);
 }
 
 }  // namespace moeq

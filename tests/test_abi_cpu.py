@@ -131,6 +131,26 @@ def test_validation_rejects_before_device_work(L):
     assert gm(2000, 16, 256, 256, p, 4) == moeq.MOEQ_ERR_UNSUPPORTED             # G > 1024
     assert moeq.lib().moe_w4a16_grouped_masked_workspace_size(8, 64, 256, 384, 48) > \
         moeq.lib().moe_w4a16_grouped_masked_workspace_size(8, 64, 256, 384, 4)   # tensor-core gather buffer
+    # expert-parallel layers: the range must be non-empty and inside [0, E); workspace by ep_local
+    ep = lambda name, base, local, wsb: _rc(L, name, p, p, 32, 7168, 2048, 384, 8, base, local, p, p, p, p, p, N, N,
+                                            p, wsb, N)
+    for name in ("moe_w4a16_forward_ep", "moe_mxfp4_forward_ep", "moe_w8a8_block_fp8_forward_ep"):
+        assert ep(name, 0, 0, 1 << 40) == moeq.MOEQ_ERR_INVALID_ARG             # empty range
+        assert ep(name, -1, 48, 1 << 40) == moeq.MOEQ_ERR_INVALID_ARG           # negative base
+        assert ep(name, 340, 48, 1 << 40) == moeq.MOEQ_ERR_INVALID_ARG          # past E
+        assert b"expert range" in L.moe_last_error()
+        assert ep(name, 336, 48, 10) == moeq.MOEQ_ERR_WORKSPACE
+    nvep = lambda g13, g2: _rc(L, "moe_nvfp4_forward_ep", p, p, 32, 7168, 2048, 384, 8, 0, 48, p, p, g13, p, p, g2,
+                               p, N, N, p, 1 << 40, N)
+    assert nvep(N, p) == moeq.MOEQ_ERR_INVALID_ARG and nvep(p, N) == moeq.MOEQ_ERR_INVALID_ARG
+    w4_full = moeq.moe_w4a16_workspace_size(32, 7168, 2048, 384, 8)
+    w4_ep = moeq.moe_w4a16_ep_workspace_size(32, 7168, 2048, 384, 8, 48)
+    assert 0 < w4_ep < w4_full                     # the alignment's capacity follows ep_local
+    assert moeq.moe_w4a16_ep_workspace_size(32, 7168, 2048, 384, 8, 384) == w4_full
+    assert moeq.moe_w4a16_ep_workspace_size(32, 7168, 2048, 384, 8, 0) == 0
+    assert moeq.moe_w8a8_block_fp8_ep_workspace_size(4096, 7168, 2048, 256, 8, 256) == \
+        moeq.moe_w8a8_block_fp8_workspace_size(4096, 7168, 2048, 256, 8)
+    assert moeq.moe_w8a8_block_fp8_ep_workspace_size(4096, 7168, 2048, 256, 8, 32) > 0
     # T == 0 / M == 0 are valid no-ops
     assert _rc(L, "moe_route_topk", N, 0, 8, 2, N, N, N) == 0
     assert _rc(L, "w8a8_block_fp8_matmul", N, N, N, N, 0, 256, 256, 128, 128, N, N) == 0
