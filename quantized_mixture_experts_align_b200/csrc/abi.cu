@@ -508,6 +508,7 @@ static int w4_layer_forward(int fmt, const char *name, const uint16_t *x, const 
         // down, routing weight applied per slot
         a.act = h;
         a.act_row_div = 1;
+        a.after_gateup = 1;
         a.wq = w2_q;
         a.ws = w2_s;
         a.wglobal = g2;

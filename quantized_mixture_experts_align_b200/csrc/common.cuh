@@ -19,6 +19,32 @@ __host__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 int set_error(int code, const char *fmt, ...);
 int check_launch(const char *what);
 
+// ---- programmatic dependent launch ----------------------------------------------------------
+// A kernel launched by launch_pdl may start while the previous kernel in its stream still runs.
+// pdl_wait() blocks until that kernel has completed and its writes are visible (it returns at
+// once in a kernel launched the ordinary way); every read of data the previous kernels wrote
+// must come after it. pdl_trigger() lets the next kernel, if launched by launch_pdl, start once
+// every CTA of this grid has triggered or exited (all of them resident, so none can starve).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // ---- bf16 / fp32 bit helpers ----------------------------------------------------------------
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }

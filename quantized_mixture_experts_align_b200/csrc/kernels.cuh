@@ -35,6 +35,10 @@ struct W4GroupedArgs {
     // 0: align blocks of BM rows. Otherwise the alignment has blocks of blk_stride rows and the
     // kernel takes only those with at most BM real rows (the rest belong to the tensor-core path)
     int blk_stride;
+    // down, blk_stride 0: the kernel directly before this one is the gate/up kernel of the same
+    // alignment (which waits for the alignment before it lets this kernel start), so the routing
+    // buffers may be read, and the weights prefetched, before waiting for h
+    int after_gateup;
 };
 
 struct F8GroupedArgs {

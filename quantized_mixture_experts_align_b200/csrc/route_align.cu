@@ -22,6 +22,7 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict
                                                          int32_t *__restrict__ local_ids, int ep_base,
                                                          int ep_local)
 {
+    pdl_trigger();  // the alignment after this kernel may launch (it waits for these ids)
     const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (t >= T) return;
@@ -100,6 +101,8 @@ __global__ void __launch_bounds__(kAlignThreads) align_kernel(const int32_t *__r
     __shared__ uint8_t hist[kMaxExperts][kAlignWarps];  // per tile: count of expert e in warp w
     __shared__ int warp_sums[kAlignWarps];
 
+    pdl_wait();     // launched by launch_pdl: the routing ids come from the previous kernel
+    pdl_trigger();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     for (int e = tid; e < E; e += kAlignThreads) { cnt[e] = 0; cursor[e] = 0; }
     for (int i = tid; i < kMaxExperts * kAlignWarps / 4; i += kAlignThreads)
@@ -333,7 +336,7 @@ void launch_align(const int32_t *topk_ids, int n, int E, int B, int32_t *sorted_
         align_scatter_kernel<<<chunks, kChunkThreads, 0, s>>>(topk_ids, n, E, scratch, sorted_ids);
         return;
     }
-    align_kernel<<<1, kAlignThreads, 0, s>>>(topk_ids, n, E, B, sorted_ids, expert_ids, ntp);
+    launch_pdl(align_kernel, dim3(1), dim3(kAlignThreads), 0, s, topk_ids, n, E, B, sorted_ids, expert_ids, ntp);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -345,6 +348,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t *__restrict
                                                       const int32_t *__restrict__ local_ids,
                                                       uint16_t *__restrict__ out)
 {
+    pdl_wait();     // launched by launch_pdl: ys comes from the previous kernel
     const int H8 = H / 8;
     const long total = (long)T * H8;
     for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < total; i += (long)gridDim.x * blockDim.x) {
@@ -376,7 +380,7 @@ void launch_combine(const uint16_t *ys, int T, int k, int H, uint16_t *out, int 
     if (T <= 0) return;
     const long total = (long)T * (H / 8);
     const int blocks = (int)((total + 255) / 256 < (long)num_sms * 8 ? (total + 255) / 256 : (long)num_sms * 8);
-    combine_kernel<<<blocks, 256, 0, s>>>(ys, T, k, H, local_ids, out);
+    launch_pdl(combine_kernel, dim3(blocks), dim3(256), 0, s, ys, T, k, H, local_ids, out);
 }
 
 }  // namespace moeq

@@ -87,24 +87,25 @@ __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4Grouped
     extern __shared__ __align__(16) unsigned char smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
+    // Launched by launch_pdl (blk_stride 0), this kernel may start before the previous one ends.
+    // A down kernel right after its gate/up kernel may read the routing buffers at once (the
+    // gate/up kernel lets it start only after waiting for the alignment) and prefetches its
+    // weights before waiting for h; otherwise every read waits. Every CTA waits before it exits,
+    // so this grid completes after the previous one.
+    const bool early = MODE == MODE_DOWN && !STRIDED && a.after_gateup;
+    if (!early) pdl_wait();
+    pdl_trigger();
     const int blk = blockIdx.x;
     const int base = blk * (STRIDED ? a.blk_stride : BM);  // first aligned row of the block
-    if (base >= __ldg(a.num_tokens_padded)) return;
-    // strided: blocks with more than BM real rows are the tensor-core path's (real rows come first)
-    if (STRIDED && __ldg(a.sorted_ids + base + BM) < a.n_slots) return;
     const int e = __ldg(a.expert_ids + blk);
-    if (e < 0 || e >= a.E) return;
-
     const int tile = blockIdx.y * WARPS + warp;
-    int rowA, rowB;
-    if (MODE == MODE_GATEUP) {
-        rowA = tile * 16;
-        if (rowA >= a.n_out) return;
-        rowB = a.n_out + rowA;
-    } else {
-        rowA = tile * 32;
-        if (rowA >= a.n_out) return;
-        rowB = rowA + 16;
+    const int rowA = tile * (MODE == MODE_GATEUP ? 16 : 32);
+    const int rowB = MODE == MODE_GATEUP ? a.n_out + rowA : rowA + 16;
+    // strided: blocks with more than BM real rows are the tensor-core path's (real rows come first)
+    if (base >= __ldg(a.num_tokens_padded) || (STRIDED && __ldg(a.sorted_ids + base + BM) < a.n_slots) || e < 0 ||
+        e >= a.E || rowA >= a.n_out) {
+        if (early) pdl_wait();
+        return;
     }
 
     // token columns this lane feeds as MMA B (column g of each sub-tile)
@@ -152,6 +153,7 @@ __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4Grouped
 
 #pragma unroll
     for (int q = 0; q < S - 1; ++q) issue(q);
+    if (early) pdl_wait();  // h comes from the gate/up kernel
 
     uint4 xcur[kActPrefetch ? MS : 1][4];
     if (kActPrefetch) {
@@ -266,7 +268,10 @@ static void launch_bm_fmt(const W4GroupedArgs &a, int max_blocks, cudaStream_t s
         attr_set = true;
     }
     dim3 grid(max_blocks, cdiv(a.n_out, rows_per_cta));
-    w4a16_grouped_mma_kernel<BM, WARPS, MODE, STRIDED, FMT><<<grid, WARPS * 32, smem, s>>>(a);
+    if (STRIDED)  // after the tensor-core kernels of the same stage: an ordinary launch
+        w4a16_grouped_mma_kernel<BM, WARPS, MODE, STRIDED, FMT><<<grid, WARPS * 32, smem, s>>>(a);
+    else
+        launch_pdl(w4a16_grouped_mma_kernel<BM, WARPS, MODE, STRIDED, FMT>, grid, dim3(WARPS * 32), smem, s, a);
 }
 
 template <int BM, int WARPS, int MODE, bool STRIDED>
