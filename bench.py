@@ -50,7 +50,7 @@ def load_peaks():
 
 
 # ---------------------------------------------------------------------------------------------
-# distributed plumbing (replicas only)
+# distributed plumbing
 # ---------------------------------------------------------------------------------------------
 
 def dist_setup(n_gpus):
