@@ -12,6 +12,13 @@
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream). Every call only
  *    enqueues work on that stream and returns; no call synchronizes with the host or reads
  *    device data back, so a sequence of calls can be captured in a CUDA graph.
+ *  - Some kernels are launched as programmatic dependents of the kernel before them in the
+ *    stream, which may be the caller's. Such a kernel may start early. Each of its CTAs waits
+ *    for that kernel to complete, with its writes visible, before reading anything that kernel
+ *    could have written, and before exiting. Stream order toward the caller's work is
+ *    therefore unchanged: a call sees everything written before it on the stream, and its
+ *    outputs are complete before the caller's next launch (ordinary, or waiting in the same
+ *    way), copy or event on the stream.
  *  - Status: 0 on success, else one of the MOEQ_ERR_* codes; the calling thread's last error
  *    message is available from moe_last_error(). Arguments are validated on the host before
  *    anything is enqueued; a rejected call enqueues nothing. No C++ exception crosses the ABI.
