@@ -14,7 +14,7 @@ import oracle
 import workloads as W
 from quantized_mixture_experts_align_b200 import sharding as S
 
-KINDS = {"w4a16": "tiny_w4a16", "nvfp4": "decode_nvfp4", "fp8": "moe_fp8"}
+KINDS = {"w4a16": "tiny_w4a16", "mxfp4": "decode_mxfp4", "nvfp4": "decode_nvfp4", "fp8": "moe_fp8"}
 
 
 def _layer(kind, T=6, E=6, k=2, H=128, I=256):
@@ -23,7 +23,7 @@ def _layer(kind, T=6, E=6, k=2, H=128, I=256):
 
 def _host(d, kind):
     """The weights as the oracle takes them, keyed as the sharding module names them (the oracle
-    reads raw NVFP4 scale bytes where the GPU path reads prepacked factors: same layout)."""
+    reads the raw MXFP4 / NVFP4 scale bytes where the GPU path reads prepacked factors: same layout)."""
     if kind == "fp8":
         return {n: W.np_bits(d[n]) for n in ("w13", "w13s", "w2", "w2s")}
     w = {"w13q": W.np_bits(d["w13q"]), "w2q": W.np_bits(d["w2q"])}
@@ -41,6 +41,8 @@ def _oracle_full(d, kind, w):
         return oracle.moe_fp8(x, lg, k, w["w13"], w["w13s"], w["w2"], w["w2s"])
     if kind == "nvfp4":
         return oracle.moe_nvfp4(x, lg, k, w["w13q"], w["w13f"], w["g13"], w["w2q"], w["w2f"], w["g2"])
+    if kind == "mxfp4":
+        return oracle.moe_mxfp4(x, lg, k, w["w13q"], w["w13f"], w["w2q"], w["w2f"])
     return oracle.moe_w4a16(x, lg, k, w["w13q"], w["w13s"], w["w2q"], w["w2s"])
 
 
@@ -50,6 +52,8 @@ def _oracle_ep(d, kind, w, base):
         return oracle.moe_fp8_ep(x, lg, k, base, w["w13"], w["w13s"], w["w2"], w["w2s"])
     if kind == "nvfp4":
         return oracle.moe_q4_ep("nvfp4", x, lg, k, base, w["w13q"], w["w13f"], w["w2q"], w["w2f"], w["g13"], w["g2"])
+    if kind == "mxfp4":
+        return oracle.moe_q4_ep("mxfp4", x, lg, k, base, w["w13q"], w["w13f"], w["w2q"], w["w2f"])
     return oracle.moe_q4_ep("w4a16", x, lg, k, base, w["w13q"], w["w13s"], w["w2q"], w["w2s"])
 
 
