@@ -105,6 +105,28 @@ def _stream(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
 
 
+def _shape(t, want, name: str):
+    """Raise unless tensor t has shape `want` (checked before any pointer is taken)."""
+    if tuple(t.shape) != tuple(want):
+        raise ValueError(f"{name} must have shape {tuple(want)}, got {tuple(t.shape)}")
+
+
+def _layer_shapes(x, logits, w13, s13, w2, s2, E_w, I, w_div, s_div, fmt="w4a16"):
+    """Shapes of a layer call: x [T, H], logits [T, E], and the weights of E_w experts: gate/up
+    [E_w, 2I, H / w_div] with scales [E_w, 2I / s_row, H / s_div], down [E_w, H, I / w_div] with
+    scales [E_w, H / s_row, I / s_div] (s_row = 128 for block FP8, else 1)."""
+    T, H = x.shape
+    if logits.dim() != 2 or logits.shape[0] != T:
+        raise ValueError(f"logits must be [T={T}, E], got {tuple(logits.shape)}")
+    if H % s_div or I % s_div:
+        raise ValueError(f"H={H} and I={I} must be multiples of {s_div}")
+    r = 128 if fmt == "fp8" else 1
+    _shape(w13, (E_w, 2 * I, H // w_div), "w13")
+    _shape(s13, (E_w, 2 * I // r, H // s_div), "w13 scales")
+    _shape(w2, (E_w, H, I // w_div), "w2")
+    _shape(s2, (E_w, H // r, I // s_div), "w2 scales")
+
+
 _BF16 = (torch.bfloat16, torch.int16, torch.uint16)
 _U8 = (torch.uint8, torch.float8_e4m3fn)
 
@@ -170,6 +192,7 @@ def moe_w4a16_forward(x, logits, k, w13_q, w13_s, w2_q, w2_s, out=None, ws=None,
     T, H = x.shape
     E = logits.shape[1]
     I = w2_q.shape[2] * 8
+    _layer_shapes(x, logits, w13_q, w13_s, w2_q, w2_s, E, I, 8, 32)
     out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device) if out is None else out
     need = moe_w4a16_workspace_size(T, H, I, E, k)
     ws = workspace(need, x.device) if ws is None else ws
@@ -198,6 +221,7 @@ def moe_mxfp4_forward(x, logits, k, w13_q, w13_f, w2_q, w2_f, out=None, ws=None,
     T, H = x.shape
     E = logits.shape[1]
     I = w2_q.shape[2] * 8
+    _layer_shapes(x, logits, w13_q, w13_f, w2_q, w2_f, E, I, 8, 32)
     out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device) if out is None else out
     need = lib().moe_mxfp4_workspace_size(T, H, I, E, k)
     ws = workspace(need, x.device) if ws is None else ws
@@ -226,6 +250,9 @@ def moe_nvfp4_forward(x, logits, k, w13_q, w13_f, w13_g, w2_q, w2_f, w2_g, out=N
     T, H = x.shape
     E = logits.shape[1]
     I = w2_q.shape[2] * 8
+    _layer_shapes(x, logits, w13_q, w13_f, w2_q, w2_f, E, I, 8, 16)
+    _shape(w13_g, (E,), "w13_g")
+    _shape(w2_g, (E,), "w2_g")
     out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device) if out is None else out
     need = lib().moe_nvfp4_workspace_size(T, H, I, E, k)
     ws = workspace(need, x.device) if ws is None else ws
@@ -260,6 +287,7 @@ def moe_w8a8_block_fp8_forward(x, logits, k, w13, w13_s, w2, w2_s, out=None, ws=
     T, H = x.shape
     E = logits.shape[1]
     I = w2.shape[2]
+    _layer_shapes(x, logits, w13, w13_s, w2, w2_s, E, I, 1, 128, fmt="fp8")
     out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device) if out is None else out
     need = moe_w8a8_block_fp8_workspace_size(T, H, I, E, k)
     ws = workspace(need, x.device) if ws is None else ws
@@ -286,6 +314,14 @@ def _ep_call(name, x, logits, k, ep_base, weights, out, ws, topk_ids_out, topk_w
     T, H = x.shape
     E = logits.shape[1]
     ep_local = weights[0][0].shape[0]
+    mats = [t for t, n, _ in weights if not n.endswith("_g")]  # codes / scales in the layer order
+    if name == "moe_w8a8_block_fp8_forward_ep":
+        _layer_shapes(x, logits, *mats, ep_local, I, 1, 128, fmt="fp8")
+    else:
+        _layer_shapes(x, logits, *mats, ep_local, I, 8, 16 if name == "moe_nvfp4_forward_ep" else 32)
+    for t, n, _ in weights:
+        if n.endswith("_g"):
+            _shape(t, (ep_local,), n)
     out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device) if out is None else out
     ws = workspace(ws_fn(T, H, I, E, k, ep_local), x.device) if ws is None else ws
     _check(getattr(lib(), name)(
@@ -335,8 +371,13 @@ def moe_w8a8_block_fp8_forward_ep(x, logits, k, ep_base, w13, w13_s, w2, w2_s, o
 
 
 def w8a8_block_fp8_matmul(A, As, B, Bs, block_size=(128, 128), out=None, stream=None):
+    """C = block-scaled A B^T in bf16: A E4M3 [M, K], As f32 [M, K/128] (per token and 128-column
+    group), B E4M3 [N, K], Bs f32 [cdiv(N, 128), cdiv(K, 128)] (per [128, 128] block)."""
     M, K = A.shape
     N = B.shape[0]
+    _shape(B, (N, K), "B")
+    _shape(As, (M, -(-K // 128)), "As")
+    _shape(Bs, (-(-N // 128), -(-K // 128)), "Bs")
     out = torch.empty((M, N), dtype=torch.bfloat16, device=A.device) if out is None else out
     _check(lib().w8a8_block_fp8_matmul(
         _dev(A, "A", _U8), _dev(As, "As", torch.float32), _dev(B, "B", _U8), _dev(Bs, "Bs", torch.float32),
@@ -364,6 +405,9 @@ def moe_w4a16_grouped_contiguous(A, w_q, w_s, m_indices, out=None, ws=None, stre
     w_s bf16 [G, N, K/32]; m_indices int32 [M]."""
     M, K = A.shape
     G, N = w_q.shape[0], w_q.shape[1]
+    _shape(w_q, (G, N, K // 8), "w_q")
+    _shape(w_s, (G, N, K // 32), "w_s")
+    _shape(m_indices, (M,), "m_indices")
     out = torch.empty((M, N), dtype=torch.bfloat16, device=A.device) if out is None else out
     ws = workspace(lib().moe_w4a16_grouped_contiguous_workspace_size(M, K, N, G), A.device) if ws is None else ws
     _check(lib().moe_w4a16_grouped_contiguous(
@@ -380,6 +424,11 @@ def moe_w4a16_grouped_masked(A, w_q, w_s, masked_m, expected_m, out=None, ws=Non
     G, N = w_q.shape[0], w_q.shape[1]
     K = A.shape[-1]
     max_m = A.numel() // (G * K)
+    if A.numel() != G * max_m * K:
+        raise ValueError(f"A must hold G={G} budgets of max_m rows of K={K}, got {tuple(A.shape)}")
+    _shape(w_q, (G, N, K // 8), "w_q")
+    _shape(w_s, (G, N, K // 32), "w_s")
+    _shape(masked_m, (G,), "masked_m")
     out = torch.empty((G * max_m, N), dtype=torch.bfloat16, device=A.device) if out is None else out
     ws = workspace(lib().moe_w4a16_grouped_masked_workspace_size(G, max_m, K, N, expected_m), A.device) \
         if ws is None else ws

@@ -160,3 +160,65 @@ def test_binding_refuses_cpu_tensors(L):
     import torch
     with pytest.raises(ValueError):
         moeq.moe_route_topk(torch.zeros(4, 8), 2)
+
+
+def test_binding_rejects_mismatched_shapes(L):
+    """The binding checks every tensor's shape against the sizes it passes to the C ABI (which
+    sees pointers only) and raises before taking any pointer (meta tensors: no memory, no GPU)."""
+    import torch
+    m = lambda *sh, dt=torch.uint8: torch.empty(sh, dtype=dt, device="meta")
+    f32, i32, bf = torch.float32, torch.int32, torch.bfloat16
+    # dense block FP8: As [M, cdiv(K,128)], Bs [cdiv(N,128), cdiv(K,128)], B [N, K]
+    A, B = m(4, 256), m(384, 256)
+    with pytest.raises(ValueError, match="Bs"):
+        moeq.w8a8_block_fp8_matmul(A, m(4, 2, dt=f32), B, m(2, 2, dt=f32))
+    with pytest.raises(ValueError, match="As"):
+        moeq.w8a8_block_fp8_matmul(A, m(4, 3, dt=f32), B, m(3, 2, dt=f32))
+    with pytest.raises(ValueError, match="B must"):
+        moeq.w8a8_block_fp8_matmul(A, m(4, 2, dt=f32), m(384, 128), m(3, 2, dt=f32))
+    # W4A16 layer (T=2, H=256, I=128, E=4): every weight tensor and the logits
+    x, lg = m(2, 256, dt=bf), m(2, 4, dt=f32)
+    good = [m(4, 256, 32, dt=i32), m(4, 256, 8, dt=bf), m(4, 256, 16, dt=i32), m(4, 256, 4, dt=bf)]
+    for i, bad in enumerate([m(3, 256, 32, dt=i32), m(4, 256, 4, dt=bf), m(4, 128, 16, dt=i32), m(4, 256, 8, dt=bf)]):
+        w = list(good)
+        w[i] = bad
+        with pytest.raises(ValueError, match="w13|w2"):
+            moeq.moe_w4a16_forward(x, lg, 2, *w)
+    with pytest.raises(ValueError, match="logits"):
+        moeq.moe_w4a16_forward(x, m(3, 4, dt=f32), 2, *good)
+    # NVFP4 group-16 scales and per-expert tensor scales
+    nv = [m(4, 256, 32, dt=i32), m(4, 256, 16, dt=bf), m(4, dt=f32), m(4, 256, 16, dt=i32), m(4, 256, 8, dt=bf),
+          m(4, dt=f32)]
+    bad = list(nv)
+    bad[2] = m(3, dt=f32)
+    with pytest.raises(ValueError, match="w13_g"):
+        moeq.moe_nvfp4_forward(x, lg, 2, *bad)
+    bad = list(nv)
+    bad[1] = m(4, 256, 8, dt=bf)                                  # group-32 scales given
+    with pytest.raises(ValueError, match="w13 scales"):
+        moeq.moe_nvfp4_forward(x, lg, 2, *bad)
+    # block-FP8 layer: scales per [128, 128] block
+    fp = [m(4, 256, 256), m(4, 2, 2, dt=f32), m(4, 256, 128), m(4, 2, 1, dt=f32)]
+    bad = list(fp)
+    bad[3] = m(4, 2, 2, dt=f32)
+    with pytest.raises(ValueError, match="w2 scales"):
+        moeq.moe_w8a8_block_fp8_forward(m(2, 256, dt=bf), lg, 2, *bad)
+    # expert-parallel share: every tensor holds the same ep_local experts
+    with pytest.raises(ValueError, match="w2"):
+        moeq.moe_w4a16_forward_ep(x, lg, 2, 2, m(2, 256, 32, dt=i32), m(2, 256, 8, dt=bf), m(3, 256, 16, dt=i32),
+                                  m(2, 256, 4, dt=bf))
+
+
+def test_grouped_binding_rejects_mismatched_shapes(L):
+    import torch
+    m = lambda *sh, dt=torch.uint8: torch.empty(sh, dtype=dt, device="meta")
+    i32, bf = torch.int32, torch.bfloat16
+    A, wq, ws = m(256, 256, dt=bf), m(4, 128, 32, dt=i32), m(4, 128, 8, dt=bf)
+    with pytest.raises(ValueError, match="w_s"):
+        moeq.moe_w4a16_grouped_contiguous(A, wq, m(4, 128, 4, dt=bf), m(256, dt=i32))
+    with pytest.raises(ValueError, match="m_indices"):
+        moeq.moe_w4a16_grouped_contiguous(A, wq, ws, m(255, dt=i32))
+    with pytest.raises(ValueError, match="masked_m"):
+        moeq.moe_w4a16_grouped_masked(m(4, 16, 256, dt=bf), wq, ws, m(3, dt=i32), 4)
+    with pytest.raises(ValueError, match="budgets"):
+        moeq.moe_w4a16_grouped_masked(m(4, 15, 256, dt=bf).view(60, 256)[:58], wq, ws, m(4, dt=i32), 4)
