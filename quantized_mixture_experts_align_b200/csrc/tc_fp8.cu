@@ -476,13 +476,11 @@ int launch_tc(const Fp8TcArgs &a, const CUtensorMap &tmA, const CUtensorMap &tmB
 {
     using Sh = Fp8TcShape<BN, PAIR, MODE>;
     constexpr int kThreads = fp8_threads(MODE);
-    static bool attr = false;
-    if (!attr) {
-        const cudaError_t e = cudaFuncSetAttribute(fp8_tc_gemm_kernel<BN, MODE, PAIR>,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Sh::kSmemBytes);
+    static int smem_enabled[tc::kMaxDevices] = {};
+    {
+        const cudaError_t e = tc::enable_smem(fp8_tc_gemm_kernel<BN, MODE, PAIR>, (int)Sh::kSmemBytes, smem_enabled);
         if (e != cudaSuccess)
             return set_error(MOEQ_ERR_CUDA, "tcgen05 FP8 GEMM: shared-memory attribute: %s", cudaGetErrorString(e));
-        attr = true;
     }
     if (grid_x <= 0 || grid_y <= 0) return MOEQ_OK;
     if (!PAIR && split <= 1) {

@@ -273,14 +273,12 @@ int launch_skinny(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B, int sp
     if (smem > 227 * 1024)
         return set_error(MOEQ_ERR_UNSUPPORTED, "tcgen05 FP8 skinny GEMM: K = %d needs %zu bytes of shared memory",
                          a.K, smem);
-    static int attr_bytes = 0;
-    if (attr_bytes < (int)smem) {
-        const cudaError_t e = cudaFuncSetAttribute(fp8_tc_skinny_kernel<MP, G, TWO, CW>,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static int smem_enabled[tc::kMaxDevices] = {};
+    {
+        const cudaError_t e = tc::enable_smem(fp8_tc_skinny_kernel<MP, G, TWO, CW>, (int)smem, smem_enabled);
         if (e != cudaSuccess)
             return set_error(MOEQ_ERR_CUDA, "tcgen05 FP8 skinny GEMM: shared-memory attribute: %s",
                              cudaGetErrorString(e));
-        attr_bytes = (int)smem;
     }
     CUtensorMap tmW, tmX;
     int rc = make_tmap_2d(&tmW, B, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.N, (uint64_t)a.K, kRows, kBK);

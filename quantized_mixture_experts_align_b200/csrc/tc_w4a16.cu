@@ -407,13 +407,11 @@ __global__ void __launch_bounds__(256) gather_bf16_perm_kernel(const uint16_t *_
 template <int MODE, int FMT>
 int launch_mode(const W4TcArgs &a, const CUtensorMap &tm, int grid_x, int grid_y, cudaStream_t s)
 {
-    static bool attr = false;
-    if (!attr) {
-        const cudaError_t e =
-            cudaFuncSetAttribute(w4a16_tc_kernel<MODE, FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    static int smem_enabled[tc::kMaxDevices] = {};
+    {
+        const cudaError_t e = tc::enable_smem(w4a16_tc_kernel<MODE, FMT>, (int)kSmemBytes, smem_enabled);
         if (e != cudaSuccess)
             return set_error(MOEQ_ERR_CUDA, "tcgen05 W4A16 GEMM: shared-memory attribute: %s", cudaGetErrorString(e));
-        attr = true;
     }
     if (grid_x <= 0 || grid_y <= 0) return MOEQ_OK;
     w4a16_tc_kernel<MODE, FMT><<<dim3(grid_x, grid_y), kThreads, kSmemBytes, s>>>(tm, a);
