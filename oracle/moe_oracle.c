@@ -15,11 +15,14 @@
  *  [CHORD]  "vLLM x Novita AI: Chord W4A16 INT4 MoE Kernel for Kimi K2.x" (Novita blog).
  *  [SGL]    "SGLang W8A8 Block FP8 quantized kernel config files: analysis and tuning guide"
  *           (xdnf.cn article on SGLang's fp8_kernel.py).
+ *  lk_moe   "Lsglang — lk_moe Hybrid Inference for sglang", "Supported models & quant formats"
+ *           (MXFP4 and NVFP4 weight formats).
  * Where the pages leave a step open, the reading taken is stated at the step.
  *
  * Parity pins: every exported function is checked, on the CPU, against hand-worked cases, closed
  * forms, invariants, brute force or a library routine (numpy matmul, torch dtype casts) by the
- * oracle tests; none is "parity unpinned".
+ * oracle tests. The expert-parallel shares are pinned to the whole layer: the full range is the
+ * layer bit for bit, and the ranks' shares sum to it. None is "parity unpinned".
  */
 #include <math.h>
 #include <stdint.h>
