@@ -127,6 +127,21 @@ def _layer_shapes(x, logits, w13, s13, w2, s2, E_w, I, w_div, s_div, fmt="w4a16"
     _shape(s2, (E_w, H // r, I // s_div), "w2 scales")
 
 
+def _layer_outputs(x, k, out, topk_ids_out, topk_w_out):
+    """The layer's output buffers: out [T, H] (allocated when None) and the optional routing
+    outputs topk_ids_out / topk_w_out [T, k]. A caller-passed buffer of another shape raises before
+    any pointer is taken: the kernels write T x H and T x k elements through the raw pointers."""
+    T, H = x.shape
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
+    _shape(out, (T, H), "out")
+    if topk_ids_out is not None:
+        _shape(topk_ids_out, (T, k), "topk_ids_out")
+    if topk_w_out is not None:
+        _shape(topk_w_out, (T, k), "topk_w_out")
+    return out
+
+
 _BF16 = (torch.bfloat16, torch.int16, torch.uint16)
 _U8 = (torch.uint8, torch.float8_e4m3fn)
 
@@ -139,6 +154,8 @@ def moe_route_topk(logits: torch.Tensor, k: int, topk_ids=None, topk_w=None, str
     T, E = logits.shape
     topk_ids = torch.empty((T, k), dtype=torch.int32, device=logits.device) if topk_ids is None else topk_ids
     topk_w = torch.empty((T, k), dtype=torch.float32, device=logits.device) if topk_w is None else topk_w
+    _shape(topk_ids, (T, k), "topk_ids")
+    _shape(topk_w, (T, k), "topk_w")
     _check(lib().moe_route_topk(_dev(logits, "logits", torch.float32), T, E, k, _dev(topk_ids, "topk_ids", torch.int32),
                                 _dev(topk_w, "topk_w", torch.float32), _stream(stream)))
     return topk_ids, topk_w
@@ -193,7 +210,7 @@ def moe_w4a16_forward(x, logits, k, w13_q, w13_s, w2_q, w2_s, out=None, ws=None,
     E = logits.shape[1]
     I = w2_q.shape[2] * 8
     _layer_shapes(x, logits, w13_q, w13_s, w2_q, w2_s, E, I, 8, 32)
-    out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device) if out is None else out
+    out = _layer_outputs(x, k, out, topk_ids_out, topk_w_out)
     need = moe_w4a16_workspace_size(T, H, I, E, k)
     ws = workspace(need, x.device) if ws is None else ws
     _check(lib().moe_w4a16_forward(
@@ -209,6 +226,7 @@ def moe_mxfp4_prepack_scales(s_ue8m0, out=None, stream=None):
     """UE8M0 group scales (uint8, any shape) -> the bf16 group factors 2^(s - 1) moe_mxfp4_forward
     takes (same shape)."""
     out = torch.empty(s_ue8m0.shape, dtype=torch.bfloat16, device=s_ue8m0.device) if out is None else out
+    _shape(out, s_ue8m0.shape, "out")
     _check(lib().moe_mxfp4_prepack_scales(_dev(s_ue8m0, "s_ue8m0", _U8), s_ue8m0.numel(), _dev(out, "out", _BF16),
                                           _stream(stream)))
     return out
@@ -222,7 +240,7 @@ def moe_mxfp4_forward(x, logits, k, w13_q, w13_f, w2_q, w2_f, out=None, ws=None,
     E = logits.shape[1]
     I = w2_q.shape[2] * 8
     _layer_shapes(x, logits, w13_q, w13_f, w2_q, w2_f, E, I, 8, 32)
-    out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device) if out is None else out
+    out = _layer_outputs(x, k, out, topk_ids_out, topk_w_out)
     need = lib().moe_mxfp4_workspace_size(T, H, I, E, k)
     ws = workspace(need, x.device) if ws is None else ws
     _check(lib().moe_mxfp4_forward(
@@ -238,6 +256,7 @@ def moe_nvfp4_prepack_scales(s_e4m3, out=None, stream=None):
     """E4M3 group scales (uint8, any shape) -> the bf16 factors E4M3(s) * 2^118 moe_nvfp4_forward
     takes (same shape)."""
     out = torch.empty(s_e4m3.shape, dtype=torch.bfloat16, device=s_e4m3.device) if out is None else out
+    _shape(out, s_e4m3.shape, "out")
     _check(lib().moe_nvfp4_prepack_scales(_dev(s_e4m3, "s_e4m3", _U8), s_e4m3.numel(), _dev(out, "out", _BF16),
                                           _stream(stream)))
     return out
@@ -253,7 +272,7 @@ def moe_nvfp4_forward(x, logits, k, w13_q, w13_f, w13_g, w2_q, w2_f, w2_g, out=N
     _layer_shapes(x, logits, w13_q, w13_f, w2_q, w2_f, E, I, 8, 16)
     _shape(w13_g, (E,), "w13_g")
     _shape(w2_g, (E,), "w2_g")
-    out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device) if out is None else out
+    out = _layer_outputs(x, k, out, topk_ids_out, topk_w_out)
     need = lib().moe_nvfp4_workspace_size(T, H, I, E, k)
     ws = workspace(need, x.device) if ws is None else ws
     _check(lib().moe_nvfp4_forward(
@@ -273,7 +292,8 @@ def moe_w4a16_forward_noalloc(x, logits, k, w13_q, w13_s, w2_q, w2_s, out=None, 
     T, H = x.shape
     E = logits.shape[1]
     I = w2_q.shape[2] * 8
-    out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device) if out is None else out
+    _layer_shapes(x, logits, w13_q, w13_s, w2_q, w2_s, E, I, 8, 32)
+    out = _layer_outputs(x, k, out, topk_ids_out, topk_w_out)
     _check(lib().moe_w4a16_forward_noalloc(
         _dev(x, "x", _BF16), _dev(logits, "logits", torch.float32), T, H, I, E, k,
         _dev(w13_q, "w13_q", torch.int32), _dev(w13_s, "w13_s", _BF16), _dev(w2_q, "w2_q", torch.int32),
@@ -288,7 +308,7 @@ def moe_w8a8_block_fp8_forward(x, logits, k, w13, w13_s, w2, w2_s, out=None, ws=
     E = logits.shape[1]
     I = w2.shape[2]
     _layer_shapes(x, logits, w13, w13_s, w2, w2_s, E, I, 1, 128, fmt="fp8")
-    out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device) if out is None else out
+    out = _layer_outputs(x, k, out, topk_ids_out, topk_w_out)
     need = moe_w8a8_block_fp8_workspace_size(T, H, I, E, k)
     ws = workspace(need, x.device) if ws is None else ws
     _check(lib().moe_w8a8_block_fp8_forward(
@@ -322,7 +342,7 @@ def _ep_call(name, x, logits, k, ep_base, weights, out, ws, topk_ids_out, topk_w
     for t, n, _ in weights:
         if n.endswith("_g"):
             _shape(t, (ep_local,), n)
-    out = torch.empty((T, H), dtype=torch.bfloat16, device=x.device) if out is None else out
+    out = _layer_outputs(x, k, out, topk_ids_out, topk_w_out)
     ws = workspace(ws_fn(T, H, I, E, k, ep_local), x.device) if ws is None else ws
     _check(getattr(lib(), name)(
         _dev(x, "x", _BF16), _dev(logits, "logits", torch.float32), T, H, I, E, k, int(ep_base), ep_local,
@@ -379,6 +399,7 @@ def w8a8_block_fp8_matmul(A, As, B, Bs, block_size=(128, 128), out=None, stream=
     _shape(As, (M, -(-K // 128)), "As")
     _shape(Bs, (-(-N // 128), -(-K // 128)), "Bs")
     out = torch.empty((M, N), dtype=torch.bfloat16, device=A.device) if out is None else out
+    _shape(out, (M, N), "out")
     _check(lib().w8a8_block_fp8_matmul(
         _dev(A, "A", _U8), _dev(As, "As", torch.float32), _dev(B, "B", _U8), _dev(Bs, "Bs", torch.float32),
         M, N, K, int(block_size[0]), int(block_size[1]), _dev(out, "out", _BF16), _stream(stream)))
@@ -393,6 +414,7 @@ def w8a8_channel_fp8_matmul(A, As, B, Bs, out=None, stream=None):
     if As.numel() != M or Bs.numel() != N:
         raise ValueError("w8a8_channel_fp8_matmul: As must hold M and Bs N scales")
     out = torch.empty((M, N), dtype=torch.bfloat16, device=A.device) if out is None else out
+    _shape(out, (M, N), "out")
     _check(lib().w8a8_channel_fp8_matmul(
         _dev(A, "A", _U8), _dev(As, "As", torch.float32), _dev(B, "B", _U8), _dev(Bs, "Bs", torch.float32),
         M, N, K, _dev(out, "out", _BF16), _stream(stream)))
@@ -409,6 +431,7 @@ def moe_w4a16_grouped_contiguous(A, w_q, w_s, m_indices, out=None, ws=None, stre
     _shape(w_s, (G, N, K // 32), "w_s")
     _shape(m_indices, (M,), "m_indices")
     out = torch.empty((M, N), dtype=torch.bfloat16, device=A.device) if out is None else out
+    _shape(out, (M, N), "out")
     ws = workspace(lib().moe_w4a16_grouped_contiguous_workspace_size(M, K, N, G), A.device) if ws is None else ws
     _check(lib().moe_w4a16_grouped_contiguous(
         _dev(A, "A", _BF16), M, K, _dev(w_q, "w_q", torch.int32), _dev(w_s, "w_s", _BF16), G, N,
@@ -430,6 +453,7 @@ def moe_w4a16_grouped_masked(A, w_q, w_s, masked_m, expected_m, out=None, ws=Non
     _shape(w_s, (G, N, K // 32), "w_s")
     _shape(masked_m, (G,), "masked_m")
     out = torch.empty((G * max_m, N), dtype=torch.bfloat16, device=A.device) if out is None else out
+    _shape(out, (G * max_m, N), "out")
     ws = workspace(lib().moe_w4a16_grouped_masked_workspace_size(G, max_m, K, N, expected_m), A.device) \
         if ws is None else ws
     _check(lib().moe_w4a16_grouped_masked(
@@ -439,7 +463,7 @@ def moe_w4a16_grouped_masked(A, w_q, w_s, masked_m, expected_m, out=None, ws=Non
     return out
 
 
-TRACE_STAGES = ("route_topk", "align", "fp8_act_quant", "gate_up", "down", "combine", "dense_fp8")
+TRACE_STAGES = ("route_topk", "align", "fp8_act_quant", "gate_up", "down", "combine", "dense_fp8", "gather")
 
 
 def moe_trace_enable(enable: bool = True):

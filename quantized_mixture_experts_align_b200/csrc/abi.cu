@@ -51,7 +51,7 @@ static int num_sms()
 // When enabled, each kernel stage of a call is bracketed by a CUDA event pair recorded on the
 // call's stream; moe_trace_read() waits for the recorded pairs and accumulates their durations.
 namespace trace {
-enum { ROUTE = 0, ALIGN, ACT_QUANT, GATE_UP, DOWN, COMBINE, DENSE, NSTAGE };
+enum { ROUTE = 0, ALIGN, ACT_QUANT, GATE_UP, DOWN, COMBINE, DENSE, GATHER, NSTAGE };
 struct Rec {
     cudaEvent_t a, b;
     int stage;
@@ -112,9 +112,8 @@ static int pick_block_m(long T, int k, int E)
     return 64;
 }
 
-// Dense block-FP8: up to 16 rows the register-fed kernel (K split over warps) streams the
-// weights; from 17 rows on, the tcgen05 kernel (128-row tiles). Chosen from measured M sweeps.
-// K split of the few-row dense FP8 GEMM (cluster size): the smallest power of two that gives
+// K split of the few-row dense FP8 GEMM (swap-AB tcgen05 tiles, used up to fp8_skinny_max_rows()
+// rows; cluster size): the smallest power of two that gives
 // every SM one CTA (16 padded rows: two, the lighter CTAs then share SMs best), at most 8.
 // Measured on 24576 x 7168 weights: 16 rows 36.9 us with split 2 vs 38.9 with 1; 32 / 64 rows
 // 41.0 / 46.6 us with split 1 vs 45.1 / 55.3 with 2.
@@ -413,7 +412,7 @@ static int w4_layer_forward(int fmt, const char *name, const uint16_t *x, const 
         if (!status) return set_error(MOEQ_ERR_CUDA, "%s: no device status word", name);
         const int cap = r.max_blocks * r.block_m;
         {
-            trace::Scope ts(trace::ACT_QUANT, s);  // the activation gather takes the act-prep slot
+            trace::Scope ts(trace::GATHER, s);
             launch_gather_bf16_perm(x, H, k, r.sorted, r.ntp, n, cap, kW4SmallRows, xg, num_sms(), s);
         }
         W4TcArgs t{};
@@ -836,7 +835,10 @@ static int fp8_layer_forward(const char *name, const uint16_t *x, const float *l
     {
         trace::Scope ts(trace::ACT_QUANT, s);
         launch_fp8_act_quant(x, T, H, xq, xs, s);
-        if (tcp) launch_gather_fp8_rows(xq, xs, H, k, r.sorted, r.ntp, n, r.max_blocks * 128, xg, xsg, num_sms(), s);
+    }
+    if (tcp) {
+        trace::Scope ts(trace::GATHER, s);
+        launch_gather_fp8_rows(xq, xs, H, k, r.sorted, r.ntp, n, r.max_blocks * 128, xg, xsg, num_sms(), s);
     }
 
     if (tcp) {

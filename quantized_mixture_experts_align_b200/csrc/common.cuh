@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "moeq.h"
 
 namespace moeq {
@@ -18,6 +20,25 @@ __host__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 // ---- error reporting (host) -------------------------------------------------------------
 int set_error(int code, const char *fmt, ...);
 int check_launch(const char *what);
+
+// ---- dynamic shared memory above the default limit (host) ----------------------------------
+// Enabled per kernel and per device (each device's context holds its own copy of the kernel).
+// `enabled` remembers, per device, the largest size set so far; the entries are atomics because
+// the launchers' tables are shared by every host thread, and setting the attribute twice from
+// two threads is harmless.
+constexpr int kMaxDevices = 64;
+template <typename F>
+inline cudaError_t enable_smem(F kernel, int bytes, std::atomic<int> (&enabled)[kMaxDevices])
+{
+    int dev = 0;
+    const cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const bool tracked = dev >= 0 && dev < kMaxDevices;
+    if (tracked && enabled[dev].load(std::memory_order_relaxed) >= bytes) return cudaSuccess;
+    const cudaError_t r = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (r == cudaSuccess && tracked) enabled[dev].store(bytes, std::memory_order_relaxed);
+    return r;
+}
 
 // ---- programmatic dependent launch ----------------------------------------------------------
 // A kernel launched by launch_pdl may start while the previous kernel in its stream still runs.

@@ -14,21 +14,6 @@ namespace tc {
 // A bounded wait that gives up sets this code in the kernel's status word.
 constexpr int kStatusTimeout = MOEQ_ERR_DEVICE_TIMEOUT;
 
-// Dynamic shared memory above the default limit is enabled per kernel and per device (each
-// device's context holds its own copy of the kernel). `enabled` remembers, per device, the
-// largest size set so far; setting it again from another thread is harmless.
-constexpr int kMaxDevices = 64;
-template <typename F>
-inline cudaError_t enable_smem(F kernel, int bytes, int (&enabled)[kMaxDevices])
-{
-    int dev = 0;
-    const cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < kMaxDevices && enabled[dev] >= bytes) return cudaSuccess;
-    const cudaError_t r = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (r == cudaSuccess && dev >= 0 && dev < kMaxDevices) enabled[dev] = bytes;
-    return r;
-}
 // try_wait polls before a wait is declared stuck (each poll may itself suspend briefly).
 constexpr uint32_t kMaxPolls = 1u << 24;
 

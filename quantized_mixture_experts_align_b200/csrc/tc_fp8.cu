@@ -476,9 +476,9 @@ int launch_tc(const Fp8TcArgs &a, const CUtensorMap &tmA, const CUtensorMap &tmB
 {
     using Sh = Fp8TcShape<BN, PAIR, MODE>;
     constexpr int kThreads = fp8_threads(MODE);
-    static int smem_enabled[tc::kMaxDevices] = {};
+    static std::atomic<int> smem_enabled[kMaxDevices];
     {
-        const cudaError_t e = tc::enable_smem(fp8_tc_gemm_kernel<BN, MODE, PAIR>, (int)Sh::kSmemBytes, smem_enabled);
+        const cudaError_t e = enable_smem(fp8_tc_gemm_kernel<BN, MODE, PAIR>, (int)Sh::kSmemBytes, smem_enabled);
         if (e != cudaSuccess)
             return set_error(MOEQ_ERR_CUDA, "tcgen05 FP8 GEMM: shared-memory attribute: %s", cudaGetErrorString(e));
     }

@@ -273,9 +273,9 @@ int launch_skinny(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B, int sp
     if (smem > 227 * 1024)
         return set_error(MOEQ_ERR_UNSUPPORTED, "tcgen05 FP8 skinny GEMM: K = %d needs %zu bytes of shared memory",
                          a.K, smem);
-    static int smem_enabled[tc::kMaxDevices] = {};
+    static std::atomic<int> smem_enabled[kMaxDevices];
     {
-        const cudaError_t e = tc::enable_smem(fp8_tc_skinny_kernel<MP, G, TWO, CW>, (int)smem, smem_enabled);
+        const cudaError_t e = enable_smem(fp8_tc_skinny_kernel<MP, G, TWO, CW>, (int)smem, smem_enabled);
         if (e != cudaSuccess)
             return set_error(MOEQ_ERR_CUDA, "tcgen05 FP8 skinny GEMM: shared-memory attribute: %s",
                              cudaGetErrorString(e));

@@ -407,9 +407,9 @@ __global__ void __launch_bounds__(256) gather_bf16_perm_kernel(const uint16_t *_
 template <int MODE, int FMT>
 int launch_mode(const W4TcArgs &a, const CUtensorMap &tm, int grid_x, int grid_y, cudaStream_t s)
 {
-    static int smem_enabled[tc::kMaxDevices] = {};
+    static std::atomic<int> smem_enabled[kMaxDevices];
     {
-        const cudaError_t e = tc::enable_smem(w4a16_tc_kernel<MODE, FMT>, (int)kSmemBytes, smem_enabled);
+        const cudaError_t e = enable_smem(w4a16_tc_kernel<MODE, FMT>, (int)kSmemBytes, smem_enabled);
         if (e != cudaSuccess)
             return set_error(MOEQ_ERR_CUDA, "tcgen05 W4A16 GEMM: shared-memory attribute: %s", cudaGetErrorString(e));
     }

@@ -261,12 +261,8 @@ static void launch_bm_fmt(const W4GroupedArgs &a, int max_blocks, cudaStream_t s
 {
     const int rows_per_cta = (MODE == MODE_GATEUP ? 16 : 32) * WARPS;
     const size_t smem = (size_t)WARPS * kW4Stages * w4_stage_bytes(FMT);
-    static bool attr_set = false;  // per template instance; the attribute is per function
-    if (!attr_set) {
-        cudaFuncSetAttribute(w4a16_grouped_mma_kernel<BM, WARPS, MODE, STRIDED, FMT>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        attr_set = true;
-    }
+    static std::atomic<int> smem_enabled[kMaxDevices];
+    enable_smem(w4a16_grouped_mma_kernel<BM, WARPS, MODE, STRIDED, FMT>, (int)smem, smem_enabled);
     dim3 grid(max_blocks, cdiv(a.n_out, rows_per_cta));
     if (STRIDED)  // after the tensor-core kernels of the same stage: an ordinary launch
         w4a16_grouped_mma_kernel<BM, WARPS, MODE, STRIDED, FMT><<<grid, WARPS * 32, smem, s>>>(a);

@@ -222,3 +222,46 @@ def test_grouped_binding_rejects_mismatched_shapes(L):
         moeq.moe_w4a16_grouped_masked(m(4, 16, 256, dt=bf), wq, ws, m(3, dt=i32), 4)
     with pytest.raises(ValueError, match="budgets"):
         moeq.moe_w4a16_grouped_masked(m(4, 15, 256, dt=bf).view(60, 256)[:58], wq, ws, m(4, dt=i32), 4)
+
+
+def test_binding_rejects_output_buffers_of_the_wrong_shape(L):
+    """Caller-passed outputs (out [T, H], topk_ids_out / topk_w_out [T, k], dense C [M, N]) are
+    checked before any pointer is taken: a smaller buffer would be written past its end."""
+    import torch
+    m = lambda *sh, dt=torch.uint8: torch.empty(sh, dtype=dt, device="meta")
+    f32, i32, bf = torch.float32, torch.int32, torch.bfloat16
+    x, lg = m(2, 256, dt=bf), m(2, 4, dt=f32)
+    w = [m(4, 256, 32, dt=i32), m(4, 256, 8, dt=bf), m(4, 256, 16, dt=i32), m(4, 256, 4, dt=bf)]
+    with pytest.raises(ValueError, match="out"):
+        moeq.moe_w4a16_forward(x, lg, 2, *w, out=m(1, 256, dt=bf))
+    with pytest.raises(ValueError, match="topk_ids_out"):
+        moeq.moe_w4a16_forward(x, lg, 2, *w, topk_ids_out=m(2, 1, dt=i32))
+    with pytest.raises(ValueError, match="topk_w_out"):
+        moeq.moe_mxfp4_forward(x, lg, 2, *w, topk_w_out=m(2, 3, dt=f32))
+    fp = [m(4, 256, 256), m(4, 2, 2, dt=f32), m(4, 256, 128), m(4, 2, 1, dt=f32)]
+    with pytest.raises(ValueError, match="out"):
+        moeq.moe_w8a8_block_fp8_forward(x, lg, 2, *fp, out=m(2, 128, dt=bf))
+    with pytest.raises(ValueError, match="out"):
+        moeq.moe_w4a16_forward_ep(x, lg, 2, 0, *w, out=m(2, 255, dt=bf))
+    with pytest.raises(ValueError, match="out"):
+        moeq.w8a8_block_fp8_matmul(m(4, 256), m(4, 2, dt=f32), m(384, 256), m(3, 2, dt=f32), out=m(4, 256, dt=bf))
+    with pytest.raises(ValueError, match="topk_ids"):
+        moeq.moe_route_topk(lg, 2, topk_ids=m(2, 3, dt=i32))
+
+
+def test_noalloc_binding_checks_shapes(L):
+    """The scratch-free forward checks its tensors like moe_w4a16_forward before any pointer."""
+    import torch
+    m = lambda *sh, dt=torch.uint8: torch.empty(sh, dtype=dt, device="meta")
+    f32, i32, bf = torch.float32, torch.int32, torch.bfloat16
+    x, lg = m(2, 256, dt=bf), m(2, 4, dt=f32)
+    good = [m(4, 256, 32, dt=i32), m(4, 256, 8, dt=bf), m(4, 256, 16, dt=i32), m(4, 256, 4, dt=bf)]
+    for i, bad in enumerate([m(3, 256, 32, dt=i32), m(4, 256, 4, dt=bf), m(4, 128, 16, dt=i32), m(4, 256, 8, dt=bf)]):
+        w = list(good)
+        w[i] = bad
+        with pytest.raises(ValueError, match="w13|w2"):
+            moeq.moe_w4a16_forward_noalloc(x, lg, 2, *w)
+    with pytest.raises(ValueError, match="logits"):
+        moeq.moe_w4a16_forward_noalloc(x, m(3, 4, dt=f32), 2, *good)
+    with pytest.raises(ValueError, match="out"):
+        moeq.moe_w4a16_forward_noalloc(x, lg, 2, *good, out=m(2, 128, dt=bf))
