@@ -326,6 +326,20 @@ MOEQ_API int moe_trace_enable(int enable);
 MOEQ_API int moe_trace_read(double *stage_ms, long long *stage_calls, int n_stages, int reset);
 
 /*
+ * Host-side cost of the entry points ("vLLM x Novita AI: Chord W4A16 INT4 MoE Kernel for Kimi
+ * K2.x", section "SM90 grouped kernels": per-launch host lookup, memoized there). Every layer
+ * forward, grouped GEMM and dense matmul adds its host wall time (validation, workspace carving,
+ * schedule choice, tensor maps, kernel launches; not the device time) to a process-wide total.
+ * The tensor maps the tensor-core kernels need are memoized on their parameters (address, type,
+ * extents, box, swizzle; a ring of 64), so a repeated call on the same buffers encodes none.
+ * Writes (each pointer may be NULL): the summed host time in microseconds, the number of calls,
+ * tensor maps encoded through the driver and reused from the memo since load. `reset` != 0 clears
+ * the time and call totals. Returns MOEQ_OK.
+ */
+MOEQ_API int moe_host_stats(double *host_us, long long *calls, long long *tmap_encoded, long long *tmap_reused,
+                            int reset);
+
+/*
  * Sticky device status of the library's kernels on the current device: 0 if no kernel has
  * reported a problem, else MOEQ_ERR_DEVICE_TIMEOUT. This call synchronizes with the device (it
  * is a diagnostic, not part of the forward path); `clear` != 0 resets the status.

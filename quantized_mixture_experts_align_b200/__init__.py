@@ -58,6 +58,7 @@ _SIGNATURES = {
     "moe_w4a16_grouped_masked": ([_V, _I, _I, _I, _V, _V, _I, _V, _I, _V, _V, _Z, _V], _I),
     "moe_trace_enable": ([_I], _I),
     "moe_trace_read": ([_V, _V, _I, _I], _I),
+    "moe_host_stats": ([_V, _V, _V, _V, _I], _I),
     "moe_device_status": ([_I], _I),
     "moe_selftest_bounded_wait": ([_V], _I),
 }
@@ -480,6 +481,16 @@ def moe_trace_read(reset: bool = False) -> dict:
     if rc != n:
         _check(rc)
     return {name: (ms[i], calls[i]) for i, name in enumerate(TRACE_STAGES)}
+
+
+def moe_host_stats(reset: bool = False) -> dict:
+    """Host time the library's entry points spent (microseconds, summed), their call count, and
+    tensor maps encoded / reused from the library's memo."""
+    us = ctypes.c_double()
+    calls, enc, reu = ctypes.c_longlong(), ctypes.c_longlong(), ctypes.c_longlong()
+    _check(lib().moe_host_stats(ctypes.byref(us), ctypes.byref(calls), ctypes.byref(enc), ctypes.byref(reu),
+                                1 if reset else 0))
+    return {"host_us": us.value, "calls": calls.value, "tmap_encoded": enc.value, "tmap_reused": reu.value}
 
 
 def moe_selftest_bounded_wait(stream=None):

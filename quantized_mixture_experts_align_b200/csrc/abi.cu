@@ -4,6 +4,8 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <atomic>
+#include <chrono>
 #include <mutex>
 #include <vector>
 
@@ -97,6 +99,22 @@ struct Scope {
     }
 };
 }  // namespace trace
+
+// ---- host submit time ------------------------------------------------------------------------
+// Wall time each entry point spends on the host (validation, workspace carving, schedule choice,
+// tensor maps, launches), summed per library; read with moe_host_stats.
+namespace host_time {
+static std::atomic<long long> ns{0}, calls{0};
+struct Scope {
+    std::chrono::steady_clock::time_point t0 = std::chrono::steady_clock::now();
+    ~Scope()
+    {
+        const auto d = std::chrono::steady_clock::now() - t0;
+        ns.fetch_add((long long)std::chrono::duration_cast<std::chrono::nanoseconds>(d).count(), std::memory_order_relaxed);
+        calls.fetch_add(1, std::memory_order_relaxed);
+    }
+};
+}  // namespace host_time
 
 // ---- schedule --------------------------------------------------------------------------------
 // The routed rows per expert (tok_e = T*k/E), not the token count, decides the tile ("vLLM x
@@ -195,8 +213,8 @@ static size_t w4a16_layout(Carve &c, long T, int H, int I, int E, int k, RouteBu
     const size_t cap = (size_t)r.max_blocks * r.block_m;
     uint16_t *hp = c.take<uint16_t>((tcp ? cap : (size_t)T * k) * I);
     uint16_t *yp = c.take<uint16_t>((size_t)T * k * H);  // weighted slot rows (bf16) for the combine
-    uint16_t *xgp = tcp ? c.take<uint16_t>(cap * H) : nullptr;
-    // small blocks of the tensor-core schedule: h in slot order, natural feature order
+    uint16_t *xgp = tcp ? c.take<uint16_t>(cap * H) : nullptr;  // routed rows of x in aligned order
+    // small blocks of the tensor-core schedule: h in slot order
     uint16_t *hsp = tcp ? c.take<uint16_t>((size_t)T * k * I) : nullptr;
     if (rb) *rb = r;
     if (h) *h = hp;
@@ -219,7 +237,9 @@ static size_t fp8_layout(Carve &c, long T, int H, int I, int E, int k, RouteBufs
     const int Es = E_sched > 0 ? E_sched : E;
     const bool tcp = fp8_use_tc(T, k, Es);
     RouteBufs r = carve_route(c, T, k, E, tcp ? 128 : pick_block_m(T, k, Es));
-    const size_t cap = (size_t)T * k + (size_t)E * (r.block_m - 1);   // aligned rows
+    // aligned rows: every block the alignment can form (the tensor-core kernels index the
+    // group-major scale arrays [groups, cap] with this row count)
+    const size_t cap = (size_t)r.max_blocks * r.block_m;
     const size_t hrows = tcp ? cap : (size_t)T * k;                     // h rows: aligned or by slot
     uint8_t *xqp = c.take<uint8_t>((size_t)T * H);
     float *xsp = c.take<float>((size_t)T * (H / 128));
@@ -365,6 +385,7 @@ static int w4_layer_forward(int fmt, const char *name, const uint16_t *x, const 
                             size_t ws_bytes, void *stream, const float *g13 = nullptr, const float *g2 = nullptr,
                             int ep_base = 0, int ep_local = 0)
 {
+    host_time::Scope host_scope;
     g_err[0] = 0;
     int rc = check_layer_shape(T, H, I, E, k);
     if (rc) return rc;
@@ -413,7 +434,7 @@ static int w4_layer_forward(int fmt, const char *name, const uint16_t *x, const 
         const int cap = r.max_blocks * r.block_m;
         {
             trace::Scope ts(trace::GATHER, s);
-            launch_gather_bf16_perm(x, H, k, r.sorted, r.ntp, n, cap, kW4SmallRows, xg, num_sms(), s);
+            launch_gather_bf16(x, H, k, r.sorted, r.ntp, n, cap, kW4SmallRows, xg, num_sms(), s, fmt == W4_INT4);
         }
         W4TcArgs t{};
         t.fmt = fmt;
@@ -630,10 +651,12 @@ int moe_mxfp4_prepack_scales(const uint8_t *ue8m0, long long n, uint16_t *factor
 // then the down-mode kernels with unit weights write each real row of C).
 // ------------------------------------------------------------------------------------------
 
+static bool grouped_use_tc(int rows_hint) { return rows_hint >= 16; }  // same rule as the layer: rows per expert
+
 static size_t grouped_layout(Carve &c, long M, int K, int G, int rows_hint, RouteBufs *rb, int32_t **ids,
                              uint16_t **xg)
 {
-    const bool tcp = rows_hint >= 16;  // same rule as the layer: rows per expert
+    const bool tcp = grouped_use_tc(rows_hint);
     int32_t *idp = c.take<int32_t>((size_t)M);
     RouteBufs r = carve_route(c, M, 1, G, tcp ? 256 : pick_block_m((long)rows_hint * G, 1, G));
     uint16_t *xgp = tcp ? c.take<uint16_t>((size_t)r.max_blocks * r.block_m * K) : nullptr;
@@ -671,6 +694,7 @@ static int grouped_forward(const char *name, const uint16_t *A, long M, int K, c
                            int G, int N, const int32_t *m_indices, const int32_t *masked_m, int max_m, int rows_hint,
                            uint16_t *C, void *ws, size_t ws_bytes, void *stream)
 {
+    host_time::Scope host_scope;
     MOEQ_REQUIRE(A);
     MOEQ_REQUIRE(wq);
     MOEQ_REQUIRE(wsc);
@@ -717,7 +741,7 @@ static int grouped_forward(const char *name, const uint16_t *A, long M, int K, c
         int *status = device_status_ptr();
         if (!status) return set_error(MOEQ_ERR_CUDA, "%s: no device status word", name);
         const int cap = r.max_blocks * r.block_m;
-        launch_gather_bf16_perm(A, K, 1, r.sorted, r.ntp, n, cap, kW4SmallRows, xg, num_sms(), s);
+        launch_gather_bf16(A, K, 1, r.sorted, r.ntp, n, cap, kW4SmallRows, xg, num_sms(), s, true);
         W4TcArgs t{};
         t.status = status;
         t.E = G;
@@ -791,6 +815,7 @@ static int fp8_layer_forward(const char *name, const uint16_t *x, const float *l
                              uint16_t *out, int32_t *topk_ids_out, float *topk_w_out, void *ws, size_t ws_bytes,
                              void *stream, int ep_base, int ep_local)
 {
+    host_time::Scope host_scope;
     g_err[0] = 0;
     int rc = check_layer_shape(T, H, I, E, k);
     if (rc) return rc;
@@ -946,6 +971,7 @@ int moe_w8a8_block_fp8_forward_ep(const uint16_t *x, const float *logits, int T,
 int w8a8_block_fp8_matmul(const uint8_t *A, const float *As, const uint8_t *B, const float *Bs, int M, int N, int K,
                           int block_n, int block_k, uint16_t *C, void *stream)
 {
+    host_time::Scope host_scope;
     g_err[0] = 0;
     if (block_n != 128 || block_k != 128)
         return set_error(MOEQ_ERR_UNSUPPORTED, "block_size must be [128, 128] (got [%d, %d])", block_n, block_k);
@@ -961,7 +987,7 @@ int w8a8_block_fp8_matmul(const uint8_t *A, const float *As, const uint8_t *B, c
     if (reinterpret_cast<uintptr_t>(A) % 16 || reinterpret_cast<uintptr_t>(B) % 16 || reinterpret_cast<uintptr_t>(C) % 16)
         return set_error(MOEQ_ERR_UNSUPPORTED, "w8a8_block_fp8_matmul: A, B and C must be 16-byte aligned");
     // up to 64 rows: swap-AB tiles with K split over a cluster (HBM bound); more rows: 128-row
-    // activation tiles (CTA pairs from 256 rows)
+    // activation tiles
     Fp8TcArgs t{};
     t.a_scale = As;
     t.b_scale = Bs;
@@ -982,6 +1008,7 @@ int w8a8_block_fp8_matmul(const uint8_t *A, const float *As, const uint8_t *B, c
 int w8a8_channel_fp8_matmul(const uint8_t *A, const float *As, const uint8_t *B, const float *Bs, int M, int N, int K,
                             uint16_t *C, void *stream)
 {
+    host_time::Scope host_scope;
     g_err[0] = 0;
     if (M < 0 || N < 1 || K < 1) return set_error(MOEQ_ERR_INVALID_ARG, "bad sizes M=%d N=%d K=%d", M, N, K);
     if (K % 128) return set_error(MOEQ_ERR_UNSUPPORTED, "K must be a multiple of 128 (got %d)", K);
@@ -1046,6 +1073,23 @@ int moe_trace_read(double *stage_ms, long long *stage_calls, int n_stages, int r
     if (reset)
         for (int i = 0; i < trace::NSTAGE; ++i) { trace::sum_ms[i] = 0.0; trace::calls[i] = 0; }
     return trace::NSTAGE;
+}
+
+int moe_host_stats(double *host_us, long long *calls, long long *tmap_encoded, long long *tmap_reused, int reset)
+{
+    g_err[0] = 0;
+    long long hits = 0, misses = 0;
+    tmap_memo_stats(&hits, &misses);
+    const long long n = host_time::calls.load(std::memory_order_relaxed);
+    if (host_us) *host_us = host_time::ns.load(std::memory_order_relaxed) * 1e-3;
+    if (calls) *calls = n;
+    if (tmap_encoded) *tmap_encoded = misses;
+    if (tmap_reused) *tmap_reused = hits;
+    if (reset) {
+        host_time::ns.store(0, std::memory_order_relaxed);
+        host_time::calls.store(0, std::memory_order_relaxed);
+    }
+    return MOEQ_OK;
 }
 
 int moe_selftest_bounded_wait(void *stream)

@@ -127,6 +127,32 @@ __device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b)
     return r;
 }
 
+__device__ __forceinline__ uint32_t f16x2_sub(uint32_t a, uint32_t b)
+{
+    uint32_t r;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t f16x2_mul(uint32_t a, uint32_t b)
+{
+    uint32_t r;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+// Two f32 -> f16x2 (nearest even), lo in bits [0,16).
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi)
+{
+    uint32_t u;
+    asm("cvt.rn.f16x2.f32 %0, %2, %1;" : "=r"(u) : "f"(lo), "f"(hi));
+    return u;
+}
+
+// bf16x2 -> f16x2: exact for magnitudes in [2^-14, 65504] (8 significant bits fit the f16
+// significand); smaller ones round into the f16 subnormals (absolute error at most 2^-25).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) { return pack_f16x2(bf16_lo(v), bf16_hi(v)); }
+
 __device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b)
 {
     uint32_t r;

@@ -99,7 +99,7 @@ struct W4TcArgs {
     const int32_t *ntp;
     int n_slots;
     const float *topk_w;
-    uint16_t *h_out;        // gate/up: [M, N] bf16, pair-permuted inside 8-element chunks
+    uint16_t *h_out;        // gate/up: [M, N], bf16 values (stored as f16 for the INT4 format)
     uint16_t *ys;           // down: [n_slots, N] bf16, routing weight applied
     int small_rows;         // blocks with at most this many real rows are left to the register-fed path
     int tiles_per_cta;      // down: output tiles of 128 rows per CTA (set by the launcher)
@@ -142,11 +142,14 @@ int launch_fp8_tc_skinny(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B,
 // each, per expert_ids / ntp) and weights W [E * rows_per_expert, K]; mode TC_GATEUP or TC_DOWN.
 int launch_fp8_tc_grouped(const Fp8TcArgs &a, int mode, const uint8_t *A, const uint8_t *W, int E, int max_blocks,
                           cudaStream_t s);
-// tcgen05 W4A16 grouped GEMM over aligned activation rows (bf16 [M, K], pair-permuted); mode
-// TC_GATEUP (h = silu(gate) * up, written pair-permuted) or TC_DOWN (weighted slot rows).
+// tcgen05 W4A16 grouped GEMM over aligned bf16 activation rows act [M, K]; mode TC_GATEUP (h =
+// silu(gate) * up in aligned order) or TC_DOWN (weighted slot rows).
 int launch_w4a16_tc(const W4TcArgs &a, int mode, const uint16_t *act, int max_blocks, cudaStream_t s);
-void launch_gather_bf16_perm(const uint16_t *x, int H, int k, const int32_t *sorted_ids, const int32_t *ntp,
-                             int n_slots, int cap_rows, int small_rows, uint16_t *xg, int num_sms, cudaStream_t s);
+// Copies the routed rows of x into aligned order (row r takes x[sorted_ids[r] / k]); only the rows
+// the tensor-core MMAs read (see the kernel). to_f16: the copies are converted to f16 (the INT4
+// tensor-core GEMMs compute in f16).
+void launch_gather_bf16(const uint16_t *x, int H, int k, const int32_t *sorted_ids, const int32_t *ntp, int n_slots,
+                        int cap_rows, int small_rows, uint16_t *xg, int num_sms, cudaStream_t s, bool to_f16);
 // Copies E4M3 rows (and their scales) of the routed slots into aligned order: row r takes token
 // sorted_ids[r] / k; padding rows become zero.
 void launch_gather_fp8_rows(const uint8_t *xq, const float *xs, int H, int k, const int32_t *sorted_ids,

@@ -355,14 +355,26 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t *__restrict
         const long t = i / H8;
         const int c = (int)(i - t * H8);
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int j = 0; j < k; ++j) {
-            if (local_ids && __ldg(local_ids + (size_t)t * k + j) < 0) continue;
-            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(ys + ((size_t)t * k + j) * H) + c);
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        const uint16_t *row0 = ys + (size_t)t * k * H;
+        // up to 8 slot rows in flight per thread (the rows are read once: no L1 allocation), then
+        // summed in slot order
+        for (int j0 = 0; j0 < k; j0 += 8) {
+            uint4 v[8];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                acc[2 * q] += __uint_as_float(w[q] << 16);
-                acc[2 * q + 1] += __uint_as_float(w[q] & 0xFFFF0000u);
+            for (int jj = 0; jj < 8; ++jj) {
+                const int j = j0 + jj;
+                const bool use = j < k && !(local_ids && __ldg(local_ids + (size_t)t * k + j) < 0);
+                v[jj] = use ? ld_stream_v4(reinterpret_cast<const uint4 *>(row0 + (size_t)j * H) + c)
+                            : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) {
+                const uint32_t w[4] = {v[jj].x, v[jj].y, v[jj].z, v[jj].w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    acc[2 * q] += __uint_as_float(w[q] << 16);
+                    acc[2 * q + 1] += __uint_as_float(w[q] & 0xFFFF0000u);
+                }
             }
         }
         uint4 o;

@@ -1,6 +1,7 @@
 // Host utilities of the tensor-core kernels: TMA tensor maps (encoded through the driver entry
 // point, so the library needs no link-time dependency on libcuda) and the device status word that
 // kernels with bounded waits write when a wait gives up.
+#include <atomic>
 #include <mutex>
 
 #include "tc_common.cuh"
@@ -18,9 +19,47 @@ EncodeTiledFn g_encode = nullptr;
 int *g_status_addr[64] = {};
 }  // namespace
 
+// Memo of encoded tensor maps. A tensor map is a pure function of its parameters (address,
+// type, extents, pitch, box, swizzle), so a repeated call with the same buffers reuses the
+// encoding instead of going through the driver again ("vLLM x Novita AI: Chord W4A16 INT4 MoE
+// Kernel for Kimi K2.x", section "SM90 grouped kernels": descriptors memoized per shape, about
+// 30 us of host work per small decode launch saved). A small ring, most recent first.
+namespace {
+struct TmapKey {
+    const void *base;
+    int dtype, elem_bytes;
+    uint64_t rows, cols;
+    uint32_t box_rows, box_cols;
+    bool swizzle128;
+    bool operator==(const TmapKey &o) const
+    {
+        return base == o.base && dtype == o.dtype && elem_bytes == o.elem_bytes && rows == o.rows && cols == o.cols &&
+               box_rows == o.box_rows && box_cols == o.box_cols && swizzle128 == o.swizzle128;
+    }
+};
+constexpr int kTmapMemo = 64;
+std::mutex g_memo_mu;
+TmapKey g_memo_key[kTmapMemo];
+CUtensorMap g_memo_map[kTmapMemo];
+int g_memo_n = 0, g_memo_next = 0;
+std::atomic<long long> g_memo_hits{0}, g_memo_misses{0};
+}  // namespace
+
 int make_tmap_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype, int elem_bytes, uint64_t rows,
                  uint64_t cols, uint32_t box_rows, uint32_t box_cols, bool swizzle128)
 {
+    const TmapKey key{base, (int)dtype, elem_bytes, rows, cols, box_rows, box_cols, swizzle128};
+    {
+        std::lock_guard<std::mutex> g(g_memo_mu);
+        for (int i = 0; i < g_memo_n; ++i) {
+            const int j = (g_memo_next - 1 - i + kTmapMemo) % kTmapMemo;
+            if (g_memo_key[j] == key) {
+                *map = g_memo_map[j];
+                g_memo_hits.fetch_add(1, std::memory_order_relaxed);
+                return MOEQ_OK;
+            }
+        }
+    }
     {
         std::lock_guard<std::mutex> g(g_mu);
         if (!g_encode) {
@@ -46,7 +85,19 @@ int make_tmap_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype, 
                                 swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return set_error(MOEQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+    g_memo_misses.fetch_add(1, std::memory_order_relaxed);
+    std::lock_guard<std::mutex> g(g_memo_mu);
+    g_memo_key[g_memo_next] = key;
+    g_memo_map[g_memo_next] = *map;
+    g_memo_next = (g_memo_next + 1) % kTmapMemo;
+    if (g_memo_n < kTmapMemo) ++g_memo_n;
     return MOEQ_OK;
+}
+
+void tmap_memo_stats(long long *hits, long long *misses)
+{
+    if (hits) *hits = g_memo_hits.load(std::memory_order_relaxed);
+    if (misses) *misses = g_memo_misses.load(std::memory_order_relaxed);
 }
 
 // A wait that can never complete (nothing arrives on the barrier), given a short poll limit: the

@@ -16,16 +16,16 @@
 // A tile serves up to 256 tokens, so each dequantized weight feeds 256 rows of MMA work: the
 // dequantization, not the MMA, bounds this kernel, and the wide tile halves it per FLOP. The
 // MMA's N is the block's real row count rounded up to 16, so padding rows cost no MMA work.
-// The nibble pairs that one shift + LOP3 extracts, (q0,q4) (q1,q5) (q2,q6) (q3,q7) of each
-// 32-bit word, become consecutive K in tensor memory, so the activations are stored with the
-// same order inside every 8-element chunk (done by the gather and by the gate/up epilogue).
+// One shift + LOP3 extracts the nibble pairs (q0,q4) (q1,q5) (q2,q6) (q3,q7) of a 32-bit code
+// word; four byte permutes put them in natural order, so the activation rows keep their own order:
+// the gather copies the routed rows of x as they are, and h is written in natural order.
 //
 // CTA = one 256-row activation block of one expert x (gate/up: 64 features, gate rows in tensor
 // lanes 0-63 and the matching up rows in lanes 64-127; down: 128 output rows):
 //   warp 0      TMA producer of the activation tiles [256 tokens x 128 inputs] (3 stages, two
-//               128-byte-swizzled halves of 64 inputs each); a
-//               tile's bytes complete on the same "stage ready" barrier the dequantization warps
-//               arrive on, and one commit per step frees both the weight stage and the tile;
+//               128-byte-swizzled halves of 64 inputs each); a tile's bytes complete on the same
+//               "stage ready" barrier the dequantization warps arrive on, and one commit per step
+//               frees both the weight stage and the tile;
 //   warp 1      tensor-memory allocation; lane 0 issues 8 MMAs (K = 16) per 128-input step into
 //               the one accumulator and commits. On sm_100a a pipeline step costs several hundred
 //               cycles of synchronization whatever work it carries (an MMA issue ~50-65 cycles, a
@@ -36,8 +36,8 @@
 //               a private 3-deep cp.async ring, and writes the dequantized slice to one of 3
 //               tensor-memory
 //               stages; then the epilogue: gate/up passes the up values through shared memory
-//               to the warps holding the gate values, which write h = bf16(silu(g) * u) in the
-//               permuted order; down writes the routing-weighted bf16 slot rows.
+//               to the warps holding the gate values, which write h = bf16(silu(g) * u); down
+//               writes the routing-weighted bf16 slot rows.
 #include "kernels.cuh"
 #include "tc_common.cuh"
 
@@ -71,28 +71,31 @@ static_assert(64 * kTok * 4 <= kBStages * kBTile, "gate/up exchange fits in the 
 
 // (q - 8) * scale (INT4) or E2M1(q) * 2^(s - 1) (FP4, see e2m1_pair_pre) in bf16 for the pairs
 // (q0,q4) (q1,q5) (q2,q6) (q3,q7) of one code word
+// INT4 runs in f16: (q - 8) * s has up to 11 significant bits (a 3-bit integer times the 8-bit
+// significand of a bf16 scale), which f16 holds exactly and bf16 does not; the f16 MMA then sees
+// the exact weights, and the bf16 activations, converted to f16, exactly too (within the f16 range).
+// MXFP4 / NVFP4 weights are exact in bf16 and stay there.
 template <int FMT>
 __device__ __forceinline__ void dequant4(uint32_t w, uint32_t scale2, uint32_t *out)
 {
+    uint32_t p[4];  // the pairs one shift + LOP3 yields: (q0,q4) (q1,q5) (q2,q6) (q3,q7)
     if (FMT == W4_FP4 || FMT == W4_NV) {
-        out[0] = bf16x2_mul(e2m1_pair_pre<0>(w), scale2);
-        out[1] = bf16x2_mul(e2m1_pair_pre<1>(w), scale2);
-        out[2] = bf16x2_mul(e2m1_pair_pre<2>(w), scale2);
-        out[3] = bf16x2_mul(e2m1_pair_pre<3>(w), scale2);
+        p[0] = bf16x2_mul(e2m1_pair_pre<0>(w), scale2);
+        p[1] = bf16x2_mul(e2m1_pair_pre<1>(w), scale2);
+        p[2] = bf16x2_mul(e2m1_pair_pre<2>(w), scale2);
+        p[3] = bf16x2_mul(e2m1_pair_pre<3>(w), scale2);
     } else {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const uint32_t v = lop3_and_or(w >> (4 * i), 0x000F000Fu, 0x43004300u);  // 128 + q, exact
-            out[i] = bf16x2_mul(bf16x2_sub(v, 0x43084308u), scale2);                  // (q - 8), then * s
+            const uint32_t v = lop3_and_or(w >> (4 * i), 0x000F000Fu, 0x64006400u);  // f16 1024 + q, exact
+            p[i] = f16x2_mul(f16x2_sub(v, 0x64086408u), scale2);                      // (q - 8) * s, exact
         }
     }
-}
-
-// position of feature f inside its 8-element chunk after the pair permutation
-__device__ __forceinline__ int perm_pos(int f)
-{
-    const int i = f & 7;
-    return (f & ~7) + (i < 4 ? 2 * i : 2 * (i - 4) + 1);
+    // natural order (q0,q1) (q2,q3) (q4,q5) (q6,q7): the activation rows need no reordering
+    out[0] = prmt(p[0], p[1], 0x5410u);
+    out[1] = prmt(p[2], p[3], 0x5410u);
+    out[2] = prmt(p[0], p[1], 0x7632u);
+    out[3] = prmt(p[2], p[3], 0x7632u);
 }
 
 template <int MODE, int FMT>
@@ -176,7 +179,8 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            const uint32_t idesc = tc::idesc_f32(tc::kFmtBF16, tc::kFmtBF16, 128, n_mma);
+            constexpr uint32_t kFmt = FMT == W4_INT4 ? tc::kFmtF16 : tc::kFmtBF16;
+            const uint32_t idesc = tc::idesc_f32(kFmt, kFmt, 128, n_mma);
             // lean issue path: stage bases precomputed, the first step peeled, then MMAs that always
             // accumulate (the dequantization warps keep this SM's issue slots busy)
             const uint32_t a_base = tmem + kAccCols;
@@ -271,7 +275,8 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
             const uint32_t sc = *reinterpret_cast<const uint32_t *>(scale_slot(slot));
             issue();  // step gs + kRing - 1: refills the slot read in step gs - 1
             // this slice's group scale, twice (group 16: words 0-1 the first, words 2-3 the second)
-            const uint32_t s2 = prmt(sc, sc, (FMT != W4_NV && (kq & 1)) ? 0x3232u : 0x1010u);
+            uint32_t s2 = prmt(sc, sc, (FMT != W4_NV && (kq & 1)) ? 0x3232u : 0x1010u);
+            if (FMT == W4_INT4) s2 = bf16x2_to_f16x2(s2);  // the group scale in f16 (exact in range)
             const uint32_t s2h = FMT == W4_NV ? prmt(sc, sc, 0x3232u) : s2;
             uint32_t pairs[16];
             dequant4<FMT>(c.x, s2, pairs + 0);
@@ -318,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
             asm volatile("bar.sync 1, %0;" ::"n"(kDeqThreads) : "memory");
             if (ok && quarter < 2) {
                 const int f = n0 + row;
-                uint16_t *hcol = a.h_out + perm_pos(f);
+                uint16_t *hcol = a.h_out + f;
                 for (int c = 0; c < kTok / kSplit / 32; ++c) {
                     const int tok0 = kq * (kTok / kSplit) + c * 32;
                     if (tok0 >= n_mma) break;
@@ -328,7 +333,10 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         const float hv = silu_f32(gsc * __uint_as_float(g[j])) * up_s[(tok0 + j) * 64 + row];
-                        hcol[(size_t)(r0 + tok0 + j) * a.N] = f32_to_bf16(hv);
+                        // h = bf16(a); the INT4 down GEMM reads it as f16 (the same value)
+                        const uint16_t hb = f32_to_bf16(hv);
+                        hcol[(size_t)(r0 + tok0 + j) * a.N] =
+                            FMT == W4_INT4 ? (uint16_t)(pack_f16x2(__uint_as_float((uint32_t)hb << 16), 0.f) & 0xFFFFu) : hb;
                     }
                 }
             }
@@ -368,15 +376,15 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
     if (warp == 1) tc::tmem_dealloc(tmem, kTmemCols);
 }
 
-// Gather of bf16 activation rows into aligned order with the pair permutation inside every
-// 8-element chunk; one warp per row. Only the rows the MMAs read are written: the real rows and
-// the zero padding up to the block's real count rounded up to 16 (the MMA's N); blocks with at
-// most small_rows real rows belong to the register-fed kernel, which reads x itself.
-__global__ void __launch_bounds__(256) gather_bf16_perm_kernel(const uint16_t *__restrict__ x, int H, int k,
-                                                               const int32_t *__restrict__ sorted_ids,
-                                                               const int32_t *__restrict__ ntp, int n_slots,
-                                                               int cap_rows, int small_rows,
-                                                               uint16_t *__restrict__ xg)
+// Gather of bf16 activation rows into aligned order (row r takes row sorted_ids[r] / k of x),
+// converted to f16 for the INT4 GEMMs (TO_F16); one warp per row, 16-byte copies. Only the rows the MMAs read are written: the real rows and the zero
+// padding up to the block's real count rounded up to 16 (the MMA's N); blocks with at most
+// small_rows real rows belong to the register-fed kernel, which reads x itself.
+template <bool TO_F16>
+__global__ void __launch_bounds__(256) gather_bf16_kernel(const uint16_t *__restrict__ x, int H, int k,
+                                                          const int32_t *__restrict__ sorted_ids,
+                                                          const int32_t *__restrict__ ntp, int n_slots, int cap_rows,
+                                                          int small_rows, uint16_t *__restrict__ xg)
 {
     const int lane = threadIdx.x & 31;
     const int rows = min(__ldg(ntp), cap_rows);
@@ -391,13 +399,12 @@ __global__ void __launch_bounds__(256) gather_bf16_perm_kernel(const uint16_t *_
         const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)(real ? slot / k : 0) * H);
         uint4 *dst = reinterpret_cast<uint4 *>(xg + (size_t)r * H);
         for (int i = lane; i < H / 8; i += 32) {
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (real) {
-                const uint4 u = __ldg(src + i);
-                v.x = prmt(u.x, u.z, 0x5410u);  // (x0, x4)
-                v.y = prmt(u.x, u.z, 0x7632u);  // (x1, x5)
-                v.z = prmt(u.y, u.w, 0x5410u);  // (x2, x6)
-                v.w = prmt(u.y, u.w, 0x7632u);  // (x3, x7)
+            uint4 v = real ? ld_stream_v4(src + i) : make_uint4(0u, 0u, 0u, 0u);
+            if (TO_F16) {
+                v.x = bf16x2_to_f16x2(v.x);
+                v.y = bf16x2_to_f16x2(v.y);
+                v.z = bf16x2_to_f16x2(v.z);
+                v.w = bf16x2_to_f16x2(v.w);
             }
             dst[i] = v;
         }
@@ -443,12 +450,15 @@ int launch_w4a16_tc(const W4TcArgs &a_in, int mode, const uint16_t *act, int max
     return launch_mode<TC_DOWN, W4_INT4>(a, tm, gx, max_blocks, s);
 }
 
-void launch_gather_bf16_perm(const uint16_t *x, int H, int k, const int32_t *sorted_ids, const int32_t *ntp,
-                             int n_slots, int cap_rows, int small_rows, uint16_t *xg, int num_sms, cudaStream_t s)
+void launch_gather_bf16(const uint16_t *x, int H, int k, const int32_t *sorted_ids, const int32_t *ntp, int n_slots,
+                        int cap_rows, int small_rows, uint16_t *xg, int num_sms, cudaStream_t s, bool to_f16)
 {
     if (cap_rows <= 0) return;
     const int blocks = min(cdiv(cap_rows, 8), num_sms * 8);
-    gather_bf16_perm_kernel<<<blocks, 256, 0, s>>>(x, H, k, sorted_ids, ntp, n_slots, cap_rows, small_rows, xg);
+    if (to_f16)
+        gather_bf16_kernel<true><<<blocks, 256, 0, s>>>(x, H, k, sorted_ids, ntp, n_slots, cap_rows, small_rows, xg);
+    else
+        gather_bf16_kernel<false><<<blocks, 256, 0, s>>>(x, H, k, sorted_ids, ntp, n_slots, cap_rows, small_rows, xg);
 }
 
 }  // namespace moeq

@@ -83,3 +83,32 @@ def sample_tokens(d: dict, n: int, seed: int = 0) -> np.ndarray:
     while len(pick) < n:
         pick.add(int(rng.integers(0, T)))
     return np.array(sorted(pick), dtype=np.int32)
+
+
+def block_tokens(d: dict, block_m: int, small_rows: int = 0, n_sampled: int = 0, seed: int = 0) -> np.ndarray:
+    """Tokens whose outputs run through chosen blocks of the aligned routing (the oracle's routing
+    and alignment): every token of the most loaded expert's first and last block_m-row block, every
+    token of one block with at most `small_rows` real rows (the few-row tail), and n_sampled more
+    tokens from the seeded sample."""
+    import oracle
+    logits = W.np_bits(d["logits"])
+    ids, _ = oracle.route_topk(logits, d["k"])
+    sorted_ids, expert_ids, ntp = oracle.align(ids, d["E"], block_m)
+    n_slots = ids.size
+    counts = np.bincount(ids.ravel(), minlength=d["E"])
+    heavy = int(np.argmax(counts))
+    blocks = [b for b in range(ntp // block_m) if expert_ids[b] == heavy]
+    pick = set()
+    for b in (blocks[0], blocks[-1]):
+        rows = sorted_ids[b * block_m:(b + 1) * block_m]
+        pick.update(int(s) // d["k"] for s in rows if s < n_slots)
+    if small_rows:
+        for b in range(ntp // block_m):
+            rows = sorted_ids[b * block_m:(b + 1) * block_m]
+            real = rows[rows < n_slots]
+            if 0 < real.size <= small_rows:
+                pick.update(int(s) // d["k"] for s in real)
+                break
+    if n_sampled:
+        pick.update(int(t) for t in sample_tokens(d, n_sampled, seed))
+    return np.array(sorted(pick), dtype=np.int32)

@@ -265,3 +265,15 @@ def test_noalloc_binding_checks_shapes(L):
         moeq.moe_w4a16_forward_noalloc(x, m(3, 4, dt=f32), 2, *good)
     with pytest.raises(ValueError, match="out"):
         moeq.moe_w4a16_forward_noalloc(x, lg, 2, *good, out=m(2, 128, dt=bf))
+
+
+def test_host_stats_counts_calls_without_a_device(L):
+    """moe_host_stats reads host-side counters only. A call rejected during validation still
+    counts its (host) time."""
+    s0 = moeq.moe_host_stats(reset=True)
+    assert s0["host_us"] >= 0 and s0["calls"] >= 0
+    N = None
+    rc = L.moe_w4a16_forward(N, N, 4, 7168, 2048, 384, 0, N, N, N, N, N, N, N, N, 0, N)  # k = 0: rejected
+    assert rc != 0
+    s1 = moeq.moe_host_stats()
+    assert s1["calls"] == 1 and s1["host_us"] >= 0

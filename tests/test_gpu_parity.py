@@ -9,7 +9,7 @@ import torch
 import oracle
 import quantized_mixture_experts_align_b200 as moeq
 import workloads as W
-from tests._util import (TOL_FP8, TOL_W4A16, assert_layer_close, bf16_to_f64, oracle_layer,
+from tests._util import (TOL_FP8, TOL_W4A16, assert_layer_close, bf16_to_f64, block_tokens, oracle_layer,
                          sample_tokens)
 
 pytestmark = pytest.mark.gpu
@@ -213,6 +213,16 @@ def test_w4a16_prefill_sampled():
     _layer_parity(d, sample_tokens(d, 10), TOL_W4A16, "prefill_w4a16")
 
 
+def test_w4a16_prefill_heavy_and_tail_blocks():
+    """Full prefill shapes (T = 8192, Zipf routing): every token of the most loaded expert's first
+    and last 256-row tensor-core block, and every token of one block with at most 8 real rows (the
+    register-fed side of the schedule)."""
+    d = workload("prefill_w4a16")
+    toks = block_tokens(d, 256, small_rows=8)
+    assert toks.size > 256
+    _layer_parity(d, toks, TOL_W4A16, "prefill_w4a16 heavy/tail blocks")
+
+
 @pytest.mark.parametrize("T,E,k,H,I,logit_mode", [
     (1, 8, 2, 512, 256, "normal"),        # one token
     (200, 8, 1, 512, 256, "one"),         # every token on one expert (block_m 64, ragged tail)
@@ -259,6 +269,16 @@ def test_fp8_moe_small_all_tokens():
 def test_fp8_moe_full_sampled():
     d = workload("moe_fp8")
     _layer_parity(d, sample_tokens(d, 8), TOL_FP8, "moe_fp8")
+
+
+def test_fp8_moe_full_heavy_tail_blocks_and_sampled():
+    """Full block-FP8 MoE shapes (T = 4096, E = 256, Zipf routing): every token of the most loaded
+    expert's first and last 128-row block, every token of one block with at most 8 real rows, and
+    64 sampled tokens."""
+    d = workload("moe_fp8")
+    toks = block_tokens(d, 128, small_rows=8, n_sampled=64, seed=3)
+    assert toks.size > 192
+    _layer_parity(d, toks, TOL_FP8, "moe_fp8 heavy/tail blocks + sampled")
 
 
 @pytest.mark.parametrize("T,E,k,H,logit_mode", [
@@ -369,3 +389,21 @@ def test_dense_fp8_closed_form_ones():
     Bs = torch.full((N // 128, K // 128), 0.5 / 448.0, device=DEV)
     C = moeq.w8a8_block_fp8_matmul(A, As, B, Bs).float().cpu().numpy()
     assert np.all(np.abs(C - 0.5 * K) <= 0.5 * K * 2 ** -8)
+
+
+def test_tensor_map_memo_reuses_encodings():
+    """A repeated tensor-core call on the same buffers reuses its encoded tensor maps (no driver
+    encode), and a call on other buffers encodes new ones; the results are unchanged."""
+    d = W.make_moe(W.WORKLOADS["moe_fp8"], device=DEV, T=256, E=8, k=2, H=512, I=256)
+    ws = moeq.workspace(moeq.moe_w8a8_block_fp8_workspace_size(256, 512, 256, 8, 2), DEV)
+    out1 = _forward(d, ws=ws)
+    s0 = moeq.moe_host_stats()
+    out2 = _forward(d, ws=ws)
+    s1 = moeq.moe_host_stats()
+    torch.cuda.synchronize()
+    assert s1["tmap_encoded"] == s0["tmap_encoded"] and s1["tmap_reused"] >= s0["tmap_reused"] + 4
+    assert s1["calls"] == s0["calls"] + 1 and s1["host_us"] > s0["host_us"]
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+    ws2 = moeq.workspace(ws.numel() + 4096, DEV)
+    _forward(d, ws=ws2)
+    assert moeq.moe_host_stats()["tmap_encoded"] > s1["tmap_encoded"]

@@ -1,12 +1,15 @@
 """Whole-layer CUDA-graph capture through the C ABI: every entry point is asynchronous on the
 caller's stream and makes no host synchronization, so a forward captured into a CUDA graph must
 replay to exactly the bytes an eager call writes (the kernels are deterministic), also after the
-inputs are overwritten in place between replays."""
+inputs are overwritten in place between replays; the replay on the new inputs is also checked
+against the oracle."""
+import numpy as np
 import pytest
 import torch
 
 import quantized_mixture_experts_align_b200 as moeq
 import workloads as W
+from tests._util import TOL_FP8, TOL_W4A16, assert_layer_close, bf16_to_f64, oracle_layer
 
 pytestmark = pytest.mark.gpu
 
@@ -71,6 +74,12 @@ def test_layer_graph_replay_matches_eager(case):
         fwd(out_eager)
         torch.cuda.synchronize()
         assert torch.equal(out_graph.view(torch.int16), out_eager.view(torch.int16)), f"{case} trial {trial}"
+    # the replay on the inputs written in place, against the oracle on those inputs (tokens
+    # sampled from the decode workload, all tokens of the small ones)
+    d_new = dict(d, x=x_in, logits=lg_in)
+    toks = np.arange(T, dtype=np.int32) if T <= 512 else np.arange(0, T, max(1, T // 16), dtype=np.int32)
+    assert_layer_close(bf16_to_f64(out_graph[torch.as_tensor(toks, device=DEV).long()]), oracle_layer(d_new, toks),
+                       TOL_W4A16 if w4 else TOL_FP8, f"{case} graph replay vs oracle")
     assert moeq.moe_device_status() == 0
 
 
