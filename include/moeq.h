@@ -217,7 +217,7 @@ MOEQ_API int moe_nvfp4_forward_ep(const uint16_t *x, const float *logits, int T,
  *    library; every GPU that loads the library holds it until the process exits.
  *  - Shapes whose moe_w4a16_workspace_size() exceeds that size are rejected with
  *    MOEQ_ERR_WORKSPACE before anything is enqueued (at H=7168, I=2048, E=384, k=8 the limit is
- *    T <= 113 tokens).
+ *    T <= 103 tokens).
  *  - The call allocates nothing: no cudaMalloc, cudaFree or other allocating routine.
  *  - The first call on each device does a one-time set-up, the lookup of the array's device
  *    address (cudaGetSymbolAddress, with that device current); make that first call before any

@@ -204,8 +204,11 @@ static_assert(kW4SmallRows == 8, "the strided register-fed instantiation is buil
 // E: experts whose weights the call holds (the alignment's capacity); E_sched (0: E): experts the
 // routing picks from, whose mean load T*k/E_sched picks the schedule (under expert parallelism a
 // rank holds E of the E_sched experts, and each of them still sees T*k/E_sched rows on average).
+// fmt: the INT4 register-fed schedule also holds x converted to f16 (xh; the INT4 GEMMs compute in
+// f16), written by the routing kernel.
 static size_t w4a16_layout(Carve &c, long T, int H, int I, int E, int k, RouteBufs *rb, uint16_t **h, uint16_t **ys,
-                           uint16_t **xg = nullptr, uint16_t **h_small = nullptr, int E_sched = 0)
+                           uint16_t **xg = nullptr, uint16_t **h_small = nullptr, int E_sched = 0, int fmt = W4_INT4,
+                           uint16_t **xh = nullptr)
 {
     const int Es = E_sched > 0 ? E_sched : E;
     const bool tcp = w4_use_tc(T, k, Es);
@@ -216,11 +219,13 @@ static size_t w4a16_layout(Carve &c, long T, int H, int I, int E, int k, RouteBu
     uint16_t *xgp = tcp ? c.take<uint16_t>(cap * H) : nullptr;  // routed rows of x in aligned order
     // small blocks of the tensor-core schedule: h in slot order
     uint16_t *hsp = tcp ? c.take<uint16_t>((size_t)T * k * I) : nullptr;
+    uint16_t *xhp = (!tcp && fmt == W4_INT4) ? c.take<uint16_t>((size_t)T * H) : nullptr;
     if (rb) *rb = r;
     if (h) *h = hp;
     if (ys) *ys = yp;
     if (xg) *xg = xgp;
     if (h_small) *h_small = hsp;
+    if (xh) *xh = xhp;
     return c.used;
 }
 
@@ -370,7 +375,7 @@ size_t moe_w4a16_ep_workspace_size(int T, int H, int I, int E, int k, int ep_loc
 {
     if (check_layer_shape(T, H, I, E, k) || check_expert_range(E, 0, ep_local)) return 0;
     Carve c(nullptr);
-    return w4a16_layout(c, T, H, I, ep_local, k, nullptr, nullptr, nullptr, nullptr, nullptr, E);
+    return w4a16_layout(c, T, H, I, ep_local, k, nullptr, nullptr, nullptr, nullptr, nullptr, E);  // INT4: the largest
 }
 
 }  // extern "C"
@@ -408,9 +413,9 @@ static int w4_layer_forward(int fmt, const char *name, const uint16_t *x, const 
     cudaStream_t s = (cudaStream_t)stream;
     Carve c(ws);
     RouteBufs r;
-    uint16_t *h, *xg, *h_small;
+    uint16_t *h, *xg, *h_small, *xh;
     uint16_t *ys;
-    w4a16_layout(c, T, H, I, Ew, k, &r, &h, &ys, &xg, &h_small, E);
+    w4a16_layout(c, T, H, I, Ew, k, &r, &h, &ys, &xg, &h_small, E, fmt, &xh);
     // global picks to the caller's buffer (if any); under expert parallelism the alignment and the
     // combine take the local ids (-1 for experts held elsewhere) in the route scratch
     int32_t *ids = topk_ids_out ? topk_ids_out : (ep ? nullptr : r.ids);
@@ -421,7 +426,7 @@ static int w4_layer_forward(int fmt, const char *name, const uint16_t *x, const 
 
     {
         trace::Scope ts(trace::ROUTE, s);
-        launch_route_topk(logits, T, E, k, ids, tw, s, lids, ep_base, ep_local);
+        launch_route_topk(logits, T, E, k, ids, tw, s, lids, ep_base, ep_local, x, H, xh);
     }
     {
         trace::Scope ts(trace::ALIGN, s);
@@ -465,6 +470,7 @@ static int w4_layer_forward(int fmt, const char *name, const uint16_t *x, const 
         g.topk_w = tw;
         g.blk_stride = r.block_m;
         g.act = x;
+        g.act_bf16 = 1;  // INT4: converted in registers (the few-row blocks only)
         g.act_row_div = k;
         g.wq = w13_q;
         g.ws = w13_s;
@@ -488,6 +494,7 @@ static int w4_layer_forward(int fmt, const char *name, const uint16_t *x, const 
         t.wglobal = g2;
         t.ys = ys;
         g.act = h_small;
+        g.act_bf16 = 0;
         g.act_row_div = 1;
         g.wq = w2_q;
         g.ws = w2_s;
@@ -511,8 +518,8 @@ static int w4_layer_forward(int fmt, const char *name, const uint16_t *x, const 
         a.num_tokens_padded = r.ntp;
         a.n_slots = n;
         a.topk_w = tw;
-        // gate/up + SiLU*up
-        a.act = x;
+        // gate/up + SiLU*up (INT4: x in f16, converted by the routing kernel)
+        a.act = xh ? xh : x;
         a.act_row_div = k;
         a.wq = w13_q;
         a.ws = w13_s;
@@ -729,6 +736,7 @@ static int grouped_forward(const char *name, const uint16_t *A, long M, int K, c
     g.n_slots = n;
     g.topk_w = nullptr;  // weight 1: plain grouped GEMM
     g.act = A;
+    g.act_bf16 = 1;      // INT4 in f16: the bf16 rows are converted in registers
     g.act_row_div = 1;   // k = 1: the slot is the row
     g.wq = wq;
     g.ws = wsc;

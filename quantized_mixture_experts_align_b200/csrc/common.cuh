@@ -153,6 +153,12 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi)
 // significand); smaller ones round into the f16 subnormals (absolute error at most 2^-25).
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) { return pack_f16x2(bf16_lo(v), bf16_hi(v)); }
 
+// h = bf16(v) (nearest even), returned as the f16 bits of that value (exact in the f16 range).
+__device__ __forceinline__ uint16_t f32_to_bf16_as_f16(float v)
+{
+    return (uint16_t)(pack_f16x2(__uint_as_float((uint32_t)f32_to_bf16(v) << 16), 0.f) & 0xFFFFu);
+}
+
 __device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b)
 {
     uint32_t r;
@@ -182,6 +188,17 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
 {
     asm volatile(
         "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// D[16x8] += A[16x16] (f16, row) * B[16x8] (f16, col), f32 accumulate.
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                              uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
         "{%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));

@@ -17,7 +17,7 @@ enum { W4_INT4 = 0, W4_FP4 = 1, W4_NV = 2 };
 struct W4GroupedArgs {
     int fmt;                 // W4_INT4 / W4_FP4 / W4_NV
     const float *wglobal;    // W4_NV: f32 tensor scale per expert [E]
-    const uint16_t *act;     // gate/up: x [T, K]; down: h [T*k, K]  (bf16)
+    const uint16_t *act;     // gate/up: x [T, K]; down: h [T*k, K] (INT4: f16 values unless act_bf16)
     int act_row_div;         // activation row of a slot = slot / act_row_div (k for x, 1 for h)
     const int32_t *wq;       // [E, n_rows, K/8]
     const uint16_t *ws;      // [E, n_rows, K/32] bf16
@@ -30,7 +30,7 @@ struct W4GroupedArgs {
     const int32_t *num_tokens_padded;
     int n_slots;             // T*k; sorted_ids entries >= n_slots are padding
     const float *topk_w;     // [T*k] (down); null: weight 1 (plain grouped GEMM)
-    uint16_t *h_out;         // [T*k, I] bf16 (gate/up)
+    uint16_t *h_out;         // [T*k, I] bf16(a) values (gate/up; f16 bits for INT4)
     uint16_t *y_out;         // [T*k, H] bf16, routing weight applied (down)
     // 0: align blocks of BM rows. Otherwise the alignment has blocks of blk_stride rows and the
     // kernel takes only those with at most BM real rows (the rest belong to the tensor-core path)
@@ -39,6 +39,9 @@ struct W4GroupedArgs {
     // alignment (which waits for the alignment before it lets this kernel start), so the routing
     // buffers may be read, and the weights prefetched, before waiting for h
     int after_gateup;
+    // INT4: 1 = act holds bf16 values, converted to f16 in registers; 0 = act is already f16 (the
+    // INT4 GEMMs compute in f16, where the dequantized weights are exact)
+    int act_bf16;
 };
 
 struct F8GroupedArgs {
@@ -107,8 +110,10 @@ struct W4TcArgs {
 
 // local_ids (nullable): the picks relative to the expert range [ep_base, ep_base + ep_local), -1
 // outside it; ids may be null when local_ids is given.
+// xh (nullable): also writes x [T, H] (bf16) as f16 into xh [T, H].
 void launch_route_topk(const float *logits, int T, int E, int k, int32_t *ids, float *w, cudaStream_t s,
-                       int32_t *local_ids = nullptr, int ep_base = 0, int ep_local = 0);
+                       int32_t *local_ids = nullptr, int ep_base = 0, int ep_local = 0, const uint16_t *x = nullptr,
+                       int H = 0, uint16_t *xh = nullptr);
 // Scratch (bytes) the alignment of n slots over E experts uses; 0 = the one-CTA kernel, which
 // also runs when launch_align gets no scratch.
 size_t align_scratch_bytes(int n, int E);

@@ -20,12 +20,26 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict
                                                          int k, int32_t *__restrict__ ids,
                                                          float *__restrict__ w,
                                                          int32_t *__restrict__ local_ids, int ep_base,
-                                                         int ep_local)
+                                                         int ep_local, const uint16_t *__restrict__ x, int H,
+                                                         uint16_t *__restrict__ xh)
 {
     pdl_trigger();  // the alignment after this kernel may launch (it waits for these ids)
     const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (t >= T) return;
+    if (xh) {
+        // the token's activation row in f16 for the INT4 GEMMs (exact for magnitudes in [2^-14, 65504])
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)t * H);
+        uint4 *dst = reinterpret_cast<uint4 *>(xh + (size_t)t * H);
+        for (int i = lane; i < H / 8; i += 32) {
+            uint4 v = __ldg(src + i);
+            v.x = bf16x2_to_f16x2(v.x);
+            v.y = bf16x2_to_f16x2(v.y);
+            v.z = bf16x2_to_f16x2(v.z);
+            v.w = bf16x2_to_f16x2(v.w);
+            dst[i] = v;
+        }
+    }
     const float *row = logits + (size_t)t * E;
     float v[kMaxExperts / 32];
 #pragma unroll
@@ -72,11 +86,12 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict
 }
 
 void launch_route_topk(const float *logits, int T, int E, int k, int32_t *ids, float *w, cudaStream_t s,
-                       int32_t *local_ids, int ep_base, int ep_local)
+                       int32_t *local_ids, int ep_base, int ep_local, const uint16_t *x, int H, uint16_t *xh)
 {
     if (T <= 0) return;
     const int warps = 8;
-    route_topk_kernel<<<cdiv(T, warps), warps * 32, 0, s>>>(logits, T, E, k, ids, w, local_ids, ep_base, ep_local);
+    route_topk_kernel<<<cdiv(T, warps), warps * 32, 0, s>>>(logits, T, E, k, ids, w, local_ids, ep_base, ep_local,
+                                                            x, H, xh);
 }
 
 // ------------------------------------------------------------------------------------------

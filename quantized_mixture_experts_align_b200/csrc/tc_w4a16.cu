@@ -398,15 +398,25 @@ __global__ void __launch_bounds__(256) gather_bf16_kernel(const uint16_t *__rest
         if (small_rows > 0 && __ldg(sorted_ids + blk0 + small_rows) >= n_slots) continue;
         const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)(real ? slot / k : 0) * H);
         uint4 *dst = reinterpret_cast<uint4 *>(xg + (size_t)r * H);
-        for (int i = lane; i < H / 8; i += 32) {
-            uint4 v = real ? ld_stream_v4(src + i) : make_uint4(0u, 0u, 0u, 0u);
-            if (TO_F16) {
-                v.x = bf16x2_to_f16x2(v.x);
-                v.y = bf16x2_to_f16x2(v.y);
-                v.z = bf16x2_to_f16x2(v.z);
-                v.w = bf16x2_to_f16x2(v.w);
+        // four 16-byte chunks in flight per lane (H / 8 is a multiple of 16)
+        for (int i0 = lane; i0 < H / 8; i0 += 4 * 32) {
+            uint4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = i0 + 32 * u;
+                v[u] = (real && i < H / 8) ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
             }
-            dst[i] = v;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = i0 + 32 * u;
+                if (TO_F16) {
+                    v[u].x = bf16x2_to_f16x2(v[u].x);
+                    v[u].y = bf16x2_to_f16x2(v[u].y);
+                    v[u].z = bf16x2_to_f16x2(v[u].z);
+                    v[u].w = bf16x2_to_f16x2(v[u].w);
+                }
+                if (i < H / 8) dst[i] = v[u];
+            }
         }
     }
 }

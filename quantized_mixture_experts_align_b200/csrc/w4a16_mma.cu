@@ -31,6 +31,8 @@ struct DeqWord {
     uint32_t p[4];  // bf16x2 pairs: (n0,n4) (n1,n5) (n2,n6) (n3,n7), already (q-8)*scale
 };
 
+// INT4 in f16: (q - 8) * s has up to 11 significant bits, exact in f16 (not in bf16), so the
+// INT4 instantiations compute in f16 with f16 activations; MXFP4 / NVFP4 weights are exact in bf16.
 template <int FMT>
 __device__ __forceinline__ DeqWord dequant_word(uint32_t w, uint32_t scale2)
 {
@@ -42,12 +44,12 @@ __device__ __forceinline__ DeqWord dequant_word(uint32_t w, uint32_t scale2)
         d.p[2] = bf16x2_mul(e2m1_pair_pre<2>(w), scale2);
         d.p[3] = bf16x2_mul(e2m1_pair_pre<3>(w), scale2);
     } else {
-        const uint32_t magic = 0x43004300u;  // bf16 128.0 in both halves
-        const uint32_t bias = 0x43084308u;   // bf16 136.0 = 128 + 8 (zero point) in both halves
+        const uint32_t magic = 0x64006400u;  // f16 1024.0 in both halves
+        const uint32_t bias = 0x64086408u;   // f16 1032.0 = 1024 + 8 (zero point) in both halves
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const uint32_t v = lop3_and_or(w >> (4 * i), 0x000F000Fu, magic);  // 128 + q, exact
-            d.p[i] = bf16x2_mul(bf16x2_sub(v, bias), scale2);                 // (q - 8) exact, then * s
+            const uint32_t v = lop3_and_or(w >> (4 * i), 0x000F000Fu, magic);  // 1024 + q, exact
+            d.p[i] = f16x2_mul(f16x2_sub(v, bias), scale2);                   // (q - 8) * s, exact
         }
     }
     return d;
@@ -78,7 +80,9 @@ __host__ __device__ constexpr int w4_stage_bytes(int fmt) { return 4 * 32 * 16 +
 //              h[slot, f] = bf16(silu(gate) * up).
 // MODE_DOWN:   rows [r0, r0+32) of W2; epilogue writes ys[slot, r] = bf16(topk_w[slot] * y) (weight 1
 //              without routing weights: the plain grouped GEMM).
-template <int BM, int WARPS, int MODE, bool STRIDED, int FMT>
+// CVT (INT4 only): the activations are bf16 and are converted to f16 in registers; otherwise they
+// are already f16 (INT4) or bf16 (MXFP4 / NVFP4).
+template <int BM, int WARPS, int MODE, bool STRIDED, int FMT, bool CVT>
 __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4GroupedArgs a)
 {
     constexpr int MS = BM / 8;  // token sub-tiles of 8 columns
@@ -180,7 +184,12 @@ __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4Grouped
                 sc[r] = reinterpret_cast<const uint32_t *>(scale_slot(st, r, g))[t];  // (lo, hi)
             } else {
                 const uint32_t s16 = reinterpret_cast<const uint16_t *>(scale_slot(st, r, g))[t];
-                sc[r] = s16 | (s16 << 16);
+                if (FMT == W4_INT4) {
+                    const float sf = __uint_as_float(s16 << 16);
+                    sc[r] = pack_f16x2(sf, sf);  // the bf16 scale in f16, both halves (exact in range)
+                } else {
+                    sc[r] = s16 | (s16 << 16);
+                }
             }
         }
         issue(q + S - 1);  // refills the slot every lane finished reading in iteration q - 1
@@ -207,13 +216,26 @@ __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4Grouped
                 uint4 xv;
                 if (kActPrefetch) xv = xcur[s][m];
                 else xv = act_row[s] ? ld_v4(act_row[s] + kofs + 8 * m) : make_uint4(0u, 0u, 0u, 0u);
+                if (FMT == W4_INT4 && CVT) {
+                    xv.x = bf16x2_to_f16x2(xv.x);
+                    xv.y = bf16x2_to_f16x2(xv.y);
+                    xv.z = bf16x2_to_f16x2(xv.z);
+                    xv.w = bf16x2_to_f16x2(xv.w);
+                }
                 uint32_t b[4];
                 act_pairs(xv, b);
                 // k-step 2m: pairs 0/1; k-step 2m+1: pairs 2/3
-                mma_bf16_16816(accA[s], d[0].p[0], d[1].p[0], d[0].p[1], d[1].p[1], b[0], b[1]);
-                mma_bf16_16816(accB[s], d[2].p[0], d[3].p[0], d[2].p[1], d[3].p[1], b[0], b[1]);
-                mma_bf16_16816(accA[s], d[0].p[2], d[1].p[2], d[0].p[3], d[1].p[3], b[2], b[3]);
-                mma_bf16_16816(accB[s], d[2].p[2], d[3].p[2], d[2].p[3], d[3].p[3], b[2], b[3]);
+                if (FMT == W4_INT4) {
+                    mma_f16_16816(accA[s], d[0].p[0], d[1].p[0], d[0].p[1], d[1].p[1], b[0], b[1]);
+                    mma_f16_16816(accB[s], d[2].p[0], d[3].p[0], d[2].p[1], d[3].p[1], b[0], b[1]);
+                    mma_f16_16816(accA[s], d[0].p[2], d[1].p[2], d[0].p[3], d[1].p[3], b[2], b[3]);
+                    mma_f16_16816(accB[s], d[2].p[2], d[3].p[2], d[2].p[3], d[3].p[3], b[2], b[3]);
+                } else {
+                    mma_bf16_16816(accA[s], d[0].p[0], d[1].p[0], d[0].p[1], d[1].p[1], b[0], b[1]);
+                    mma_bf16_16816(accB[s], d[2].p[0], d[3].p[0], d[2].p[1], d[3].p[1], b[0], b[1]);
+                    mma_bf16_16816(accA[s], d[0].p[2], d[1].p[2], d[0].p[3], d[1].p[3], b[2], b[3]);
+                    mma_bf16_16816(accB[s], d[2].p[2], d[3].p[2], d[2].p[3], d[3].p[3], b[2], b[3]);
+                }
             }
         }
         if (kActPrefetch) {
@@ -242,8 +264,11 @@ __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4Grouped
             if (slot >= a.n_slots) continue;
             if (MODE == MODE_GATEUP) {
                 uint16_t *h = a.h_out + (size_t)slot * a.n_out;
-                h[rowA + g] = f32_to_bf16(silu_f32(accA[s][c]) * accB[s][c]);
-                h[rowA + g + 8] = f32_to_bf16(silu_f32(accA[s][2 + c]) * accB[s][2 + c]);
+                // h = bf16(silu(g) * u), stored as f16 for the INT4 down GEMM (the same value)
+                const float h0 = silu_f32(accA[s][c]) * accB[s][c];
+                const float h1 = silu_f32(accA[s][2 + c]) * accB[s][2 + c];
+                h[rowA + g] = FMT == W4_INT4 ? f32_to_bf16_as_f16(h0) : f32_to_bf16(h0);
+                h[rowA + g + 8] = FMT == W4_INT4 ? f32_to_bf16_as_f16(h1) : f32_to_bf16(h1);
             } else {
                 const float wt = a.topk_w ? __ldg(a.topk_w + slot) : 1.f;
                 uint16_t *y = a.y_out + (size_t)slot * a.n_out;
@@ -256,26 +281,27 @@ __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4Grouped
     }
 }
 
-template <int BM, int WARPS, int MODE, bool STRIDED, int FMT>
+template <int BM, int WARPS, int MODE, bool STRIDED, int FMT, bool CVT>
 static void launch_bm_fmt(const W4GroupedArgs &a, int max_blocks, cudaStream_t s)
 {
     const int rows_per_cta = (MODE == MODE_GATEUP ? 16 : 32) * WARPS;
     const size_t smem = (size_t)WARPS * kW4Stages * w4_stage_bytes(FMT);
     static std::atomic<int> smem_enabled[kMaxDevices];
-    enable_smem(w4a16_grouped_mma_kernel<BM, WARPS, MODE, STRIDED, FMT>, (int)smem, smem_enabled);
+    enable_smem(w4a16_grouped_mma_kernel<BM, WARPS, MODE, STRIDED, FMT, CVT>, (int)smem, smem_enabled);
     dim3 grid(max_blocks, cdiv(a.n_out, rows_per_cta));
     if (STRIDED)  // after the tensor-core kernels of the same stage: an ordinary launch
-        w4a16_grouped_mma_kernel<BM, WARPS, MODE, STRIDED, FMT><<<grid, WARPS * 32, smem, s>>>(a);
+        w4a16_grouped_mma_kernel<BM, WARPS, MODE, STRIDED, FMT, CVT><<<grid, WARPS * 32, smem, s>>>(a);
     else
-        launch_pdl(w4a16_grouped_mma_kernel<BM, WARPS, MODE, STRIDED, FMT>, grid, dim3(WARPS * 32), smem, s, a);
+        launch_pdl(w4a16_grouped_mma_kernel<BM, WARPS, MODE, STRIDED, FMT, CVT>, grid, dim3(WARPS * 32), smem, s, a);
 }
 
 template <int BM, int WARPS, int MODE, bool STRIDED>
 static void launch_bm(const W4GroupedArgs &a, int max_blocks, cudaStream_t s)
 {
-    if (a.fmt == W4_FP4) launch_bm_fmt<BM, WARPS, MODE, STRIDED, W4_FP4>(a, max_blocks, s);
-    else if (a.fmt == W4_NV) launch_bm_fmt<BM, WARPS, MODE, STRIDED, W4_NV>(a, max_blocks, s);
-    else launch_bm_fmt<BM, WARPS, MODE, STRIDED, W4_INT4>(a, max_blocks, s);
+    if (a.fmt == W4_FP4) launch_bm_fmt<BM, WARPS, MODE, STRIDED, W4_FP4, false>(a, max_blocks, s);
+    else if (a.fmt == W4_NV) launch_bm_fmt<BM, WARPS, MODE, STRIDED, W4_NV, false>(a, max_blocks, s);
+    else if (a.act_bf16) launch_bm_fmt<BM, WARPS, MODE, STRIDED, W4_INT4, true>(a, max_blocks, s);
+    else launch_bm_fmt<BM, WARPS, MODE, STRIDED, W4_INT4, false>(a, max_blocks, s);
 }
 
 // UE8M0 -> bf16 2^(s - 1): exponent field s + 126 (s <= 128); larger codes give +inf
