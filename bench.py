@@ -281,12 +281,17 @@ def launch_overhead_w4a16(moeq, d, steps, warmup):
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) / steps, host_us
 
+    moeq.moe_host_stats(reset=True)
     eager_ms, eager_host = back_to_back(step)
+    lib = moeq.moe_host_stats(reset=True)
     graph_ms, graph_host = back_to_back(g.replay)
     del g
+    lib_us = lib["host_us"] / max(lib["calls"], 1)
     return {"eager_ms_per_step": eager_ms, "graph_ms_per_step": graph_ms, "eager_host_submit_us": eager_host,
+            "eager_library_host_us": lib_us, "eager_binding_host_us": eager_host - lib_us,
             "graph_host_submit_us": graph_host, "steps": steps,
-            "how": "back-to-back steps on one stream, no L2 flush; host time = enqueue time per step"}
+            "how": "back-to-back steps on one stream, no L2 flush; host time = enqueue time per step; library = "
+                   "the C entry point's own wall time (moe_host_stats), binding = the rest (Python + ctypes)"}
 
 
 def run_w4a16(moeq, d, steps, warmup, flush, world, trace=False):
@@ -627,6 +632,7 @@ def main():
         also["fp8_peak"] = fp8m
         dp = W.make_moe(W.WORKLOADS["prefill_w4a16"], device="cuda")
         pms, _, _ = run_w4a16(moeq, dp, max(3, args.steps // 4), 3, None, world, trace=False)
+        phost = moeq.moe_host_stats(reset=True)  # the timed calls above (warm-up included)
         _, pst, _ = run_w4a16(moeq, dp, 3, 3, None, world, trace=True)
         pflops = W.moe_flops(dp["T"], dp["k"], dp["H"], dp["I"])
         pstep = max_over_ranks(statistics.mean(pms), world)
@@ -652,6 +658,8 @@ def main():
                          "algorithmic_flops_per_launch": pgu_flops, "launch_ms": pgu_avg,
                          "peak_source": f"{peak_src} bf16_tflops (burst)"},
             "skew_aware_roof_ms": proof, "frac_of_skew_aware_roof": proof / pstep,
+            "host": {"library_us_per_call": phost["host_us"] / max(phost["calls"], 1),
+                     "tensor_maps_encoded": phost["tmap_encoded"], "tensor_maps_reused": phost["tmap_reused"]},
             "weight_gbs": pbytes / (pstep * 1e-3) / 1e9, "active_experts": int((prows > 0).sum()),
             "stages_ms": {k: v[0] / max(v[1], 1) for k, v in pst.items() if v[1]}}
         # MXFP4 weights (E2M1 codes, UE8M0 group-32 scales) on the same layer: decode (T = 32,

@@ -32,10 +32,9 @@
 //               barrier wait ~47 even when the phase is complete, more under load), so the steps
 //               are long and the MMA thread waits on one barrier and commits once per step;
 //   warps 2-17  dequantization: a thread owns one weight row (tensor lane) and a 32-input slice
-//               of each 128-input step (16 bytes of codes, 1 group scale), prefetches them through
-//               a private 3-deep cp.async ring, and writes the dequantized slice to one of 3
-//               tensor-memory
-//               stages; then the epilogue: gate/up passes the up values through shared memory
+//               of each 128-input step (16 bytes of codes, 1 group scale), fetches them into
+//               registers four steps ahead, and writes the dequantized slice to one of 3
+//               tensor-memory stages; then the epilogue: gate/up passes the up values through shared memory
 //               to the warps holding the gate values, which write h = bf16(silu(g) * u); down
 //               writes the routing-weighted bf16 slot rows.
 #include "kernels.cuh"
@@ -50,7 +49,7 @@ constexpr int kKs = 128;      // inputs per pipeline step (8 MMAs per barrier ro
 constexpr int kStages = 3;    // dequantized weight stages (tensor memory)
 constexpr int kDownTilesPerCta = 4;  // down GEMM: 128-row output tiles run by one CTA
 constexpr int kBStages = 3;   // activation tiles (shared memory)
-constexpr int kRing = 3;      // per-thread packed-code prefetch depth, in steps
+constexpr int kPf = 4;        // per-thread packed-code prefetch depth (registers), in steps
 constexpr int kDeqWarps = 16;  // 4 per tensor-memory lane quarter, each a quarter of every step
 constexpr int kDeqThreads = kDeqWarps * 32;
 constexpr int kSplit = kDeqWarps / 4;           // K slices of a step (one per warp of a lane quarter)
@@ -62,9 +61,7 @@ constexpr int kAStageCols = kKs / 2;            // 128 bf16 inputs = 64 columns
 constexpr int kTmemCols = 512;                  // 256 + 3 x 64 used, power of two allocated
 constexpr int kBTile = kTok * kKs * 2;          // 64 KB: two 128-byte-swizzled halves of 64 inputs
 constexpr int kBHalf = kBTile / 2;
-constexpr size_t kCodeRing = (size_t)kRing * kDeqThreads * 16;
-constexpr size_t kScaleRing = (size_t)kRing * kDeqThreads * 4;
-constexpr size_t kSmemBytes = 1024 + (size_t)kBStages * kBTile + kCodeRing + kScaleRing + 256;
+constexpr size_t kSmemBytes = 1024 + (size_t)kBStages * kBTile + 256;
 static_assert(kAccCols + kStages * kAStageCols <= kTmemCols, "tensor memory budget");
 static_assert(kBStages == kStages, "one stage-free barrier serves the activation and weight stages");
 static_assert(64 * kTok * 4 <= kBStages * kBTile, "gate/up exchange fits in the activation ring");
@@ -105,9 +102,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *btiles = smem;
-    uint8_t *code_ring = btiles + kBStages * kBTile;
-    uint8_t *scale_ring = code_ring + kCodeRing;
-    uint64_t *a_full = reinterpret_cast<uint64_t *>(scale_ring + kScaleRing);
+    uint64_t *a_full = reinterpret_cast<uint64_t *>(btiles + kBStages * kBTile);
     uint64_t *empty = a_full + kStages;
     uint64_t *acc_full = empty + kStages;
     uint64_t *mma_done = acc_full + 1;
@@ -232,18 +227,19 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
         constexpr int GS = FMT == W4_NV ? 16 : 32;
         const uint16_t *srow = a.ws + (size_t)grow * (K / GS) + (FMT == W4_NV ? 2 * kq : (kq & ~1));
         const size_t stile = (size_t)128 * (K / GS);
-        auto code_slot = [&](int slot) { return code_ring + ((size_t)slot * kDeqThreads + t) * 16; };
-        auto scale_slot = [&](int slot) { return scale_ring + ((size_t)slot * kDeqThreads + t) * 4; };
-        // prefetch position (global step pg = tile pt, K step pk): advanced by one per issue, so the
-        // ring runs on into the next tile's weights without a division
+        // Codes and scales run kPf steps ahead in registers (fetch position: global step pg = tile
+        // pt, K step pk, advanced by one per fetch, so the prefetch runs on into the next tile's
+        // weights without a division). Every access is aligned: a row holds K / 2 bytes (K a
+        // multiple of 128) and a thread's slice starts at 16 kq bytes.
         int pg = 0, pk = 0;
         const int32_t *pw = wrow;
         const uint16_t *ps = srow;
-        auto issue = [&]() {
+        uint4 cq[kPf];
+        uint32_t sq[kPf];
+        auto fetch = [&](uint4 &c, uint32_t &sc) {
             if (pg < NT) {
-                const int slot = pg % kRing;
-                cp_async16_stream(code_slot(slot), pw + pk * (kKs / 8));
-                cp_async4_ca(scale_slot(slot), ps + pk * (kKs / GS));
+                c = __ldg(reinterpret_cast<const uint4 *>(pw + pk * (kKs / 8)));
+                sc = __ldg(reinterpret_cast<const uint32_t *>(ps + pk * (kKs / GS)));
                 ++pg;
                 if (++pk == NS) {
                     pk = 0;
@@ -251,10 +247,13 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
                     ps += stile;
                 }
             }
-            cp_async_commit();
         };
 #pragma unroll
-        for (int gs = 0; gs < kRing - 1; ++gs) issue();
+        for (int i = 0; i < kPf; ++i) {
+            cq[i] = make_uint4(0u, 0u, 0u, 0u);
+            sq[i] = 0u;
+            fetch(cq[i], sq[i]);
+        }
         // The stores of step ks are waited for (tcgen05.wait::st) only after the dequantization of
         // step ks + 1, so the tensor-memory write latency hides behind that work.
         auto stage_ready = [&](int j) -> bool {
@@ -269,11 +268,14 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
         for (int tt = 0; tt < nt && ok; ++tt) {
         for (int ks = 0; ks < NS && ok; ++ks) {
             const int gs = tt * NS + ks;
-            cp_async_wait<kRing - 2>();
-            const int slot = gs % kRing;
-            const uint4 c = *reinterpret_cast<const uint4 *>(code_slot(slot));  // a warp reads 512 contiguous bytes
-            const uint32_t sc = *reinterpret_cast<const uint32_t *>(scale_slot(slot));
-            issue();  // step gs + kRing - 1: refills the slot read in step gs - 1
+            const uint4 c = cq[0];
+            const uint32_t sc = sq[0];
+#pragma unroll
+            for (int i = 0; i < kPf - 1; ++i) {
+                cq[i] = cq[i + 1];
+                sq[i] = sq[i + 1];
+            }
+            fetch(cq[kPf - 1], sq[kPf - 1]);  // step gs + kPf
             // this slice's group scale, twice (group 16: words 0-1 the first, words 2-3 the second)
             uint32_t s2 = prmt(sc, sc, (FMT != W4_NV && (kq & 1)) ? 0x3232u : 0x1010u);
             if (FMT == W4_INT4) s2 = bf16x2_to_f16x2(s2);  // the group scale in f16 (exact in range)
@@ -368,7 +370,6 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
             if (lane == 0) tc::mbar_arrive(acc_empty);
         }
         }  // output tiles
-        cp_async_wait<0>();
     }
     tc::fence_before_sync();
     __syncthreads();
