@@ -643,19 +643,23 @@ def main():
         proof = skew_roof_ms(prows, W.w4a16_expert_bytes(dp["H"], dp["I"]), dp["H"], dp["I"], peaks["hbm_gbs"],
                              bf16_peak)
         ptf = pflops / (pstep * 1e-3) / 1e12
-        # dominant kernel: the gate/up stage (tcgen05 blocks + the register-fed few-row blocks),
-        # algorithmic FLOPs of the real routed rows only (padding excluded)
+        # dominant kernel: the tcgen05 gate/up GEMM (stage gate_up; the expert blocks with at most
+        # 8 routed rows run in the few_rows stage), algorithmic FLOPs of the real routed rows of
+        # its blocks only (padding excluded)
         pgu_ms, pgu_calls = pst["gate_up"]
         pgu_avg = pgu_ms / max(pgu_calls, 1)
-        pgu_flops = 2.0 * dp["T"] * dp["k"] * 2 * dp["I"] * dp["H"]
+        tail = prows % 256
+        few = int(tail[(tail > 0) & (tail <= 8)].sum())
+        pgu_flops = 2.0 * (dp["T"] * dp["k"] - few) * 2 * dp["I"] * dp["H"]
         prefill = {
             "metric": "prefill W4A16 MoE layer TFLOP/s", "value": ptf, "unit": "TFLOP/s",
             "workload": "prefill_w4a16 T=8192 H=7168 I=2048 E=384 k=8, Zipf-biased routing (INT4 group-32)",
             "ms_per_step": pstep, "steps": len(pms), "frac_of_bf16_burst": ptf / bf16_peak,
             "roofline": {"bound": "tensor", "achieved": pgu_flops / (pgu_avg * 1e-3) / 1e12, "peak": bf16_peak,
                          "unit": "TFLOP/s", "frac": pgu_flops / (pgu_avg * 1e-3) / 1e12 / bf16_peak, "traffic": None,
-                         "kernel": "w4a16_tc_kernel<GATEUP> + w4a16_grouped_mma_kernel<8,4,GATEUP,strided> (gate/up)",
+                         "kernel": "w4a16_tc_kernel<GATEUP> (gate/up + SiLU*up, blocks of more than 8 rows)",
                          "algorithmic_flops_per_launch": pgu_flops, "launch_ms": pgu_avg,
+                         "rows_in_few_row_blocks": few,
                          "peak_source": f"{peak_src} bf16_tflops (burst)"},
             "skew_aware_roof_ms": proof, "frac_of_skew_aware_roof": proof / pstep,
             "host": {"library_us_per_call": phost["host_us"] / max(phost["calls"], 1),

@@ -315,12 +315,13 @@ MOEQ_API int w8a8_channel_fp8_matmul(const uint8_t *A, const float *As, const ui
  * brackets each of its kernel stages with a pair of CUDA events recorded on the call's stream
  * (the library creates the events on first use, on the current device; do not enable tracing
  * during stream capture). moe_trace_read() waits for the recorded events, adds their durations
- * to per-stage totals and writes the first min(n_stages, 8) totals (milliseconds) and call
- * counts (either pointer may be NULL); it returns 8, the number of stages, or MOEQ_ERR_CUDA.
+ * to per-stage totals and writes the first min(n_stages, 9) totals (milliseconds) and call
+ * counts (either pointer may be NULL); it returns 9, the number of stages, or MOEQ_ERR_CUDA.
  * `reset` != 0 clears the totals after reading. Stage indices: 0 route_topk, 1 align,
  * 2 fp8_act_quant, 3 gate_up (with SiLU*up), 4 down (with the routing weight), 5 combine,
  * 6 dense block-FP8 matmul, 7 gather (routed activation rows copied into aligned order for the
- * tensor-core GEMMs).
+ * tensor-core GEMMs), 8 few_rows (gate/up and down of the expert blocks with at most 8 routed
+ * rows on the 4-bit layers' tensor-core schedule, run by the register-fed kernel).
  */
 MOEQ_API int moe_trace_enable(int enable);
 MOEQ_API int moe_trace_read(double *stage_ms, long long *stage_calls, int n_stages, int reset);

@@ -464,7 +464,8 @@ def moe_w4a16_grouped_masked(A, w_q, w_s, masked_m, expected_m, out=None, ws=Non
     return out
 
 
-TRACE_STAGES = ("route_topk", "align", "fp8_act_quant", "gate_up", "down", "combine", "dense_fp8", "gather")
+TRACE_STAGES = ("route_topk", "align", "fp8_act_quant", "gate_up", "down", "combine", "dense_fp8", "gather",
+                "few_rows")
 
 
 def moe_trace_enable(enable: bool = True):

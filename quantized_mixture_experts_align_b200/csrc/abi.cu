@@ -53,7 +53,7 @@ static int num_sms()
 // When enabled, each kernel stage of a call is bracketed by a CUDA event pair recorded on the
 // call's stream; moe_trace_read() waits for the recorded pairs and accumulates their durations.
 namespace trace {
-enum { ROUTE = 0, ALIGN, ACT_QUANT, GATE_UP, DOWN, COMBINE, DENSE, GATHER, NSTAGE };
+enum { ROUTE = 0, ALIGN, ACT_QUANT, GATE_UP, DOWN, COMBINE, DENSE, GATHER, FEW_ROWS, NSTAGE };
 struct Rec {
     cudaEvent_t a, b;
     int stage;
@@ -483,6 +483,9 @@ static int w4_layer_forward(int fmt, const char *name, const uint16_t *x, const 
         {
             trace::Scope ts(trace::GATE_UP, s);
             rc = launch_w4a16_tc(t, TC_GATEUP, xg, r.max_blocks, s);
+        }
+        {
+            trace::Scope ts(trace::FEW_ROWS, s);
             launch_w4a16_grouped_mma(g, MODE_GATEUP, kW4SmallRows, r.max_blocks, s);
         }
         if (rc) return rc;
@@ -506,6 +509,9 @@ static int w4_layer_forward(int fmt, const char *name, const uint16_t *x, const 
         {
             trace::Scope ts(trace::DOWN, s);
             rc = launch_w4a16_tc(t, TC_DOWN, h, r.max_blocks, s);
+        }
+        {
+            trace::Scope ts(trace::FEW_ROWS, s);
             launch_w4a16_grouped_mma(g, MODE_DOWN, kW4SmallRows, r.max_blocks, s);
         }
         if (rc) return rc;
