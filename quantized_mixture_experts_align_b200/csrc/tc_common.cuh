@@ -52,6 +52,31 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
     return ok != 0;
 }
 
+// One poll of the barrier at a shared-memory address (same meaning as mbar_try_wait).
+__device__ __forceinline__ bool mbar_try_wait_addr(uint32_t bar_addr, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar_addr), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Arrival of lane 0 of the calling warp (predicated, no branch).
+__device__ __forceinline__ void mbar_arrive_lane0(uint32_t bar_addr, int lane)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.eq.s32 p, %1, 0;\n\t"
+        "@p mbarrier.arrive.shared::cta.b64 _, [%0];\n\t}"
+        ::"r"(bar_addr), "r"(lane)
+        : "memory");
+}
+
 // Wait for the phase with the given parity to complete; false (and `*abort` set, status word
 // written) if it does not within kMaxPolls polls or if another thread already gave up.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort, int *status,

@@ -227,77 +227,89 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
         constexpr int GS = FMT == W4_NV ? 16 : 32;
         const uint16_t *srow = a.ws + (size_t)grow * (K / GS) + (FMT == W4_NV ? 2 * kq : (kq & ~1));
         const size_t stile = (size_t)128 * (K / GS);
-        // Codes and scales run kPf steps ahead in registers (fetch position: global step pg = tile
-        // pt, K step pk, advanced by one per fetch, so the prefetch runs on into the next tile's
-        // weights without a division). Every access is aligned: a row holds K / 2 bytes (K a
-        // multiple of 128) and a thread's slice starts at 16 kq bytes.
-        int pg = 0, pk = 0;
-        const int32_t *pw = wrow;
-        const uint16_t *ps = srow;
+        // Codes and scales run kPf steps ahead in registers. A tile's steps are counted over NSP =
+        // NS rounded up to kPf (the steps past NS do nothing), so the register slot of a step is its
+        // index mod kPf: a constant in the loop unrolled by kPf, where slot j is consumed and refilled
+        // in place. Every access is aligned: a row holds K / 2 bytes (K a multiple of 128) and a
+        // thread's slice starts at 16 kq bytes.
+        const int NSP = (NS + kPf - 1) / kPf * kPf;
         uint4 cq[kPf];
         uint32_t sq[kPf];
-        auto fetch = [&](uint4 &c, uint32_t &sc) {
-            if (pg < NT) {
-                c = __ldg(reinterpret_cast<const uint4 *>(pw + pk * (kKs / 8)));
-                sc = __ldg(reinterpret_cast<const uint32_t *>(ps + pk * (kKs / GS)));
-                ++pg;
-                if (++pk == NS) {
-                    pk = 0;
-                    pw += wtile;
-                    ps += stile;
-                }
-            }
-        };
 #pragma unroll
-        for (int i = 0; i < kPf; ++i) {
-            cq[i] = make_uint4(0u, 0u, 0u, 0u);
-            sq[i] = 0u;
-            fetch(cq[i], sq[i]);
+        for (int j = 0; j < kPf; ++j) {
+            cq[j] = make_uint4(0u, 0u, 0u, 0u);
+            sq[j] = 0u;
+            if (j < NS) {
+                cq[j] = __ldg(reinterpret_cast<const uint4 *>(wrow + j * (kKs / 8)));
+                sq[j] = __ldg(reinterpret_cast<const uint32_t *>(srow + j * (kKs / GS)));
+            }
         }
-        // The stores of step ks are waited for (tcgen05.wait::st) only after the dequantization of
-        // step ks + 1, so the tensor-memory write latency hides behind that work.
-        auto stage_ready = [&](int j) -> bool {
+        const uint32_t a_full0 = smem_addr(a_full), empty0 = smem_addr(empty);
+        // this thread's slot of weight stage 0 (tensor-memory lane quarter, K slice); stage s adds
+        // s * kAStageCols columns
+        const uint32_t tst0 = tmem + ((uint32_t)(quarter * 32) << 16) + kAccCols + kq * (kThrK / 2);
+        // the stores of a step are waited for (tcgen05.wait::st) only after the dequantization of
+        // the next step, so the tensor-memory write latency hides behind that work
+        auto stage_ready = [&](uint32_t st) {
             tc::tmem_wait_st();
             tc::fence_before_sync();
             __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&a_full[j % kStages]);
-            return true;
+            tc::mbar_arrive_lane0(a_full0 + 8u * st, lane);
         };
         bool ok = true;
-        int pending = -1;
+        int gs = 0;                        // steps stored so far (all tiles)
+        uint32_t s = 0, ph = 0;            // stage of the next step, parity of its use count
+        int pending = -1;                  // stage stored by the previous step, not yet published
         for (int tt = 0; tt < nt && ok; ++tt) {
-        for (int ks = 0; ks < NS && ok; ++ks) {
-            const int gs = tt * NS + ks;
-            const uint4 c = cq[0];
-            const uint32_t sc = sq[0];
+        for (int ks0 = 0; ks0 < NSP && ok; ks0 += kPf) {
+            // the slots refilled in this round: steps ks0 + kPf .. of this tile, or the next
+            // tile's first kPf steps
+            const bool wrap = ks0 + kPf == NSP;
+            const int ft = wrap ? tt + 1 : tt, fp0 = wrap ? 0 : ks0 + kPf;
+            const int32_t *fw = wrow + (size_t)ft * wtile + fp0 * (kKs / 8);
+            const uint16_t *fsc = srow + (size_t)ft * stile + fp0 * (kKs / GS);
 #pragma unroll
-            for (int i = 0; i < kPf - 1; ++i) {
-                cq[i] = cq[i + 1];
-                sq[i] = sq[i + 1];
-            }
-            fetch(cq[kPf - 1], sq[kPf - 1]);  // step gs + kPf
-            // this slice's group scale, twice (group 16: words 0-1 the first, words 2-3 the second)
-            uint32_t s2 = prmt(sc, sc, (FMT != W4_NV && (kq & 1)) ? 0x3232u : 0x1010u);
-            if (FMT == W4_INT4) s2 = bf16x2_to_f16x2(s2);  // the group scale in f16 (exact in range)
-            const uint32_t s2h = FMT == W4_NV ? prmt(sc, sc, 0x3232u) : s2;
-            uint32_t pairs[16];
-            dequant4<FMT>(c.x, s2, pairs + 0);
-            dequant4<FMT>(c.y, s2, pairs + 4);
-            dequant4<FMT>(c.z, s2h, pairs + 8);
-            dequant4<FMT>(c.w, s2h, pairs + 12);
-            if (pending >= 0) {
-                ok = stage_ready(pending);
+            for (int j = 0; j < kPf; ++j) {
+                const uint4 c = cq[j];
+                const uint32_t sc = sq[j];
+                if (ft < nt && fp0 + j < NS) {
+                    cq[j] = __ldg(reinterpret_cast<const uint4 *>(fw + j * (kKs / 8)));
+                    sq[j] = __ldg(reinterpret_cast<const uint32_t *>(fsc + j * (kKs / GS)));
+                }
+                if (ks0 + j >= NS || !ok) continue;  // padding step (uniform over the warp)
+                uint32_t s2, s2h;
+                if (FMT == W4_INT4) {
+                    // this slice's group scale, bf16 -> f32 -> f16 (exact in range), twice
+                    const float sf = __uint_as_float(prmt(sc, 0u, (kq & 1) ? 0x3244u : 0x1044u));
+                    s2 = s2h = pack_f16x2(sf, sf);
+                } else {
+                    // group 32: this slice's scale twice; group 16: words 0-1 the first, 2-3 the second
+                    s2 = prmt(sc, sc, (FMT != W4_NV && (kq & 1)) ? 0x3232u : 0x1010u);
+                    s2h = FMT == W4_NV ? prmt(sc, sc, 0x3232u) : s2;
+                }
+                uint32_t pairs[16];
+                dequant4<FMT>(c.x, s2, pairs + 0);
+                dequant4<FMT>(c.y, s2, pairs + 4);
+                dequant4<FMT>(c.z, s2h, pairs + 8);
+                dequant4<FMT>(c.w, s2h, pairs + 12);
+                if (pending >= 0) stage_ready((uint32_t)pending);
                 pending = -1;
-                if (!ok) break;
+                // the stage's previous contents have been read by the MMAs (all lanes poll once;
+                // a bounded warp-wide wait only when the phase is not complete yet)
+                if (gs >= kStages && !__all_sync(0xFFFFFFFFu, tc::mbar_try_wait_addr(empty0 + 8u * s, ph ^ 1u)))
+                    ok = tc::mbar_wait_warp(&empty[s], ph ^ 1u, abort_flag, a.status);
+                if (!ok) continue;
+                tc::fence_after_sync();
+                tc::tmem_st16(tst0 + s * kAStageCols, pairs);
+                pending = (int)s;
+                ++gs;
+                if (++s == kStages) {
+                    s = 0;
+                    ph ^= 1u;
+                }
             }
-            const int s = gs % kStages;
-            if (gs >= kStages) ok = tc::mbar_wait_warp(&empty[s], ((gs / kStages) & 1) ^ 1, abort_flag, a.status);
-            if (!ok) break;
-            tc::fence_after_sync();
-            tc::tmem_st16(tmem + ((uint32_t)(quarter * 32) << 16) + kAccCols + s * kAStageCols + kq * (kThrK / 2), pairs);
-            pending = gs;
         }
-        if (pending >= 0 && ok) ok = stage_ready(pending);
+        if (pending >= 0 && ok) stage_ready((uint32_t)pending);
         pending = -1;
 
         // ---- epilogue of tile tt: tokens [64 kq, 64 kq + 64), chunks of 32 ----
