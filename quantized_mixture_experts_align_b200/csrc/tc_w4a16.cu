@@ -20,8 +20,10 @@
 // word; four byte permutes put them in natural order, so the activation rows keep their own order:
 // the gather copies the routed rows of x as they are, and h is written in natural order.
 //
-// CTA = one 256-row activation block of one expert x (gate/up: 64 features, gate rows in tensor
-// lanes 0-63 and the matching up rows in lanes 64-127; down: 128 output rows):
+// CTA = one 256-row activation block of one expert x consecutive output tiles, run back to back
+// through one pipeline (gate/up: tiles of 64 features, each tensor-memory lane quarter holding the
+// gate rows of 16 features in lanes 0-15 and their up rows in lanes 16-31; down: tiles of 128
+// output rows):
 //   warp 0      TMA producer of the activation tiles [256 tokens x 128 inputs] (3 stages, two
 //               128-byte-swizzled halves of 64 inputs each); a tile's bytes complete on the same
 //               "stage ready" barrier the dequantization warps arrive on, and one commit per step
@@ -34,9 +36,9 @@
 //   warps 2-17  dequantization: a thread owns one weight row (tensor lane) and a 32-input slice
 //               of each 128-input step (16 bytes of codes, 1 group scale), fetches them into
 //               registers four steps ahead, and writes the dequantized slice to one of 3
-//               tensor-memory stages; then the epilogue: gate/up passes the up values through shared memory
-//               to the warps holding the gate values, which write h = bf16(silu(g) * u); down
-//               writes the routing-weighted bf16 slot rows.
+//               tensor-memory stages; then the epilogue of each tile: gate/up pairs every gate
+//               lane with its up lane by shuffles and writes h = bf16(silu(g) * u); down writes
+//               the routing-weighted bf16 slot rows.
 #include "kernels.cuh"
 #include "tc_common.cuh"
 
@@ -47,7 +49,8 @@ namespace {
 constexpr int kTok = 256;     // tokens per tile = aligned block size
 constexpr int kKs = 128;      // inputs per pipeline step (8 MMAs per barrier round trip)
 constexpr int kStages = 3;    // dequantized weight stages (tensor memory)
-constexpr int kDownTilesPerCta = 4;  // down GEMM: 128-row output tiles run by one CTA
+constexpr int kDownTilesPerCta = 4;    // down GEMM: 128-row output tiles run by one CTA
+constexpr int kGateUpTilesPerCta = 2;  // gate/up GEMM: 64-feature output tiles run by one CTA
 constexpr int kBStages = 3;   // activation tiles (shared memory)
 constexpr int kPf = 4;        // per-thread packed-code prefetch depth (registers), in steps
 constexpr int kDeqWarps = 16;  // 4 per tensor-memory lane quarter, each a quarter of every step
@@ -64,7 +67,6 @@ constexpr int kBHalf = kBTile / 2;
 constexpr size_t kSmemBytes = 1024 + (size_t)kBStages * kBTile + 256;
 static_assert(kAccCols + kStages * kAStageCols <= kTmemCols, "tensor memory budget");
 static_assert(kBStages == kStages, "one stage-free barrier serves the activation and weight stages");
-static_assert(64 * kTok * 4 <= kBStages * kBTile, "gate/up exchange fits in the activation ring");
 
 // (q - 8) * scale (INT4) or E2M1(q) * 2^(s - 1) (FP4, see e2m1_pair_pre) in bf16 for the pairs
 // (q0,q4) (q1,q5) (q2,q6) (q3,q7) of one code word
@@ -106,7 +108,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
     uint64_t *empty = a_full + kStages;
     uint64_t *acc_full = empty + kStages;
     uint64_t *mma_done = acc_full + 1;
-    uint64_t *acc_empty = mma_done + 1;  // down, several output tiles: the accumulator has been read
+    uint64_t *acc_empty = mma_done + 1;  // several output tiles: the accumulator has been read
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -118,13 +120,14 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
     if (r0 >= __ldg(a.ntp)) return;  // uniform over the CTA, before any barrier or allocation
     const int e = __ldg(a.expert_ids + blockIdx.y);
     if (e < 0 || e >= a.E) return;
-    // gate/up: one tile of 64 features; down: nt consecutive 128-row output tiles of the block, run
-    // back to back through one pipeline (the setup, the ring fill and the prefetch of the next
-    // tile's weights are shared; only the accumulator drains between tiles)
-    const int tpc = GU ? 1 : a.tiles_per_cta;
+    // nt consecutive output tiles of the block, run back to back through one pipeline (the setup,
+    // the ring fill and the prefetch of the next tile's weights are shared; only the accumulator
+    // drains between tiles)
+    constexpr int kTileW = GU ? 64 : 128;  // output features (gate/up) or rows (down) of a tile
+    const int tpc = a.tiles_per_cta;
     const int tile0 = blockIdx.x * tpc;
-    const int nt = GU ? 1 : min(tpc, a.N / 128 - tile0);
-    const int n0 = tile0 * (GU ? 64 : 128);  // first output feature (gate/up) or row (down)
+    const int nt = min(tpc, a.N / kTileW - tile0);
+    const int n0 = tile0 * kTileW;  // first output feature (gate/up) or row (down)
     const int K = a.K, NS = K / kKs, NT = nt * NS;  // K steps per tile, in all
     // real rows of this block: the expert's slots come first, padding after
     const int valid = __syncthreads_count(threadIdx.x < kTok && __ldg(a.sorted_ids + r0 + threadIdx.x) < a.n_slots);
@@ -217,16 +220,18 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
         const int dw = warp - 2, quarter = warp & 3, kq = dw >> 2;  // lane quarter, K slice
         const int t = dw * 32 + lane;                            // ring slot owner
         const int row = quarter * 32 + lane;                     // tensor-memory lane = weight row
-        const int grow = GU ? e * a.rows_per_expert + (row < 64 ? 0 : a.N) + n0 + (row & 63)
+        // gate/up: lanes 0-15 of each lane quarter hold the gate rows of 16 features, lanes 16-31
+        // the up rows of the same features (the epilogue pairs them with one shuffle)
+        const int grow = GU ? e * a.rows_per_expert + ((lane & 16) ? a.N : 0) + n0 + 16 * quarter + (lane & 15)
                             : e * a.rows_per_expert + n0 + row;
         const int32_t *wrow = a.wq + (size_t)grow * (K / 8) + kq * 4;  // 4 words = 32 inputs
-        const size_t wtile = (size_t)128 * (K / 8);                     // next output tile (down)
+        const size_t wtile = (size_t)kTileW * (K / 8);                  // next output tile
         // the group-32 scale of this thread's 32 inputs comes with its neighbour's in one aligned
         // 4-byte copy (rows are K/16 bytes apart, K a multiple of 128); group 16: its own two
         // scales, the same aligned 4 bytes
         constexpr int GS = FMT == W4_NV ? 16 : 32;
         const uint16_t *srow = a.ws + (size_t)grow * (K / GS) + (FMT == W4_NV ? 2 * kq : (kq & ~1));
-        const size_t stile = (size_t)128 * (K / GS);
+        const size_t stile = (size_t)kTileW * (K / GS);
         // Codes and scales run kPf steps ahead in registers. A tile's steps are counted over NSP =
         // NS rounded up to kPf (the steps past NS do nothing), so the register slot of a step is its
         // index mod kPf: a constant in the loop unrolled by kPf, where slot j is consumed and refilled
@@ -319,37 +324,29 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
         // NVFP4: the accumulator carries 2^-8 / (tensor scale) of the product
         const float gsc = FMT == W4_NV ? __ldg(a.wglobal + e) * 256.f : 1.f;
         if (GU) {
-            // up values (lanes 64-127) go through shared memory (the activation ring is free once
-            // every MMA has completed) to the warps holding the matching gate values (lanes 0-63)
-            float *up_s = reinterpret_cast<float *>(btiles);  // [token][feature 0..63]
-            if (ok) tc::fence_after_sync();
-            if (ok && quarter >= 2) {
+            // lane l < 16 holds gate row f, lane l + 16 the up row of the same feature: per token
+            // pair one shuffle gives each its partner's value; the gate lane finishes tokens
+            // 0-15 of a 32-token chunk, the up lane tokens 16-31
+            if (ok) {
+                tc::fence_after_sync();
+                const bool is_gate = lane < 16;
+                uint16_t *hcol = a.h_out + n0 + tt * 64 + 16 * quarter + (lane & 15);
                 for (int c = 0; c < kTok / kSplit / 32; ++c) {
                     const int tok0 = kq * (kTok / kSplit) + c * 32;
                     if (tok0 >= n_mma) break;
-                    uint32_t u[32];
-                    tc::tmem_ld32(lane_base + tok0, u);
+                    uint32_t v[32];
+                    tc::tmem_ld32(lane_base + tok0, v);
                     tc::tmem_wait_ld();
+                    uint16_t *hrow = hcol + (size_t)(r0 + tok0 + (is_gate ? 0 : 16)) * a.N;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) up_s[(tok0 + j) * 64 + (row - 64)] = gsc * __uint_as_float(u[j]);
-                }
-            }
-            asm volatile("bar.sync 1, %0;" ::"n"(kDeqThreads) : "memory");
-            if (ok && quarter < 2) {
-                const int f = n0 + row;
-                uint16_t *hcol = a.h_out + f;
-                for (int c = 0; c < kTok / kSplit / 32; ++c) {
-                    const int tok0 = kq * (kTok / kSplit) + c * 32;
-                    if (tok0 >= n_mma) break;
-                    uint32_t g[32];
-                    tc::tmem_ld32(lane_base + tok0, g);
-                    tc::tmem_wait_ld();
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const float hv = silu_f32(gsc * __uint_as_float(g[j])) * up_s[(tok0 + j) * 64 + row];
+                    for (int m = 0; m < 16; ++m) {
+                        const uint32_t mine = is_gate ? v[m] : v[16 + m];
+                        const uint32_t other = __shfl_xor_sync(0xFFFFFFFFu, is_gate ? v[16 + m] : v[m], 16);
+                        const float g = gsc * __uint_as_float(is_gate ? mine : other);
+                        const float u = gsc * __uint_as_float(is_gate ? other : mine);
                         // h = bf16(a); the INT4 down GEMM reads it as f16 (the same value)
-                        const uint16_t hb = f32_to_bf16(hv);
-                        hcol[(size_t)(r0 + tok0 + j) * a.N] =
+                        const uint16_t hb = f32_to_bf16(silu_f32(g) * u);
+                        hrow[(size_t)m * a.N] =
                             FMT == W4_INT4 ? (uint16_t)(pack_f16x2(__uint_as_float((uint32_t)hb << 16), 0.f) & 0xFFFFu) : hb;
                     }
                 }
@@ -376,11 +373,11 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
                     }
                 }
             }
-            // this warp has read its accumulator lanes: the next tile's MMAs may overwrite them
-            tc::fence_before_sync();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(acc_empty);
         }
+        // this warp has read its accumulator lanes: the next tile's MMAs may overwrite them
+        tc::fence_before_sync();
+        __syncwarp();
+        tc::mbar_arrive_lane0(smem_addr(acc_empty), lane);
         }  // output tiles
     }
     tc::fence_before_sync();
@@ -456,11 +453,11 @@ int launch_w4a16_tc(const W4TcArgs &a_in, int mode, const uint16_t *act, int max
     const int rc = make_tmap_2d(&tm, act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)a_in.M, (uint64_t)a_in.K,
                                 kTok, kKs / 2);
     if (rc) return rc;
-    // down: several 128-row output tiles per CTA share one pipeline (set-up, ring fill, weight
-    // prefetch across the tile boundary)
+    // several output tiles per CTA share one pipeline (set-up, ring fill, weight prefetch across
+    // the tile boundary)
     W4TcArgs a = a_in;
-    a.tiles_per_cta = mode == TC_GATEUP ? 1 : kDownTilesPerCta;
-    const int gx = mode == TC_GATEUP ? a.N / 64 : cdiv(a.N / 128, a.tiles_per_cta);
+    a.tiles_per_cta = mode == TC_GATEUP ? kGateUpTilesPerCta : kDownTilesPerCta;
+    const int gx = cdiv(a.N / (mode == TC_GATEUP ? 64 : 128), a.tiles_per_cta);
     if (a.fmt == W4_FP4) {
         if (mode == TC_GATEUP) return launch_mode<TC_GATEUP, W4_FP4>(a, tm, gx, max_blocks, s);
         return launch_mode<TC_DOWN, W4_FP4>(a, tm, gx, max_blocks, s);
