@@ -66,6 +66,18 @@ __device__ __forceinline__ bool mbar_try_wait_addr(uint32_t bar_addr, uint32_t p
     return ok != 0;
 }
 
+// True in exactly one lane of the (converged) calling warp.
+__device__ __forceinline__ bool elect_one()
+{
+    uint32_t pred;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "elect.sync _|p, 0xFFFFFFFF;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
+}
+
 // Arrival of lane 0 of the calling warp (predicated, no branch).
 __device__ __forceinline__ void mbar_arrive_lane0(uint32_t bar_addr, int lane)
 {
@@ -191,6 +203,12 @@ __device__ __forceinline__ void mma_f16_ts_acc(uint32_t d_tmem, uint32_t a_tmem,
 __device__ __forceinline__ void mma_commit(uint64_t *bar)
 {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void mma_commit_addr(uint32_t bar_addr)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar_addr)
                  : "memory");
 }
 

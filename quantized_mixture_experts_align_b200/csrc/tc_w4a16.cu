@@ -176,45 +176,59 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
                 tc::mbar_drain(&a_full[gs % kBStages], (gs / kBStages) & 1, a.status);
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            constexpr uint32_t kFmt = FMT == W4_INT4 ? tc::kFmtF16 : tc::kFmtBF16;
-            const uint32_t idesc = tc::idesc_f32(kFmt, kFmt, 128, n_mma);
-            // lean issue path: stage bases precomputed, the first step peeled, then MMAs that always
-            // accumulate (the dequantization warps keep this SM's issue slots busy)
-            const uint32_t a_base = tmem + kAccCols;
-            const uint64_t b_base = tc::smem_desc_sw128(btiles);
-            bool live = true;
-            for (int tt = 0, gs = 0; tt < nt && live; ++tt) {
+        // The whole warp runs the issue loop, so its operands stay warp-uniform; one elected lane
+        // issues each step's MMAs and its commit. (Issued by lane 0 alone inside a divergent
+        // branch, the loop took ~1100 cycles per step for 8 MMAs whatever their N: its operand
+        // set-up competed for issue slots with the dequantization warps of its sub-partition.)
+        constexpr uint32_t kFmt = FMT == W4_INT4 ? tc::kFmtF16 : tc::kFmtBF16;
+        const uint32_t idesc = tc::idesc_f32(kFmt, kFmt, 128, n_mma);
+        const uint32_t a_base = tmem + kAccCols;
+        const uint64_t b_base = tc::smem_desc_sw128(btiles);
+        const uint32_t a_full0 = smem_addr(a_full), empty0 = smem_addr(empty);
+        uint32_t s = 0, ph = 0;  // stage of the next step (weights and activation tile), its parity
+        bool live = true;
+        for (int tt = 0; tt < nt && live; ++tt) {
             // a new tile overwrites the accumulator: the previous tile's epilogue has read it
-            if (tt > 0 && !tc::mbar_wait(acc_empty, (tt - 1) & 1, abort_flag, a.status)) break;
-            for (int ks = 0; ks < NS; ++ks, ++gs) {
-                const int s = gs % kStages, sb = gs % kBStages;  // equal: one stage index
+            if (tt > 0 && !tc::mbar_wait_warp(acc_empty, (tt - 1) & 1, abort_flag, a.status)) break;
+            for (int ks = 0; ks < NS; ++ks) {
                 // one wait per step: a_full completes when the weight stage and the activation tile
                 // are both in place
-                if (!tc::mbar_wait(&a_full[s], (gs / kStages) & 1, abort_flag, a.status)) {
+                if (!__all_sync(0xFFFFFFFFu, tc::mbar_try_wait_addr(a_full0 + 8u * s, ph)) &&
+                    !tc::mbar_wait_warp(&a_full[s], ph, abort_flag, a.status)) {
                     live = false;
                     break;
                 }
                 tc::fence_after_sync();
-                const uint64_t bdesc = b_base + (uint64_t)((sb * kBTile) >> 4);
+                const uint64_t bdesc = b_base + (uint64_t)(s * (kBTile >> 4));
                 const uint32_t astage = a_base + s * kAStageCols;
-                if (ks == 0) {
+                if (tc::elect_one()) {
+                    if (ks == 0) {
 #pragma unroll
-                    for (int kk = 0; kk < kKs / 16; ++kk)
-                        tc::mma_f16_ts(tmem, astage + kk * 8, bdesc + (kk >> 2) * (kBHalf >> 4) + 2 * (kk & 3), idesc,
-                                       kk > 0 ? 1u : 0u);
-                } else {
+                        for (int kk = 0; kk < kKs / 16; ++kk)
+                            tc::mma_f16_ts(tmem, astage + kk * 8, bdesc + (kk >> 2) * (kBHalf >> 4) + 2 * (kk & 3), idesc,
+                                           kk > 0 ? 1u : 0u);
+                    } else {
 #pragma unroll
-                    for (int kk = 0; kk < kKs / 16; ++kk)
-                        tc::mma_f16_ts_acc(tmem, astage + kk * 8, bdesc + (kk >> 2) * (kBHalf >> 4) + 2 * (kk & 3), idesc);
+                        for (int kk = 0; kk < kKs / 16; ++kk)
+                            tc::mma_f16_ts_acc(tmem, astage + kk * 8, bdesc + (kk >> 2) * (kBHalf >> 4) + 2 * (kk & 3),
+                                               idesc);
+                    }
+                    tc::mma_commit_addr(empty0 + 8u * s);  // frees the weight stage and the activation tile
                 }
-                tc::mma_commit(&empty[s]);  // frees the weight stage and the activation tile
+                __syncwarp();
+                if (++s == kStages) {
+                    s = 0;
+                    ph ^= 1u;
+                }
             }
-            if (live) tc::mma_commit(acc_full);  // this tile's accumulator is complete
-            }
-            tc::mma_commit(mma_done);
-            tc::mbar_drain(mma_done, 0, a.status);
+            if (live && tc::elect_one()) tc::mma_commit(acc_full);  // this tile's accumulator is complete
+            __syncwarp();
         }
+        // every MMA issued must finish before tensor memory is released (the commit comes from
+        // the lane that issued them: elect.sync picks the same lane of the converged warp)
+        if (tc::elect_one()) tc::mma_commit(mma_done);
+        __syncwarp();
+        if (lane == 0) tc::mbar_drain(mma_done, 0, a.status);
     } else {
         // ---- dequantization ----
         const int dw = warp - 2, quarter = warp & 3, kq = dw >> 2;  // lane quarter, K slice
