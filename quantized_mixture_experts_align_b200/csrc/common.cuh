@@ -216,6 +216,10 @@ __device__ __forceinline__ void mma_e4m3_16832(float (&d)[4], uint32_t a0, uint3
 }
 
 __device__ __forceinline__ float silu_f32(float g) { return g / (1.0f + expf(-g)); }
+// The same with the fast exponential and division (relative error a few f32 ulp, far below the
+// bf16 rounding of h = bf16(silu(g) * u) in the 4-bit tensor-core GEMM); e^-g overflowing to +inf
+// gives -0.
+__device__ __forceinline__ float silu_fast_f32(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 }  // namespace moeq
 

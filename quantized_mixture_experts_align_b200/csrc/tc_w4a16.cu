@@ -17,8 +17,10 @@
 // dequantization, not the MMA, bounds this kernel, and the wide tile halves it per FLOP. The
 // MMA's N is the block's real row count rounded up to 16, so padding rows cost no MMA work.
 // One shift + LOP3 extracts the nibble pairs (q0,q4) (q1,q5) (q2,q6) (q3,q7) of a 32-bit code
-// word; four byte permutes put them in natural order, so the activation rows keep their own order:
-// the gather copies the routed rows of x as they are, and h is written in natural order.
+// word, and the weights enter tensor memory in that order: within every 8 inputs the K order is
+// 0 4 1 5 2 6 3 7. The activations take the same order (the gather permutes each 8-input group of
+// the routed rows it copies, the gate/up epilogue writes h that way), so the sum over K is
+// unchanged and the dequantization needs no byte permutes.
 //
 // CTA = one 256-row activation block of one expert x consecutive output tiles, run back to back
 // through one pipeline (gate/up: tiles of 64 features, each tensor-memory lane quarter holding the
@@ -90,11 +92,11 @@ __device__ __forceinline__ void dequant4(uint32_t w, uint32_t scale2, uint32_t *
             p[i] = f16x2_mul(f16x2_sub(v, 0x64086408u), scale2);                      // (q - 8) * s, exact
         }
     }
-    // natural order (q0,q1) (q2,q3) (q4,q5) (q6,q7): the activation rows need no reordering
-    out[0] = prmt(p[0], p[1], 0x5410u);
-    out[1] = prmt(p[2], p[3], 0x5410u);
-    out[2] = prmt(p[0], p[1], 0x7632u);
-    out[3] = prmt(p[2], p[3], 0x7632u);
+    // K order 0 4 1 5 2 6 3 7 (the activations are permuted alike)
+    out[0] = p[0];
+    out[1] = p[1];
+    out[2] = p[2];
+    out[3] = p[3];
 }
 
 template <int MODE, int FMT>
@@ -344,7 +346,9 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
             if (ok) {
                 tc::fence_after_sync();
                 const bool is_gate = lane < 16;
-                uint16_t *hcol = a.h_out + n0 + tt * 64 + 16 * quarter + (lane & 15);
+                // feature f goes to column f of h with the 8-group K order 0 4 1 5 2 6 3 7
+                const int j8 = lane & 7;
+                uint16_t *hcol = a.h_out + n0 + tt * 64 + 16 * quarter + (lane & 8) + (j8 < 4 ? 2 * j8 : 2 * j8 - 7);
                 for (int c = 0; c < kTok / kSplit / 32; ++c) {
                     const int tok0 = kq * (kTok / kSplit) + c * 32;
                     if (tok0 >= n_mma) break;
@@ -359,7 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
                         const float g = gsc * __uint_as_float(is_gate ? mine : other);
                         const float u = gsc * __uint_as_float(is_gate ? other : mine);
                         // h = bf16(a); the INT4 down GEMM reads it as f16 (the same value)
-                        const uint16_t hb = f32_to_bf16(silu_f32(g) * u);
+                        const uint16_t hb = f32_to_bf16(silu_fast_f32(g) * u);
                         hrow[(size_t)m * a.N] =
                             FMT == W4_INT4 ? (uint16_t)(pack_f16x2(__uint_as_float((uint32_t)hb << 16), 0.f) & 0xFFFFu) : hb;
                     }
@@ -400,8 +404,9 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
     if (warp == 1) tc::tmem_dealloc(tmem, kTmemCols);
 }
 
-// Gather of bf16 activation rows into aligned order (row r takes row sorted_ids[r] / k of x),
-// converted to f16 for the INT4 GEMMs (TO_F16); one warp per row, 16-byte copies. Only the rows the MMAs read are written: the real rows and the zero
+// Gather of bf16 activation rows into aligned order (row r takes row sorted_ids[r] / k of x), each
+// 8-input group in the K order of the dequantized weights (0 4 1 5 2 6 3 7), converted to f16 for
+// the INT4 GEMMs (TO_F16); one warp per row, 16-byte copies. Only the rows the MMAs read are written: the real rows and the zero
 // padding up to the block's real count rounded up to 16 (the MMA's N); blocks with at most
 // small_rows real rows belong to the register-fed kernel, which reads x itself.
 template <bool TO_F16>
@@ -433,6 +438,12 @@ __global__ void __launch_bounds__(256) gather_bf16_kernel(const uint16_t *__rest
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const int i = i0 + 32 * u;
+                // (x0 x1) (x2 x3) (x4 x5) (x6 x7) -> (x0 x4) (x1 x5) (x2 x6) (x3 x7)
+                const uint4 w = v[u];
+                v[u].x = prmt(w.x, w.z, 0x5410u);
+                v[u].y = prmt(w.x, w.z, 0x7632u);
+                v[u].z = prmt(w.y, w.w, 0x5410u);
+                v[u].w = prmt(w.y, w.w, 0x7632u);
                 if (TO_F16) {
                     v[u].x = bf16x2_to_f16x2(v[u].x);
                     v[u].y = bf16x2_to_f16x2(v[u].y);
