@@ -37,7 +37,7 @@
 //               are long and the MMA thread waits on one barrier and commits once per step;
 //   warps 2-17  dequantization: a thread owns one weight row (tensor lane) and a 32-input slice
 //               of each 128-input step (16 bytes of codes, 1 group scale), fetches them into
-//               registers four steps ahead, and writes the dequantized slice to one of 3
+//               registers two steps ahead, and writes the dequantized slice to one of 3
 //               tensor-memory stages; then the epilogue of each tile: gate/up pairs every gate
 //               lane with its up lane by shuffles and writes h = bf16(silu(g) * u); down writes
 //               the routing-weighted bf16 slot rows.
@@ -54,7 +54,13 @@ constexpr int kStages = 3;    // dequantized weight stages (tensor memory)
 constexpr int kDownTilesPerCta = 4;    // down GEMM: 128-row output tiles run by one CTA
 constexpr int kGateUpTilesPerCta = 2;  // gate/up GEMM: 64-feature output tiles run by one CTA
 constexpr int kBStages = 3;   // activation tiles (shared memory)
-constexpr int kPf = 4;        // per-thread packed-code prefetch depth (registers), in steps
+// Per-thread packed-code prefetch depth (registers), in steps. The code loads go through L1: the
+// four warps of a lane quarter read the four 16-byte quarters of each row's 64-byte step chunk, so
+// the first warp's miss serves the other three (no-allocate loads ran 35 % slower). In-flight loads
+// therefore hold L1 lines, and L1 is what shared memory leaves of the SM's 256 KB: measured, 2
+// steps ran 2 % faster than 4 and 6 much slower, and 30 KB more shared memory made gate/up 47 %
+// slower.
+constexpr int kPf = 2;
 constexpr int kDeqWarps = 16;  // 4 per tensor-memory lane quarter, each a quarter of every step
 constexpr int kDeqThreads = kDeqWarps * 32;
 constexpr int kSplit = kDeqWarps / 4;           // K slices of a step (one per warp of a lane quarter)
