@@ -218,16 +218,23 @@ __global__ void __launch_bounds__(fp8_threads(MODE), 1)
             // the peer issues nothing; it waits (bounded) until the pair's MMAs, which write its
             // tensor memory and read its shared memory, are done
             if (lane == 0) tc::mbar_drain(mma_done, 0, a.status);
-        } else if (lane == 0) {
+        } else {
+            // The whole warp runs the issue loop, so its operands stay warp-uniform; one elected
+            // lane issues each K block's MMAs and commits (a lane-0 loop inside a divergent branch
+            // competes for issue slots with the promotion warps of its sub-partition).
             constexpr uint32_t idesc = tc::idesc_f32(tc::kFmtE4M3, tc::kFmtE4M3, PAIR ? 2 * kBM : kBM, BN);
             const uint64_t a_base = tc::smem_desc_sw128(smem);
+            const uint32_t full0 = smem_addr(full), tempty0 = smem_addr(tempty);
+            uint32_t s = 0, ph = 0;      // ring stage of the next K block, its parity
+            uint32_t buf = 0, pbuf = 0;  // partial buffer of the next K block, its parity
             bool live = true;
             for (int tt = 0, gs = 0; tt < ntl && live; ++tt)
             for (int kb = 0; kb < nkb; ++kb, ++gs) {
-                const int s = gs % kStages, buf = gs % NB;
-                if (!tc::mbar_wait(&full[s], (gs / kStages) & 1, abort_flag, a.status) ||
+                if ((!__all_sync(0xFFFFFFFFu, tc::mbar_try_wait_addr(full0 + 8u * s, ph)) &&
+                     !tc::mbar_wait_warp(&full[s], ph, abort_flag, a.status)) ||
                     (MODE != TC_DENSE_CW && gs >= NB &&
-                     !tc::mbar_wait(&tempty[buf], ((gs / NB) & 1) ^ 1, abort_flag, a.status))) {
+                     !__all_sync(0xFFFFFFFFu, tc::mbar_try_wait_addr(tempty0 + 8u * buf, pbuf ^ 1u)) &&
+                     !tc::mbar_wait_warp(&tempty[buf], pbuf ^ 1u, abort_flag, a.status))) {
                     live = false;
                     break;
                 }
@@ -239,31 +246,48 @@ __global__ void __launch_bounds__(fp8_threads(MODE), 1)
                 const uint32_t d = tmem + buf * BN;
                 // channelwise: only the very first MMA starts the accumulator
                 const uint32_t first_acc = (MODE == TC_DENSE_CW && kb > 0) ? 1u : 0u;
-                if (PAIR) {
-                    tc::mma_f8f6f4_ss_pair(d, adesc, bdesc, idesc, first_acc);
+                if (tc::elect_one()) {
+                    if (PAIR) {
+                        tc::mma_f8f6f4_ss_pair(d, adesc, bdesc, idesc, first_acc);
 #pragma unroll
-                    for (int kk = 1; kk < kBK / 32; ++kk)
-                        tc::mma_f8f6f4_ss_pair_acc(d, adesc + 2 * kk, bdesc + 2 * kk, idesc);
-                    tc::mma_commit_pair(&empty[s], 0x3);
-                    if (MODE != TC_DENSE_CW) tc::mma_commit_pair(&tfull[buf], 0x3);
-                } else {
-                    tc::mma_f8f6f4_ss(d, adesc, bdesc, idesc, first_acc);
+                        for (int kk = 1; kk < kBK / 32; ++kk)
+                            tc::mma_f8f6f4_ss_pair_acc(d, adesc + 2 * kk, bdesc + 2 * kk, idesc);
+                        tc::mma_commit_pair(&empty[s], 0x3);
+                        if (MODE != TC_DENSE_CW) tc::mma_commit_pair(&tfull[buf], 0x3);
+                    } else {
+                        tc::mma_f8f6f4_ss(d, adesc, bdesc, idesc, first_acc);
 #pragma unroll
-                    for (int kk = 1; kk < kBK / 32; ++kk)
-                        tc::mma_f8f6f4_ss_acc(d, adesc + 2 * kk, bdesc + 2 * kk, idesc);
-                    tc::mma_commit(&empty[s]);
-                    if (MODE != TC_DENSE_CW) tc::mma_commit(&tfull[buf]);
+                        for (int kk = 1; kk < kBK / 32; ++kk)
+                            tc::mma_f8f6f4_ss_acc(d, adesc + 2 * kk, bdesc + 2 * kk, idesc);
+                        tc::mma_commit(&empty[s]);
+                        if (MODE != TC_DENSE_CW) tc::mma_commit(&tfull[buf]);
+                    }
+                }
+                __syncwarp();
+                if (++s == (uint32_t)kStages) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+                if (++buf == (uint32_t)NB) {
+                    buf = 0;
+                    pbuf ^= 1u;
                 }
             }
+            // (the commits below come from the lane that issued the MMAs: elect.sync picks the
+            // same lane of the converged warp)
             // channelwise: the accumulator is complete once every MMA issued so far has finished
-            if (MODE == TC_DENSE_CW) {
+            if (MODE == TC_DENSE_CW && tc::elect_one()) {
                 if (PAIR) tc::mma_commit_pair(&tfull[0], 0x3);
                 else tc::mma_commit(&tfull[0]);
             }
+            __syncwarp();
             // every MMA issued must finish before tensor memory is released
-            if (PAIR) tc::mma_commit_pair(mma_done, 0x3);
-            else tc::mma_commit(mma_done);
-            tc::mbar_drain(mma_done, 0, a.status);
+            if (tc::elect_one()) {
+                if (PAIR) tc::mma_commit_pair(mma_done, 0x3);
+                else tc::mma_commit(mma_done);
+            }
+            __syncwarp();
+            if (lane == 0) tc::mbar_drain(mma_done, 0, a.status);
         }
     } else if (MODE == TC_DENSE_CW) {
         // warp w: tensor-memory lanes 32 (w % 4) .. +31 (= tile rows) and column slice cq; one
