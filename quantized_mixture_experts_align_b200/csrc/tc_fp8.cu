@@ -174,45 +174,55 @@ __global__ void __launch_bounds__(fp8_threads(MODE), 1)
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
+        // the whole warp runs the producer loop (warp-uniform operands); one elected lane issues
+        // each stage's copies
         if (lane == 0) {
             tc::prefetch_tmap(&tmA);
             tc::prefetch_tmap(&tmB);
-            int issued = 0;
-            bool live = true;
-            for (int tt = 0, gs = 0; tt < ntl && live; ++tt)
-            for (int kb = 0; kb < nkb; ++kb, ++gs) {  // local K index, x = (kb0 + kb) * kBK; gs over tiles
-                const int s = gs % kStages;
-                if (gs >= kStages && !tc::mbar_wait(&empty[s], ((gs / kStages) & 1) ^ 1, abort_flag, a.status)) {
-                    live = false;
-                    break;
-                }
-                uint8_t *sa = smem + s * Sh::kStageBytes;
+        }
+        const uint32_t empty0 = smem_addr(empty);
+        uint32_t s = 0, ph = 0;  // ring stage of the next K block, its parity
+        int issued = 0;
+        bool live = true;
+        for (int tt = 0, gs = 0; tt < ntl && live; ++tt)
+        for (int kb = 0; kb < nkb; ++kb, ++gs) {  // local K index, x = (kb0 + kb) * kBK; gs over tiles
+            if (gs >= kStages && !__all_sync(0xFFFFFFFFu, tc::mbar_try_wait_addr(empty0 + 8u * s, ph ^ 1u)) &&
+                !tc::mbar_wait_warp(&empty[s], ph ^ 1u, abort_flag, a.status)) {
+                live = false;
+                break;
+            }
+            uint8_t *sa = smem + s * Sh::kStageBytes;
+            if (tc::elect_one()) {
                 if (PAIR) {
                     // both CTAs' bytes complete on rank 0's barrier, which alone expects them
                     const uint32_t fb = tc::cluster_addr(&full[s], 0);
                     if (rank == 0) tc::mbar_arrive_expect_tx(&full[s], 2 * Sh::kStageBytes);
                     tc::tma_load_2d_pair(sa, &tmA, fb, kb * kBK, m0);
                     tc::tma_load_2d_pair(sa + Sh::kABytes, &tmB, fb, kb * kBK, brow_own);
-                    issued = gs + 1;
-                    continue;
-                }
-                tc::mbar_arrive_expect_tx(&full[s], Sh::kStageBytes);
-                const int x = (kb0 + kb) * kBK;
-                tc::tma_load_2d(sa, &tmA, &full[s], x, m0);
-                if (MODE == TC_GATEUP) {
-                    tc::tma_load_2d(sa + Sh::kABytes, &tmB, &full[s], x, brow0);
-                    tc::tma_load_2d(sa + Sh::kABytes + 128 * kBK, &tmB, &full[s], x, brow1);
                 } else {
-                    tc::tma_load_2d(sa + Sh::kABytes, &tmB, &full[s], x, brow0 + tt * BN);
+                    tc::mbar_arrive_expect_tx(&full[s], Sh::kStageBytes);
+                    const int x = (kb0 + kb) * kBK;
+                    tc::tma_load_2d(sa, &tmA, &full[s], x, m0);
+                    if (MODE == TC_GATEUP) {
+                        tc::tma_load_2d(sa + Sh::kABytes, &tmB, &full[s], x, brow0);
+                        tc::tma_load_2d(sa + Sh::kABytes + 128 * kBK, &tmB, &full[s], x, brow1);
+                    } else {
+                        tc::tma_load_2d(sa + Sh::kABytes, &tmB, &full[s], x, brow0 + tt * BN);
+                    }
                 }
-                issued = gs + 1;
             }
-            // no copy may still be landing in shared memory when the CTA exits (pair: rank 0's
-            // barrier counts both CTAs' bytes; rank 1 is held by the final cluster barrier)
-            if (!PAIR || rank == 0)
-                for (int gs = issued - kStages > 0 ? issued - kStages : 0; gs < issued; ++gs)
-                    tc::mbar_drain(&full[gs % kStages], (gs / kStages) & 1, a.status);
+            __syncwarp();
+            issued = gs + 1;
+            if (++s == (uint32_t)kStages) {
+                s = 0;
+                ph ^= 1u;
+            }
         }
+        // no copy may still be landing in shared memory when the CTA exits (pair: rank 0's
+        // barrier counts both CTAs' bytes; rank 1 is held by the final cluster barrier)
+        if (lane == 0 && (!PAIR || rank == 0))
+            for (int gs = issued - kStages > 0 ? issued - kStages : 0; gs < issued; ++gs)
+                tc::mbar_drain(&full[gs % kStages], (gs / kStages) & 1, a.status);
     } else if (warp == 1) {
         if (PAIR && rank != 0) {
             // the peer issues nothing; it waits (bounded) until the pair's MMAs, which write its

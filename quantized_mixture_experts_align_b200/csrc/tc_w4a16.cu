@@ -160,29 +160,38 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
-        if (lane == 0) {
-            tc::prefetch_tmap(&tmX);
-            int issued = 0;
-            bool live = true;
-            for (int tt = 0, gs = 0; tt < nt && live; ++tt) {
-                for (int ks = 0; ks < NS; ++ks, ++gs) {  // gs: global step over the tiles
-                    const int s = gs % kBStages;
-                    if (gs >= kBStages &&
-                        !tc::mbar_wait(&empty[s], ((gs / kBStages) & 1) ^ 1, abort_flag, a.status)) {
-                        live = false;
-                        break;
-                    }
-                    // the tile's bytes complete on the stage's a_full barrier (dequantization warps +
-                    // this arrival): the MMA thread waits on one barrier per step
+        // the whole warp runs the producer loop (warp-uniform operands); one elected lane issues
+        // each tile's copies
+        if (lane == 0) tc::prefetch_tmap(&tmX);
+        const uint32_t empty0 = smem_addr(empty);
+        uint32_t s = 0, ph = 0;  // stage of the next step, its parity
+        int issued = 0;
+        bool live = true;
+        for (int tt = 0, gs = 0; tt < nt && live; ++tt) {
+            for (int ks = 0; ks < NS; ++ks, ++gs) {  // gs: global step over the tiles
+                if (gs >= kBStages && !__all_sync(0xFFFFFFFFu, tc::mbar_try_wait_addr(empty0 + 8u * s, ph ^ 1u)) &&
+                    !tc::mbar_wait_warp(&empty[s], ph ^ 1u, abort_flag, a.status)) {
+                    live = false;
+                    break;
+                }
+                // the tile's bytes complete on the stage's a_full barrier (dequantization warps +
+                // this arrival): the MMA warp waits on one barrier per step
+                if (tc::elect_one()) {
                     tc::mbar_arrive_expect_tx(&a_full[s], kBTile);
                     tc::tma_load_2d(btiles + s * kBTile, &tmX, &a_full[s], ks * kKs, r0);
                     tc::tma_load_2d(btiles + s * kBTile + kBHalf, &tmX, &a_full[s], ks * kKs + kKs / 2, r0);
-                    issued = gs + 1;
+                }
+                __syncwarp();
+                issued = gs + 1;
+                if (++s == kBStages) {
+                    s = 0;
+                    ph ^= 1u;
                 }
             }
+        }
+        if (lane == 0)
             for (int gs = issued - kBStages > 0 ? issued - kBStages : 0; gs < issued; ++gs)
                 tc::mbar_drain(&a_full[gs % kBStages], (gs / kBStages) & 1, a.status);
-        }
     } else if (warp == 1) {
         // The whole warp runs the issue loop, so its operands stay warp-uniform; one elected lane
         // issues each step's MMAs and its commit. (Issued by lane 0 alone inside a divergent
