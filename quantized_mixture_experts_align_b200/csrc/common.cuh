@@ -134,6 +134,27 @@ __device__ __forceinline__ uint32_t f16x2_sub(uint32_t a, uint32_t b)
     return r;
 }
 
+__device__ __forceinline__ uint32_t f16x2_fma(uint32_t a, uint32_t b, uint32_t c)
+{
+    uint32_t r;
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+    return r;
+}
+
+// Unsigned INT4 nibble pairs of a code word minus the zero point 8, as exact f16x2 values
+// (q - 8 in [-8, 7]): pair i holds nibbles i and i + 4. Nibbles 0 and 4 (2, 6 after a shift by 8)
+// are ORed into the mantissa of 1024 (f16 1024 + q) and take 1032 off; nibbles 1 and 5 (3, 7)
+// are masked in place, giving 1024 + 16 q, and one FMA by 1/16 minus 72 yields q - 8, saving their
+// shift. Every intermediate is an integer or a power-of-two fraction that f16 holds exactly.
+__device__ __forceinline__ void int4_pairs_minus8(uint32_t w, uint32_t (&p)[4])
+{
+    const uint32_t w8 = w >> 8;
+    p[0] = f16x2_sub(lop3_and_or(w, 0x000F000Fu, 0x64006400u), 0x64086408u);
+    p[1] = f16x2_fma(lop3_and_or(w, 0x00F000F0u, 0x64006400u), 0x2C002C00u, 0xD480D480u);  // x/16 - 72
+    p[2] = f16x2_sub(lop3_and_or(w8, 0x000F000Fu, 0x64006400u), 0x64086408u);
+    p[3] = f16x2_fma(lop3_and_or(w8, 0x00F000F0u, 0x64006400u), 0x2C002C00u, 0xD480D480u);
+}
+
 __device__ __forceinline__ uint32_t f16x2_mul(uint32_t a, uint32_t b)
 {
     uint32_t r;

@@ -16,8 +16,8 @@
 // A tile serves up to 256 tokens, so each dequantized weight feeds 256 rows of MMA work: the
 // dequantization, not the MMA, bounds this kernel, and the wide tile halves it per FLOP. The
 // MMA's N is the block's real row count rounded up to 16, so padding rows cost no MMA work.
-// One shift + LOP3 extracts the nibble pairs (q0,q4) (q1,q5) (q2,q6) (q3,q7) of a 32-bit code
-// word, and the weights enter tensor memory in that order: within every 8 inputs the K order is
+// LOP3s (one shift per word) extract the nibble pairs (q0,q4) (q1,q5) (q2,q6) (q3,q7) of a 32-bit
+// code word, and the weights enter tensor memory in that order: within every 8 inputs the K order is
 // 0 4 1 5 2 6 3 7. The activations take the same order (the gather permutes each 8-input group of
 // the routed rows it copies, the gate/up epilogue writes h that way), so the sum over K is
 // unchanged and the dequantization needs no byte permutes.
@@ -85,18 +85,16 @@ static_assert(kBStages == kStages, "one stage-free barrier serves the activation
 template <int FMT>
 __device__ __forceinline__ void dequant4(uint32_t w, uint32_t scale2, uint32_t *out)
 {
-    uint32_t p[4];  // the pairs one shift + LOP3 yields: (q0,q4) (q1,q5) (q2,q6) (q3,q7)
+    uint32_t p[4];  // the nibble pairs (q0,q4) (q1,q5) (q2,q6) (q3,q7)
     if (FMT == W4_FP4 || FMT == W4_NV) {
         p[0] = bf16x2_mul(e2m1_pair_pre<0>(w), scale2);
         p[1] = bf16x2_mul(e2m1_pair_pre<1>(w), scale2);
         p[2] = bf16x2_mul(e2m1_pair_pre<2>(w), scale2);
         p[3] = bf16x2_mul(e2m1_pair_pre<3>(w), scale2);
     } else {
+        int4_pairs_minus8(w, p);  // q - 8, exact
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint32_t v = lop3_and_or(w >> (4 * i), 0x000F000Fu, 0x64006400u);  // f16 1024 + q, exact
-            p[i] = f16x2_mul(f16x2_sub(v, 0x64086408u), scale2);                      // (q - 8) * s, exact
-        }
+        for (int i = 0; i < 4; ++i) p[i] = f16x2_mul(p[i], scale2);  // (q - 8) * s, exact
     }
     // K order 0 4 1 5 2 6 3 7 (the activations are permuted alike)
     out[0] = p[0];

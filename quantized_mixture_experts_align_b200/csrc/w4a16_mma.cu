@@ -17,9 +17,10 @@
 // Input permutation. The sum over K does not care about order, so inside a 128-input
 // "quad-group" lane t (of a 4-lane quad) takes the 32 inputs of group t = 16 contiguous bytes of
 // the row, which keeps each element with its own group scale. Word m of that group feeds
-// k-steps 2m and 2m+1; its nibble pairs (0,4), (1,5), (2,6), (3,7) are extracted with one shift
-// and one LOP3 each (magic 0x4300 = bf16 128.0, nibble in the low mantissa bits), so the
-// activation fragments take the same pairs, rebuilt with PRMT from a 16-byte load.
+// k-steps 2m and 2m+1; its nibble pairs (0,4), (1,5), (2,6), (3,7) are extracted with one LOP3
+// each (INT4: the nibble ORed into the mantissa of f16 1024, one shift by 8 per word; E2M1: see
+// e2m1_pair_pre), so the activation fragments take the same pairs, rebuilt with PRMT from a
+// 16-byte load.
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -44,13 +45,10 @@ __device__ __forceinline__ DeqWord dequant_word(uint32_t w, uint32_t scale2)
         d.p[2] = bf16x2_mul(e2m1_pair_pre<2>(w), scale2);
         d.p[3] = bf16x2_mul(e2m1_pair_pre<3>(w), scale2);
     } else {
-        const uint32_t magic = 0x64006400u;  // f16 1024.0 in both halves
-        const uint32_t bias = 0x64086408u;   // f16 1032.0 = 1024 + 8 (zero point) in both halves
+        uint32_t q8[4];
+        int4_pairs_minus8(w, q8);  // q - 8, exact
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint32_t v = lop3_and_or(w >> (4 * i), 0x000F000Fu, magic);  // 1024 + q, exact
-            d.p[i] = f16x2_mul(f16x2_sub(v, bias), scale2);                   // (q - 8) * s, exact
-        }
+        for (int i = 0; i < 4; ++i) d.p[i] = f16x2_mul(q8[i], scale2);  // (q - 8) * s, exact
     }
     return d;
 }
