@@ -28,16 +28,17 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict
     const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (t >= T) return;
     if (xh) {
-        // the token's activation row in f16 for the INT4 GEMMs (exact for magnitudes in [2^-14, 65504])
+        // the token's activation row in f16 for the INT4 GEMMs (exact for magnitudes in [2^-14, 65504]),
+        // each 8-input group in the nibble-pair order of the register-fed kernels' weight words:
+        // (x0 x4) (x1 x5) (x2 x6) (x3 x7)
         const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)t * H);
         uint4 *dst = reinterpret_cast<uint4 *>(xh + (size_t)t * H);
         for (int i = lane; i < H / 8; i += 32) {
-            uint4 v = __ldg(src + i);
-            v.x = bf16x2_to_f16x2(v.x);
-            v.y = bf16x2_to_f16x2(v.y);
-            v.z = bf16x2_to_f16x2(v.z);
-            v.w = bf16x2_to_f16x2(v.w);
-            dst[i] = v;
+            const uint4 v = __ldg(src + i);
+            const uint32_t a0 = bf16x2_to_f16x2(v.x), a1 = bf16x2_to_f16x2(v.y);
+            const uint32_t a2 = bf16x2_to_f16x2(v.z), a3 = bf16x2_to_f16x2(v.w);
+            dst[i] = make_uint4(prmt(a0, a2, 0x5410u), prmt(a0, a2, 0x7632u), prmt(a1, a3, 0x5410u),
+                                prmt(a1, a3, 0x7632u));
         }
     }
     const float *row = logits + (size_t)t * E;

@@ -80,6 +80,13 @@ __host__ __device__ constexpr int w4_stage_bytes(int fmt) { return 4 * 32 * 16 +
 //              without routing weights: the plain grouped GEMM).
 // CVT (INT4 only): the activations are bf16 and are converted to f16 in registers; otherwise they
 // are already f16 (INT4) or bf16 (MXFP4 / NVFP4).
+// Paired activations: the library's own activation rows (the routing kernel's f16 copy of x and
+// every h this file writes) hold each 8-input group in the nibble-pair order (x0 x4) (x1 x5)
+// (x2 x6) (x3 x7), so a 16-byte load is the four MMA B registers as they are; rows the caller
+// passes (bf16 x of the gate/up GEMM in MXFP4 / NVFP4 and in the few-row blocks, the grouped
+// GEMM's A) are paired in registers.
+template <int MODE, int FMT, bool CVT>
+__host__ __device__ constexpr bool act_paired() { return !CVT && (MODE == MODE_DOWN || FMT == W4_INT4); }
 template <int BM, int WARPS, int MODE, bool STRIDED, int FMT, bool CVT>
 __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4GroupedArgs a)
 {
@@ -221,7 +228,14 @@ __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4Grouped
                     xv.w = bf16x2_to_f16x2(xv.w);
                 }
                 uint32_t b[4];
-                act_pairs(xv, b);
+                if (act_paired<MODE, FMT, CVT>()) {
+                    b[0] = xv.x;
+                    b[1] = xv.y;
+                    b[2] = xv.z;
+                    b[3] = xv.w;
+                } else {
+                    act_pairs(xv, b);
+                }
                 // k-step 2m: pairs 0/1; k-step 2m+1: pairs 2/3
                 if (FMT == W4_INT4) {
                     mma_f16_16816(accA[s], d[0].p[0], d[1].p[0], d[0].p[1], d[1].p[1], b[0], b[1]);
@@ -265,8 +279,11 @@ __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4Grouped
                 // h = bf16(silu(g) * u), stored as f16 for the INT4 down GEMM (the same value)
                 const float h0 = silu_f32(accA[s][c]) * accB[s][c];
                 const float h1 = silu_f32(accA[s][2 + c]) * accB[s][2 + c];
-                h[rowA + g] = FMT == W4_INT4 ? f32_to_bf16_as_f16(h0) : f32_to_bf16(h0);
-                h[rowA + g + 8] = FMT == W4_INT4 ? f32_to_bf16_as_f16(h1) : f32_to_bf16(h1);
+                // features rowA + g and rowA + 8 + g at their paired columns (the down GEMM reads h
+                // paired): position 2j of an 8-group holds input j < 4, position 2(j - 4) + 1 input j
+                const int pg = g < 4 ? 2 * g : 2 * g - 7;
+                h[rowA + pg] = FMT == W4_INT4 ? f32_to_bf16_as_f16(h0) : f32_to_bf16(h0);
+                h[rowA + 8 + pg] = FMT == W4_INT4 ? f32_to_bf16_as_f16(h1) : f32_to_bf16(h1);
             } else {
                 const float wt = a.topk_w ? __ldg(a.topk_w + slot) : 1.f;
                 uint16_t *y = a.y_out + (size_t)slot * a.n_out;
