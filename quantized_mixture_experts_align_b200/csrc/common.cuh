@@ -202,6 +202,10 @@ __device__ __forceinline__ uint4 ld_v4(const void *p)
     return __ldg(reinterpret_cast<const uint4 *>(p));
 }
 
+// An ordinary (coherent) 16-byte load: for data an earlier kernel of a programmatic-launch chain
+// writes, which must not be read ahead of the wait for that kernel (as __ldg may be scheduled).
+__device__ __forceinline__ uint4 ld_v4_coherent(const void *p) { return *reinterpret_cast<const uint4 *>(p); }
+
 // ---- tensor-core MMA (warp-level, register operands) ----------------------------------------
 // D[16x8] += A[16x16] (bf16, row) * B[16x8] (bf16, col), f32 accumulate.
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,

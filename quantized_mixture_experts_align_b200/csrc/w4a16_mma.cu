@@ -106,12 +106,15 @@ __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4Grouped
     pdl_trigger();
     const int blk = blockIdx.x;
     const int base = blk * (STRIDED ? a.blk_stride : BM);  // first aligned row of the block
-    const int e = __ldg(a.expert_ids + blk);
+    // Data earlier kernels of the chain write (the alignment, the routing weights, h) is read with
+    // ordinary loads, never __ldg: a read-only (non-coherent) load may be scheduled ahead of the
+    // programmatic-launch wait, and these kernels can start while their predecessor still runs.
+    const int e = a.expert_ids[blk];
     const int tile = blockIdx.y * WARPS + warp;
     const int rowA = tile * (MODE == MODE_GATEUP ? 16 : 32);
     const int rowB = MODE == MODE_GATEUP ? a.n_out + rowA : rowA + 16;
     // strided: blocks with more than BM real rows are the tensor-core path's (real rows come first)
-    if (base >= __ldg(a.num_tokens_padded) || (STRIDED && __ldg(a.sorted_ids + base + BM) < a.n_slots) || e < 0 ||
+    if (base >= *a.num_tokens_padded || (STRIDED && a.sorted_ids[base + BM] < a.n_slots) || e < 0 ||
         e >= a.E || rowA >= a.n_out) {
         if (early) pdl_wait();
         return;
@@ -126,7 +129,7 @@ __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4Grouped
     const uint16_t *act_row[MS];
 #pragma unroll
     for (int s = 0; s < MS; ++s) {
-        const int slot = __ldg(a.sorted_ids + base + 8 * s + g);
+        const int slot = a.sorted_ids[base + 8 * s + g];
         act_row[s] = (slot < a.n_slots) ? a.act + (size_t)(slot / a.act_row_div) * K : nullptr;
     }
 
@@ -170,7 +173,7 @@ __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4Grouped
         for (int s = 0; s < MS; ++s)
 #pragma unroll
             for (int m = 0; m < 4; ++m)
-                xcur[s][m] = act_row[s] ? ld_v4(act_row[s] + 32 * t + 8 * m) : make_uint4(0u, 0u, 0u, 0u);
+                xcur[s][m] = act_row[s] ? ld_v4_coherent(act_row[s] + 32 * t + 8 * m) : make_uint4(0u, 0u, 0u, 0u);
     }
 
     for (int q = 0; q < NQ; ++q) {
@@ -207,7 +210,7 @@ __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4Grouped
             for (int s = 0; s < MS; ++s)
 #pragma unroll
                 for (int m = 0; m < 4; ++m)
-                    xnext[s][m] = act_row[s] ? ld_v4(act_row[s] + kn + 8 * m) : make_uint4(0u, 0u, 0u, 0u);
+                    xnext[s][m] = act_row[s] ? ld_v4_coherent(act_row[s] + kn + 8 * m) : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
@@ -220,7 +223,7 @@ __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4Grouped
             for (int s = 0; s < MS; ++s) {
                 uint4 xv;
                 if (kActPrefetch) xv = xcur[s][m];
-                else xv = act_row[s] ? ld_v4(act_row[s] + kofs + 8 * m) : make_uint4(0u, 0u, 0u, 0u);
+                else xv = act_row[s] ? ld_v4_coherent(act_row[s] + kofs + 8 * m) : make_uint4(0u, 0u, 0u, 0u);
                 if (FMT == W4_INT4 && CVT) {
                     xv.x = bf16x2_to_f16x2(xv.x);
                     xv.y = bf16x2_to_f16x2(xv.y);
@@ -272,7 +275,7 @@ __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4Grouped
     for (int s = 0; s < MS; ++s) {
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
-            const int slot = __ldg(a.sorted_ids + base + 8 * s + 2 * t + c);
+            const int slot = a.sorted_ids[base + 8 * s + 2 * t + c];
             if (slot >= a.n_slots) continue;
             if (MODE == MODE_GATEUP) {
                 uint16_t *h = a.h_out + (size_t)slot * a.n_out;
@@ -285,7 +288,7 @@ __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4Grouped
                 h[rowA + pg] = FMT == W4_INT4 ? f32_to_bf16_as_f16(h0) : f32_to_bf16(h0);
                 h[rowA + 8 + pg] = FMT == W4_INT4 ? f32_to_bf16_as_f16(h1) : f32_to_bf16(h1);
             } else {
-                const float wt = a.topk_w ? __ldg(a.topk_w + slot) : 1.f;
+                const float wt = a.topk_w ? a.topk_w[slot] : 1.f;
                 uint16_t *y = a.y_out + (size_t)slot * a.n_out;
                 y[rowA + g] = f32_to_bf16(wt * accA[s][c]);
                 y[rowA + g + 8] = f32_to_bf16(wt * accA[s][2 + c]);
