@@ -204,8 +204,9 @@ static_assert(kW4SmallRows == 8, "the strided register-fed instantiation is buil
 // E: experts whose weights the call holds (the alignment's capacity); E_sched (0: E): experts the
 // routing picks from, whose mean load T*k/E_sched picks the schedule (under expert parallelism a
 // rank holds E of the E_sched experts, and each of them still sees T*k/E_sched rows on average).
-// fmt: the INT4 register-fed schedule also holds x converted to f16 (xh; the INT4 GEMMs compute in
-// f16), written by the routing kernel.
+// The register-fed (decode) schedule also holds a copy of x in nibble-pair order (xh: f16 for
+// INT4, whose GEMMs compute in f16; bf16 for MXFP4 / NVFP4), written by the routing kernel.
+// (fmt is kept for callers; the layout is the same for every 4-bit format.)
 static size_t w4a16_layout(Carve &c, long T, int H, int I, int E, int k, RouteBufs *rb, uint16_t **h, uint16_t **ys,
                            uint16_t **xg = nullptr, uint16_t **h_small = nullptr, int E_sched = 0, int fmt = W4_INT4,
                            uint16_t **xh = nullptr)
@@ -219,7 +220,8 @@ static size_t w4a16_layout(Carve &c, long T, int H, int I, int E, int k, RouteBu
     uint16_t *xgp = tcp ? c.take<uint16_t>(cap * H) : nullptr;  // routed rows of x in aligned order
     // small blocks of the tensor-core schedule: h in slot order
     uint16_t *hsp = tcp ? c.take<uint16_t>((size_t)T * k * I) : nullptr;
-    uint16_t *xhp = (!tcp && fmt == W4_INT4) ? c.take<uint16_t>((size_t)T * H) : nullptr;
+    // the decode schedule's copy of x in nibble-pair order (f16 for INT4), written by the routing kernel
+    uint16_t *xhp = !tcp ? c.take<uint16_t>((size_t)T * H) : nullptr;
     if (rb) *rb = r;
     if (h) *h = hp;
     if (ys) *ys = yp;
@@ -426,7 +428,7 @@ static int w4_layer_forward(int fmt, const char *name, const uint16_t *x, const 
 
     {
         trace::Scope ts(trace::ROUTE, s);
-        launch_route_topk(logits, T, E, k, ids, tw, s, lids, ep_base, ep_local, x, H, xh);
+        launch_route_topk(logits, T, E, k, ids, tw, s, lids, ep_base, ep_local, x, H, xh, fmt == W4_INT4);
     }
     {
         trace::Scope ts(trace::ALIGN, s);
@@ -524,8 +526,8 @@ static int w4_layer_forward(int fmt, const char *name, const uint16_t *x, const 
         a.num_tokens_padded = r.ntp;
         a.n_slots = n;
         a.topk_w = tw;
-        // gate/up + SiLU*up (INT4: x in f16, converted by the routing kernel)
-        a.act = xh ? xh : x;
+        // gate/up + SiLU*up on the routing kernel's copy of x (nibble-pair order; f16 for INT4)
+        a.act = xh;
         a.act_row_div = k;
         a.wq = w13_q;
         a.ws = w13_s;

@@ -110,10 +110,11 @@ struct W4TcArgs {
 
 // local_ids (nullable): the picks relative to the expert range [ep_base, ep_base + ep_local), -1
 // outside it; ids may be null when local_ids is given.
-// xh (nullable): also writes x [T, H] (bf16) as f16 into xh [T, H].
+// xh (nullable): also copies x [T, H] (bf16) into xh [T, H], each 8-input group in nibble-pair
+// order, converted to f16 when xh_f16.
 void launch_route_topk(const float *logits, int T, int E, int k, int32_t *ids, float *w, cudaStream_t s,
                        int32_t *local_ids = nullptr, int ep_base = 0, int ep_local = 0, const uint16_t *x = nullptr,
-                       int H = 0, uint16_t *xh = nullptr);
+                       int H = 0, uint16_t *xh = nullptr, bool xh_f16 = true);
 // Scratch (bytes) the alignment of n slots over E experts uses; 0 = the one-CTA kernel, which
 // also runs when launch_align gets no scratch.
 size_t align_scratch_bytes(int n, int E);

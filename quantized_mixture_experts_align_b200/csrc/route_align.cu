@@ -21,22 +21,22 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict
                                                          float *__restrict__ w,
                                                          int32_t *__restrict__ local_ids, int ep_base,
                                                          int ep_local, const uint16_t *__restrict__ x, int H,
-                                                         uint16_t *__restrict__ xh)
+                                                         uint16_t *__restrict__ xh, int xh_f16)
 {
     pdl_trigger();  // the alignment after this kernel may launch (it waits for these ids)
     const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (t >= T) return;
     if (xh) {
-        // the token's activation row in f16 for the INT4 GEMMs (exact for magnitudes in [2^-14, 65504]),
-        // each 8-input group in the nibble-pair order of the register-fed kernels' weight words:
-        // (x0 x4) (x1 x5) (x2 x6) (x3 x7)
+        // the token's activation row for the register-fed GEMMs, each 8-input group in the
+        // nibble-pair order of their weight words: (x0 x4) (x1 x5) (x2 x6) (x3 x7); in f16 for the
+        // INT4 GEMMs (xh_f16; exact for magnitudes in [2^-14, 65504]), else bf16 as it is
         const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)t * H);
         uint4 *dst = reinterpret_cast<uint4 *>(xh + (size_t)t * H);
         for (int i = lane; i < H / 8; i += 32) {
             const uint4 v = __ldg(src + i);
-            const uint32_t a0 = bf16x2_to_f16x2(v.x), a1 = bf16x2_to_f16x2(v.y);
-            const uint32_t a2 = bf16x2_to_f16x2(v.z), a3 = bf16x2_to_f16x2(v.w);
+            const uint32_t a0 = xh_f16 ? bf16x2_to_f16x2(v.x) : v.x, a1 = xh_f16 ? bf16x2_to_f16x2(v.y) : v.y;
+            const uint32_t a2 = xh_f16 ? bf16x2_to_f16x2(v.z) : v.z, a3 = xh_f16 ? bf16x2_to_f16x2(v.w) : v.w;
             dst[i] = make_uint4(prmt(a0, a2, 0x5410u), prmt(a0, a2, 0x7632u), prmt(a1, a3, 0x5410u),
                                 prmt(a1, a3, 0x7632u));
         }
@@ -87,12 +87,13 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict
 }
 
 void launch_route_topk(const float *logits, int T, int E, int k, int32_t *ids, float *w, cudaStream_t s,
-                       int32_t *local_ids, int ep_base, int ep_local, const uint16_t *x, int H, uint16_t *xh)
+                       int32_t *local_ids, int ep_base, int ep_local, const uint16_t *x, int H, uint16_t *xh,
+                       bool xh_f16)
 {
     if (T <= 0) return;
     const int warps = 8;
     route_topk_kernel<<<cdiv(T, warps), warps * 32, 0, s>>>(logits, T, E, k, ids, w, local_ids, ep_base, ep_local,
-                                                            x, H, xh);
+                                                            x, H, xh, xh_f16 ? 1 : 0);
 }
 
 // ------------------------------------------------------------------------------------------

@@ -80,13 +80,13 @@ __host__ __device__ constexpr int w4_stage_bytes(int fmt) { return 4 * 32 * 16 +
 //              without routing weights: the plain grouped GEMM).
 // CVT (INT4 only): the activations are bf16 and are converted to f16 in registers; otherwise they
 // are already f16 (INT4) or bf16 (MXFP4 / NVFP4).
-// Paired activations: the library's own activation rows (the routing kernel's f16 copy of x and
-// every h this file writes) hold each 8-input group in the nibble-pair order (x0 x4) (x1 x5)
-// (x2 x6) (x3 x7), so a 16-byte load is the four MMA B registers as they are; rows the caller
-// passes (bf16 x of the gate/up GEMM in MXFP4 / NVFP4 and in the few-row blocks, the grouped
-// GEMM's A) are paired in registers.
-template <int MODE, int FMT, bool CVT>
-__host__ __device__ constexpr bool act_paired() { return !CVT && (MODE == MODE_DOWN || FMT == W4_INT4); }
+// Paired activations: the library's own activation rows (the routing kernel's copy of x for the
+// decode schedule and every h this file writes) hold each 8-input group in the nibble-pair order
+// (x0 x4) (x1 x5) (x2 x6) (x3 x7), so a 16-byte load is the four MMA B registers as they are; rows
+// the caller passes (bf16 x in the few-row blocks (STRIDED) of the tensor-core schedule, the
+// grouped GEMM's A, both with CVT for INT4) are paired in registers.
+template <int MODE, bool STRIDED, bool CVT>
+__host__ __device__ constexpr bool act_paired() { return !CVT && (MODE == MODE_DOWN || !STRIDED); }
 template <int BM, int WARPS, int MODE, bool STRIDED, int FMT, bool CVT>
 __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4GroupedArgs a)
 {
@@ -231,7 +231,7 @@ __global__ void __launch_bounds__(WARPS * 32) w4a16_grouped_mma_kernel(W4Grouped
                     xv.w = bf16x2_to_f16x2(xv.w);
                 }
                 uint32_t b[4];
-                if (act_paired<MODE, FMT, CVT>()) {
+                if (act_paired<MODE, STRIDED, CVT>()) {
                     b[0] = xv.x;
                     b[1] = xv.y;
                     b[2] = xv.z;
