@@ -8,9 +8,9 @@
 // grouped kernels"). Re-derived for tcgen05:
 //
 // Weights take the MMA's A side and live in TENSOR memory: dequantization warps turn the packed
-// codes into bf16 in registers and store them with tcgen05.st, so dequantized weights never pass
-// through shared memory (a bf16 B-side tile would cost its shared-memory bandwidth twice, on
-// write and on every MMA read). The activations (routed rows gathered in aligned order, one
+// codes into f16 (INT4, exact) or bf16 (MXFP4 / NVFP4) in registers and store them with
+// tcgen05.st, so dequantized weights never pass through shared memory (a 16-bit B-side tile would
+// cost its shared-memory bandwidth twice, on write and on every MMA read). The activations (routed rows gathered in aligned order, one
 // expert per 256-row block) are the B side, loaded by TMA with the 128-byte swizzle.
 //   D[weight rows, tokens] += A_tmem[128 weight rows, K] * B_smem[tokens, K]^T   (M = 128, K = 16)
 // A tile serves up to 256 tokens, so each dequantized weight feeds 256 rows of MMA work: the
@@ -27,14 +27,16 @@
 // gate rows of 16 features in lanes 0-15 and their up rows in lanes 16-31; down: tiles of 128
 // output rows):
 //   warp 0      TMA producer of the activation tiles [256 tokens x 128 inputs] (3 stages, two
-//               128-byte-swizzled halves of 64 inputs each); a tile's bytes complete on the same
-//               "stage ready" barrier the dequantization warps arrive on, and one commit per step
-//               frees both the weight stage and the tile;
-//   warp 1      tensor-memory allocation; lane 0 issues 8 MMAs (K = 16) per 128-input step into
-//               the one accumulator and commits. On sm_100a a pipeline step costs several hundred
-//               cycles of synchronization whatever work it carries (an MMA issue ~50-65 cycles, a
-//               barrier wait ~47 even when the phase is complete, more under load), so the steps
-//               are long and the MMA thread waits on one barrier and commits once per step;
+//               128-byte-swizzled halves of 64 inputs each; the warp runs the loop, one elected
+//               lane issues the copies); a tile's bytes complete on the same "stage ready" barrier
+//               the dequantization warps arrive on, and one commit per step frees both the weight
+//               stage and the tile;
+//   warp 1      tensor-memory allocation; the whole warp runs the issue loop and one elected lane
+//               issues 8 MMAs (K = 16) per 128-input step into the one accumulator and commits.
+//               A pipeline step costs several hundred cycles of synchronization whatever work it
+//               carries (an MMA issue ~50-65 cycles, a barrier wait ~47 even when the phase is
+//               complete, more under load), so the steps are long and the issuing warp waits on
+//               one barrier and commits once per step;
 //   warps 2-17  dequantization: a thread owns one weight row (tensor lane) and a 32-input slice
 //               of each 128-input step (16 bytes of codes, 1 group scale), fetches them into
 //               registers two steps ahead, and writes the dequantized slice to one of 3
