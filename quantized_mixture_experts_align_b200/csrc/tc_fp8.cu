@@ -11,9 +11,10 @@
 // CTA = one 128 x BN output tile, 18 warps:
 //   warp 0      TMA producer: A [128 x 128 B] and B [BN x 128 B] tiles per K block, 128-byte
 //               swizzle, into a 4-stage shared-memory ring (mbarrier transaction counts);
-//   warp 1      allocates tensor memory; lane 0 issues 4 tcgen05.mma (K = 32 each) per K block
-//               into partial buffer kb % 2 and commits to the stage's "empty" and the buffer's
-//               "full" barriers;
+//   warp 1      allocates tensor memory; one elected lane issues 4 tcgen05.mma (K = 32 each) per
+//               K block into partial buffer kb % 2 and commits to the stage's "empty" and the
+//               buffer's "full" barriers (warps 0 and 1 run their loops warp-wide, one elected
+//               lane issuing, so the operands stay warp-uniform);
 //   warps 2-17  promotion and epilogue: warp w reads tensor-memory lanes 32 (w % 4) .. +31
 //               (= tile rows) and one quarter of the columns, keeps the running f32 sums in
 //               registers (the next block's scales are loaded while the partial is awaited),
