@@ -249,7 +249,6 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
     } else {
         // ---- dequantization ----
         const int dw = warp - 2, quarter = warp & 3, kq = dw >> 2;  // lane quarter, K slice
-        const int t = dw * 32 + lane;                            // ring slot owner
         const int row = quarter * 32 + lane;                     // tensor-memory lane = weight row
         // gate/up: lanes 0-15 of each lane quarter hold the gate rows of 16 features, lanes 16-31
         // the up rows of the same features (the epilogue pairs them with one shuffle)
@@ -419,6 +418,30 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
     if (warp == 1) tc::tmem_dealloc(tmem, kTmemCols);
 }
 
+// L2 policy for the gather's reads of x: each token's row is read once per routed slot, so keep it
+// resident (the gathered rows written meanwhile are streamed out, evict-first).
+__device__ __forceinline__ uint64_t l2_evict_last_policy()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+__device__ __forceinline__ uint4 ld_keep_v4(const uint4 *p, uint64_t pol)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p), "l"(pol));
+    return v;
+}
+
+__device__ __forceinline__ void st_stream_v4(uint4 *p, const uint4 &v)
+{
+    asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
 // Gather of bf16 activation rows into aligned order (row r takes row sorted_ids[r] / k of x), each
 // 8-input group in the K order of the dequantized weights (0 4 1 5 2 6 3 7), converted to f16 for
 // the INT4 GEMMs (TO_F16); one warp per row, 16-byte copies. Only the rows the MMAs read are written: the real rows and the zero
@@ -432,6 +455,7 @@ __global__ void __launch_bounds__(256) gather_bf16_kernel(const uint16_t *__rest
 {
     const int lane = threadIdx.x & 31;
     const int rows = min(__ldg(ntp), cap_rows);
+    const uint64_t keep = l2_evict_last_policy();
     for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += gridDim.x * (blockDim.x >> 5)) {
         const int slot = __ldg(sorted_ids + r);
         const bool real = slot < n_slots;
@@ -448,7 +472,7 @@ __global__ void __launch_bounds__(256) gather_bf16_kernel(const uint16_t *__rest
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const int i = i0 + 32 * u;
-                v[u] = (real && i < H / 8) ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
+                v[u] = (real && i < H / 8) ? ld_keep_v4(src + i, keep) : make_uint4(0u, 0u, 0u, 0u);
             }
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
@@ -465,7 +489,7 @@ __global__ void __launch_bounds__(256) gather_bf16_kernel(const uint16_t *__rest
                     v[u].z = bf16x2_to_f16x2(v[u].z);
                     v[u].w = bf16x2_to_f16x2(v[u].w);
                 }
-                if (i < H / 8) dst[i] = v[u];
+                if (i < H / 8) st_stream_v4(dst + i, v[u]);
             }
         }
     }
