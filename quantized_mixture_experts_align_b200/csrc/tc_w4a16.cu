@@ -136,7 +136,7 @@ __global__ void __launch_bounds__(kThreads, 1) w4a16_tc_kernel(const __grid_cons
     const int tile0 = blockIdx.x * tpc;
     const int nt = min(tpc, a.N / kTileW - tile0);
     const int n0 = tile0 * kTileW;  // first output feature (gate/up) or row (down)
-    const int K = a.K, NS = K / kKs, NT = nt * NS;  // K steps per tile, in all
+    const int K = a.K, NS = K / kKs;  // K steps per tile
     // real rows of this block: the expert's slots come first, padding after
     const int valid = __syncthreads_count(threadIdx.x < kTok && __ldg(a.sorted_ids + r0 + threadIdx.x) < a.n_slots);
     const int n_mma = (valid + 15) & ~15;  // MMA N: multiple of 16 in [16, 256]
