@@ -64,7 +64,6 @@ constexpr int kBStages = 3;   // activation tiles (shared memory)
 // slower.
 constexpr int kPf = 2;
 constexpr int kDeqWarps = 16;  // 4 per tensor-memory lane quarter, each a quarter of every step
-constexpr int kDeqThreads = kDeqWarps * 32;
 constexpr int kSplit = kDeqWarps / 4;           // K slices of a step (one per warp of a lane quarter)
 constexpr int kThrK = kKs / kSplit;             // 32 inputs per thread per step: 4 code words, 1 group
 static_assert(kThrK == 32, "one scale group per thread and step");
