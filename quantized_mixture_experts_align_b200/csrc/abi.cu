@@ -130,16 +130,18 @@ static int pick_block_m(long T, int k, int E)
     return 64;
 }
 
-// K split of the few-row dense FP8 GEMM (swap-AB tcgen05 tiles, used up to fp8_skinny_max_rows()
-// rows; cluster size): the smallest power of two that gives
-// every SM one CTA (16 padded rows: two, the lighter CTAs then share SMs best), at most 8.
-// Measured on 24576 x 7168 weights: 16 rows 36.9 us with split 2 vs 38.9 with 1; 32 / 64 rows
-// 41.0 / 46.6 us with split 1 vs 45.1 / 55.3 with 2.
-static int pick_skinny_split(int M, int N, int K)
+// K split of the few-row dense FP8 GEMM (swap-AB tcgen05 tiles, used up to
+// fp8_skinny_max_rows(channelwise) rows; cluster size): the smallest power of two that gives every
+// SM one CTA, or two where the CTAs are light enough to share an SM (16 padded rows; 32 with
+// block scales, whose CTAs there run three to an SM), at most 8. Measured on 24576 x 7168
+// weights: 16 rows 36.9 us with split 2 vs 38.9 with 1; block scales at 32 rows 38.2-38.9 us with
+// split 2 (three CTAs per SM) vs 41.0 with 1. The two-CTA form that the channelwise GEMM keeps
+// took 41.0 / 46.6 us at 32 / 64 rows with split 1 vs 45.1 / 55.3 with 2 (block scales).
+static int pick_skinny_split(int M, int N, int K, bool channelwise)
 {
     (void)K;
     const int tiles = N / 128;
-    const int want = (M <= 16 ? 2 : 1) * 148;
+    const int want = (M <= 16 || (!channelwise && M <= 32) ? 2 : 1) * 148;
     int split = 1;
     while (split < 8 && tiles * split < want) split *= 2;
     return split;
@@ -1002,7 +1004,7 @@ int w8a8_block_fp8_matmul(const uint8_t *A, const float *As, const uint8_t *B, c
     MOEQ_REQUIRE(C);
     if (reinterpret_cast<uintptr_t>(A) % 16 || reinterpret_cast<uintptr_t>(B) % 16 || reinterpret_cast<uintptr_t>(C) % 16)
         return set_error(MOEQ_ERR_UNSUPPORTED, "w8a8_block_fp8_matmul: A, B and C must be 16-byte aligned");
-    // up to 64 rows: swap-AB tiles with K split over a cluster (HBM bound); more rows: 128-row
+    // up to 32 rows: swap-AB tiles with K split over a cluster (HBM bound); more rows: 128-row
     // activation tiles
     Fp8TcArgs t{};
     t.a_scale = As;
@@ -1014,8 +1016,8 @@ int w8a8_block_fp8_matmul(const uint8_t *A, const float *As, const uint8_t *B, c
     t.status = device_status_ptr();
     if (!t.status) return set_error(MOEQ_ERR_CUDA, "w8a8_block_fp8_matmul: no device status word");
     trace::Scope ts(trace::DENSE, (cudaStream_t)stream);
-    const int rc = M <= fp8_skinny_max_rows()
-                       ? launch_fp8_tc_skinny(t, A, B, pick_skinny_split(M, N, K), false, (cudaStream_t)stream)
+    const int rc = M <= fp8_skinny_max_rows(false)
+                       ? launch_fp8_tc_skinny(t, A, B, pick_skinny_split(M, N, K, false), false, (cudaStream_t)stream)
                        : launch_fp8_tc_gemm(t, A, B, (cudaStream_t)stream);
     if (rc) return rc;
     return check_launch("w8a8_block_fp8_matmul");
@@ -1049,8 +1051,8 @@ int w8a8_channel_fp8_matmul(const uint8_t *A, const float *As, const uint8_t *B,
     t.status = device_status_ptr();
     if (!t.status) return set_error(MOEQ_ERR_CUDA, "w8a8_channel_fp8_matmul: no device status word");
     trace::Scope ts(trace::DENSE, (cudaStream_t)stream);
-    const int rc = M <= fp8_skinny_max_rows()
-                       ? launch_fp8_tc_skinny(t, A, B, pick_skinny_split(M, N, K), true, (cudaStream_t)stream)
+    const int rc = M <= fp8_skinny_max_rows(true)
+                       ? launch_fp8_tc_skinny(t, A, B, pick_skinny_split(M, N, K, true), true, (cudaStream_t)stream)
                        : launch_fp8_tc_channel(t, A, B, (cudaStream_t)stream);
     if (rc) return rc;
     return check_launch("w8a8_channel_fp8_matmul");

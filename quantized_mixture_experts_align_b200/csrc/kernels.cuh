@@ -135,11 +135,11 @@ void launch_w4a16_grouped_mma(const W4GroupedArgs &a, int mode, int block_m, int
 void launch_fp8_grouped_mma(const F8GroupedArgs &a, int mode, int block_m, int max_blocks, cudaStream_t s);
 // tcgen05 block-FP8 GEMM: A [M, K] and B [N, K] E4M3, K % 128 == 0, N % 128 == 0. Returns a status.
 int launch_fp8_tc_gemm(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B, cudaStream_t s);
-// Dense channelwise FP8 GEMM (a_scale [M], b_scale [N]) for M > fp8_skinny_max_rows().
+// Dense channelwise FP8 GEMM (a_scale [M], b_scale [N]) for M > fp8_skinny_max_rows(true).
 int launch_fp8_tc_channel(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B, cudaStream_t s);
-// Dense block-FP8 GEMM for M <= fp8_skinny_max_rows() rows (swap-AB tcgen05 tiles of 128 weight
-// rows, K split over a cluster of `split` CTAs reduced through distributed shared memory).
-int fp8_skinny_max_rows();
+// Dense FP8 GEMM for M <= fp8_skinny_max_rows(channelwise) rows (swap-AB tcgen05 tiles of 128
+// weight rows, K split over a cluster of `split` CTAs reduced through distributed shared memory).
+int fp8_skinny_max_rows(bool channelwise);
 // channelwise: a_scale [M] per token and b_scale [N] per channel, the whole K accumulated in one
 // tensor-memory buffer.
 int launch_fp8_tc_skinny(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B, int split, bool channelwise,

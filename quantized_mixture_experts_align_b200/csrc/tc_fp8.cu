@@ -572,7 +572,7 @@ static DenseSchedule pick_dense_schedule(int M, int N, int K, int bn, bool chann
 
 int launch_fp8_tc_gemm(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B, cudaStream_t s)
 {
-    // Rows past 64 (fewer go to the swap-AB kernel): 256-column tiles (more weight bytes in flight
+    // Rows past 32 (fewer go to the swap-AB kernel): 256-column tiles (more weight bytes in flight
     // per SM, fewer activation re-reads; tensor bound for many rows), chosen from measured M sweeps.
     const int bn = (a.N % 256 == 0) ? 256 : 128;
     const DenseSchedule sch = pick_dense_schedule(a.M, a.N, a.K, bn, false);

@@ -1,4 +1,5 @@
-// Block-FP8 GEMM for few activation rows (M <= 64) on the 5th-generation tensor cores.
+// Dense FP8 GEMM for few activation rows (block scales: M <= 32; channelwise: M <= 64) on the
+// 5th-generation tensor cores.
 //
 // "SGLang W8A8 Block FP8 quantized kernel config files", section "Background", defines
 //   C[m, n] = sum over 128-wide K blocks kb of As[m, kb] * Bs[n/128, kb] * (A_q[m, kb] . B_q[n, kb]).
@@ -10,7 +11,7 @@
 // of S CTAs; each CTA promotes its K blocks into registers and the S partial tiles are summed
 // through distributed shared memory (no workspace, no second launch).
 //
-// CTA = 128 weight rows x MP rows x K/S, 2 + EW warps (two CTAs per SM). The pipeline moves G
+// CTA = 128 weight rows x MP rows x K/S, 2 + EW warps (NC CTAs per SM). The pipeline moves G
 // K blocks per step:
 //   warp 0        TMA producer: per K block a weight tile [128 x 128 B] and an activation tile
 //                 [MP x 128 B], 128-byte swizzle, into a shared-memory ring of steps;
@@ -36,22 +37,27 @@ constexpr int kWBytes = kRows * kBK;
 
 // MP padded rows; G K blocks per pipeline step (one wait, one MMA batch, one commit and one
 // promotion pass per step: the hand-offs between the roles, not the bytes, set the time of a
-// step); TWO: the shared memory of two CTAs fits on one SM; CW: channelwise scales (per token,
-// per channel), the CTA's whole K range accumulated in one buffer and scaled once.
-template <int MP, int G, bool TWO, bool CW>
+// step); NC CTAs share an SM (1, 2 or 3: the ring is sized so that their shared memory fits);
+// CW: channelwise scales (per token, per channel), the CTA's whole K range accumulated in one
+// buffer and scaled once.
+template <int MP, int G, int NC, bool CW>
 struct SkinnyShape {
     static constexpr int kEpiWarps = MP <= 64 ? 4 : 8;        // <= 64 accumulators per thread
     static constexpr int kThreads = (2 + kEpiWarps) * 32;
     static constexpr int kCols = MP / (kEpiWarps / 4);        // columns per promotion warp
     static constexpr int kKbBytes = kWBytes + MP * kBK;       // one K block: weights + activations
     static constexpr int kStageBytes = G * kKbBytes;          // multiple of 1024 (MP >= 16)
-    static constexpr int kStages = (TWO ? 104 * 1024 : 200 * 1024) / kStageBytes;
+    static constexpr int kRing = NC == 1 ? 200 * 1024 : NC == 2 ? 104 * 1024 : 64 * 1024;
+    static constexpr int kStages = kRing / kStageBytes;
     static constexpr int kBufCols = CW ? MP : G * MP;         // one partial buffer: G blocks
     static constexpr int kTmemCols = 2 * kBufCols < 32 ? 32 : 2 * kBufCols;
     static_assert(kStages >= 2, "at least two pipeline stages");
-    static_assert(kTmemCols <= (TWO ? 256 : 512), "tensor memory of the CTAs on one SM");
+    static_assert(NC >= 1 && NC <= 3, "one to three CTAs per SM");
+    static_assert(kTmemCols * NC <= 512, "tensor memory of the CTAs on one SM");
     static_assert(kStages * kStageBytes >= MP * kRows * 4, "partial tile must fit in the ring");
     static_assert(kKbBytes % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
+    // shared memory one CTA may take when NC of them share the SM's 228 KB (1 KB each reserved)
+    static constexpr size_t kSmemCap = (NC == 1 ? 227 : 228 / NC - 1) * 1024;
     static constexpr size_t smem_bytes(int nkb_max)
     {
         return 1024 + (size_t)kStages * kStageBytes + (size_t)nkb_max * MP * 4 + (2 * kStages + 5) * 8 + 16;
@@ -68,12 +74,12 @@ __device__ __forceinline__ float4 ld_cluster_f32x4(uint32_t addr)
     return v;
 }
 
-template <int MP, int G, bool TWO, bool CW>
-__global__ void __launch_bounds__(SkinnyShape<MP, G, TWO, CW>::kThreads, TWO ? 2 : 1)
+template <int MP, int G, int NC, bool CW>
+__global__ void __launch_bounds__(SkinnyShape<MP, G, NC, CW>::kThreads, NC)
     fp8_tc_skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                          Fp8TcArgs a, int split)
 {
-    using Sh = SkinnyShape<MP, G, TWO, CW>;
+    using Sh = SkinnyShape<MP, G, NC, CW>;
     constexpr int kStages = Sh::kStages, kEpiWarps = Sh::kEpiWarps, COLS = Sh::kCols;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -262,20 +268,20 @@ __global__ void __launch_bounds__(SkinnyShape<MP, G, TWO, CW>::kThreads, TWO ? 2
     if (warp == 1) tc::tmem_dealloc(tmem, Sh::kTmemCols);
 }
 
-template <int MP, int G, bool TWO, bool CW>
+template <int MP, int G, int NC, bool CW>
 int launch_skinny(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B, int split, cudaStream_t s)
 {
-    using Sh = SkinnyShape<MP, G, TWO, CW>;
+    using Sh = SkinnyShape<MP, G, NC, CW>;
     const int KB = a.K / kBK;
     // the per-block scale table grows with K / split: more CTAs per tile for very deep K
-    while (Sh::smem_bytes((KB + split - 1) / split) > (TWO ? 113 : 227) * 1024 && split < 8 && split < KB) ++split;
+    while (Sh::smem_bytes((KB + split - 1) / split) > Sh::kSmemCap && split < 8 && split < KB) ++split;
     const size_t smem = Sh::smem_bytes((KB + split - 1) / split);
     if (smem > 227 * 1024)
         return set_error(MOEQ_ERR_UNSUPPORTED, "tcgen05 FP8 skinny GEMM: K = %d needs %zu bytes of shared memory",
                          a.K, smem);
     static std::atomic<int> smem_enabled[kMaxDevices];
     {
-        const cudaError_t e = enable_smem(fp8_tc_skinny_kernel<MP, G, TWO, CW>, (int)smem, smem_enabled);
+        const cudaError_t e = enable_smem(fp8_tc_skinny_kernel<MP, G, NC, CW>, (int)smem, smem_enabled);
         if (e != cudaSuccess)
             return set_error(MOEQ_ERR_CUDA, "tcgen05 FP8 skinny GEMM: shared-memory attribute: %s",
                              cudaGetErrorString(e));
@@ -297,33 +303,39 @@ int launch_skinny(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B, int sp
     at[0].val.clusterDim.z = 1;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, fp8_tc_skinny_kernel<MP, G, TWO, CW>, tmW, tmX, a, split);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, fp8_tc_skinny_kernel<MP, G, NC, CW>, tmW, tmX, a, split);
     if (e != cudaSuccess) return set_error(MOEQ_ERR_CUDA, "tcgen05 FP8 skinny GEMM launch: %s", cudaGetErrorString(e));
     return MOEQ_OK;
 }
 
 }  // namespace
 
-int fp8_skinny_max_rows() { return 64; }
+// Up to 32 rows the block-scaled GEMM streams the weights faster through this kernel; from 33 rows
+// the 128-row tile kernel (one wave of 128 x 256 tiles for N = 24576) is as fast or faster:
+// 24576 x 7168 weights at 33-64 rows 41.0 us there against 46.6 us here (L2 flushed, alternating
+// runs). The channelwise GEMM keeps this kernel up to 64 rows.
+int fp8_skinny_max_rows(bool channelwise) { return channelwise ? 64 : 32; }
 
 int launch_fp8_tc_skinny(const Fp8TcArgs &a, const uint8_t *A, const uint8_t *B, int split, bool channelwise,
                          cudaStream_t s)
 {
     const int KB = a.K / kBK;
-    if (a.M < 1 || a.M > fp8_skinny_max_rows() || a.N % kRows || a.K % kBK)
+    if (a.M < 1 || a.M > fp8_skinny_max_rows(channelwise) || a.N % kRows || a.K % kBK)
         return set_error(MOEQ_ERR_UNSUPPORTED, "tcgen05 FP8 skinny GEMM: M = %d, N = %d, K = %d", a.M, a.N, a.K);
     if (split < 1) split = 1;
     if (split > 8) split = 8;  // portable cluster size
     if (split > KB) split = KB;
-    // two K blocks per step, two CTAs per SM (measured best for every row count up to 64)
+    // two K blocks per step and two CTAs per SM, except block scales at 17-32 rows: one K block per
+    // step and three CTAs per SM (with a K split of 2 every CTA of 24576 / 128 tiles is resident:
+    // 38.2-38.9 us against 41.0 at 32 rows; at 16 rows both forms measured 36.9 us; the
+    // channelwise GEMM keeps the two-block form it was measured with)
     if (channelwise) {
-        if (a.M <= 16) return launch_skinny<16, 2, true, true>(a, A, B, split, s);
-        if (a.M <= 32) return launch_skinny<32, 2, true, true>(a, A, B, split, s);
-        return launch_skinny<64, 2, true, true>(a, A, B, split, s);
+        if (a.M <= 16) return launch_skinny<16, 2, 2, true>(a, A, B, split, s);
+        if (a.M <= 32) return launch_skinny<32, 2, 2, true>(a, A, B, split, s);
+        return launch_skinny<64, 2, 2, true>(a, A, B, split, s);
     }
-    if (a.M <= 16) return launch_skinny<16, 2, true, false>(a, A, B, split, s);
-    if (a.M <= 32) return launch_skinny<32, 2, true, false>(a, A, B, split, s);
-    return launch_skinny<64, 2, true, false>(a, A, B, split, s);
+    if (a.M <= 16) return launch_skinny<16, 2, 2, false>(a, A, B, split, s);
+    return launch_skinny<32, 1, 3, false>(a, A, B, split, s);
 }
 
 }  // namespace moeq

@@ -327,10 +327,12 @@ def test_dense_fp8_small_shapes_all_rows(M):
 
 
 @pytest.mark.parametrize("M,N,K", [(5, 256, 896), (70, 1280, 2944), (17, 384, 384), (128, 384, 1024),
-                                   (120, 128, 7168), (33, 24576 // 16, 7168)])
+                                   (120, 128, 7168), (33, 24576 // 16, 7168), (24, 24576 // 8, 7168),
+                                   (32, 24576, 1152), (20, 640, 7168)])
 def test_dense_fp8_skinny_split_shapes_all_rows(M, N, K):
     """The few-row path splits K over a cluster of CTAs: cluster sizes that do not divide the K
-    blocks (7 CTAs over 7 blocks, 8 CTAs over 23), every padded row count (16 .. 128), one tile."""
+    blocks (7 CTAs over 7 blocks, 8 CTAs over 23), every padded row count (16 .. 128), one tile;
+    17-32 rows on the three-CTAs-per-SM form with K splits of 2 (full N) and 8 (fewer tiles)."""
     _dense_parity(M, N, K, np.arange(M, dtype=np.int32))
 
 
@@ -344,7 +346,7 @@ def test_dense_fp8_tensor_core_shapes_all_rows(M, N, K):
     _dense_parity(M, N, K, np.arange(M, dtype=np.int32))
 
 
-@pytest.mark.parametrize("M", [1, 16, 128, 1000, 4096])
+@pytest.mark.parametrize("M", [1, 16, 32, 64, 128, 1000, 4096])
 def test_dense_fp8_full_shape_sampled(M):
     rows = np.unique(np.array([0, M - 1, M // 2, M // 3], np.int32))
     _dense_parity(M, 24576, 7168, rows)

@@ -85,6 +85,7 @@ def test_layer_graph_replay_matches_eager(case):
 
 @pytest.mark.parametrize("kind,M,N,K", [
     ("block", 8, 512, 1024),       # swap-AB tiles, K split over a cluster of 8
+    ("block", 24, 512, 1024),      # swap-AB tiles, three CTAs per SM, K split over a cluster of 8
     ("block", 100, 512, 1024),     # 128-row tiles, K split over a cluster of 4
     ("block", 512, 8192, 1024),    # 128-row tiles, no split
     ("channel", 40, 512, 1024),    # channelwise swap-AB
